@@ -1,0 +1,177 @@
+"""Python access to the CPU oracle (ssd_oracle.c).
+
+TEST INFRASTRUCTURE ONLY.  Only the test-suite, ``__graft_entry__.smoke()``
+and the CPU-baseline leg of ``bench.py`` may import this package.  The GPU
+library never calls it, and it imports nothing from the GPU library.
+
+All arithmetic lives in the C file; this module only marshals numpy arrays
+(float32 inputs holding the exact I/O-dtype values, float64 outputs).
+"""
+import ctypes
+
+import numpy as np
+
+from .build import build as _build
+
+_lib = None
+
+
+def _bind(path):
+    lib = ctypes.CDLL(path)
+    f32p = ctypes.POINTER(ctypes.c_float)
+    f64p = ctypes.POINTER(ctypes.c_double)
+    i32p = ctypes.POINTER(ctypes.c_int)
+    i64 = ctypes.c_int64
+    lib.oracle_conv.argtypes = [ctypes.c_int, i64, ctypes.c_int, f32p, f32p, f32p,
+                                f32p, ctypes.c_int, f32p, f32p]
+    lib.oracle_conv.restype = None
+    lib.oracle_scan.argtypes = [ctypes.c_int, i64, ctypes.c_int, ctypes.c_int,
+                                ctypes.c_int, ctypes.c_int, i64,
+                                f32p, i64, i64, f32p, i64, i64, f32p, i64, i64,
+                                f32p, f32p, f32p, f64p, i32p, ctypes.c_int,
+                                f64p, f64p, f64p]
+    lib.oracle_scan.restype = None
+    lib.oracle_round_bf16.argtypes = [ctypes.c_double]
+    lib.oracle_round_bf16.restype = ctypes.c_double
+    lib.oracle_num_threads.argtypes = []
+    lib.oracle_num_threads.restype = ctypes.c_int
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = _bind(_build())
+    return _lib
+
+
+def use_library(path):
+    """Point this module at another build of the oracle source (returns the old one).
+
+    Used by the mutation test, which compiles a deliberately broken copy of
+    ssd_oracle.c and checks that the pins reject it.
+    """
+    global _lib
+    old = _lib
+    _lib = _bind(path) if isinstance(path, str) else path
+    return old
+
+
+def _f32(a):
+    if a is None:
+        return None
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    return a
+
+
+def _p32(a):
+    return None if a is None else a.ctypes.data_as(ctypes.POINTER(ctypes.c_float))
+
+
+def _p64(a):
+    return None if a is None else a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+IO_ROUND = {"none": 0, "f32": 1, "bf16": 2}
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def round_bf16(values):
+    """Round each float64 value to the nearest bfloat16 (ties to even)."""
+    lib = _load()
+    flat = np.asarray(values, dtype=np.float64).ravel()
+    out = np.array([lib.oracle_round_bf16(float(v)) for v in flat])
+    return out.reshape(np.shape(values))
+
+
+def conv(u, w, bias=None, tail_in=None, io_round="none"):
+    """Causal depthwise conv1d (kernel 4) + SiLU.
+
+    u: [b, L, Cch]; w: [Cch, 4]; bias: [Cch] or None; tail_in: [b, 3, Cch] or None.
+    Returns (v [b, L, Cch] float32 rounded per ``io_round``, tail_out [b, 3, Cch]).
+    """
+    lib = _load()
+    u = _f32(u)
+    b, L, cch = u.shape
+    w = _f32(w)
+    assert w.shape == (cch, 4)
+    bias = _f32(bias)
+    tail_in = _f32(tail_in)
+    if tail_in is not None:
+        assert tail_in.shape == (b, 3, cch)
+    v = np.empty((b, L, cch), dtype=np.float32)
+    tail_out = np.empty((b, 3, cch), dtype=np.float32)
+    lib.oracle_conv(b, L, cch, _p32(u), _p32(w), _p32(bias), _p32(tail_in),
+                    IO_ROUND[io_round], _p32(v), _p32(tail_out))
+    return v, tail_out
+
+
+def scan(x, B, C, dt, A, D=None, h0=None, s=0, heads=None, H=None, P=None, G=1,
+         want_ckpt=True):
+    """Literal per-token selective-state recurrence in fp64.
+
+    x: [b, L, >= H*P] (x[:, :, h*P + p] for head h), B and C: [b, L, >= G*N]
+    (group g occupies columns g*N .. g*N+N-1), dt: [b, L, H], A: [H], D: [H]
+    or None, h0: [b, H, P, N] (float64, any exact state) or None.  ``heads`` selects a subset of heads.
+    Returns dict y [b, L, nh, P], h_final [b, nh, P, N], h_ckpt [b, L//s, nh, P, N].
+    """
+    lib = _load()
+    x = np.asarray(x)
+    B = np.asarray(B)
+    C = np.asarray(C)
+    b, L = x.shape[0], x.shape[1]
+    dt = _f32(dt)
+    H = dt.shape[2] if H is None else H
+    assert dt.shape == (b, L, H)
+    N = B.shape[2] // G
+    if P is None:
+        P = x.shape[2] // H
+    A = _f32(A)
+    D = _f32(D)
+    if h0 is not None:
+        h0 = np.ascontiguousarray(h0, dtype=np.float64)
+        assert h0.shape == (b, H, P, N)
+
+    def strided(a):
+        a = _f32(a)
+        return a, a.shape[1] * a.shape[2], a.shape[2]
+
+    x, xbs, xrs = strided(x)
+    B, Bbs, Brs = strided(B)
+    C, Cbs, Crs = strided(C)
+    if heads is None:
+        hsel = None
+        nh = H
+    else:
+        hsel = np.ascontiguousarray(heads, dtype=np.int32)
+        nh = len(hsel)
+    y = np.empty((b, L, nh, P), dtype=np.float64)
+    h_final = np.empty((b, nh, P, N), dtype=np.float64)
+    n_ckpt = L // s if s > 0 else 0
+    h_ckpt = np.empty((b, n_ckpt, nh, P, N), dtype=np.float64) if want_ckpt else None
+    lib.oracle_scan(b, L, H, P, N, G, int(s), _p32(x), xbs, xrs, _p32(B), Bbs, Brs,
+                    _p32(C), Cbs, Crs, _p32(dt), _p32(A), _p32(D), _p64(h0),
+                    None if hsel is None else hsel.ctypes.data_as(ctypes.POINTER(ctypes.c_int)),
+                    nh, _p64(y), _p64(h_final), _p64(h_ckpt))
+    return {"y": y, "h_final": h_final, "h_ckpt": h_ckpt}
+
+
+def layer(u, w, dt, A, D=None, bias=None, tail_in=None, h0=None, H=None, P=None, N=None,
+          G=1, s=0, io_round="none", heads=None, want_ckpt=True):
+    """conv1d+SiLU on the packed x|B|C stream, then the recurrence.
+
+    u: [b, L, H*P + 2*G*N] pre-conv stream, channel order x, then B, then C.
+    Returns the scan dict plus ``v`` (the rounded conv output) and ``tail_out``.
+    """
+    v, tail_out = conv(u, w, bias, tail_in, io_round)
+    d_inner = H * P
+    x = v[:, :, :d_inner]
+    Bm = v[:, :, d_inner:d_inner + G * N]
+    Cm = v[:, :, d_inner + G * N:d_inner + 2 * G * N]
+    out = scan(x, Bm, Cm, dt, A, D, h0, s, heads=heads, H=H, P=P, G=G, want_ckpt=want_ckpt)
+    out["v"] = v
+    out["tail_out"] = tail_out
+    return out

@@ -1,0 +1,69 @@
+"""Plant plausible mistakes in copies of the oracle and check the pins catch each.
+
+Every mutant is a one-line edit of oracle/ssd_oracle.c (a dropped term, a
+wrong sign or index, a swapped operand), compiled to a temporary library on
+the CPU.  The test passes only if at least one pin rejects every mutant.
+"""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from oracle_pins import PINS
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                   "oracle", "ssd_oracle.c")
+
+MUTANTS = {
+    "drop_D_skip": ("yt[p] = acc + Dh * xp;", "yt[p] = acc;"),
+    "decay_sign": ("const double a = exp(dtv * Ah);", "const double a = exp(-dtv * Ah);"),
+    "decay_missing_dt": ("const double a = exp(dtv * Ah);", "const double a = exp(Ah);"),
+    "input_missing_dt": ("const double u = dtv * xp;", "const double u = xp;"),
+    "output_uses_B": ("acc += (double)Ct[n] * Sp[n];", "acc += (double)Bt[n] * Sp[n];"),
+    "output_before_update": (
+        "Sp[n] = a * Sp[n] + u * (double)Bt[n];\n                    acc += (double)Ct[n] * Sp[n];",
+        "acc += (double)Ct[n] * Sp[n];\n                    Sp[n] = a * Sp[n] + u * (double)Bt[n];"),
+    "h0_ignored": ("S[i] = h0 ? h0[(((int64_t)bi * H + h) * P) * N + i] : 0.0;", "S[i] = 0.0;"),
+    "group_index": ("const int g = (int)((int64_t)h * G / H);", "const int g = h % G;"),
+    "ckpt_off_by_one": ("if (h_ckpt && s > 0 && (t + 1) % s == 0) {\n                const int64_t k = (t + 1) / s - 1;",
+                        "if (h_ckpt && s > 0 && t % s == 0 && t > 0) {\n                const int64_t k = t / s - 1;"),
+    "conv_shift": ("int64_t tt = t - (ORACLE_CONV_K - 1) + k;",
+                   "int64_t tt = t - (ORACLE_CONV_K - 1) + k - 1;"),
+    "conv_weight_flip": ("z += (double)w[c * ORACLE_CONV_K + k] * val;",
+                         "z += (double)w[c * ORACLE_CONV_K + (ORACLE_CONV_K - 1 - k)] * val;"),
+    "conv_tail_order": ("else val = tb ? (double)tb[(3 + tt) * Cch + c] : 0.0;",
+                        "else val = tb ? (double)tb[(-1 - tt) * Cch + c] : 0.0;"),
+    "silu_sign": ("double silu = z / (1.0 + exp(-z));", "double silu = z / (1.0 + exp(z));"),
+    "tail_out_shift": ("int64_t pos = L - 3 + r;", "int64_t pos = L - 4 + r;"),
+    "bf16_ties_away": ("double r = nearbyint(ldexp(fabs(d), -q));", "double r = round(ldexp(fabs(d), -q));"),
+    "bias_dropped": ("double z = bias ? (double)bias[c] : 0.0;", "double z = 0.0;"),
+}
+
+
+def _build_mutant(tmp_path, name, old, new):
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not unique/found"
+    path = tmp_path / f"{name}.c"
+    path.write_text(src.replace(old, new))
+    lib = tmp_path / f"lib_{name}.so"
+    subprocess.check_call(["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp",
+                           "-fPIC", "-shared", "-std=c11", str(path), "-o", str(lib), "-lm"])
+    return str(lib)
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(tmp_path, name):
+    old, new = MUTANTS[name]
+    lib = _build_mutant(tmp_path, name, old, new)
+    prev = oracle.use_library(lib)
+    caught = []
+    try:
+        for pin in PINS:
+            try:
+                pin()
+            except AssertionError:
+                caught.append(pin.__name__)
+    finally:
+        oracle.use_library(prev)
+    assert caught, f"no pin rejects mutant {name}"
