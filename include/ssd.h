@@ -1,0 +1,200 @@
+/*
+ * ssd.h -- C ABI of the B200 (sm_100a) Mamba-2 selective-state (SSD) layer.
+ *
+ * The layer (Video-Ma2mba / VAMBA backbone; pith.science verdict record for
+ * arXiv 2411.19460):
+ *   v = silu(causal_conv1d_k4(u))        on the packed x|B|C stream
+ *       (skeptic_critique.load_bearing_attack: "causal Conv1d", kernel 4)
+ *   per head h:  h_t = exp(dt_t*A_h) h_{t-1} + dt_t * x_t B_t^T
+ *                y_t = C_t^T h_t + D_h x_t
+ *       (pith_extraction.core_discovery, Eq. (1) h_t = A_t h_{t-1} + B_t x_t,
+ *        discretised per Mamba-2 head)
+ *   h_ckpt[k] = state after (k+1)*s tokens
+ *       (pith_extraction.key_machinery, "Algorithm 1" sequence checkpoint Sckpt)
+ *
+ * Conventions for every entry point
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates, frees or retains them.  Strides are in ELEMENTS.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream).  The return value reports argument errors and launch
+ *    failures detected on the host.  Errors detected on the device (a bounded
+ *    wait that timed out) are latched in a per-device status word and read by
+ *    ssd_sync_status().
+ *  - Every call returns an ssd_status.  On error nothing is launched, and
+ *    ssd_last_error_string() (thread-local) describes the failure.
+ *  - The library computes everything in its own CUDA kernels; there is no CPU
+ *    fallback.  Shapes the GPU kernels do not support return
+ *    SSD_ERR_UNSUPPORTED.
+ *  - dtype SSD_BF16: x/B/C, u, v, y and the conv tails are bfloat16; SSD_F32:
+ *    they are float.  dt, A, D, conv weights/bias, h0, h_final and h_ckpt are
+ *    always float (fp32 state).
+ */
+#ifndef SSD_H_
+#define SSD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SSD_API __attribute__((visibility("default")))
+#else
+#define SSD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *ssd_stream_t; /* same type as cudaStream_t */
+
+typedef enum ssd_dtype { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
+
+typedef enum ssd_status {
+    SSD_OK = 0,
+    SSD_ERR_NULL = 1,        /* a required pointer is NULL */
+    SSD_ERR_SHAPE = 2,       /* inconsistent or out-of-range sizes */
+    SSD_ERR_ALIGN = 3,       /* a pointer or row stride breaks 16-byte alignment */
+    SSD_ERR_STRIDE = 4,      /* strides smaller than the rows they step over */
+    SSD_ERR_DTYPE = 5,       /* unknown dtype code */
+    SSD_ERR_UNSUPPORTED = 6, /* valid, but no GPU kernel for this shape */
+    SSD_ERR_LAUNCH = 7,      /* CUDA launch or runtime error */
+    SSD_ERR_TIMEOUT = 8,     /* a bounded device-side wait gave up (device status) */
+    SSD_ERR_WORKSPACE = 9    /* workspace missing or smaller than required */
+} ssd_status;
+
+/*
+ * ssd_conv_forward -- depthwise causal conv1d (kernel 4) + SiLU.
+ * Defines: v[bi,t,c] = silu(bias[c] + sum_{k=0..3} w[c,k] * u[bi,t-3+k,c]),
+ * silu(z) = z / (1 + exp(-z)); u at t < 0 is tail_in[bi, 3+t, c] (zeros when
+ * tail_in is NULL).  tail_out[bi, r, c] = u at position L-3+r (from tail_in
+ * when that position is negative): the conv buffer that, with the SSD state,
+ * makes a resumed call exact (skeptic_critique.headline, desk_editor.letter).
+ *   u        [b][L][C_ch], element (bi,t,c) at u[bi*u_batch_stride + t*u_row_stride + c]
+ *   w        [C_ch][4] float; bias [C_ch] float or NULL (zero bias)
+ *   tail_in  [b][3][C_ch] contiguous or NULL; tail_out same layout or NULL.
+ *            tail_out may alias tail_in (it is written after all reads).
+ *   v        [b][L][C_ch] output, strides like u; must not overlap u.
+ * Requirements: C_ch a multiple of 8 (bf16) or 4 (f32); u, v, tails 16-byte
+ * aligned and row/batch strides multiples of 16 bytes (SSD_ERR_ALIGN).
+ */
+SSD_API int ssd_conv_forward(const void *u, int64_t u_batch_stride, int64_t u_row_stride,
+                     const float *w, const float *bias,
+                     const void *tail_in, void *tail_out,
+                     void *v, int64_t v_batch_stride, int64_t v_row_stride,
+                     int b, int64_t L, int C_ch, int dtype, ssd_stream_t stream);
+
+/*
+ * Arguments of the selective scan (see ssd_scan_forward).
+ *   x   element (bi,t,h,p) at x[bi*x_batch_stride + t*x_row_stride + h*P + p]
+ *   B,C element (bi,t,g,n) at B[bi*B_batch_stride + t*B_row_stride + g*N + n]
+ *       (x, B and C may be column slices of the conv output v)
+ *   dt  [b][L][H] float, contiguous, > 0
+ *   A   [H] float (A <= 0 expected; not checked), D [H] float or NULL (no skip)
+ *   h0  [b][H][P][N] float or NULL (zero state); may alias h_final
+ *   y   element (bi,t,h,p) at y[bi*y_batch_stride + t*y_row_stride + h*P + p]
+ *   h_final [b][H][P][N] float or NULL
+ *   h_ckpt  [b][floor(L/s)][H][P][N] float or NULL (no checkpoints written)
+ *   s   checkpoint stride in tokens, a multiple of Q, or 0 (none)
+ *   Q   chunk length: 32, 64 or 128
+ *   workspace: device scratch of at least ssd_scan_workspace_size() bytes,
+ *       256-byte aligned; NULL allowed when that size is 0.  Contents on
+ *       entry are ignored; the call overwrites them.
+ */
+typedef struct ssd_scan_args {
+    int dtype;
+    int b;
+    int64_t L;
+    int H, P, N, G, Q;
+    int64_t s;
+    const void *x;
+    int64_t x_batch_stride, x_row_stride;
+    const void *B;
+    int64_t B_batch_stride, B_row_stride;
+    const void *C;
+    int64_t C_batch_stride, C_row_stride;
+    const float *dt;
+    const float *A;
+    const float *D;
+    const float *h0;
+    void *y;
+    int64_t y_batch_stride, y_row_stride;
+    float *h_final;
+    float *h_ckpt;
+    void *workspace;
+    size_t workspace_bytes;
+} ssd_scan_args;
+
+/*
+ * ssd_scan_forward -- chunked selective scan with state checkpoints.
+ * Computes, for every batch row and head, the recurrence stated at the top
+ * of this header from h0, writing y for every token, h_ckpt every s tokens
+ * and h_final after the last token.  H must be a multiple of G; P and N in
+ * {16, 32, 64, 128}; L >= 0 (L need not be a multiple of Q or s).
+ */
+SSD_API int ssd_scan_forward(const ssd_scan_args *args, ssd_stream_t stream);
+
+/* Bytes of workspace ssd_scan_forward / ssd_stream_forward need for this shape. */
+SSD_API size_t ssd_scan_workspace_size(int b, int64_t L, int H, int P, int N, int Q);
+
+/*
+ * Arguments of one streamed segment (see ssd_stream_forward).  u is the
+ * segment's pre-conv x|B|C stream [b][L][C_ch], C_ch = H*P + 2*G*N, channel
+ * order x, then B, then C.  v receives the conv output (the scan reads its
+ * column slices).  tail_in/h0 carry the previous segment's conv buffer and
+ * state; tail_out/h_final receive this segment's (they may alias them).
+ */
+typedef struct ssd_stream_args {
+    int dtype;
+    int b;
+    int64_t L;
+    int H, P, N, G, Q;
+    int64_t s;
+    const void *u;
+    int64_t u_batch_stride, u_row_stride;
+    const float *conv_w;
+    const float *conv_bias;
+    const void *tail_in;
+    void *tail_out;
+    void *v;
+    int64_t v_batch_stride, v_row_stride;
+    const float *dt;
+    const float *A;
+    const float *D;
+    const float *h0;
+    void *y;
+    int64_t y_batch_stride, y_row_stride;
+    float *h_final;
+    float *h_ckpt;
+    void *workspace;
+    size_t workspace_bytes;
+} ssd_stream_args;
+
+/*
+ * ssd_stream_forward -- one segment of a long stream: conv (tail_in ->
+ * tail_out) then scan (h0 -> h_final, checkpoints every s tokens of this
+ * segment).  Calling it on consecutive segments, each resumed from the
+ * previous (h_final, tail_out), equals one call on the whole sequence
+ * (sequence-axis checkpointing of pith_extraction.key_machinery, with the
+ * conv buffer the skeptic_critique asks for).
+ */
+SSD_API int ssd_stream_forward(const ssd_stream_args *args, ssd_stream_t stream);
+
+/*
+ * ssd_sync_status -- synchronise `stream`, then return SSD_ERR_LAUNCH if the
+ * CUDA runtime reports an error, else the device status word latched by
+ * this library's kernels on the current device (SSD_OK or SSD_ERR_TIMEOUT),
+ * which it then clears.
+ */
+SSD_API int ssd_sync_status(ssd_stream_t stream);
+
+/* Description of the last error on this host thread ("" if none). */
+SSD_API const char *ssd_last_error_string(void);
+
+/* ABI version: major*10000 + minor*100 + patch. */
+SSD_API int ssd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_H_ */

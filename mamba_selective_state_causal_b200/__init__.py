@@ -1,0 +1,225 @@
+"""Python binding of the B200 SSD layer library (libssd.so, C ABI in include/ssd.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  torch tensors supply device memory and the CUDA stream.  If the
+compiled library is missing, importing the binding's functions raises: there
+is no fallback implementation.
+"""
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libssd.so")
+
+SSD_F32, SSD_BF16 = 0, 1
+STATUS = {0: "SSD_OK", 1: "SSD_ERR_NULL", 2: "SSD_ERR_SHAPE", 3: "SSD_ERR_ALIGN",
+          4: "SSD_ERR_STRIDE", 5: "SSD_ERR_DTYPE", 6: "SSD_ERR_UNSUPPORTED",
+          7: "SSD_ERR_LAUNCH", 8: "SSD_ERR_TIMEOUT", 9: "SSD_ERR_WORKSPACE"}
+
+_i64 = ctypes.c_int64
+_vp = ctypes.c_void_p
+
+
+class SSDError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"{STATUS.get(code, code)}: {msg}")
+        self.code = code
+
+
+class ScanArgs(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int), ("b", ctypes.c_int), ("L", _i64),
+                ("H", ctypes.c_int), ("P", ctypes.c_int), ("N", ctypes.c_int),
+                ("G", ctypes.c_int), ("Q", ctypes.c_int), ("s", _i64),
+                ("x", _vp), ("x_batch_stride", _i64), ("x_row_stride", _i64),
+                ("B", _vp), ("B_batch_stride", _i64), ("B_row_stride", _i64),
+                ("C", _vp), ("C_batch_stride", _i64), ("C_row_stride", _i64),
+                ("dt", _vp), ("A", _vp), ("D", _vp), ("h0", _vp),
+                ("y", _vp), ("y_batch_stride", _i64), ("y_row_stride", _i64),
+                ("h_final", _vp), ("h_ckpt", _vp),
+                ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
+
+
+class StreamArgs(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int), ("b", ctypes.c_int), ("L", _i64),
+                ("H", ctypes.c_int), ("P", ctypes.c_int), ("N", ctypes.c_int),
+                ("G", ctypes.c_int), ("Q", ctypes.c_int), ("s", _i64),
+                ("u", _vp), ("u_batch_stride", _i64), ("u_row_stride", _i64),
+                ("conv_w", _vp), ("conv_bias", _vp), ("tail_in", _vp), ("tail_out", _vp),
+                ("v", _vp), ("v_batch_stride", _i64), ("v_row_stride", _i64),
+                ("dt", _vp), ("A", _vp), ("D", _vp), ("h0", _vp),
+                ("y", _vp), ("y_batch_stride", _i64), ("y_row_stride", _i64),
+                ("h_final", _vp), ("h_ckpt", _vp),
+                ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libssd.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -c 'import __graft_entry__ as g; g.build()'`")
+        L = ctypes.CDLL(LIB_PATH)
+        L.ssd_conv_forward.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _i64, _i64,
+                                       ctypes.c_int, _i64, ctypes.c_int, ctypes.c_int, _vp]
+        L.ssd_conv_forward.restype = ctypes.c_int
+        L.ssd_scan_forward.argtypes = [ctypes.POINTER(ScanArgs), _vp]
+        L.ssd_scan_forward.restype = ctypes.c_int
+        L.ssd_stream_forward.argtypes = [ctypes.POINTER(StreamArgs), _vp]
+        L.ssd_stream_forward.restype = ctypes.c_int
+        L.ssd_scan_workspace_size.argtypes = [ctypes.c_int, _i64, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_int, ctypes.c_int]
+        L.ssd_scan_workspace_size.restype = ctypes.c_size_t
+        L.ssd_sync_status.argtypes = [_vp]
+        L.ssd_sync_status.restype = ctypes.c_int
+        L.ssd_last_error_string.argtypes = []
+        L.ssd_last_error_string.restype = ctypes.c_char_p
+        L.ssd_version.argtypes = []
+        L.ssd_version.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(rc):
+    if rc != 0:
+        raise SSDError(rc, lib().ssd_last_error_string().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return SSD_BF16
+    if t.dtype == torch.float32:
+        return SSD_F32
+    raise TypeError(f"unsupported I/O dtype {t.dtype}")
+
+
+def _cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors")
+
+
+def _f32(t, name):
+    if t is not None and (t.dtype != torch.float32 or not t.is_contiguous()):
+        raise TypeError(f"{name} must be a contiguous float32 tensor")
+    return t
+
+
+def workspace_size(b, L, H, P, N, Q):
+    return int(lib().ssd_scan_workspace_size(b, L, H, P, N, Q))
+
+
+def alloc_workspace(b, L, H, P, N, Q, device=None):
+    n = workspace_size(b, L, H, P, N, Q)
+    return torch.empty(max(n, 1), dtype=torch.uint8, device=device or "cuda")
+
+
+def sync_status(stream=None):
+    _check(lib().ssd_sync_status(_stream(stream)))
+
+
+def conv_forward(u, w, bias=None, tail_in=None, tail_out=None, v=None, stream=None):
+    """v = silu(causal_conv1d_k4(u)); returns (v, tail_out)."""
+    _cuda(u, w, bias, tail_in, tail_out, v)
+    b, L, cch = u.shape
+    if v is None:
+        v = torch.empty_like(u)
+    _f32(w, "w")
+    _f32(bias, "bias")
+    rc = lib().ssd_conv_forward(_ptr(u), u.stride(0), u.stride(1), _ptr(w), _ptr(bias),
+                                _ptr(tail_in), _ptr(tail_out), _ptr(v), v.stride(0), v.stride(1),
+                                b, L, cch, _dtype_code(u), _stream(stream))
+    _check(rc)
+    return v, tail_out
+
+
+def scan_forward(x, B, C, dt, A, D=None, h0=None, *, H, G=1, Q=128, s=0, y=None,
+                 h_final=None, h_ckpt=None, workspace=None, stream=None):
+    """Chunked selective scan; returns (y, h_final, h_ckpt).
+
+    x: [b, L, >=H*P] view (may be a column slice of the conv output),
+    B, C: [b, L, >=G*N] views, dt: [b, L, H] float32, A/D: [H] float32,
+    h0: [b, H, P, N] float32 or None.
+    """
+    _cuda(x, B, C, dt, A, D, h0, y, h_final, h_ckpt, workspace)
+    b, L = x.shape[0], x.shape[1]
+    P = x.shape[2] // H
+    N = B.shape[2] // G
+    dev = x.device
+    if y is None:
+        y = torch.empty(b, L, H, P, dtype=x.dtype, device=dev)
+    if h_final is None:
+        h_final = torch.empty(b, H, P, N, dtype=torch.float32, device=dev)
+    if h_ckpt is None and s > 0:
+        h_ckpt = torch.empty(b, L // s, H, P, N, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = alloc_workspace(b, L, H, P, N, Q, dev)
+    for t, n in ((dt, "dt"), (A, "A"), (D, "D"), (h0, "h0"), (h_final, "h_final"), (h_ckpt, "h_ckpt")):
+        _f32(t, n)
+    a = ScanArgs()
+    a.dtype = _dtype_code(x); a.b = b; a.L = L; a.H = H; a.P = P; a.N = N; a.G = G; a.Q = Q; a.s = s
+    a.x = x.data_ptr(); a.x_batch_stride = x.stride(0); a.x_row_stride = x.stride(1)
+    a.B = B.data_ptr(); a.B_batch_stride = B.stride(0); a.B_row_stride = B.stride(1)
+    a.C = C.data_ptr(); a.C_batch_stride = C.stride(0); a.C_row_stride = C.stride(1)
+    a.dt = dt.data_ptr(); a.A = A.data_ptr(); a.D = D.data_ptr() if D is not None else None
+    a.h0 = h0.data_ptr() if h0 is not None else None
+    y2 = y.view(b, L, H * P)
+    a.y = y.data_ptr(); a.y_batch_stride = y2.stride(0); a.y_row_stride = y2.stride(1)
+    a.h_final = h_final.data_ptr() if h_final is not None else None
+    a.h_ckpt = h_ckpt.data_ptr() if h_ckpt is not None else None
+    a.workspace = workspace.data_ptr(); a.workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().ssd_scan_forward(ctypes.byref(a), _stream(stream)))
+    return y, h_final, h_ckpt
+
+
+def stream_forward(u, conv_w, dt, A, D=None, *, H, P, N, G=1, Q=128, s=0, conv_bias=None,
+                   tail_in=None, tail_out=None, h0=None, v=None, y=None, h_final=None,
+                   h_ckpt=None, workspace=None, stream=None):
+    """One streamed segment: conv (tail_in -> tail_out), then scan (h0 -> h_final)."""
+    _cuda(u, conv_w, dt, A, D, conv_bias, tail_in, tail_out, h0, v, y, h_final, h_ckpt, workspace)
+    b, L, cch = u.shape
+    assert cch == H * P + 2 * G * N, "u must hold x|B|C channels"
+    dev = u.device
+    if v is None:
+        v = torch.empty_like(u)
+    if y is None:
+        y = torch.empty(b, L, H, P, dtype=u.dtype, device=dev)
+    if h_final is None:
+        h_final = torch.empty(b, H, P, N, dtype=torch.float32, device=dev)
+    if tail_out is None:
+        tail_out = torch.empty(b, 3, cch, dtype=u.dtype, device=dev)
+    if h_ckpt is None and s > 0:
+        h_ckpt = torch.empty(b, L // s, H, P, N, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = alloc_workspace(b, L, H, P, N, Q, dev)
+    a = StreamArgs()
+    a.dtype = _dtype_code(u); a.b = b; a.L = L; a.H = H; a.P = P; a.N = N; a.G = G; a.Q = Q; a.s = s
+    a.u = u.data_ptr(); a.u_batch_stride = u.stride(0); a.u_row_stride = u.stride(1)
+    a.conv_w = conv_w.data_ptr(); a.conv_bias = conv_bias.data_ptr() if conv_bias is not None else None
+    a.tail_in = tail_in.data_ptr() if tail_in is not None else None
+    a.tail_out = tail_out.data_ptr()
+    a.v = v.data_ptr(); a.v_batch_stride = v.stride(0); a.v_row_stride = v.stride(1)
+    a.dt = dt.data_ptr(); a.A = A.data_ptr(); a.D = D.data_ptr() if D is not None else None
+    a.h0 = h0.data_ptr() if h0 is not None else None
+    y2 = y.view(b, L, H * P)
+    a.y = y.data_ptr(); a.y_batch_stride = y2.stride(0); a.y_row_stride = y2.stride(1)
+    a.h_final = h_final.data_ptr()
+    a.h_ckpt = h_ckpt.data_ptr() if h_ckpt is not None else None
+    a.workspace = workspace.data_ptr(); a.workspace_bytes = workspace.numel()
+    _check(lib().ssd_stream_forward(ctypes.byref(a), _stream(stream)))
+    return {"v": v, "y": y, "h_final": h_final, "h_ckpt": h_ckpt, "tail_out": tail_out}

@@ -1,0 +1,190 @@
+// conv1d_silu.cu -- depthwise causal conv1d (kernel 4) + SiLU over the packed
+// x|B|C stream (pith.science verdict for arXiv 2411.19460,
+// skeptic_critique.load_bearing_attack: the causal Conv1d in front of the SSD,
+// output at t uses inputs t-3..t; concrete_test: kernel = 4).
+//
+// Pure HBM stream: each thread owns one 16-byte channel vector (8 bf16 or
+// 4 fp32 channels) over a block of TT consecutive tokens.  The 3-token halo
+// lives in registers and slides along the token block, so every input row is
+// read once (plus a 3-row halo per token block) and written once.
+#include "ssd_common.cuh"
+
+namespace ssd {
+namespace {
+
+constexpr int kTokensPerThread = 64;
+constexpr int kUnroll = 8;
+
+struct alignas(16) Vec16 { uint32_t w[4]; };
+
+__device__ __forceinline__ Vec16 ld_stream(const void *p)
+{
+    Vec16 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.w[0]), "=r"(r.w[1]), "=r"(r.w[2]), "=r"(r.w[3])
+                 : "l"(p));
+    return r;
+}
+
+// Unpack a 16-byte vector into floats (8 bf16 or 4 fp32).
+template <typename T> struct VecIO;
+template <> struct VecIO<__nv_bfloat16> {
+    static constexpr int kN = 8;
+    __device__ __forceinline__ static void unpack(const Vec16 &v, float *f)
+    {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) { f[2 * i] = bf16_lo(v.w[i]); f[2 * i + 1] = bf16_hi(v.w[i]); }
+    }
+    __device__ __forceinline__ static Vec16 pack(const float *f)
+    {
+        Vec16 v;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v.w[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
+        return v;
+    }
+    // fast SiLU; the result is rounded to bf16 right after
+    __device__ __forceinline__ static float silu(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
+};
+template <> struct VecIO<float> {
+    static constexpr int kN = 4;
+    __device__ __forceinline__ static void unpack(const Vec16 &v, float *f)
+    {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) f[i] = __uint_as_float(v.w[i]);
+    }
+    __device__ __forceinline__ static Vec16 pack(const float *f)
+    {
+        Vec16 v;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v.w[i] = __float_as_uint(f[i]);
+        return v;
+    }
+    // accurate SiLU for the fp32 I/O path
+    __device__ __forceinline__ static float silu(float z) { return z / (1.0f + expf(-z)); }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256) conv1d_silu_kernel(ConvParams p, int64_t n_tblk)
+{
+    using IO = VecIO<T>;
+    constexpr int V = IO::kN;
+    const int ncv = p.C_ch / V;
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int cv = (int)(gid % ncv);
+    const int64_t rest = gid / ncv;
+    const int64_t tb = rest % n_tblk;
+    const int64_t bi = rest / n_tblk;
+    if (bi >= p.b) return;
+    const int c0 = cv * V;
+
+    float w0[V], w1[V], w2[V], w3[V], bs[V];
+    {
+        const float4 *wp = reinterpret_cast<const float4 *>(p.w + (int64_t)c0 * 4);
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            float4 q = __ldg(wp + i);
+            w0[i] = q.x; w1[i] = q.y; w2[i] = q.z; w3[i] = q.w;
+            bs[i] = p.bias ? __ldg(p.bias + c0 + i) : 0.0f;
+        }
+    }
+    const T *u = reinterpret_cast<const T *>(p.u) + bi * p.ubs + c0;
+    T *v = reinterpret_cast<T *>(p.v) + bi * p.vbs + c0;
+    const T *tin = p.tail_in ? reinterpret_cast<const T *>(p.tail_in) + bi * 3 * p.C_ch + c0 : nullptr;
+
+    const int64_t t0 = tb * kTokensPerThread;
+    const int64_t t1 = min(p.L, t0 + kTokensPerThread);
+
+    // halo: m3 = u[t-3], m2 = u[t-2], m1 = u[t-1]
+    float m3[V], m2[V], m1[V];
+    {
+        float *dst[3] = {m3, m2, m1};
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+            const int64_t pos = t0 - 3 + k;
+            if (pos >= 0) {
+                IO::unpack(ld_stream(u + pos * p.urs), dst[k]);
+            } else if (tin) {
+                IO::unpack(*reinterpret_cast<const Vec16 *>(tin + (3 + pos) * p.C_ch), dst[k]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < V; ++i) dst[k][i] = 0.0f;
+            }
+        }
+    }
+
+    for (int64_t t = t0; t < t1; t += kUnroll) {
+        Vec16 raw[kUnroll];
+#pragma unroll
+        for (int j = 0; j < kUnroll; ++j)
+            if (t + j < t1) raw[j] = ld_stream(u + (t + j) * p.urs);
+#pragma unroll
+        for (int j = 0; j < kUnroll; ++j) {
+            if (t + j < t1) {
+                float cur[V], out[V];
+                IO::unpack(raw[j], cur);
+#pragma unroll
+                for (int i = 0; i < V; ++i) {
+                    float z = bs[i];
+                    z = fmaf(w0[i], m3[i], z);
+                    z = fmaf(w1[i], m2[i], z);
+                    z = fmaf(w2[i], m1[i], z);
+                    z = fmaf(w3[i], cur[i], z);
+                    out[i] = IO::silu(z);
+                    m3[i] = m2[i]; m2[i] = m1[i]; m1[i] = cur[i];
+                }
+                *reinterpret_cast<Vec16 *>(v + (t + j) * p.vrs) = IO::pack(out);
+            }
+        }
+    }
+}
+
+// tail_out[bi, r, c] = u at position L-3+r, or tail_in[bi, 3+pos, c] when pos < 0,
+// or 0.  Runs after the conv kernel on the same stream, so tail_out may alias
+// tail_in; each thread reads its three values before writing any.
+template <typename T>
+__global__ void conv_tail_kernel(ConvParams p)
+{
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= (int64_t)p.b * p.C_ch) return;
+    const int64_t bi = gid / p.C_ch;
+    const int c = (int)(gid % p.C_ch);
+    const T *u = reinterpret_cast<const T *>(p.u) + bi * p.ubs + c;
+    const T *tin = p.tail_in ? reinterpret_cast<const T *>(p.tail_in) + bi * 3 * p.C_ch + c : nullptr;
+    T vals[3];
+#pragma unroll
+    for (int r = 0; r < 3; ++r) {
+        const int64_t pos = p.L - 3 + r;
+        if (pos >= 0) vals[r] = u[pos * p.urs];
+        else vals[r] = tin ? tin[(3 + pos) * p.C_ch] : from_f32<T>(0.0f);
+    }
+    T *tout = reinterpret_cast<T *>(p.tail_out) + bi * 3 * p.C_ch + c;
+#pragma unroll
+    for (int r = 0; r < 3; ++r) tout[r * p.C_ch] = vals[r];
+}
+
+template <typename T>
+int launch_conv_t(const ConvParams &p, cudaStream_t st)
+{
+    constexpr int V = VecIO<T>::kN;
+    if (p.b > 0 && p.L > 0) {
+        const int64_t n_tblk = (p.L + kTokensPerThread - 1) / kTokensPerThread;
+        const int64_t threads = (int64_t)p.b * n_tblk * (p.C_ch / V);
+        const int64_t blocks = (threads + 255) / 256;
+        if (blocks > 0x7fffffffLL) return 2;
+        conv1d_silu_kernel<T><<<(unsigned)blocks, 256, 0, st>>>(p, n_tblk);
+    }
+    if (p.tail_out && p.b > 0) {
+        const int64_t n = (int64_t)p.b * p.C_ch;
+        conv_tail_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p);
+    }
+    return cudaGetLastError() == cudaSuccess ? 0 : 7;
+}
+
+}  // namespace
+
+int launch_conv(const ConvParams &p, int dtype, cudaStream_t st)
+{
+    return dtype == 1 ? launch_conv_t<__nv_bfloat16>(p, st) : launch_conv_t<float>(p, st);
+}
+
+}  // namespace ssd

@@ -1,0 +1,275 @@
+// ssd_api.cu -- the C ABI declared in include/ssd.h: argument checks, the
+// stripe plan, workspace carving and dispatch to the CUDA kernels.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "../../include/ssd.h"
+#include "ssd_common.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char *fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+int ok()
+{
+    g_last_error.clear();
+    return SSD_OK;
+}
+
+// Per-device status word written by kernels when a bounded wait gives up.
+__device__ unsigned int g_device_status;
+
+constexpr int kMaxDevices = 64;
+unsigned int *g_status_ptr[kMaxDevices] = {nullptr};
+
+unsigned int *status_ptr()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    if (!g_status_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+        g_status_ptr[dev] = static_cast<unsigned int *>(p);
+    }
+    return g_status_ptr[dev];
+}
+
+size_t elem_size(int dtype) { return dtype == SSD_BF16 ? 2 : 4; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool pow2_dim(int v) { return v == 16 || v == 32 || v == 64 || v == 128; }
+
+// Stripe plan: the sequence is split into stripes of T tokens (a multiple of
+// Q) so that b * stripes * H gives about a thousand independent (stripe, head)
+// units of work, with T between Q and 32*Q.
+struct Plan {
+    int64_t T = 0, ns = 0;
+    size_t off_S = 0, off_hin = 0, off_dA = 0, bytes = 0;
+};
+
+size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
+
+Plan make_plan(int b, int64_t L, int H, int P, int N, int Q)
+{
+    Plan pl;
+    if (b <= 0 || L <= 0 || H <= 0 || Q <= 0) return pl;
+    int64_t m = ((int64_t)b * L * H) / (1024LL * Q);
+    if (m < 1) m = 1;
+    if (m > 32) m = 32;
+    pl.T = m * Q;
+    pl.ns = (L + pl.T - 1) / pl.T;
+    if (pl.ns > 1) {
+        const size_t state = sizeof(float) * (size_t)b * pl.ns * H * P * N;
+        pl.off_S = 0;
+        pl.off_hin = round256(state);
+        pl.off_dA = pl.off_hin + round256(state);
+        pl.bytes = pl.off_dA + round256(sizeof(float) * (size_t)b * pl.ns * H);
+    }
+    return pl;
+}
+
+int check_scan_shape(int dtype, int b, int64_t L, int H, int P, int N, int G, int Q, int64_t s)
+{
+    if (dtype != SSD_F32 && dtype != SSD_BF16) return fail(SSD_ERR_DTYPE, "unknown dtype %d", dtype);
+    if (b < 0 || L < 0) return fail(SSD_ERR_SHAPE, "negative b (%d) or L (%lld)", b, (long long)L);
+    if (H <= 0 || G <= 0 || H % G != 0)
+        return fail(SSD_ERR_SHAPE, "need H > 0, G > 0 and H %% G == 0 (H=%d, G=%d)", H, G);
+    if (!pow2_dim(P) || !pow2_dim(N))
+        return fail(SSD_ERR_SHAPE, "P and N must be 16, 32, 64 or 128 (P=%d, N=%d)", P, N);
+    if (Q != 32 && Q != 64 && Q != 128) return fail(SSD_ERR_SHAPE, "Q must be 32, 64 or 128 (Q=%d)", Q);
+    if (s < 0 || (s > 0 && s % Q != 0))
+        return fail(SSD_ERR_SHAPE, "checkpoint stride s=%lld must be 0 or a multiple of Q=%d",
+                    (long long)s, Q);
+    return SSD_OK;
+}
+
+int check_rows(const char *name, const void *ptr, int64_t bs, int64_t rs, int64_t width,
+               int b, int64_t L, int dtype, bool need_align)
+{
+    if (!ptr) return fail(SSD_ERR_NULL, "%s is NULL", name);
+    if (rs < width) return fail(SSD_ERR_STRIDE, "%s row stride %lld < row width %lld", name,
+                                (long long)rs, (long long)width);
+    if (b > 1 && bs < rs * L)
+        return fail(SSD_ERR_STRIDE, "%s batch stride %lld < L * row stride", name, (long long)bs);
+    if (bs < 0) return fail(SSD_ERR_STRIDE, "%s batch stride is negative", name);
+    if (need_align) {
+        const size_t es = elem_size(dtype);
+        if (!aligned16(ptr) || (rs * es) % 16 != 0 || (bs * es) % 16 != 0)
+            return fail(SSD_ERR_ALIGN, "%s must be 16-byte aligned with 16-byte row/batch strides", name);
+    }
+    return SSD_OK;
+}
+
+int scan_impl(const ssd_scan_args *a, cudaStream_t st)
+{
+    if (!a) return fail(SSD_ERR_NULL, "args is NULL");
+    int rc = check_scan_shape(a->dtype, a->b, a->L, a->H, a->P, a->N, a->G, a->Q, a->s);
+    if (rc) return rc;
+    if (a->b == 0) return ok();
+    if (a->L > 0) {
+        if ((rc = check_rows("x", a->x, a->x_batch_stride, a->x_row_stride, (int64_t)a->H * a->P, a->b, a->L, a->dtype, true))) return rc;
+        if ((rc = check_rows("B", a->B, a->B_batch_stride, a->B_row_stride, (int64_t)a->G * a->N, a->b, a->L, a->dtype, true))) return rc;
+        if ((rc = check_rows("C", a->C, a->C_batch_stride, a->C_row_stride, (int64_t)a->G * a->N, a->b, a->L, a->dtype, true))) return rc;
+        if ((rc = check_rows("y", a->y, a->y_batch_stride, a->y_row_stride, (int64_t)a->H * a->P, a->b, a->L, a->dtype, true))) return rc;
+        if (!a->dt) return fail(SSD_ERR_NULL, "dt is NULL");
+        if (!a->A) return fail(SSD_ERR_NULL, "A is NULL");
+    }
+    const Plan pl = make_plan(a->b, a->L, a->H, a->P, a->N, a->Q);
+    if (pl.bytes > 0) {
+        if (!a->workspace || a->workspace_bytes < pl.bytes)
+            return fail(SSD_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", pl.bytes,
+                        a->workspace ? a->workspace_bytes : (size_t)0);
+        if ((reinterpret_cast<uintptr_t>(a->workspace) & 255u) != 0)
+            return fail(SSD_ERR_ALIGN, "workspace must be 256-byte aligned");
+    }
+    const size_t state_bytes = sizeof(float) * (size_t)a->b * a->H * a->P * a->N;
+    if (a->L == 0) {
+        // no token: the final state is the initial state
+        if (a->h_final && a->h_final != a->h0) {
+            cudaError_t e = a->h0 ? cudaMemcpyAsync(a->h_final, a->h0, state_bytes, cudaMemcpyDeviceToDevice, st)
+                                  : cudaMemsetAsync(a->h_final, 0, state_bytes, st);
+            if (e != cudaSuccess) return fail(SSD_ERR_LAUNCH, "%s", cudaGetErrorString(e));
+        }
+        return ok();
+    }
+    ssd::ScanParams p{};
+    p.b = a->b; p.L = a->L; p.H = a->H; p.P = a->P; p.N = a->N; p.G = a->G; p.Q = a->Q; p.s = a->s;
+    p.x = a->x; p.xbs = a->x_batch_stride; p.xrs = a->x_row_stride;
+    p.B = a->B; p.Bbs = a->B_batch_stride; p.Brs = a->B_row_stride;
+    p.C = a->C; p.Cbs = a->C_batch_stride; p.Crs = a->C_row_stride;
+    p.dt = a->dt; p.A = a->A; p.D = a->D; p.h0 = a->h0;
+    p.y = a->y; p.ybs = a->y_batch_stride; p.yrs = a->y_row_stride;
+    p.h_final = a->h_final; p.h_ckpt = a->h_ckpt;
+    p.T = pl.T; p.ns = pl.ns;
+    char *ws = static_cast<char *>(a->workspace);
+    p.ws_S = pl.bytes ? reinterpret_cast<float *>(ws + pl.off_S) : nullptr;
+    p.ws_hin = pl.bytes ? reinterpret_cast<float *>(ws + pl.off_hin) : nullptr;
+    p.ws_dA = pl.bytes ? reinterpret_cast<float *>(ws + pl.off_dA) : nullptr;
+    p.status = status_ptr();
+    if (!p.status) return fail(SSD_ERR_LAUNCH, "no CUDA device available");
+    if (ssd::tc_scan_supported(p, a->dtype))
+        rc = ssd::launch_scan_tc(p, st);
+    else
+        rc = ssd::launch_scan_generic(p, a->dtype, st);
+    if (rc == 6) return fail(SSD_ERR_UNSUPPORTED, "no GPU kernel for this shape (P=%d N=%d Q=%d)", a->P, a->N, a->Q);
+    if (rc) return fail(SSD_ERR_LAUNCH, "scan launch failed: %s", cudaGetErrorString(cudaGetLastError()));
+    return ok();
+}
+
+int conv_impl(const void *u, int64_t ubs, int64_t urs, const float *w, const float *bias,
+              const void *tail_in, void *tail_out, void *v, int64_t vbs, int64_t vrs,
+              int b, int64_t L, int C_ch, int dtype, cudaStream_t st)
+{
+    if (dtype != SSD_F32 && dtype != SSD_BF16) return fail(SSD_ERR_DTYPE, "unknown dtype %d", dtype);
+    if (b < 0 || L < 0 || C_ch <= 0) return fail(SSD_ERR_SHAPE, "need b >= 0, L >= 0, C_ch > 0");
+    const int vec = (int)(16 / elem_size(dtype));
+    if (C_ch % vec != 0) return fail(SSD_ERR_SHAPE, "C_ch=%d must be a multiple of %d", C_ch, vec);
+    if (b == 0) return ok();
+    int rc;
+    if (L > 0) {
+        if ((rc = check_rows("u", u, ubs, urs, C_ch, b, L, dtype, true))) return rc;
+        if ((rc = check_rows("v", v, vbs, vrs, C_ch, b, L, dtype, true))) return rc;
+        if (!w) return fail(SSD_ERR_NULL, "conv weight w is NULL");
+        if (!aligned16(w)) return fail(SSD_ERR_ALIGN, "conv weight w must be 16-byte aligned");
+    } else if (!u && tail_out) {
+        // tail_out from tail_in only; u is never read
+    }
+    if ((tail_in && !aligned16(tail_in)) || (tail_out && !aligned16(tail_out)))
+        return fail(SSD_ERR_ALIGN, "conv tails must be 16-byte aligned");
+    ssd::ConvParams p{};
+    p.u = u; p.ubs = ubs; p.urs = urs; p.w = w; p.bias = bias; p.tail_in = tail_in;
+    p.tail_out = tail_out; p.v = v; p.vbs = vbs; p.vrs = vrs; p.b = b; p.L = L; p.C_ch = C_ch;
+    rc = ssd::launch_conv(p, dtype, st);
+    if (rc == 2) return fail(SSD_ERR_SHAPE, "conv grid too large");
+    if (rc) return fail(SSD_ERR_LAUNCH, "conv launch failed: %s", cudaGetErrorString(cudaGetLastError()));
+    return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+int ssd_conv_forward(const void *u, int64_t u_batch_stride, int64_t u_row_stride,
+                     const float *w, const float *bias, const void *tail_in, void *tail_out,
+                     void *v, int64_t v_batch_stride, int64_t v_row_stride,
+                     int b, int64_t L, int C_ch, int dtype, ssd_stream_t stream)
+{
+    return conv_impl(u, u_batch_stride, u_row_stride, w, bias, tail_in, tail_out, v,
+                     v_batch_stride, v_row_stride, b, L, C_ch, dtype, (cudaStream_t)stream);
+}
+
+int ssd_scan_forward(const ssd_scan_args *args, ssd_stream_t stream)
+{
+    return scan_impl(args, (cudaStream_t)stream);
+}
+
+size_t ssd_scan_workspace_size(int b, int64_t L, int H, int P, int N, int Q)
+{
+    return make_plan(b, L, H, P, N, Q).bytes;
+}
+
+int ssd_stream_forward(const ssd_stream_args *a, ssd_stream_t stream)
+{
+    if (!a) return fail(SSD_ERR_NULL, "args is NULL");
+    int rc = check_scan_shape(a->dtype, a->b, a->L, a->H, a->P, a->N, a->G, a->Q, a->s);
+    if (rc) return rc;
+    const int d_inner = a->H * a->P;
+    const int C_ch = d_inner + 2 * a->G * a->N;
+    if (a->L > 0 && !a->v) return fail(SSD_ERR_NULL, "v is NULL");
+    rc = conv_impl(a->u, a->u_batch_stride, a->u_row_stride, a->conv_w, a->conv_bias, a->tail_in,
+                   a->tail_out, a->v, a->v_batch_stride, a->v_row_stride, a->b, a->L, C_ch,
+                   a->dtype, (cudaStream_t)stream);
+    if (rc) return rc;
+    const size_t es = elem_size(a->dtype);
+    const char *v = static_cast<const char *>(a->v);
+    ssd_scan_args s{};
+    s.dtype = a->dtype; s.b = a->b; s.L = a->L; s.H = a->H; s.P = a->P; s.N = a->N; s.G = a->G;
+    s.Q = a->Q; s.s = a->s;
+    s.x = v; s.x_batch_stride = a->v_batch_stride; s.x_row_stride = a->v_row_stride;
+    s.B = v ? v + es * d_inner : nullptr;
+    s.B_batch_stride = a->v_batch_stride; s.B_row_stride = a->v_row_stride;
+    s.C = v ? v + es * (d_inner + (size_t)a->G * a->N) : nullptr;
+    s.C_batch_stride = a->v_batch_stride; s.C_row_stride = a->v_row_stride;
+    s.dt = a->dt; s.A = a->A; s.D = a->D; s.h0 = a->h0;
+    s.y = a->y; s.y_batch_stride = a->y_batch_stride; s.y_row_stride = a->y_row_stride;
+    s.h_final = a->h_final; s.h_ckpt = a->h_ckpt;
+    s.workspace = a->workspace; s.workspace_bytes = a->workspace_bytes;
+    return scan_impl(&s, (cudaStream_t)stream);
+}
+
+int ssd_sync_status(ssd_stream_t stream)
+{
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return fail(SSD_ERR_LAUNCH, "CUDA error: %s", cudaGetErrorString(e));
+    unsigned int *sp = status_ptr();
+    if (!sp) return fail(SSD_ERR_LAUNCH, "no CUDA device available");
+    unsigned int v = 0;
+    e = cudaMemcpy(&v, sp, sizeof v, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return fail(SSD_ERR_LAUNCH, "CUDA error: %s", cudaGetErrorString(e));
+    if (v != 0) {
+        const unsigned int zero = 0;
+        cudaMemcpy(sp, &zero, sizeof zero, cudaMemcpyHostToDevice);
+        return fail((int)v, "device status %u (a bounded wait gave up)", v);
+    }
+    return ok();
+}
+
+const char *ssd_last_error_string(void) { return g_last_error.c_str(); }
+
+int ssd_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,87 @@
+// ssd_common.cuh -- types and small device helpers shared by the SSD kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ssd {
+
+// Device status codes latched by kernels (mirrors ssd_status in include/ssd.h).
+enum : unsigned int { kDevOk = 0u, kDevTimeout = 8u };
+
+// Everything a scan kernel needs, passed by value.
+struct ScanParams {
+    int b;
+    int64_t L;
+    int H, P, N, G, Q;
+    int64_t s;
+    const void *x;
+    int64_t xbs, xrs;
+    const void *B;
+    int64_t Bbs, Brs;
+    const void *C;
+    int64_t Cbs, Crs;
+    const float *dt;
+    const float *A;
+    const float *D;
+    const float *h0;
+    void *y;
+    int64_t ybs, yrs;
+    float *h_final;
+    float *h_ckpt;
+    // stripe decomposition of the sequence (see make_plan)
+    int64_t T;          // stripe length in tokens, a multiple of Q
+    int64_t ns;         // number of stripes = ceil(L / T)
+    float *ws_S;        // [b][ns][H][P][N] stripe state from a zero start
+    float *ws_hin;      // [b][ns][H][P][N] exact state entering each stripe
+    float *ws_dA;       // [b][ns][H] sum of dt*A over the stripe
+    unsigned int *status;
+};
+
+struct ConvParams {
+    const void *u;
+    int64_t ubs, urs;
+    const float *w;
+    const float *bias;
+    const void *tail_in;
+    void *tail_out;
+    void *v;
+    int64_t vbs, vrs;
+    int b;
+    int64_t L;
+    int C_ch;
+};
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    __nv_bfloat162 r = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&r);
+}
+
+template <typename T> __device__ __forceinline__ float to_f32(T v);
+template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v)
+{
+    return __bfloat162float(v);
+}
+
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v)
+{
+    return __float2bfloat16_rn(v);
+}
+
+}  // namespace ssd
+
+// Launchers (defined in the .cu files).
+namespace ssd {
+int launch_conv(const ConvParams &p, int dtype, cudaStream_t st);
+int launch_scan_generic(const ScanParams &p, int dtype, cudaStream_t st);
+bool tc_scan_supported(const ScanParams &p, int dtype);
+int launch_scan_tc(const ScanParams &p, cudaStream_t st);
+}  // namespace ssd
