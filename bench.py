@@ -1,0 +1,441 @@
+#!/usr/bin/env python
+"""Benchmark of the SSD mixer forward (conv1d+SiLU then chunked selective scan).
+
+One step = the whole layer over one batch of the workload: by default the
+Video-Ma2mba-0.3B mixer shape (32 heads, P=64, N=128, Q=128, bf16) over a
+1,048,576-token stream processed as 8 consecutive 131072-token segments, each
+resumed from the previous segment's (state, conv tail), with state
+checkpoints every 4096 tokens.  Inputs are seeded synthetic tensors already
+resident in HBM (u alone is 4.8 GB, far larger than the 126 MB L2).
+
+Prints ONE JSON line (rank 0).  Multi-GPU: `torchrun --nproc-per-node N
+bench.py --gpus N`; every rank runs its own independent stream (weak
+scaling, no data-path collective), NCCL only for the barrier and the
+max-over-ranks time.  `--impl reference` times the CPU oracle instead.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import ssd_synth  # noqa: E402
+
+METRIC = "SSD mixer fwd tokens/s at 0.3B shape, L=1M; % of HBM/tensor roofline"
+DEFAULT_WORKLOAD = "mamba2-0.3b-L1M-stream8"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(ssd_synth.BY_NAME))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=131072)
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------- bytes model
+def algorithmic_bytes_per_token(wl):
+    """Minimum HBM bytes per token of the two-call path (conv, then scan)."""
+    e = 2 if wl.dtype == "bf16" else 4
+    conv = 2 * wl.cch * e                              # read u, write v
+    scan = (2 * wl.d_inner * e                         # read x, write y
+            + 2 * wl.G * wl.N * e                      # read B, C
+            + 4 * wl.H                                 # read dt
+            + (4 * wl.H * wl.P * wl.N / wl.s if wl.s else 0))  # write checkpoints
+    return conv, scan
+
+
+# ----------------------------------------------------------------- peaks
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def recorded_traffic(kernel):
+    """DRAM bytes per token of `kernel` from the committed ncu summary, or None
+    when the kernel's source changed since those counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        rec = d[kernel]
+        src = os.path.join(ROOT, rec["source"])
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if digest != rec["source_sha256_16"]:
+            return None
+        return float(rec["dram_bytes_per_token"])
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append({"sm": float(parts[1]), "max": float(parts[2]), "power": float(parts[3]),
+                             "hw": parts[5], "hw_thermal": parts[6], "sw_thermal": parts[7],
+                             "sw_power": parts[8]})
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        loaded = [r for r in rows if r["power"] > 200] or rows
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hw_thermal", "hw_thermal_slowdown"),
+                              ("sw_thermal", "sw_thermal_slowdown"), ("sw_power", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded),
+                "sm_max_mhz": max(r["max"] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows), "samples_under_load": len(loaded)}
+
+
+# ----------------------------------------------------------------- distributed
+def dist_setup(backend=None):
+    """One process per GPU (RANK/LOCAL_RANK/WORLD_SIZE from torchrun).  NCCL on
+    GPUs; gloo when no GPU is present (the CPU tests of the multi-rank logic)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if backend is None:
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def _nccl():
+    import torch.distributed as dist
+    return dist.is_initialized() and dist.get_backend() == "nccl"
+
+
+def barrier(world, local):
+    if world > 1:
+        import torch.distributed as dist
+        if _nccl():
+            dist.barrier(device_ids=[local])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(world, value):
+    """Max of a per-rank scalar (the device time of the timed region)."""
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda" if _nccl() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(wl, rank):
+    """Every rank runs its own independent sequence (weak scaling)."""
+    return wl.seed + 100 * rank
+
+
+def job_throughput(wl, world, steps, ms_max):
+    """Tokens of all ranks over the slowest rank's time."""
+    return wl.tokens * world * steps / (ms_max / 1e3)
+
+
+# ----------------------------------------------------------------- the workload
+class Layer:
+    """Device buffers and one step of the layer for a workload (one rank)."""
+
+    def __init__(self, wl, seed):
+        import mamba_selective_state_causal_b200 as ssd
+        self.ssd = ssd
+        self.wl = wl
+        d = torch.device("cuda", torch.cuda.current_device())
+        self.dev = d
+        prm = ssd_synth.make_params(wl, device=d, seed=seed)
+        self.w, self.bias, self.A, self.D = prm["w"], prm["bias"], prm["A"], prm["D"]
+        self.u = ssd_synth.make_u(wl, device=d, seed=seed)
+        self.dt = ssd_synth.make_dt(wl, prm["dt_bias"], device=d, seed=seed)
+        seg = wl.seg_len
+        self.seg = seg
+        tdt = ssd_synth.torch_dtype(wl.dtype)
+        self.v = torch.empty(wl.b, seg, wl.cch, dtype=tdt, device=d)
+        self.y = torch.empty(wl.b, wl.L, wl.H, wl.P, dtype=tdt, device=d)
+        self.h = torch.empty(wl.b, wl.H, wl.P, wl.N, dtype=torch.float32, device=d)
+        self.tail = torch.empty(wl.b, 3, wl.cch, dtype=tdt, device=d)
+        n_ck = seg // wl.s if wl.s else 0
+        self.ckpt = torch.empty(wl.b, wl.segments * n_ck, wl.H, wl.P, wl.N, dtype=torch.float32, device=d)
+        self.ws = ssd.alloc_workspace(wl.b, seg, wl.H, wl.P, wl.N, wl.Q, d)
+        self.n_ck = n_ck
+
+    def step(self, stream=None):
+        wl, ssd = self.wl, self.ssd
+        for k in range(wl.segments):
+            t0, t1 = k * self.seg, (k + 1) * self.seg
+            ssd.stream_forward(
+                self.u[:, t0:t1], self.w, self.dt[:, t0:t1], self.A, self.D, H=wl.H, P=wl.P, N=wl.N,
+                G=wl.G, Q=wl.Q, s=wl.s, conv_bias=self.bias,
+                tail_in=None if k == 0 else self.tail, tail_out=self.tail,
+                h0=None if k == 0 else self.h, h_final=self.h, v=self.v, y=self.y[:, t0:t1],
+                h_ckpt=self.ckpt[:, k * self.n_ck:(k + 1) * self.n_ck] if self.n_ck else None,
+                workspace=self.ws, stream=stream)
+
+
+def time_steps(fn, steps, warmup, world, local):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(world, local)
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(steps):
+        fn()
+    e1.record(st)
+    torch.cuda.synchronize()
+    barrier(world, local)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def cpu_baseline(wl, sample_tokens):
+    """The CPU oracle (as it stands) on a bounded sample of the same workload."""
+    import oracle
+    sw = ssd_synth.scaled(wl, L=sample_tokens, b=1, segments=1)
+    prm = ssd_synth.make_params(sw)
+    u = ssd_synth.make_u(sw).float().numpy()
+    dt = ssd_synth.make_dt(sw, prm["dt_bias"]).numpy()
+    args = (u, prm["w"].numpy(), dt, prm["A"].numpy(), prm["D"].numpy(), prm["bias"].numpy())
+    t0 = time.perf_counter()
+    oracle.layer(*args, None, None, H=sw.H, P=sw.P, N=sw.N, G=sw.G, s=sw.s,
+                 io_round="bf16" if sw.dtype == "bf16" else "f32", want_ckpt=True)
+    el = time.perf_counter() - t0
+    return {"value": sample_tokens / el, "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{wl.name} shape, first {sample_tokens} tokens of one sequence, all {wl.H} heads, "
+                      f"conv1d+SiLU then the per-token recurrence in fp64 ({el:.1f} s)"}
+
+
+def run_reference(args, wl, world, rank):
+    """--impl reference: the CPU oracle timed per step on a bounded sample."""
+    if rank != 0:
+        return
+    import oracle
+    sample = min(16384, wl.seg_len)
+    sw = ssd_synth.scaled(wl, L=sample, b=1, segments=1)
+    prm = ssd_synth.make_params(sw)
+    u = ssd_synth.make_u(sw).float().numpy()
+    dt = ssd_synth.make_dt(sw, prm["dt_bias"]).numpy()
+
+    def step():
+        oracle.layer(u, prm["w"].numpy(), dt, prm["A"].numpy(), prm["D"].numpy(), prm["bias"].numpy(),
+                     None, None, H=sw.H, P=sw.P, N=sw.N, G=sw.G, s=sw.s, io_round="bf16")
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    value = sample * args.steps / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "sample_tokens_per_step": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"{wl.name} shape, {sample} tokens of one sequence per step, all heads"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_e2e(layer, steps=3):
+    """Same metric through the library with host buffers: inputs copied in from
+    pinned host memory and the outputs copied back, every step."""
+    wl = layer.wl
+    st = torch.cuda.current_stream()
+    h_u = torch.empty(layer.u.shape, dtype=layer.u.dtype, pin_memory=True)
+    h_dt = torch.empty(layer.dt.shape, dtype=layer.dt.dtype, pin_memory=True)
+    h_u.copy_(layer.u)
+    h_dt.copy_(layer.dt)
+    o_y = torch.empty(layer.y.shape, dtype=layer.y.dtype, pin_memory=True)
+    o_h = torch.empty(layer.h.shape, dtype=layer.h.dtype, pin_memory=True)
+    o_ck = torch.empty(layer.ckpt.shape, dtype=layer.ckpt.dtype, pin_memory=True)
+
+    def step():
+        layer.u.copy_(h_u, non_blocking=True)
+        layer.dt.copy_(h_dt, non_blocking=True)
+        layer.step()
+        o_y.copy_(layer.y, non_blocking=True)
+        o_h.copy_(layer.h, non_blocking=True)
+        o_ck.copy_(layer.ckpt, non_blocking=True)
+    step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(steps):
+        step()
+    e1.record(st)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    h2d = h_u.numel() * h_u.element_size() + h_dt.numel() * h_dt.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in (o_y, o_h, o_ck))
+    return {"value": wl.tokens / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}
+
+
+def main():
+    args = parse_args()
+    wl = ssd_synth.BY_NAME[args.workload]
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        run_reference(args, wl, world, rank)
+        return
+    import __graft_entry__
+    __graft_entry__.build()
+    layer = Layer(wl, seed=rank_seed(wl, rank))
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    ms = time_steps(layer.step, args.steps, args.warmup, world, local)
+    clk = clocks.stop()
+    layer.ssd.sync_status()
+    ms = max_over_ranks(world, ms)
+    ms_step = ms / args.steps
+    value = job_throughput(wl, world, args.steps, ms)
+
+    # per-kernel times over a second, profiled pass of the same steps
+    layer.ssd.profile_begin()
+    prof_steps = min(args.steps, 5)
+    for _ in range(prof_steps):
+        layer.step()
+    torch.cuda.synchronize()
+    prof = layer.ssd.profile_end()
+    launches_per_step = sum(v["launches"] for v in prof.values()) / prof_steps
+
+    conv_b, scan_b = algorithmic_bytes_per_token(wl)
+    peak, peak_src = hbm_peak()
+    per_launch = {k: v["total_ms"] / v["launches"] for k, v in prof.items()}
+    dom = max(prof, key=lambda k: prof[k]["total_ms"])
+    tokens_per_launch = {
+        "conv1d_silu": wl.b * wl.seg_len, "chunk_output_tc": wl.b * wl.seg_len,
+        "chunk_output_generic": wl.b * wl.seg_len, "stripe_state_tc": wl.b * wl.seg_len,
+        "stripe_state_generic": wl.b * wl.seg_len}
+    alg_per_token = {"conv1d_silu": conv_b, "chunk_output_tc": scan_b, "chunk_output_generic": scan_b,
+                     # pass A's own necessary reads: x, B, dt
+                     "stripe_state_tc": 2 * wl.d_inner + 2 * wl.G * wl.N + 4 * wl.H,
+                     "stripe_state_generic": 2 * wl.d_inner + 2 * wl.G * wl.N + 4 * wl.H}
+    dom_alg = alg_per_token.get(dom, 0) * tokens_per_launch.get(dom, 0)
+    achieved = dom_alg / (per_launch[dom] / 1e3) / 1e9
+    traffic_pt = recorded_traffic(dom)
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_source": peak_src,
+                "traffic": None if traffic_pt is None else traffic_pt * tokens_per_launch.get(dom, 0),
+                "algorithmic_bytes_per_launch": dom_alg}
+    step_bytes = (conv_b + scan_b) * wl.tokens
+    step_frac = step_bytes / (ms_step / 1e3) / 1e9 / peak
+    kernels = {k: {"launches_per_step": v["launches"] / prof_steps, "ms_per_launch": per_launch[k],
+                   "share": v["total_ms"] / sum(x["total_ms"] for x in prof.values())}
+               for k, v in prof.items()}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, args.cpu_sample_tokens)
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(layer)
+        if world > 1:
+            e2e_ms = max_over_ranks(world, e2e["ms_per_step"])
+            e2e["value"] = wl.tokens * world / (e2e_ms / 1e3)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.b, "seq_len": wl.L, "segments": wl.segments,
+                   "heads": wl.H, "headdim": wl.P, "d_state": wl.N, "chunk": wl.Q,
+                   "ckpt_stride": wl.s, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (u alone %.1f GB)" % (layer.u.numel() * 2 / 1e9)},
+        "roofline": roofline,
+        "step_roofline": {"bound": "hbm", "algorithmic_bytes_per_token": conv_b + scan_b,
+                          "achieved": step_bytes / (ms_step / 1e3) / 1e9, "peak": peak, "frac": step_frac},
+        "kernels": kernels,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": int(round(launches_per_step * args.steps)),
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -187,6 +187,25 @@ SSD_API int ssd_stream_forward(const ssd_stream_args *args, ssd_stream_t stream)
  */
 SSD_API int ssd_sync_status(ssd_stream_t stream);
 
+/*
+ * Per-kernel timing (tracing).  Between ssd_profile_begin() and
+ * ssd_profile_end(), every kernel this library launches from the calling
+ * host thread is bracketed by two CUDA events recorded on the launch stream.
+ * ssd_profile_end() waits for those events and fills `out` (up to
+ * `capacity` entries; *count receives the number of distinct kernels) with
+ * the launch count and the summed event time of each kernel, by name.  The
+ * names are static strings owned by the library.  Profiling adds two event
+ * records per launch; time the workload without it when the total matters.
+ */
+typedef struct ssd_kernel_stat {
+    const char *name;
+    int64_t launches;
+    double total_ms;
+} ssd_kernel_stat;
+
+SSD_API int ssd_profile_begin(void);
+SSD_API int ssd_profile_end(ssd_kernel_stat *out, int capacity, int *count);
+
 /* Description of the last error on this host thread ("" if none). */
 SSD_API const char *ssd_last_error_string(void);
 

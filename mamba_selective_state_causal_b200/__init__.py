@@ -28,6 +28,10 @@ class SSDError(RuntimeError):
         self.code = code
 
 
+class KernelStat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char_p), ("launches", _i64), ("total_ms", ctypes.c_double)]
+
+
 class ScanArgs(ctypes.Structure):
     _fields_ = [("dtype", ctypes.c_int), ("b", ctypes.c_int), ("L", _i64),
                 ("H", ctypes.c_int), ("P", ctypes.c_int), ("N", ctypes.c_int),
@@ -81,6 +85,11 @@ def lib():
         L.ssd_last_error_string.restype = ctypes.c_char_p
         L.ssd_version.argtypes = []
         L.ssd_version.restype = ctypes.c_int
+        L.ssd_profile_begin.argtypes = []
+        L.ssd_profile_begin.restype = ctypes.c_int
+        L.ssd_profile_end.argtypes = [ctypes.POINTER(KernelStat), ctypes.c_int,
+                                      ctypes.POINTER(ctypes.c_int)]
+        L.ssd_profile_end.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -127,6 +136,21 @@ def workspace_size(b, L, H, P, N, Q):
 def alloc_workspace(b, L, H, P, N, Q, device=None):
     n = workspace_size(b, L, H, P, N, Q)
     return torch.empty(max(n, 1), dtype=torch.uint8, device=device or "cuda")
+
+
+def profile_begin():
+    """Start timing every kernel the library launches from this thread."""
+    _check(lib().ssd_profile_begin())
+
+
+def profile_end():
+    """Stop timing; returns {kernel name: {"launches": n, "total_ms": t}}."""
+    cap = 32
+    arr = (KernelStat * cap)()
+    n = ctypes.c_int(0)
+    _check(lib().ssd_profile_end(arr, cap, ctypes.byref(n)))
+    return {arr[i].name.decode(): {"launches": int(arr[i].launches), "total_ms": float(arr[i].total_ms)}
+            for i in range(min(n.value, cap))}
 
 
 def sync_status(stream=None):

@@ -13,7 +13,7 @@ namespace ssd {
 namespace {
 
 constexpr int kTokensPerThread = 64;
-constexpr int kUnroll = 8;
+constexpr int kUnroll = 4;
 
 struct alignas(16) Vec16 { uint32_t w[4]; };
 
@@ -64,7 +64,7 @@ template <> struct VecIO<float> {
 };
 
 template <typename T>
-__global__ void __launch_bounds__(256) conv1d_silu_kernel(ConvParams p, int64_t n_tblk)
+__global__ void __launch_bounds__(256, 2) conv1d_silu_kernel(ConvParams p, int64_t n_tblk)
 {
     using IO = VecIO<T>;
     constexpr int V = IO::kN;
@@ -171,11 +171,15 @@ int launch_conv_t(const ConvParams &p, cudaStream_t st)
         const int64_t threads = (int64_t)p.b * n_tblk * (p.C_ch / V);
         const int64_t blocks = (threads + 255) / 256;
         if (blocks > 0x7fffffffLL) return 2;
+        prof_begin(st, kKConv);
         conv1d_silu_kernel<T><<<(unsigned)blocks, 256, 0, st>>>(p, n_tblk);
+        prof_end(st, kKConv);
     }
     if (p.tail_out && p.b > 0) {
         const int64_t n = (int64_t)p.b * p.C_ch;
+        prof_begin(st, kKConvTail);
         conv_tail_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p);
+        prof_end(st, kKConvTail);
     }
     return cudaGetLastError() == cudaSuccess ? 0 : 7;
 }

@@ -23,6 +23,7 @@
 #include "ssd_common.cuh"
 
 namespace ssd {
+int launch_chain(const ScanParams &p, cudaStream_t st);
 namespace {
 
 constexpr int kThreads = 256;
@@ -238,15 +239,28 @@ int launch_t(const ScanParams &p, cudaStream_t st)
     if (p.ns > 65535 || p.H > 65535 || p.b > 65535) return 6;
     const dim3 grid((unsigned)p.ns, (unsigned)p.H, (unsigned)p.b);
     if (p.ns > 1) {
+        prof_begin(st, kKStateGeneric);
         stripe_state_kernel<T><<<grid, kThreads, smA, st>>>(p);
-        const dim3 gchain((unsigned)((P * N + kThreads - 1) / kThreads), (unsigned)p.H, (unsigned)p.b);
-        stripe_chain_kernel<<<gchain, kThreads, 0, st>>>(p);
+        prof_end(st, kKStateGeneric);
+        const int rc = launch_chain(p, st);
+        if (rc) return rc;
     }
+    prof_begin(st, kKOutputGeneric);
     chunk_output_kernel<T><<<grid, kThreads, smC, st>>>(p);
+    prof_end(st, kKOutputGeneric);
     return cudaGetLastError() == cudaSuccess ? 0 : 7;
 }
 
 }  // namespace
+
+int launch_chain(const ScanParams &p, cudaStream_t st)
+{
+    const dim3 g((unsigned)((p.P * p.N + kThreads - 1) / kThreads), (unsigned)p.H, (unsigned)p.b);
+    prof_begin(st, kKChain);
+    stripe_chain_kernel<<<g, kThreads, 0, st>>>(p);
+    prof_end(st, kKChain);
+    return cudaGetLastError() == cudaSuccess ? 0 : 7;
+}
 
 int launch_scan_generic(const ScanParams &p, int dtype, cudaStream_t st)
 {

@@ -2,8 +2,10 @@
 // stripe plan, workspace carving and dispatch to the CUDA kernels.
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <string>
+#include <vector>
 
 #include "../../include/ssd.h"
 #include "ssd_common.cuh"
@@ -161,10 +163,19 @@ int scan_impl(const ssd_scan_args *a, cudaStream_t st)
     p.ws_dA = pl.bytes ? reinterpret_cast<float *>(ws + pl.off_dA) : nullptr;
     p.status = status_ptr();
     if (!p.status) return fail(SSD_ERR_LAUNCH, "no CUDA device available");
-    if (ssd::tc_scan_supported(p, a->dtype))
-        rc = ssd::launch_scan_tc(p, st);
-    else
-        rc = ssd::launch_scan_generic(p, a->dtype, st);
+    {
+        const char *lim = getenv("SSD_WAIT_LIMIT_MS");
+        const long long ms = lim ? atoll(lim) : 2000;
+        p.wait_limit_ns = (uint64_t)(ms > 0 ? ms : 2000) * 1000000ull;
+        const char *drop = getenv("SSD_TEST_DROP_UNIT");
+        p.test_drop_unit = drop ? atoll(drop) : -1;
+    }
+    // SSD_SCAN_PATH=generic forces the CUDA-core kernels (used to cross-check the paths)
+    const char *path = getenv("SSD_SCAN_PATH");
+    const bool force_generic = path && strcmp(path, "generic") == 0;
+    rc = 6;
+    if (!force_generic && ssd::tc_scan_supported(p, a->dtype)) rc = ssd::launch_scan_tc(p, st);
+    if (rc == 6) rc = ssd::launch_scan_generic(p, a->dtype, st);
     if (rc == 6) return fail(SSD_ERR_UNSUPPORTED, "no GPU kernel for this shape (P=%d N=%d Q=%d)", a->P, a->N, a->Q);
     if (rc) return fail(SSD_ERR_LAUNCH, "scan launch failed: %s", cudaGetErrorString(cudaGetLastError()));
     return ok();
@@ -199,9 +210,90 @@ int conv_impl(const void *u, int64_t ubs, int64_t urs, const float *w, const flo
     return ok();
 }
 
+// ---------------------------------------------------------------- kernel timing
+const char *const kKernelNames[ssd::kKCount] = {
+    "conv1d_silu", "conv_tail", "stripe_state_tc", "stripe_chain", "chunk_output_tc",
+    "stripe_state_generic", "chunk_output_generic"};
+
+struct ProfRecord {
+    int id;
+    cudaEvent_t a, b;
+};
+
+struct ProfState {
+    bool on = false;
+    std::vector<ProfRecord> recs;
+    std::vector<cudaEvent_t> pool;
+    cudaEvent_t pending = nullptr;
+    cudaEvent_t take()
+    {
+        if (!pool.empty()) {
+            cudaEvent_t e = pool.back();
+            pool.pop_back();
+            return e;
+        }
+        cudaEvent_t e = nullptr;
+        cudaEventCreate(&e);
+        return e;
+    }
+};
+
+thread_local ProfState g_prof;
+
 }  // namespace
 
+namespace ssd {
+void prof_begin(cudaStream_t st, int)
+{
+    if (!g_prof.on) return;
+    g_prof.pending = g_prof.take();
+    cudaEventRecord(g_prof.pending, st);
+}
+void prof_end(cudaStream_t st, int id)
+{
+    if (!g_prof.on || !g_prof.pending) return;
+    cudaEvent_t e = g_prof.take();
+    cudaEventRecord(e, st);
+    g_prof.recs.push_back({id, g_prof.pending, e});
+    g_prof.pending = nullptr;
+}
+}  // namespace ssd
+
 extern "C" {
+
+int ssd_profile_begin(void)
+{
+    for (auto &r : g_prof.recs) { g_prof.pool.push_back(r.a); g_prof.pool.push_back(r.b); }
+    g_prof.recs.clear();
+    g_prof.on = true;
+    return ok();
+}
+
+int ssd_profile_end(ssd_kernel_stat *out, int capacity, int *count)
+{
+    g_prof.on = false;
+    int64_t launches[ssd::kKCount] = {0};
+    double ms[ssd::kKCount] = {0};
+    for (auto &r : g_prof.recs) {
+        float t = 0.0f;
+        cudaError_t e = cudaEventSynchronize(r.b);
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&t, r.a, r.b);
+        if (e != cudaSuccess) return fail(SSD_ERR_LAUNCH, "profiling events: %s", cudaGetErrorString(e));
+        launches[r.id] += 1;
+        ms[r.id] += t;
+    }
+    int n = 0;
+    for (int i = 0; i < ssd::kKCount; ++i) {
+        if (!launches[i]) continue;
+        if (out && n < capacity) out[n] = ssd_kernel_stat{kKernelNames[i], launches[i], ms[i]};
+        ++n;
+    }
+    if (count) *count = n;
+    for (auto &r : g_prof.recs) { g_prof.pool.push_back(r.a); g_prof.pool.push_back(r.b); }
+    g_prof.recs.clear();
+    return ok();
+}
+
 
 int ssd_conv_forward(const void *u, int64_t u_batch_stride, int64_t u_row_stride,
                      const float *w, const float *bias, const void *tail_in, void *tail_out,

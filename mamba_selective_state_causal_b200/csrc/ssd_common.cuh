@@ -37,6 +37,11 @@ struct ScanParams {
     float *ws_hin;      // [b][ns][H][P][N] exact state entering each stripe
     float *ws_dA;       // [b][ns][H] sum of dt*A over the stripe
     unsigned int *status;
+    // bounded waits give up after this many nanoseconds (SSD_WAIT_LIMIT_MS)
+    uint64_t wait_limit_ns;
+    // failure-detection test hook (SSD_TEST_DROP_UNIT): the work unit whose
+    // loads are never issued, so that its waits run out; -1 = none
+    int64_t test_drop_unit;
 };
 
 struct ConvParams {
@@ -76,10 +81,15 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(v);
 }
 
-}  // namespace ssd
+// Kernel timing hooks (ssd_api.cu): no-ops unless ssd_profile_begin() is active
+// on the calling thread.
+enum KernelId : int {
+    kKConv = 0, kKConvTail, kKStateTc, kKChain, kKOutputTc, kKStateGeneric, kKOutputGeneric, kKCount
+};
+void prof_begin(cudaStream_t st, int id);
+void prof_end(cudaStream_t st, int id);
 
 // Launchers (defined in the .cu files).
-namespace ssd {
 int launch_conv(const ConvParams &p, int dtype, cudaStream_t st);
 int launch_scan_generic(const ScanParams &p, int dtype, cudaStream_t st);
 bool tc_scan_supported(const ScanParams &p, int dtype);

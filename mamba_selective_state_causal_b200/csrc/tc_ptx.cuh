@@ -58,8 +58,9 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
 }
 
 // Wait for phase `parity` of `bar`, giving up after `limit_ns` nanoseconds or
-// as soon as *abort is set by another thread of the CTA.  Returns false when
-// it gave up; the caller then raises the CTA abort flag and unwinds.
+// as soon as *abort is set by another thread of the CTA (abort may be NULL:
+// no early exit, used when draining work in flight).  Returns false when it
+// gave up; the caller then raises the CTA abort flag and unwinds.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                           uint64_t limit_ns = 2000000000ull)
 {
@@ -67,7 +68,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (*abort) return false;
+        if (abort && *abort) return false;
         if (globaltimer_ns() - t0 > limit_ns) return false;
     }
 }

@@ -91,7 +91,7 @@ def test_03b_L16k_workload_all_heads():
 @pytest.mark.parametrize("segments", [2, 8])
 def test_streamed_segments_equal_unsplit(segments):
     """Split/resume invariant: consecutive resumed calls reproduce the unsplit layer."""
-    wl = ssd_synth.scaled(W[2], L=8 * 2048, H=4)
+    wl = ssd_synth.scaled(W[2], L=8 * 2048, H=4, s=1024)
     prm = ssd_synth.make_params(wl)
     u = ssd_synth.make_u(wl)
     dt = ssd_synth.make_dt(wl, prm["dt_bias"])

@@ -112,3 +112,15 @@ def test_scan_linearity_in_h0():
                                 (2 * ha).to(d), H=wl.H, Q=wl.Q, s=0)
     ssd.sync_status()
     assert rel_l2(host(y2), 2 * host(ya)) < 1e-6
+
+
+def test_tensor_core_path_matches_cuda_core_path(monkeypatch):
+    """The tcgen05 path (bf16, P=64, N=128, Q=128) and the CUDA-core path agree,
+    and both stay within tolerance of the oracle."""
+    wl = ssd_synth.scaled(W[1], L=3000, H=4, b=2)
+    fast, ref = run_case(wl)
+    monkeypatch.setenv("SSD_SCAN_PATH", "generic")
+    slow, _ = run_case(wl)
+    check_outputs(fast, ref, TOL["bf16"])
+    check_outputs(slow, ref, TOL["bf16"])
+    assert rel_l2(host(fast["y"]), host(slow["y"])) < 1e-2
