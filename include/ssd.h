@@ -180,6 +180,31 @@ typedef struct ssd_stream_args {
 SSD_API int ssd_stream_forward(const ssd_stream_args *args, ssd_stream_t stream);
 
 /*
+ * ssd_scan_forward_static_scratch -- ssd_scan_forward for callers that cannot
+ * allocate device memory.  (The pages have no counterpart: this is a
+ * deployment aid of this library, not part of the layer they describe.)
+ *
+ * ssd_scan_forward needs a caller-allocated `workspace`.  Callers that may not
+ * call cudaMalloc (a memory pool that forbids new allocations, plugin code
+ * that is handed only its input and output buffers, code that must not risk
+ * the device synchronisation or out-of-memory failure an allocation can
+ * bring) use this variant instead: the scratch comes from a fixed 80 MiB array
+ * compiled into the library.  The `workspace` fields of `args` are ignored;
+ * all other arguments, results and errors are those of ssd_scan_forward.
+ *  - Every GPU that loads the library holds those 80 MiB until process exit.
+ *  - A shape whose ssd_scan_workspace_size() exceeds 80 MiB is rejected with
+ *    SSD_ERR_WORKSPACE before anything is launched.
+ *  - The first call on each device looks up the array's device address, with
+ *    that device current; make that first call before any stream capture.
+ *  - All calls on a device share the array, which keeps the last call's
+ *    contents (each call writes every element it reads, so nothing needs to
+ *    start at zero).  Calls whose kernels overlap on the GPU race on it:
+ *    serialise them (one stream, or synchronise between streams).
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ */
+SSD_API int ssd_scan_forward_static_scratch(const ssd_scan_args *args, ssd_stream_t stream);
+
+/*
  * ssd_sync_status -- synchronise `stream`, then return SSD_ERR_LAUNCH if the
  * CUDA runtime reports an error, else the device status word latched by
  * this library's kernels on the current device (SSD_OK or SSD_ERR_TIMEOUT),

@@ -85,6 +85,8 @@ def lib():
         L.ssd_last_error_string.restype = ctypes.c_char_p
         L.ssd_version.argtypes = []
         L.ssd_version.restype = ctypes.c_int
+        L.ssd_scan_forward_static_scratch.argtypes = [ctypes.POINTER(ScanArgs), _vp]
+        L.ssd_scan_forward_static_scratch.restype = ctypes.c_int
         L.ssd_profile_begin.argtypes = []
         L.ssd_profile_begin.restype = ctypes.c_int
         L.ssd_profile_end.argtypes = [ctypes.POINTER(KernelStat), ctypes.c_int,

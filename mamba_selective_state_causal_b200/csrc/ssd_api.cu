@@ -243,6 +243,8 @@ thread_local ProfState g_prof;
 }  // namespace
 
 namespace ssd {
+int set_error(int code, const char *msg) { return fail(code, "%s", msg); }
+
 void prof_begin(cudaStream_t st, int)
 {
     if (!g_prof.on) return;
