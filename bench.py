@@ -46,6 +46,9 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=131072)
+    # profiling aids: run a shorter stream of the same shape (not a bench line)
+    ap.add_argument("--seq-len", type=int, default=None)
+    ap.add_argument("--segments", type=int, default=None)
     return ap.parse_args()
 
 
@@ -351,6 +354,9 @@ def run_e2e(layer, steps=3):
 def main():
     args = parse_args()
     wl = ssd_synth.BY_NAME[args.workload]
+    if args.seq_len or args.segments:
+        wl = ssd_synth.scaled(wl, L=args.seq_len or wl.L, segments=args.segments or wl.segments,
+                              name=wl.name + f"-profile-L{args.seq_len or wl.L}")
     world, rank, local = dist_setup()
     if args.impl == "reference":
         run_reference(args, wl, world, rank)

@@ -120,11 +120,16 @@ __device__ __forceinline__ void raise_timeout(const ScanParams &p, volatile int 
 }
 
 // =============================================================== pass A
+// Two heads per CTA: S^T[(h,p)][n] = sum_j (w_h o X_h)[j][p] B[j][n] for the
+// head pair, accumulated in TMEM over the whole stripe (M = 128 rows = 2 heads
+// x 64, N = 128 as two N=64 halves).  Chunks are walked backwards so that the
+// decay from each chunk to the stripe end (a suffix sum) is known when the
+// chunk is scaled.
 struct SmemA {
-    uint8_t stage[3][3 * kBox + kDtBox];  // B (two boxes), X, dt
-    uint8_t xw[2][kBox];
-    float scratch[2][4];
-    uint64_t full[3], empty[3], xw_full[2], xw_empty[2], acc_full, fin, epi;
+    uint8_t stage[2][4 * kBox + kDtBox];  // B (two boxes), X of head h0, X of head h1, dt
+    uint8_t xw[2][2 * kBox];              // w o X for both heads (h0 box, h1 box)
+    float scratch[2][8];
+    uint64_t full[2], empty[2], xw_full[2], xw_empty[2], acc_full, fin, epi;
     uint32_t tmem;
     int abort;
 };
@@ -136,17 +141,23 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
     SmemA &s = *reinterpret_cast<SmemA *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t unit = blockIdx.x;
-    const int h = (int)(unit % p.H);
-    const int64_t k = (unit / p.H) % p.ns;
-    const int bi = (int)(unit / ((int64_t)p.H * p.ns));
-    const int g = (int)((int64_t)h * p.G / p.H);
+    const int hpairs = p.H / 2;
+    const int h0 = 2 * (int)(unit % hpairs);
+    const int64_t k = (unit / hpairs) % p.ns;
+    const int bi = (int)(unit / ((int64_t)hpairs * p.ns));
+    const int g = (int)((int64_t)h0 * p.G / p.H);  // both heads of the pair share a group (H/G even)
     const int64_t s0 = k * p.T;
     const int64_t s1 = min(p.L, s0 + p.T);
     const int nc = (int)((s1 - s0 + kQ - 1) / kQ);
+    const uint64_t lim = p.wait_limit_ns;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 3; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], 1 + 128); }
-        for (int i = 0; i < 2; ++i) { mbar_init(&s.xw_full[i], 128); mbar_init(&s.xw_empty[i], 1); }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s.full[i], 1);
+            mbar_init(&s.empty[i], 1 + 128);
+            mbar_init(&s.xw_full[i], 128);
+            mbar_init(&s.xw_empty[i], 1);
+        }
         mbar_init(&s.acc_full, 1);
         mbar_init(&s.fin, 1);
         mbar_init(&s.epi, 128);
@@ -158,7 +169,7 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
         prefetch_tmap(&maps.B);
         prefetch_tmap(&maps.dt);
     }
-    if (warp == 1) { tmem_alloc(&s.tmem, 64); tmem_relinquish(); }
+    if (warp == 1) { tmem_alloc(&s.tmem, 128); tmem_relinquish(); }
     __syncthreads();
     tc_fence_after();
     const uint32_t tS = s.tmem;
@@ -168,42 +179,43 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
         if (lane == 0) {
             int issued = 0;
             for (int it = 0; it < nc; ++it) {
-                const int st = it % 3, u = it / 3;
-                if (it >= 3 && !mbar_wait(&s.empty[st], (u - 1) & 1, abort, p.wait_limit_ns)) { raise_timeout(p, abort); break; }
+                const int st = it & 1, u = it >> 1;
+                if (it >= 2 && !mbar_wait(&s.empty[st], (u - 1) & 1, abort, lim)) { raise_timeout(p, abort); break; }
                 if (unit == p.test_drop_unit) break;  // test hook: this unit's loads never arrive
                 const int c = nc - 1 - it;  // chunks in reverse order
                 const int t0 = (int)(s0 + (int64_t)c * kQ);
                 uint8_t *sb = s.stage[st];
-                mbar_arrive_expect_tx(&s.full[st], 3 * kBox + kDtBox);
+                mbar_arrive_expect_tx(&s.full[st], 4 * kBox + kDtBox);
                 tma_load_3d(sb, &maps.B, &s.full[st], g * kN, t0, bi);
                 tma_load_3d(sb + kBox, &maps.B, &s.full[st], g * kN + 64, t0, bi);
-                tma_load_3d(sb + 2 * kBox, &maps.x, &s.full[st], h * kP, t0, bi);
-                tma_load_3d(sb + 3 * kBox, &maps.dt, &s.full[st], h & ~3, t0, bi);
+                tma_load_3d(sb + 2 * kBox, &maps.x, &s.full[st], h0 * kP, t0, bi);
+                tma_load_3d(sb + 3 * kBox, &maps.x, &s.full[st], (h0 + 1) * kP, t0, bi);
+                tma_load_3d(sb + 4 * kBox, &maps.dt, &s.full[st], h0 & ~3, t0, bi);
                 issued = it + 1;
             }
             if (*abort) {  // let copies in flight land before the CTA exits
-                for (int it = max(0, issued - 3); it < issued; ++it)
-                    mbar_wait(&s.full[it % 3], (it / 3) & 1, nullptr, 100000000ull);
+                for (int it = max(0, issued - 2); it < issued; ++it)
+                    mbar_wait(&s.full[it & 1], (it >> 1) & 1, nullptr, 100000000ull);
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t id = idesc_bf16(128, 64, 1, 1);
-            bool okk = true;
-            for (int it = 0; it < nc && okk; ++it) {
-                const int st = it % 3, u = it / 3, xb = it & 1;
-                if (!mbar_wait(&s.full[st], u & 1, abort, p.wait_limit_ns) || !mbar_wait(&s.xw_full[xb], (it >> 1) & 1, abort, p.wait_limit_ns)) {
+            for (int it = 0; it < nc; ++it) {
+                const int st = it & 1, u = it >> 1, xb = it & 1;
+                if (!mbar_wait(&s.full[st], u & 1, abort, lim) || !mbar_wait(&s.xw_full[xb], (it >> 1) & 1, abort, lim)) {
                     raise_timeout(p, abort);
-                    okk = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t sB = smem_u32(s.stage[st]);
                 const uint32_t sXw = smem_u32(s.xw[xb]);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tS, smem_desc(sB + kk * 2048, kBox, 1024), smem_desc(sXw + kk * 2048, 0, 1024), id,
-                           it > 0 || kk > 0);
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t da = smem_desc(sXw + kk * 2048, kBox, 1024);  // rows (h,p): two atoms
+                    mma_ss(tS, da, smem_desc(sB + kk * 2048, 0, 1024), id, it > 0 || kk > 0);
+                    mma_ss(tS + 64, da, smem_desc(sB + kBox + kk * 2048, 0, 1024), id, it > 0 || kk > 0);
+                }
                 mma_commit(&s.empty[st]);
                 mma_commit(&s.xw_empty[xb]);
             }
@@ -212,98 +224,126 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
             mbar_wait(&s.fin, 0, nullptr, 200000000ull);
         }
     } else {
-        const int r = 32 * (warp & 3) + lane;  // token row / TMEM lane
-        const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-        const float A2 = p.A[h] * kLog2e;
-        float suf2 = 0.0f;
+        const int q = warp & 3;
+        const int r = 32 * q + lane;  // token row j; TMEM lane (h,p) for the result
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        const float A2a = p.A[h0] * kLog2e, A2b = p.A[h0 + 1] * kLog2e;
+        float sufa = 0.0f, sufb = 0.0f;
         bool okk = true;
         uint32_t eph = 0;
         for (int it = 0; it < nc; ++it) {
-            const int st = it % 3, u = it / 3, xb = it & 1;
-            if (!ewait(&s.full[st], u & 1, abort, p.wait_limit_ns)) { raise_timeout(p, abort); okk = false; break; }
+            const int st = it & 1, u = it >> 1, xb = it & 1;
+            if (!ewait(&s.full[st], u & 1, abort, lim)) { raise_timeout(p, abort); okk = false; break; }
             const uint8_t *sb = s.stage[st];
-            const float dt_r = reinterpret_cast<const float *>(sb + 3 * kBox)[r * 4 + (h & 3)];
-            float tot2, cs2 = dt_r * A2;
-            if (!epi_scan(cs2, r, s.scratch[it & 1], tot2, &s.epi, eph, abort, p.wait_limit_ns)) {
-                raise_timeout(p, abort);
-                okk = false;
-                break;
-            }
-            const float w = dt_r * ex2((tot2 - cs2) + suf2);
-            if (it >= 2 && !ewait(&s.xw_empty[xb], ((it >> 1) - 1) & 1, abort, p.wait_limit_ns)) {
-                raise_timeout(p, abort);
-                okk = false;
-                break;
-            }
-            const uint8_t *xrow = sb + 2 * kBox;
-            uint8_t *xwt = s.xw[xb];
+            const float *dtrow = reinterpret_cast<const float *>(sb + 4 * kBox) + r * 4 + (h0 & 3);
+            const float dta = dtrow[0], dtb = dtrow[1];
+            float va = dta * A2a, vb = dtb * A2b;
+            const int lq = r & 31;
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-                const uint32_t o = swz(r, cc);
-                uint4 v = lds128(xrow + o);
-                v.x = scale_bf16x2(v.x, w); v.y = scale_bf16x2(v.y, w);
-                v.z = scale_bf16x2(v.z, w); v.w = scale_bf16x2(v.w, w);
-                sts128(xwt + o, v);
+            for (int o = 1; o < 32; o <<= 1) {
+                const float ta = __shfl_up_sync(0xffffffffu, va, o);
+                const float tb = __shfl_up_sync(0xffffffffu, vb, o);
+                if (lq >= o) { va += ta; vb += tb; }
+            }
+            float *scr = s.scratch[it & 1];
+            if (lq == 31) { scr[q] = va; scr[4 + q] = vb; }
+            if (!epi_sync(&s.epi, eph, abort, lim)) { raise_timeout(p, abort); okk = false; break; }
+            float prea = 0.0f, preb = 0.0f;
+            if (q > 0) { prea += scr[0]; preb += scr[4]; }
+            if (q > 1) { prea += scr[1]; preb += scr[5]; }
+            if (q > 2) { prea += scr[2]; preb += scr[6]; }
+            const float tota = ((scr[0] + scr[1]) + scr[2]) + scr[3];
+            const float totb = ((scr[4] + scr[5]) + scr[6]) + scr[7];
+            const float wa = dta * ex2((tota - (va + prea)) + sufa);
+            const float wb = dtb * ex2((totb - (vb + preb)) + sufb);
+            if (it >= 2 && !ewait(&s.xw_empty[xb], ((it >> 1) - 1) & 1, abort, lim)) {
+                raise_timeout(p, abort);
+                okk = false;
+                break;
+            }
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const uint8_t *xrow = sb + (2 + hh) * kBox;
+                uint8_t *xwt = s.xw[xb] + hh * kBox;
+                const float w = hh ? wb : wa;
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    const uint32_t o = swz(r, cc);
+                    uint4 vv = lds128(xrow + o);
+                    vv.x = scale_bf16x2(vv.x, w); vv.y = scale_bf16x2(vv.y, w);
+                    vv.z = scale_bf16x2(vv.z, w); vv.w = scale_bf16x2(vv.w, w);
+                    sts128(xwt + o, vv);
+                }
             }
             fence_proxy_async_smem();
             mbar_arrive(&s.xw_full[xb]);
             mbar_arrive(&s.empty[st]);
-            suf2 += tot2;
+            sufa += tota;
+            sufb += totb;
         }
-        if (okk && ewait(&s.acc_full, 0, abort, p.wait_limit_ns)) {
+        if (okk && ewait(&s.acc_full, 0, abort, lim)) {
             tc_fence_after();
-            uint32_t a[32], b[32];
-            tmem_ld32(tS + lane_base, a);
-            tmem_ld32(tS + lane_base + 32, b);
-            tmem_wait_ld();
-            float *dst = p.ws_S + (((int64_t)bi * p.ns + k) * p.H + h) * (kP * kN) + r;
+            const int hh = r >> 6, pp = r & 63;  // lane r holds state row p of head h0 + hh
+            float *dst = p.ws_S + (((int64_t)bi * p.ns + k) * p.H + h0 + hh) * (kP * kN) + (int64_t)pp * kN;
 #pragma unroll
-            for (int pp = 0; pp < 32; ++pp) dst[pp * kN] = __uint_as_float(a[pp]);
+            for (int c32 = 0; c32 < 4; ++c32) {
+                uint32_t a[32];
+                tmem_ld32(tS + lane_base + 32 * c32, a);
+                tmem_wait_ld();
 #pragma unroll
-            for (int pp = 0; pp < 32; ++pp) dst[(pp + 32) * kN] = __uint_as_float(b[pp]);
-            if (r == 0) p.ws_dA[((int64_t)bi * p.ns + k) * p.H + h] = suf2 * kLn2;
+                for (int i = 0; i < 8; ++i)
+                    reinterpret_cast<uint4 *>(dst + 32 * c32)[i] = make_uint4(a[4 * i], a[4 * i + 1], a[4 * i + 2], a[4 * i + 3]);
+            }
+            if (r == 0) {
+                p.ws_dA[((int64_t)bi * p.ns + k) * p.H + h0] = sufa * kLn2;
+                p.ws_dA[((int64_t)bi * p.ns + k) * p.H + h0 + 1] = sufb * kLn2;
+            }
         } else if (okk) {
             raise_timeout(p, abort);
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) tmem_dealloc(tS, 64);
+    if (warp == 1) tmem_dealloc(tS, 128);
 }
 
 // =============================================================== pass C
+// One CTA per (stripe, head), two CTAs per SM: each CTA walks its chunks in a
+// plain sequence and the two co-resident CTAs hide each other's latencies.
+// Per chunk (all 256 threads; thread = TMEM lane quarter q, column half hs):
+//   G  = C B^T                         one elected thread issues the MMAs
+//   cumsum of dt*A (each warp on its own), Pm from G, D x into Y
+//   EC = exp(cs_i) C_i (bf16, TMEM) ; w o X written over the spent C tile
+//   Y += Pm X ; Y += EC h_prev^T ; S = B^T (w o X)      (one commit)
+//   -> every input slot is free: the next chunk's TMA is issued here
+//   y = Y -> global ; h = exp(cs_last) h + S ; h_prev (bf16) -> smem ; checkpoints
+// TMEM (256 columns): G 0..127, then EC 0..63 and S 64..127 | Pm 128..191 | Y 192..255.
+constexpr int kThreadsC = 256;
+
 struct SmemC {
-    uint8_t stage[2][5 * kBox + kDtBox];  // C (two boxes), B (two boxes), X, dt
-    uint8_t xw[kBox];
-    uint8_t hp[kBox];                     // bf16 h_prev, rows n, 128B-swizzled
-    float cs2[kQ];
-    float dts[kQ];
-    float scratch[2][4];
-    uint64_t full[2], empty[2], g_full[2], pm_full[2], pm_free[2];
-    uint64_t y_full, acc_empty, xw_full, xw_empty, s_full, s_empty, hp_full, fin, epi;
+    uint8_t cb[4 * kBox];      // C (two boxes: K 0..63, 64..127), B (two boxes); C is reused for w o X
+    uint8_t x[kBox];           // X, rows j (tokens), 128B-swizzled
+    uint8_t hp[kBox];          // bf16 h_prev, rows n, 128B-swizzled
+    float dt[kQ * 4];          // dt box: [128 tokens][4 heads]
+    uint64_t full, g_done, mma_done, fin;
     uint32_t tmem;
     int abort;
 };
 
-__device__ __forceinline__ void write_hp(uint8_t *hp, int n, const float (&hr)[64])
+__device__ __forceinline__ float sel4(const float (&v)[4], int i)
 {
-#pragma unroll
-    for (int cc = 0; cc < 8; ++cc) {
-        uint4 v;
-        v.x = pack_bf16x2(hr[8 * cc + 0], hr[8 * cc + 1]);
-        v.y = pack_bf16x2(hr[8 * cc + 2], hr[8 * cc + 3]);
-        v.z = pack_bf16x2(hr[8 * cc + 4], hr[8 * cc + 5]);
-        v.w = pack_bf16x2(hr[8 * cc + 6], hr[8 * cc + 7]);
-        sts128(hp + swz(n, cc), v);
-    }
+    return i == 0 ? v[0] : (i == 1 ? v[1] : (i == 2 ? v[2] : v[3]));
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsC, 2)
 chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
 {
     extern __shared__ uint8_t smraw[];
     SmemC &s = *reinterpret_cast<SmemC *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q = warp & 3, hs = warp >> 2;
+    const int r = 32 * q + lane;                 // token row / TMEM lane / state column n
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     const int64_t unit = blockIdx.x;
     const int h = (int)(unit % p.H);
     const int64_t k = (unit / p.H) % p.ns;
@@ -312,275 +352,299 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
     const int64_t s0 = k * p.T;
     const int64_t s1 = min(p.L, s0 + p.T);
     const int nc = (int)((s1 - s0 + kQ - 1) / kQ);
+    const uint64_t lim = p.wait_limit_ns;
+    const int PN = kP * kN;
 
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&s.full[i], 1);
-            mbar_init(&s.empty[i], 1 + 128);
-            mbar_init(&s.g_full[i], 1);
-            mbar_init(&s.pm_full[i], 128);
-            mbar_init(&s.pm_free[i], 1);
-        }
-        mbar_init(&s.y_full, 1);
-        mbar_init(&s.acc_empty, 128);
-        mbar_init(&s.xw_full, 128);
-        mbar_init(&s.xw_empty, 1);
-        mbar_init(&s.s_full, 1);
-        mbar_init(&s.s_empty, 128);
-        mbar_init(&s.hp_full, 128);
+    if (tid == 0) {
+        mbar_init(&s.full, 1);
+        mbar_init(&s.g_done, 1);
+        mbar_init(&s.mma_done, 1);
         mbar_init(&s.fin, 1);
-        mbar_init(&s.epi, 128);
         s.abort = 0;
         fence_mbar_init();
-    }
-    if (warp == 0 && lane == 0) {
         prefetch_tmap(&maps.x);
         prefetch_tmap(&maps.B);
         prefetch_tmap(&maps.C);
         prefetch_tmap(&maps.dt);
     }
-    if (warp == 1) { tmem_alloc(&s.tmem, 512); tmem_relinquish(); }
+    if (warp == 0) { tmem_alloc(&s.tmem, 256); tmem_relinquish(); }
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = s.tmem;
-    const uint32_t tYd = tm + 256, tYo = tm + 320, tS = tm + 384;
+    const uint32_t tG = tm, tEC = tm, tS = tm + 64, tPm = tm + 128, tY = tm + 192;
     volatile int *abort = &s.abort;
 
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer
-        if (lane == 0) {
-            int issued = 0;
-            for (int c = 0; c < nc; ++c) {
-                const int st = c & 1, u = c >> 1;
-                if (c >= 2 && !mbar_wait(&s.empty[st], (u - 1) & 1, abort, p.wait_limit_ns)) { raise_timeout(p, abort); break; }
-                if (unit == p.test_drop_unit) break;  // test hook: this unit's loads never arrive
-                const int t0 = (int)(s0 + (int64_t)c * kQ);
-                uint8_t *sb = s.stage[st];
-                mbar_arrive_expect_tx(&s.full[st], 5 * kBox + kDtBox);
-                tma_load_3d(sb, &maps.C, &s.full[st], g * kN, t0, bi);
-                tma_load_3d(sb + kBox, &maps.C, &s.full[st], g * kN + 64, t0, bi);
-                tma_load_3d(sb + 2 * kBox, &maps.B, &s.full[st], g * kN, t0, bi);
-                tma_load_3d(sb + 3 * kBox, &maps.B, &s.full[st], g * kN + 64, t0, bi);
-                tma_load_3d(sb + 4 * kBox, &maps.x, &s.full[st], h * kP, t0, bi);
-                tma_load_3d(sb + 5 * kBox, &maps.dt, &s.full[st], h & ~3, t0, bi);
-                issued = c + 1;
-            }
-            if (*abort) {
-                for (int c = max(0, issued - 2); c < issued; ++c)
-                    mbar_wait(&s.full[c & 1], (c >> 1) & 1, nullptr, 100000000ull);
-            }
+    auto issue_loads = [&](int c) {
+        const int t0 = (int)(s0 + (int64_t)c * kQ);
+        mbar_arrive_expect_tx(&s.full, 5 * kBox + kDtBox);
+        tma_load_3d(s.cb, &maps.C, &s.full, g * kN, t0, bi);
+        tma_load_3d(s.cb + kBox, &maps.C, &s.full, g * kN + 64, t0, bi);
+        tma_load_3d(s.cb + 2 * kBox, &maps.B, &s.full, g * kN, t0, bi);
+        tma_load_3d(s.cb + 3 * kBox, &maps.B, &s.full, g * kN + 64, t0, bi);
+        tma_load_3d(s.x, &maps.x, &s.full, h * kP, t0, bi);
+        tma_load_3d(s.dt, &maps.dt, &s.full, h & ~3, t0, bi);
+    };
+    int pending = -1;   // (thread 0) chunk whose loads are issued but not yet waited for
+    if (tid == 0 && nc > 0 && unit != p.test_drop_unit) { issue_loads(0); pending = 0; }
+
+    // state entering the stripe: thread (r = n, hs) owns h[32 hs .. 32 hs + 31][n]
+    float hr[32];
+    {
+        const float *hin = (k == 0) ? (p.h0 ? p.h0 + ((int64_t)bi * p.H + h) * PN : nullptr)
+                                    : p.ws_hin + (((int64_t)bi * p.ns + k) * p.H + h) * PN;
+#pragma unroll
+        for (int pp = 0; pp < 32; ++pp) hr[pp] = hin ? hin[(32 * hs + pp) * kN + r] : 0.0f;
+    }
+    auto write_hp = [&]() {
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+            uint4 v;
+            v.x = pack_bf16x2(hr[8 * c4 + 0], hr[8 * c4 + 1]);
+            v.y = pack_bf16x2(hr[8 * c4 + 2], hr[8 * c4 + 3]);
+            v.z = pack_bf16x2(hr[8 * c4 + 4], hr[8 * c4 + 5]);
+            v.w = pack_bf16x2(hr[8 * c4 + 6], hr[8 * c4 + 7]);
+            sts128(s.hp + swz(r, 4 * hs + c4), v);
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t id_g = idesc_bf16(128, 128, 0, 0);
-            const uint32_t id_kmn = idesc_bf16(128, 64, 0, 1);
-            const uint32_t id_mnmn = idesc_bf16(128, 64, 1, 1);
-            const uint32_t sHp = smem_u32(s.hp), sXw = smem_u32(s.xw);
-            for (int c = 0; c < nc; ++c) {
-                const int st = c & 1, u = c >> 1, buf = c & 1;
-                const uint32_t tG = tm + 128 * buf;
-                if (!mbar_wait(&s.full[st], u & 1, abort, p.wait_limit_ns)) { raise_timeout(p, abort); break; }
-                if (c >= 2 && !mbar_wait(&s.pm_free[buf], ((c >> 1) - 1) & 1, abort, p.wait_limit_ns)) { raise_timeout(p, abort); break; }
-                tc_fence_after();
-                const uint32_t sC = smem_u32(s.stage[st]);
-                const uint32_t sB = sC + 2 * kBox, sX = sC + 4 * kBox;
-                // G = C B^T
+    };
+    write_hp();
+    fence_proxy_async_smem();
+
+    const float A2 = p.A[h] * kLog2e;
+    const float Dh = p.D ? p.D[h] : 0.0f;
+    const int64_t n_ckpt = p.s > 0 ? p.L / p.s : 0;
+    __nv_bfloat16 *ybase = reinterpret_cast<__nv_bfloat16 *>(p.y) + (int64_t)bi * p.ybs + (int64_t)h * kP + 32 * hs;
+    const uint32_t id_g = idesc_bf16(128, 128, 0, 0);
+    const uint32_t id_kmn = idesc_bf16(128, 64, 0, 1);
+    const uint32_t id_mnmn = idesc_bf16(128, 64, 1, 1);
+
+    for (int c = 0; c < nc; ++c) {
+        const int64_t t0 = s0 + (int64_t)c * kQ;
+        // ---- operands of this chunk
+        bool ok = mbar_wait(&s.full, c & 1, abort, lim);
+        if (!__syncthreads_and(ok)) { raise_timeout(p, abort); break; }
+        pending = -1;
+        tc_fence_after();
+        if (tid == 0) {
+            const uint32_t sC = smem_u32(s.cb), sB = sC + 2 * kBox;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-                    mma_ss(tG, smem_desc(sC + off, 16, 1024), smem_desc(sB + off, 16, 1024), id_g, kk > 0);
-                }
-                mma_commit(&s.g_full[buf]);
-                // Yo = C h_prev^T
-                if (!mbar_wait(&s.hp_full, c & 1, abort, p.wait_limit_ns)) { raise_timeout(p, abort); break; }
-                if (c >= 1 && !mbar_wait(&s.acc_empty, (c - 1) & 1, abort, p.wait_limit_ns)) { raise_timeout(p, abort); break; }
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-                    mma_ss(tYo, smem_desc(sC + off, 16, 1024), smem_desc(sHp + kk * 2048, 0, 1024), id_kmn, kk > 0);
-                }
-                // Yd = Pm X   (Pm: bf16 in TMEM, written over G)
-                if (!mbar_wait(&s.pm_full[buf], (c >> 1) & 1, abort, p.wait_limit_ns)) { raise_timeout(p, abort); break; }
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tYd, tG + kk * 8, smem_desc(sX + kk * 2048, 0, 1024), id_kmn, kk > 0);
-                mma_commit(&s.y_full);
-                mma_commit(&s.pm_free[buf]);
-                // S = B^T (w o X)
-                if (!mbar_wait(&s.xw_full, c & 1, abort, p.wait_limit_ns)) { raise_timeout(p, abort); break; }
-                if (c >= 1 && !mbar_wait(&s.s_empty, (c - 1) & 1, abort, p.wait_limit_ns)) { raise_timeout(p, abort); break; }
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tS, smem_desc(sB + kk * 2048, kBox, 1024), smem_desc(sXw + kk * 2048, 0, 1024),
-                           id_mnmn, kk > 0);
-                mma_commit(&s.s_full);
-                mma_commit(&s.xw_empty);
-                mma_commit(&s.empty[st]);
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+                mma_ss(tG, smem_desc(sC + off, 16, 1024), smem_desc(sB + off, 16, 1024), id_g, kk > 0);
             }
-            mma_commit(&s.fin);
-            mbar_wait(&s.fin, 0, nullptr, 200000000ull);
+            mma_commit(&s.g_done);
         }
-    } else {
-        // ------------------------------------------------ epilogue: rows r = TMEM lanes
-        const int q = warp & 3;
-        const int r = 32 * q + lane;
-        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        const float A2 = p.A[h] * kLog2e;
-        const float Dh = p.D ? p.D[h] : 0.0f;
-        const int64_t n_ckpt = p.s > 0 ? p.L / p.s : 0;
-        const int PN = kP * kN;
-        float hr[64];
+        // ---- chunk cumsum (each warp on its own: lane l holds rows l + 32 J)
+        float dv[4], cv[4], fv[4], r2[4];
+#pragma unroll
+        for (int J = 0; J < 4; ++J) dv[J] = s.dt[(lane + 32 * J) * 4 + (h & 3)];
+#pragma unroll
+        for (int J = 0; J < 4; ++J) {
+            float v = dv[J] * A2;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float t = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += t;
+            }
+            cv[J] = v;
+        }
         {
-            const float *hin = (k == 0) ? (p.h0 ? p.h0 + ((int64_t)bi * p.H + h) * PN : nullptr)
-                                        : p.ws_hin + (((int64_t)bi * p.ns + k) * p.H + h) * PN;
+            float run = 0.0f;
 #pragma unroll
-            for (int pp = 0; pp < 64; ++pp) hr[pp] = hin ? hin[pp * kN + r] : 0.0f;
-        }
-        write_hp(s.hp, r, hr);
-        fence_proxy_async_smem();
-        mbar_arrive(&s.hp_full);
-
-        __nv_bfloat16 *ybase = reinterpret_cast<__nv_bfloat16 *>(p.y) + (int64_t)bi * p.ybs + (int64_t)h * kP;
-        uint32_t eph = 0;
-        for (int c = 0; c < nc; ++c) {
-            const int st = c & 1, u = c >> 1, buf = c & 1;
-            const uint32_t tG = tm + 128 * buf;
-            const int64_t t0 = s0 + (int64_t)c * kQ;
-            if (!ewait(&s.full[st], u & 1, abort, p.wait_limit_ns)) { raise_timeout(p, abort); break; }
-            const uint8_t *sb = s.stage[st];
-            const uint8_t *xt = sb + 4 * kBox;
-            const float dt_r = reinterpret_cast<const float *>(sb + 5 * kBox)[r * 4 + (h & 3)];
-            float tot2, cs2 = dt_r * A2;
-            if (!epi_scan(cs2, r, s.scratch[c & 1], tot2, &s.epi, eph, abort, p.wait_limit_ns)) { raise_timeout(p, abort); break; }
-            s.cs2[r] = cs2;
-            s.dts[r] = dt_r;
-            if (!epi_sync(&s.epi, eph, abort, p.wait_limit_ns)) { raise_timeout(p, abort); break; }
-
-            // ---- w o X for the state update
-            if (c >= 1 && !ewait(&s.xw_empty, (c - 1) & 1, abort, p.wait_limit_ns)) { raise_timeout(p, abort); break; }
-            {
-                const float w = dt_r * ex2(tot2 - cs2);
-#pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
-                    const uint32_t o = swz(r, cc);
-                    uint4 v = lds128(xt + o);
-                    v.x = scale_bf16x2(v.x, w); v.y = scale_bf16x2(v.y, w);
-                    v.z = scale_bf16x2(v.z, w); v.w = scale_bf16x2(v.w, w);
-                    sts128(s.xw + o, v);
-                }
-                fence_proxy_async_smem();
-                mbar_arrive(&s.xw_full);
+            for (int J = 0; J < 4; ++J) {
+                const float bt = __shfl_sync(0xffffffffu, cv[J], 31);
+                cv[J] += run;
+                run += bt;
+                r2[J] = run;
             }
-
-            // ---- masked decay: Pm[r][j] = G[r][j] * exp(cs_r - cs_j) * dt_j for j <= r
-            if (!ewait(&s.g_full[buf], (c >> 1) & 1, abort, p.wait_limit_ns)) { raise_timeout(p, abort); break; }
-            tc_fence_after();
+        }
+        const float tot2 = r2[3];
 #pragma unroll
-            for (int jb = 0; jb < 4; ++jb) {
+        for (int J = 0; J < 4; ++J) fv[J] = dv[J] * ex2(r2[J] - cv[J]);
+        const float cs2 = sel4(cv, q);
+        const float dt_r = sel4(dv, q);
+        // ---- D x into Y (this half's 32 columns of p)
+        {
+            uint32_t dx[32];
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const uint4 xv = lds128(s.x + swz(r, 4 * hs + c4));
+                const uint32_t w4[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    dx[8 * c4 + 2 * i] = __float_as_uint(Dh * bf16_lo(w4[i]));
+                    dx[8 * c4 + 2 * i + 1] = __float_as_uint(Dh * bf16_hi(w4[i]));
+                }
+            }
+            uint32_t d0[16], d1[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) { d0[i] = dx[i]; d1[i] = dx[16 + i]; }
+            tmem_st16(tY + lane_base + 32 * hs, d0);
+            tmem_st16(tY + lane_base + 32 * hs + 16, d1);
+        }
+        // ---- masked decay Pm[r][j] = G[r][j] exp(cs_r - cs_j) dt_j (j <= r): blocks {hs, hs + 2}
+        ok = mbar_wait(&s.g_done, c & 1, abort, lim);
+        if (!__all_sync(0xffffffffu, ok)) { *abort = 1; }
+        tc_fence_after();
+        if (!*abort) {
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const int J = 2 * jj + hs;
                 uint32_t pk[16];
-                if (jb <= q) {
+                if (J < q) {
+                    const float E = ex2(cs2 - sel4(r2, J));
                     uint32_t gv[32];
-                    tmem_ld32(tG + lane_base + 32 * jb, gv);
+                    tmem_ld32(tG + lane_base + 32 * J, gv);
                     tmem_wait_ld();
+                    const float fJ = sel4(fv, J);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const int j0 = 32 * jb + 2 * i;
-                        float v0 = __uint_as_float(gv[2 * i]) * ex2(cs2 - s.cs2[j0]) * s.dts[j0];
-                        float v1 = __uint_as_float(gv[2 * i + 1]) * ex2(cs2 - s.cs2[j0 + 1]) * s.dts[j0 + 1];
-                        if (j0 > r) v0 = 0.0f;
-                        if (j0 + 1 > r) v1 = 0.0f;
+                        const float f0 = __shfl_sync(0xffffffffu, fJ, 2 * i);
+                        const float f1 = __shfl_sync(0xffffffffu, fJ, 2 * i + 1);
+                        pk[i] = pack_bf16x2(__uint_as_float(gv[2 * i]) * f0 * E,
+                                            __uint_as_float(gv[2 * i + 1]) * f1 * E);
+                    }
+                } else if (J == q) {
+                    uint32_t gv[32];
+                    tmem_ld32(tG + lane_base + 32 * J, gv);
+                    tmem_wait_ld();
+                    const float cJ = sel4(cv, J), dJ = sel4(dv, J);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float c0 = __shfl_sync(0xffffffffu, cJ, 2 * i);
+                        const float c1 = __shfl_sync(0xffffffffu, cJ, 2 * i + 1);
+                        const float d0 = __shfl_sync(0xffffffffu, dJ, 2 * i);
+                        const float d1 = __shfl_sync(0xffffffffu, dJ, 2 * i + 1);
+                        float v0 = __uint_as_float(gv[2 * i]) * ex2(cs2 - c0) * d0;
+                        float v1 = __uint_as_float(gv[2 * i + 1]) * ex2(cs2 - c1) * d1;
+                        if (2 * i > lane) v0 = 0.0f;
+                        if (2 * i + 1 > lane) v1 = 0.0f;
                         pk[i] = pack_bf16x2(v0, v1);
                     }
                 } else {
 #pragma unroll
                     for (int i = 0; i < 16; ++i) pk[i] = 0u;
                 }
-                tmem_st16(tG + lane_base + 16 * jb, pk);
+                tmem_st16(tPm + lane_base + 16 * J, pk);
             }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&s.pm_full[buf]);
-
-            // ---- outputs y = Yd + exp(cs_r) Yo + D x
-            if (!ewait(&s.y_full, c & 1, abort, p.wait_limit_ns)) { raise_timeout(p, abort); break; }
-            tc_fence_after();
-            {
-                const float e = ex2(cs2);
-                const bool valid = t0 + r < s1;
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        if (__syncthreads_or(*abort)) { raise_timeout(p, abort); break; }   // all reads of G done
+        tc_fence_after();
+        // ---- EC = exp(cs_r) C_r over G's columns 0..63 (this half: K = 64 hs .. 64 hs + 63)
+        {
+            const float e = ex2(cs2);
+            const uint8_t *cbox = s.cb + hs * kBox;
+#pragma unroll
+            for (int q2 = 0; q2 < 2; ++q2) {
+                uint32_t ev[16];
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const uint4 cvv = lds128(cbox + swz(r, 4 * q2 + c4));
+                    ev[4 * c4 + 0] = scale_bf16x2(cvv.x, e);
+                    ev[4 * c4 + 1] = scale_bf16x2(cvv.y, e);
+                    ev[4 * c4 + 2] = scale_bf16x2(cvv.z, e);
+                    ev[4 * c4 + 3] = scale_bf16x2(cvv.w, e);
+                }
+                tmem_st16(tEC + lane_base + 32 * hs + 16 * q2, ev);
+            }
+        }
+        tmem_wait_st();
+        __syncthreads();   // every read of C is done: w o X may overwrite it
+        // ---- w o X for the state update, written over C's first box (rows j, same swizzle)
+        {
+            const float w = dt_r * ex2(tot2 - cs2);
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const int cc = 4 * hs + c4;
+                uint4 vv = lds128(s.x + swz(r, cc));
+                vv.x = scale_bf16x2(vv.x, w); vv.y = scale_bf16x2(vv.y, w);
+                vv.z = scale_bf16x2(vv.z, w); vv.w = scale_bf16x2(vv.w, w);
+                sts128(s.cb + swz(r, cc), vv);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (tid == 0) {
+            const uint32_t sX = smem_u32(s.x), sHp = smem_u32(s.hp), sXw = smem_u32(s.cb);
+            const uint32_t sB = sXw + 2 * kBox;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                mma_ts(tY, tPm + kk * 8, smem_desc(sX + kk * 2048, 0, 1024), id_kmn, true);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                mma_ts(tY, tEC + kk * 8, smem_desc(sHp + kk * 2048, 0, 1024), id_kmn, true);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                mma_ss(tS, smem_desc(sB + kk * 2048, kBox, 1024), smem_desc(sXw + kk * 2048, 0, 1024),
+                       id_mnmn, kk > 0);
+            mma_commit(&s.mma_done);
+        }
+        ok = mbar_wait(&s.mma_done, c & 1, abort, lim);
+        if (!__syncthreads_and(ok)) { raise_timeout(p, abort); break; }
+        tc_fence_after();
+        // every operand slot is free: fetch the next chunk while this one finishes
+        if (tid == 0 && c + 1 < nc) {
+            issue_loads(c + 1);
+            pending = c + 1;
+        }
+        // ---- y = Y, this half's 32 columns
+        {
+            uint32_t yv[32];
+            tmem_ld32(tY + lane_base + 32 * hs, yv);
+            tmem_wait_ld();
+            if (t0 + r < s1) {
                 __nv_bfloat16 *yrow = ybase + (t0 + r) * p.yrs;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t yd[32], yo[32];
-                    tmem_ld32(tYd + lane_base + 32 * half, yd);
-                    tmem_ld32(tYo + lane_base + 32 * half, yo);
-                    tmem_wait_ld();
-                    if (half == 1) {
-                        tc_fence_before();
-                        mbar_arrive(&s.acc_empty);
-                    }
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    uint32_t o4[4];
 #pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        const int cc = 4 * half + c4;
-                        const uint4 xv = lds128(xt + swz(r, cc));
-                        const uint32_t xw4[4] = {xv.x, xv.y, xv.z, xv.w};
-                        uint32_t o4[4];
-#pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2) {
-                            const int i0 = 8 * c4 + 2 * e2;
-                            const float a0 = __uint_as_float(yd[i0]) + e * __uint_as_float(yo[i0]) + Dh * bf16_lo(xw4[e2]);
-                            const float a1 = __uint_as_float(yd[i0 + 1]) + e * __uint_as_float(yo[i0 + 1]) + Dh * bf16_hi(xw4[e2]);
-                            o4[e2] = pack_bf16x2(a0, a1);
-                        }
-                        if (valid) *reinterpret_cast<uint4 *>(yrow + 8 * cc) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
-                    }
-                }
-            }
-            mbar_arrive(&s.empty[st]);
-
-            // ---- state update h = exp(cs_last) h + S  (thread r owns state column n = r)
-            if (!ewait(&s.s_full, c & 1, abort, p.wait_limit_ns)) { raise_timeout(p, abort); break; }
-            tc_fence_after();
-            {
-                uint32_t sa[32], sbv[32];
-                tmem_ld32(tS + lane_base, sa);
-                tmem_ld32(tS + lane_base + 32, sbv);
-                tmem_wait_ld();
-                tc_fence_before();
-                mbar_arrive(&s.s_empty);
-                const float dec = ex2(tot2);
-#pragma unroll
-                for (int pp = 0; pp < 32; ++pp) hr[pp] = fmaf(dec, hr[pp], __uint_as_float(sa[pp]));
-#pragma unroll
-                for (int pp = 0; pp < 32; ++pp) hr[pp + 32] = fmaf(dec, hr[pp + 32], __uint_as_float(sbv[pp]));
-            }
-            if (c + 1 < nc) {
-                write_hp(s.hp, r, hr);
-                fence_proxy_async_smem();
-                mbar_arrive(&s.hp_full);
-            }
-            const int64_t t_end = t0 + kQ;
-            if (p.h_ckpt && p.s > 0 && t_end <= s1 && t_end % p.s == 0) {
-                const int64_t kk = t_end / p.s - 1;
-                if (kk < n_ckpt) {
-                    float *dst = p.h_ckpt + (((int64_t)bi * n_ckpt + kk) * p.H + h) * PN + r;
-#pragma unroll
-                    for (int pp = 0; pp < 64; ++pp) dst[pp * kN] = hr[pp];
+                    for (int e2 = 0; e2 < 4; ++e2)
+                        o4[e2] = pack_bf16x2(__uint_as_float(yv[8 * c4 + 2 * e2]), __uint_as_float(yv[8 * c4 + 2 * e2 + 1]));
+                    *reinterpret_cast<uint4 *>(yrow + 8 * c4) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
                 }
             }
         }
-        if (!*abort && p.h_final && s1 == p.L) {
-            float *dst = p.h_final + ((int64_t)bi * p.H + h) * PN + r;
+        // ---- state: h = exp(cs_last) h + S  (columns p of this half, state column n = r)
+        {
+            uint32_t sa[32];
+            tmem_ld32(tS + lane_base + 32 * hs, sa);
+            tmem_wait_ld();
+            const float dec = ex2(tot2);
 #pragma unroll
-            for (int pp = 0; pp < 64; ++pp) dst[pp * kN] = hr[pp];
+            for (int pp = 0; pp < 32; ++pp) hr[pp] = fmaf(dec, hr[pp], __uint_as_float(sa[pp]));
         }
+        if (c + 1 < nc) {
+            write_hp();
+            fence_proxy_async_smem();   // before the barrier that orders it with the next MMAs
+        }
+        const int64_t t_end = t0 + kQ;
+        if (p.h_ckpt && p.s > 0 && t_end <= s1 && t_end % p.s == 0) {
+            const int64_t kk = t_end / p.s - 1;
+            if (kk < n_ckpt) {
+                float *dst = p.h_ckpt + (((int64_t)bi * n_ckpt + kk) * p.H + h) * PN + (int64_t)(32 * hs) * kN + r;
+#pragma unroll
+                for (int pp = 0; pp < 32; ++pp) dst[pp * kN] = hr[pp];
+            }
+        }
+        tc_fence_before();
+    }
+    if (!*abort && p.h_final && s1 == p.L) {
+        float *dst = p.h_final + ((int64_t)bi * p.H + h) * PN + (int64_t)(32 * hs) * kN + r;
+#pragma unroll
+        for (int pp = 0; pp < 32; ++pp) dst[pp * kN] = hr[pp];
+    }
+    // drain: MMAs and loads that may still be in flight after an abort
+    if (tid == 0 && *abort) {
+        mma_commit(&s.fin);
+        mbar_wait(&s.fin, 0, nullptr, 100000000ull);
+        if (pending >= 0) mbar_wait(&s.full, pending & 1, nullptr, 100000000ull);
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) tmem_dealloc(tm, 512);
+    if (warp == 0) tmem_dealloc(tm, 256);
 }
 
 // =============================================================== host side
@@ -639,7 +703,7 @@ static_assert(kSmemA <= 232448, "pass A shared memory");
 bool tc_scan_supported(const ScanParams &p, int dtype)
 {
     if (dtype != 1 || p.P != kP || p.N != kN || p.Q != kQ) return false;
-    if (p.H % 4 != 0) return false;
+    if (p.H % 4 != 0 || (p.H / p.G) % 2 != 0) return false;  // head pairs share a B/C group
     if ((reinterpret_cast<uintptr_t>(p.dt) & 15u) != 0) return false;
     if (p.L >= (1LL << 31) || (int64_t)p.b * p.ns * p.H >= (1LL << 31)) return false;
     return encode_fn() != nullptr;
@@ -668,13 +732,13 @@ int launch_scan_tc(const ScanParams &p, cudaStream_t st)
     const int64_t units = (int64_t)p.b * p.ns * p.H;
     if (p.ns > 1) {
         prof_begin(st, kKStateTc);
-        stripe_state_tc_kernel<<<(unsigned)units, kThreads, kSmemA, st>>>(maps, p);
+        stripe_state_tc_kernel<<<(unsigned)(units / 2), kThreads, kSmemA, st>>>(maps, p);
         prof_end(st, kKStateTc);
         const int rc = launch_chain(p, st);
         if (rc) return rc;
     }
     prof_begin(st, kKOutputTc);
-    chunk_output_tc_kernel<<<(unsigned)units, kThreads, kSmemC, st>>>(maps, p);
+    chunk_output_tc_kernel<<<(unsigned)units, kThreadsC, kSmemC, st>>>(maps, p);
     prof_end(st, kKOutputTc);
     return cudaGetLastError() == cudaSuccess ? 0 : 7;
 }
