@@ -11,21 +11,20 @@
 // Per chunk of 128 tokens of one head (cs = chunk-local cumulative dt*A, kept
 // in log2 units so that exp(x) = ex2(x * log2 e)):
 //   G  = C B^T                                     tcgen05, 128x128x128, TMEM
-//   Pm = G o [exp(cs_i - cs_j) dt_j, j <= i]       CUDA cores, TMEM -> TMEM (bf16)
+//   Pm = G o [exp(cs_i - cs_j) dt_j, j <= i] + D I CUDA cores, TMEM -> TMEM (bf16)
 //   Yd = Pm X                                      tcgen05, A from TMEM, 128x64x128
 //   Yo = C h_prev^T                                tcgen05, 128x64x128
-//   y  = Yd + exp(cs_i) Yo + D x                   CUDA cores -> global (bf16)
+//   y  = Yd + exp(cs_i) Yo                         CUDA cores -> smem -> TMA store
 //   S  = B^T (w o X),  w_j = dt_j exp(cs_last - cs_j)   tcgen05, 128x64x128
 //   h  = exp(cs_last) h + S                        CUDA cores, fp32 state in registers
 // Only non-positive differences of cs are exponentiated.  The state is kept in
-// fp32; its bf16 copy only feeds the C h_prev^T product.
+// fp32; its bf16 copy only feeds the C h_prev^T product.  Both kernels take
+// two heads per CTA: they share B (and C), so G is computed once per pair and
+// the products with a shared operand run at N = 128.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads into a 2-stage ring,
-// warp 1 issues the MMAs (one thread), warps 2..5 (128 threads, one per
-// token row / TMEM lane) do the masked decay, the outputs and the state.
 // All waits are bounded (tc::mbar_wait): on a timeout the CTA raises an abort
-// flag, every role unwinds, outstanding MMAs are drained, TMEM is freed and
-// the device status word reports SSD_ERR_TIMEOUT.
+// flag, every thread unwinds, outstanding MMAs and loads are drained, TMEM is
+// freed and the device status word reports SSD_ERR_TIMEOUT.
 #include <cuda.h>
 
 #include "ssd_common.cuh"
@@ -47,7 +46,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kThreads = 192;
 
 struct Maps {
-    CUtensorMap x, B, C, dt;
+    CUtensorMap x, B, C, dt, y;
 };
 
 __device__ __forceinline__ float ex2(float x)
@@ -87,30 +86,6 @@ __device__ __forceinline__ void sts128(uint8_t *p, uint4 v) { *reinterpret_cast<
 __device__ __forceinline__ uint32_t scale_bf16x2(uint32_t v, float w)
 {
     return pack_bf16x2(bf16_lo(v) * w, bf16_hi(v) * w);
-}
-
-// Inclusive scan of one value per epilogue thread (row r) over the 128 rows.
-// scratch holds two buffers of 4 floats, used alternately by consecutive
-// calls (a thread can be at most one call ahead of the slowest one).
-__device__ __forceinline__ bool epi_scan(float &v, int r, float *scratch, float &total, uint64_t *bar,
-                                         uint32_t &ph, volatile int *abort, uint64_t limit_ns)
-{
-    const int lane = r & 31, q = r >> 5;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const float t = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += t;
-    }
-    if (lane == 31) scratch[q] = v;
-    if (!epi_sync(bar, ph, abort, limit_ns)) return false;
-    const float s0 = scratch[0], s1 = scratch[1], s2 = scratch[2], s3 = scratch[3];
-    float pre = 0.0f;
-    if (q > 0) pre += s0;
-    if (q > 1) pre += s1;
-    if (q > 2) pre += s2;
-    total = ((s0 + s1) + s2) + s3;
-    v = q == 3 ? v + ((s0 + s1) + s2) : v + pre;
-    return true;
 }
 
 __device__ __forceinline__ void raise_timeout(const ScanParams &p, volatile int *abort)
@@ -308,56 +283,71 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
 }
 
 // =============================================================== pass C
-// One CTA per (stripe, head), two CTAs per SM: each CTA walks its chunks in a
-// plain sequence and the two co-resident CTAs hide each other's latencies.
-// Per chunk (all 256 threads; thread = TMEM lane quarter q, column half hs):
-//   G  = C B^T                         one elected thread issues the MMAs
-//   cumsum of dt*A (each warp on its own), Pm from G, D x into Y
-//   EC = exp(cs_i) C_i (bf16, TMEM) ; w o X written over the spent C tile
-//   Y += Pm X ; Y += EC h_prev^T ; S = B^T (w o X)      (one commit)
-//   -> every input slot is free: the next chunk's TMA is issued here
-//   y = Y -> global ; h = exp(cs_last) h + S ; h_prev (bf16) -> smem ; checkpoints
-// TMEM (256 columns): G 0..127, then EC 0..63 and S 64..127 | Pm 128..191 | Y 192..255.
-constexpr int kThreadsC = 256;
+// One CTA per (stripe, head pair), one CTA per SM.  The two heads share their
+// B and C tiles and G = C B^T; the chunks of the stripe are walked in order.
+// Thread = TMEM lane quarter q (warp & 3) x column slice cs (warp >> 2); the
+// column slices 0,1 belong to head a, 2,3 to head b.  Per chunk c:
+//   scan      warps 0 and 8: chunk cumsum of dt*A of head a / b -> smem
+//   mask a    Pm_a = G o [exp(cs_i - cs_j) dt_j]_{j<=i} (+ D on the diagonal),
+//             then Y_a = Pm_a X_a is issued
+//   mask b    likewise; then Y_b = Pm_b X_b and Ys = C [hp_a | hp_b]^T (into
+//             G's columns, G being spent) are issued
+//   w o X     written over X_h once Y_h is done; S = B^T [Xw_a | Xw_b] issued
+//   ->        the B/C slot is refilled and G of chunk c+1 is issued into the
+//             columns Pm used
+//   state     h = exp(cs_last) h + S; bf16 copy -> hp; checkpoints
+//   y         Y + exp(cs_i) Ys -> bf16 -> the X slot -> TMA store
+// D x rides on the diagonal of Pm (Pm[i][i] = G[i][i] dt_i + D), so it costs
+// nothing beyond the Pm X product.
+// TMEM (512 columns): R0 = 0..127 and R1 = 128..255 alternate between {G, Ys}
+// and {Pm_a, Pm_b} by chunk parity; Y = 256..383 (a | b); S = 384..511 (a | b).
+// Shared memory: B/C ring of 2, X ring of 2 (each X slot then holds w o X and
+// finally the chunk's y), hp, and the per-head scan values (about 227 KB).
+constexpr int kThreadsC = 512;
 
 struct SmemC {
-    uint8_t cb[4 * kBox];      // C (two boxes: K 0..63, 64..127), B (two boxes); C is reused for w o X
-    uint8_t x[kBox];           // X, rows j (tokens), 128B-swizzled
-    uint8_t hp[kBox];          // bf16 h_prev, rows n, 128B-swizzled
-    float dt[kQ * 4];          // dt box: [128 tokens][4 heads]
-    uint64_t full, g_done, mma_done, fin;
+    uint8_t bc[2][4 * kBox];   // ring slot: C box 0, C box 1, B box 0, B box 1
+    uint8_t x[2][2 * kBox];    // ring slot: X of head a, X of head b
+    uint8_t hp[2 * kBox];      // bf16 h_prev of head a, head b (rows n, cols p), 128B-swizzled
+    float cvs[2][kQ];          // chunk-inclusive cumsum of dt*A (log2 units), per head
+    float dvs[2][kQ];          // dt, per head
+    float fs[2][3 * 32];       // dt_j exp(cs_end(J) - cs_j) for the 32-token blocks J = 0..2
+    uint64_t full_bc[2], full_x[2], g_done, m2a, m2b, mma_done, fin;
     uint32_t tmem;
     int abort;
 };
 
-__device__ __forceinline__ float sel4(const float (&v)[4], int i)
-{
-    return i == 0 ? v[0] : (i == 1 ? v[1] : (i == 2 ? v[2] : v[3]));
-}
-
-__global__ void __launch_bounds__(kThreadsC, 2)
+__global__ void __launch_bounds__(kThreadsC, 1)
 chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
 {
-    extern __shared__ uint8_t smraw[];
-    SmemC &s = *reinterpret_cast<SmemC *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smc_raw[];
+    SmemC &s = *reinterpret_cast<SmemC *>(smc_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int q = warp & 3, hs = warp >> 2;
-    const int r = 32 * q + lane;                 // token row / TMEM lane / state column n
+    const int q = warp & 3, cs = warp >> 2, hd = cs >> 1, p0 = 32 * (cs & 1);
+    const int r = 32 * q + lane;                 // token row / TMEM lane / state row n
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    const int HP = p.H >> 1;
     const int64_t unit = blockIdx.x;
-    const int h = (int)(unit % p.H);
-    const int64_t k = (unit / p.H) % p.ns;
-    const int bi = (int)(unit / ((int64_t)p.H * p.ns));
-    const int g = (int)((int64_t)h * p.G / p.H);
+    const int ha = 2 * (int)(unit % HP);         // head a; head b = ha + 1
+    const int64_t k = (unit / HP) % p.ns;
+    const int bi = (int)(unit / ((int64_t)HP * p.ns));
+    const int g = (int)((int64_t)ha * p.G / p.H);
     const int64_t s0 = k * p.T;
     const int64_t s1 = min(p.L, s0 + p.T);
     const int nc = (int)((s1 - s0 + kQ - 1) / kQ);
     const uint64_t lim = p.wait_limit_ns;
-    const int PN = kP * kN;
+    constexpr int PN = kP * kN;
 
+    // the 128B-swizzled tiles need a 1024-byte aligned base (no room to pad)
+    if (smem_u32(smc_raw) & 1023u) {
+        if (tid == 0) atomicOr(p.status, kDevUnsupported);
+        return;
+    }
     if (tid == 0) {
-        mbar_init(&s.full, 1);
+        for (int i = 0; i < 2; ++i) { mbar_init(&s.full_bc[i], 1); mbar_init(&s.full_x[i], 1); }
         mbar_init(&s.g_done, 1);
+        mbar_init(&s.m2a, 1);
+        mbar_init(&s.m2b, 1);
         mbar_init(&s.mma_done, 1);
         mbar_init(&s.fin, 1);
         s.abort = 0;
@@ -365,37 +355,71 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
         prefetch_tmap(&maps.x);
         prefetch_tmap(&maps.B);
         prefetch_tmap(&maps.C);
-        prefetch_tmap(&maps.dt);
+        prefetch_tmap(&maps.y);
     }
-    if (warp == 0) { tmem_alloc(&s.tmem, 256); tmem_relinquish(); }
+    if (warp == 0) { tmem_alloc(&s.tmem, 512); tmem_relinquish(); }
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = s.tmem;
-    const uint32_t tG = tm, tEC = tm, tS = tm + 64, tPm = tm + 128, tY = tm + 192;
+    const uint32_t tY = tm + 256, tS = tm + 384;
     volatile int *abort = &s.abort;
+    const bool live = unit != p.test_drop_unit;
 
-    auto issue_loads = [&](int c) {
+    // ---- thread 0: loads (and the bookkeeping needed to drain them on an abort)
+    int bc_issued = 0, bc_waited = 0, x_issued = 0, x_waited = 0;
+    auto issue_bc = [&](int c) {
         const int t0 = (int)(s0 + (int64_t)c * kQ);
-        mbar_arrive_expect_tx(&s.full, 5 * kBox + kDtBox);
-        tma_load_3d(s.cb, &maps.C, &s.full, g * kN, t0, bi);
-        tma_load_3d(s.cb + kBox, &maps.C, &s.full, g * kN + 64, t0, bi);
-        tma_load_3d(s.cb + 2 * kBox, &maps.B, &s.full, g * kN, t0, bi);
-        tma_load_3d(s.cb + 3 * kBox, &maps.B, &s.full, g * kN + 64, t0, bi);
-        tma_load_3d(s.x, &maps.x, &s.full, h * kP, t0, bi);
-        tma_load_3d(s.dt, &maps.dt, &s.full, h & ~3, t0, bi);
+        uint8_t *d = s.bc[c & 1];
+        uint64_t *bar = &s.full_bc[c & 1];
+        mbar_arrive_expect_tx(bar, 4 * kBox);
+        tma_load_3d(d, &maps.C, bar, g * kN, t0, bi);
+        tma_load_3d(d + kBox, &maps.C, bar, g * kN + 64, t0, bi);
+        tma_load_3d(d + 2 * kBox, &maps.B, bar, g * kN, t0, bi);
+        tma_load_3d(d + 3 * kBox, &maps.B, bar, g * kN + 64, t0, bi);
+        ++bc_issued;
     };
-    int pending = -1;   // (thread 0) chunk whose loads are issued but not yet waited for
-    if (tid == 0 && nc > 0 && unit != p.test_drop_unit) { issue_loads(0); pending = 0; }
+    auto issue_x = [&](int c) {
+        const int t0 = (int)(s0 + (int64_t)c * kQ);
+        uint8_t *d = s.x[c & 1];
+        uint64_t *bar = &s.full_x[c & 1];
+        mbar_arrive_expect_tx(bar, 2 * kBox);
+        tma_load_3d(d, &maps.x, bar, ha * kP, t0, bi);
+        tma_load_3d(d + kBox, &maps.x, bar, (ha + 1) * kP, t0, bi);
+        ++x_issued;
+    };
+    // G = C B^T of chunk c into the TMEM columns at tG (waits for the chunk's B/C)
+    auto issue_g = [&](int c, uint32_t tG) -> bool {
+        if (!mbar_wait(&s.full_bc[c & 1], (c >> 1) & 1, abort, lim)) return false;
+        ++bc_waited;
+        tc_fence_after();
+        const uint32_t sC = smem_u32(s.bc[c & 1]), sB = sC + 2 * kBox;
+        const uint32_t id_g = idesc_bf16(128, 128, 0, 0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+            mma_ss(tG, smem_desc(sC + off, 16, 1024), smem_desc(sB + off, 16, 1024), id_g, kk > 0);
+        }
+        mma_commit(&s.g_done);
+        return true;
+    };
+    if (tid == 0 && live) {
+        issue_bc(0);
+        if (nc > 1) issue_bc(1);
+        issue_x(0);
+        if (!issue_g(0, tm)) raise_timeout(p, abort);
+    }
 
-    // state entering the stripe: thread (r = n, hs) owns h[32 hs .. 32 hs + 31][n]
+    // ---- state entering the stripe: thread (n = r, cs) owns h[p0 .. p0 + 31][n] of head hd
+    const int hh = ha + hd;
     float hr[32];
     {
-        const float *hin = (k == 0) ? (p.h0 ? p.h0 + ((int64_t)bi * p.H + h) * PN : nullptr)
-                                    : p.ws_hin + (((int64_t)bi * p.ns + k) * p.H + h) * PN;
+        const float *hin = (k == 0) ? (p.h0 ? p.h0 + ((int64_t)bi * p.H + hh) * PN : nullptr)
+                                    : p.ws_hin + (((int64_t)bi * p.ns + k) * p.H + hh) * PN;
 #pragma unroll
-        for (int pp = 0; pp < 32; ++pp) hr[pp] = hin ? hin[(32 * hs + pp) * kN + r] : 0.0f;
+        for (int pp = 0; pp < 32; ++pp) hr[pp] = hin ? hin[(p0 + pp) * kN + r] : 0.0f;
     }
     auto write_hp = [&]() {
+        uint8_t *dst = s.hp + hd * kBox;
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
             uint4 v;
@@ -403,51 +427,58 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
             v.y = pack_bf16x2(hr[8 * c4 + 2], hr[8 * c4 + 3]);
             v.z = pack_bf16x2(hr[8 * c4 + 4], hr[8 * c4 + 5]);
             v.w = pack_bf16x2(hr[8 * c4 + 6], hr[8 * c4 + 7]);
-            sts128(s.hp + swz(r, 4 * hs + c4), v);
+            sts128(dst + swz(r, (p0 >> 3) + c4), v);
         }
     };
     write_hp();
     fence_proxy_async_smem();
 
-    const float A2 = p.A[h] * kLog2e;
-    const float Dh = p.D ? p.D[h] : 0.0f;
+    // ---- chunk cumsum: warp 0 (head a) and warp 8 (head b); dt prefetched a chunk ahead
+    const bool scan_warp = (q == 0) && ((cs & 1) == 0);
+    const float A2 = p.A[hh] * kLog2e;
+    float dvn[4];
+    auto load_dt = [&](int c) {
+        const int64_t t0 = s0 + (int64_t)c * kQ;
+#pragma unroll
+        for (int J = 0; J < 4; ++J) {
+            const int64_t t = t0 + lane + 32 * J;
+            dvn[J] = t < s1 ? p.dt[((int64_t)bi * p.L + t) * p.H + hh] : 0.0f;
+        }
+    };
+    if (scan_warp) load_dt(0);
+
+    const float Dv[2] = {p.D ? p.D[ha] : 0.0f, p.D ? p.D[ha + 1] : 0.0f};
     const int64_t n_ckpt = p.s > 0 ? p.L / p.s : 0;
-    __nv_bfloat16 *ybase = reinterpret_cast<__nv_bfloat16 *>(p.y) + (int64_t)bi * p.ybs + (int64_t)h * kP + 32 * hs;
-    const uint32_t id_g = idesc_bf16(128, 128, 0, 0);
-    const uint32_t id_kmn = idesc_bf16(128, 64, 0, 1);
-    const uint32_t id_mnmn = idesc_bf16(128, 64, 1, 1);
+    const uint32_t id_pm = idesc_bf16(128, 64, 0, 1);     // A = Pm (TMEM), B = X (MN-major)
+    const uint32_t id_ys = idesc_bf16(128, 128, 0, 1);    // A = C (K-major), B = hp (MN-major)
+    const uint32_t id_s = idesc_bf16(128, 128, 1, 1);     // A = B^T (MN-major), B = w o X (MN-major)
 
     for (int c = 0; c < nc; ++c) {
         const int64_t t0 = s0 + (int64_t)c * kQ;
-        // ---- operands of this chunk
-        bool ok = mbar_wait(&s.full, c & 1, abort, lim);
-        if (!__syncthreads_and(ok)) { raise_timeout(p, abort); break; }
-        pending = -1;
-        tc_fence_after();
-        if (tid == 0) {
-            const uint32_t sC = smem_u32(s.cb), sB = sC + 2 * kBox;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-                mma_ss(tG, smem_desc(sC + off, 16, 1024), smem_desc(sB + off, 16, 1024), id_g, kk > 0);
-            }
-            mma_commit(&s.g_done);
+        const uint32_t tG = tm + ((c & 1) ? 128u : 0u);   // G, later Ys
+        const uint32_t tPm = tm + ((c & 1) ? 0u : 128u);  // Pm_a | Pm_b
+        uint8_t *xs = s.x[c & 1];
+
+        // the other X slot is refilled once the y store that used it has read it
+        if (tid == 0 && live && c + 1 < nc) {
+            tma_store_wait_read<0>();
+            issue_x(c + 1);
         }
-        // ---- chunk cumsum (each warp on its own: lane l holds rows l + 32 J)
-        float dv[4], cv[4], fv[4], r2[4];
+        if (scan_warp) {
+            float dv[4], cv[4], r2[4];
 #pragma unroll
-        for (int J = 0; J < 4; ++J) dv[J] = s.dt[(lane + 32 * J) * 4 + (h & 3)];
+            for (int J = 0; J < 4; ++J) dv[J] = dvn[J];
+            if (c + 1 < nc) load_dt(c + 1);
 #pragma unroll
-        for (int J = 0; J < 4; ++J) {
-            float v = dv[J] * A2;
+            for (int J = 0; J < 4; ++J) {
+                float v = dv[J] * A2;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float t = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += t;
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float t = __shfl_up_sync(0xffffffffu, v, o);
+                    if (lane >= o) v += t;
+                }
+                cv[J] = v;
             }
-            cv[J] = v;
-        }
-        {
             float run = 0.0f;
 #pragma unroll
             for (int J = 0; J < 4; ++J) {
@@ -456,195 +487,210 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
                 run += bt;
                 r2[J] = run;
             }
-        }
-        const float tot2 = r2[3];
 #pragma unroll
-        for (int J = 0; J < 4; ++J) fv[J] = dv[J] * ex2(r2[J] - cv[J]);
-        const float cs2 = sel4(cv, q);
-        const float dt_r = sel4(dv, q);
-        // ---- D x into Y (this half's 32 columns of p)
-        {
-            uint32_t dx[32];
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                const uint4 xv = lds128(s.x + swz(r, 4 * hs + c4));
-                const uint32_t w4[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    dx[8 * c4 + 2 * i] = __float_as_uint(Dh * bf16_lo(w4[i]));
-                    dx[8 * c4 + 2 * i + 1] = __float_as_uint(Dh * bf16_hi(w4[i]));
-                }
-            }
-            uint32_t d0[16], d1[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) { d0[i] = dx[i]; d1[i] = dx[16 + i]; }
-            tmem_st16(tY + lane_base + 32 * hs, d0);
-            tmem_st16(tY + lane_base + 32 * hs + 16, d1);
-        }
-        // ---- masked decay Pm[r][j] = G[r][j] exp(cs_r - cs_j) dt_j (j <= r): blocks {hs, hs + 2}
-        ok = mbar_wait(&s.g_done, c & 1, abort, lim);
-        if (!__all_sync(0xffffffffu, ok)) { *abort = 1; }
-        tc_fence_after();
-        if (!*abort) {
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                const int J = 2 * jj + hs;
-                uint32_t pk[16];
-                if (J < q) {
-                    const float E = ex2(cs2 - sel4(r2, J));
-                    uint32_t gv[32];
-                    tmem_ld32(tG + lane_base + 32 * J, gv);
-                    tmem_wait_ld();
-                    const float fJ = sel4(fv, J);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float f0 = __shfl_sync(0xffffffffu, fJ, 2 * i);
-                        const float f1 = __shfl_sync(0xffffffffu, fJ, 2 * i + 1);
-                        pk[i] = pack_bf16x2(__uint_as_float(gv[2 * i]) * f0 * E,
-                                            __uint_as_float(gv[2 * i + 1]) * f1 * E);
-                    }
-                } else if (J == q) {
-                    uint32_t gv[32];
-                    tmem_ld32(tG + lane_base + 32 * J, gv);
-                    tmem_wait_ld();
-                    const float cJ = sel4(cv, J), dJ = sel4(dv, J);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float c0 = __shfl_sync(0xffffffffu, cJ, 2 * i);
-                        const float c1 = __shfl_sync(0xffffffffu, cJ, 2 * i + 1);
-                        const float d0 = __shfl_sync(0xffffffffu, dJ, 2 * i);
-                        const float d1 = __shfl_sync(0xffffffffu, dJ, 2 * i + 1);
-                        float v0 = __uint_as_float(gv[2 * i]) * ex2(cs2 - c0) * d0;
-                        float v1 = __uint_as_float(gv[2 * i + 1]) * ex2(cs2 - c1) * d1;
-                        if (2 * i > lane) v0 = 0.0f;
-                        if (2 * i + 1 > lane) v1 = 0.0f;
-                        pk[i] = pack_bf16x2(v0, v1);
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) pk[i] = 0u;
-                }
-                tmem_st16(tPm + lane_base + 16 * J, pk);
+            for (int J = 0; J < 4; ++J) {
+                s.cvs[hd][lane + 32 * J] = cv[J];
+                s.dvs[hd][lane + 32 * J] = dv[J];
+                if (J < 3) s.fs[hd][lane + 32 * J] = dv[J] * ex2(r2[J] - cv[J]);
             }
         }
-        tmem_wait_st();
-        tc_fence_before();
-        if (__syncthreads_or(*abort)) { raise_timeout(p, abort); break; }   // all reads of G done
-        tc_fence_after();
-        // ---- EC = exp(cs_r) C_r over G's columns 0..63 (this half: K = 64 hs .. 64 hs + 63)
-        {
-            const float e = ex2(cs2);
-            const uint8_t *cbox = s.cb + hs * kBox;
-#pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-                uint32_t ev[16];
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    const uint4 cvv = lds128(cbox + swz(r, 4 * q2 + c4));
-                    ev[4 * c4 + 0] = scale_bf16x2(cvv.x, e);
-                    ev[4 * c4 + 1] = scale_bf16x2(cvv.y, e);
-                    ev[4 * c4 + 2] = scale_bf16x2(cvv.z, e);
-                    ev[4 * c4 + 3] = scale_bf16x2(cvv.w, e);
-                }
-                tmem_st16(tEC + lane_base + 32 * hs + 16 * q2, ev);
-            }
-        }
-        tmem_wait_st();
-        __syncthreads();   // every read of C is done: w o X may overwrite it
-        // ---- w o X for the state update, written over C's first box (rows j, same swizzle)
-        {
-            const float w = dt_r * ex2(tot2 - cs2);
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                const int cc = 4 * hs + c4;
-                uint4 vv = lds128(s.x + swz(r, cc));
-                vv.x = scale_bf16x2(vv.x, w); vv.y = scale_bf16x2(vv.y, w);
-                vv.z = scale_bf16x2(vv.z, w); vv.w = scale_bf16x2(vv.w, w);
-                sts128(s.cb + swz(r, cc), vv);
-            }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
         __syncthreads();
+
+        // ---- masked decay of head hm into Pm_hm: this warp takes column block J = cs of its rows
+        auto mask = [&](int hm) {
+            const int J = cs;
+            uint32_t pk[16];
+            if (J < q) {
+                const float E = ex2(s.cvs[hm][r] - s.cvs[hm][32 * J + 31]);
+                uint32_t gv[32];
+                tmem_ld32(tG + lane_base + 32 * J, gv);
+                tmem_wait_ld();
+                const float4 *f4 = reinterpret_cast<const float4 *>(&s.fs[hm][32 * J]);
+#pragma unroll
+                for (int i4 = 0; i4 < 8; ++i4) {
+                    const float4 f = f4[i4];
+                    pk[2 * i4] = pack_bf16x2(__uint_as_float(gv[4 * i4]) * (f.x * E),
+                                             __uint_as_float(gv[4 * i4 + 1]) * (f.y * E));
+                    pk[2 * i4 + 1] = pack_bf16x2(__uint_as_float(gv[4 * i4 + 2]) * (f.z * E),
+                                                 __uint_as_float(gv[4 * i4 + 3]) * (f.w * E));
+                }
+            } else if (J == q) {
+                const float csr = s.cvs[hm][r];
+                const float Dm = Dv[hm];
+                uint32_t gv[32];
+                tmem_ld32(tG + lane_base + 32 * J, gv);
+                tmem_wait_ld();
+                const float4 *c4 = reinterpret_cast<const float4 *>(&s.cvs[hm][32 * J]);
+                const float4 *d4 = reinterpret_cast<const float4 *>(&s.dvs[hm][32 * J]);
+#pragma unroll
+                for (int i4 = 0; i4 < 8; ++i4) {
+                    const float4 cc = c4[i4], dd = d4[i4];
+                    const float ca[4] = {cc.x, cc.y, cc.z, cc.w}, da[4] = {dd.x, dd.y, dd.z, dd.w};
+                    float v[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = 4 * i4 + e;
+                        const float t = __uint_as_float(gv[i]) * ex2(csr - ca[e]) * da[e];
+                        v[e] = i > lane ? 0.0f : (i == lane ? t + Dm : t);
+                    }
+                    pk[2 * i4] = pack_bf16x2(v[0], v[1]);
+                    pk[2 * i4 + 1] = pack_bf16x2(v[2], v[3]);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pk[i] = 0u;
+            }
+            tmem_st16(tPm + lane_base + 64 * hm + 16 * J, pk);
+        };
+
+        // ---- head a
+        bool ok = ewait(&s.g_done, c & 1, abort, lim);
         tc_fence_after();
+        if (ok) mask(0);
+        tmem_wait_st();
+        tc_fence_before();
+        if (__syncthreads_or(!ok || *abort)) { raise_timeout(p, abort); break; }
         if (tid == 0) {
-            const uint32_t sX = smem_u32(s.x), sHp = smem_u32(s.hp), sXw = smem_u32(s.cb);
-            const uint32_t sB = sXw + 2 * kBox;
+            tc_fence_after();
+            if (mbar_wait(&s.full_x[c & 1], (c >> 1) & 1, abort, lim)) {
+                ++x_waited;
+                const uint32_t sX = smem_u32(xs);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tY, tPm + kk * 8, smem_desc(sX + kk * 2048, 0, 1024), id_pm, kk > 0);
+                mma_commit(&s.m2a);
+            } else {
+                raise_timeout(p, abort);
+            }
+        }
+        // ---- head b, then C hp^T over the spent G
+        mask(1);
+        tmem_wait_st();
+        tc_fence_before();
+        if (__syncthreads_or(*abort)) { raise_timeout(p, abort); break; }
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t sX = smem_u32(xs) + kBox;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                mma_ts(tY, tPm + kk * 8, smem_desc(sX + kk * 2048, 0, 1024), id_kmn, true);
+                mma_ts(tY + 64, tPm + 64 + kk * 8, smem_desc(sX + kk * 2048, 0, 1024), id_pm, kk > 0);
+            mma_commit(&s.m2b);
+            const uint32_t sC = smem_u32(s.bc[c & 1]), sHp = smem_u32(s.hp);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+                mma_ss(tG, smem_desc(sC + off, 16, 1024), smem_desc(sHp + kk * 2048, kBox, 1024), id_ys, kk > 0);
+            }
+        }
+        // ---- w o X over X_h once Y_h has read X_h; 4 threads per token row
+        auto xw = [&](int hm) {
+            const int j = tid >> 2, ch = 2 * (tid & 3);
+            const float w = s.dvs[hm][j] * ex2(s.cvs[hm][kQ - 1] - s.cvs[hm][j]);
+            uint8_t *base = xs + hm * kBox;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                uint4 v = lds128(base + swz(j, ch + u));
+                v.x = scale_bf16x2(v.x, w); v.y = scale_bf16x2(v.y, w);
+                v.z = scale_bf16x2(v.z, w); v.w = scale_bf16x2(v.w, w);
+                sts128(base + swz(j, ch + u), v);
+            }
+        };
+        // (X_c's landing is waited for here too, so that its bytes are visible to this thread)
+        ok = mbar_wait(&s.full_x[c & 1], (c >> 1) & 1, abort, lim) && mbar_wait(&s.m2a, c & 1, abort, lim);
+        if (ok) xw(0);
+        ok = ok && mbar_wait(&s.m2b, c & 1, abort, lim);
+        if (ok) xw(1);
+        fence_proxy_async_smem();
+        if (__syncthreads_or(!ok || *abort)) { raise_timeout(p, abort); break; }
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t sB = smem_u32(s.bc[c & 1]) + 2 * kBox, sXw = smem_u32(xs);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                mma_ts(tY, tEC + kk * 8, smem_desc(sHp + kk * 2048, 0, 1024), id_kmn, true);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                mma_ss(tS, smem_desc(sB + kk * 2048, kBox, 1024), smem_desc(sXw + kk * 2048, 0, 1024),
-                       id_mnmn, kk > 0);
+                mma_ss(tS, smem_desc(sB + kk * 2048, kBox, 1024), smem_desc(sXw + kk * 2048, kBox, 1024), id_s, kk > 0);
             mma_commit(&s.mma_done);
         }
-        ok = mbar_wait(&s.mma_done, c & 1, abort, lim);
-        if (!__syncthreads_and(ok)) { raise_timeout(p, abort); break; }
+        ok = ewait(&s.mma_done, c & 1, abort, lim);
         tc_fence_after();
-        // every operand slot is free: fetch the next chunk while this one finishes
-        if (tid == 0 && c + 1 < nc) {
-            issue_loads(c + 1);
-            pending = c + 1;
+        // every operand of chunk c is consumed: refill its B/C slot, start G of chunk c+1
+        if (tid == 0 && ok && live) {
+            if (c + 2 < nc) issue_bc(c + 2);
+            if (c + 1 < nc && !issue_g(c + 1, tPm)) raise_timeout(p, abort);
         }
-        // ---- y = Y, this half's 32 columns
-        {
-            uint32_t yv[32];
-            tmem_ld32(tY + lane_base + 32 * hs, yv);
-            tmem_wait_ld();
-            if (t0 + r < s1) {
-                __nv_bfloat16 *yrow = ybase + (t0 + r) * p.yrs;
+        if (ok) {
+            // ---- state: h = exp(cs_last) h + S (columns p0.. of head hd, state row n = r)
+            {
+                uint32_t sa[32];
+                tmem_ld32(tS + lane_base + 32 * cs, sa);
+                tmem_wait_ld();
+                const float dec = ex2(s.cvs[hd][kQ - 1]);
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    uint32_t o4[4];
+                for (int pp = 0; pp < 32; ++pp) hr[pp] = fmaf(dec, hr[pp], __uint_as_float(sa[pp]));
+            }
+            if (c + 1 < nc) write_hp();
+            // ---- y = Y + exp(cs_r) Ys -> bf16, staged in the X slot (same swizzle as the y map)
+            {
+                const float e = ex2(s.cvs[hd][r]);
+                uint8_t *dst = xs + hd * kBox;
 #pragma unroll
-                    for (int e2 = 0; e2 < 4; ++e2)
-                        o4[e2] = pack_bf16x2(__uint_as_float(yv[8 * c4 + 2 * e2]), __uint_as_float(yv[8 * c4 + 2 * e2 + 1]));
-                    *reinterpret_cast<uint4 *>(yrow + 8 * c4) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t yv[16], ys[16];
+                    tmem_ld16(tY + lane_base + 32 * cs + 16 * hf, yv);
+                    tmem_ld16(tG + lane_base + 32 * cs + 16 * hf, ys);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c2 = 0; c2 < 2; ++c2) {
+                        uint4 v;
+                        uint32_t *vw = reinterpret_cast<uint32_t *>(&v);
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            const int i = 8 * c2 + 2 * e2;
+                            vw[e2] = pack_bf16x2(fmaf(e, __uint_as_float(ys[i]), __uint_as_float(yv[i])),
+                                                 fmaf(e, __uint_as_float(ys[i + 1]), __uint_as_float(yv[i + 1])));
+                        }
+                        sts128(dst + swz(r, (p0 >> 3) + 2 * hf + c2), v);
+                    }
+                }
+            }
+            const int64_t t_end = t0 + kQ;
+            if (p.h_ckpt && p.s > 0 && t_end <= s1 && t_end % p.s == 0) {
+                const int64_t kc = t_end / p.s - 1;
+                if (kc < n_ckpt) {
+                    float *dst = p.h_ckpt + (((int64_t)bi * n_ckpt + kc) * p.H + hh) * PN + (int64_t)p0 * kN + r;
+#pragma unroll
+                    for (int pp = 0; pp < 32; ++pp) dst[pp * kN] = hr[pp];
                 }
             }
         }
-        // ---- state: h = exp(cs_last) h + S  (columns p of this half, state column n = r)
-        {
-            uint32_t sa[32];
-            tmem_ld32(tS + lane_base + 32 * hs, sa);
-            tmem_wait_ld();
-            const float dec = ex2(tot2);
-#pragma unroll
-            for (int pp = 0; pp < 32; ++pp) hr[pp] = fmaf(dec, hr[pp], __uint_as_float(sa[pp]));
-        }
-        if (c + 1 < nc) {
-            write_hp();
-            fence_proxy_async_smem();   // before the barrier that orders it with the next MMAs
-        }
-        const int64_t t_end = t0 + kQ;
-        if (p.h_ckpt && p.s > 0 && t_end <= s1 && t_end % p.s == 0) {
-            const int64_t kk = t_end / p.s - 1;
-            if (kk < n_ckpt) {
-                float *dst = p.h_ckpt + (((int64_t)bi * n_ckpt + kk) * p.H + h) * PN + (int64_t)(32 * hs) * kN + r;
-#pragma unroll
-                for (int pp = 0; pp < 32; ++pp) dst[pp * kN] = hr[pp];
-            }
-        }
+        fence_proxy_async_smem();   // hp for the next C hp^T, y for the store
         tc_fence_before();
+        if (__syncthreads_or(!ok || *abort)) { raise_timeout(p, abort); break; }
+        if (tid == 0 && live) {
+            tma_store_3d(&maps.y, xs, ha * kP, (int)t0, bi);
+            tma_store_3d(&maps.y, xs + kBox, (ha + 1) * kP, (int)t0, bi);
+            tma_store_commit();
+        }
     }
     if (!*abort && p.h_final && s1 == p.L) {
-        float *dst = p.h_final + ((int64_t)bi * p.H + h) * PN + (int64_t)(32 * hs) * kN + r;
+        float *dst = p.h_final + ((int64_t)bi * p.H + hh) * PN + (int64_t)p0 * kN + r;
 #pragma unroll
         for (int pp = 0; pp < 32; ++pp) dst[pp * kN] = hr[pp];
     }
-    // drain: MMAs and loads that may still be in flight after an abort
-    if (tid == 0 && *abort) {
-        mma_commit(&s.fin);
-        mbar_wait(&s.fin, 0, nullptr, 100000000ull);
-        if (pending >= 0) mbar_wait(&s.full, pending & 1, nullptr, 100000000ull);
+    if (tid == 0) {
+        if (*abort) {
+            // drain: MMAs, then every load still in flight
+            mma_commit(&s.fin);
+            mbar_wait(&s.fin, 0, nullptr, 100000000ull);
+            for (int i = bc_waited; i < bc_issued; ++i)
+                mbar_wait(&s.full_bc[i & 1], (i >> 1) & 1, nullptr, 100000000ull);
+            for (int i = x_waited; i < x_issued; ++i)
+                mbar_wait(&s.full_x[i & 1], (i >> 1) & 1, nullptr, 100000000ull);
+        }
+        tma_store_wait<0>();
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tm, 256);
+    if (warp == 0) tmem_dealloc(tm, 512);
 }
 
 // =============================================================== host side
@@ -694,7 +740,7 @@ bool encode_dt(EncodeTiledFn enc, CUtensorMap *m, const float *dt, int H, int64_
 }
 
 constexpr size_t kSmemA = sizeof(SmemA) + 1024;
-constexpr size_t kSmemC = sizeof(SmemC) + 1024;
+constexpr size_t kSmemC = sizeof(SmemC);   // no alignment pad: the base is checked in the kernel
 static_assert(kSmemC <= 232448, "pass C shared memory");
 static_assert(kSmemA <= 232448, "pass A shared memory");
 
@@ -718,7 +764,8 @@ int launch_scan_tc(const ScanParams &p, cudaStream_t st)
     if (!encode_bf16(enc, &maps.x, p.x, (int64_t)p.H * p.P, p.L, p.b, p.xrs, p.xbs) ||
         !encode_bf16(enc, &maps.B, p.B, gn, p.L, p.b, p.Brs, p.Bbs) ||
         !encode_bf16(enc, &maps.C, p.C, gn, p.L, p.b, p.Crs, p.Cbs) ||
-        !encode_dt(enc, &maps.dt, p.dt, p.H, p.L, p.b))
+        !encode_dt(enc, &maps.dt, p.dt, p.H, p.L, p.b) ||
+        !encode_bf16(enc, &maps.y, p.y, (int64_t)p.H * p.P, p.L, p.b, p.yrs, p.ybs))
         return 6;
     static bool attr_set[64] = {false};
     int dev = 0;
@@ -738,7 +785,7 @@ int launch_scan_tc(const ScanParams &p, cudaStream_t st)
         if (rc) return rc;
     }
     prof_begin(st, kKOutputTc);
-    chunk_output_tc_kernel<<<(unsigned)units, kThreadsC, kSmemC, st>>>(maps, p);
+    chunk_output_tc_kernel<<<(unsigned)(units / 2), kThreadsC, kSmemC, st>>>(maps, p);
     prof_end(st, kKOutputTc);
     return cudaGetLastError() == cudaSuccess ? 0 : 7;
 }

@@ -8,7 +8,7 @@
 namespace ssd {
 
 // Device status codes latched by kernels (mirrors ssd_status in include/ssd.h).
-enum : unsigned int { kDevOk = 0u, kDevTimeout = 8u };
+enum : unsigned int { kDevOk = 0u, kDevUnsupported = 6u, kDevTimeout = 8u };
 
 // Everything a scan kernel needs, passed by value.
 struct ScanParams {
