@@ -283,27 +283,39 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
 }
 
 // =============================================================== pass C
-// One CTA per (stripe, head pair), one CTA per SM.  The two heads share their
-// B and C tiles and G = C B^T; the chunks of the stripe are walked in order.
-// Thread = TMEM lane quarter q (warp & 3) x column slice cs (warp >> 2); the
-// column slices 0,1 belong to head a, 2,3 to head b.  Per chunk c:
-//   scan      warps 0 and 8: chunk cumsum of dt*A of head a / b -> smem
-//   mask a    Pm_a = G o [exp(cs_i - cs_j) dt_j]_{j<=i} (+ D on the diagonal),
-//             then Y_a = Pm_a X_a is issued
-//   mask b    likewise; then Y_b = Pm_b X_b and Ys = C [hp_a | hp_b]^T (into
-//             G's columns, G being spent) are issued
-//   w o X     written over X_h once Y_h is done; S = B^T [Xw_a | Xw_b] issued
-//   ->        the B/C slot is refilled and G of chunk c+1 is issued into the
-//             columns Pm used
-//   state     h = exp(cs_last) h + S; bf16 copy -> hp; checkpoints
-//   y         Y + exp(cs_i) Ys -> bf16 -> the X slot -> TMA store
-// D x rides on the diagonal of Pm (Pm[i][i] = G[i][i] dt_i + D), so it costs
-// nothing beyond the Pm X product.
+// One CTA per (stripe, head pair), one CTA per SM: 16 compute warps and one
+// issuing warp.  The two heads share their B and C tiles and G = C B^T; the
+// chunks of the stripe are walked in order.
+//
+// Issuing warp, per chunk c (the whole warp waits, one lane issues):
+//   Pm ready -> Y_a = Pm_a X_a, Y_b = Pm_b X_b, Ys = C [hp_a | hp_b]^T (into G's
+//   columns, G being spent), then the other X slot (y of chunk c-1, stored by
+//   now) is refilled with chunk c+1; w o X ready -> S = B^T [Xw_a | Xw_b],
+//   accumulated straight into the fp32 state H in TMEM;
+//   products done -> refill the B/C slot, G of chunk c+1 into the columns Pm used;
+//   y staged -> TMA store of y.
+// Warp 4 (no masked-decay work of its own) also publishes the chunk cumsum of
+// dt*A of both heads for chunk c+1 once the products of chunk c are done.
+// Compute warp (TMEM lane quarter q = warp & 3, column slice cs = warp >> 2 of
+// the 128 (head, p) columns; head hd = cs >> 1), per chunk:
+//   mask: Pm columns 32 cs .. 32 cs + 31, i.e. head hd's 32-token column
+//         blocks 2 (cs & 1) and 2 (cs & 1) + 1 of its 32 rows:
+//         Pm[i][j] = G[i][j] exp(cs_i - cs_j) dt_j (j <= i), + D on the diagonal
+//   w o X over X_hd (rows split over the head's 8 warps) once Y_hd is done
+//   state (before the mask): H holds h after the previous chunk; its bf16 copy
+//         -> hp, checkpoint, then H = exp(cs_last) H, to which S is added
+//   y = Y + exp(cs_i) Ys -> bf16 -> the X slot (same swizzle as the y map)
+// A warp writes Pm into exactly the columns it read Ys from one chunk earlier,
+// and reads Y / S / Ys columns only it owns, so no barrier among the compute
+// warps is needed; hand-offs go through mbarriers (one arrival per warp).
+// D x rides on the diagonal of Pm (Pm[i][i] = G[i][i] dt_i + D).
 // TMEM (512 columns): R0 = 0..127 and R1 = 128..255 alternate between {G, Ys}
-// and {Pm_a, Pm_b} by chunk parity; Y = 256..383 (a | b); S = 384..511 (a | b).
+// and {Pm_a, Pm_b} by chunk parity; Y = 256..383 (a | b); H = 384..511 (a | b),
+// the fp32 state, rows n.
 // Shared memory: B/C ring of 2, X ring of 2 (each X slot then holds w o X and
 // finally the chunk's y), hp, and the per-head scan values (about 227 KB).
-constexpr int kThreadsC = 512;
+constexpr int kComputeWarps = 16;
+constexpr int kThreadsC = 32 * (kComputeWarps + 1);
 
 struct SmemC {
     uint8_t bc[2][4 * kBox];   // ring slot: C box 0, C box 1, B box 0, B box 1
@@ -312,10 +324,23 @@ struct SmemC {
     float cvs[2][kQ];          // chunk-inclusive cumsum of dt*A (log2 units), per head
     float dvs[2][kQ];          // dt, per head
     float fs[2][3 * 32];       // dt_j exp(cs_end(J) - cs_j) for the 32-token blocks J = 0..2
-    uint64_t full_bc[2], full_x[2], g_done, m2a, m2b, mma_done, fin;
+    uint64_t full_bc[2], full_x[2], g_done, m2a, m2b, mma_done, fin;   // TMA / MMA -> warps
+    uint64_t pm_ready, xw_ready, y_ready, scan_ready;                  // warps -> issuing warp
     uint32_t tmem;
     int abort;
 };
+
+// two fp32 products in one instruction (sm_100 packed fp32)
+__device__ __forceinline__ float2 mul2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
 
 __global__ void __launch_bounds__(kThreadsC, 1)
 chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
@@ -323,9 +348,6 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
     extern __shared__ __align__(1024) uint8_t smc_raw[];
     SmemC &s = *reinterpret_cast<SmemC *>(smc_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int q = warp & 3, cs = warp >> 2, hd = cs >> 1, p0 = 32 * (cs & 1);
-    const int r = 32 * q + lane;                 // token row / TMEM lane / state row n
-    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     const int HP = p.H >> 1;
     const int64_t unit = blockIdx.x;
     const int ha = 2 * (int)(unit % HP);         // head a; head b = ha + 1
@@ -350,6 +372,10 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
         mbar_init(&s.m2b, 1);
         mbar_init(&s.mma_done, 1);
         mbar_init(&s.fin, 1);
+        mbar_init(&s.pm_ready, kComputeWarps);
+        mbar_init(&s.xw_ready, kComputeWarps);
+        mbar_init(&s.y_ready, kComputeWarps);
+        mbar_init(&s.scan_ready, 1);
         s.abort = 0;
         fence_mbar_init();
         prefetch_tmap(&maps.x);
@@ -361,276 +387,220 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = s.tmem;
-    const uint32_t tY = tm + 256, tS = tm + 384;
+    const uint32_t tY = tm + 256, tH = tm + 384;
     volatile int *abort = &s.abort;
     const bool live = unit != p.test_drop_unit;
 
-    // ---- thread 0: loads (and the bookkeeping needed to drain them on an abort)
-    int bc_issued = 0, bc_waited = 0, x_issued = 0, x_waited = 0;
-    auto issue_bc = [&](int c) {
-        const int t0 = (int)(s0 + (int64_t)c * kQ);
-        uint8_t *d = s.bc[c & 1];
-        uint64_t *bar = &s.full_bc[c & 1];
-        mbar_arrive_expect_tx(bar, 4 * kBox);
-        tma_load_3d(d, &maps.C, bar, g * kN, t0, bi);
-        tma_load_3d(d + kBox, &maps.C, bar, g * kN + 64, t0, bi);
-        tma_load_3d(d + 2 * kBox, &maps.B, bar, g * kN, t0, bi);
-        tma_load_3d(d + 3 * kBox, &maps.B, bar, g * kN + 64, t0, bi);
-        ++bc_issued;
-    };
-    auto issue_x = [&](int c) {
-        const int t0 = (int)(s0 + (int64_t)c * kQ);
-        uint8_t *d = s.x[c & 1];
-        uint64_t *bar = &s.full_x[c & 1];
-        mbar_arrive_expect_tx(bar, 2 * kBox);
-        tma_load_3d(d, &maps.x, bar, ha * kP, t0, bi);
-        tma_load_3d(d + kBox, &maps.x, bar, (ha + 1) * kP, t0, bi);
-        ++x_issued;
-    };
-    // G = C B^T of chunk c into the TMEM columns at tG (waits for the chunk's B/C)
-    auto issue_g = [&](int c, uint32_t tG) -> bool {
-        if (!mbar_wait(&s.full_bc[c & 1], (c >> 1) & 1, abort, lim)) return false;
-        ++bc_waited;
-        tc_fence_after();
-        const uint32_t sC = smem_u32(s.bc[c & 1]), sB = sC + 2 * kBox;
-        const uint32_t id_g = idesc_bf16(128, 128, 0, 0);
+    if (warp < kComputeWarps) {
+        // ================================================= compute warps
+        const int q = warp & 3, cs = warp >> 2, hd = cs >> 1, p0 = 32 * (cs & 1);
+        const int r = 32 * q + lane;             // token row / TMEM lane / state row n
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        const int hh = ha + hd;
+        auto fail = [&]() { if (lane == 0) raise_timeout(p, abort); };
+
+        // state entering the stripe -> H: thread (n = r, cs) owns h[p0 .. p0 + 31][n] of head hh
+        {
+            const float *hin = (k == 0) ? (p.h0 ? p.h0 + ((int64_t)bi * p.H + hh) * PN : nullptr)
+                                        : p.ws_hin + (((int64_t)bi * p.ns + k) * p.H + hh) * PN;
+            uint32_t hv[32];
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-            mma_ss(tG, smem_desc(sC + off, 16, 1024), smem_desc(sB + off, 16, 1024), id_g, kk > 0);
+            for (int pp = 0; pp < 32; ++pp) hv[pp] = __float_as_uint(hin ? hin[(p0 + pp) * kN + r] : 0.0f);
+            tmem_st32(tH + lane_base + 32 * cs, hv);
+            tmem_wait_st();
         }
-        mma_commit(&s.g_done);
-        return true;
-    };
-    if (tid == 0 && live) {
-        issue_bc(0);
-        if (nc > 1) issue_bc(1);
-        issue_x(0);
-        if (!issue_g(0, tm)) raise_timeout(p, abort);
-    }
-
-    // ---- state entering the stripe: thread (n = r, cs) owns h[p0 .. p0 + 31][n] of head hd
-    const int hh = ha + hd;
-    float hr[32];
-    {
-        const float *hin = (k == 0) ? (p.h0 ? p.h0 + ((int64_t)bi * p.H + hh) * PN : nullptr)
-                                    : p.ws_hin + (((int64_t)bi * p.ns + k) * p.H + hh) * PN;
+        // the checkpoint slot of the state after the chunk ending at t_end, or -1
+        const int64_t n_ckpt = p.s > 0 ? p.L / p.s : 0;
+        auto ckpt_slot = [&](int64_t t_end) -> int64_t {
+            if (!p.h_ckpt || p.s <= 0 || t_end > s1 || t_end % p.s != 0) return -1;
+            const int64_t kc = t_end / p.s - 1;
+            return kc < n_ckpt ? kc : -1;
+        };
+        auto store_state = [&](float *dst, const uint32_t (&hv)[32]) {
 #pragma unroll
-        for (int pp = 0; pp < 32; ++pp) hr[pp] = hin ? hin[(p0 + pp) * kN + r] : 0.0f;
-    }
-    auto write_hp = [&]() {
-        uint8_t *dst = s.hp + hd * kBox;
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-            uint4 v;
-            v.x = pack_bf16x2(hr[8 * c4 + 0], hr[8 * c4 + 1]);
-            v.y = pack_bf16x2(hr[8 * c4 + 2], hr[8 * c4 + 3]);
-            v.z = pack_bf16x2(hr[8 * c4 + 4], hr[8 * c4 + 5]);
-            v.w = pack_bf16x2(hr[8 * c4 + 6], hr[8 * c4 + 7]);
-            sts128(dst + swz(r, (p0 >> 3) + c4), v);
-        }
-    };
-    write_hp();
-    fence_proxy_async_smem();
-
-    // ---- chunk cumsum: warp 0 (head a) and warp 8 (head b); dt prefetched a chunk ahead
-    const bool scan_warp = (q == 0) && ((cs & 1) == 0);
-    const float A2 = p.A[hh] * kLog2e;
-    float dvn[4];
-    auto load_dt = [&](int c) {
-        const int64_t t0 = s0 + (int64_t)c * kQ;
-#pragma unroll
-        for (int J = 0; J < 4; ++J) {
-            const int64_t t = t0 + lane + 32 * J;
-            dvn[J] = t < s1 ? p.dt[((int64_t)bi * p.L + t) * p.H + hh] : 0.0f;
-        }
-    };
-    if (scan_warp) load_dt(0);
-
-    const float Dv[2] = {p.D ? p.D[ha] : 0.0f, p.D ? p.D[ha + 1] : 0.0f};
-    const int64_t n_ckpt = p.s > 0 ? p.L / p.s : 0;
-    const uint32_t id_pm = idesc_bf16(128, 64, 0, 1);     // A = Pm (TMEM), B = X (MN-major)
-    const uint32_t id_ys = idesc_bf16(128, 128, 0, 1);    // A = C (K-major), B = hp (MN-major)
-    const uint32_t id_s = idesc_bf16(128, 128, 1, 1);     // A = B^T (MN-major), B = w o X (MN-major)
-
-    for (int c = 0; c < nc; ++c) {
-        const int64_t t0 = s0 + (int64_t)c * kQ;
-        const uint32_t tG = tm + ((c & 1) ? 128u : 0u);   // G, later Ys
-        const uint32_t tPm = tm + ((c & 1) ? 0u : 128u);  // Pm_a | Pm_b
-        uint8_t *xs = s.x[c & 1];
-
-        // the other X slot is refilled once the y store that used it has read it
-        if (tid == 0 && live && c + 1 < nc) {
-            tma_store_wait_read<0>();
-            issue_x(c + 1);
-        }
-        if (scan_warp) {
-            float dv[4], cv[4], r2[4];
-#pragma unroll
-            for (int J = 0; J < 4; ++J) dv[J] = dvn[J];
-            if (c + 1 < nc) load_dt(c + 1);
-#pragma unroll
-            for (int J = 0; J < 4; ++J) {
-                float v = dv[J] * A2;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float t = __shfl_up_sync(0xffffffffu, v, o);
-                    if (lane >= o) v += t;
-                }
-                cv[J] = v;
-            }
-            float run = 0.0f;
-#pragma unroll
-            for (int J = 0; J < 4; ++J) {
-                const float bt = __shfl_sync(0xffffffffu, cv[J], 31);
-                cv[J] += run;
-                run += bt;
-                r2[J] = run;
-            }
-#pragma unroll
-            for (int J = 0; J < 4; ++J) {
-                s.cvs[hd][lane + 32 * J] = cv[J];
-                s.dvs[hd][lane + 32 * J] = dv[J];
-                if (J < 3) s.fs[hd][lane + 32 * J] = dv[J] * ex2(r2[J] - cv[J]);
-            }
-        }
-        __syncthreads();
-
-        // ---- masked decay of head hm into Pm_hm: this warp takes column block J = cs of its rows
-        auto mask = [&](int hm) {
-            const int J = cs;
-            uint32_t pk[16];
-            if (J < q) {
-                const float E = ex2(s.cvs[hm][r] - s.cvs[hm][32 * J + 31]);
-                uint32_t gv[32];
-                tmem_ld32(tG + lane_base + 32 * J, gv);
-                tmem_wait_ld();
-                const float4 *f4 = reinterpret_cast<const float4 *>(&s.fs[hm][32 * J]);
-#pragma unroll
-                for (int i4 = 0; i4 < 8; ++i4) {
-                    const float4 f = f4[i4];
-                    pk[2 * i4] = pack_bf16x2(__uint_as_float(gv[4 * i4]) * (f.x * E),
-                                             __uint_as_float(gv[4 * i4 + 1]) * (f.y * E));
-                    pk[2 * i4 + 1] = pack_bf16x2(__uint_as_float(gv[4 * i4 + 2]) * (f.z * E),
-                                                 __uint_as_float(gv[4 * i4 + 3]) * (f.w * E));
-                }
-            } else if (J == q) {
-                const float csr = s.cvs[hm][r];
-                const float Dm = Dv[hm];
-                uint32_t gv[32];
-                tmem_ld32(tG + lane_base + 32 * J, gv);
-                tmem_wait_ld();
-                const float4 *c4 = reinterpret_cast<const float4 *>(&s.cvs[hm][32 * J]);
-                const float4 *d4 = reinterpret_cast<const float4 *>(&s.dvs[hm][32 * J]);
-#pragma unroll
-                for (int i4 = 0; i4 < 8; ++i4) {
-                    const float4 cc = c4[i4], dd = d4[i4];
-                    const float ca[4] = {cc.x, cc.y, cc.z, cc.w}, da[4] = {dd.x, dd.y, dd.z, dd.w};
-                    float v[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i = 4 * i4 + e;
-                        const float t = __uint_as_float(gv[i]) * ex2(csr - ca[e]) * da[e];
-                        v[e] = i > lane ? 0.0f : (i == lane ? t + Dm : t);
-                    }
-                    pk[2 * i4] = pack_bf16x2(v[0], v[1]);
-                    pk[2 * i4 + 1] = pack_bf16x2(v[2], v[3]);
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) pk[i] = 0u;
-            }
-            tmem_st16(tPm + lane_base + 64 * hm + 16 * J, pk);
+            for (int pp = 0; pp < 32; ++pp) dst[pp * kN] = __uint_as_float(hv[pp]);
+        };
+        auto ckpt_ptr = [&](int64_t kc) {
+            return p.h_ckpt + (((int64_t)bi * n_ckpt + kc) * p.H + hh) * PN + (int64_t)p0 * kN + r;
         };
 
-        // ---- head a
-        bool ok = ewait(&s.g_done, c & 1, abort, lim);
-        tc_fence_after();
-        if (ok) mask(0);
-        tmem_wait_st();
-        tc_fence_before();
-        if (__syncthreads_or(!ok || *abort)) { raise_timeout(p, abort); break; }
-        if (tid == 0) {
-            tc_fence_after();
-            if (mbar_wait(&s.full_x[c & 1], (c >> 1) & 1, abort, lim)) {
-                ++x_waited;
-                const uint32_t sX = smem_u32(xs);
+        // chunk cumsum of both heads (warp 4, which has no masked-decay work): lane l holds
+        // tokens 4 l .. 4 l + 3; dt is prefetched a chunk ahead
+        const float A2a = p.A[ha] * kLog2e, A2b = p.A[ha + 1] * kLog2e;
+        float2 dtn[4];
+        auto load_dt = [&](int c) {
+            const int64_t t0 = s0 + (int64_t)c * kQ;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tY, tPm + kk * 8, smem_desc(sX + kk * 2048, 0, 1024), id_pm, kk > 0);
-                mma_commit(&s.m2a);
-            } else {
-                raise_timeout(p, abort);
-            }
-        }
-        // ---- head b, then C hp^T over the spent G
-        mask(1);
-        tmem_wait_st();
-        tc_fence_before();
-        if (__syncthreads_or(*abort)) { raise_timeout(p, abort); break; }
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t sX = smem_u32(xs) + kBox;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                mma_ts(tY + 64, tPm + 64 + kk * 8, smem_desc(sX + kk * 2048, 0, 1024), id_pm, kk > 0);
-            mma_commit(&s.m2b);
-            const uint32_t sC = smem_u32(s.bc[c & 1]), sHp = smem_u32(s.hp);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-                mma_ss(tG, smem_desc(sC + off, 16, 1024), smem_desc(sHp + kk * 2048, kBox, 1024), id_ys, kk > 0);
-            }
-        }
-        // ---- w o X over X_h once Y_h has read X_h; 4 threads per token row
-        auto xw = [&](int hm) {
-            const int j = tid >> 2, ch = 2 * (tid & 3);
-            const float w = s.dvs[hm][j] * ex2(s.cvs[hm][kQ - 1] - s.cvs[hm][j]);
-            uint8_t *base = xs + hm * kBox;
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                uint4 v = lds128(base + swz(j, ch + u));
-                v.x = scale_bf16x2(v.x, w); v.y = scale_bf16x2(v.y, w);
-                v.z = scale_bf16x2(v.z, w); v.w = scale_bf16x2(v.w, w);
-                sts128(base + swz(j, ch + u), v);
+            for (int kq = 0; kq < 4; ++kq) {
+                const int64_t t = t0 + 4 * lane + kq;
+                dtn[kq] = t < s1 ? *reinterpret_cast<const float2 *>(p.dt + ((int64_t)bi * p.L + t) * p.H + ha)
+                                 : make_float2(0.0f, 0.0f);
             }
         };
-        // (X_c's landing is waited for here too, so that its bytes are visible to this thread)
-        ok = mbar_wait(&s.full_x[c & 1], (c >> 1) & 1, abort, lim) && mbar_wait(&s.m2a, c & 1, abort, lim);
-        if (ok) xw(0);
-        ok = ok && mbar_wait(&s.m2b, c & 1, abort, lim);
-        if (ok) xw(1);
-        fence_proxy_async_smem();
-        if (__syncthreads_or(!ok || *abort)) { raise_timeout(p, abort); break; }
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t sB = smem_u32(s.bc[c & 1]) + 2 * kBox, sXw = smem_u32(xs);
+        auto scan = [&]() {
+            float ca[4], cb[4];
+            float sa = 0.0f, sb = 0.0f;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                mma_ss(tS, smem_desc(sB + kk * 2048, kBox, 1024), smem_desc(sXw + kk * 2048, kBox, 1024), id_s, kk > 0);
-            mma_commit(&s.mma_done);
+            for (int kq = 0; kq < 4; ++kq) {
+                sa += dtn[kq].x * A2a; ca[kq] = sa;
+                sb += dtn[kq].y * A2b; cb[kq] = sb;
+            }
+            float ia = sa, ib = sb;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float ta = __shfl_up_sync(0xffffffffu, ia, o);
+                const float tb = __shfl_up_sync(0xffffffffu, ib, o);
+                if (lane >= o) { ia += ta; ib += tb; }
+            }
+            float xa = __shfl_up_sync(0xffffffffu, ia, 1), xb = __shfl_up_sync(0xffffffffu, ib, 1);
+            if (lane == 0) { xa = 0.0f; xb = 0.0f; }
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq) { ca[kq] += xa; cb[kq] += xb; }
+            // cumsum at the end of this lane's 32-token block (token 32 J + 31 = lane 8 J + 7)
+            const float ea = __shfl_sync(0xffffffffu, ca[3], lane | 7);
+            const float eb = __shfl_sync(0xffffffffu, cb[3], lane | 7);
+            reinterpret_cast<float4 *>(s.cvs[0])[lane] = make_float4(ca[0], ca[1], ca[2], ca[3]);
+            reinterpret_cast<float4 *>(s.cvs[1])[lane] = make_float4(cb[0], cb[1], cb[2], cb[3]);
+            reinterpret_cast<float4 *>(s.dvs[0])[lane] = make_float4(dtn[0].x, dtn[1].x, dtn[2].x, dtn[3].x);
+            reinterpret_cast<float4 *>(s.dvs[1])[lane] = make_float4(dtn[0].y, dtn[1].y, dtn[2].y, dtn[3].y);
+            if (lane < 24) {
+                reinterpret_cast<float4 *>(s.fs[0])[lane] =
+                    make_float4(dtn[0].x * ex2(ea - ca[0]), dtn[1].x * ex2(ea - ca[1]),
+                                dtn[2].x * ex2(ea - ca[2]), dtn[3].x * ex2(ea - ca[3]));
+                reinterpret_cast<float4 *>(s.fs[1])[lane] =
+                    make_float4(dtn[0].y * ex2(eb - cb[0]), dtn[1].y * ex2(eb - cb[1]),
+                                dtn[2].y * ex2(eb - cb[2]), dtn[3].y * ex2(eb - cb[3]));
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.scan_ready);
+        };
+
+        const bool scan_warp = warp == 4;
+        if (scan_warp && live) {
+            load_dt(0);
+            scan();
+            if (nc > 1) load_dt(1);
         }
-        ok = ewait(&s.mma_done, c & 1, abort, lim);
-        tc_fence_after();
-        // every operand of chunk c is consumed: refill its B/C slot, start G of chunk c+1
-        if (tid == 0 && ok && live) {
-            if (c + 2 < nc) issue_bc(c + 2);
-            if (c + 1 < nc && !issue_g(c + 1, tPm)) raise_timeout(p, abort);
-        }
-        if (ok) {
-            // ---- state: h = exp(cs_last) h + S (columns p0.. of head hd, state row n = r)
+        const float Dh = p.D ? p.D[hh] : 0.0f;
+        for (int c = 0; c < nc; ++c) {
+            const int64_t t0 = s0 + (int64_t)c * kQ;
+            const uint32_t tG = tm + ((c & 1) ? 128u : 0u);   // G, later Ys
+            const uint32_t tPm = tm + ((c & 1) ? 0u : 128u);  // Pm_a | Pm_b
+            uint8_t *xs = s.x[c & 1];
+
+            if (!ewait(&s.scan_ready, c & 1, abort, lim)) { fail(); break; }
+            // ---- state: H = h after chunk c-1 -> bf16 copy for C hp^T, checkpoint; H *= exp(cs_last)
             {
-                uint32_t sa[32];
-                tmem_ld32(tS + lane_base + 32 * cs, sa);
+                uint32_t hv[32];
+                tmem_ld32(tH + lane_base + 32 * cs, hv);
                 tmem_wait_ld();
+                const int64_t kc = c > 0 ? ckpt_slot(t0) : -1;
+                if (kc >= 0) store_state(ckpt_ptr(kc), hv);
+                uint8_t *dst = s.hp + hd * kBox;
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    uint4 v;
+                    v.x = pack_bf16x2(__uint_as_float(hv[8 * c4 + 0]), __uint_as_float(hv[8 * c4 + 1]));
+                    v.y = pack_bf16x2(__uint_as_float(hv[8 * c4 + 2]), __uint_as_float(hv[8 * c4 + 3]));
+                    v.z = pack_bf16x2(__uint_as_float(hv[8 * c4 + 4]), __uint_as_float(hv[8 * c4 + 5]));
+                    v.w = pack_bf16x2(__uint_as_float(hv[8 * c4 + 6]), __uint_as_float(hv[8 * c4 + 7]));
+                    sts128(dst + swz(r, (p0 >> 3) + c4), v);
+                }
                 const float dec = ex2(s.cvs[hd][kQ - 1]);
 #pragma unroll
-                for (int pp = 0; pp < 32; ++pp) hr[pp] = fmaf(dec, hr[pp], __uint_as_float(sa[pp]));
+                for (int pp = 0; pp < 32; ++pp) hv[pp] = __float_as_uint(dec * __uint_as_float(hv[pp]));
+                tmem_st32(tH + lane_base + 32 * cs, hv);
             }
-            if (c + 1 < nc) write_hp();
-            // ---- y = Y + exp(cs_r) Ys -> bf16, staged in the X slot (same swizzle as the y map)
+            // ---- masked decay: column blocks J = 2 (cs & 1) + jb of head hd, rows of quarter q
+            if (!ewait(&s.g_done, c & 1, abort, lim)) { fail(); break; }
+            tc_fence_after();
             {
-                const float e = ex2(s.cvs[hd][r]);
+                const float csr = s.cvs[hd][r];
+#pragma unroll
+                for (int jb = 0; jb < 2; ++jb) {
+                    const int J = 2 * (cs & 1) + jb;
+                    uint32_t pk[16];
+                    if (J < q) {
+                        const float E = ex2(csr - s.cvs[hd][32 * J + 31]);
+                        const float2 E2 = make_float2(E, E);
+                        uint32_t gv[32];
+                        tmem_ld32(tG + lane_base + 32 * J, gv);
+                        tmem_wait_ld();
+                        const float4 *f4 = reinterpret_cast<const float4 *>(&s.fs[hd][32 * J]);
+#pragma unroll
+                        for (int i4 = 0; i4 < 8; ++i4) {
+                            const float4 f = f4[i4];
+                            const float2 a = mul2(make_float2(__uint_as_float(gv[4 * i4]), __uint_as_float(gv[4 * i4 + 1])),
+                                                  mul2(make_float2(f.x, f.y), E2));
+                            const float2 b = mul2(make_float2(__uint_as_float(gv[4 * i4 + 2]), __uint_as_float(gv[4 * i4 + 3])),
+                                                  mul2(make_float2(f.z, f.w), E2));
+                            pk[2 * i4] = pack_bf16x2(a.x, a.y);
+                            pk[2 * i4 + 1] = pack_bf16x2(b.x, b.y);
+                        }
+                    } else if (J == q) {
+                        uint32_t gv[32];
+                        tmem_ld32(tG + lane_base + 32 * J, gv);
+                        tmem_wait_ld();
+                        const float4 *c4 = reinterpret_cast<const float4 *>(&s.cvs[hd][32 * J]);
+                        const float4 *d4 = reinterpret_cast<const float4 *>(&s.dvs[hd][32 * J]);
+#pragma unroll
+                        for (int i4 = 0; i4 < 8; ++i4) {
+                            const float4 cc = c4[i4], dd = d4[i4];
+                            const float ca[4] = {cc.x, cc.y, cc.z, cc.w}, da[4] = {dd.x, dd.y, dd.z, dd.w};
+                            float v[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int i = 4 * i4 + e;
+                                const float t = __uint_as_float(gv[i]) * ex2(csr - ca[e]) * da[e];
+                                v[e] = i > lane ? 0.0f : (i == lane ? t + Dh : t);
+                            }
+                            pk[2 * i4] = pack_bf16x2(v[0], v[1]);
+                            pk[2 * i4 + 1] = pack_bf16x2(v[2], v[3]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) pk[i] = 0u;
+                    }
+                    tmem_st16(tPm + lane_base + 16 * (2 * cs + jb), pk);
+                }
+            }
+            tmem_wait_st();
+            fence_proxy_async_smem();   // hp, read by C hp^T
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.pm_ready);
+            // the epilogue's factor (the scan buffer is rewritten once w o X is done)
+            const float e_r = ex2(s.cvs[hd][r]);
+
+            // ---- w o X over X_hd once Y_hd has read it: 4 chunks of 16 B per thread
+            if (!(ewait(&s.full_x[c & 1], (c >> 1) & 1, abort, lim) &&
+                  ewait(hd ? &s.m2b : &s.m2a, c & 1, abort, lim))) { fail(); break; }
+            {
+                const int ti = 32 * (warp & 7) + lane;
+                const int j = ti >> 1, ch = 4 * (ti & 1);
+                const float w = s.dvs[hd][j] * ex2(s.cvs[hd][kQ - 1] - s.cvs[hd][j]);
+                uint8_t *base = xs + hd * kBox;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    uint4 v = lds128(base + swz(j, ch + u));
+                    v.x = scale_bf16x2(v.x, w); v.y = scale_bf16x2(v.y, w);
+                    v.z = scale_bf16x2(v.z, w); v.w = scale_bf16x2(v.w, w);
+                    sts128(base + swz(j, ch + u), v);
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.xw_ready);
+
+            // ---- y once every product of the chunk is done
+            if (!ewait(&s.mma_done, c & 1, abort, lim)) { fail(); break; }
+            tc_fence_after();
+            // every warp has read this chunk's scan values (M4 waited for them): publish the next chunk's
+            if (scan_warp && c + 1 < nc) {
+                scan();
+                if (c + 2 < nc) load_dt(c + 2);
+            }
+            {
                 uint8_t *dst = xs + hd * kBox;
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
@@ -645,48 +615,161 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
 #pragma unroll
                         for (int e2 = 0; e2 < 4; ++e2) {
                             const int i = 8 * c2 + 2 * e2;
-                            vw[e2] = pack_bf16x2(fmaf(e, __uint_as_float(ys[i]), __uint_as_float(yv[i])),
-                                                 fmaf(e, __uint_as_float(ys[i + 1]), __uint_as_float(yv[i + 1])));
+                            vw[e2] = pack_bf16x2(fmaf(e_r, __uint_as_float(ys[i]), __uint_as_float(yv[i])),
+                                                 fmaf(e_r, __uint_as_float(ys[i + 1]), __uint_as_float(yv[i + 1])));
                         }
                         sts128(dst + swz(r, (p0 >> 3) + 2 * hf + c2), v);
                     }
                 }
             }
-            const int64_t t_end = t0 + kQ;
-            if (p.h_ckpt && p.s > 0 && t_end <= s1 && t_end % p.s == 0) {
-                const int64_t kc = t_end / p.s - 1;
-                if (kc < n_ckpt) {
-                    float *dst = p.h_ckpt + (((int64_t)bi * n_ckpt + kc) * p.H + hh) * PN + (int64_t)p0 * kN + r;
+            fence_proxy_async_smem();   // y, read by the TMA store
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.y_ready);
+        }
+        if (!__any_sync(0xffffffffu, *abort != 0)) {
+            // the state after the stripe's last chunk
+            uint32_t hv[32];
+            tmem_ld32(tH + lane_base + 32 * cs, hv);
+            tmem_wait_ld();
+            const int64_t kc = ckpt_slot(s0 + (int64_t)nc * kQ);
+            if (kc >= 0) store_state(ckpt_ptr(kc), hv);
+            if (p.h_final && s1 == p.L) store_state(p.h_final + ((int64_t)bi * p.H + hh) * PN + (int64_t)p0 * kN + r, hv);
+        }
+    } else {
+        // ================================================= issuing warp
+        int bc_issued = 0, bc_waited = 0, x_issued = 0, x_waited = 0;   // lane 0's bookkeeping
+        auto issue_bc = [&](int c) {
+            const int t0 = (int)(s0 + (int64_t)c * kQ);
+            uint8_t *d = s.bc[c & 1];
+            uint64_t *bar = &s.full_bc[c & 1];
+            mbar_arrive_expect_tx(bar, 4 * kBox);
+            tma_load_3d(d, &maps.C, bar, g * kN, t0, bi);
+            tma_load_3d(d + kBox, &maps.C, bar, g * kN + 64, t0, bi);
+            tma_load_3d(d + 2 * kBox, &maps.B, bar, g * kN, t0, bi);
+            tma_load_3d(d + 3 * kBox, &maps.B, bar, g * kN + 64, t0, bi);
+            ++bc_issued;
+        };
+        auto issue_x = [&](int c) {
+            const int t0 = (int)(s0 + (int64_t)c * kQ);
+            uint8_t *d = s.x[c & 1];
+            uint64_t *bar = &s.full_x[c & 1];
+            mbar_arrive_expect_tx(bar, 2 * kBox);
+            tma_load_3d(d, &maps.x, bar, ha * kP, t0, bi);
+            tma_load_3d(d + kBox, &maps.x, bar, (ha + 1) * kP, t0, bi);
+            ++x_issued;
+        };
+        // G = C B^T of chunk c into the TMEM columns at tG (its B/C slot has landed)
+        auto issue_g = [&](int c, uint32_t tG) {
+            const uint32_t sC = smem_u32(s.bc[c & 1]), sB = sC + 2 * kBox;
+            const uint32_t id_g = idesc_bf16(128, 128, 0, 0);
 #pragma unroll
-                    for (int pp = 0; pp < 32; ++pp) dst[pp * kN] = hr[pp];
-                }
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+                mma_ss(tG, smem_desc(sC + off, 16, 1024), smem_desc(sB + off, 16, 1024), id_g, kk > 0);
+            }
+            mma_commit(&s.g_done);
+        };
+        const uint32_t id_pm = idesc_bf16(128, 64, 0, 1);     // A = Pm (TMEM), B = X (MN-major)
+        const uint32_t id_ys = idesc_bf16(128, 128, 0, 1);    // A = C (K-major), B = hp (MN-major)
+        const uint32_t id_s = idesc_bf16(128, 128, 1, 1);     // A = B^T (MN-major), B = w o X (MN-major)
+        // The whole warp waits (warp-uniform outcome); lane 0 issues.
+        bool ok = live;
+        if (ok) {
+            if (lane == 0) {
+                issue_bc(0);
+                if (nc > 1) issue_bc(1);
+                issue_x(0);
+                if (nc > 1) issue_x(1);
+            }
+            ok = ewait(&s.full_bc[0], 0, abort, lim);
+            if (ok) {
+                tc_fence_after();
+                if (lane == 0) { ++bc_waited; issue_g(0, tm); }
+                __syncwarp();
             }
         }
-        fence_proxy_async_smem();   // hp for the next C hp^T, y for the store
-        tc_fence_before();
-        if (__syncthreads_or(!ok || *abort)) { raise_timeout(p, abort); break; }
-        if (tid == 0 && live) {
-            tma_store_3d(&maps.y, xs, ha * kP, (int)t0, bi);
-            tma_store_3d(&maps.y, xs + kBox, (ha + 1) * kP, (int)t0, bi);
-            tma_store_commit();
-        }
-    }
-    if (!*abort && p.h_final && s1 == p.L) {
-        float *dst = p.h_final + ((int64_t)bi * p.H + hh) * PN + (int64_t)p0 * kN + r;
+        for (int c = 0; ok && c < nc; ++c) {
+            const int64_t t0 = s0 + (int64_t)c * kQ;
+            const uint32_t tG = tm + ((c & 1) ? 128u : 0u);
+            const uint32_t tPm = tm + ((c & 1) ? 0u : 128u);
+            uint8_t *xs = s.x[c & 1];
+            // Pm and X of chunk c: Y_a, Y_b, then C hp^T over the spent G
+            ok = ewait(&s.pm_ready, c & 1, abort, lim) && ewait(&s.full_x[c & 1], (c >> 1) & 1, abort, lim);
+            if (!ok) break;
+            tc_fence_after();
+            if (lane == 0) {
+                ++x_waited;
+                const uint32_t sX = smem_u32(xs);
 #pragma unroll
-        for (int pp = 0; pp < 32; ++pp) dst[pp * kN] = hr[pp];
-    }
-    if (tid == 0) {
-        if (*abort) {
-            // drain: MMAs, then every load still in flight
-            mma_commit(&s.fin);
-            mbar_wait(&s.fin, 0, nullptr, 100000000ull);
-            for (int i = bc_waited; i < bc_issued; ++i)
-                mbar_wait(&s.full_bc[i & 1], (i >> 1) & 1, nullptr, 100000000ull);
-            for (int i = x_waited; i < x_issued; ++i)
-                mbar_wait(&s.full_x[i & 1], (i >> 1) & 1, nullptr, 100000000ull);
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tY, tPm + kk * 8, smem_desc(sX + kk * 2048, 0, 1024), id_pm, kk > 0);
+                mma_commit(&s.m2a);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tY + 64, tPm + 64 + kk * 8, smem_desc(sX + kBox + kk * 2048, 0, 1024), id_pm, kk > 0);
+                mma_commit(&s.m2b);
+                const uint32_t sC = smem_u32(s.bc[c & 1]), sHp = smem_u32(s.hp);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+                    mma_ss(tG, smem_desc(sC + off, 16, 1024), smem_desc(sHp + kk * 2048, kBox, 1024), id_ys, kk > 0);
+                }
+                // the other X slot held y of chunk c-1, whose store has been read by now: chunk c+1 goes there
+                if (c >= 1 && c + 1 < nc) {
+                    tma_store_wait_read<0>();
+                    issue_x(c + 1);
+                }
+            }
+            __syncwarp();
+            // w o X of both heads: S = B^T [Xw_a | Xw_b] accumulates into H
+            ok = ewait(&s.xw_ready, c & 1, abort, lim);
+            if (!ok) break;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t sB = smem_u32(s.bc[c & 1]) + 2 * kBox, sXw = smem_u32(xs);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(tH, smem_desc(sB + kk * 2048, kBox, 1024), smem_desc(sXw + kk * 2048, kBox, 1024), id_s, true);
+                mma_commit(&s.mma_done);
+            }
+            __syncwarp();
+            // products done: refill the B/C slot, G of chunk c+1 into the columns Pm used
+            ok = ewait(&s.mma_done, c & 1, abort, lim);
+            if (!ok) break;
+            tc_fence_after();
+            if (lane == 0 && c + 2 < nc) issue_bc(c + 2);
+            if (c + 1 < nc) {
+                ok = ewait(&s.full_bc[(c + 1) & 1], ((c + 1) >> 1) & 1, abort, lim);
+                if (!ok) break;
+                tc_fence_after();
+                if (lane == 0) { ++bc_waited; issue_g(c + 1, tPm); }
+                __syncwarp();
+            }
+            // y staged: store it (the slot is refilled once the next chunk's products are issued)
+            ok = ewait(&s.y_ready, c & 1, abort, lim);
+            if (!ok) break;
+            if (lane == 0) {
+                tma_store_3d(&maps.y, xs, ha * kP, (int)t0, bi);
+                tma_store_3d(&maps.y, xs + kBox, (ha + 1) * kP, (int)t0, bi);
+                tma_store_commit();
+            }
+            __syncwarp();
         }
-        tma_store_wait<0>();
+        if (lane == 0) {
+            if (live && !ok) raise_timeout(p, abort);
+            if (*abort) {
+                // drain: MMAs, then every load still in flight
+                mma_commit(&s.fin);
+                mbar_wait(&s.fin, 0, nullptr, 100000000ull);
+                for (int i = bc_waited; i < bc_issued; ++i)
+                    mbar_wait(&s.full_bc[i & 1], (i >> 1) & 1, nullptr, 100000000ull);
+                for (int i = x_waited; i < x_issued; ++i)
+                    mbar_wait(&s.full_x[i & 1], (i >> 1) & 1, nullptr, 100000000ull);
+            }
+            tma_store_wait<0>();
+        }
+        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();
