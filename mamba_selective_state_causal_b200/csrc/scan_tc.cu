@@ -88,6 +88,18 @@ __device__ __forceinline__ uint32_t scale_bf16x2(uint32_t v, float w)
     return pack_bf16x2(bf16_lo(v) * w, bf16_hi(v) * w);
 }
 
+// fp32 pair -> bf16x2 by integer rounding (half an ulp added, ties away from zero), on the
+// integer pipe so that it runs beside the conversion unit; inputs are finite
+__device__ __forceinline__ uint32_t pack_bf16x2_int(float lo, float hi)
+{
+    return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
+}
+
+__device__ __forceinline__ uint32_t scale_bf16x2_int(uint32_t v, float w)
+{
+    return pack_bf16x2_int(bf16_lo(v) * w, bf16_hi(v) * w);
+}
+
 __device__ __forceinline__ void raise_timeout(const ScanParams &p, volatile int *abort)
 {
     *abort = 1;
@@ -289,10 +301,10 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
 //
 // Issuing warp, per chunk c (the whole warp waits, one lane issues):
 //   Pm ready -> Y_a = Pm_a X_a, Y_b = Pm_b X_b, Ys = C [hp_a | hp_b]^T (into G's
-//   columns, G being spent), then the other X slot (y of chunk c-1, stored by
-//   now) is refilled with chunk c+1; w o X ready -> S = B^T [Xw_a | Xw_b],
-//   accumulated straight into the fp32 state H in TMEM;
-//   products done -> refill the B/C slot, G of chunk c+1 into the columns Pm used;
+//   columns, G being spent); w o X ready -> S = B^T [Xw_a | Xw_b], accumulated
+//   straight into the fp32 state H in TMEM, then the other X slot (y of chunk
+//   c-1, stored by now) is refilled with chunk c+1; products done -> G of chunk
+//   c+1 into the columns Pm used, then the B/C slot is refilled;
 //   y staged -> TMA store of y.
 // Warp 4 (no masked-decay work of its own) also publishes the chunk cumsum of
 // dt*A of both heads for chunk c+1 once the products of chunk c are done.
@@ -482,35 +494,58 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
             if (nc > 1) load_dt(1);
         }
         const float Dh = p.D ? p.D[hh] : 0.0f;
-        for (int c = 0; c < nc; ++c) {
-            const int64_t t0 = s0 + (int64_t)c * kQ;
+
+        // H = h after chunk c-1: its bf16 copy feeds C hp^T of chunk c (checkpointed when a
+        // checkpoint ends there), then H *= exp(cs_last(c)), to which chunk c's S is added.
+        auto state_step = [&](int c, uint32_t (&hv)[32]) {
+            const int64_t kc = c > 0 ? ckpt_slot(s0 + (int64_t)c * kQ) : -1;
+            if (kc >= 0) store_state(ckpt_ptr(kc), hv);
+            uint8_t *dst = s.hp + hd * kBox;
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                uint4 v;
+                v.x = pack_bf16x2_int(__uint_as_float(hv[8 * c4 + 0]), __uint_as_float(hv[8 * c4 + 1]));
+                v.y = pack_bf16x2_int(__uint_as_float(hv[8 * c4 + 2]), __uint_as_float(hv[8 * c4 + 3]));
+                v.z = pack_bf16x2_int(__uint_as_float(hv[8 * c4 + 4]), __uint_as_float(hv[8 * c4 + 5]));
+                v.w = pack_bf16x2_int(__uint_as_float(hv[8 * c4 + 6]), __uint_as_float(hv[8 * c4 + 7]));
+                sts128(dst + swz(r, (p0 >> 3) + c4), v);
+            }
+            const float dec = ex2(s.cvs[hd][kQ - 1]);
+#pragma unroll
+            for (int pp = 0; pp < 32; ++pp) hv[pp] = __float_as_uint(dec * __uint_as_float(hv[pp]));
+            tmem_st32(tH + lane_base + 32 * cs, hv);
+        };
+        // y = Y + exp(cs_r) Ys for 16 columns -> bf16 -> the X slot (same swizzle as the y map)
+        auto y_half = [&](uint8_t *xs, const uint32_t (&yv)[16], const uint32_t (&ys)[16], float e_r, int hf) {
+            uint8_t *dst = xs + hd * kBox;
+#pragma unroll
+            for (int c2 = 0; c2 < 2; ++c2) {
+                uint4 v;
+                uint32_t *vw = reinterpret_cast<uint32_t *>(&v);
+#pragma unroll
+                for (int e2 = 0; e2 < 4; ++e2) {
+                    const int i = 8 * c2 + 2 * e2;
+                    vw[e2] = pack_bf16x2(fmaf(e_r, __uint_as_float(ys[i]), __uint_as_float(yv[i])),
+                                         fmaf(e_r, __uint_as_float(ys[i + 1]), __uint_as_float(yv[i + 1])));
+                }
+                sts128(dst + swz(r, (p0 >> 3) + 2 * hf + c2), v);
+            }
+        };
+
+        bool ok = ewait(&s.scan_ready, 0, abort, lim);
+        if (ok) {
+            uint32_t hv[32];
+            tmem_ld32(tH + lane_base + 32 * cs, hv);
+            tmem_wait_ld();
+            state_step(0, hv);
+        } else {
+            fail();
+        }
+        for (int c = 0; ok && c < nc; ++c) {
             const uint32_t tG = tm + ((c & 1) ? 128u : 0u);   // G, later Ys
             const uint32_t tPm = tm + ((c & 1) ? 0u : 128u);  // Pm_a | Pm_b
             uint8_t *xs = s.x[c & 1];
 
-            if (!ewait(&s.scan_ready, c & 1, abort, lim)) { fail(); break; }
-            // ---- state: H = h after chunk c-1 -> bf16 copy for C hp^T, checkpoint; H *= exp(cs_last)
-            {
-                uint32_t hv[32];
-                tmem_ld32(tH + lane_base + 32 * cs, hv);
-                tmem_wait_ld();
-                const int64_t kc = c > 0 ? ckpt_slot(t0) : -1;
-                if (kc >= 0) store_state(ckpt_ptr(kc), hv);
-                uint8_t *dst = s.hp + hd * kBox;
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    uint4 v;
-                    v.x = pack_bf16x2(__uint_as_float(hv[8 * c4 + 0]), __uint_as_float(hv[8 * c4 + 1]));
-                    v.y = pack_bf16x2(__uint_as_float(hv[8 * c4 + 2]), __uint_as_float(hv[8 * c4 + 3]));
-                    v.z = pack_bf16x2(__uint_as_float(hv[8 * c4 + 4]), __uint_as_float(hv[8 * c4 + 5]));
-                    v.w = pack_bf16x2(__uint_as_float(hv[8 * c4 + 6]), __uint_as_float(hv[8 * c4 + 7]));
-                    sts128(dst + swz(r, (p0 >> 3) + c4), v);
-                }
-                const float dec = ex2(s.cvs[hd][kQ - 1]);
-#pragma unroll
-                for (int pp = 0; pp < 32; ++pp) hv[pp] = __float_as_uint(dec * __uint_as_float(hv[pp]));
-                tmem_st32(tH + lane_base + 32 * cs, hv);
-            }
             // ---- masked decay: column blocks J = 2 (cs & 1) + jb of head hd, rows of quarter q
             if (!ewait(&s.g_done, c & 1, abort, lim)) { fail(); break; }
             tc_fence_after();
@@ -521,6 +556,7 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
                     const int J = 2 * (cs & 1) + jb;
                     uint32_t pk[16];
                     if (J < q) {
+                        // whole block below the diagonal: exp(cs_r - cs_j) = exp(cs_r - m_J) exp(m_J - cs_j)
                         const float E = ex2(csr - s.cvs[hd][32 * J + 31]);
                         const float2 E2 = make_float2(E, E);
                         uint32_t gv[32];
@@ -538,24 +574,33 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
                             pk[2 * i4 + 1] = pack_bf16x2(b.x, b.y);
                         }
                     } else if (J == q) {
+                        // diagonal block as 16x16 quarters: the two on the diagonal exponentiate each
+                        // entry; the one below factors through m = cs at the block's column 15
                         uint32_t gv[32];
                         tmem_ld32(tG + lane_base + 32 * J, gv);
                         tmem_wait_ld();
-                        const float4 *c4 = reinterpret_cast<const float4 *>(&s.cvs[hd][32 * J]);
-                        const float4 *d4 = reinterpret_cast<const float4 *>(&s.dvs[hd][32 * J]);
+                        const float *cvb = &s.cvs[hd][32 * J], *dvb = &s.dvs[hd][32 * J];
+                        const float m16 = cvb[15];
+                        const bool lo = lane < 16;
+                        const float a_r = ex2(csr - m16);                                   // <= 1 for lane >= 16
+                        const float b_own = dvb[lane & 15] * ex2(m16 - cvb[lane & 15]);     // <= dt for lane < 16
+                        const int xo = lo ? 0 : 16;
 #pragma unroll
-                        for (int i4 = 0; i4 < 8; ++i4) {
-                            const float4 cc = c4[i4], dd = d4[i4];
-                            const float ca[4] = {cc.x, cc.y, cc.z, cc.w}, da[4] = {dd.x, dd.y, dd.z, dd.w};
-                            float v[4];
+                        for (int k2 = 0; k2 < 8; ++k2) {
+                            float vl[2], vh[2];
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int i = 4 * i4 + e;
-                                const float t = __uint_as_float(gv[i]) * ex2(csr - ca[e]) * da[e];
-                                v[e] = i > lane ? 0.0f : (i == lane ? t + Dh : t);
+                            for (int e = 0; e < 2; ++e) {
+                                const int k = 2 * k2 + e;
+                                const int x = xo + k;
+                                const float g_x = __uint_as_float(lo ? gv[k] : gv[16 + k]);
+                                float t = g_x * ex2(csr - cvb[x]) * dvb[x];
+                                t = x > lane ? 0.0f : (x == lane ? t + Dh : t);
+                                const float bk = __shfl_sync(0xffffffffu, b_own, k);
+                                vl[e] = lo ? t : __uint_as_float(gv[k]) * (a_r * bk);
+                                vh[e] = lo ? 0.0f : t;
                             }
-                            pk[2 * i4] = pack_bf16x2(v[0], v[1]);
-                            pk[2 * i4 + 1] = pack_bf16x2(v[2], v[3]);
+                            pk[k2] = pack_bf16x2(vl[0], vl[1]);
+                            pk[8 + k2] = pack_bf16x2(vh[0], vh[1]);
                         }
                     } else {
 #pragma unroll
@@ -583,46 +628,49 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     uint4 v = lds128(base + swz(j, ch + u));
-                    v.x = scale_bf16x2(v.x, w); v.y = scale_bf16x2(v.y, w);
-                    v.z = scale_bf16x2(v.z, w); v.w = scale_bf16x2(v.w, w);
+                    v.x = scale_bf16x2_int(v.x, w); v.y = scale_bf16x2_int(v.y, w);
+                    v.z = scale_bf16x2_int(v.z, w); v.w = scale_bf16x2_int(v.w, w);
                     sts128(base + swz(j, ch + u), v);
                 }
             }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.xw_ready);
-
-            // ---- y once every product of the chunk is done
-            if (!ewait(&s.mma_done, c & 1, abort, lim)) { fail(); break; }
-            tc_fence_after();
-            // every warp has read this chunk's scan values (M4 waited for them): publish the next chunk's
+            // every warp has read this chunk's scan values once all w o X are written: publish the next chunk's
             if (scan_warp && c + 1 < nc) {
+                if (!ewait(&s.xw_ready, c & 1, abort, lim)) { fail(); break; }
                 scan();
                 if (c + 2 < nc) load_dt(c + 2);
             }
-            {
-                uint8_t *dst = xs + hd * kBox;
+
+            // ---- once every product of the chunk is done: y of chunk c and the state step of chunk c+1
+            if (!ewait(&s.mma_done, c & 1, abort, lim)) { fail(); break; }
+            tc_fence_after();
+            if (c + 1 < nc) {
+                if (!ewait(&s.scan_ready, (c + 1) & 1, abort, lim)) { fail(); break; }
+                uint32_t hv[32], yv[16], ys[16];
+                tmem_ld32(tH + lane_base + 32 * cs, hv);
+                tmem_ld16(tY + lane_base + 32 * cs, yv);
+                tmem_ld16(tG + lane_base + 32 * cs, ys);
+                tmem_wait_ld();
+                y_half(xs, yv, ys, e_r, 0);
+                tmem_ld16(tY + lane_base + 32 * cs + 16, yv);
+                tmem_ld16(tG + lane_base + 32 * cs + 16, ys);
+                state_step(c + 1, hv);
+                tmem_wait_ld();
+                y_half(xs, yv, ys, e_r, 1);
+            } else {
+                uint32_t yv[16], ys[16];
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
-                    uint32_t yv[16], ys[16];
                     tmem_ld16(tY + lane_base + 32 * cs + 16 * hf, yv);
                     tmem_ld16(tG + lane_base + 32 * cs + 16 * hf, ys);
                     tmem_wait_ld();
-#pragma unroll
-                    for (int c2 = 0; c2 < 2; ++c2) {
-                        uint4 v;
-                        uint32_t *vw = reinterpret_cast<uint32_t *>(&v);
-#pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2) {
-                            const int i = 8 * c2 + 2 * e2;
-                            vw[e2] = pack_bf16x2(fmaf(e_r, __uint_as_float(ys[i]), __uint_as_float(yv[i])),
-                                                 fmaf(e_r, __uint_as_float(ys[i + 1]), __uint_as_float(yv[i + 1])));
-                        }
-                        sts128(dst + swz(r, (p0 >> 3) + 2 * hf + c2), v);
-                    }
+                    y_half(xs, yv, ys, e_r, hf);
                 }
             }
-            fence_proxy_async_smem();   // y, read by the TMA store
+            tmem_wait_st();
+            fence_proxy_async_smem();   // y for the store, hp for the next C hp^T
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.y_ready);
@@ -715,11 +763,6 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
                     const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
                     mma_ss(tG, smem_desc(sC + off, 16, 1024), smem_desc(sHp + kk * 2048, kBox, 1024), id_ys, kk > 0);
                 }
-                // the other X slot held y of chunk c-1, whose store has been read by now: chunk c+1 goes there
-                if (c >= 1 && c + 1 < nc) {
-                    tma_store_wait_read<0>();
-                    issue_x(c + 1);
-                }
             }
             __syncwarp();
             // w o X of both heads: S = B^T [Xw_a | Xw_b] accumulates into H
@@ -732,20 +775,25 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ss(tH, smem_desc(sB + kk * 2048, kBox, 1024), smem_desc(sXw + kk * 2048, kBox, 1024), id_s, true);
                 mma_commit(&s.mma_done);
+                // the other X slot held y of chunk c-1, whose store has been read by now: chunk c+1 goes there
+                if (c >= 1 && c + 1 < nc) {
+                    tma_store_wait_read<0>();
+                    issue_x(c + 1);
+                }
             }
             __syncwarp();
-            // products done: refill the B/C slot, G of chunk c+1 into the columns Pm used
+            // products done: G of chunk c+1 into the columns Pm used, then refill this B/C slot
             ok = ewait(&s.mma_done, c & 1, abort, lim);
             if (!ok) break;
             tc_fence_after();
-            if (lane == 0 && c + 2 < nc) issue_bc(c + 2);
             if (c + 1 < nc) {
                 ok = ewait(&s.full_bc[(c + 1) & 1], ((c + 1) >> 1) & 1, abort, lim);
                 if (!ok) break;
                 tc_fence_after();
                 if (lane == 0) { ++bc_waited; issue_g(c + 1, tPm); }
-                __syncwarp();
             }
+            if (lane == 0 && c + 2 < nc) issue_bc(c + 2);
+            __syncwarp();
             // y staged: store it (the slot is refilled once the next chunk's products are issued)
             ok = ewait(&s.y_ready, c & 1, abort, lim);
             if (!ok) break;
