@@ -40,13 +40,11 @@ using namespace tc;
 
 constexpr int kQ = 128, kP = 64, kN = 128;
 constexpr uint32_t kBox = 128 * 64 * 2;   // one 128-row x 64-col bf16 TMA box (16 KB)
-constexpr uint32_t kDtBox = 128 * 4 * 4;  // dt box: [128 tokens][4 heads] fp32 (2 KB)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr int kThreads = 192;
 
 struct Maps {
-    CUtensorMap x, B, C, dt, y;
+    CUtensorMap x, B, C, y;
 };
 
 __device__ __forceinline__ float ex2(float x)
@@ -63,17 +61,6 @@ __device__ __forceinline__ bool ewait(uint64_t *bar, uint32_t parity, volatile i
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, limit_ns));
 }
 
-// Barrier among the 128 epilogue threads, built on an mbarrier so that the
-// wait is bounded like every other wait (a bar.sync could not be abandoned).
-// `ph` counts the completed phases of `bar` seen by this thread.
-__device__ __forceinline__ bool epi_sync(uint64_t *bar, uint32_t &ph, volatile int *abort, uint64_t limit_ns)
-{
-    mbar_arrive(bar);
-    const bool ok = ewait(bar, ph & 1, abort, limit_ns);
-    ++ph;
-    return ok;
-}
-
 // byte offset of 16-byte chunk c of row r in a 128B-swizzled tile of 128-byte rows
 __device__ __forceinline__ uint32_t swz(int r, int c)
 {
@@ -83,10 +70,6 @@ __device__ __forceinline__ uint32_t swz(int r, int c)
 __device__ __forceinline__ uint4 lds128(const uint8_t *p) { return *reinterpret_cast<const uint4 *>(p); }
 __device__ __forceinline__ void sts128(uint8_t *p, uint4 v) { *reinterpret_cast<uint4 *>(p) = v; }
 
-__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t v, float w)
-{
-    return pack_bf16x2(bf16_lo(v) * w, bf16_hi(v) * w);
-}
 
 // fp32 pair -> bf16x2 by integer rounding (half an ulp added, ties away from zero), on the
 // integer pipe so that it runs beside the conversion unit; inputs are finite
@@ -107,191 +90,231 @@ __device__ __forceinline__ void raise_timeout(const ScanParams &p, volatile int 
 }
 
 // =============================================================== pass A
-// Two heads per CTA: S^T[(h,p)][n] = sum_j (w_h o X_h)[j][p] B[j][n] for the
-// head pair, accumulated in TMEM over the whole stripe (M = 128 rows = 2 heads
-// x 64, N = 128 as two N=64 halves).  Chunks are walked backwards so that the
-// decay from each chunk to the stripe end (a suffix sum) is known when the
-// chunk is scaled.
+// One CTA per (stripe, head pair): S[n][(h,p)] = sum_j B[j][n] (w_h o X_h)[j][p]
+// over the whole stripe, both heads side by side on N = 128, accumulated in
+// TMEM.  Chunks are walked backwards so that the decay from each chunk to the
+// stripe end (a suffix sum) is known when the chunk is scaled:
+//   w_j = dt_j exp(sum of dt*A after token j, up to the stripe end).
+// Warps 0..15 scale X in place (half a token row of one head per thread);
+// warp 16 issues the TMA loads (B and X of both heads, 3-stage ring) and the
+// MMAs; warp 17 runs the dt scan that yields w, up to three chunks ahead.
+constexpr int kStagesA = 3;
+constexpr int kScaleWarpsA = 16;
+constexpr int kThreadsA = 32 * (kScaleWarpsA + 2);
+
 struct SmemA {
-    uint8_t stage[2][4 * kBox + kDtBox];  // B (two boxes), X of head h0, X of head h1, dt
-    uint8_t xw[2][2 * kBox];              // w o X for both heads (h0 box, h1 box)
-    float scratch[2][8];
-    uint64_t full[2], empty[2], xw_full[2], xw_empty[2], acc_full, fin, epi;
+    uint8_t stage[kStagesA][4 * kBox];   // B box 0, B box 1, X of head a, X of head b
+    float w[kStagesA][2][kQ];            // w_j of head a / b for the chunk in the stage
+    uint64_t full[kStagesA], w_ready[kStagesA], xw_ready[kStagesA], empty[kStagesA];
+    uint64_t acc_full, fin;
     uint32_t tmem;
     int abort;
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsA, 1)
 stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
 {
-    extern __shared__ uint8_t smraw[];
-    SmemA &s = *reinterpret_cast<SmemA *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t sma_raw[];
+    SmemA &s = *reinterpret_cast<SmemA *>((reinterpret_cast<uintptr_t>(sma_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t unit = blockIdx.x;
     const int hpairs = p.H / 2;
-    const int h0 = 2 * (int)(unit % hpairs);
+    const int ha = 2 * (int)(unit % hpairs);
     const int64_t k = (unit / hpairs) % p.ns;
     const int bi = (int)(unit / ((int64_t)hpairs * p.ns));
-    const int g = (int)((int64_t)h0 * p.G / p.H);  // both heads of the pair share a group (H/G even)
+    const int g = (int)((int64_t)ha * p.G / p.H);  // both heads of the pair share a group (H/G even)
     const int64_t s0 = k * p.T;
     const int64_t s1 = min(p.L, s0 + p.T);
     const int nc = (int)((s1 - s0 + kQ - 1) / kQ);
     const uint64_t lim = p.wait_limit_ns;
+    constexpr int PN = kP * kN;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kStagesA; ++i) {
             mbar_init(&s.full[i], 1);
-            mbar_init(&s.empty[i], 1 + 128);
-            mbar_init(&s.xw_full[i], 128);
-            mbar_init(&s.xw_empty[i], 1);
+            mbar_init(&s.w_ready[i], 1);
+            mbar_init(&s.xw_ready[i], kScaleWarpsA);
+            mbar_init(&s.empty[i], 1);
         }
         mbar_init(&s.acc_full, 1);
         mbar_init(&s.fin, 1);
-        mbar_init(&s.epi, 128);
         s.abort = 0;
         fence_mbar_init();
-    }
-    if (warp == 0 && lane == 0) {
         prefetch_tmap(&maps.x);
         prefetch_tmap(&maps.B);
-        prefetch_tmap(&maps.dt);
     }
-    if (warp == 1) { tmem_alloc(&s.tmem, 128); tmem_relinquish(); }
+    if (warp == 0) { tmem_alloc(&s.tmem, 128); tmem_relinquish(); }
     __syncthreads();
     tc_fence_after();
     const uint32_t tS = s.tmem;
     volatile int *abort = &s.abort;
+    const bool live = unit != p.test_drop_unit;
 
-    if (warp == 0) {
-        if (lane == 0) {
-            int issued = 0;
-            for (int it = 0; it < nc; ++it) {
-                const int st = it & 1, u = it >> 1;
-                if (it >= 2 && !mbar_wait(&s.empty[st], (u - 1) & 1, abort, lim)) { raise_timeout(p, abort); break; }
-                if (unit == p.test_drop_unit) break;  // test hook: this unit's loads never arrive
-                const int c = nc - 1 - it;  // chunks in reverse order
-                const int t0 = (int)(s0 + (int64_t)c * kQ);
-                uint8_t *sb = s.stage[st];
-                mbar_arrive_expect_tx(&s.full[st], 4 * kBox + kDtBox);
-                tma_load_3d(sb, &maps.B, &s.full[st], g * kN, t0, bi);
-                tma_load_3d(sb + kBox, &maps.B, &s.full[st], g * kN + 64, t0, bi);
-                tma_load_3d(sb + 2 * kBox, &maps.x, &s.full[st], h0 * kP, t0, bi);
-                tma_load_3d(sb + 3 * kBox, &maps.x, &s.full[st], (h0 + 1) * kP, t0, bi);
-                tma_load_3d(sb + 4 * kBox, &maps.dt, &s.full[st], h0 & ~3, t0, bi);
-                issued = it + 1;
-            }
-            if (*abort) {  // let copies in flight land before the CTA exits
-                for (int it = max(0, issued - 2); it < issued; ++it)
-                    mbar_wait(&s.full[it & 1], (it >> 1) & 1, nullptr, 100000000ull);
-            }
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            const uint32_t id = idesc_bf16(128, 64, 1, 1);
-            for (int it = 0; it < nc; ++it) {
-                const int st = it & 1, u = it >> 1, xb = it & 1;
-                if (!mbar_wait(&s.full[st], u & 1, abort, lim) || !mbar_wait(&s.xw_full[xb], (it >> 1) & 1, abort, lim)) {
-                    raise_timeout(p, abort);
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t sB = smem_u32(s.stage[st]);
-                const uint32_t sXw = smem_u32(s.xw[xb]);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t da = smem_desc(sXw + kk * 2048, kBox, 1024);  // rows (h,p): two atoms
-                    mma_ss(tS, da, smem_desc(sB + kk * 2048, 0, 1024), id, it > 0 || kk > 0);
-                    mma_ss(tS + 64, da, smem_desc(sB + kBox + kk * 2048, 0, 1024), id, it > 0 || kk > 0);
-                }
-                mma_commit(&s.empty[st]);
-                mma_commit(&s.xw_empty[xb]);
-            }
-            mma_commit(&s.acc_full);
-            mma_commit(&s.fin);
-            mbar_wait(&s.fin, 0, nullptr, 200000000ull);
-        }
-    } else {
-        const int q = warp & 3;
-        const int r = 32 * q + lane;  // token row j; TMEM lane (h,p) for the result
-        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        const float A2a = p.A[h0] * kLog2e, A2b = p.A[h0 + 1] * kLog2e;
-        float sufa = 0.0f, sufb = 0.0f;
-        bool okk = true;
-        uint32_t eph = 0;
+    if (warp < kScaleWarpsA) {
+        // ================================================= scaling warps
+        const int hd = warp >> 3, j = 32 * (warp & 3) + lane, c0 = 4 * ((warp >> 2) & 1);
+        bool ok = true;
         for (int it = 0; it < nc; ++it) {
-            const int st = it & 1, u = it >> 1, xb = it & 1;
-            if (!ewait(&s.full[st], u & 1, abort, lim)) { raise_timeout(p, abort); okk = false; break; }
-            const uint8_t *sb = s.stage[st];
-            const float *dtrow = reinterpret_cast<const float *>(sb + 4 * kBox) + r * 4 + (h0 & 3);
-            const float dta = dtrow[0], dtb = dtrow[1];
-            float va = dta * A2a, vb = dtb * A2b;
-            const int lq = r & 31;
+            const int st = it % kStagesA;
+            const uint32_t ph = (uint32_t)(it / kStagesA) & 1;
+            ok = ewait(&s.full[st], ph, abort, lim) && ewait(&s.w_ready[st], ph, abort, lim);
+            if (!ok) break;
+            const float w = s.w[st][hd][j];
+            uint8_t *xrow = s.stage[st] + (2 + hd) * kBox;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float ta = __shfl_up_sync(0xffffffffu, va, o);
-                const float tb = __shfl_up_sync(0xffffffffu, vb, o);
-                if (lq >= o) { va += ta; vb += tb; }
-            }
-            float *scr = s.scratch[it & 1];
-            if (lq == 31) { scr[q] = va; scr[4 + q] = vb; }
-            if (!epi_sync(&s.epi, eph, abort, lim)) { raise_timeout(p, abort); okk = false; break; }
-            float prea = 0.0f, preb = 0.0f;
-            if (q > 0) { prea += scr[0]; preb += scr[4]; }
-            if (q > 1) { prea += scr[1]; preb += scr[5]; }
-            if (q > 2) { prea += scr[2]; preb += scr[6]; }
-            const float tota = ((scr[0] + scr[1]) + scr[2]) + scr[3];
-            const float totb = ((scr[4] + scr[5]) + scr[6]) + scr[7];
-            const float wa = dta * ex2((tota - (va + prea)) + sufa);
-            const float wb = dtb * ex2((totb - (vb + preb)) + sufb);
-            if (it >= 2 && !ewait(&s.xw_empty[xb], ((it >> 1) - 1) & 1, abort, lim)) {
-                raise_timeout(p, abort);
-                okk = false;
-                break;
-            }
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const uint8_t *xrow = sb + (2 + hh) * kBox;
-                uint8_t *xwt = s.xw[xb] + hh * kBox;
-                const float w = hh ? wb : wa;
-#pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
-                    const uint32_t o = swz(r, cc);
-                    uint4 vv = lds128(xrow + o);
-                    vv.x = scale_bf16x2(vv.x, w); vv.y = scale_bf16x2(vv.y, w);
-                    vv.z = scale_bf16x2(vv.z, w); vv.w = scale_bf16x2(vv.w, w);
-                    sts128(xwt + o, vv);
-                }
+            for (int cc = 0; cc < 4; ++cc) {
+                const uint32_t o = swz(j, c0 + cc);
+                uint4 vv = lds128(xrow + o);
+                vv.x = scale_bf16x2_int(vv.x, w); vv.y = scale_bf16x2_int(vv.y, w);
+                vv.z = scale_bf16x2_int(vv.z, w); vv.w = scale_bf16x2_int(vv.w, w);
+                sts128(xrow + o, vv);
             }
             fence_proxy_async_smem();
-            mbar_arrive(&s.xw_full[xb]);
-            mbar_arrive(&s.empty[st]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.xw_ready[st]);
+        }
+        if (!ok) {
+            if (lane == 0) raise_timeout(p, abort);
+        } else if (warp < 8) {
+            if (ewait(&s.acc_full, 0, abort, lim)) {
+                // S[n][(h,p)]: lane quarter q holds state rows n = 32 q .. 32 q + 31; warp 4 hd' + q takes head hd'
+                tc_fence_after();
+                const int q = warp & 3, hq = warp >> 2, n = 32 * q + lane;
+                const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+                float *dst = p.ws_S + (((int64_t)bi * p.ns + k) * p.H + ha + hq) * PN + n;
+#pragma unroll
+                for (int c32 = 0; c32 < 2; ++c32) {
+                    uint32_t a[32];
+                    tmem_ld32(tS + lane_base + 64 * hq + 32 * c32, a);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int pp = 0; pp < 32; ++pp) dst[(int64_t)(32 * c32 + pp) * kN] = __uint_as_float(a[pp]);
+                }
+            } else if (lane == 0) {
+                raise_timeout(p, abort);
+            }
+        }
+    } else if (warp == kScaleWarpsA) {
+        // ================================================= issuing warp (the whole warp waits, lane 0 issues)
+        int issued = 0;   // lane 0: loads issued (consumed loads are those of the MMAs issued)
+        auto issue_load = [&](int it) {
+            const int st = it % kStagesA;
+            const int t0 = (int)(s0 + (int64_t)(nc - 1 - it) * kQ);
+            uint8_t *sb = s.stage[st];
+            mbar_arrive_expect_tx(&s.full[st], 4 * kBox);
+            tma_load_3d(sb, &maps.B, &s.full[st], g * kN, t0, bi);
+            tma_load_3d(sb + kBox, &maps.B, &s.full[st], g * kN + 64, t0, bi);
+            tma_load_3d(sb + 2 * kBox, &maps.x, &s.full[st], ha * kP, t0, bi);
+            tma_load_3d(sb + 3 * kBox, &maps.x, &s.full[st], (ha + 1) * kP, t0, bi);
+            ++issued;
+        };
+        const uint32_t id_s = idesc_bf16(128, 128, 1, 1);   // A = B^T (MN-major), B = w o X (MN-major)
+        bool ok = live;
+        int mmas = 0;
+        if (ok && lane == 0)
+            for (int it = 0; it < min(nc, kStagesA); ++it) issue_load(it);
+        for (int it = 0; ok && it < nc; ++it) {
+            const int st = it % kStagesA;
+            ok = ewait(&s.xw_ready[st], (uint32_t)(it / kStagesA) & 1, abort, lim);
+            if (!ok) break;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t sB = smem_u32(s.stage[st]), sXw = sB + 2 * kBox;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(tS, smem_desc(sB + kk * 2048, kBox, 1024), smem_desc(sXw + kk * 2048, kBox, 1024), id_s,
+                           it > 0 || kk > 0);
+                mma_commit(&s.empty[st]);
+            }
+            ++mmas;
+            __syncwarp();
+            // the previous step's product has read its stage by now: refill it with step it + 2
+            if (it >= 1 && it + 2 < nc) {
+                const int pst = (it - 1) % kStagesA;
+                ok = ewait(&s.empty[pst], (uint32_t)((it - 1) / kStagesA) & 1, abort, lim);
+                if (!ok) break;
+                if (lane == 0) issue_load(it + 2);
+                __syncwarp();
+            }
+        }
+        if (lane == 0) {
+            if (live && !ok) raise_timeout(p, abort);
+            mma_commit(&s.acc_full);
+            mma_commit(&s.fin);
+            mbar_wait(&s.fin, 0, nullptr, 100000000ull);
+            if (*abort) {
+                // drain: every load issued but not consumed by an MMA
+                for (int it = mmas; it < issued; ++it)
+                    mbar_wait(&s.full[it % kStagesA], (uint32_t)(it / kStagesA) & 1, nullptr, 100000000ull);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ================================================= scan warp: w of every step, in order
+        const float A2a = p.A[ha] * kLog2e, A2b = p.A[ha + 1] * kLog2e;
+        float sufa = 0.0f, sufb = 0.0f;     // sum of dt*A (log2 units) after the chunks scanned so far
+        float2 dtn[4];                      // dt of tokens 4 lane .. 4 lane + 3 of the next chunk
+        auto load_dt = [&](int it) {
+            const int64_t t0 = s0 + (int64_t)(nc - 1 - it) * kQ;
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq) {
+                const int64_t t = t0 + 4 * lane + kq;
+                dtn[kq] = t < s1 ? *reinterpret_cast<const float2 *>(p.dt + ((int64_t)bi * p.L + t) * p.H + ha)
+                                 : make_float2(0.0f, 0.0f);
+            }
+        };
+        bool ok = live;
+        if (ok) load_dt(0);
+        for (int it = 0; ok && it < nc; ++it) {
+            const int st = it % kStagesA;
+            // the scaling warps are done with w[st] once step it - 3 is scaled
+            if (it >= kStagesA) {
+                ok = ewait(&s.xw_ready[st], (uint32_t)(it / kStagesA - 1) & 1, abort, lim);
+                if (!ok) break;
+            }
+            float ca[4], cb[4];
+            float sa = 0.0f, sb = 0.0f;
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq) {
+                sa += dtn[kq].x * A2a; ca[kq] = sa;
+                sb += dtn[kq].y * A2b; cb[kq] = sb;
+            }
+            const float2 dcur[4] = {dtn[0], dtn[1], dtn[2], dtn[3]};
+            if (it + 1 < nc) load_dt(it + 1);
+            float ia = sa, ib = sb;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float ta = __shfl_up_sync(0xffffffffu, ia, o);
+                const float tb = __shfl_up_sync(0xffffffffu, ib, o);
+                if (lane >= o) { ia += ta; ib += tb; }
+            }
+            float xa = __shfl_up_sync(0xffffffffu, ia, 1), xb = __shfl_up_sync(0xffffffffu, ib, 1);
+            if (lane == 0) { xa = 0.0f; xb = 0.0f; }
+            const float tota = __shfl_sync(0xffffffffu, ia, 31), totb = __shfl_sync(0xffffffffu, ib, 31);
+            // decay from token j (exclusive) to the stripe end: tot - cs_j + suffix of the later chunks
+            reinterpret_cast<float4 *>(s.w[st][0])[lane] =
+                make_float4(dcur[0].x * ex2(tota - (ca[0] + xa) + sufa), dcur[1].x * ex2(tota - (ca[1] + xa) + sufa),
+                            dcur[2].x * ex2(tota - (ca[2] + xa) + sufa), dcur[3].x * ex2(tota - (ca[3] + xa) + sufa));
+            reinterpret_cast<float4 *>(s.w[st][1])[lane] =
+                make_float4(dcur[0].y * ex2(totb - (cb[0] + xb) + sufb), dcur[1].y * ex2(totb - (cb[1] + xb) + sufb),
+                            dcur[2].y * ex2(totb - (cb[2] + xb) + sufb), dcur[3].y * ex2(totb - (cb[3] + xb) + sufb));
             sufa += tota;
             sufb += totb;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.w_ready[st]);
         }
-        if (okk && ewait(&s.acc_full, 0, abort, lim)) {
-            tc_fence_after();
-            const int hh = r >> 6, pp = r & 63;  // lane r holds state row p of head h0 + hh
-            float *dst = p.ws_S + (((int64_t)bi * p.ns + k) * p.H + h0 + hh) * (kP * kN) + (int64_t)pp * kN;
-#pragma unroll
-            for (int c32 = 0; c32 < 4; ++c32) {
-                uint32_t a[32];
-                tmem_ld32(tS + lane_base + 32 * c32, a);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    reinterpret_cast<uint4 *>(dst + 32 * c32)[i] = make_uint4(a[4 * i], a[4 * i + 1], a[4 * i + 2], a[4 * i + 3]);
+        if (lane == 0) {
+            if (live && !ok) raise_timeout(p, abort);
+            if (ok && !*abort) {
+                p.ws_dA[((int64_t)bi * p.ns + k) * p.H + ha] = sufa * kLn2;
+                p.ws_dA[((int64_t)bi * p.ns + k) * p.H + ha + 1] = sufb * kLn2;
             }
-            if (r == 0) {
-                p.ws_dA[((int64_t)bi * p.ns + k) * p.H + h0] = sufa * kLn2;
-                p.ws_dA[((int64_t)bi * p.ns + k) * p.H + h0 + 1] = sufb * kLn2;
-            }
-        } else if (okk) {
-            raise_timeout(p, abort);
         }
+        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) tmem_dealloc(tS, 128);
+    if (warp == 0) tmem_dealloc(tS, 128);
 }
 
 // =============================================================== pass C
@@ -859,16 +882,6 @@ bool encode_bf16(EncodeTiledFn enc, CUtensorMap *m, const void *base, int64_t co
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool encode_dt(EncodeTiledFn enc, CUtensorMap *m, const float *dt, int H, int64_t L, int b)
-{
-    const cuuint64_t dims[3] = {(cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)b};
-    const cuuint64_t strides[2] = {(cuuint64_t)H * 4, (cuuint64_t)H * 4 * L};
-    const cuuint32_t box[3] = {4, 128, 1};
-    const cuuint32_t es[3] = {1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(dt), dims, strides, box, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 constexpr size_t kSmemA = sizeof(SmemA) + 1024;
 constexpr size_t kSmemC = sizeof(SmemC);   // no alignment pad: the base is checked in the kernel
@@ -880,8 +893,8 @@ static_assert(kSmemA <= 232448, "pass A shared memory");
 bool tc_scan_supported(const ScanParams &p, int dtype)
 {
     if (dtype != 1 || p.P != kP || p.N != kN || p.Q != kQ) return false;
-    if (p.H % 4 != 0 || (p.H / p.G) % 2 != 0) return false;  // head pairs share a B/C group
-    if ((reinterpret_cast<uintptr_t>(p.dt) & 15u) != 0) return false;
+    if (p.H % 2 != 0 || (p.H / p.G) % 2 != 0) return false;  // head pairs share a B/C group
+    if ((reinterpret_cast<uintptr_t>(p.dt) & 7u) != 0) return false;  // dt of a head pair read as float2
     if (p.L >= (1LL << 31) || (int64_t)p.b * p.ns * p.H >= (1LL << 31)) return false;
     return encode_fn() != nullptr;
 }
@@ -895,7 +908,6 @@ int launch_scan_tc(const ScanParams &p, cudaStream_t st)
     if (!encode_bf16(enc, &maps.x, p.x, (int64_t)p.H * p.P, p.L, p.b, p.xrs, p.xbs) ||
         !encode_bf16(enc, &maps.B, p.B, gn, p.L, p.b, p.Brs, p.Bbs) ||
         !encode_bf16(enc, &maps.C, p.C, gn, p.L, p.b, p.Crs, p.Cbs) ||
-        !encode_dt(enc, &maps.dt, p.dt, p.H, p.L, p.b) ||
         !encode_bf16(enc, &maps.y, p.y, (int64_t)p.H * p.P, p.L, p.b, p.yrs, p.ybs))
         return 6;
     static bool attr_set[64] = {false};
@@ -910,7 +922,7 @@ int launch_scan_tc(const ScanParams &p, cudaStream_t st)
     const int64_t units = (int64_t)p.b * p.ns * p.H;
     if (p.ns > 1) {
         prof_begin(st, kKStateTc);
-        stripe_state_tc_kernel<<<(unsigned)(units / 2), kThreads, kSmemA, st>>>(maps, p);
+        stripe_state_tc_kernel<<<(unsigned)(units / 2), kThreadsA, kSmemA, st>>>(maps, p);
         prof_end(st, kKStateTc);
         const int rc = launch_chain(p, st);
         if (rc) return rc;

@@ -204,12 +204,6 @@ int conv_impl(const void *u, int64_t ubs, int64_t urs, const float *w, const flo
     ssd::ConvParams p{};
     p.u = u; p.ubs = ubs; p.urs = urs; p.w = w; p.bias = bias; p.tail_in = tail_in;
     p.tail_out = tail_out; p.v = v; p.vbs = vbs; p.vrs = vrs; p.b = b; p.L = L; p.C_ch = C_ch;
-    p.status = L > 0 ? status_ptr() : nullptr;
-    {
-        const char *lim = getenv("SSD_WAIT_LIMIT_MS");
-        const long long ms = lim ? atoll(lim) : 2000;
-        p.wait_limit_ns = (uint64_t)(ms > 0 ? ms : 2000) * 1000000ull;
-    }
     rc = ssd::launch_conv(p, dtype, st);
     if (rc == 2) return fail(SSD_ERR_SHAPE, "conv grid too large");
     if (rc) return fail(SSD_ERR_LAUNCH, "conv launch failed: %s", cudaGetErrorString(cudaGetLastError()));

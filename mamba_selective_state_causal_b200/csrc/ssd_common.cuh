@@ -56,8 +56,6 @@ struct ConvParams {
     int b;
     int64_t L;
     int C_ch;
-    unsigned int *status;       // device status word (bounded waits); NULL: register kernel only
-    uint64_t wait_limit_ns;
 };
 
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
