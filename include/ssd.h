@@ -133,7 +133,8 @@ typedef struct ssd_scan_args {
  */
 SSD_API int ssd_scan_forward(const ssd_scan_args *args, ssd_stream_t stream);
 
-/* Bytes of workspace ssd_scan_forward / ssd_stream_forward need for this shape. */
+/* Bytes of workspace ssd_scan_forward / ssd_stream_forward need for this shape
+ * on the current device (the stripe plan depends on its SM count). */
 SSD_API size_t ssd_scan_workspace_size(int b, int64_t L, int H, int P, int N, int Q);
 
 /*

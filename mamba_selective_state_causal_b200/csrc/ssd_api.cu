@@ -3,6 +3,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
+#include <algorithm>
 #include <cstring>
 #include <string>
 #include <vector>
@@ -55,9 +56,6 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 bool pow2_dim(int v) { return v == 16 || v == 32 || v == 64 || v == 128; }
 
-// Stripe plan: the sequence is split into stripes of T tokens (a multiple of
-// Q) so that b * stripes * H gives about a thousand independent (stripe, head)
-// units of work, with T between Q and 32*Q.
 struct Plan {
     int64_t T = 0, ns = 0;
     size_t off_S = 0, off_hin = 0, off_dA = 0, bytes = 0;
@@ -65,14 +63,44 @@ struct Plan {
 
 size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
 
+// Stripe plan: the sequence is split into stripes of T tokens (a multiple of Q).
+// The tensor-core passes run one CTA per SM and one (stripe, head pair) unit
+// per CTA, so a pass takes about
+//     waves x (chunks per stripe + 2),   waves = ceil(units / SMs),
+// the 2 standing for a unit's fixed cost (pipeline fill and drain) in chunks.
+// The plan takes the stripe length that minimises it on the current device and,
+// among equal costs, the fewest stripes (less chain work, smaller workspace).
+int sm_count()
+{
+    static int cached[kMaxDevices] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
 Plan make_plan(int b, int64_t L, int H, int P, int N, int Q)
 {
     Plan pl;
     if (b <= 0 || L <= 0 || H <= 0 || Q <= 0) return pl;
-    int64_t m = ((int64_t)b * L * H) / (1024LL * Q);
-    if (m < 1) m = 1;
-    if (m > 32) m = 32;
-    pl.T = m * Q;
+    const int64_t nchunks = (L + Q - 1) / Q;
+    const int64_t hp = (H % 2 == 0) ? H / 2 : H;
+    const int64_t nsm = sm_count();
+    int64_t best_cost = -1, best_tc = nchunks;
+    const int64_t max_ns = std::min<int64_t>(nchunks, 16384);
+    for (int64_t ns = 1; ns <= max_ns; ++ns) {
+        const int64_t tc = (nchunks + ns - 1) / ns;      // chunks per stripe
+        const int64_t real_ns = (nchunks + tc - 1) / tc;
+        if (real_ns != ns) continue;                     // the same plan as a smaller ns
+        const int64_t waves = ((int64_t)b * real_ns * hp + nsm - 1) / nsm;
+        const int64_t cost = waves * (tc + 2);
+        if (best_cost < 0 || cost < best_cost) { best_cost = cost; best_tc = tc; }
+    }
+    pl.T = best_tc * Q;
     pl.ns = (L + pl.T - 1) / pl.T;
     if (pl.ns > 1) {
         const size_t state = sizeof(float) * (size_t)b * pl.ns * H * P * N;

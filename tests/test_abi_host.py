@@ -44,15 +44,33 @@ def test_library_exports_every_declared_symbol(ssd):
     assert lib.ssd_version() >= 100
 
 
-def _plan_bytes(b, L, H, P, N, Q):
-    m = max(1, min(32, (b * L * H) // (1024 * Q)))
-    T = m * Q
-    ns = -(-L // T)
+def _plan_bytes(b, L, H, P, N, Q, nsm=148):
+    """Workspace of the stripe plan: the stripe length (whole chunks) minimising
+    waves x (chunks per stripe + 2), waves = ceil(b * stripes * head pairs / SMs),
+    fewest stripes among equals.  Without a GPU the library assumes 148 SMs."""
+    if b <= 0 or L <= 0:
+        return 0
+    nch = -(-L // Q)
+    hp = H // 2 if H % 2 == 0 else H
+    best = None
+    for ns in range(1, min(nch, 16384) + 1):
+        tc = -(-nch // ns)
+        if -(-nch // tc) != ns:
+            continue
+        cost = -(-(b * ns * hp) // nsm) * (tc + 2)
+        if best is None or cost < best[0]:
+            best = (cost, tc)
+    ns = -(-L // (best[1] * Q))
     if ns <= 1:
         return 0
     r = lambda v: (v + 255) // 256 * 256
     state = 4 * b * ns * H * P * N
     return 2 * r(state) + r(4 * b * ns * H)
+
+
+def test_plan_fills_whole_waves():
+    """The 0.3B 131072-token segment: 9 stripes x 16 head pairs = 144 CTAs, one wave of 148 SMs."""
+    assert _plan_bytes(1, 131072, 32, 64, 128, 128) == 2 * 4 * 9 * 32 * 64 * 128 + 9 * 32 * 4 + 256 - (9 * 32 * 4) % 256
 
 
 @pytest.mark.parametrize("shape", [(1, 16384, 32, 64, 128, 128), (1, 131072, 32, 64, 128, 128),
