@@ -4,9 +4,11 @@
 // output at t uses inputs t-3..t; concrete_test: kernel = 4).
 //
 // Pure HBM stream: each thread owns one 16-byte channel vector (8 bf16 or
-// 4 fp32 channels) over a block of TT consecutive tokens.  The 3-token halo
-// lives in registers and slides along the token block, so every input row is
-// read once (plus a 3-row halo per token block) and written once.
+// 4 fp32 channels) over a block of 64 consecutive tokens.  Its rows stream in
+// through a private 16-row ring in shared memory filled by cp.async, which
+// keeps 128 KB of loads in flight per SM without holding registers.  The
+// 3-token halo lives in registers and slides along the token block, so every
+// input row is read once (plus a 3-row halo per token block) and written once.
 #include <algorithm>
 
 #include "ssd_common.cuh"
@@ -15,7 +17,6 @@ namespace ssd {
 namespace {
 
 constexpr int kTokensPerThread = 64;
-constexpr int kUnroll = 4;
 
 struct alignas(16) Vec16 { uint32_t w[4]; };
 
@@ -72,21 +73,52 @@ template <> struct VecIO<float> {
     __device__ __forceinline__ static float silu(float z) { return z / (1.0f + expf(-z)); }
 };
 
+// cp.async of one 16-byte vector into shared memory (its own commit group per row)
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)),
+                 "l"(gmem)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+constexpr int kRing = 16;          // rows in flight per thread, staged in shared memory
+constexpr int kConvThreads = 256;
+
 template <typename T>
-__global__ void __launch_bounds__(256, 2) conv1d_silu_kernel(ConvParams p, int64_t n_tblk)
+__global__ void __launch_bounds__(kConvThreads, 2) conv1d_silu_kernel(ConvParams p, int64_t n_tblk)
 {
     using IO = VecIO<T>;
     constexpr int V = IO::kN;
+    // each thread streams its own rows through its own ring slots: [row slot][thread]
+    extern __shared__ Vec16 ring_raw[];
+    Vec16 (*ring)[kConvThreads] = reinterpret_cast<Vec16 (*)[kConvThreads]>(ring_raw);
     const int ncv = p.C_ch / V;
     const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int cv = (int)(gid % ncv);
     const int64_t rest = gid / ncv;
     const int64_t tb = rest % n_tblk;
     const int64_t bi = rest / n_tblk;
-    if (bi >= p.b) return;
+    const bool active = bi < p.b;
     const int c0 = cv * V;
 
     float w0[V], w1[V], w2[V], w3[V], bs[V];
+    const T *u = reinterpret_cast<const T *>(p.u) + bi * p.ubs + c0;
+    T *v = reinterpret_cast<T *>(p.v) + bi * p.vbs + c0;
+    const T *tin = p.tail_in ? reinterpret_cast<const T *>(p.tail_in) + bi * 3 * p.C_ch + c0 : nullptr;
+    const int64_t t0 = tb * kTokensPerThread;
+    const int n = active ? (int)(min(p.L, t0 + kTokensPerThread) - t0) : 0;
+    Vec16 *slot = &ring[0][threadIdx.x];
+    const T *up = u + t0 * p.urs;
+    // fill the ring: one commit group per row (empty groups past the end keep the count uniform)
+#pragma unroll
+    for (int j = 0; j < kRing; ++j) {
+        if (j < n) cp_async16(slot + j * kConvThreads, up + j * p.urs);
+        cp_async_commit();
+    }
+    if (!active) return;
     {
         const float4 *wp = reinterpret_cast<const float4 *>(p.w + (int64_t)c0 * 4);
 #pragma unroll
@@ -96,13 +128,6 @@ __global__ void __launch_bounds__(256, 2) conv1d_silu_kernel(ConvParams p, int64
             bs[i] = p.bias ? __ldg(p.bias + c0 + i) : 0.0f;
         }
     }
-    const T *u = reinterpret_cast<const T *>(p.u) + bi * p.ubs + c0;
-    T *v = reinterpret_cast<T *>(p.v) + bi * p.vbs + c0;
-    const T *tin = p.tail_in ? reinterpret_cast<const T *>(p.tail_in) + bi * 3 * p.C_ch + c0 : nullptr;
-
-    const int64_t t0 = tb * kTokensPerThread;
-    const int64_t t1 = min(p.L, t0 + kTokensPerThread);
-
     // halo: m3 = u[t-3], m2 = u[t-2], m1 = u[t-1]
     float m3[V], m2[V], m1[V];
     {
@@ -120,17 +145,19 @@ __global__ void __launch_bounds__(256, 2) conv1d_silu_kernel(ConvParams p, int64
             }
         }
     }
-
-    for (int64_t t = t0; t < t1; t += kUnroll) {
-        Vec16 raw[kUnroll];
+    T *vp = v + t0 * p.vrs;
+    up += kRing * p.urs;
+    for (int i0 = 0; i0 < n; i0 += kRing) {
 #pragma unroll
-        for (int j = 0; j < kUnroll; ++j)
-            if (t + j < t1) raw[j] = ld_stream(u + (t + j) * p.urs);
-#pragma unroll
-        for (int j = 0; j < kUnroll; ++j) {
-            if (t + j < t1) {
+        for (int j = 0; j < kRing; ++j) {
+            if (i0 + j < n) {
+                cp_async_wait<kRing - 1>();      // row i0 + j has landed (its group is the oldest)
                 float cur[V], out[V];
-                IO::unpack(raw[j], cur);
+                IO::unpack(slot[j * kConvThreads], cur);
+                // refill the slot with row i0 + j + kRing
+                if (i0 + j + kRing < n) cp_async16(slot + j * kConvThreads, up);
+                cp_async_commit();
+                up += p.urs;
 #pragma unroll
                 for (int i = 0; i < V; ++i) {
                     float z = bs[i];
@@ -141,10 +168,12 @@ __global__ void __launch_bounds__(256, 2) conv1d_silu_kernel(ConvParams p, int64
                     out[i] = IO::silu(z);
                     m3[i] = m2[i]; m2[i] = m1[i]; m1[i] = cur[i];
                 }
-                *reinterpret_cast<Vec16 *>(v + (t + j) * p.vrs) = IO::pack(out);
+                *reinterpret_cast<Vec16 *>(vp) = IO::pack(out);
+                vp += p.vrs;
             }
         }
     }
+    cp_async_wait<0>();
 }
 
 // tail_out[bi, r, c] = u at position L-3+r, or tail_in[bi, 3+pos, c] when pos < 0,
@@ -179,9 +208,18 @@ int launch_conv_t(const ConvParams &p, cudaStream_t st)
         prof_begin(st, kKConv);
         const int64_t n_tblk = (p.L + kTokensPerThread - 1) / kTokensPerThread;
         const int64_t threads = (int64_t)p.b * n_tblk * (p.C_ch / V);
-        const int64_t blocks = (threads + 255) / 256;
+        const int64_t blocks = (threads + kConvThreads - 1) / kConvThreads;
         if (blocks > 0x7fffffffLL) return 2;
-        conv1d_silu_kernel<T><<<(unsigned)blocks, 256, 0, st>>>(p, n_tblk);
+        constexpr int smem = kRing * kConvThreads * (int)sizeof(Vec16);
+        static bool attr_set[64] = {false};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+            if (cudaFuncSetAttribute(conv1d_silu_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+                return 7;
+            attr_set[dev] = true;
+        }
+        conv1d_silu_kernel<T><<<(unsigned)blocks, kConvThreads, smem, st>>>(p, n_tblk);
         prof_end(st, kKConv);
     }
     if (p.tail_out && p.b > 0) {
