@@ -228,12 +228,12 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
             }
             ++mmas;
             __syncwarp();
-            // the previous step's product has read its stage by now: refill it with step it + 2
-            if (it >= 1 && it + 2 < nc) {
-                const int pst = (it - 1) % kStagesA;
-                ok = ewait(&s.empty[pst], (uint32_t)((it - 1) / kStagesA) & 1, abort, lim);
+            // refill this stage with step it + 3 once the product has read it, so that three
+            // stages stay in flight (the next product cannot start before this one ends anyway)
+            if (it + kStagesA < nc) {
+                ok = ewait(&s.empty[st], (uint32_t)(it / kStagesA) & 1, abort, lim);
                 if (!ok) break;
-                if (lane == 0) issue_load(it + 2);
+                if (lane == 0) issue_load(it + kStagesA);
                 __syncwarp();
             }
         }
