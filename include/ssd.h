@@ -181,6 +181,51 @@ typedef struct ssd_stream_args {
 SSD_API int ssd_stream_forward(const ssd_stream_args *args, ssd_stream_t stream);
 
 /*
+ * Arguments of one decode step: a single new token of b independent streams
+ * (online inference on a video consumed as one continuous stream at 1 FPS --
+ * video-ma2mba-0.3b catalog page, "What is Video-Ma2mba?").  Per stream:
+ *   u       [b][C_ch] this token's pre-conv x|B|C (I/O dtype), C_ch = H*P + 2*G*N,
+ *           batch stride u_batch_stride elements, 16-byte aligned rows
+ *   conv_w  [C_ch][4] fp32, conv_bias [C_ch] fp32 or NULL
+ *   tail_in [b][3][C_ch] the three previous pre-conv tokens (oldest first), or
+ *           NULL for zeros (the first token of a stream)
+ *   tail_out[b][3][C_ch] receives [tail_in[1], tail_in[2], u]; may alias tail_in; NULL: not kept
+ *   dt      [b][H] fp32 (positive), A [H] fp32, D [H] fp32 or NULL
+ *   h_in    [b][H][P][N] fp32 state before the token, or NULL for zeros
+ *   h_out   [b][H][P][N] fp32 state after the token; may alias h_in
+ *   y       [b][H*P] (I/O dtype), batch stride y_batch_stride elements
+ * P, N in {16, 32, 64, 128}; H % G == 0.
+ */
+typedef struct ssd_decode_args {
+    int dtype;
+    int b;
+    int H, P, N, G;
+    const void *u;
+    int64_t u_batch_stride;
+    const float *conv_w;
+    const float *conv_bias;
+    const void *tail_in;
+    void *tail_out;
+    const float *dt;
+    const float *A;
+    const float *D;
+    const float *h_in;
+    float *h_out;
+    void *y;
+    int64_t y_batch_stride;
+} ssd_decode_args;
+
+/*
+ * ssd_decode_step -- the layer on one token: v = silu(causal conv4 of
+ * (tail, u)), then h = exp(dt*A) h + dt x B^T and y = C h + D x per head
+ * (Eq. (1) of the pages with the discretisation of the selective scan).
+ * Equal, up to rounding, to ssd_stream_forward on a one-token segment; a
+ * sequence of decode steps equals one call on the whole sequence.
+ * Asynchronous on `stream`; status as for the other entry points.
+ */
+SSD_API int ssd_decode_step(const ssd_decode_args *args, ssd_stream_t stream);
+
+/*
  * ssd_scan_forward_static_scratch -- ssd_scan_forward for callers that cannot
  * allocate device memory.  (The pages have no counterpart: this is a
  * deployment aid of this library, not part of the layer they describe.)

@@ -58,6 +58,15 @@ class StreamArgs(ctypes.Structure):
                 ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
 
 
+class DecodeArgs(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int), ("b", ctypes.c_int),
+                ("H", ctypes.c_int), ("P", ctypes.c_int), ("N", ctypes.c_int), ("G", ctypes.c_int),
+                ("u", _vp), ("u_batch_stride", _i64),
+                ("conv_w", _vp), ("conv_bias", _vp), ("tail_in", _vp), ("tail_out", _vp),
+                ("dt", _vp), ("A", _vp), ("D", _vp), ("h_in", _vp), ("h_out", _vp),
+                ("y", _vp), ("y_batch_stride", _i64)]
+
+
 _lib = None
 
 
@@ -76,6 +85,8 @@ def lib():
         L.ssd_scan_forward.restype = ctypes.c_int
         L.ssd_stream_forward.argtypes = [ctypes.POINTER(StreamArgs), _vp]
         L.ssd_stream_forward.restype = ctypes.c_int
+        L.ssd_decode_step.argtypes = [ctypes.POINTER(DecodeArgs), _vp]
+        L.ssd_decode_step.restype = ctypes.c_int
         L.ssd_scan_workspace_size.argtypes = [ctypes.c_int, _i64, ctypes.c_int, ctypes.c_int,
                                               ctypes.c_int, ctypes.c_int]
         L.ssd_scan_workspace_size.restype = ctypes.c_size_t
@@ -249,3 +260,32 @@ def stream_forward(u, conv_w, dt, A, D=None, *, H, P, N, G=1, Q=128, s=0, conv_b
     a.workspace = workspace.data_ptr(); a.workspace_bytes = workspace.numel()
     _check(lib().ssd_stream_forward(ctypes.byref(a), _stream(stream)))
     return {"v": v, "y": y, "h_final": h_final, "h_ckpt": h_ckpt, "tail_out": tail_out}
+
+
+def decode_step(u, conv_w, dt, A, D=None, *, H, P, N, G=1, conv_bias=None, tail_in=None,
+                tail_out=None, h_in=None, h_out=None, y=None, stream=None):
+    """One token of b streams: u [b, C_ch] (pre-conv x|B|C), dt [b, H].  Returns
+    {"y": [b, H, P], "h_out": [b, H, P, N], "tail_out": [b, 3, C_ch]}; h_out may be h_in
+    and tail_out may be tail_in (updated in place)."""
+    _cuda(u, conv_w, dt, A, D, conv_bias, tail_in, tail_out, h_in, h_out, y)
+    b, cch = u.shape
+    assert cch == H * P + 2 * G * N, "u must hold x|B|C channels"
+    dev = u.device
+    if y is None:
+        y = torch.empty(b, H, P, dtype=u.dtype, device=dev)
+    if h_out is None:
+        h_out = torch.empty(b, H, P, N, dtype=torch.float32, device=dev)
+    if tail_out is None:
+        tail_out = torch.empty(b, 3, cch, dtype=u.dtype, device=dev)
+    a = DecodeArgs()
+    a.dtype = _dtype_code(u); a.b = b; a.H = H; a.P = P; a.N = N; a.G = G
+    a.u = u.data_ptr(); a.u_batch_stride = u.stride(0)
+    a.conv_w = conv_w.data_ptr(); a.conv_bias = conv_bias.data_ptr() if conv_bias is not None else None
+    a.tail_in = tail_in.data_ptr() if tail_in is not None else None
+    a.tail_out = tail_out.data_ptr()
+    a.dt = dt.data_ptr(); a.A = A.data_ptr(); a.D = D.data_ptr() if D is not None else None
+    a.h_in = h_in.data_ptr() if h_in is not None else None
+    a.h_out = h_out.data_ptr()
+    a.y = y.data_ptr(); a.y_batch_stride = y.view(b, H * P).stride(0)
+    _check(lib().ssd_decode_step(ctypes.byref(a), _stream(stream)))
+    return {"y": y, "h_out": h_out, "tail_out": tail_out}

@@ -1,0 +1,143 @@
+// decode.cu -- one token of b independent streams (online inference, video
+// consumed as one continuous stream at 1 FPS: video-ma2mba-0.3b catalog page,
+// "What is Video-Ma2mba?").
+//
+// Per stream and token, the layer of the selective scan (Eq. (1) with the
+// discretisation exp(dt A), dt B x^T, C^T h + D x; causal conv1d of width 4
+// and SiLU on x|B|C in front, as in the pith.science verdict for arXiv
+// 2411.19460, skeptic_critique.load_bearing_attack):
+//   v = silu(bias + w0 tail[0] + w1 tail[1] + w2 tail[2] + w3 u)  (rounded to the I/O dtype)
+//   h = exp(dt A) h + dt x B^T,   y = C h + D x
+// The state is the traffic: 2 * P * N * 4 bytes per (stream, head), read and
+// written once.  One CTA per (stream, head): it recomputes the conv of the
+// channels it reads (its head's x, its group's B and C) from tail_in, then
+// streams its state with float4 loads (lane = 4 state columns, warp = P/8 rows)
+// and reduces y over n with shuffles.  The tail shift runs as a second kernel
+// after it, so that tail_out may alias tail_in.
+#include <algorithm>
+
+#include "ssd_common.cuh"
+
+namespace ssd {
+namespace {
+
+constexpr int kDecThreads = 256;
+
+template <typename T> __device__ __forceinline__ float dec_silu(float z);
+// one hardware tanh, the result is rounded to bf16 right after
+template <> __device__ __forceinline__ float dec_silu<__nv_bfloat16>(float z)
+{
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
+    return z * fmaf(0.5f, t, 0.5f);
+}
+template <> __device__ __forceinline__ float dec_silu<float>(float z) { return z / (1.0f + expf(-z)); }
+
+template <typename T>
+__global__ void __launch_bounds__(kDecThreads) decode_step_kernel(DecodeParams p)
+{
+    extern __shared__ float dsm[];          // x [P], B [N], C [N] of this (stream, head)
+    float *xs = dsm, *Bs = dsm + p.P, *Cs = Bs + p.N;
+    const int bi = blockIdx.x / p.H, h = blockIdx.x % p.H;
+    const int g = (int)((int64_t)h * p.G / p.H);
+    const int din = p.H * p.P;
+    const int C_ch = din + 2 * p.G * p.N;
+    const T *u = reinterpret_cast<const T *>(p.u) + (int64_t)bi * p.ubs;
+    const T *tin = p.tail_in ? reinterpret_cast<const T *>(p.tail_in) + (int64_t)bi * 3 * C_ch : nullptr;
+
+    // conv + SiLU of the P + 2N channels this head reads
+    for (int i = threadIdx.x; i < p.P + 2 * p.N; i += blockDim.x) {
+        const int c = i < p.P ? h * p.P + i : (i < p.P + p.N ? din + g * p.N + (i - p.P)
+                                                             : din + p.G * p.N + g * p.N + (i - p.P - p.N));
+        const float4 w = reinterpret_cast<const float4 *>(p.w)[c];
+        float z = p.bias ? p.bias[c] : 0.0f;
+        if (tin) {
+            z = fmaf(w.x, to_f32(tin[c]), z);
+            z = fmaf(w.y, to_f32(tin[C_ch + c]), z);
+            z = fmaf(w.z, to_f32(tin[2 * C_ch + c]), z);
+        }
+        z = fmaf(w.w, to_f32(u[c]), z);
+        dsm[i] = to_f32(from_f32<T>(dec_silu<T>(z)));   // v is an I/O-dtype tensor in the layer
+    }
+    __syncthreads();
+
+    const float dt = p.dt[(int64_t)bi * p.H + h];
+    const float a = exp2f(dt * p.A[h] * 1.4426950408889634f);
+    const float Dh = p.D ? p.D[h] : 0.0f;
+    const int64_t PN = (int64_t)p.P * p.N;
+    const float *hin = p.h_in ? p.h_in + ((int64_t)bi * p.H + h) * PN : nullptr;
+    float *hout = p.h_out + ((int64_t)bi * p.H + h) * PN;
+    T *y = reinterpret_cast<T *>(p.y) + (int64_t)bi * p.ybs + (int64_t)h * p.P;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nw = blockDim.x >> 5;
+    const int nq = p.N >> 2;                // float4 columns per state row (4 .. 32)
+    // lanes take 4 state columns each; a warp covers 32 / nq rows at a time
+    const int rows_per_pass = 32 / nq;
+    const int sub = lane / nq, col = lane % nq;
+    const float4 Bv = reinterpret_cast<const float4 *>(Bs)[col];
+    const float4 Cv = reinterpret_cast<const float4 *>(Cs)[col];
+    for (int p0 = warp * rows_per_pass; p0 < p.P; p0 += nw * rows_per_pass) {
+        const int pr = p0 + sub;
+        float part = 0.0f;
+        if (pr < p.P) {
+            const float4 hv = hin ? reinterpret_cast<const float4 *>(hin + (int64_t)pr * p.N)[col]
+                                  : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            const float dx = dt * xs[pr];
+            float4 o;
+            o.x = fmaf(a, hv.x, dx * Bv.x);
+            o.y = fmaf(a, hv.y, dx * Bv.y);
+            o.z = fmaf(a, hv.z, dx * Bv.z);
+            o.w = fmaf(a, hv.w, dx * Bv.w);
+            reinterpret_cast<float4 *>(hout + (int64_t)pr * p.N)[col] = o;
+            part = fmaf(Cv.x, o.x, fmaf(Cv.y, o.y, fmaf(Cv.z, o.z, Cv.w * o.w)));
+        }
+        // sum over the nq lanes of this row
+        for (int o = 1; o < nq; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if (col == 0 && pr < p.P) y[pr] = from_f32<T>(fmaf(Dh, xs[pr], part));
+    }
+}
+
+// tail_out[bi] = [tail_in[bi][1], tail_in[bi][2], u[bi]] (zeros for a NULL tail_in);
+// each thread reads its channel's values before writing, so tail_out may alias tail_in
+template <typename T>
+__global__ void decode_tail_kernel(DecodeParams p)
+{
+    const int C_ch = p.H * p.P + 2 * p.G * p.N;
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= (int64_t)p.b * C_ch) return;
+    const int64_t bi = gid / C_ch;
+    const int c = (int)(gid % C_ch);
+    const T *tin = p.tail_in ? reinterpret_cast<const T *>(p.tail_in) + bi * 3 * C_ch + c : nullptr;
+    const T t1 = tin ? tin[C_ch] : from_f32<T>(0.0f);
+    const T t2 = tin ? tin[2 * C_ch] : from_f32<T>(0.0f);
+    const T uc = reinterpret_cast<const T *>(p.u)[bi * p.ubs + c];
+    T *tout = reinterpret_cast<T *>(p.tail_out) + bi * 3 * C_ch + c;
+    tout[0] = t1;
+    tout[C_ch] = t2;
+    tout[2 * C_ch] = uc;
+}
+
+template <typename T>
+int launch_decode_t(const DecodeParams &p, cudaStream_t st)
+{
+    if (p.b > 0) {
+        const size_t smem = sizeof(float) * (size_t)(p.P + 2 * p.N);
+        prof_begin(st, kKDecode);
+        decode_step_kernel<T><<<(unsigned)(p.b * p.H), kDecThreads, smem, st>>>(p);
+        prof_end(st, kKDecode);
+        if (p.tail_out) {
+            const int64_t n = (int64_t)p.b * (p.H * p.P + 2 * p.G * p.N);
+            decode_tail_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p);
+        }
+    }
+    return cudaGetLastError() == cudaSuccess ? 0 : 7;
+}
+
+}  // namespace
+
+int launch_decode(const DecodeParams &p, int dtype, cudaStream_t st)
+{
+    return dtype == 1 ? launch_decode_t<__nv_bfloat16>(p, st) : launch_decode_t<float>(p, st);
+}
+
+}  // namespace ssd

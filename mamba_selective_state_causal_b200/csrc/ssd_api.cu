@@ -241,7 +241,7 @@ int conv_impl(const void *u, int64_t ubs, int64_t urs, const float *w, const flo
 // ---------------------------------------------------------------- kernel timing
 const char *const kKernelNames[ssd::kKCount] = {
     "conv1d_silu", "conv_tail", "stripe_state_tc", "stripe_chain", "chunk_output_tc",
-    "stripe_state_generic", "chunk_output_generic"};
+    "stripe_state_generic", "chunk_output_generic", "decode_step"};
 
 struct ProfRecord {
     int id;
@@ -371,6 +371,36 @@ int ssd_stream_forward(const ssd_stream_args *a, ssd_stream_t stream)
     s.h_final = a->h_final; s.h_ckpt = a->h_ckpt;
     s.workspace = a->workspace; s.workspace_bytes = a->workspace_bytes;
     return scan_impl(&s, (cudaStream_t)stream);
+}
+
+int ssd_decode_step(const ssd_decode_args *a, ssd_stream_t stream)
+{
+    if (!a) return fail(SSD_ERR_NULL, "args is NULL");
+    if (a->dtype != SSD_F32 && a->dtype != SSD_BF16) return fail(SSD_ERR_DTYPE, "unknown dtype %d", a->dtype);
+    if (a->b < 0) return fail(SSD_ERR_SHAPE, "negative b (%d)", a->b);
+    if (a->H <= 0 || a->G <= 0 || a->H % a->G != 0)
+        return fail(SSD_ERR_SHAPE, "need H > 0, G > 0 and H %% G == 0 (H=%d, G=%d)", a->H, a->G);
+    if (!pow2_dim(a->P) || !pow2_dim(a->N))
+        return fail(SSD_ERR_SHAPE, "P and N must be 16, 32, 64 or 128 (P=%d, N=%d)", a->P, a->N);
+    if (a->b == 0) return ok();
+    const int64_t C_ch = (int64_t)a->H * a->P + 2LL * a->G * a->N;
+    const size_t es = elem_size(a->dtype);
+    if (!a->u || !a->conv_w || !a->dt || !a->A || !a->h_out || !a->y)
+        return fail(SSD_ERR_NULL, "u, conv_w, dt, A, h_out and y must not be NULL");
+    if (a->u_batch_stride < C_ch || (a->b > 1 && a->y_batch_stride < (int64_t)a->H * a->P) || a->y_batch_stride < 0)
+        return fail(SSD_ERR_STRIDE, "batch strides smaller than a row");
+    if (!aligned16(a->u) || (a->u_batch_stride * es) % 16 != 0 || !aligned16(a->conv_w) ||
+        (a->tail_in && !aligned16(a->tail_in)) || (a->tail_out && !aligned16(a->tail_out)) ||
+        (a->h_in && !aligned16(a->h_in)) || !aligned16(a->h_out))
+        return fail(SSD_ERR_ALIGN, "u rows, conv_w, tails and states must be 16-byte aligned");
+    ssd::DecodeParams p{};
+    p.b = a->b; p.H = a->H; p.P = a->P; p.N = a->N; p.G = a->G;
+    p.u = a->u; p.ubs = a->u_batch_stride; p.w = a->conv_w; p.bias = a->conv_bias;
+    p.tail_in = a->tail_in; p.tail_out = a->tail_out; p.dt = a->dt; p.A = a->A; p.D = a->D;
+    p.h_in = a->h_in; p.h_out = a->h_out; p.y = a->y; p.ybs = a->y_batch_stride;
+    const int rc = ssd::launch_decode(p, a->dtype, (cudaStream_t)stream);
+    if (rc) return fail(SSD_ERR_LAUNCH, "decode launch failed: %s", cudaGetErrorString(cudaGetLastError()));
+    return ok();
 }
 
 int ssd_sync_status(ssd_stream_t stream)

@@ -58,6 +58,24 @@ struct ConvParams {
     int C_ch;
 };
 
+// One decode step (decode.cu).
+struct DecodeParams {
+    int b, H, P, N, G;
+    const void *u;
+    int64_t ubs;
+    const float *w;
+    const float *bias;
+    const void *tail_in;
+    void *tail_out;
+    const float *dt;
+    const float *A;
+    const float *D;
+    const float *h_in;
+    float *h_out;
+    void *y;
+    int64_t ybs;
+};
+
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
@@ -84,13 +102,14 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // Kernel timing hooks (ssd_api.cu): no-ops unless ssd_profile_begin() is active
 // on the calling thread.
 enum KernelId : int {
-    kKConv = 0, kKConvTail, kKStateTc, kKChain, kKOutputTc, kKStateGeneric, kKOutputGeneric, kKCount
+    kKConv = 0, kKConvTail, kKStateTc, kKChain, kKOutputTc, kKStateGeneric, kKOutputGeneric, kKDecode, kKCount
 };
 void prof_begin(cudaStream_t st, int id);
 void prof_end(cudaStream_t st, int id);
 
 // Launchers (defined in the .cu files).
 int launch_conv(const ConvParams &p, int dtype, cudaStream_t st);
+int launch_decode(const DecodeParams &p, int dtype, cudaStream_t st);
 int launch_scan_generic(const ScanParams &p, int dtype, cudaStream_t st);
 bool tc_scan_supported(const ScanParams &p, int dtype);
 int launch_scan_tc(const ScanParams &p, cudaStream_t st);
