@@ -49,6 +49,9 @@ def parse_args():
     # profiling aids: run a shorter stream of the same shape (not a bench line)
     ap.add_argument("--seq-len", type=int, default=None)
     ap.add_argument("--segments", type=int, default=None)
+    # the decode step instead of the headline step: this many independent streams of the
+    # 0.3B shape, each advancing one token per step (its own JSON line)
+    ap.add_argument("--decode-streams", type=int, default=0)
     return ap.parse_args()
 
 
@@ -351,6 +354,63 @@ def run_e2e(layer, steps=3):
             "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}
 
 
+def run_decode(args, world, rank, local):
+    """Decode steps: each of B independent streams of the 0.3B shape takes one token per step
+    (conv tail and state updated in place), timed with CUDA events like the headline step."""
+    import __graft_entry__
+    __graft_entry__.build()
+    import mamba_selective_state_causal_b200 as ssd
+    nb = args.decode_streams
+    base = ssd_synth.BY_NAME[DEFAULT_WORKLOAD]
+    n_tok = args.warmup + args.steps
+    wl = ssd_synth.scaled(base, b=nb, L=n_tok, segments=1, name=f"decode-0.3b-{nb}streams")
+    d = torch.device("cuda", torch.cuda.current_device())
+    seed = rank_seed(wl, rank)
+    prm = ssd_synth.make_params(wl, device=d, seed=seed)
+    u_steps = ssd_synth.make_u(wl, device=d, seed=seed).transpose(0, 1).contiguous()     # [T][B][C_ch]
+    dt_steps = ssd_synth.make_dt(wl, prm["dt_bias"], device=d, seed=seed).transpose(0, 1).contiguous()
+    h = torch.zeros(nb, wl.H, wl.P, wl.N, dtype=torch.float32, device=d)
+    tail = torch.zeros(nb, 3, wl.cch, dtype=u_steps.dtype, device=d)
+    y = torch.empty(nb, wl.H, wl.P, dtype=u_steps.dtype, device=d)
+    t = [0]
+
+    def step():
+        ssd.decode_step(u_steps[t[0]], prm["w"], dt_steps[t[0]], prm["A"], prm["D"], H=wl.H, P=wl.P,
+                        N=wl.N, G=wl.G, conv_bias=prm["bias"], tail_in=tail, tail_out=tail,
+                        h_in=h, h_out=h, y=y)
+        t[0] += 1
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    ms = time_steps(step, args.steps, args.warmup, world, local)
+    clk = clocks.stop()
+    ssd.sync_status()
+    ms = max_over_ranks(world, ms)
+    e = 2
+    step_bytes = nb * (2 * 4 * wl.H * wl.P * wl.N          # state read + write
+                       + e * wl.cch + 2 * e * 3 * wl.cch     # token in, conv tail read + write
+                       + e * wl.H * wl.P + 4 * wl.H)         # y out, dt in
+    peak, peak_src = hbm_peak()
+    achieved = step_bytes / (ms / args.steps / 1e3) / 1e9
+    line = {
+        "metric": "SSD decode step tokens/s (independent streams of the 0.3B shape)",
+        "value": nb * world * args.steps / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "streams": nb, "heads": wl.H, "headdim": wl.P, "d_state": wl.N,
+                   "l2": "state larger than L2 (%.0f MB)" % (nb * wl.H * wl.P * wl.N * 4 / 1e6)
+                   if nb * wl.H * wl.P * wl.N * 4 > 126e6 else "state fits in L2"},
+        "roofline": {"bound": "hbm", "kernel": "decode_step", "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": achieved / peak, "peak_source": peak_src, "traffic": None,
+                     "algorithmic_bytes_per_launch": step_bytes},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     wl = ssd_synth.BY_NAME[args.workload]
@@ -360,6 +420,9 @@ def main():
     world, rank, local = dist_setup()
     if args.impl == "reference":
         run_reference(args, wl, world, rank)
+        return
+    if args.decode_streams > 0:
+        run_decode(args, world, rank, local)
         return
     import __graft_entry__
     __graft_entry__.build()

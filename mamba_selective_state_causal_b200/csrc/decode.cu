@@ -76,24 +76,36 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(DecodeParams p
     const int sub = lane / nq, col = lane % nq;
     const float4 Bv = reinterpret_cast<const float4 *>(Bs)[col];
     const float4 Cv = reinterpret_cast<const float4 *>(Cs)[col];
-    for (int p0 = warp * rows_per_pass; p0 < p.P; p0 += nw * rows_per_pass) {
-        const int pr = p0 + sub;
-        float part = 0.0f;
-        if (pr < p.P) {
-            const float4 hv = hin ? reinterpret_cast<const float4 *>(hin + (int64_t)pr * p.N)[col]
-                                  : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            const float dx = dt * xs[pr];
-            float4 o;
-            o.x = fmaf(a, hv.x, dx * Bv.x);
-            o.y = fmaf(a, hv.y, dx * Bv.y);
-            o.z = fmaf(a, hv.z, dx * Bv.z);
-            o.w = fmaf(a, hv.w, dx * Bv.w);
-            reinterpret_cast<float4 *>(hout + (int64_t)pr * p.N)[col] = o;
-            part = fmaf(Cv.x, o.x, fmaf(Cv.y, o.y, fmaf(Cv.z, o.z, Cv.w * o.w)));
+    // rows of this thread: pr = p0 + sub for p0 = warp * rows_per_pass + k * stride; their state
+    // loads are issued kBatch at a time before any is used, to keep several in flight
+    constexpr int kBatch = 4;
+    const int stride = nw * rows_per_pass;
+    for (int pb = warp * rows_per_pass; pb < p.P; pb += kBatch * stride) {
+        float4 hv[kBatch];
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) {
+            const int pr = pb + k * stride + sub;
+            hv[k] = (hin && pr < p.P) ? reinterpret_cast<const float4 *>(hin + (int64_t)pr * p.N)[col]
+                                      : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         }
-        // sum over the nq lanes of this row
-        for (int o = 1; o < nq; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-        if (col == 0 && pr < p.P) y[pr] = from_f32<T>(fmaf(Dh, xs[pr], part));
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) {
+            const int pr = pb + k * stride + sub;
+            float part = 0.0f;
+            if (pr < p.P) {
+                const float dx = dt * xs[pr];
+                float4 o;
+                o.x = fmaf(a, hv[k].x, dx * Bv.x);
+                o.y = fmaf(a, hv[k].y, dx * Bv.y);
+                o.z = fmaf(a, hv[k].z, dx * Bv.z);
+                o.w = fmaf(a, hv[k].w, dx * Bv.w);
+                reinterpret_cast<float4 *>(hout + (int64_t)pr * p.N)[col] = o;
+                part = fmaf(Cv.x, o.x, fmaf(Cv.y, o.y, fmaf(Cv.z, o.z, Cv.w * o.w)));
+            }
+            // sum over the nq lanes of this row
+            for (int o = 1; o < nq; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+            if (col == 0 && pr < p.P) y[pr] = from_f32<T>(fmaf(Dh, xs[pr], part));
+        }
     }
 }
 
