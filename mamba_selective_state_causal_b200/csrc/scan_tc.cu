@@ -325,10 +325,13 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
 // Issuing warp, per chunk c (the whole warp waits, one lane issues):
 //   Pm ready -> Y_a = Pm_a X_a, Y_b = Pm_b X_b, Ys = C [hp_a | hp_b]^T (into G's
 //   columns, G being spent); w o X ready -> S = B^T [Xw_a | Xw_b], accumulated
-//   straight into the fp32 state H in TMEM, then the other X slot (y of chunk
-//   c-1, stored by now) is refilled with chunk c+1; products done -> G of chunk
-//   c+1 into the columns Pm used, then the B/C slot is refilled;
-//   y staged -> TMA store of y.
+//   straight into the fp32 state H in TMEM; products done -> G of chunk c+1
+//   into the columns Pm used, the B/C slot is refilled, and X of chunk c+1 is
+//   loaded into the X slot w o X came from; y staged -> TMA store of y, then,
+//   once the store has read its slot, chunk c+1 may write its w o X there.
+// The two X slots alternate: chunk c's X sits in slot c & 1, its w o X goes
+// to slot (c + 1) & 1 (so that scaling X never waits for Y = Pm X to read it)
+// and its y is staged back in slot c & 1.
 // Warp 4 (no masked-decay work of its own) also publishes the chunk cumsum of
 // dt*A of both heads for chunk c+1 once the products of chunk c are done.
 // Compute warp (TMEM lane quarter q = warp & 3, column slice cs = warp >> 2 of
@@ -336,7 +339,7 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
 //   mask: Pm columns 32 cs .. 32 cs + 31, i.e. head hd's 32-token column
 //         blocks 2 (cs & 1) and 2 (cs & 1) + 1 of its 32 rows:
 //         Pm[i][j] = G[i][j] exp(cs_i - cs_j) dt_j (j <= i), + D on the diagonal
-//   w o X over X_hd (rows split over the head's 8 warps) once Y_hd is done
+//   w o X of head hd into the other X slot (rows split over the head's 8 warps)
 //   state (before the mask): H holds h after the previous chunk; its bf16 copy
 //         -> hp, checkpoint, then H = exp(cs_last) H, to which S is added
 //   y = Y + exp(cs_i) Ys -> bf16 -> the X slot (same swizzle as the y map)
@@ -359,7 +362,7 @@ struct SmemC {
     float cvs[2][kQ];          // chunk-inclusive cumsum of dt*A (log2 units), per head
     float dvs[2][kQ];          // dt, per head
     float fs[2][3 * 32];       // dt_j exp(cs_end(J) - cs_j) for the 32-token blocks J = 0..2
-    uint64_t full_bc[2], full_x[2], g_done, m2a, m2b, mma_done, fin;   // TMA / MMA -> warps
+    uint64_t full_bc[2], full_x[2], g_done, mma_done, fin, xslot_free; // TMA / MMA / issuer -> warps
     uint64_t pm_ready, xw_ready, y_ready, scan_ready;                  // warps -> issuing warp
     uint32_t tmem;
     int abort;
@@ -403,8 +406,7 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) { mbar_init(&s.full_bc[i], 1); mbar_init(&s.full_x[i], 1); }
         mbar_init(&s.g_done, 1);
-        mbar_init(&s.m2a, 1);
-        mbar_init(&s.m2b, 1);
+        mbar_init(&s.xslot_free, 1);
         mbar_init(&s.mma_done, 1);
         mbar_init(&s.fin, 1);
         mbar_init(&s.pm_ready, kComputeWarps);
@@ -640,20 +642,22 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
             // the epilogue's factor (the scan buffer is rewritten once w o X is done)
             const float e_r = ex2(s.cvs[hd][r]);
 
-            // ---- w o X over X_hd once Y_hd has read it: 4 chunks of 16 B per thread
+            // ---- w o X of head hd into the other X slot (free once the previous y store has read it),
+            //      so that it need not wait for Y = Pm X: 4 chunks of 16 B per thread
             if (!(ewait(&s.full_x[c & 1], (c >> 1) & 1, abort, lim) &&
-                  ewait(hd ? &s.m2b : &s.m2a, c & 1, abort, lim))) { fail(); break; }
+                  ewait(&s.xslot_free, c & 1, abort, lim))) { fail(); break; }
             {
                 const int ti = 32 * (warp & 7) + lane;
                 const int j = ti >> 1, ch = 4 * (ti & 1);
                 const float w = s.dvs[hd][j] * ex2(s.cvs[hd][kQ - 1] - s.cvs[hd][j]);
-                uint8_t *base = xs + hd * kBox;
+                const uint8_t *src = xs + hd * kBox;
+                uint8_t *dst = s.x[(c + 1) & 1] + hd * kBox;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    uint4 v = lds128(base + swz(j, ch + u));
+                    uint4 v = lds128(src + swz(j, ch + u));
                     v.x = scale_bf16x2_int(v.x, w); v.y = scale_bf16x2_int(v.y, w);
                     v.z = scale_bf16x2_int(v.z, w); v.w = scale_bf16x2_int(v.w, w);
-                    sts128(base + swz(j, ch + u), v);
+                    sts128(dst + swz(j, ch + u), v);
                 }
             }
             fence_proxy_async_smem();
@@ -751,7 +755,7 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
                 issue_bc(0);
                 if (nc > 1) issue_bc(1);
                 issue_x(0);
-                if (nc > 1) issue_x(1);
+                mbar_arrive(&s.xslot_free);   // chunk 0's w o X goes into the untouched slot 1
             }
             ok = ewait(&s.full_bc[0], 0, abort, lim);
             if (ok) {
@@ -775,11 +779,9 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ts(tY, tPm + kk * 8, smem_desc(sX + kk * 2048, 0, 1024), id_pm, kk > 0);
-                mma_commit(&s.m2a);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ts(tY + 64, tPm + 64 + kk * 8, smem_desc(sX + kBox + kk * 2048, 0, 1024), id_pm, kk > 0);
-                mma_commit(&s.m2b);
                 const uint32_t sC = smem_u32(s.bc[c & 1]), sHp = smem_u32(s.hp);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -793,16 +795,11 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
             if (!ok) break;
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t sB = smem_u32(s.bc[c & 1]) + 2 * kBox, sXw = smem_u32(xs);
+                const uint32_t sB = smem_u32(s.bc[c & 1]) + 2 * kBox, sXw = smem_u32(s.x[(c + 1) & 1]);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ss(tH, smem_desc(sB + kk * 2048, kBox, 1024), smem_desc(sXw + kk * 2048, kBox, 1024), id_s, true);
                 mma_commit(&s.mma_done);
-                // the other X slot held y of chunk c-1, whose store has been read by now: chunk c+1 goes there
-                if (c >= 1 && c + 1 < nc) {
-                    tma_store_wait_read<0>();
-                    issue_x(c + 1);
-                }
             }
             __syncwarp();
             // products done: G of chunk c+1 into the columns Pm used, then refill this B/C slot
@@ -816,6 +813,8 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
                 if (lane == 0) { ++bc_waited; issue_g(c + 1, tPm); }
             }
             if (lane == 0 && c + 2 < nc) issue_bc(c + 2);
+            // S has read w o X from the other X slot: chunk c+1's X goes there
+            if (lane == 0 && c + 1 < nc) issue_x(c + 1);
             __syncwarp();
             // y staged: store it (the slot is refilled once the next chunk's products are issued)
             ok = ewait(&s.y_ready, c & 1, abort, lim);
@@ -824,6 +823,9 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
                 tma_store_3d(&maps.y, xs, ha * kP, (int)t0, bi);
                 tma_store_3d(&maps.y, xs + kBox, (ha + 1) * kP, (int)t0, bi);
                 tma_store_commit();
+                // once the store has read the slot, chunk c+1 may write its w o X there
+                tma_store_wait_read<0>();
+                mbar_arrive(&s.xslot_free);
             }
             __syncwarp();
         }
