@@ -13,10 +13,10 @@
 //   G  = C B^T                                     tcgen05, 128x128x128, TMEM
 //   Pm = G o [exp(cs_i - cs_j) dt_j, j <= i] + D I CUDA cores, TMEM -> TMEM (bf16)
 //   Yd = Pm X                                      tcgen05, A from TMEM, 128x64x128
-//   Yo = C h_prev^T                                tcgen05, 128x64x128
+//   Yo = C h_prev^T                                tcgen05, 128x128x128 (both heads)
 //   y  = Yd + exp(cs_i) Yo                         CUDA cores -> smem -> TMA store
-//   S  = B^T (w o X),  w_j = dt_j exp(cs_last - cs_j)   tcgen05, 128x64x128
-//   h  = exp(cs_last) h + S                        CUDA cores, fp32 state in registers
+//   S  = B^T (w o X),  w_j = dt_j exp(cs_last - cs_j)   tcgen05, 128x128x128 (both heads)
+//   h  = exp(cs_last) h + S                        fp32 state in TMEM, S accumulated into it
 // Only non-positive differences of cs are exponentiated.  The state is kept in
 // fp32; its bf16 copy only feeds the C h_prev^T product.  Both kernels take
 // two heads per CTA: they share B (and C), so G is computed once per pair and
@@ -333,16 +333,16 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
 // to slot (c + 1) & 1 (so that scaling X never waits for Y = Pm X to read it)
 // and its y is staged back in slot c & 1.
 // Warp 4 (no masked-decay work of its own) also publishes the chunk cumsum of
-// dt*A of both heads for chunk c+1 once the products of chunk c are done.
+// dt*A of both heads for chunk c+1 once every warp has written chunk c's w o X.
 // Compute warp (TMEM lane quarter q = warp & 3, column slice cs = warp >> 2 of
 // the 128 (head, p) columns; head hd = cs >> 1), per chunk:
 //   mask: Pm columns 32 cs .. 32 cs + 31, i.e. head hd's 32-token column
 //         blocks 2 (cs & 1) and 2 (cs & 1) + 1 of its 32 rows:
 //         Pm[i][j] = G[i][j] exp(cs_i - cs_j) dt_j (j <= i), + D on the diagonal
 //   w o X of head hd into the other X slot (rows split over the head's 8 warps)
-//   state (before the mask): H holds h after the previous chunk; its bf16 copy
-//         -> hp, checkpoint, then H = exp(cs_last) H, to which S is added
-//   y = Y + exp(cs_i) Ys -> bf16 -> the X slot (same swizzle as the y map)
+//   y = Y + exp(cs_i) Ys -> bf16 -> the X slot (same swizzle as the y map), and
+//   with it the state step of chunk c+1: H (h after chunk c) -> bf16 copy hp,
+//         checkpoint, then H = exp(cs_last(c+1)) H, to which S of chunk c+1 is added
 // A warp writes Pm into exactly the columns it read Ys from one chunk earlier,
 // and reads Y / S / Ys columns only it owns, so no barrier among the compute
 // warps is needed; hand-offs go through mbarriers (one arrival per warp).
@@ -350,14 +350,14 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
 // TMEM (512 columns): R0 = 0..127 and R1 = 128..255 alternate between {G, Ys}
 // and {Pm_a, Pm_b} by chunk parity; Y = 256..383 (a | b); H = 384..511 (a | b),
 // the fp32 state, rows n.
-// Shared memory: B/C ring of 2, X ring of 2 (each X slot then holds w o X and
-// finally the chunk's y), hp, and the per-head scan values (about 227 KB).
+// Shared memory: B/C ring of 2, two X slots (a slot holds a chunk's X, then its
+// y, then the next chunk's w o X), hp, and the per-head scan values (about 227 KB).
 constexpr int kComputeWarps = 16;
 constexpr int kThreadsC = 32 * (kComputeWarps + 1);
 
 struct SmemC {
     uint8_t bc[2][4 * kBox];   // ring slot: C box 0, C box 1, B box 0, B box 1
-    uint8_t x[2][2 * kBox];    // ring slot: X of head a, X of head b
+    uint8_t x[2][2 * kBox];    // X slot: head a box, head b box (X, then y, then the next chunk's w o X)
     uint8_t hp[2 * kBox];      // bf16 h_prev of head a, head b (rows n, cols p), 128B-swizzled
     float cvs[2][kQ];          // chunk-inclusive cumsum of dt*A (log2 units), per head
     float dvs[2][kQ];          // dt, per head

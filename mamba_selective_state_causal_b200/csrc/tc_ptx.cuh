@@ -251,16 +251,6 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar)
                  : "memory");
 }
 
-__device__ __forceinline__ uint32_t elect_one()
-{
-    uint32_t pred = 0;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t.reg .b32 r;\n\t"
-        "elect.sync r|p, 0xffffffff;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(pred));
-    return pred;
-}
 
 }  // namespace tc
 }  // namespace ssd
