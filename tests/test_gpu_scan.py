@@ -46,6 +46,7 @@ W = ssd_synth.WORKLOADS
     ssd_synth.scaled(W[0], L=500, H=4, G=2, P=32, N=32, Q=64, s=128),      # two groups, fp32
     ssd_synth.scaled(W[4], L=4096, H=6, b=2),                              # long dt: decay underflow
     ssd_synth.scaled(W[1], L=5000, H=5, P=128, N=16, Q=64, s=64, b=1),     # P=128, N=16
+    ssd_synth.scaled(W[1], L=1500, H=8, G=2, b=1),                         # tensor cores, two B/C groups
 ], ids=lambda w: f"{w.dtype}-b{w.b}-L{w.L}-H{w.H}-P{w.P}-N{w.N}-G{w.G}-Q{w.Q}-s{w.s}")
 def test_scan_matches_oracle(wl):
     out, ref = run_case(wl)
