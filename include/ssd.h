@@ -122,6 +122,14 @@ typedef struct ssd_scan_args {
     float *h_ckpt;
     void *workspace;
     size_t workspace_bytes;
+    /* dt as given, or dt_eff = clamp(f(dt + dt_bias[h]), dt_min, dt_max): dt_bias [H]
+     * fp32 or NULL (none), f = softplus(v) = log(1 + e^v) when dt_softplus != 0 and
+     * the identity otherwise, the clamp applied only when dt_max > 0.  A
+     * zero-initialised struct leaves dt unchanged.  (The Mamba-2 block's
+     * dt_bias + softplus, fused here; the pages give dt itself.) */
+    const float *dt_bias;
+    int dt_softplus;
+    float dt_min, dt_max;
 } ssd_scan_args;
 
 /*
@@ -134,7 +142,10 @@ typedef struct ssd_scan_args {
 SSD_API int ssd_scan_forward(const ssd_scan_args *args, ssd_stream_t stream);
 
 /* Bytes of workspace ssd_scan_forward / ssd_stream_forward need for this shape
- * on the current device (the stripe plan depends on its SM count). */
+ * on the current device (the stripe plan depends on its SM count): the stripe
+ * states, then room for the effective dt [b][L][H] fp32.  Calls that ask for
+ * none of dt_bias / softplus / clamp need only the first part, which is 0 when
+ * the sequence is a single stripe. */
 SSD_API size_t ssd_scan_workspace_size(int b, int64_t L, int H, int P, int N, int Q);
 
 /*
@@ -168,6 +179,14 @@ typedef struct ssd_stream_args {
     float *h_ckpt;
     void *workspace;
     size_t workspace_bytes;
+    /* dt as given, or dt_eff = clamp(f(dt + dt_bias[h]), dt_min, dt_max): dt_bias [H]
+     * fp32 or NULL (none), f = softplus(v) = log(1 + e^v) when dt_softplus != 0 and
+     * the identity otherwise, the clamp applied only when dt_max > 0.  A
+     * zero-initialised struct leaves dt unchanged.  (The Mamba-2 block's
+     * dt_bias + softplus, fused here; the pages give dt itself.) */
+    const float *dt_bias;
+    int dt_softplus;
+    float dt_min, dt_max;
 } ssd_stream_args;
 
 /*
@@ -213,6 +232,14 @@ typedef struct ssd_decode_args {
     float *h_out;
     void *y;
     int64_t y_batch_stride;
+    /* dt as given, or dt_eff = clamp(f(dt + dt_bias[h]), dt_min, dt_max): dt_bias [H]
+     * fp32 or NULL (none), f = softplus(v) = log(1 + e^v) when dt_softplus != 0 and
+     * the identity otherwise, the clamp applied only when dt_max > 0.  A
+     * zero-initialised struct leaves dt unchanged.  (The Mamba-2 block's
+     * dt_bias + softplus, fused here; the pages give dt itself.) */
+    const float *dt_bias;
+    int dt_softplus;
+    float dt_min, dt_max;
 } ssd_decode_args;
 
 /*

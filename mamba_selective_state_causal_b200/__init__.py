@@ -42,7 +42,9 @@ class ScanArgs(ctypes.Structure):
                 ("dt", _vp), ("A", _vp), ("D", _vp), ("h0", _vp),
                 ("y", _vp), ("y_batch_stride", _i64), ("y_row_stride", _i64),
                 ("h_final", _vp), ("h_ckpt", _vp),
-                ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
+                ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
+                ("dt_bias", _vp), ("dt_softplus", ctypes.c_int),
+                ("dt_min", ctypes.c_float), ("dt_max", ctypes.c_float)]
 
 
 class StreamArgs(ctypes.Structure):
@@ -55,7 +57,9 @@ class StreamArgs(ctypes.Structure):
                 ("dt", _vp), ("A", _vp), ("D", _vp), ("h0", _vp),
                 ("y", _vp), ("y_batch_stride", _i64), ("y_row_stride", _i64),
                 ("h_final", _vp), ("h_ckpt", _vp),
-                ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
+                ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
+                ("dt_bias", _vp), ("dt_softplus", ctypes.c_int),
+                ("dt_min", ctypes.c_float), ("dt_max", ctypes.c_float)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -64,7 +68,9 @@ class DecodeArgs(ctypes.Structure):
                 ("u", _vp), ("u_batch_stride", _i64),
                 ("conv_w", _vp), ("conv_bias", _vp), ("tail_in", _vp), ("tail_out", _vp),
                 ("dt", _vp), ("A", _vp), ("D", _vp), ("h_in", _vp), ("h_out", _vp),
-                ("y", _vp), ("y_batch_stride", _i64)]
+                ("y", _vp), ("y_batch_stride", _i64),
+                ("dt_bias", _vp), ("dt_softplus", ctypes.c_int),
+                ("dt_min", ctypes.c_float), ("dt_max", ctypes.c_float)]
 
 
 _lib = None
@@ -185,13 +191,25 @@ def conv_forward(u, w, bias=None, tail_in=None, tail_out=None, v=None, stream=No
     return v, tail_out
 
 
+
+def _set_dt(a, dt_bias, dt_softplus, dt_limit):
+    """The optional dt_bias [H] float32 / softplus / (lo, hi) clamp of the arguments."""
+    _cuda(dt_bias)
+    _f32(dt_bias, "dt_bias")
+    a.dt_bias = dt_bias.data_ptr() if dt_bias is not None else None
+    a.dt_softplus = 1 if dt_softplus else 0
+    lo, hi = dt_limit if dt_limit is not None else (0.0, 0.0)
+    a.dt_min, a.dt_max = float(lo), float(hi)
+
 def scan_forward(x, B, C, dt, A, D=None, h0=None, *, H, G=1, Q=128, s=0, y=None,
-                 h_final=None, h_ckpt=None, workspace=None, stream=None):
+                 h_final=None, h_ckpt=None, workspace=None, stream=None, dt_bias=None,
+                 dt_softplus=False, dt_limit=None):
     """Chunked selective scan; returns (y, h_final, h_ckpt).
 
     x: [b, L, >=H*P] view (may be a column slice of the conv output),
     B, C: [b, L, >=G*N] views, dt: [b, L, H] float32, A/D: [H] float32,
-    h0: [b, H, P, N] float32 or None.
+    h0: [b, H, P, N] float32 or None.  dt_bias [H] / dt_softplus / dt_limit (lo, hi):
+    the kernels use clamp(softplus(dt + dt_bias)) instead of dt (each part optional).
     """
     _cuda(x, B, C, dt, A, D, h0, y, h_final, h_ckpt, workspace)
     b, L = x.shape[0], x.shape[1]
@@ -220,13 +238,15 @@ def scan_forward(x, B, C, dt, A, D=None, h0=None, *, H, G=1, Q=128, s=0, y=None,
     a.h_final = h_final.data_ptr() if h_final is not None else None
     a.h_ckpt = h_ckpt.data_ptr() if h_ckpt is not None else None
     a.workspace = workspace.data_ptr(); a.workspace_bytes = workspace.numel() * workspace.element_size()
+    _set_dt(a, dt_bias, dt_softplus, dt_limit)
     _check(lib().ssd_scan_forward(ctypes.byref(a), _stream(stream)))
     return y, h_final, h_ckpt
 
 
 def stream_forward(u, conv_w, dt, A, D=None, *, H, P, N, G=1, Q=128, s=0, conv_bias=None,
                    tail_in=None, tail_out=None, h0=None, v=None, y=None, h_final=None,
-                   h_ckpt=None, workspace=None, stream=None):
+                   h_ckpt=None, workspace=None, stream=None, dt_bias=None, dt_softplus=False,
+                   dt_limit=None):
     """One streamed segment: conv (tail_in -> tail_out), then scan (h0 -> h_final)."""
     _cuda(u, conv_w, dt, A, D, conv_bias, tail_in, tail_out, h0, v, y, h_final, h_ckpt, workspace)
     b, L, cch = u.shape
@@ -258,12 +278,14 @@ def stream_forward(u, conv_w, dt, A, D=None, *, H, P, N, G=1, Q=128, s=0, conv_b
     a.h_final = h_final.data_ptr()
     a.h_ckpt = h_ckpt.data_ptr() if h_ckpt is not None else None
     a.workspace = workspace.data_ptr(); a.workspace_bytes = workspace.numel()
+    _set_dt(a, dt_bias, dt_softplus, dt_limit)
     _check(lib().ssd_stream_forward(ctypes.byref(a), _stream(stream)))
     return {"v": v, "y": y, "h_final": h_final, "h_ckpt": h_ckpt, "tail_out": tail_out}
 
 
 def decode_step(u, conv_w, dt, A, D=None, *, H, P, N, G=1, conv_bias=None, tail_in=None,
-                tail_out=None, h_in=None, h_out=None, y=None, stream=None):
+                tail_out=None, h_in=None, h_out=None, y=None, stream=None, dt_bias=None,
+                dt_softplus=False, dt_limit=None):
     """One token of b streams: u [b, C_ch] (pre-conv x|B|C), dt [b, H].  Returns
     {"y": [b, H, P], "h_out": [b, H, P, N], "tail_out": [b, 3, C_ch]}; h_out may be h_in
     and tail_out may be tail_in (updated in place)."""
@@ -287,5 +309,6 @@ def decode_step(u, conv_w, dt, A, D=None, *, H, P, N, G=1, conv_bias=None, tail_
     a.h_in = h_in.data_ptr() if h_in is not None else None
     a.h_out = h_out.data_ptr()
     a.y = y.data_ptr(); a.y_batch_stride = y.view(b, H * P).stride(0)
+    _set_dt(a, dt_bias, dt_softplus, dt_limit)
     _check(lib().ssd_decode_step(ctypes.byref(a), _stream(stream)))
     return {"y": y, "h_out": h_out, "tail_out": tail_out}

@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(DecodeParams p
     }
     __syncthreads();
 
-    const float dt = p.dt[(int64_t)bi * p.H + h];
+    const float dt = dt_effective(p.dt[(int64_t)bi * p.H + h], p.dt_bias, h, p.dt_softplus, p.dt_min, p.dt_max);
     const float a = exp2f(dt * p.A[h] * 1.4426950408889634f);
     const float Dh = p.D ? p.D[h] : 0.0f;
     const int64_t PN = (int64_t)p.P * p.N;

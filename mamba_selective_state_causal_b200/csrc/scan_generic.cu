@@ -20,6 +20,8 @@
 //           checkpoints that fall in the stripe (state after every s tokens,
 //           "Algorithm 1" Sckpt of pith_extraction.key_machinery) and h_final.
 // This file is the general path: any supported P, N, Q and both dtypes.
+#include <algorithm>
+
 #include "ssd_common.cuh"
 
 namespace ssd {
@@ -251,6 +253,14 @@ int launch_t(const ScanParams &p, cudaStream_t st)
     return cudaGetLastError() == cudaSuccess ? 0 : 7;
 }
 
+// dt_eff[b][L][H] = dt_effective(dt) for the scan kernels, which then read it as plain dt
+__global__ void dt_prepare_kernel(ScanParams p, float *out)
+{
+    const int64_t n = (int64_t)p.b * p.L * p.H;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        out[i] = dt_effective(p.dt[i], p.dt_bias, (int)(i % p.H), p.dt_softplus, p.dt_min, p.dt_max);
+}
+
 }  // namespace
 
 int launch_chain(const ScanParams &p, cudaStream_t st)
@@ -266,6 +276,16 @@ int launch_scan_generic(const ScanParams &p, int dtype, cudaStream_t st)
 {
     if (p.P * p.N > kThreads * kMaxEPT) return 6;
     return dtype == 1 ? launch_t<__nv_bfloat16>(p, st) : launch_t<float>(p, st);
+}
+
+int launch_dt_prepare(const ScanParams &p, float *out, cudaStream_t st)
+{
+    const int64_t n = (int64_t)p.b * p.L * p.H;
+    if (n > 0) {
+        const int64_t blocks = std::min<int64_t>((n + 255) / 256, 148 * 16);
+        dt_prepare_kernel<<<(unsigned)blocks, 256, 0, st>>>(p, out);
+    }
+    return cudaGetLastError() == cudaSuccess ? 0 : 7;
 }
 
 }  // namespace ssd

@@ -59,6 +59,9 @@ bool pow2_dim(int v) { return v == 16 || v == 32 || v == 64 || v == 128; }
 struct Plan {
     int64_t T = 0, ns = 0;
     size_t off_S = 0, off_hin = 0, off_dA = 0, bytes = 0;
+    // the dt surroundings' buffer (effective dt [b][L][H] fp32) follows the stripe states;
+    // it is needed only when a call asks for dt_bias / softplus / a clamp
+    size_t off_dt = 0, bytes_dt = 0;
 };
 
 size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -109,6 +112,8 @@ Plan make_plan(int b, int64_t L, int H, int P, int N, int Q)
         pl.off_dA = pl.off_hin + round256(state);
         pl.bytes = pl.off_dA + round256(sizeof(float) * (size_t)b * pl.ns * H);
     }
+    pl.off_dt = round256(pl.bytes);
+    pl.bytes_dt = pl.off_dt + round256(sizeof(float) * (size_t)b * L * H);
     return pl;
 }
 
@@ -159,9 +164,11 @@ int scan_impl(const ssd_scan_args *a, cudaStream_t st)
         if (!a->A) return fail(SSD_ERR_NULL, "A is NULL");
     }
     const Plan pl = make_plan(a->b, a->L, a->H, a->P, a->N, a->Q);
-    if (pl.bytes > 0) {
-        if (!a->workspace || a->workspace_bytes < pl.bytes)
-            return fail(SSD_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", pl.bytes,
+    const bool dtx = a->dt_bias || a->dt_softplus || a->dt_max > 0.0f;
+    const size_t need = dtx ? pl.bytes_dt : pl.bytes;
+    if (need > 0) {
+        if (!a->workspace || a->workspace_bytes < need)
+            return fail(SSD_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
                         a->workspace ? a->workspace_bytes : (size_t)0);
         if ((reinterpret_cast<uintptr_t>(a->workspace) & 255u) != 0)
             return fail(SSD_ERR_ALIGN, "workspace must be 256-byte aligned");
@@ -182,6 +189,7 @@ int scan_impl(const ssd_scan_args *a, cudaStream_t st)
     p.B = a->B; p.Bbs = a->B_batch_stride; p.Brs = a->B_row_stride;
     p.C = a->C; p.Cbs = a->C_batch_stride; p.Crs = a->C_row_stride;
     p.dt = a->dt; p.A = a->A; p.D = a->D; p.h0 = a->h0;
+    p.dt_bias = a->dt_bias; p.dt_softplus = a->dt_softplus; p.dt_min = a->dt_min; p.dt_max = a->dt_max;
     p.y = a->y; p.ybs = a->y_batch_stride; p.yrs = a->y_row_stride;
     p.h_final = a->h_final; p.h_ckpt = a->h_ckpt;
     p.T = pl.T; p.ns = pl.ns;
@@ -189,6 +197,14 @@ int scan_impl(const ssd_scan_args *a, cudaStream_t st)
     p.ws_S = pl.bytes ? reinterpret_cast<float *>(ws + pl.off_S) : nullptr;
     p.ws_hin = pl.bytes ? reinterpret_cast<float *>(ws + pl.off_hin) : nullptr;
     p.ws_dA = pl.bytes ? reinterpret_cast<float *>(ws + pl.off_dA) : nullptr;
+    if (dtx) {
+        // the effective dt goes to the workspace first; the scan kernels read it as plain dt
+        float *dte = reinterpret_cast<float *>(ws + pl.off_dt);
+        if (ssd::launch_dt_prepare(p, dte, st))
+            return fail(SSD_ERR_LAUNCH, "dt launch failed: %s", cudaGetErrorString(cudaGetLastError()));
+        p.dt = dte;
+        p.dt_bias = nullptr; p.dt_softplus = 0; p.dt_min = 0.0f; p.dt_max = 0.0f;
+    }
     p.status = status_ptr();
     if (!p.status) return fail(SSD_ERR_LAUNCH, "no CUDA device available");
     {
@@ -341,7 +357,7 @@ int ssd_scan_forward(const ssd_scan_args *args, ssd_stream_t stream)
 
 size_t ssd_scan_workspace_size(int b, int64_t L, int H, int P, int N, int Q)
 {
-    return make_plan(b, L, H, P, N, Q).bytes;
+    return make_plan(b, L, H, P, N, Q).bytes_dt;
 }
 
 int ssd_stream_forward(const ssd_stream_args *a, ssd_stream_t stream)
@@ -367,6 +383,7 @@ int ssd_stream_forward(const ssd_stream_args *a, ssd_stream_t stream)
     s.C = v ? v + es * (d_inner + (size_t)a->G * a->N) : nullptr;
     s.C_batch_stride = a->v_batch_stride; s.C_row_stride = a->v_row_stride;
     s.dt = a->dt; s.A = a->A; s.D = a->D; s.h0 = a->h0;
+    s.dt_bias = a->dt_bias; s.dt_softplus = a->dt_softplus; s.dt_min = a->dt_min; s.dt_max = a->dt_max;
     s.y = a->y; s.y_batch_stride = a->y_batch_stride; s.y_row_stride = a->y_row_stride;
     s.h_final = a->h_final; s.h_ckpt = a->h_ckpt;
     s.workspace = a->workspace; s.workspace_bytes = a->workspace_bytes;
@@ -398,6 +415,7 @@ int ssd_decode_step(const ssd_decode_args *a, ssd_stream_t stream)
     p.u = a->u; p.ubs = a->u_batch_stride; p.w = a->conv_w; p.bias = a->conv_bias;
     p.tail_in = a->tail_in; p.tail_out = a->tail_out; p.dt = a->dt; p.A = a->A; p.D = a->D;
     p.h_in = a->h_in; p.h_out = a->h_out; p.y = a->y; p.ybs = a->y_batch_stride;
+    p.dt_bias = a->dt_bias; p.dt_softplus = a->dt_softplus; p.dt_min = a->dt_min; p.dt_max = a->dt_max;
     const int rc = ssd::launch_decode(p, a->dtype, (cudaStream_t)stream);
     if (rc) return fail(SSD_ERR_LAUNCH, "decode launch failed: %s", cudaGetErrorString(cudaGetLastError()));
     return ok();

@@ -42,6 +42,11 @@ struct ScanParams {
     // failure-detection test hook (SSD_TEST_DROP_UNIT): the work unit whose
     // loads are never issued, so that its waits run out; -1 = none
     int64_t test_drop_unit;
+    // the dt surroundings (dt_effective): applied by a pre-pass into the workspace, so the
+    // scan kernels themselves always read plain dt
+    const float *dt_bias;
+    int dt_softplus;
+    float dt_min, dt_max;
 };
 
 struct ConvParams {
@@ -74,7 +79,23 @@ struct DecodeParams {
     float *h_out;
     void *y;
     int64_t ybs;
+    const float *dt_bias;
+    int dt_softplus;
+    float dt_min, dt_max;
 };
+
+// The step size a kernel uses for a raw dt value of head h: dt + dt_bias[h]
+// (bias optional), through softplus(v) = log(1 + e^v) when asked (v itself
+// above 20, where the two agree in fp32), clamped to [dt_min, dt_max] when
+// dt_max > 0.  With no bias, no softplus and dt_max <= 0 it is dt unchanged.
+__device__ __forceinline__ float dt_effective(float raw, const float *bias, int h, int softplus, float lo,
+                                              float hi)
+{
+    float v = bias ? raw + bias[h] : raw;
+    if (softplus) v = v > 20.0f ? v : log1pf(__expf(v));
+    if (hi > 0.0f) v = fminf(fmaxf(v, lo), hi);
+    return v;
+}
 
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
@@ -111,6 +132,7 @@ void prof_end(cudaStream_t st, int id);
 int launch_conv(const ConvParams &p, int dtype, cudaStream_t st);
 int launch_decode(const DecodeParams &p, int dtype, cudaStream_t st);
 int launch_scan_generic(const ScanParams &p, int dtype, cudaStream_t st);
+int launch_dt_prepare(const ScanParams &p, float *out, cudaStream_t st);
 bool tc_scan_supported(const ScanParams &p, int dtype);
 int launch_scan_tc(const ScanParams &p, cudaStream_t st);
 }  // namespace ssd

@@ -159,6 +159,21 @@ def scan(x, B, C, dt, A, D=None, h0=None, s=0, heads=None, H=None, P=None, G=1,
     return {"y": y, "h_final": h_final, "h_ckpt": h_ckpt}
 
 
+def dt_effective(dt, dt_bias=None, softplus=False, dt_min=0.0, dt_max=0.0):
+    """The step size from a raw dt, fp64: v = dt + dt_bias[h] (bias optional),
+    then softplus(v) = log(1 + e^v) when asked, then clamped to [dt_min, dt_max]
+    when dt_max > 0.  These are the Mamba-2 block's dt surroundings, which the
+    pages leave out (they give dt itself); dt is [..., H]."""
+    v = np.asarray(dt, dtype=np.float64)
+    if dt_bias is not None:
+        v = v + np.asarray(dt_bias, dtype=np.float64)
+    if softplus:
+        v = np.logaddexp(0.0, v)
+    if dt_max > 0:
+        v = np.clip(v, dt_min, dt_max)
+    return v
+
+
 def layer(u, w, dt, A, D=None, bias=None, tail_in=None, h0=None, H=None, P=None, N=None,
           G=1, s=0, io_round="none", heads=None, want_ckpt=True):
     """conv1d+SiLU on the packed x|B|C stream, then the recurrence.

@@ -95,6 +95,15 @@ def make_params(wl: Workload, device="cpu", seed=None):
     return {"A": A, "D": D, "w": w, "bias": bias, "dt_bias": dt_bias}
 
 
+def make_dt_raw(wl: Workload, L=None, b=None, device="cpu", seed=None):
+    """The raw draws z ~ N(0, 0.5^2) [b, L, H] fp32 that make_dt turns into dt
+    (for the entry points that take dt before its bias and softplus)."""
+    L = wl.L if L is None else L
+    b = wl.b if b is None else b
+    g = _gen((wl.seed if seed is None else seed) + 1000, device)
+    return torch.randn(b, L, wl.H, device=device, dtype=torch.float32, generator=g) * 0.5
+
+
 def make_dt(wl: Workload, dt_bias, L=None, b=None, device="cpu", seed=None):
     """dt [b, L, H] fp32 > 0 from the softplus recipe."""
     L = wl.L if L is None else L

@@ -61,16 +61,16 @@ def _plan_bytes(b, L, H, P, N, Q, nsm=148):
         if best is None or cost < best[0]:
             best = (cost, tc)
     ns = -(-L // (best[1] * Q))
-    if ns <= 1:
-        return 0
     r = lambda v: (v + 255) // 256 * 256
-    state = 4 * b * ns * H * P * N
-    return 2 * r(state) + r(4 * b * ns * H)
+    stripes = 0 if ns <= 1 else 2 * r(4 * b * ns * H * P * N) + r(4 * b * ns * H)
+    # followed by room for the effective dt [b][L][H] fp32 (used when dt_bias / softplus / a clamp is asked)
+    return r(stripes) + r(4 * b * L * H)
 
 
 def test_plan_fills_whole_waves():
     """The 0.3B 131072-token segment: 9 stripes x 16 head pairs = 144 CTAs, one wave of 148 SMs."""
-    assert _plan_bytes(1, 131072, 32, 64, 128, 128) == 2 * 4 * 9 * 32 * 64 * 128 + 9 * 32 * 4 + 256 - (9 * 32 * 4) % 256
+    stripes = 2 * 4 * 9 * 32 * 64 * 128 + 9 * 32 * 4 + 256 - (9 * 32 * 4) % 256
+    assert _plan_bytes(1, 131072, 32, 64, 128, 128) == stripes + 4 * 131072 * 32
 
 
 @pytest.mark.parametrize("shape", [(1, 16384, 32, 64, 128, 128), (1, 131072, 32, 64, 128, 128),
