@@ -209,6 +209,14 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
             ++issued;
         };
         const uint32_t id_s = idesc_bf16(128, 128, 1, 1);   // A = B^T (MN-major), B = w o X (MN-major)
+        // descriptors of each stage's B^T and w o X, built once; a K-step adds 2048 B (128 units)
+        uint64_t dB[kStagesA], dXw[kStagesA];
+#pragma unroll
+        for (int i = 0; i < kStagesA; ++i) {
+            const uint32_t sb = smem_u32(s.stage[i]);
+            dB[i] = smem_desc(sb, kBox, 1024);
+            dXw[i] = smem_desc(sb + 2 * kBox, kBox, 1024);
+        }
         bool ok = live;
         int mmas = 0;
         if (ok && lane == 0)
@@ -219,11 +227,11 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
             if (!ok) break;
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t sB = smem_u32(s.stage[st]), sXw = sB + 2 * kBox;
+                const uint64_t db = st == 0 ? dB[0] : (st == 1 ? dB[1] : dB[2]);
+                const uint64_t dx = st == 0 ? dXw[0] : (st == 1 ? dXw[1] : dXw[2]);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tS, smem_desc(sB + kk * 2048, kBox, 1024), smem_desc(sXw + kk * 2048, kBox, 1024), id_s,
-                           it > 0 || kk > 0);
+                    mma_ss(tS, db + (uint64_t)(kk * 128), dx + (uint64_t)(kk * 128), id_s, it > 0 || kk > 0);
                 mma_commit(&s.empty[st]);
             }
             ++mmas;
@@ -735,14 +743,24 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
             ++x_issued;
         };
         // G = C B^T of chunk c into the TMEM columns at tG (its B/C slot has landed)
+        // shared-memory descriptors of every operand tile, built once per slot: a K-step only adds
+        // a constant to the start-address field (in 16-byte units; addresses stay below 256 KB)
+        const uint32_t bc0 = smem_u32(s.bc[0]), bc1 = smem_u32(s.bc[1]);
+        const uint32_t x0 = smem_u32(s.x[0]), x1 = smem_u32(s.x[1]);
+        const uint64_t dC0 = smem_desc(bc0, 16, 1024), dC1 = smem_desc(bc1, 16, 1024);   // C, K-major
+        const uint64_t dBk0 = smem_desc(bc0 + 2 * kBox, 16, 1024), dBk1 = smem_desc(bc1 + 2 * kBox, 16, 1024);  // B, K-major
+        const uint64_t dBt0 = smem_desc(bc0 + 2 * kBox, kBox, 1024), dBt1 = smem_desc(bc1 + 2 * kBox, kBox, 1024);  // B^T, MN-major
+        const uint64_t dX0 = smem_desc(x0, 0, 1024), dX1 = smem_desc(x1, 0, 1024);           // X of one head, MN-major, N = 64
+        const uint64_t dXw0 = smem_desc(x0, kBox, 1024), dXw1 = smem_desc(x1, kBox, 1024);    // w o X of both heads, N = 128
+        const uint64_t dHp = smem_desc(smem_u32(s.hp), kBox, 1024);                          // hp of both heads, N = 128
+        constexpr uint64_t kBoxD = kBox >> 4;
+        auto koff = [](int kk) -> uint64_t { return (uint64_t)((kk >> 2) * kBoxD + (kk & 3) * 2); };  // K-major K-step
+        auto moff = [](int kk) -> uint64_t { return (uint64_t)(kk * 128); };                          // MN-major K-step
         auto issue_g = [&](int c, uint32_t tG) {
-            const uint32_t sC = smem_u32(s.bc[c & 1]), sB = sC + 2 * kBox;
+            const uint64_t dc = (c & 1) ? dC1 : dC0, db = (c & 1) ? dBk1 : dBk0;
             const uint32_t id_g = idesc_bf16(128, 128, 0, 0);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-                mma_ss(tG, smem_desc(sC + off, 16, 1024), smem_desc(sB + off, 16, 1024), id_g, kk > 0);
-            }
+            for (int kk = 0; kk < 8; ++kk) mma_ss(tG, dc + koff(kk), db + koff(kk), id_g, kk > 0);
             mma_commit(&s.g_done);
         };
         const uint32_t id_pm = idesc_bf16(128, 64, 0, 1);     // A = Pm (TMEM), B = X (MN-major)
@@ -775,19 +793,13 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
             tc_fence_after();
             if (lane == 0) {
                 ++x_waited;
-                const uint32_t sX = smem_u32(xs);
+                const uint64_t dx = (c & 1) ? dX1 : dX0, dc = (c & 1) ? dC1 : dC0;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tY, tPm + kk * 8, smem_desc(sX + kk * 2048, 0, 1024), id_pm, kk > 0);
+                for (int kk = 0; kk < 8; ++kk) mma_ts(tY, tPm + kk * 8, dx + moff(kk), id_pm, kk > 0);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tY + 64, tPm + 64 + kk * 8, smem_desc(sX + kBox + kk * 2048, 0, 1024), id_pm, kk > 0);
-                const uint32_t sC = smem_u32(s.bc[c & 1]), sHp = smem_u32(s.hp);
+                for (int kk = 0; kk < 8; ++kk) mma_ts(tY + 64, tPm + 64 + kk * 8, dx + kBoxD + moff(kk), id_pm, kk > 0);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-                    mma_ss(tG, smem_desc(sC + off, 16, 1024), smem_desc(sHp + kk * 2048, kBox, 1024), id_ys, kk > 0);
-                }
+                for (int kk = 0; kk < 8; ++kk) mma_ss(tG, dc + koff(kk), dHp + moff(kk), id_ys, kk > 0);
             }
             __syncwarp();
             // w o X of both heads: S = B^T [Xw_a | Xw_b] accumulates into H
@@ -795,10 +807,9 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
             if (!ok) break;
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t sB = smem_u32(s.bc[c & 1]) + 2 * kBox, sXw = smem_u32(s.x[(c + 1) & 1]);
+                const uint64_t dbt = (c & 1) ? dBt1 : dBt0, dxw = (c & 1) ? dXw0 : dXw1;   // w o X is in slot (c+1) & 1
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tH, smem_desc(sB + kk * 2048, kBox, 1024), smem_desc(sXw + kk * 2048, kBox, 1024), id_s, true);
+                for (int kk = 0; kk < 8; ++kk) mma_ss(tH, dbt + moff(kk), dxw + moff(kk), id_s, true);
                 mma_commit(&s.mma_done);
             }
             __syncwarp();
