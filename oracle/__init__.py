@@ -31,6 +31,12 @@ def _bind(path):
                                 f32p, f32p, f32p, f64p, i32p, ctypes.c_int,
                                 f64p, f64p, f64p]
     lib.oracle_scan.restype = None
+    lib.oracle_scan_backward.argtypes = [ctypes.c_int, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_int, i64,
+                                         f32p, i64, i64, f32p, i64, i64, f32p, i64, i64,
+                                         f32p, f32p, f32p, f64p, f64p, f64p, f64p,
+                                         f64p, f64p, f64p, f64p, f64p, f64p, f64p]
+    lib.oracle_scan_backward.restype = None
     lib.oracle_round_bf16.argtypes = [ctypes.c_double]
     lib.oracle_round_bf16.restype = ctypes.c_double
     lib.oracle_num_threads.argtypes = []
@@ -157,6 +163,69 @@ def scan(x, B, C, dt, A, D=None, h0=None, s=0, heads=None, H=None, P=None, G=1,
                     None if hsel is None else hsel.ctypes.data_as(ctypes.POINTER(ctypes.c_int)),
                     nh, _p64(y), _p64(h_final), _p64(h_ckpt))
     return {"y": y, "h_final": h_final, "h_ckpt": h_ckpt}
+
+
+def scan_backward(x, B, C, dt, A, D, dy, h0=None, h_ckpt=None, dh_final=None, s=0, H=None, P=None, G=1):
+    """Gradients of the recurrence, fp64, by its literal reverse mode.
+
+    Shapes as in ``scan`` (all heads); dy: [b, L, H, P] and dh_final:
+    [b, H, P, N] (or None) are the loss's gradients with respect to y and
+    h_final.  With ``h_ckpt`` ([b, L//s, H, P, N], the forward's checkpoints)
+    and s > 0, each cell of s tokens is recomputed from its checkpoint;
+    without it, the states come from one pass over the whole sequence.
+    Returns dict dx [b, L, H, P], dB and dC [b, L, G, N] (summed over the
+    heads of each group), ddt [b, L, H], dA and dD [H] (summed over b),
+    dh0 [b, H, P, N], and the per-head dB_h, dC_h [b, L, H, N].
+    """
+    lib = _load()
+    x, B, C = np.asarray(x), np.asarray(B), np.asarray(C)
+    b, L = x.shape[0], x.shape[1]
+    dt = _f32(dt)
+    H = dt.shape[2] if H is None else H
+    N = B.shape[2] // G
+    if P is None:
+        P = x.shape[2] // H
+    A = _f32(A)
+    D = _f32(D)
+
+    def strided(a):
+        a = _f32(a)
+        return a, a.shape[1] * a.shape[2], a.shape[2]
+
+    def f64(a, shape):
+        if a is None:
+            return None
+        a = np.ascontiguousarray(a, dtype=np.float64)
+        assert a.shape == shape, (a.shape, shape)
+        return a
+
+    x, xbs, xrs = strided(x)
+    B, Bbs, Brs = strided(B)
+    C, Cbs, Crs = strided(C)
+    h0 = f64(h0, (b, H, P, N))
+    n_ckpt = L // s if s > 0 else 0
+    h_ckpt = f64(h_ckpt, (b, n_ckpt, H, P, N))
+    dy = f64(dy, (b, L, H, P))
+    dh_final = f64(dh_final, (b, H, P, N))
+    dx = np.empty((b, L, H, P))
+    dB_h = np.empty((b, L, H, N))
+    dC_h = np.empty((b, L, H, N))
+    ddt = np.empty((b, L, H))
+    dA_b = np.empty((b, H))
+    dD_b = np.empty((b, H))
+    dh0 = np.empty((b, H, P, N))
+    lib.oracle_scan_backward(b, L, H, P, N, G, int(s), _p32(x), xbs, xrs, _p32(B), Bbs, Brs,
+                             _p32(C), Cbs, Crs, _p32(dt), _p32(A), _p32(D), _p64(h0), _p64(h_ckpt),
+                             _p64(dy), _p64(dh_final), _p64(dx), _p64(dB_h), _p64(dC_h), _p64(ddt),
+                             _p64(dA_b), _p64(dD_b), _p64(dh0))
+    grp = (np.arange(H) * G) // H
+    dB = np.zeros((b, L, G, N))
+    dC = np.zeros((b, L, G, N))
+    for h in range(H):
+        dB[:, :, grp[h]] += dB_h[:, :, h]
+        dC[:, :, grp[h]] += dC_h[:, :, h]
+    return {"dx": dx, "dB": dB, "dC": dC, "ddt": ddt, "dA": dA_b.sum(0), "dD": dD_b.sum(0),
+            "dh0": dh0, "dB_h": dB_h, "dC_h": dC_h}
 
 
 def dt_effective(dt, dt_bias=None, softplus=False, dt_min=0.0, dt_max=0.0):

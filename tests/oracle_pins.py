@@ -308,7 +308,122 @@ def pin_resume_needs_conv_tail():
     assert _rel(bad["y"], full["y"][:, m:]) > 1e-4
 
 
+def _scan_loss(x, B, C, dt, A, D, h0, dy, dhf, H, P, G):
+    """The scalar sum(dy * y) + sum(dhf * h_final) through the forward oracle."""
+    out = oracle.scan(x, B, C, dt, A, D, h0, s=0, H=H, P=P, G=G, want_ckpt=False)
+    return float(np.sum(out["y"] * dy) + np.sum(out["h_final"] * dhf))
+
+
+def _fd_grad(f, arr, rel_step=None, abs_step=2.0 ** -5):
+    """Central differences of f with respect to every element of arr.
+
+    float32 inputs are perturbed in float32 and divided by the step actually
+    taken.  With rel_step the step scales with the element and the estimate is
+    Richardson-extrapolated (error O(step^4)); without it the step is fixed,
+    which is exact for inputs the loss is linear in.
+    """
+    g = np.zeros(arr.shape)
+    for i in range(arr.size):
+        def diff(step):
+            up, dn = arr.copy(), arr.copy()
+            up.flat[i] = arr.flat[i] + step
+            dn.flat[i] = arr.flat[i] - step
+            width = float(up.flat[i]) - float(dn.flat[i])
+            return (f(up) - f(dn)) / width
+        if rel_step is None:
+            g.flat[i] = diff(abs_step)
+        else:
+            st = rel_step * abs(float(arr.flat[i]))
+            g.flat[i] = (4.0 * diff(st / 2) - diff(st)) / 3.0
+    return g
+
+
+def pin_backward_finite_differences():
+    """Every gradient of the reverse mode against central differences of the forward."""
+    rng = RNG(30)
+    b, L, H, P, N, G = 2, 7, 4, 2, 2, 2
+    x, B, C, dt, A, D, h0 = _inputs(rng, b, L, H, P, N, G=G, dt_range=(0.05, 0.4))
+    dy = rng.standard_normal((b, L, H, P))
+    dhf = rng.standard_normal((b, H, P, N))
+    args = dict(x=x, B=B, C=C, dt=dt, A=A, D=D, h0=h0)
+    bw = oracle.scan_backward(x, B, C, dt, A, D, dy, h0=h0, dh_final=dhf, H=H, P=P, G=G)
+
+    def loss_wrt(name):
+        def f(v):
+            kw = dict(args)
+            kw[name] = v
+            return _scan_loss(kw["x"], kw["B"], kw["C"], kw["dt"], kw["A"], kw["D"], kw["h0"],
+                              dy, dhf, H, P, G)
+        return f
+
+    # the loss is linear in x, B, C, D and h0: fixed steps give exact differences
+    for name, key in [("x", "dx"), ("B", "dB"), ("C", "dC"), ("D", "dD"), ("h0", "dh0")]:
+        fd = _fd_grad(loss_wrt(name), args[name])
+        got = bw[key]
+        if name == "x":
+            got = got.reshape(b, L, H * P)
+        elif name in ("B", "C"):
+            got = got.reshape(b, L, G * N)
+        assert _rel(got, fd) < 1e-9, (name, _rel(got, fd))
+    for name, key in [("dt", "ddt"), ("A", "dA")]:
+        fd = _fd_grad(loss_wrt(name), args[name], rel_step=1e-2)
+        assert _rel(bw[key], fd) < 1e-7, (name, _rel(bw[key], fd))
+
+
+def pin_backward_cells_equal_full():
+    """Recomputing each cell from its checkpoint gives bitwise the gradients of
+    one pass that keeps every state, including a ragged last cell."""
+    rng = RNG(31)
+    b, L, H, P, N, s = 2, 37, 2, 3, 4, 8
+    x, B, C, dt, A, D, h0 = _inputs(rng, b, L, H, P, N)
+    dy = rng.standard_normal((b, L, H, P))
+    dhf = rng.standard_normal((b, H, P, N))
+    fwd = oracle.scan(x, B, C, dt, A, D, h0, s=s)
+    full = oracle.scan_backward(x, B, C, dt, A, D, dy, h0=h0, dh_final=dhf)
+    cells = oracle.scan_backward(x, B, C, dt, A, D, dy, h0=h0, h_ckpt=fwd["h_ckpt"], dh_final=dhf, s=s)
+    for k in full:
+        assert np.array_equal(full[k], cells[k]), k
+
+
+def pin_backward_without_input():
+    """B = 0 leaves h_t = exp(A cumsum(dt)) h0, whose gradients have closed forms."""
+    rng = RNG(32)
+    b, L, H, P, N = 2, 11, 2, 3, 4
+    x, B, C, dt, A, D, h0 = _inputs(rng, b, L, H, P, N)
+    B = np.zeros_like(B)
+    dy = rng.standard_normal((b, L, H, P))
+    dhf = rng.standard_normal((b, H, P, N))
+    bw = oracle.scan_backward(x, B, C, dt, A, D, dy, h0=h0, dh_final=dhf)
+    xh = x.reshape(b, L, H, P).astype(np.float64)
+    assert np.array_equal(bw["dx"], D.astype(np.float64)[None, None, :, None] * dy)
+    assert abs(bw["dD"] - np.einsum("blhp,blhp->h", dy, xh)).max() < 1e-12 * np.abs(dy).sum()
+    Cd = C.astype(np.float64)
+    dC = np.zeros((b, L, N))
+    dh0 = np.zeros((b, H, P, N))
+    ddt = np.zeros((b, L, H))
+    dA = np.zeros(H)
+    for bi in range(b):
+        for h in range(H):
+            cum = np.cumsum(dt[bi, :, h].astype(np.float64))
+            e = np.exp(float(A[h]) * cum)
+            # r_t = dLoss/d(decay_t) for the factor e_t that multiplies h0 in h_t
+            r = np.array([dy[bi, t, h] @ h0[bi, h] @ Cd[bi, t] for t in range(L)])
+            r[-1] += np.sum(dhf[bi, h] * h0[bi, h])
+            for t in range(L):
+                dC[bi, t] += e[t] * (dy[bi, t, h] @ h0[bi, h])
+                dh0[bi, h] += e[t] * np.outer(dy[bi, t, h], Cd[bi, t])
+            dh0[bi, h] += e[-1] * dhf[bi, h]
+            re = r * e
+            ddt[bi, :, h] = float(A[h]) * np.cumsum(re[::-1])[::-1]
+            dA[h] += np.sum(cum * re)
+    assert _rel(bw["dC"][:, :, 0], dC) < 1e-12
+    assert _rel(bw["dh0"], dh0) < 1e-12
+    assert _rel(bw["ddt"], ddt) < 1e-12
+    assert _rel(bw["dA"], dA) < 1e-12
+
+
 PINS = [pin_quadratic_form, pin_A_zero_prefix_sum, pin_constant_geometric, pin_skip_only,
         pin_single_impulse, pin_linearity, pin_conv_torch, pin_conv_delta_weights,
         pin_bf16_rounding, pin_ckpt_indexing, pin_split_resume_bitwise,
-        pin_resume_needs_conv_tail]
+        pin_resume_needs_conv_tail, pin_backward_finite_differences, pin_backward_cells_equal_full,
+        pin_backward_without_input]
