@@ -52,6 +52,9 @@ def parse_args():
     # the decode step instead of the headline step: this many independent streams of the
     # 0.3B shape, each advancing one token per step (its own JSON line)
     ap.add_argument("--decode-streams", type=int, default=0)
+    # the backward pass of the scan instead of the headline step: gradients from the
+    # forward's checkpoints, on the 0.3B 16384-token workload (its own JSON line)
+    ap.add_argument("--backward", action="store_true")
     return ap.parse_args()
 
 
@@ -437,6 +440,85 @@ def run_decode(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+# fp32 FMA issue of the CUDA cores: 148 SMs x 128 lanes x 2 flops x 1.965 GHz (max SM clock)
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def bwd_flops_per_chunk_head(P, N, Q=64):
+    """Multiply-add flops of one (64-token chunk, head) in the backward kernels:
+    summaries S and Gl (2 x 2QPN); gradients: C.B and dy.x (2Q^2 N + 2Q^2 P),
+    dx (2Q^2 P + 2QNP), dB (2Q^2 N + 2QPN), dC (2QPN + 2Q^2 N)."""
+    summary = 2 * 2 * Q * P * N
+    grad = Q * Q * (6 * N + 4 * P) + 6 * Q * P * N
+    return summary, grad
+
+
+def run_backward(args, world, rank, local):
+    """Gradients through the scan from the forward's checkpoints (cell recompute), timed
+    with CUDA events like the headline step; the forward runs once, before the timing."""
+    import __graft_entry__
+    __graft_entry__.build()
+    import mamba_selective_state_causal_b200 as ssd
+    wl = ssd_synth.BY_NAME["mamba2-0.3b-L16k"]
+    d = torch.device("cuda", torch.cuda.current_device())
+    seed = rank_seed(wl, rank)
+    prm = ssd_synth.make_params(wl, device=d, seed=seed)
+    dt = ssd_synth.make_dt(wl, prm["dt_bias"], device=d, seed=seed)
+    x, Bm, Cm = ssd_synth.make_xbc(wl, device=d, seed=seed)
+    dy, dhf = ssd_synth.make_grads(wl, device=d, seed=seed)
+    _, _, ck = ssd.scan_forward(x, Bm, Cm, dt, prm["A"], prm["D"], H=wl.H, Q=wl.Q, s=wl.s)
+    ws = torch.empty(ssd.backward_workspace_size(wl.b, wl.L, wl.H, wl.P, wl.N), dtype=torch.uint8, device=d)
+    out = {"dx": torch.empty(wl.b, wl.L, wl.H, wl.P, device=d), "dB": torch.empty(wl.b, wl.L, wl.G, wl.N, device=d),
+           "dC": torch.empty(wl.b, wl.L, wl.G, wl.N, device=d), "ddt": torch.empty(wl.b, wl.L, wl.H, device=d),
+           "dA": torch.empty(wl.H, device=d), "dD": torch.empty(wl.H, device=d),
+           "dh0": torch.empty(wl.b, wl.H, wl.P, wl.N, device=d)}
+
+    def step():
+        ssd.scan_backward(x, Bm, Cm, dt, prm["A"], prm["D"], dy, h_ckpt=ck, dh_final=dhf, H=wl.H, G=wl.G,
+                          s=wl.s, workspace=ws, out=out)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    ms = time_steps(step, args.steps, args.warmup, world, local)
+    clk = clocks.stop()
+    ssd.sync_status()
+    ms = max_over_ranks(world, ms)
+    ssd.profile_begin()
+    prof_steps = min(args.steps, 5)
+    for _ in range(prof_steps):
+        step()
+    torch.cuda.synchronize()
+    prof = ssd.profile_end()
+    per_launch = {k: v["total_ms"] / v["launches"] for k, v in prof.items()}
+    nch = -(-wl.L // 64)
+    f_sum, f_grad = bwd_flops_per_chunk_head(wl.P, wl.N)
+    grad_flops = f_grad * nch * wl.H * wl.b
+    achieved = grad_flops / (per_launch["bwd_chunk_grad"] / 1e3) / 1e12
+    step_flops = (f_sum + f_grad) * nch * wl.H * wl.b
+    line = {
+        "metric": "SSD scan backward tokens/s (0.3B shape, L=16384, cells recomputed from checkpoints)",
+        "value": wl.tokens * world * args.steps / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": wl.name + "-backward", "batch": wl.b, "seq_len": wl.L, "heads": wl.H,
+                   "headdim": wl.P, "d_state": wl.N, "ckpt_stride": wl.s, "io_dtype": wl.dtype,
+                   "l2": "workspace and outputs larger than L2 (%.1f GB)" % (ws.numel() / 1e9)},
+        "roofline": {"bound": "alu", "kernel": "bwd_chunk_grad", "achieved": achieved, "peak": FP32_ALU_TFLOPS,
+                     "unit": "TFLOP/s", "frac": achieved / FP32_ALU_TFLOPS,
+                     "peak_source": "derived: 148 SMs x 128 fp32 FMA lanes x 2 x 1.965 GHz", "traffic": None,
+                     "algorithmic_flops_per_launch": grad_flops},
+        "step_flops": step_flops,
+        "kernels": {k: {"launches_per_step": v["launches"] / prof_steps, "ms_per_launch": per_launch[k]}
+                    for k, v in prof.items()},
+        # per step: summary, two chains, gradients, two reductions
+        "gpu_launches": 6 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     wl = ssd_synth.BY_NAME[args.workload]
@@ -449,6 +531,9 @@ def main():
         return
     if args.decode_streams > 0:
         run_decode(args, world, rank, local)
+        return
+    if args.backward:
+        run_backward(args, world, rank, local)
         return
     import __graft_entry__
     __graft_entry__.build()

@@ -253,6 +253,65 @@ typedef struct ssd_decode_args {
 SSD_API int ssd_decode_step(const ssd_decode_args *args, ssd_stream_t stream);
 
 /*
+ * Arguments of the backward pass of the scan (see ssd_scan_backward).
+ *   dtype, b, L, H, P, N, G, x, B, C, dt, A, D, h0: as given to the forward
+ *           call whose gradients are wanted (dt is the step size the scan
+ *           used; x, B, C laid out and aligned as for ssd_scan_forward).
+ *   h_ckpt  [b][floor(L/s)][H][P][N] float: that call's checkpoints, s their
+ *           stride (a multiple of 64).  Or NULL (s ignored): the states are
+ *           then rebuilt from h0 over the whole sequence.
+ *   dy      element (bi,t,h,p) at dy[bi*dy_batch_stride + t*dy_row_stride + h*P + p],
+ *           I/O dtype, 16-byte aligned rows: dLoss/dy.
+ *   dh_final [b][H][P][N] float or NULL (zero): dLoss/dh_final.
+ * Outputs, float, contiguous, every element written:
+ *   dx [b][L][H][P]; dB, dC [b][L][G][N] (summed over the heads of each
+ *   group); ddt [b][L][H]; dA [H]; dD [H] or NULL (both summed over the batch
+ *   rows); dh0 [b][H][P][N] or NULL.  They must not overlap the inputs.
+ *   workspace: at least ssd_scan_backward_workspace_size() bytes, 256-byte
+ *   aligned; contents on entry are ignored.
+ */
+typedef struct ssd_scan_bwd_args {
+    int dtype;
+    int b;
+    int64_t L;
+    int H, P, N, G;
+    int64_t s;
+    const void *x;
+    int64_t x_batch_stride, x_row_stride;
+    const void *B;
+    int64_t B_batch_stride, B_row_stride;
+    const void *C;
+    int64_t C_batch_stride, C_row_stride;
+    const float *dt;
+    const float *A;
+    const float *D;
+    const float *h0;
+    const float *h_ckpt;
+    const void *dy;
+    int64_t dy_batch_stride, dy_row_stride;
+    const float *dh_final;
+    float *dx, *dB, *dC, *ddt, *dA, *dD, *dh0;
+    void *workspace;
+    size_t workspace_bytes;
+} ssd_scan_bwd_args;
+
+/*
+ * ssd_scan_backward -- gradients of a scalar loss through the scan, given
+ * dLoss/dy and dLoss/dh_final: the reverse mode of the recurrence at the top
+ * of this header.  With checkpoints, the states of each cell of s tokens are
+ * rebuilt from the checkpoint that starts it (h0 for the first cell), and no
+ * state is carried across cells: the grid-cell recompute of MA-GC
+ * (pith_extraction.key_machinery, "Algorithm 1") on the sequence axis, whose
+ * gradients must match plain backpropagation (skeptic_critique.concrete_test).
+ * All arithmetic is fp32 on CUDA cores.  Asynchronous on `stream`.
+ */
+SSD_API int ssd_scan_backward(const ssd_scan_bwd_args *args, ssd_stream_t stream);
+
+/* Bytes of workspace ssd_scan_backward needs: per 64-token chunk and head two
+ * P x N fp32 states, and per token and head two N-vectors of fp32. */
+SSD_API size_t ssd_scan_backward_workspace_size(int b, int64_t L, int H, int P, int N);
+
+/*
  * ssd_scan_forward_static_scratch -- ssd_scan_forward for callers that cannot
  * allocate device memory.  (The pages have no counterpart: this is a
  * deployment aid of this library, not part of the layer they describe.)

@@ -73,6 +73,21 @@ class DecodeArgs(ctypes.Structure):
                 ("dt_min", ctypes.c_float), ("dt_max", ctypes.c_float)]
 
 
+class ScanBwdArgs(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int), ("b", ctypes.c_int), ("L", _i64),
+                ("H", ctypes.c_int), ("P", ctypes.c_int), ("N", ctypes.c_int),
+                ("G", ctypes.c_int), ("s", _i64),
+                ("x", _vp), ("x_batch_stride", _i64), ("x_row_stride", _i64),
+                ("B", _vp), ("B_batch_stride", _i64), ("B_row_stride", _i64),
+                ("C", _vp), ("C_batch_stride", _i64), ("C_row_stride", _i64),
+                ("dt", _vp), ("A", _vp), ("D", _vp), ("h0", _vp), ("h_ckpt", _vp),
+                ("dy", _vp), ("dy_batch_stride", _i64), ("dy_row_stride", _i64),
+                ("dh_final", _vp),
+                ("dx", _vp), ("dB", _vp), ("dC", _vp), ("ddt", _vp), ("dA", _vp), ("dD", _vp),
+                ("dh0", _vp),
+                ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
+
+
 _lib = None
 
 
@@ -93,6 +108,11 @@ def lib():
         L.ssd_stream_forward.restype = ctypes.c_int
         L.ssd_decode_step.argtypes = [ctypes.POINTER(DecodeArgs), _vp]
         L.ssd_decode_step.restype = ctypes.c_int
+        L.ssd_scan_backward.argtypes = [ctypes.POINTER(ScanBwdArgs), _vp]
+        L.ssd_scan_backward.restype = ctypes.c_int
+        L.ssd_scan_backward_workspace_size.argtypes = [ctypes.c_int, _i64, ctypes.c_int, ctypes.c_int,
+                                                       ctypes.c_int]
+        L.ssd_scan_backward_workspace_size.restype = ctypes.c_size_t
         L.ssd_scan_workspace_size.argtypes = [ctypes.c_int, _i64, ctypes.c_int, ctypes.c_int,
                                               ctypes.c_int, ctypes.c_int]
         L.ssd_scan_workspace_size.restype = ctypes.c_size_t
@@ -312,3 +332,54 @@ def decode_step(u, conv_w, dt, A, D=None, *, H, P, N, G=1, conv_bias=None, tail_
     _set_dt(a, dt_bias, dt_softplus, dt_limit)
     _check(lib().ssd_decode_step(ctypes.byref(a), _stream(stream)))
     return {"y": y, "h_out": h_out, "tail_out": tail_out}
+
+
+def backward_workspace_size(b, L, H, P, N):
+    return int(lib().ssd_scan_backward_workspace_size(b, L, H, P, N))
+
+
+def scan_backward(x, B, C, dt, A, D, dy, h0=None, h_ckpt=None, dh_final=None, *, H, G=1, s=0,
+                  workspace=None, out=None, stream=None):
+    """Gradients through scan_forward: returns dict dx, dB, dC, ddt, dA, dD, dh0 (float32).
+
+    x, B, C, dt, A, D, h0: the forward's inputs (views as for scan_forward);
+    dy: [b, L, >=H*P] (I/O dtype) = dLoss/dy, dh_final: [b, H, P, N] float32
+    or None.  h_ckpt: the forward's checkpoints [b, L//s, H, P, N] with stride
+    s, or None to rebuild the states from h0 over the whole sequence.
+    ``out`` may hold preallocated outputs under the same keys.
+    """
+    _cuda(x, B, C, dt, A, D, dy, h0, h_ckpt, dh_final, workspace)
+    b, L = x.shape[0], x.shape[1]
+    P = x.shape[2] // H
+    N = B.shape[2] // G
+    dev = x.device
+    o = dict(out or {})
+    shapes = {"dx": (b, L, H, P), "dB": (b, L, G, N), "dC": (b, L, G, N), "ddt": (b, L, H),
+              "dA": (H,), "dD": (H,), "dh0": (b, H, P, N)}
+    for k, shp in shapes.items():
+        if k not in o:
+            o[k] = torch.empty(shp, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(backward_workspace_size(b, L, H, P, N), 1), dtype=torch.uint8, device=dev)
+    for t, n in ((dt, "dt"), (A, "A"), (D, "D"), (h0, "h0"), (h_ckpt, "h_ckpt"), (dh_final, "dh_final"),
+                 *((o[k], k) for k in shapes)):
+        _f32(t, n)
+    a = ScanBwdArgs()
+    a.dtype = _dtype_code(x); a.b = b; a.L = L; a.H = H; a.P = P; a.N = N; a.G = G
+    a.s = s if h_ckpt is not None else 0
+    a.x = x.data_ptr(); a.x_batch_stride = x.stride(0); a.x_row_stride = x.stride(1)
+    a.B = B.data_ptr(); a.B_batch_stride = B.stride(0); a.B_row_stride = B.stride(1)
+    a.C = C.data_ptr(); a.C_batch_stride = C.stride(0); a.C_row_stride = C.stride(1)
+    a.dt = dt.data_ptr(); a.A = A.data_ptr(); a.D = D.data_ptr() if D is not None else None
+    a.h0 = h0.data_ptr() if h0 is not None else None
+    a.h_ckpt = h_ckpt.data_ptr() if h_ckpt is not None else None
+    dy3 = dy.reshape(b, L, -1) if dy.dim() == 4 else dy
+    a.dy = dy3.data_ptr(); a.dy_batch_stride = dy3.stride(0); a.dy_row_stride = dy3.stride(1)
+    a.dh_final = dh_final.data_ptr() if dh_final is not None else None
+    a.dx = o["dx"].data_ptr(); a.dB = o["dB"].data_ptr(); a.dC = o["dC"].data_ptr()
+    a.ddt = o["ddt"].data_ptr(); a.dA = o["dA"].data_ptr()
+    a.dD = o["dD"].data_ptr() if o["dD"] is not None else None
+    a.dh0 = o["dh0"].data_ptr() if o["dh0"] is not None else None
+    a.workspace = workspace.data_ptr(); a.workspace_bytes = workspace.numel()
+    _check(lib().ssd_scan_backward(ctypes.byref(a), _stream(stream)))
+    return o

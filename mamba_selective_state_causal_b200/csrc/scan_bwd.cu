@@ -1,0 +1,578 @@
+// scan_bwd.cu -- gradients of the selective scan, recomputing each cell of s
+// tokens from its checkpoint (CUDA cores, fp32 math).
+//
+// The layer is the recurrence h_t = a_t h_{t-1} + dt_t x_t B_t^T,
+// y_t = C_t^T h_t + D x_t with a_t = exp(dt_t A) (pith.science verdict for
+// arXiv 2411.19460, pith_extraction.core_discovery, Eq. (1)).  Its
+// checkpoints h_ckpt[k] (state after (k+1)s tokens, "Algorithm 1" Sckpt of
+// pith_extraction.key_machinery) let the backward pass rebuild the states of
+// one cell at a time instead of keeping all of them: that is the grid-cell
+// recompute of MA-GC on the sequence axis.
+//
+// Given dy = dLoss/dy and dh_final, the adjoint g_t = dLoss/dh_t obeys
+// g_t = dy_t C_t^T + a_{t+1} g_{t+1}.  Everything is organised in chunks of
+// kQb = 64 tokens with chunk-local inclusive log-decay cs_i = sum_{k<=i} dt_k A
+// and lam = cs_last; with h_prev the state entering the chunk and Gam the
+// adjoint arriving at its last token from later tokens (dh_final for the last
+// chunk):
+//   dx_j   = D dy_j + dt_j [ sum_{t>=j} e^{cs_t-cs_j} (C_t.B_j) dy_t + e^{lam-cs_j} Gam B_j ]
+//   dBr_j  = sum_{t>=j} e^{cs_t-cs_j} (dy_t.x_j) C_t + e^{lam-cs_j} x_j^T Gam,   dB_j = dt_j dBr_j
+//   dC_t   = e^{cs_t} dy_t^T h_prev + sum_{j<=t} e^{cs_t-cs_j} dt_j (dy_t.x_j) B_j
+//   dl_t   = dLoss/d(dt_t A) = <g_t, a_t h_{t-1}>
+//          = sum_{t'>=t} al_t' + sum_{t'>=t} sum_{j<t} K[t'][j] + e^{lam} <Gam, h_prev> + sum_{j<t} be_j
+//     with al_t = e^{cs_t} dy_t^T h_prev C_t,  K[t][j] = e^{cs_t-cs_j} dt_j (dy_t.x_j)(C_t.B_j),
+//          be_j = e^{lam-cs_j} dt_j x_j^T Gam B_j
+//   ddt_t  = A dl_t + B_t . dBr_t,   dA = sum_t dt_t dl_t,   dD = sum_t dy_t . x_t
+// (the last line because d/d(dt_t) of the input term dt_t x_t B_t^T gives
+// <g_t, x_t B_t^T> = B_t . dBr_t).  The chunk-entry states and adjoints come
+// from two chains over per-chunk summaries:
+//   S_c   = sum_j dt_j e^{lam-cs_j} x_j B_j^T,        h_prev[c+1] = e^{lam_c} h_prev[c] + S_c
+//   Gl_c  = sum_t e^{cs_t} dy_t C_t^T,                Gam[c-1]    = e^{lam_c} Gam[c] + Gl_c
+// The state chain restarts at every cell from its checkpoint (h0 for the
+// first), so no state is carried further than one cell; the adjoint chain
+// runs over the whole sequence, last chunk first, and ends in dh0.
+// Only non-positive differences of cs are exponentiated.
+#include <algorithm>
+
+#include "ssd_common.cuh"
+
+namespace ssd {
+namespace {
+
+constexpr int kQb = 64;           // tokens per backward chunk
+constexpr int kBwdThreads = 256;
+constexpr int kQ1 = kQb + 1;      // padded row of the chunk x chunk matrices
+
+template <typename T>
+__device__ __forceinline__ void load_rows(float *dst, int dst_rs, const T *src, int64_t src_rs, int rows_valid,
+                                          int cols)
+{
+    for (int i = threadIdx.x; i < kQb * cols; i += blockDim.x) {
+        const int r = i / cols, col = i % cols;
+        dst[r * dst_rs + col] = r < rows_valid ? to_f32<T>(src[(int64_t)r * src_rs + col]) : 0.0f;
+    }
+}
+
+// acc[r][c] += sum_k a[(r0 + r) * ars + k * acs] * b[k * brs + (c0 + c) * bcs]
+__device__ __forceinline__ void mm4x4(float (&acc)[4][4], const float *a, int ars, int acs, const float *b, int brs,
+                                      int bcs, int K, int r0, int c0)
+{
+    for (int k = 0; k < K; ++k) {
+        float av[4], bv[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) av[r] = a[(r0 + r) * ars + k * acs];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) bv[c] = b[(int64_t)k * brs + (int64_t)(c0 + c) * bcs];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
+    }
+}
+
+__device__ __forceinline__ void zero4x4(float (&acc)[4][4])
+{
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[r][c] = 0.0f;
+}
+
+// chunk-local inclusive cumsum of dt*A (serial, deterministic)
+__device__ __forceinline__ void chunk_cumsum(const float *dts, float *cum, float A)
+{
+    if (threadIdx.x == 0) {
+        float acc = 0.0f;
+        for (int i = 0; i < kQb; ++i) { acc = fmaf(dts[i], A, acc); cum[i] = acc; }
+    }
+}
+
+// ---------------------------------------------------------------- summaries
+// One CTA per (chunk, head, batch row): S_c, Gl_c and lam_c.
+template <typename T>
+__global__ void __launch_bounds__(kBwdThreads) bwd_chunk_summary_kernel(BwdParams p)
+{
+    extern __shared__ float sm[];
+    const int c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
+    const int P = p.P, N = p.N, P1 = P + 1, N1 = N + 1;
+    const int g = (int)((int64_t)h * p.G / p.H);
+    const int64_t t0 = (int64_t)c * kQb;
+    const int rows = (int)(p.L - t0 < kQb ? p.L - t0 : kQb);
+    float *xs = sm;                 // [Qb][P1]  dt_j e^{lam-cs_j} x_j
+    float *gs = xs + kQb * P1;      // [Qb][P1]  e^{cs_t} dy_t
+    float *bs = gs + kQb * P1;      // [Qb][N1]
+    float *cs = bs + kQb * N1;      // [Qb][N1]
+    float *dts = cs + kQb * N1;     // [Qb]
+    float *cum = dts + kQb;         // [Qb]
+    float *wx = cum + kQb;          // [Qb]
+    float *wg = wx + kQb;           // [Qb]
+
+    load_rows(xs, P1, reinterpret_cast<const T *>(p.x) + bi * p.xbs + t0 * p.xrs + (int64_t)h * P, p.xrs, rows, P);
+    load_rows(gs, P1, reinterpret_cast<const T *>(p.dy) + bi * p.dybs + t0 * p.dyrs + (int64_t)h * P, p.dyrs, rows,
+              P);
+    load_rows(bs, N1, reinterpret_cast<const T *>(p.B) + bi * p.Bbs + t0 * p.Brs + (int64_t)g * N, p.Brs, rows, N);
+    load_rows(cs, N1, reinterpret_cast<const T *>(p.C) + bi * p.Cbs + t0 * p.Crs + (int64_t)g * N, p.Crs, rows, N);
+    for (int i = threadIdx.x; i < kQb; i += blockDim.x)
+        dts[i] = i < rows ? p.dt[((int64_t)bi * p.L + t0 + i) * p.H + h] : 0.0f;
+    __syncthreads();
+    chunk_cumsum(dts, cum, p.A[h]);
+    __syncthreads();
+    const float lam = cum[kQb - 1];
+    for (int i = threadIdx.x; i < kQb; i += blockDim.x) {
+        wx[i] = dts[i] * expf(lam - cum[i]);
+        wg[i] = expf(cum[i]);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < kQb * P; i += blockDim.x) {
+        const int r = i / P, col = i % P;
+        xs[r * P1 + col] *= wx[r];
+        gs[r * P1 + col] *= wg[r];
+    }
+    const int64_t unit = ((int64_t)bi * p.H + h) * p.nch + c;
+    if (threadIdx.x == 0) p.ws_lam[unit] = lam;
+    __syncthreads();
+
+    float *S = p.ws_h + unit * P * N;
+    float *Gl = p.ws_g + unit * P * N;
+    const int ct = N / 4;
+    for (int tile = threadIdx.x; tile < (P / 4) * ct; tile += blockDim.x) {
+        const int p0 = (tile / ct) * 4, n0 = (tile % ct) * 4;
+        float acc[4][4];
+        zero4x4(acc);
+        mm4x4(acc, xs, 1, P1, bs, N1, 1, kQb, p0, n0);
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+            *reinterpret_cast<float4 *>(S + (int64_t)(p0 + r) * N + n0) =
+                make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+        zero4x4(acc);
+        mm4x4(acc, gs, 1, P1, cs, N1, 1, kQb, p0, n0);
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+            *reinterpret_cast<float4 *>(Gl + (int64_t)(p0 + r) * N + n0) =
+                make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+    }
+}
+
+// ---------------------------------------------------------------- chains
+__device__ __forceinline__ float4 f4_fma(float a, float4 x, float4 y)
+{
+    return make_float4(fmaf(a, x.x, y.x), fmaf(a, x.y, y.y), fmaf(a, x.z, y.z), fmaf(a, x.w, y.w));
+}
+
+constexpr int kChainAhead = 8;    // chunk summaries loaded ahead of the chain
+
+// State entering every chunk, per cell: h = start of the cell (h0 or the
+// checkpoint before it); for each chunk c of the cell: slot c := h, then
+// h = e^{lam_c} h + S_c (the slot held S_c).  Grid: (slices * cells, H, b);
+// a thread carries 4 consecutive state elements.
+__global__ void __launch_bounds__(kBwdThreads) bwd_state_chain_kernel(BwdParams p)
+{
+    const int64_t PN = (int64_t)p.P * p.N;
+    const int slices = (int)((PN + 4 * kBwdThreads - 1) / (4 * kBwdThreads));
+    const int sl = blockIdx.x % slices;
+    const int64_t k = blockIdx.x / slices;
+    const int h = blockIdx.y, bi = blockIdx.z;
+    const int64_t e = (int64_t)sl * 4 * kBwdThreads + 4 * threadIdx.x;
+    if (e >= PN) return;
+    const int64_t hu = (int64_t)bi * p.H + h;
+    float4 hv = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (k == 0) {
+        if (p.h0) hv = *reinterpret_cast<const float4 *>(p.h0 + hu * PN + e);
+    } else {
+        hv = *reinterpret_cast<const float4 *>(p.h_ckpt + (((int64_t)bi * p.n_ckpt + (k - 1)) * p.H + h) * PN + e);
+    }
+    const int64_t c0 = k * p.cell_chunks;
+    const int64_t c1 = p.nch < c0 + p.cell_chunks ? p.nch : c0 + p.cell_chunks;
+    float *base = p.ws_h + hu * p.nch * PN + e;
+    const float *lam = p.ws_lam + hu * p.nch;
+    for (int64_t cb = c0; cb < c1; cb += kChainAhead) {
+        float4 sv[kChainAhead];
+        float lv[kChainAhead];
+#pragma unroll
+        for (int i = 0; i < kChainAhead; ++i) {
+            const bool in = cb + i < c1;
+            sv[i] = in ? *reinterpret_cast<const float4 *>(base + (cb + i) * PN) : make_float4(0.f, 0.f, 0.f, 0.f);
+            lv[i] = in ? lam[cb + i] : 0.0f;
+        }
+#pragma unroll
+        for (int i = 0; i < kChainAhead; ++i) {
+            if (cb + i < c1) {
+                *reinterpret_cast<float4 *>(base + (cb + i) * PN) = hv;
+                hv = f4_fma(expf(lv[i]), hv, sv[i]);
+            }
+        }
+    }
+}
+
+// Adjoint arriving at the last token of every chunk, over the whole
+// sequence, last chunk first: G = dh_final; for c = nch-1 .. 0: slot c := G,
+// then G = e^{lam_c} G + Gl_c (the slot held Gl_c).  dh0 = G at the end.
+// Grid: (slices, H, b).
+__global__ void __launch_bounds__(kBwdThreads) bwd_adjoint_chain_kernel(BwdParams p)
+{
+    const int64_t PN = (int64_t)p.P * p.N;
+    const int sl = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
+    const int64_t e = (int64_t)sl * 4 * kBwdThreads + 4 * threadIdx.x;
+    if (e >= PN) return;
+    const int64_t hu = (int64_t)bi * p.H + h;
+    float4 gv = p.dh_final ? *reinterpret_cast<const float4 *>(p.dh_final + hu * PN + e)
+                           : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    float *base = p.ws_g + hu * p.nch * PN + e;
+    const float *lam = p.ws_lam + hu * p.nch;
+    for (int64_t cb = p.nch - 1; cb >= 0; cb -= kChainAhead) {
+        float4 sv[kChainAhead];
+        float lv[kChainAhead];
+#pragma unroll
+        for (int i = 0; i < kChainAhead; ++i) {
+            const bool in = cb - i >= 0;
+            sv[i] = in ? *reinterpret_cast<const float4 *>(base + (cb - i) * PN) : make_float4(0.f, 0.f, 0.f, 0.f);
+            lv[i] = in ? lam[cb - i] : 0.0f;
+        }
+#pragma unroll
+        for (int i = 0; i < kChainAhead; ++i) {
+            if (cb - i >= 0) {
+                *reinterpret_cast<float4 *>(base + (cb - i) * PN) = gv;
+                gv = f4_fma(expf(lv[i]), gv, sv[i]);
+            }
+        }
+    }
+    if (p.dh0) *reinterpret_cast<float4 *>(p.dh0 + hu * PN + e) = gv;
+}
+
+// ---------------------------------------------------------------- gradients
+// One CTA per (chunk, head, batch row).
+template <typename T>
+__global__ void __launch_bounds__(kBwdThreads) bwd_chunk_grad_kernel(BwdParams p)
+{
+    extern __shared__ float sm[];
+    const int c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
+    const int P = p.P, N = p.N, P1 = P + 1, N1 = N + 1;
+    const int g = (int)((int64_t)h * p.G / p.H);
+    const int64_t t0 = (int64_t)c * kQb;
+    const int rows = (int)(p.L - t0 < kQb ? p.L - t0 : kQb);
+    const int tid = threadIdx.x;
+    float *xs = sm;                  // [Qb][P1]
+    float *gs = xs + kQb * P1;       // [Qb][P1] dy
+    float *bs = gs + kQb * P1;       // [Qb][N1]
+    float *cs = bs + kQb * N1;       // [Qb][N1]
+    float *CB = cs + kQb * N1;       // [Qb][Q1] C_t.B_j, then masked and decayed
+    float *GX = CB + kQb * kQ1;      // [Qb][Q1] dy_t.x_j, then masked and decayed
+    float *KK = GX + kQb * kQ1;      // [Qb][Q1] K, then its row prefix sums, then GX * dt_j
+    float *dts = KK + kQb * kQ1;     // [Qb]
+    float *cum = dts + kQb;
+    float *ecs = cum + kQb;          // e^{cs_t}
+    float *eend = ecs + kQb;         // e^{lam - cs_j}
+    float *al = eend + kQb;          // al_t
+    float *be = al + kQb;            // be_j
+    float *din = be + kQb;           // B_t . dBr_t
+    float *rr = din + kQb;           // sum_{t'>=t} sum_{j<t} K[t'][j]
+    float *red = rr + kQb;           // [2][Qb][32] row partials over column tiles
+    float *misc = red + 2 * kQb * 32;   // [kBwdThreads / 32]
+
+    const int64_t hu = (int64_t)bi * p.H + h;
+    const int64_t unit = hu * p.nch + c;
+    const float *hprev = p.ws_h + unit * P * N;
+    const float *Gam = p.ws_g + unit * P * N;
+    const float Ah = p.A[h];
+    const float Dh = p.D ? p.D[h] : 0.0f;
+
+    load_rows(xs, P1, reinterpret_cast<const T *>(p.x) + bi * p.xbs + t0 * p.xrs + (int64_t)h * P, p.xrs, rows, P);
+    load_rows(gs, P1, reinterpret_cast<const T *>(p.dy) + bi * p.dybs + t0 * p.dyrs + (int64_t)h * P, p.dyrs, rows,
+              P);
+    load_rows(bs, N1, reinterpret_cast<const T *>(p.B) + bi * p.Bbs + t0 * p.Brs + (int64_t)g * N, p.Brs, rows, N);
+    load_rows(cs, N1, reinterpret_cast<const T *>(p.C) + bi * p.Cbs + t0 * p.Crs + (int64_t)g * N, p.Crs, rows, N);
+    for (int i = tid; i < kQb; i += blockDim.x) dts[i] = i < rows ? p.dt[((int64_t)bi * p.L + t0 + i) * p.H + h] : 0.0f;
+    __syncthreads();
+    chunk_cumsum(dts, cum, Ah);
+    // <Gam, h_prev>, reduced in a fixed order
+    float part = 0.0f;
+    for (int64_t i = tid; i < (int64_t)P * N; i += blockDim.x) part = fmaf(Gam[i], hprev[i], part);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if ((tid & 31) == 0) misc[tid >> 5] = part;
+    __syncthreads();
+    const float lam = cum[kQb - 1];
+    for (int i = tid; i < kQb; i += blockDim.x) {
+        ecs[i] = expf(cum[i]);
+        eend[i] = expf(lam - cum[i]);
+    }
+    // CB[t][j] = C_t . B_j and GX[t][j] = dy_t . x_j, all t, j
+    for (int tile = tid; tile < (kQb / 4) * (kQb / 4); tile += blockDim.x) {
+        const int r0 = (tile / (kQb / 4)) * 4, c0 = (tile % (kQb / 4)) * 4;
+        float acc[4][4];
+        zero4x4(acc);
+        mm4x4(acc, cs, N1, 1, bs, 1, N1, N, r0, c0);
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) CB[(r0 + r) * kQ1 + c0 + q] = acc[r][q];
+        zero4x4(acc);
+        mm4x4(acc, gs, P1, 1, xs, 1, P1, P, r0, c0);
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) GX[(r0 + r) * kQ1 + c0 + q] = acc[r][q];
+    }
+    __syncthreads();
+    float gam_h = 0.0f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) gam_h += misc[w];
+    const float term3 = expf(lam) * gam_h;
+    // K (strictly below the diagonal), then CB and GX masked and decayed in place
+    for (int i = tid; i < kQb * kQb; i += blockDim.x) {
+        const int t = i / kQb, j = i % kQb;
+        float kv = 0.0f, cb = 0.0f, gx = 0.0f;
+        if (j <= t) {
+            const float seg = expf(cum[t] - cum[j]);
+            cb = seg * CB[t * kQ1 + j];
+            gx = seg * GX[t * kQ1 + j];
+            if (j < t) kv = gx * dts[j] * CB[t * kQ1 + j];
+        }
+        KK[t * kQ1 + j] = kv;
+        CB[t * kQ1 + j] = cb;
+        GX[t * kQ1 + j] = gx;
+    }
+    __syncthreads();
+    // dD of this chunk: the diagonal of GX (decay 1 there)
+    if (tid == kQb) {
+        float sD = 0.0f;
+        for (int t = 0; t < kQb; ++t) sD += GX[t * kQ1 + t];
+        p.ws_pD[unit] = sD;
+    }
+    // row-exclusive prefix sums of K: KK[t][u] := sum_{j<u} K[t][j]
+    if (tid < kQb) {
+        float run = 0.0f;
+        for (int u = 0; u < kQb; ++u) {
+            const float v = KK[tid * kQ1 + u];
+            KK[tid * kQ1 + u] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+    if (tid < kQb) {
+        float s = 0.0f;
+        for (int t = tid; t < kQb; ++t) s += KK[t * kQ1 + tid];
+        rr[tid] = s;
+    }
+    __syncthreads();
+    // KK := GX * dt_j, the weights of dC's intra-chunk term
+    for (int i = tid; i < kQb * kQb; i += blockDim.x) {
+        const int t = i / kQb, j = i % kQb;
+        KK[t * kQ1 + j] = GX[t * kQ1 + j] * dts[j];
+    }
+
+    // dx[j][p] = D dy_j + dt_j (sum_t CB[t][j] dy_t[p] + eend_j sum_n Gam[p][n] B_j[n])
+    float *dx = p.dx + ((int64_t)bi * p.L + t0) * p.H * P + (int64_t)h * P;
+    {
+        const int ct = P / 4;
+        for (int tile = tid; tile < (kQb / 4) * ct; tile += blockDim.x) {
+            const int j0 = (tile / ct) * 4, p0 = (tile % ct) * 4;
+            float a1[4][4], a2[4][4];
+            zero4x4(a1);
+            zero4x4(a2);
+            mm4x4(a1, CB, 1, kQ1, gs, P1, 1, kQb, j0, p0);
+            mm4x4(a2, bs, N1, 1, Gam, 1, N, N, j0, p0);
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int j = j0 + r;
+                if (j < rows) {
+                    float o[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        o[q] = fmaf(Dh, gs[j * P1 + p0 + q], dts[j] * fmaf(eend[j], a2[r][q], a1[r][q]));
+                    *reinterpret_cast<float4 *>(dx + (int64_t)j * p.H * P + p0) = make_float4(o[0], o[1], o[2], o[3]);
+                }
+            }
+        }
+    }
+    __syncthreads();   // KK complete before dC reads it
+
+    // dBr[j][n] = sum_t GX[t][j] C_t[n] + eend_j sum_p x_j[p] Gam[p][n]
+    float *dBh = p.ws_dBh + (((int64_t)bi * p.L + t0) * p.H + h) * N;
+    float *dCh = p.ws_dCh + (((int64_t)bi * p.L + t0) * p.H + h) * N;
+    const int ctn = N / 4;
+    for (int tile = tid; tile < (kQb / 4) * ctn; tile += blockDim.x) {
+        const int j0 = (tile / ctn) * 4, n0 = (tile % ctn) * 4, nt = tile % ctn;
+        float a1[4][4], a2[4][4];
+        zero4x4(a1);
+        zero4x4(a2);
+        mm4x4(a1, GX, 1, kQ1, cs, N1, 1, kQb, j0, n0);
+        mm4x4(a2, xs, P1, 1, Gam, N, 1, P, j0, n0);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int j = j0 + r;
+            float o[4], sin = 0.0f, sbe = 0.0f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float br = fmaf(eend[j], a2[r][q], a1[r][q]);
+                const float bv = bs[j * N1 + n0 + q];
+                sin = fmaf(bv, br, sin);
+                sbe = fmaf(bv, a2[r][q], sbe);
+                o[q] = dts[j] * br;
+            }
+            red[j * 32 + nt] = sin;
+            red[kQb * 32 + j * 32 + nt] = sbe;
+            if (j < rows)
+                *reinterpret_cast<float4 *>(dBh + (int64_t)j * p.H * N + n0) = make_float4(o[0], o[1], o[2], o[3]);
+        }
+    }
+    __syncthreads();
+    if (tid < kQb) {
+        float s1 = 0.0f, s2 = 0.0f;
+        for (int q = 0; q < ctn; ++q) {
+            s1 += red[tid * 32 + q];
+            s2 += red[kQb * 32 + tid * 32 + q];
+        }
+        din[tid] = s1;
+        be[tid] = eend[tid] * dts[tid] * s2;
+    }
+    __syncthreads();
+
+    // dC[t][n] = ecs_t sum_p dy_t[p] h_prev[p][n] + sum_j GX[t][j] dt_j B_j[n]
+    for (int tile = tid; tile < (kQb / 4) * ctn; tile += blockDim.x) {
+        const int r0 = (tile / ctn) * 4, n0 = (tile % ctn) * 4, nt = tile % ctn;
+        float a1[4][4], a2[4][4];
+        zero4x4(a1);
+        zero4x4(a2);
+        mm4x4(a1, gs, P1, 1, hprev, N, 1, P, r0, n0);
+        mm4x4(a2, KK, kQ1, 1, bs, N1, 1, kQb, r0, n0);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int t = r0 + r;
+            float o[4], sal = 0.0f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                sal = fmaf(a1[r][q], cs[t * N1 + n0 + q], sal);
+                o[q] = fmaf(ecs[t], a1[r][q], a2[r][q]);
+            }
+            red[t * 32 + nt] = sal;
+            if (t < rows)
+                *reinterpret_cast<float4 *>(dCh + (int64_t)t * p.H * N + n0) = make_float4(o[0], o[1], o[2], o[3]);
+        }
+    }
+    __syncthreads();
+    if (tid < kQb) {
+        float s = 0.0f;
+        for (int q = 0; q < ctn; ++q) s += red[tid * 32 + q];
+        al[tid] = ecs[tid] * s;
+    }
+    __syncthreads();
+
+    // dl_t, ddt_t, and this chunk's share of dA
+    if (tid < kQb) {
+        const int t = tid;
+        float suf = 0.0f, pre = 0.0f;
+        for (int u = t; u < kQb; ++u) suf += al[u];
+        for (int j = 0; j < t; ++j) pre += be[j];
+        const float dl = suf + rr[t] + term3 + pre;
+        if (t < rows) p.ddt[((int64_t)bi * p.L + t0 + t) * p.H + h] = fmaf(Ah, dl, din[t]);
+        misc[t] = dts[t] * dl;     // misc is free again (gam_h was read before)
+    }
+    __syncthreads();
+    if (tid == 0) {
+        float sA = 0.0f;
+        for (int t = 0; t < kQb; ++t) sA += misc[t];
+        p.ws_pA[unit] = sA;
+    }
+}
+
+// dB, dC: sum of the per-head partials over the heads of each group;
+// one thread per (batch row, token, group, n).
+__global__ void bwd_group_sum_kernel(BwdParams p)
+{
+    const int64_t total = (int64_t)p.b * p.L * p.G * p.N;
+    const int hpg = p.H / p.G;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int n = (int)(i % p.N);
+        const int64_t r = i / p.N;
+        const int g = (int)(r % p.G);
+        const int64_t bt = r / p.G;            // bi * L + t
+        const float *sb = p.ws_dBh + (bt * p.H + (int64_t)g * hpg) * p.N + n;
+        const float *sc = p.ws_dCh + (bt * p.H + (int64_t)g * hpg) * p.N + n;
+        float ab = 0.0f, ac = 0.0f;
+        for (int k = 0; k < hpg; ++k) {
+            ab += sb[(int64_t)k * p.N];
+            ac += sc[(int64_t)k * p.N];
+        }
+        p.dB[i] = ab;
+        p.dC[i] = ac;
+    }
+}
+
+// dA[h], dD[h]: sums of the per-(batch row, chunk) partials, in a fixed order.
+__global__ void __launch_bounds__(kBwdThreads) bwd_param_sum_kernel(BwdParams p)
+{
+    __shared__ float sa[kBwdThreads], sd[kBwdThreads];
+    const int h = blockIdx.x;
+    float a = 0.0f, d = 0.0f;
+    for (int64_t i = threadIdx.x; i < (int64_t)p.b * p.nch; i += blockDim.x) {
+        const int64_t bi = i / p.nch, c = i % p.nch;
+        const int64_t unit = (bi * p.H + h) * p.nch + c;
+        a += p.ws_pA[unit];
+        d += p.ws_pD[unit];
+    }
+    sa[threadIdx.x] = a;
+    sd[threadIdx.x] = d;
+    __syncthreads();
+    for (int o = kBwdThreads / 2; o > 0; o >>= 1) {
+        if ((int)threadIdx.x < o) {
+            sa[threadIdx.x] += sa[threadIdx.x + o];
+            sd[threadIdx.x] += sd[threadIdx.x + o];
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        p.dA[h] = sa[0];
+        if (p.dD) p.dD[h] = sd[0];
+    }
+}
+
+size_t summary_smem(int P, int N) { return sizeof(float) * ((size_t)2 * kQb * (P + 1) + 2 * kQb * (N + 1) + 4 * kQb); }
+
+size_t grad_smem(int P, int N)
+{
+    return sizeof(float) * ((size_t)2 * kQb * (P + 1) + 2 * kQb * (N + 1) + 3 * kQb * kQ1 + 9 * kQb + 2 * kQb * 32 +
+                            kBwdThreads / 32 + kQb);
+}
+
+template <typename T>
+int launch_bwd_t(const BwdParams &p, cudaStream_t st)
+{
+    const size_t s1 = summary_smem(p.P, p.N), s2 = grad_smem(p.P, p.N);
+    if (cudaFuncSetAttribute(bwd_chunk_summary_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(bwd_chunk_grad_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2) !=
+            cudaSuccess)
+        return 7;
+    const dim3 grid((unsigned)p.nch, (unsigned)p.H, (unsigned)p.b);
+    prof_begin(st, kKBwdSummary);
+    bwd_chunk_summary_kernel<T><<<grid, kBwdThreads, s1, st>>>(p);
+    prof_end(st, kKBwdSummary);
+    const int64_t PN = (int64_t)p.P * p.N;
+    const unsigned slices = (unsigned)((PN + 4 * kBwdThreads - 1) / (4 * kBwdThreads));
+    const int64_t cells = (p.nch + p.cell_chunks - 1) / p.cell_chunks;
+    prof_begin(st, kKBwdChain);
+    bwd_state_chain_kernel<<<dim3(slices * (unsigned)cells, (unsigned)p.H, (unsigned)p.b), kBwdThreads, 0, st>>>(p);
+    bwd_adjoint_chain_kernel<<<dim3(slices, (unsigned)p.H, (unsigned)p.b), kBwdThreads, 0, st>>>(p);
+    prof_end(st, kKBwdChain);
+    prof_begin(st, kKBwdGrad);
+    bwd_chunk_grad_kernel<T><<<grid, kBwdThreads, s2, st>>>(p);
+    prof_end(st, kKBwdGrad);
+    prof_begin(st, kKBwdReduce);
+    const int64_t total = (int64_t)p.b * p.L * p.G * p.N;
+    const unsigned blocks = (unsigned)std::min<int64_t>((total + 255) / 256, 148 * 16);
+    bwd_group_sum_kernel<<<blocks, 256, 0, st>>>(p);
+    bwd_param_sum_kernel<<<(unsigned)p.H, kBwdThreads, 0, st>>>(p);
+    prof_end(st, kKBwdReduce);
+    return cudaGetLastError() == cudaSuccess ? 0 : 7;
+}
+
+}  // namespace
+
+size_t bwd_grad_smem_bytes(int P, int N) { return grad_smem(P, N); }
+
+int launch_scan_backward(const BwdParams &p, int dtype, cudaStream_t st)
+{
+    return dtype == 1 ? launch_bwd_t<__nv_bfloat16>(p, st) : launch_bwd_t<float>(p, st);
+}
+
+}  // namespace ssd

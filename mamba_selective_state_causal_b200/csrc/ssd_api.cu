@@ -225,6 +225,102 @@ int scan_impl(const ssd_scan_args *a, cudaStream_t st)
     return ok();
 }
 
+// Backward workspace: ws_h, ws_g [b][H][nch][P][N]; ws_lam, ws_pA, ws_pD [b][H][nch];
+// ws_dBh, ws_dCh [b][L][H][N] (all fp32, each part 256-byte aligned).
+struct BwdPlan {
+    int64_t nch = 0;
+    size_t off_h = 0, off_g = 0, off_lam = 0, off_pA = 0, off_pD = 0, off_dB = 0, off_dC = 0, bytes = 0;
+};
+
+BwdPlan make_bwd_plan(int b, int64_t L, int H, int P, int N)
+{
+    BwdPlan pl;
+    if (b <= 0 || L <= 0 || H <= 0 || P <= 0 || N <= 0) return pl;
+    pl.nch = (L + 63) / 64;
+    const size_t states = sizeof(float) * (size_t)b * H * pl.nch * P * N;
+    const size_t per_chunk = sizeof(float) * (size_t)b * H * pl.nch;
+    const size_t per_token = sizeof(float) * (size_t)b * L * H * N;
+    pl.off_h = 0;
+    pl.off_g = round256(states);
+    pl.off_lam = pl.off_g + round256(states);
+    pl.off_pA = pl.off_lam + round256(per_chunk);
+    pl.off_pD = pl.off_pA + round256(per_chunk);
+    pl.off_dB = pl.off_pD + round256(per_chunk);
+    pl.off_dC = pl.off_dB + round256(per_token);
+    pl.bytes = pl.off_dC + round256(per_token);
+    return pl;
+}
+
+int scan_bwd_impl(const ssd_scan_bwd_args *a, cudaStream_t st)
+{
+    if (!a) return fail(SSD_ERR_NULL, "args is NULL");
+    const bool ck = a->h_ckpt != nullptr;
+    int rc = check_scan_shape(a->dtype, a->b, a->L, a->H, a->P, a->N, a->G, 64, ck ? a->s : 0);
+    if (rc) return rc;
+    if (ck && a->s <= 0) return fail(SSD_ERR_SHAPE, "h_ckpt given with checkpoint stride s=%lld", (long long)a->s);
+    if (a->b == 0) return ok();
+    const size_t state_bytes = sizeof(float) * (size_t)a->b * a->H * a->P * a->N;
+    if (!a->dA) return fail(SSD_ERR_NULL, "dA is NULL");
+    if (a->L == 0) {
+        // no token: dh0 = dh_final, every parameter gradient is zero
+        cudaError_t e = cudaMemsetAsync(a->dA, 0, sizeof(float) * a->H, st);
+        if (e == cudaSuccess && a->dD) e = cudaMemsetAsync(a->dD, 0, sizeof(float) * a->H, st);
+        if (e == cudaSuccess && a->dh0)
+            e = a->dh_final ? cudaMemcpyAsync(a->dh0, a->dh_final, state_bytes, cudaMemcpyDeviceToDevice, st)
+                            : cudaMemsetAsync(a->dh0, 0, state_bytes, st);
+        if (e != cudaSuccess) return fail(SSD_ERR_LAUNCH, "%s", cudaGetErrorString(e));
+        return ok();
+    }
+    if ((rc = check_rows("x", a->x, a->x_batch_stride, a->x_row_stride, (int64_t)a->H * a->P, a->b, a->L, a->dtype, true))) return rc;
+    if ((rc = check_rows("B", a->B, a->B_batch_stride, a->B_row_stride, (int64_t)a->G * a->N, a->b, a->L, a->dtype, true))) return rc;
+    if ((rc = check_rows("C", a->C, a->C_batch_stride, a->C_row_stride, (int64_t)a->G * a->N, a->b, a->L, a->dtype, true))) return rc;
+    if ((rc = check_rows("dy", a->dy, a->dy_batch_stride, a->dy_row_stride, (int64_t)a->H * a->P, a->b, a->L, a->dtype, true))) return rc;
+    if (!a->dt || !a->A) return fail(SSD_ERR_NULL, "dt and A must not be NULL");
+    if (!a->dx || !a->dB || !a->dC || !a->ddt) return fail(SSD_ERR_NULL, "dx, dB, dC and ddt must not be NULL");
+    const void *vec[] = {a->h0, a->h_ckpt, a->dh_final, a->dx, a->dB, a->dC, a->dh0};
+    for (const void *v : vec)
+        if (v && !aligned16(v)) return fail(SSD_ERR_ALIGN, "states and gradient outputs must be 16-byte aligned");
+    const BwdPlan pl = make_bwd_plan(a->b, a->L, a->H, a->P, a->N);
+    if (!a->workspace || a->workspace_bytes < pl.bytes)
+        return fail(SSD_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", pl.bytes,
+                    a->workspace ? a->workspace_bytes : (size_t)0);
+    if ((reinterpret_cast<uintptr_t>(a->workspace) & 255u) != 0)
+        return fail(SSD_ERR_ALIGN, "workspace must be 256-byte aligned");
+    int dev = 0, smem_optin = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        return fail(SSD_ERR_LAUNCH, "no CUDA device available");
+    if (ssd::bwd_grad_smem_bytes(a->P, a->N) > (size_t)smem_optin)
+        return fail(SSD_ERR_UNSUPPORTED, "backward needs %zu bytes of shared memory, the device has %d",
+                    ssd::bwd_grad_smem_bytes(a->P, a->N), smem_optin);
+    ssd::BwdParams p{};
+    p.b = a->b; p.L = a->L; p.H = a->H; p.P = a->P; p.N = a->N; p.G = a->G;
+    p.s = ck ? a->s : 0;
+    p.n_ckpt = ck ? a->L / a->s : 0;
+    p.nch = pl.nch;
+    p.cell_chunks = ck ? a->s / 64 : pl.nch;
+    p.x = a->x; p.xbs = a->x_batch_stride; p.xrs = a->x_row_stride;
+    p.B = a->B; p.Bbs = a->B_batch_stride; p.Brs = a->B_row_stride;
+    p.C = a->C; p.Cbs = a->C_batch_stride; p.Crs = a->C_row_stride;
+    p.dy = a->dy; p.dybs = a->dy_batch_stride; p.dyrs = a->dy_row_stride;
+    p.dt = a->dt; p.A = a->A; p.D = a->D; p.h0 = a->h0; p.h_ckpt = a->h_ckpt; p.dh_final = a->dh_final;
+    p.dx = a->dx; p.dB = a->dB; p.dC = a->dC; p.ddt = a->ddt; p.dA = a->dA; p.dD = a->dD; p.dh0 = a->dh0;
+    char *ws = static_cast<char *>(a->workspace);
+    p.ws_h = reinterpret_cast<float *>(ws + pl.off_h);
+    p.ws_g = reinterpret_cast<float *>(ws + pl.off_g);
+    p.ws_lam = reinterpret_cast<float *>(ws + pl.off_lam);
+    p.ws_pA = reinterpret_cast<float *>(ws + pl.off_pA);
+    p.ws_pD = reinterpret_cast<float *>(ws + pl.off_pD);
+    p.ws_dBh = reinterpret_cast<float *>(ws + pl.off_dB);
+    p.ws_dCh = reinterpret_cast<float *>(ws + pl.off_dC);
+    if (p.nch > 2147483647LL || (int64_t)p.b * p.H > 65535LL * 65535LL)
+        return fail(SSD_ERR_SHAPE, "sequence too long for the backward grid");
+    if (a->H > 65535 || a->b > 65535) return fail(SSD_ERR_SHAPE, "H and b must be at most 65535");
+    rc = ssd::launch_scan_backward(p, a->dtype, st);
+    if (rc) return fail(SSD_ERR_LAUNCH, "backward launch failed: %s", cudaGetErrorString(cudaGetLastError()));
+    return ok();
+}
+
 int conv_impl(const void *u, int64_t ubs, int64_t urs, const float *w, const float *bias,
               const void *tail_in, void *tail_out, void *v, int64_t vbs, int64_t vrs,
               int b, int64_t L, int C_ch, int dtype, cudaStream_t st)
@@ -257,7 +353,8 @@ int conv_impl(const void *u, int64_t ubs, int64_t urs, const float *w, const flo
 // ---------------------------------------------------------------- kernel timing
 const char *const kKernelNames[ssd::kKCount] = {
     "conv1d_silu", "conv_tail", "stripe_state_tc", "stripe_chain", "chunk_output_tc",
-    "stripe_state_generic", "chunk_output_generic", "decode_step"};
+    "stripe_state_generic", "chunk_output_generic", "decode_step", "bwd_chunk_summary", "bwd_chains",
+    "bwd_chunk_grad", "bwd_reduce"};
 
 struct ProfRecord {
     int id;
@@ -388,6 +485,16 @@ int ssd_stream_forward(const ssd_stream_args *a, ssd_stream_t stream)
     s.h_final = a->h_final; s.h_ckpt = a->h_ckpt;
     s.workspace = a->workspace; s.workspace_bytes = a->workspace_bytes;
     return scan_impl(&s, (cudaStream_t)stream);
+}
+
+int ssd_scan_backward(const ssd_scan_bwd_args *args, ssd_stream_t stream)
+{
+    return scan_bwd_impl(args, (cudaStream_t)stream);
+}
+
+size_t ssd_scan_backward_workspace_size(int b, int64_t L, int H, int P, int N)
+{
+    return make_bwd_plan(b, L, H, P, N).bytes;
 }
 
 int ssd_decode_step(const ssd_decode_args *a, ssd_stream_t stream)

@@ -84,6 +84,36 @@ struct DecodeParams {
     float dt_min, dt_max;
 };
 
+// The backward pass of the scan (scan_bwd.cu).
+struct BwdParams {
+    int b;
+    int64_t L;
+    int H, P, N, G;
+    int64_t s, n_ckpt;
+    int64_t nch;            // chunks of kQb = 64 tokens
+    int64_t cell_chunks;    // chunks per recompute cell (s / 64, or nch without checkpoints)
+    const void *x;
+    int64_t xbs, xrs;
+    const void *B;
+    int64_t Bbs, Brs;
+    const void *C;
+    int64_t Cbs, Crs;
+    const void *dy;
+    int64_t dybs, dyrs;
+    const float *dt;
+    const float *A;
+    const float *D;
+    const float *h0;
+    const float *h_ckpt;
+    const float *dh_final;
+    float *dx, *dB, *dC, *ddt, *dA, *dD, *dh0;
+    float *ws_h;            // [b][H][nch][P][N] S_c, then the state entering chunk c
+    float *ws_g;            // [b][H][nch][P][N] Gl_c, then the adjoint leaving chunk c
+    float *ws_lam;          // [b][H][nch] sum of dt*A over the chunk
+    float *ws_dBh, *ws_dCh; // [b][L][H][N] per-head dB and dC
+    float *ws_pA, *ws_pD;   // [b][H][nch] per-chunk dA and dD
+};
+
 // The step size a kernel uses for a raw dt value of head h: dt + dt_bias[h]
 // (bias optional), through softplus(v) = log(1 + e^v) when asked (v itself
 // above 20, where the two agree in fp32), clamped to [dt_min, dt_max] when
@@ -123,7 +153,8 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // Kernel timing hooks (ssd_api.cu): no-ops unless ssd_profile_begin() is active
 // on the calling thread.
 enum KernelId : int {
-    kKConv = 0, kKConvTail, kKStateTc, kKChain, kKOutputTc, kKStateGeneric, kKOutputGeneric, kKDecode, kKCount
+    kKConv = 0, kKConvTail, kKStateTc, kKChain, kKOutputTc, kKStateGeneric, kKOutputGeneric, kKDecode,
+    kKBwdSummary, kKBwdChain, kKBwdGrad, kKBwdReduce, kKCount
 };
 void prof_begin(cudaStream_t st, int id);
 void prof_end(cudaStream_t st, int id);
@@ -134,5 +165,7 @@ int launch_decode(const DecodeParams &p, int dtype, cudaStream_t st);
 int launch_scan_generic(const ScanParams &p, int dtype, cudaStream_t st);
 int launch_dt_prepare(const ScanParams &p, float *out, cudaStream_t st);
 bool tc_scan_supported(const ScanParams &p, int dtype);
+int launch_scan_backward(const BwdParams &p, int dtype, cudaStream_t st);
+size_t bwd_grad_smem_bytes(int P, int N);
 int launch_scan_tc(const ScanParams &p, cudaStream_t st);
 }  // namespace ssd

@@ -14,6 +14,7 @@ Distributions:
        bias_h = inverse softplus of dt0_h,  dt0_h ~ logU[dt_min, dt_max]
   A_h = -exp(U[log 1, log 16]),  D_h ~ N(0, 1),  conv w ~ U(-0.5, 0.5), conv bias 0
   h0 = 0 and zero conv tail unless a test asks for random ones.
+  backward: dy ~ N(0, 1) in the I/O dtype, dh_final ~ N(0, 1).
 """
 from dataclasses import dataclass, field
 import math
@@ -153,6 +154,17 @@ def make_tail(wl: Workload, b=None, device="cpu", seed=None):
     b = wl.b if b is None else b
     g = _gen((wl.seed if seed is None else seed) + 5000, device)
     return torch.randn(b, 3, wl.cch, device=device, generator=g).to(torch_dtype(wl.dtype))
+
+
+def make_grads(wl: Workload, L=None, b=None, device="cpu", seed=None):
+    """Upstream gradients for the backward pass: dy [b, L, H*P] ~ N(0,1) in the
+    I/O dtype and dh_final [b, H, P, N] ~ N(0,1) fp32."""
+    L = wl.L if L is None else L
+    b = wl.b if b is None else b
+    g = _gen((wl.seed if seed is None else seed) + 6000, device)
+    dy = torch.randn(b, L, wl.d_inner, device=device, generator=g).to(torch_dtype(wl.dtype))
+    dhf = torch.randn(b, wl.H, wl.P, wl.N, device=device, generator=g)
+    return dy, dhf
 
 
 def scaled(wl: Workload, **changes) -> Workload:
