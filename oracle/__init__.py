@@ -37,6 +37,9 @@ def _bind(path):
                                          f32p, f32p, f32p, f64p, f64p, f64p, f64p,
                                          f64p, f64p, f64p, f64p, f64p, f64p, f64p]
     lib.oracle_scan_backward.restype = None
+    lib.oracle_gated_rmsnorm.argtypes = [i64, ctypes.c_int, ctypes.c_int, f32p, i64, f32p, i64, f32p,
+                                         ctypes.c_double, ctypes.c_int, f32p, i64]
+    lib.oracle_gated_rmsnorm.restype = None
     lib.oracle_round_bf16.argtypes = [ctypes.c_double]
     lib.oracle_round_bf16.restype = ctypes.c_double
     lib.oracle_num_threads.argtypes = []
@@ -226,6 +229,29 @@ def scan_backward(x, B, C, dt, A, D, dy, h0=None, h_ckpt=None, dh_final=None, s=
         dC[:, :, grp[h]] += dC_h[:, :, h]
     return {"dx": dx, "dB": dB, "dC": dC, "ddt": ddt, "dA": dA_b.sum(0), "dD": dD_b.sum(0),
             "dh0": dh0, "dB_h": dB_h, "dC_h": dC_h}
+
+
+def gated_rmsnorm(y, z, w, eps=1e-5, group=None, io_round="none"):
+    """out = v / sqrt(mean over the group of v^2 + eps) * w with v = y * silu(z), fp64.
+
+    y, z: [..., d] (the exact I/O values), w: [d]; groups of ``group``
+    consecutive channels (default: all d).  Returns float32 rounded per
+    ``io_round``, shaped like y.
+    """
+    lib = _load()
+    y = _f32(y)
+    z = _f32(z)
+    shape = y.shape
+    d = shape[-1]
+    group = d if group is None else group
+    assert z.shape == shape and d % group == 0
+    y2 = y.reshape(-1, d)
+    z2 = z.reshape(-1, d)
+    w = _f32(w)
+    out = np.empty_like(y2)
+    lib.oracle_gated_rmsnorm(y2.shape[0], d, group, _p32(y2), d, _p32(z2), d, _p32(w), float(eps),
+                             IO_ROUND[io_round], _p32(out), d)
+    return out.reshape(shape)
 
 
 def dt_effective(dt, dt_bias=None, softplus=False, dt_min=0.0, dt_max=0.0):

@@ -297,6 +297,39 @@ void oracle_scan_backward(int b, int64_t L, int H, int P, int N, int G, int64_t 
     }
 }
 
+/* ---- gated RMS normalisation of the layer output ------------------------
+ * The Mamba-2 block's output norm (not on the pages, which end at y; the
+ * plainest block surroundings): for every row r and channel c of d,
+ *   v[c]   = y[r,c] * silu(z[r,c]),   silu(z) = z / (1 + e^-z)
+ *   ms_g   = (1/group) * sum_{c' in group g} v[c']^2     (groups of `group`
+ *            consecutive channels)
+ *   out[r,c] = v[c] / sqrt(ms_g + eps) * w[c]
+ * rounded to the I/O dtype.  Rows are y[r*y_rs + c], z[r*z_rs + c],
+ * out[r*out_rs + c]; w is [d].
+ */
+void oracle_gated_rmsnorm(int64_t rows, int d, int group,
+                          const float *y, int64_t y_rs, const float *z, int64_t z_rs,
+                          const float *w, double eps, int io_round,
+                          float *out, int64_t out_rs)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        double *v = (double *)malloc(sizeof(double) * (size_t)d);
+        for (int c = 0; c < d; ++c) {
+            const double zc = z[r * z_rs + c];
+            v[c] = (double)y[r * y_rs + c] * (zc / (1.0 + exp(-zc)));
+        }
+        for (int g0 = 0; g0 < d; g0 += group) {
+            double ss = 0.0;
+            for (int c = g0; c < g0 + group; ++c) ss += v[c] * v[c];
+            const double scale = 1.0 / sqrt(ss / group + eps);
+            for (int c = g0; c < g0 + group; ++c)
+                out[r * out_rs + c] = (float)round_io(v[c] * scale * (double)w[c], io_round);
+        }
+        free(v);
+    }
+}
+
 /* Number of OpenMP threads the oracle would use (for reporting). */
 int oracle_num_threads(void)
 {

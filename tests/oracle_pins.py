@@ -422,8 +422,45 @@ def pin_backward_without_input():
     assert _rel(bw["dA"], dA) < 1e-12
 
 
+def pin_gated_norm_torch():
+    """The gated RMS norm against torch's rms_norm of y * silu(z) in fp64, four groups of 8."""
+    rng = RNG(40)
+    y = rng.standard_normal((3, 5, 32)).astype(np.float32)
+    z = (2 * rng.standard_normal((3, 5, 32))).astype(np.float32)
+    w = rng.standard_normal(32).astype(np.float32)
+    eps = 1e-2
+    got = oracle.gated_rmsnorm(y, z, w, eps=eps, group=8)
+    v = torch.from_numpy(y).double() * torch.nn.functional.silu(torch.from_numpy(z).double())
+    ref = torch.nn.functional.rms_norm(v.reshape(3, 5, 4, 8), (8,), eps=eps).reshape(3, 5, 32)
+    ref = (ref * torch.from_numpy(w).double()).numpy()
+    assert _rel(got, ref) < 1e-7, _rel(got, ref)
+    # one group over all channels
+    got1 = oracle.gated_rmsnorm(y, z, w, eps=eps)
+    ref1 = (torch.nn.functional.rms_norm(v, (32,), eps=eps) * torch.from_numpy(w).double()).numpy()
+    assert _rel(got1, ref1) < 1e-7
+
+
+def pin_gated_norm_invariants():
+    """A closed gate gives zero; without eps the norm ignores a power-of-two scale of y;
+    the normalised squares of a group average to ms / (ms + eps)."""
+    rng = RNG(41)
+    y = rng.standard_normal((4, 64)).astype(np.float32)
+    z = rng.standard_normal((4, 64)).astype(np.float32)
+    w = rng.uniform(0.5, 2.0, 64).astype(np.float32)
+    assert np.array_equal(oracle.gated_rmsnorm(y, np.zeros_like(z), w, group=16), np.zeros_like(y))
+    a = oracle.gated_rmsnorm(y, z, w, eps=0.0, group=16)
+    b = oracle.gated_rmsnorm(4 * y, z, w, eps=0.0, group=16)
+    assert np.array_equal(a, b)
+    eps = 0.25
+    out = oracle.gated_rmsnorm(y, z, w, eps=eps, group=16).astype(np.float64) / w
+    v = y.astype(np.float64) * (z / (1 + np.exp(-z.astype(np.float64))))
+    ms = (v.reshape(4, 4, 16) ** 2).mean(-1)
+    got = (out.reshape(4, 4, 16) ** 2).mean(-1)
+    assert np.abs(got - ms / (ms + eps)).max() < 1e-6
+
+
 PINS = [pin_quadratic_form, pin_A_zero_prefix_sum, pin_constant_geometric, pin_skip_only,
         pin_single_impulse, pin_linearity, pin_conv_torch, pin_conv_delta_weights,
         pin_bf16_rounding, pin_ckpt_indexing, pin_split_resume_bitwise,
         pin_resume_needs_conv_tail, pin_backward_finite_differences, pin_backward_cells_equal_full,
-        pin_backward_without_input]
+        pin_backward_without_input, pin_gated_norm_torch, pin_gated_norm_invariants]

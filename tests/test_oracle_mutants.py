@@ -51,6 +51,15 @@ MUTANTS = {
     "bwd_dA_missing_dt": ("dA_acc += dtv * dA_t;", "dA_acc += dA_t;"),
     "bwd_wrong_checkpoint": ("else v = h_ckpt[(((int64_t)bi * n_ckpt + (k - 1)) * H + h) * PN + i];",
                              "else v = h_ckpt[(((int64_t)bi * n_ckpt + (k > 1 ? k - 2 : 0)) * H + h) * PN + i];"),
+    # gated RMS norm
+    "norm_gate_dropped": ("v[c] = (double)y[r * y_rs + c] * (zc / (1.0 + exp(-zc)));",
+                          "v[c] = (double)y[r * y_rs + c];"),
+    "norm_eps_outside_sqrt": ("const double scale = 1.0 / sqrt(ss / group + eps);",
+                              "const double scale = 1.0 / (sqrt(ss / group) + eps);"),
+    "norm_mean_over_all_channels": ("const double scale = 1.0 / sqrt(ss / group + eps);",
+                                    "const double scale = 1.0 / sqrt(ss / d + eps);"),
+    "norm_weight_dropped": ("out[r * out_rs + c] = (float)round_io(v[c] * scale * (double)w[c], io_round);",
+                            "out[r * out_rs + c] = (float)round_io(v[c] * scale, io_round);"),
     "bwd_adjoint_after_output": ("Gs[(int64_t)p * N + n] += dyt[p] * (double)Ct[n];",
                                  "Gs[(int64_t)p * N + n] += 0.0 * dyt[p] * (double)Ct[n];"),
 }
