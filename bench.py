@@ -55,6 +55,8 @@ def parse_args():
     # the backward pass of the scan instead of the headline step: gradients from the
     # forward's checkpoints, on the 0.3B 16384-token workload (its own JSON line)
     ap.add_argument("--backward", action="store_true")
+    # the gated RMS norm of the layer output on one 131072-token segment of the 0.3B shape
+    ap.add_argument("--gated-norm", action="store_true")
     return ap.parse_args()
 
 
@@ -99,6 +101,65 @@ def recorded_traffic(kernel):
 
 
 # ----------------------------------------------------------------- clocks
+class NvmlClockSampler:
+    """SM clock, power and throttle reasons every 2 ms from a thread (NVML), so that
+    timed regions of a few milliseconds are still sampled while they run."""
+
+    def __init__(self, device_index):
+        import threading
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        # NVML numbers the physical GPUs; find this process's CUDA device by its PCI address
+        prop = torch.cuda.get_device_properties(device_index)
+        bus = "%08X:%02X:%02X.0" % (prop.pci_domain_id, prop.pci_bus_id, prop.pci_device_id)
+        try:
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except pynvml.NVMLError:
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+        self.rows = []
+        self.stop_flag = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+
+    def _sample(self):
+        nv = self.nv
+        r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        self.rows.append({"sm": nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
+                          "max": nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM),
+                          "power": nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0, "bits": r})
+
+    def _run(self):
+        while not self.stop_flag.is_set():
+            self._sample()
+            time.sleep(0.002)
+
+    def start(self):
+        self._sample()
+        self.thread.start()
+
+    def stop(self):
+        self.stop_flag.set()
+        self.thread.join(timeout=5)
+        self._sample()
+        rows = self.rows[1:-1] or self.rows
+        nv = self.nv
+        names = ((nv.nvmlClocksEventReasonHwSlowdown, "hw_slowdown"),
+                 (nv.nvmlClocksEventReasonHwThermalSlowdown, "hw_thermal_slowdown"),
+                 (nv.nvmlClocksEventReasonSwThermalSlowdown, "sw_thermal_slowdown"),
+                 (nv.nvmlClocksEventReasonSwPowerCap, "sw_power_cap"))
+        reasons = sorted({name for r in rows for bit, name in names if r["bits"] & bit})
+        loaded = [r for r in rows if r["power"] > 200] or rows
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(loaded), "source": "nvml"}
+
+
+def clock_sampler(device_index):
+    try:
+        return NvmlClockSampler(device_index)
+    except Exception:
+        return ClockSampler(device_index)
+
+
 class ClockSampler:
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -409,7 +470,7 @@ def run_decode(args, world, rank, local):
                         h_in=h, h_out=h, y=y)
         t[0] += 1
 
-    clocks = ClockSampler(local)
+    clocks = clock_sampler(local)
     clocks.start()
     ms = time_steps(step, args.steps, args.warmup, world, local)
     clk = clocks.stop()
@@ -477,7 +538,7 @@ def run_backward(args, world, rank, local):
         ssd.scan_backward(x, Bm, Cm, dt, prm["A"], prm["D"], dy, h_ckpt=ck, dh_final=dhf, H=wl.H, G=wl.G,
                           s=wl.s, workspace=ws, out=out)
 
-    clocks = ClockSampler(local)
+    clocks = clock_sampler(local)
     clocks.start()
     ms = time_steps(step, args.steps, args.warmup, world, local)
     clk = clocks.stop()
@@ -519,6 +580,49 @@ def run_backward(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_gated_norm(args, world, rank, local):
+    """out = rmsnorm(y * silu(z)) * w on 131072 rows of the 0.3B d_inner (2048), bf16, one group."""
+    import __graft_entry__
+    __graft_entry__.build()
+    import mamba_selective_state_causal_b200 as ssd
+    rows, d = 131072, 2048
+    dev = torch.device("cuda", torch.cuda.current_device())
+    g = torch.Generator(device=dev)
+    g.manual_seed(100 * rank + 7)
+    y = torch.randn(rows, d, device=dev, generator=g).to(torch.bfloat16)
+    z = torch.randn(rows, d, device=dev, generator=g).to(torch.bfloat16)
+    w = torch.randn(d, device=dev, generator=g)
+    out = torch.empty_like(y)
+
+    def step():
+        ssd.gated_rmsnorm(y, z, w, eps=1e-5, out=out)
+
+    clocks = clock_sampler(local)
+    clocks.start()
+    ms = time_steps(step, args.steps, args.warmup, world, local)
+    clk = clocks.stop()
+    ssd.sync_status()
+    ms = max_over_ranks(world, ms)
+    step_bytes = rows * d * 2 * 3
+    peak, peak_src = hbm_peak()
+    achieved = step_bytes / (ms / args.steps / 1e3) / 1e9
+    line = {
+        "metric": "gated RMS norm rows/s (0.3B d_inner = 2048, bf16)",
+        "value": rows * world * args.steps / (ms / 1e3), "unit": "rows/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "gated-rmsnorm-0.3b-131072rows", "rows": rows, "d": d, "group": d,
+                   "l2": "inputs larger than L2 (%.2f GB)" % (2 * rows * d * 2 / 1e9)},
+        "roofline": {"bound": "hbm", "kernel": "gated_rmsnorm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": peak_src, "traffic": None,
+                     "algorithmic_bytes_per_launch": step_bytes},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     wl = ssd_synth.BY_NAME[args.workload]
@@ -535,11 +639,14 @@ def main():
     if args.backward:
         run_backward(args, world, rank, local)
         return
+    if args.gated_norm:
+        run_gated_norm(args, world, rank, local)
+        return
     import __graft_entry__
     __graft_entry__.build()
     layer = Layer(wl, seed=rank_seed(wl, rank))
 
-    clocks = ClockSampler(local)
+    clocks = clock_sampler(local)
     clocks.start()
     ms = time_steps(layer.step, args.steps, args.warmup, world, local)
     clk = clocks.stop()

@@ -312,6 +312,25 @@ SSD_API int ssd_scan_backward(const ssd_scan_bwd_args *args, ssd_stream_t stream
 SSD_API size_t ssd_scan_backward_workspace_size(int b, int64_t L, int H, int P, int N);
 
 /*
+ * ssd_gated_rmsnorm_forward -- the output norm of the Mamba-2 block on the
+ * layer's y (the pages end at y; this is the plainest reading of the block
+ * around it: normalise after gating, over groups of consecutive channels):
+ *   v = y * silu(z),  silu(z) = z / (1 + exp(-z))
+ *   out[r,c] = v[r,c] / sqrt(mean_{c' in group(c)} v[r,c']^2 + eps) * weight[c]
+ *   y, z, out  rows r = 0..rows-1 of d channels, element (r,c) at ptr[r*row_stride + c],
+ *              I/O dtype; a [b][L][d] tensor is rows = b*L when its batches
+ *              are consecutive rows.  out may alias y (same stride).
+ *   weight     [d] float;  eps >= 0;  group_size: channels per group, a
+ *              multiple of 8 dividing d, or 0 for one group of all d.
+ * d a multiple of 8, at most 8192; pointers and row strides 16-byte aligned.
+ * Asynchronous on `stream`.
+ */
+SSD_API int ssd_gated_rmsnorm_forward(const void *y, int64_t y_row_stride, const void *z, int64_t z_row_stride,
+                                      const float *weight, float eps, int group_size,
+                                      void *out, int64_t out_row_stride, int64_t rows, int d, int dtype,
+                                      ssd_stream_t stream);
+
+/*
  * ssd_scan_forward_static_scratch -- ssd_scan_forward for callers that cannot
  * allocate device memory.  (The pages have no counterpart: this is a
  * deployment aid of this library, not part of the layer they describe.)

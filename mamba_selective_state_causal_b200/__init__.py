@@ -108,6 +108,9 @@ def lib():
         L.ssd_stream_forward.restype = ctypes.c_int
         L.ssd_decode_step.argtypes = [ctypes.POINTER(DecodeArgs), _vp]
         L.ssd_decode_step.restype = ctypes.c_int
+        L.ssd_gated_rmsnorm_forward.argtypes = [_vp, _i64, _vp, _i64, _vp, ctypes.c_float, ctypes.c_int, _vp, _i64,
+                                                _i64, ctypes.c_int, ctypes.c_int, _vp]
+        L.ssd_gated_rmsnorm_forward.restype = ctypes.c_int
         L.ssd_scan_backward.argtypes = [ctypes.POINTER(ScanBwdArgs), _vp]
         L.ssd_scan_backward.restype = ctypes.c_int
         L.ssd_scan_backward_workspace_size.argtypes = [ctypes.c_int, _i64, ctypes.c_int, ctypes.c_int,
@@ -383,3 +386,26 @@ def scan_backward(x, B, C, dt, A, D, dy, h0=None, h_ckpt=None, dh_final=None, *,
     a.workspace = workspace.data_ptr(); a.workspace_bytes = workspace.numel()
     _check(lib().ssd_scan_backward(ctypes.byref(a), _stream(stream)))
     return o
+
+
+def gated_rmsnorm(y, z, weight, eps=1e-5, group_size=0, out=None, stream=None):
+    """out = rmsnorm(y * silu(z)) * weight over groups of ``group_size`` channels (0: all).
+
+    y, z: [..., d] with the same leading shape, rows of d contiguous channels
+    (z may be a column slice of a wider tensor); weight: [d] float32.
+    """
+    _cuda(y, z, weight, out)
+    _f32(weight, "weight")
+    d = y.shape[-1]
+    y2 = y.reshape(-1, d)
+    z2 = z.reshape(-1, d) if z.is_contiguous() else z.flatten(0, -2)
+    if out is None:
+        out = torch.empty_like(y)
+    o2 = out.view(-1, d)
+    if z2.dtype != y2.dtype or o2.dtype != y2.dtype:
+        raise TypeError("y, z and out must share the I/O dtype")
+    rc = lib().ssd_gated_rmsnorm_forward(_ptr(y2), y2.stride(0), _ptr(z2), z2.stride(0), _ptr(weight), float(eps),
+                                         int(group_size), _ptr(o2), o2.stride(0), y2.shape[0], d, _dtype_code(y2),
+                                         _stream(stream))
+    _check(rc)
+    return out

@@ -53,16 +53,20 @@ __device__ __forceinline__ void load_rows(float *dst, int dst_rs, const T *src, 
     }
 }
 
-// acc[r][c] += sum_k a[(r0 + r) * ars + k * acs] * b[k * brs + (c0 + c) * bcs]
+// acc[r][c] += sum_k a[(r0 + r*rs) * ars + k * acs] * b[k * brs + (c0 + c*cs) * bcs]
+// A thread's 4 x 4 tile takes rows r0 + r*rs and columns c0 + c*cs: the callers step
+// consecutive threads over consecutive columns (or rows), so that a warp's
+// shared-memory reads fall in distinct banks and its global reads are contiguous.
 __device__ __forceinline__ void mm4x4(float (&acc)[4][4], const float *a, int ars, int acs, const float *b, int brs,
-                                      int bcs, int K, int r0, int c0)
+                                      int bcs, int K, int r0, int rs, int c0, int cs)
 {
+#pragma unroll 4
     for (int k = 0; k < K; ++k) {
         float av[4], bv[4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) av[r] = a[(r0 + r) * ars + k * acs];
+        for (int r = 0; r < 4; ++r) av[r] = a[(r0 + r * rs) * ars + k * acs];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) bv[c] = b[(int64_t)k * brs + (int64_t)(c0 + c) * bcs];
+        for (int c = 0; c < 4; ++c) bv[c] = b[(int64_t)k * brs + (int64_t)(c0 + c * cs) * bcs];
 #pragma unroll
         for (int r = 0; r < 4; ++r)
 #pragma unroll
@@ -134,22 +138,22 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_chunk_summary_kernel(BwdParam
 
     float *S = p.ws_h + unit * P * N;
     float *Gl = p.ws_g + unit * P * N;
-    const int ct = N / 4;
+    const int ct = N / 4;   // a tile's columns are n0 + c * ct
     for (int tile = threadIdx.x; tile < (P / 4) * ct; tile += blockDim.x) {
-        const int p0 = (tile / ct) * 4, n0 = (tile % ct) * 4;
+        const int p0 = (tile / ct) * 4, n0 = tile % ct;
         float acc[4][4];
         zero4x4(acc);
-        mm4x4(acc, xs, 1, P1, bs, N1, 1, kQb, p0, n0);
+        mm4x4(acc, xs, 1, P1, bs, N1, 1, kQb, p0, 1, n0, ct);
 #pragma unroll
         for (int r = 0; r < 4; ++r)
-            *reinterpret_cast<float4 *>(S + (int64_t)(p0 + r) * N + n0) =
-                make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) S[(int64_t)(p0 + r) * N + n0 + c * ct] = acc[r][c];
         zero4x4(acc);
-        mm4x4(acc, gs, 1, P1, cs, N1, 1, kQb, p0, n0);
+        mm4x4(acc, gs, 1, P1, cs, N1, 1, kQb, p0, 1, n0, ct);
 #pragma unroll
         for (int r = 0; r < 4; ++r)
-            *reinterpret_cast<float4 *>(Gl + (int64_t)(p0 + r) * N + n0) =
-                make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) Gl[(int64_t)(p0 + r) * N + n0 + c * ct] = acc[r][c];
     }
 }
 
@@ -266,13 +270,18 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_chunk_grad_kernel(BwdParams p
     float *be = al + kQb;            // be_j
     float *din = be + kQb;           // B_t . dBr_t
     float *rr = din + kQb;           // sum_{t'>=t} sum_{j<t} K[t'][j]
-    float *red = rr + kQb;           // [2][Qb][32] row partials over column tiles
-    float *misc = red + 2 * kQb * 32;   // [kBwdThreads / 32]
+    float *misc = rr + kQb;          // [kBwdThreads / 32 + kQb]
+    float *red = CB;                 // [2][Qb][32] row partials over column tiles, once CB is spent
+    float *gam_s = misc + kBwdThreads / 32 + kQb;   // [P][N] copies of Gam and h_prev, when staged
+    float *hpv_s = gam_s + P * N;
 
     const int64_t hu = (int64_t)bi * p.H + h;
     const int64_t unit = hu * p.nch + c;
-    const float *hprev = p.ws_h + unit * P * N;
-    const float *Gam = p.ws_g + unit * P * N;
+    const float *hprev_g = p.ws_h + unit * P * N;
+    const float *Gam_g = p.ws_g + unit * P * N;
+    // with room in shared memory the chunk's Gam and h_prev are copied there once
+    const float *Gam = p.stage_adjoint ? gam_s : Gam_g;
+    const float *hprev = p.stage_adjoint ? hpv_s : hprev_g;
     const float Ah = p.A[h];
     const float Dh = p.D ? p.D[h] : 0.0f;
 
@@ -282,6 +291,12 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_chunk_grad_kernel(BwdParams p
     load_rows(bs, N1, reinterpret_cast<const T *>(p.B) + bi * p.Bbs + t0 * p.Brs + (int64_t)g * N, p.Brs, rows, N);
     load_rows(cs, N1, reinterpret_cast<const T *>(p.C) + bi * p.Cbs + t0 * p.Crs + (int64_t)g * N, p.Crs, rows, N);
     for (int i = tid; i < kQb; i += blockDim.x) dts[i] = i < rows ? p.dt[((int64_t)bi * p.L + t0 + i) * p.H + h] : 0.0f;
+    if (p.stage_adjoint) {
+        for (int i = tid; i < P * N / 4; i += blockDim.x) {
+            reinterpret_cast<float4 *>(gam_s)[i] = reinterpret_cast<const float4 *>(Gam_g)[i];
+            reinterpret_cast<float4 *>(hpv_s)[i] = reinterpret_cast<const float4 *>(hprev_g)[i];
+        }
+    }
     __syncthreads();
     chunk_cumsum(dts, cum, Ah);
     // <Gam, h_prev>, reduced in a fixed order
@@ -296,22 +311,23 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_chunk_grad_kernel(BwdParams p
         ecs[i] = expf(cum[i]);
         eend[i] = expf(lam - cum[i]);
     }
-    // CB[t][j] = C_t . B_j and GX[t][j] = dy_t . x_j, all t, j
-    for (int tile = tid; tile < (kQb / 4) * (kQb / 4); tile += blockDim.x) {
-        const int r0 = (tile / (kQb / 4)) * 4, c0 = (tile % (kQb / 4)) * 4;
+    // CB[t][j] = C_t . B_j and GX[t][j] = dy_t . x_j, all t, j (a tile's columns are c0 + 16q)
+    constexpr int kQt = kQb / 4;
+    for (int tile = tid; tile < kQt * kQt; tile += blockDim.x) {
+        const int r0 = (tile / kQt) * 4, c0 = tile % kQt;
         float acc[4][4];
         zero4x4(acc);
-        mm4x4(acc, cs, N1, 1, bs, 1, N1, N, r0, c0);
+        mm4x4(acc, cs, N1, 1, bs, 1, N1, N, r0, 1, c0, kQt);
 #pragma unroll
         for (int r = 0; r < 4; ++r)
 #pragma unroll
-            for (int q = 0; q < 4; ++q) CB[(r0 + r) * kQ1 + c0 + q] = acc[r][q];
+            for (int q = 0; q < 4; ++q) CB[(r0 + r) * kQ1 + c0 + q * kQt] = acc[r][q];
         zero4x4(acc);
-        mm4x4(acc, gs, P1, 1, xs, 1, P1, P, r0, c0);
+        mm4x4(acc, gs, P1, 1, xs, 1, P1, P, r0, 1, c0, kQt);
 #pragma unroll
         for (int r = 0; r < 4; ++r)
 #pragma unroll
-            for (int q = 0; q < 4; ++q) GX[(r0 + r) * kQ1 + c0 + q] = acc[r][q];
+            for (int q = 0; q < 4; ++q) GX[(r0 + r) * kQ1 + c0 + q * kQt] = acc[r][q];
     }
     __syncthreads();
     float gam_h = 0.0f;
@@ -363,17 +379,18 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_chunk_grad_kernel(BwdParams p
     // dx[j][p] = D dy_j + dt_j (sum_t CB[t][j] dy_t[p] + eend_j sum_n Gam[p][n] B_j[n])
     float *dx = p.dx + ((int64_t)bi * p.L + t0) * p.H * P + (int64_t)h * P;
     {
-        const int ct = P / 4;
-        for (int tile = tid; tile < (kQb / 4) * ct; tile += blockDim.x) {
-            const int j0 = (tile / ct) * 4, p0 = (tile % ct) * 4;
+        // a tile's rows are j0 + 16 r (consecutive threads, consecutive rows), its columns
+        // p0 .. p0+3, shared by 16 threads: Gam is read along its rows
+        for (int tile = tid; tile < kQt * (P / 4); tile += blockDim.x) {
+            const int j0 = tile % kQt, p0 = (tile / kQt) * 4;
             float a1[4][4], a2[4][4];
             zero4x4(a1);
             zero4x4(a2);
-            mm4x4(a1, CB, 1, kQ1, gs, P1, 1, kQb, j0, p0);
-            mm4x4(a2, bs, N1, 1, Gam, 1, N, N, j0, p0);
+            mm4x4(a1, CB, 1, kQ1, gs, P1, 1, kQb, j0, kQt, p0, 1);
+            mm4x4(a2, bs, N1, 1, Gam, 1, N, N, j0, kQt, p0, 1);
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
-                const int j = j0 + r;
+                const int j = j0 + r * kQt;
                 if (j < rows) {
                     float o[4];
 #pragma unroll
@@ -391,28 +408,27 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_chunk_grad_kernel(BwdParams p
     float *dCh = p.ws_dCh + (((int64_t)bi * p.L + t0) * p.H + h) * N;
     const int ctn = N / 4;
     for (int tile = tid; tile < (kQb / 4) * ctn; tile += blockDim.x) {
-        const int j0 = (tile / ctn) * 4, n0 = (tile % ctn) * 4, nt = tile % ctn;
+        const int j0 = (tile / ctn) * 4, nt = tile % ctn;    // columns nt + q * ctn
         float a1[4][4], a2[4][4];
         zero4x4(a1);
         zero4x4(a2);
-        mm4x4(a1, GX, 1, kQ1, cs, N1, 1, kQb, j0, n0);
-        mm4x4(a2, xs, P1, 1, Gam, N, 1, P, j0, n0);
+        mm4x4(a1, GX, 1, kQ1, cs, N1, 1, kQb, j0, 1, nt, ctn);
+        mm4x4(a2, xs, P1, 1, Gam, N, 1, P, j0, 1, nt, ctn);
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             const int j = j0 + r;
-            float o[4], sin = 0.0f, sbe = 0.0f;
+            float sin = 0.0f, sbe = 0.0f;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
+                const int n = nt + q * ctn;
                 const float br = fmaf(eend[j], a2[r][q], a1[r][q]);
-                const float bv = bs[j * N1 + n0 + q];
+                const float bv = bs[j * N1 + n];
                 sin = fmaf(bv, br, sin);
                 sbe = fmaf(bv, a2[r][q], sbe);
-                o[q] = dts[j] * br;
+                if (j < rows) dBh[(int64_t)j * p.H * N + n] = dts[j] * br;
             }
             red[j * 32 + nt] = sin;
             red[kQb * 32 + j * 32 + nt] = sbe;
-            if (j < rows)
-                *reinterpret_cast<float4 *>(dBh + (int64_t)j * p.H * N + n0) = make_float4(o[0], o[1], o[2], o[3]);
         }
     }
     __syncthreads();
@@ -429,24 +445,23 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_chunk_grad_kernel(BwdParams p
 
     // dC[t][n] = ecs_t sum_p dy_t[p] h_prev[p][n] + sum_j GX[t][j] dt_j B_j[n]
     for (int tile = tid; tile < (kQb / 4) * ctn; tile += blockDim.x) {
-        const int r0 = (tile / ctn) * 4, n0 = (tile % ctn) * 4, nt = tile % ctn;
+        const int r0 = (tile / ctn) * 4, nt = tile % ctn;    // columns nt + q * ctn
         float a1[4][4], a2[4][4];
         zero4x4(a1);
         zero4x4(a2);
-        mm4x4(a1, gs, P1, 1, hprev, N, 1, P, r0, n0);
-        mm4x4(a2, KK, kQ1, 1, bs, N1, 1, kQb, r0, n0);
+        mm4x4(a1, gs, P1, 1, hprev, N, 1, P, r0, 1, nt, ctn);
+        mm4x4(a2, KK, kQ1, 1, bs, N1, 1, kQb, r0, 1, nt, ctn);
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             const int t = r0 + r;
-            float o[4], sal = 0.0f;
+            float sal = 0.0f;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                sal = fmaf(a1[r][q], cs[t * N1 + n0 + q], sal);
-                o[q] = fmaf(ecs[t], a1[r][q], a2[r][q]);
+                const int n = nt + q * ctn;
+                sal = fmaf(a1[r][q], cs[t * N1 + n], sal);
+                if (t < rows) dCh[(int64_t)t * p.H * N + n] = fmaf(ecs[t], a1[r][q], a2[r][q]);
             }
             red[t * 32 + nt] = sal;
-            if (t < rows)
-                *reinterpret_cast<float4 *>(dCh + (int64_t)t * p.H * N + n0) = make_float4(o[0], o[1], o[2], o[3]);
         }
     }
     __syncthreads();
@@ -528,16 +543,27 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_param_sum_kernel(BwdParams p)
 
 size_t summary_smem(int P, int N) { return sizeof(float) * ((size_t)2 * kQb * (P + 1) + 2 * kQb * (N + 1) + 4 * kQb); }
 
-size_t grad_smem(int P, int N)
+size_t grad_smem(int P, int N, bool staged)
 {
-    return sizeof(float) * ((size_t)2 * kQb * (P + 1) + 2 * kQb * (N + 1) + 3 * kQb * kQ1 + 9 * kQb + 2 * kQb * 32 +
-                            kBwdThreads / 32 + kQb);
+    return sizeof(float) * ((size_t)2 * kQb * (P + 1) + 2 * kQb * (N + 1) + 3 * kQb * kQ1 + 8 * kQb +
+                            kBwdThreads / 32 + kQb + (staged ? (size_t)2 * P * N : 0));
+}
+
+int smem_optin()
+{
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        return 0;
+    return v;
 }
 
 template <typename T>
-int launch_bwd_t(const BwdParams &p, cudaStream_t st)
+int launch_bwd_t(BwdParams p, cudaStream_t st)
 {
-    const size_t s1 = summary_smem(p.P, p.N), s2 = grad_smem(p.P, p.N);
+    const size_t s1 = summary_smem(p.P, p.N);
+    p.stage_adjoint = grad_smem(p.P, p.N, true) <= (size_t)smem_optin() ? 1 : 0;
+    const size_t s2 = grad_smem(p.P, p.N, p.stage_adjoint != 0);
     if (cudaFuncSetAttribute(bwd_chunk_summary_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1) !=
             cudaSuccess ||
         cudaFuncSetAttribute(bwd_chunk_grad_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2) !=
@@ -568,7 +594,7 @@ int launch_bwd_t(const BwdParams &p, cudaStream_t st)
 
 }  // namespace
 
-size_t bwd_grad_smem_bytes(int P, int N) { return grad_smem(P, N); }
+size_t bwd_grad_smem_bytes(int P, int N) { return grad_smem(P, N, false); }
 
 int launch_scan_backward(const BwdParams &p, int dtype, cudaStream_t st)
 {

@@ -354,7 +354,7 @@ int conv_impl(const void *u, int64_t ubs, int64_t urs, const float *w, const flo
 const char *const kKernelNames[ssd::kKCount] = {
     "conv1d_silu", "conv_tail", "stripe_state_tc", "stripe_chain", "chunk_output_tc",
     "stripe_state_generic", "chunk_output_generic", "decode_step", "bwd_chunk_summary", "bwd_chains",
-    "bwd_chunk_grad", "bwd_reduce"};
+    "bwd_chunk_grad", "bwd_reduce", "gated_rmsnorm"};
 
 struct ProfRecord {
     int id;
@@ -495,6 +495,34 @@ int ssd_scan_backward(const ssd_scan_bwd_args *args, ssd_stream_t stream)
 size_t ssd_scan_backward_workspace_size(int b, int64_t L, int H, int P, int N)
 {
     return make_bwd_plan(b, L, H, P, N).bytes;
+}
+
+int ssd_gated_rmsnorm_forward(const void *y, int64_t y_row_stride, const void *z, int64_t z_row_stride,
+                              const float *weight, float eps, int group_size, void *out, int64_t out_row_stride,
+                              int64_t rows, int d, int dtype, ssd_stream_t stream)
+{
+    if (dtype != SSD_F32 && dtype != SSD_BF16) return fail(SSD_ERR_DTYPE, "unknown dtype %d", dtype);
+    if (rows < 0) return fail(SSD_ERR_SHAPE, "negative rows (%lld)", (long long)rows);
+    if (d <= 0 || d % 8 != 0 || d > 8192)
+        return fail(SSD_ERR_SHAPE, "d=%d must be a positive multiple of 8, at most 8192", d);
+    const int group = group_size == 0 ? d : group_size;
+    if (group <= 0 || group % 8 != 0 || d % group != 0)
+        return fail(SSD_ERR_SHAPE, "group_size=%d must be a multiple of 8 that divides d=%d", group_size, d);
+    if (!(eps >= 0.0f)) return fail(SSD_ERR_SHAPE, "eps must be >= 0");
+    if (rows == 0) return ok();
+    if (!y || !z || !weight || !out) return fail(SSD_ERR_NULL, "y, z, weight and out must not be NULL");
+    if (y_row_stride < d || z_row_stride < d || out_row_stride < d)
+        return fail(SSD_ERR_STRIDE, "row strides must be at least d");
+    const size_t es = elem_size(dtype);
+    if (!aligned16(y) || !aligned16(z) || !aligned16(out) || !aligned16(weight) || (y_row_stride * es) % 16 != 0 ||
+        (z_row_stride * es) % 16 != 0 || (out_row_stride * es) % 16 != 0)
+        return fail(SSD_ERR_ALIGN, "y, z, out, weight and the row strides must be 16-byte aligned");
+    ssd::NormParams p{};
+    p.y = y; p.yrs = y_row_stride; p.z = z; p.zrs = z_row_stride; p.w = weight; p.eps = eps; p.group = group;
+    p.out = out; p.ors = out_row_stride; p.rows = rows; p.d = d;
+    if (ssd::launch_gated_norm(p, dtype, (cudaStream_t)stream))
+        return fail(SSD_ERR_LAUNCH, "norm launch failed: %s", cudaGetErrorString(cudaGetLastError()));
+    return ok();
 }
 
 int ssd_decode_step(const ssd_decode_args *a, ssd_stream_t stream)

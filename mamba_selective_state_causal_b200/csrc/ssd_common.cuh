@@ -112,6 +112,22 @@ struct BwdParams {
     float *ws_lam;          // [b][H][nch] sum of dt*A over the chunk
     float *ws_dBh, *ws_dCh; // [b][L][H][N] per-head dB and dC
     float *ws_pA, *ws_pD;   // [b][H][nch] per-chunk dA and dD
+    int stage_adjoint;      // set by the launcher: copy Gam and h_prev into shared memory
+};
+
+// The gated RMS norm of the layer output (gated_norm.cu).
+struct NormParams {
+    const void *y;
+    int64_t yrs;
+    const void *z;
+    int64_t zrs;
+    const float *w;
+    float eps;
+    int group;
+    void *out;
+    int64_t ors;
+    int64_t rows;
+    int d;
 };
 
 // The step size a kernel uses for a raw dt value of head h: dt + dt_bias[h]
@@ -154,7 +170,7 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // on the calling thread.
 enum KernelId : int {
     kKConv = 0, kKConvTail, kKStateTc, kKChain, kKOutputTc, kKStateGeneric, kKOutputGeneric, kKDecode,
-    kKBwdSummary, kKBwdChain, kKBwdGrad, kKBwdReduce, kKCount
+    kKBwdSummary, kKBwdChain, kKBwdGrad, kKBwdReduce, kKGatedNorm, kKCount
 };
 void prof_begin(cudaStream_t st, int id);
 void prof_end(cudaStream_t st, int id);
@@ -167,5 +183,6 @@ int launch_dt_prepare(const ScanParams &p, float *out, cudaStream_t st);
 bool tc_scan_supported(const ScanParams &p, int dtype);
 int launch_scan_backward(const BwdParams &p, int dtype, cudaStream_t st);
 size_t bwd_grad_smem_bytes(int P, int N);
+int launch_gated_norm(const NormParams &p, int dtype, cudaStream_t st);
 int launch_scan_tc(const ScanParams &p, cudaStream_t st);
 }  // namespace ssd
