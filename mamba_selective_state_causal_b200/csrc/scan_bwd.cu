@@ -41,6 +41,7 @@ namespace {
 
 constexpr int kQb = 64;           // tokens per backward chunk
 constexpr int kBwdThreads = 256;
+constexpr int kGradThreads = 512; // the gradient kernel: 16 warps per SM hide its load latency
 constexpr int kQ1 = kQb + 1;      // padded row of the chunk x chunk matrices
 
 template <typename T>
@@ -246,7 +247,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_adjoint_chain_kernel(BwdParam
 // ---------------------------------------------------------------- gradients
 // One CTA per (chunk, head, batch row).
 template <typename T>
-__global__ void __launch_bounds__(kBwdThreads) bwd_chunk_grad_kernel(BwdParams p)
+__global__ void __launch_bounds__(kGradThreads) bwd_chunk_grad_kernel(BwdParams p)
 {
     extern __shared__ float sm[];
     const int c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
@@ -270,9 +271,9 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_chunk_grad_kernel(BwdParams p
     float *be = al + kQb;            // be_j
     float *din = be + kQb;           // B_t . dBr_t
     float *rr = din + kQb;           // sum_{t'>=t} sum_{j<t} K[t'][j]
-    float *misc = rr + kQb;          // [kBwdThreads / 32 + kQb]
+    float *misc = rr + kQb;          // [kGradThreads / 32 + kQb]
     float *red = CB;                 // [2][Qb][32] row partials over column tiles, once CB is spent
-    float *gam_s = misc + kBwdThreads / 32 + kQb;   // [P][N] copies of Gam and h_prev, when staged
+    float *gam_s = misc + kGradThreads / 32 + kQb;  // [P][N] copies of Gam and h_prev, when staged
     float *hpv_s = gam_s + P * N;
 
     const int64_t hu = (int64_t)bi * p.H + h;
@@ -546,7 +547,7 @@ size_t summary_smem(int P, int N) { return sizeof(float) * ((size_t)2 * kQb * (P
 size_t grad_smem(int P, int N, bool staged)
 {
     return sizeof(float) * ((size_t)2 * kQb * (P + 1) + 2 * kQb * (N + 1) + 3 * kQb * kQ1 + 8 * kQb +
-                            kBwdThreads / 32 + kQb + (staged ? (size_t)2 * P * N : 0));
+                            kGradThreads / 32 + kQb + (staged ? (size_t)2 * P * N : 0));
 }
 
 int smem_optin()
@@ -581,7 +582,7 @@ int launch_bwd_t(BwdParams p, cudaStream_t st)
     bwd_adjoint_chain_kernel<<<dim3(slices, (unsigned)p.H, (unsigned)p.b), kBwdThreads, 0, st>>>(p);
     prof_end(st, kKBwdChain);
     prof_begin(st, kKBwdGrad);
-    bwd_chunk_grad_kernel<T><<<grid, kBwdThreads, s2, st>>>(p);
+    bwd_chunk_grad_kernel<T><<<grid, kGradThreads, s2, st>>>(p);
     prof_end(st, kKBwdGrad);
     prof_begin(st, kKBwdReduce);
     const int64_t total = (int64_t)p.b * p.L * p.G * p.N;
