@@ -92,7 +92,11 @@ __global__ void __launch_bounds__(1024) gated_rmsnorm_kernel(NormParams p)
             }
 #pragma unroll
             for (int k = 0; k < kVec; ++k) {
-                v[k] = yv[k] * (zv[k] / (1.0f + expf(-zv[k])));
+                // silu(z) = z / (1 + e^-z) with the hardware exponential and a fast division; z is
+                // clamped at -80 inside the exponential so the divisor stays below 2^126 (below -80
+                // silu is below 1e-33 either way)
+                const float e = __expf(-fmaxf(zv[k], -80.0f));
+                v[k] = yv[k] * __fdividef(zv[k], 1.0f + e);
                 ss = fmaf(v[k], v[k], ss);
             }
         }
