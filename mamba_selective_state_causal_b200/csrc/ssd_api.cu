@@ -575,6 +575,6 @@ int ssd_sync_status(ssd_stream_t stream)
 
 const char *ssd_last_error_string(void) { return g_last_error.c_str(); }
 
-int ssd_version(void) { return 100; }
+int ssd_version(void) { return 200; }   // 0.2.0: backward, its workspace size, gated norm
 
 }  // extern "C"
