@@ -28,6 +28,16 @@
  *  - dtype SSD_BF16: x/B/C, u, v, y and the conv tails are bfloat16; SSD_F32:
  *    they are float.  dt, A, D, conv weights/bias, h0, h_final and h_ckpt are
  *    always float (fp32 state).
+ *  - Environment variables, read once per process at the first scan call
+ *    (test and diagnostic hooks; leave them unset in production):
+ *      SSD_WAIT_LIMIT_MS   bound of every device-side wait in milliseconds
+ *                          (default 2000); a wait that runs out latches
+ *                          SSD_ERR_TIMEOUT in the device status word.
+ *      SSD_TEST_DROP_UNIT  index of one work unit (CTA) of the tensor-core
+ *                          scan whose loads are never issued, so that its
+ *                          waits run out (failure-detection test); it applies
+ *                          to the first scan call of the process only.
+ *      SSD_SCAN_PATH       "generic" forces the CUDA-core scan kernels.
  */
 #ifndef SSD_H_
 #define SSD_H_
@@ -255,8 +265,13 @@ SSD_API int ssd_decode_step(const ssd_decode_args *args, ssd_stream_t stream);
 /*
  * Arguments of the backward pass of the scan (see ssd_scan_backward).
  *   dtype, b, L, H, P, N, G, x, B, C, dt, A, D, h0: as given to the forward
- *           call whose gradients are wanted (dt is the step size the scan
- *           used; x, B, C laid out and aligned as for ssd_scan_forward).
+ *           call whose gradients are wanted (x, B, C laid out and aligned as
+ *           for ssd_scan_forward).  dt is the step size the scan USED: when
+ *           the forward applied dt_bias / softplus / a clamp, pass the
+ *           effective dt_eff = clamp(f(dt + dt_bias)) (the forward keeps it only
+ *           in its workspace), and ddt is then dLoss/d(dt_eff): the chain
+ *           rule through the bias, softplus and clamp is the caller's
+ *           elementwise step.
  *   h_ckpt  [b][floor(L/s)][H][P][N] float: that call's checkpoints, s their
  *           stride (a multiple of 64).  Or NULL (s ignored): the states are
  *           then rebuilt from h0 over the whole sequence.

@@ -10,6 +10,7 @@
 // 3-token halo lives in registers and slides along the token block, so every
 // input row is read once (plus a 3-row halo per token block) and written once.
 #include <algorithm>
+#include <atomic>
 
 #include "ssd_common.cuh"
 
@@ -211,7 +212,7 @@ int launch_conv_t(const ConvParams &p, cudaStream_t st)
         const int64_t blocks = (threads + kConvThreads - 1) / kConvThreads;
         if (blocks > 0x7fffffffLL) return 2;
         constexpr int smem = kRing * kConvThreads * (int)sizeof(Vec16);
-        static bool attr_set[64] = {false};
+        static std::atomic<bool> attr_set[64];   // set once per device (a repeat is harmless)
         int dev = 0;
         cudaGetDevice(&dev);
         if (dev >= 0 && dev < 64 && !attr_set[dev]) {

@@ -25,6 +25,8 @@
 // All waits are bounded (tc::mbar_wait): on a timeout the CTA raises an abort
 // flag, every thread unwinds, outstanding MMAs and loads are drained, TMEM is
 // freed and the device status word reports SSD_ERR_TIMEOUT.
+#include <atomic>
+
 #include <cuda.h>
 
 #include "ssd_common.cuh"
@@ -868,16 +870,15 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
 
 EncodeTiledFn encode_fn()
 {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
+    // looked up once per process (a function-local static is initialised thread-safely)
+    static const EncodeTiledFn fn = [] {
         void *f = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(f);
-    }
+            return reinterpret_cast<EncodeTiledFn>(f);
+        return (EncodeTiledFn) nullptr;
+    }();
     return fn;
 }
 
@@ -923,7 +924,7 @@ int launch_scan_tc(const ScanParams &p, cudaStream_t st)
         !encode_bf16(enc, &maps.C, p.C, gn, p.L, p.b, p.Crs, p.Cbs) ||
         !encode_bf16(enc, &maps.y, p.y, (int64_t)p.H * p.P, p.L, p.b, p.yrs, p.ybs))
         return 6;
-    static bool attr_set[64] = {false};
+    static std::atomic<bool> attr_set[64];   // set once per device (a repeat is harmless)
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {

@@ -4,6 +4,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <algorithm>
+#include <atomic>
 #include <cstring>
 #include <string>
 #include <vector>
@@ -36,18 +37,51 @@ int ok()
 __device__ unsigned int g_device_status;
 
 constexpr int kMaxDevices = 64;
-unsigned int *g_status_ptr[kMaxDevices] = {nullptr};
+// Looked up once per device.  Host threads may race on the first lookup; they all
+// store the same value, and the atomics make that race well defined.
+std::atomic<unsigned int *> g_status_ptr[kMaxDevices];
 
 unsigned int *status_ptr()
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    if (!g_status_ptr[dev]) {
+    unsigned int *sp = g_status_ptr[dev].load(std::memory_order_acquire);
+    if (!sp) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
-        g_status_ptr[dev] = static_cast<unsigned int *>(p);
+        sp = static_cast<unsigned int *>(p);
+        g_status_ptr[dev].store(sp, std::memory_order_release);
     }
-    return g_status_ptr[dev];
+    return sp;
+}
+
+// Test and diagnostic hooks, read from the environment once per process (the
+// first scan call) and documented in include/ssd.h:
+//   SSD_WAIT_LIMIT_MS   bound of every device-side wait, in ms (default 2000)
+//   SSD_TEST_DROP_UNIT  index of one work unit of the first scan call of the process
+//                       whose loads are never issued, so that its waits run out
+//                       (failure-detection test); later calls run normally
+//   SSD_SCAN_PATH       "generic" forces the CUDA-core scan kernels
+struct EnvHooks {
+    uint64_t wait_limit_ns;
+    int64_t test_drop_unit;
+    bool force_generic;
+};
+
+const EnvHooks &env_hooks()
+{
+    static const EnvHooks h = [] {
+        EnvHooks e{};
+        const char *lim = getenv("SSD_WAIT_LIMIT_MS");
+        const long long ms = lim ? atoll(lim) : 2000;
+        e.wait_limit_ns = (uint64_t)(ms > 0 ? ms : 2000) * 1000000ull;
+        const char *drop = getenv("SSD_TEST_DROP_UNIT");
+        e.test_drop_unit = drop ? atoll(drop) : -1;
+        const char *path = getenv("SSD_SCAN_PATH");
+        e.force_generic = path && strcmp(path, "generic") == 0;
+        return e;
+    }();
+    return h;
 }
 
 size_t elem_size(int dtype) { return dtype == SSD_BF16 ? 2 : 4; }
@@ -75,15 +109,15 @@ size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
 // among equal costs, the fewest stripes (less chain work, smaller workspace).
 int sm_count()
 {
-    static int cached[kMaxDevices] = {0};
+    static std::atomic<int> cached[kMaxDevices];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
-    if (cached[dev] == 0) {
-        int n = 0;
+    int n = cached[dev].load(std::memory_order_acquire);
+    if (n == 0) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-        cached[dev] = n;
+        cached[dev].store(n, std::memory_order_release);
     }
-    return cached[dev];
+    return n;
 }
 
 Plan make_plan(int b, int64_t L, int H, int P, int N, int Q)
@@ -207,16 +241,12 @@ int scan_impl(const ssd_scan_args *a, cudaStream_t st)
     }
     p.status = status_ptr();
     if (!p.status) return fail(SSD_ERR_LAUNCH, "no CUDA device available");
-    {
-        const char *lim = getenv("SSD_WAIT_LIMIT_MS");
-        const long long ms = lim ? atoll(lim) : 2000;
-        p.wait_limit_ns = (uint64_t)(ms > 0 ? ms : 2000) * 1000000ull;
-        const char *drop = getenv("SSD_TEST_DROP_UNIT");
-        p.test_drop_unit = drop ? atoll(drop) : -1;
-    }
+    const EnvHooks &hooks = env_hooks();
+    p.wait_limit_ns = hooks.wait_limit_ns;
+    static std::atomic<bool> drop_used{false};
+    p.test_drop_unit = (hooks.test_drop_unit >= 0 && !drop_used.exchange(true)) ? hooks.test_drop_unit : -1;
     // SSD_SCAN_PATH=generic forces the CUDA-core kernels (used to cross-check the paths)
-    const char *path = getenv("SSD_SCAN_PATH");
-    const bool force_generic = path && strcmp(path, "generic") == 0;
+    const bool force_generic = hooks.force_generic;
     rc = 6;
     if (!force_generic && ssd::tc_scan_supported(p, a->dtype)) rc = ssd::launch_scan_tc(p, st);
     if (rc == 6) rc = ssd::launch_scan_generic(p, a->dtype, st);

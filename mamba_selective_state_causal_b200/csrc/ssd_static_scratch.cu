@@ -23,6 +23,7 @@
 //  - The array's address is looked up (cudaGetSymbolAddress) by the first
 //    call made on each device, with that device current.  Make that first
 //    call before any stream capture on that device.
+#include <atomic>
 #include <cstdio>
 
 #include "../../include/ssd.h"
@@ -42,7 +43,9 @@ constexpr size_t kStaticScratchBytes = size_t(80) << 20;  // 80 MiB
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
 constexpr int kMaxDevices = 64;
-void *g_scratch_addr[kMaxDevices] = {nullptr};
+// One address per device.  Host threads making their first call together may
+// both look it up; they store the same value, and the atomics make that well defined.
+std::atomic<void *> g_scratch_addr[kMaxDevices];
 
 // Device address of the scratch on the current device (looked up once per device).
 int scratch_address(void **out)
@@ -51,7 +54,8 @@ int scratch_address(void **out)
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return ssd::set_error(SSD_ERR_LAUNCH, "static scratch: no usable current CUDA device");
-    if (!g_scratch_addr[dev]) {
+    void *addr = g_scratch_addr[dev].load(std::memory_order_acquire);
+    if (!addr) {
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_static_scratch);
         if (e != cudaSuccess || !p) {
@@ -60,9 +64,10 @@ int scratch_address(void **out)
                      cudaGetErrorString(e));
             return ssd::set_error(SSD_ERR_LAUNCH, msg);
         }
-        g_scratch_addr[dev] = p;
+        g_scratch_addr[dev].store(p, std::memory_order_release);
+        addr = p;
     }
-    *out = g_scratch_addr[dev];
+    *out = addr;
     return SSD_OK;
 }
 
