@@ -37,6 +37,11 @@ def _bind(path):
                                          f32p, f32p, f32p, f64p, f64p, f64p, f64p,
                                          f64p, f64p, f64p, f64p, f64p, f64p, f64p]
     lib.oracle_scan_backward.restype = None
+    lib.oracle_layer_backward.argtypes = [ctypes.c_int, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, i64, f32p, f32p, f32p, f32p, f32p, f32p, f32p,
+                                          f64p, f64p, f32p, f64p, f64p, f64p, ctypes.c_int,
+                                          f64p, f64p, f64p, f64p, f64p, f64p, f64p, f64p]
+    lib.oracle_layer_backward.restype = None
     lib.oracle_gated_rmsnorm.argtypes = [i64, ctypes.c_int, ctypes.c_int, f32p, i64, f32p, i64, f32p,
                                          ctypes.c_double, ctypes.c_int, f32p, i64]
     lib.oracle_gated_rmsnorm.restype = None
@@ -229,6 +234,67 @@ def scan_backward(x, B, C, dt, A, D, dy, h0=None, h_ckpt=None, dh_final=None, s=
         dC[:, :, grp[h]] += dC_h[:, :, h]
     return {"dx": dx, "dB": dB, "dC": dC, "ddt": ddt, "dA": dA_b.sum(0), "dD": dD_b.sum(0),
             "dh0": dh0, "dB_h": dB_h, "dC_h": dC_h}
+
+
+def layer_backward(u, w, dt, A, D, dy, bias=None, tail_in=None, h0=None, h_ckpt=None, conv_ckpt=None,
+                   dh_final=None, dtail_out=None, H=None, P=None, N=None, G=1, s=0, io_round="none"):
+    """Gradients of the whole layer (conv1d + SiLU, then the recurrence), fp64, by its
+    literal reverse mode.
+
+    Inputs as for ``layer``; dy [b, L, H, P], dh_final [b, H, P, N] and dtail_out
+    [b, 3, Cch] (each optional) are the loss's gradients with respect to y,
+    h_final and tail_out.  With ``h_ckpt`` [b, L//s, H, P, N] and ``conv_ckpt``
+    [b, L//s, 3, Cch] (the state and the 3 rows of u at every checkpoint) and
+    s > 0, each cell of s tokens is rebuilt from its own checkpoint and rows;
+    without them, from h0 and tail_in over the whole sequence.
+    Returns dict du [b, L, Cch], dtail_in [b, 3, Cch], dw [Cch, 4] and dbias
+    [Cch] (summed over b), ddt [b, L, H], dA and dD [H] (summed over b), dh0
+    [b, H, P, N].
+    """
+    lib = _load()
+    u = _f32(u)
+    b, L, cch = u.shape
+    assert cch == H * P + 2 * G * N
+    w = _f32(w)
+    assert w.shape == (cch, 4)
+    bias = _f32(bias)
+    tail_in = _f32(tail_in)
+    dt = _f32(dt)
+    assert dt.shape == (b, L, H)
+    A = _f32(A)
+    D = _f32(D)
+
+    def f64(a, shape):
+        if a is None:
+            return None
+        a = np.ascontiguousarray(a, dtype=np.float64)
+        assert a.shape == shape, (a.shape, shape)
+        return a
+
+    n_ckpt = L // s if s > 0 else 0
+    h0 = f64(h0, (b, H, P, N))
+    h_ckpt = f64(h_ckpt, (b, n_ckpt, H, P, N))
+    conv_ckpt = _f32(conv_ckpt)
+    if conv_ckpt is not None:
+        assert conv_ckpt.shape == (b, n_ckpt, 3, cch)
+    dy = f64(dy, (b, L, H, P))
+    dh_final = f64(dh_final, (b, H, P, N))
+    dtail_out = f64(dtail_out, (b, 3, cch))
+    du = np.empty((b, L, cch))
+    dtail_in = np.empty((b, 3, cch))
+    dw_b = np.empty((b, cch, 4))
+    dbias_b = np.empty((b, cch))
+    ddt = np.empty((b, L, H))
+    dA_b = np.empty((b, H))
+    dD_b = np.empty((b, H))
+    dh0 = np.empty((b, H, P, N))
+    lib.oracle_layer_backward(b, L, H, P, N, G, int(s), _p32(u), _p32(w), _p32(bias), _p32(tail_in),
+                              _p32(dt), _p32(A), _p32(D), _p64(h0), _p64(h_ckpt), _p32(conv_ckpt),
+                              _p64(dy), _p64(dh_final), _p64(dtail_out), IO_ROUND[io_round],
+                              _p64(du), _p64(dtail_in), _p64(dw_b), _p64(dbias_b), _p64(ddt),
+                              _p64(dA_b), _p64(dD_b), _p64(dh0))
+    return {"du": du, "dtail_in": dtail_in, "dw": dw_b.sum(0), "dbias": dbias_b.sum(0), "ddt": ddt,
+            "dA": dA_b.sum(0), "dD": dD_b.sum(0), "dh0": dh0}
 
 
 def gated_rmsnorm(y, z, w, eps=1e-5, group=None, io_round="none"):

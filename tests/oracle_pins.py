@@ -459,8 +459,110 @@ def pin_gated_norm_invariants():
     assert np.abs(got - ms / (ms + eps)).max() < 1e-6
 
 
+def _torch_layer_grads(u, w, bias, tail, dt, A, D, h0, dy, dhf, dto, H, P, N, G):
+    """Gradients of sum(dy*y) + sum(dhf*h_final) + sum(dto*tail_out) for the layer written
+    out in torch fp64 (grouped conv1d + silu, then the recurrence one token at a time), by
+    torch's autograd."""
+    f = lambda a: torch.tensor(np.asarray(a, dtype=np.float64), requires_grad=True)
+    ut, wt, bt, tt, dtt, At, Dt, h0t = map(f, (u, w, bias, tail, dt, A, D, h0))
+    b, L, cch = u.shape
+    seq = torch.cat([tt, ut], 1)                                                  # [b, L+3, cch]
+    z = torch.nn.functional.conv1d(seq.transpose(1, 2), wt.unsqueeze(1), bt, groups=cch)
+    v = torch.nn.functional.silu(z).transpose(1, 2)                             # [b, L, cch]
+    x = v[:, :, :H * P].reshape(b, L, H, P)
+    grp = [(h * G) // H for h in range(H)]
+    Bm = v[:, :, H * P:H * P + G * N].reshape(b, L, G, N)[:, :, grp]             # [b, L, H, N]
+    Cm = v[:, :, H * P + G * N:].reshape(b, L, G, N)[:, :, grp]
+    h = h0t
+    ys = []
+    for t in range(L):
+        a = torch.exp(dtt[:, t] * At)                                             # [b, H]
+        h = a[:, :, None, None] * h + dtt[:, t, :, None, None] * x[:, t, :, :, None] * Bm[:, t, :, None, :]
+        ys.append((h * Cm[:, t, :, None, :]).sum(-1) + Dt[None, :, None] * x[:, t])
+    y = torch.stack(ys, 1)
+    loss = (y * torch.from_numpy(dy)).sum() + (h * torch.from_numpy(dhf)).sum() + \
+        (seq[:, -3:] * torch.from_numpy(dto)).sum()
+    loss.backward()
+    return {"du": ut.grad.numpy(), "dtail_in": tt.grad.numpy(), "dw": wt.grad.numpy(),
+            "dbias": bt.grad.numpy(), "ddt": dtt.grad.numpy(), "dA": At.grad.numpy(),
+            "dD": Dt.grad.numpy(), "dh0": h0t.grad.numpy()}
+
+
+def _layer_grad_inputs(rng, b, L, H, P, N, G):
+    cch = H * P + 2 * G * N
+    u = rng.standard_normal((b, L, cch)).astype(np.float32)
+    w = rng.uniform(-0.5, 0.5, (cch, 4)).astype(np.float32)
+    bias = (rng.standard_normal(cch) * 0.3).astype(np.float32)
+    dt = rng.uniform(1e-2, 0.3, (b, L, H)).astype(np.float32)
+    A = (-np.exp(rng.uniform(0, math.log(16), H))).astype(np.float32)
+    D = rng.standard_normal(H).astype(np.float32)
+    h0 = rng.standard_normal((b, H, P, N))
+    tail = rng.standard_normal((b, 3, cch)).astype(np.float32)
+    dy = rng.standard_normal((b, L, H, P))
+    dhf = rng.standard_normal((b, H, P, N))
+    dto = rng.standard_normal((b, 3, cch))
+    return u, w, bias, tail, dt, A, D, h0, dy, dhf, dto
+
+
+def pin_layer_backward_torch_autograd():
+    """Every gradient of the layer's reverse mode (conv and scan) against torch autograd of
+    an independent fp64 torch statement of the same layer; two groups, and L < 3."""
+    rng = RNG(40)
+    for (b, L, H, P, N, G) in [(2, 23, 2, 3, 4, 1), (1, 17, 4, 2, 3, 2), (1, 2, 2, 2, 2, 1)]:
+        u, w, bias, tail, dt, A, D, h0, dy, dhf, dto = _layer_grad_inputs(rng, b, L, H, P, N, G)
+        got = oracle.layer_backward(u, w, dt, A, D, dy, bias=bias, tail_in=tail, h0=h0, dh_final=dhf,
+                                    dtail_out=dto, H=H, P=P, N=N, G=G, io_round="none")
+        ref = _torch_layer_grads(u, w, bias, tail, dt, A, D, h0, dy, dhf, dto, H, P, N, G)
+        for k in ref:
+            assert _rel(got[k], ref[k]) < 1e-10, (k, (b, L, H, P, N, G), _rel(got[k], ref[k]))
+
+
+def _conv_ckpt_from_u(u, s):
+    """The 3 rows of u before every checkpoint boundary: [b, L//s, 3, Cch]."""
+    b, L, cch = u.shape
+    n = L // s
+    return np.stack([u[:, (k + 1) * s - 3:(k + 1) * s] for k in range(n)], 1) if n else \
+        np.zeros((b, 0, 3, cch), np.float32)
+
+
+def pin_layer_backward_cells_equal_full():
+    """Rebuilding each cell of s tokens from its state checkpoint and its 3-row conv buffer
+    gives bitwise the gradients of the full reverse mode (exact checkpoints from the
+    forward oracle; f32 and bf16 rounding of v, a ragged last cell)."""
+    rng = RNG(41)
+    for (b, L, H, P, N, s, io) in [(2, 96, 2, 4, 3, 32, "f32"), (1, 100, 2, 3, 2, 16, "bf16"),
+                                   (1, 66, 2, 2, 3, 32, "f32")]:
+        u, w, bias, tail, dt, A, D, h0, dy, dhf, dto = _layer_grad_inputs(rng, b, L, H, P, N, 1)
+        fwd = oracle.layer(u, w, dt, A, D, bias, tail, h0, H=H, P=P, N=N, s=s, io_round=io)
+        kw = dict(bias=bias, tail_in=tail, h0=h0, dh_final=dhf, dtail_out=dto, H=H, P=P, N=N, s=s,
+                  io_round=io)
+        full = oracle.layer_backward(u, w, dt, A, D, dy, **kw)
+        cells = oracle.layer_backward(u, w, dt, A, D, dy, h_ckpt=fwd["h_ckpt"],
+                                      conv_ckpt=_conv_ckpt_from_u(u, s), **kw)
+        for k in full:
+            assert np.array_equal(full[k], cells[k]), (k, L, s)
+
+
+def pin_layer_backward_needs_conv_buffer():
+    """Negative control: cells rebuilt with the state checkpoints but without their conv
+    buffers (zeros) give wrong gradients of u and w."""
+    rng = RNG(42)
+    b, L, H, P, N, s = 1, 64, 2, 3, 2, 16
+    u, w, bias, tail, dt, A, D, h0, dy, dhf, dto = _layer_grad_inputs(rng, b, L, H, P, N, 1)
+    fwd = oracle.layer(u, w, dt, A, D, bias, tail, h0, H=H, P=P, N=N, s=s, io_round="f32")
+    kw = dict(bias=bias, tail_in=tail, h0=h0, dh_final=dhf, H=H, P=P, N=N, s=s, io_round="f32")
+    good = oracle.layer_backward(u, w, dt, A, D, dy, h_ckpt=fwd["h_ckpt"], conv_ckpt=_conv_ckpt_from_u(u, s), **kw)
+    bad = oracle.layer_backward(u, w, dt, A, D, dy, h_ckpt=fwd["h_ckpt"],
+                                conv_ckpt=np.zeros((b, L // s, 3, H * P + 2 * N), np.float32), **kw)
+    full = oracle.layer_backward(u, w, dt, A, D, dy, **kw)
+    assert np.array_equal(good["du"], full["du"])
+    assert _rel(bad["dw"], full["dw"]) > 1e-3 and _rel(bad["du"], full["du"]) > 1e-4
+
+
 PINS = [pin_quadratic_form, pin_A_zero_prefix_sum, pin_constant_geometric, pin_skip_only,
         pin_single_impulse, pin_linearity, pin_conv_torch, pin_conv_delta_weights,
         pin_bf16_rounding, pin_ckpt_indexing, pin_split_resume_bitwise,
         pin_resume_needs_conv_tail, pin_backward_finite_differences, pin_backward_cells_equal_full,
-        pin_backward_without_input, pin_gated_norm_torch, pin_gated_norm_invariants]
+        pin_backward_without_input, pin_gated_norm_torch, pin_gated_norm_invariants,
+        pin_layer_backward_torch_autograd, pin_layer_backward_cells_equal_full,
+        pin_layer_backward_needs_conv_buffer]

@@ -60,6 +60,23 @@ MUTANTS = {
                                     "const double scale = 1.0 / sqrt(ss / d + eps);"),
     "norm_weight_dropped": ("out[r * out_rs + c] = (float)round_io(v[c] * scale * (double)w[c], io_round);",
                             "out[r * out_rs + c] = (float)round_io(v[c] * scale, io_round);"),
+    # reverse mode of the whole layer (conv + SiLU, then the recurrence)
+    "layer_bwd_silu_grad_dropped": ("const double dz = dv[j * Cch + c] * (sg * (1.0 + zz * (1.0 - sg)));",
+                                    "const double dz = dv[j * Cch + c];"),
+    "layer_bwd_sigmoid_grad_instead": ("const double dz = dv[j * Cch + c] * (sg * (1.0 + zz * (1.0 - sg)));",
+                                       "const double dz = dv[j * Cch + c] * (sg * (1.0 - sg));"),
+    "layer_bwd_cell_buffer_zero": ("else val = conv_ckpt[(((int64_t)bi * n_ckpt + (k - 1)) * 3 + r) * Cch + c];",
+                                   "else val = 0.0;"),
+    "layer_bwd_tail_grad_dropped": ("else dtb[(3 + tt) * Cch + c] += wv * dz;",
+                                    "else dtb[(3 + tt) * Cch + c] += 0.0 * wv * dz;"),
+    "layer_bwd_dw_taps_flipped": ("dwb[c * ORACLE_CONV_K + kk] += dz * val;",
+                                  "dwb[c * ORACLE_CONV_K + (ORACLE_CONV_K - 1 - kk)] += dz * val;"),
+    "layer_bwd_dB_heads_not_summed": ("dvt[HP + grp * N + n] += dtv * b_acc;",
+                                      "dvt[HP + grp * N + n] = dtv * b_acc;"),
+    "layer_bwd_tail_out_grad_ignored": ("if (at >= 0) dub[at * Cch + c] += g;",
+                                        "if (at >= 0) dub[at * Cch + c] += 0.0 * g;"),
+    "layer_bwd_du_misplaced": ("if (tt >= 0) dub[tt * Cch + c] += wv * dz;",
+                               "if (tt >= 0) dub[t * Cch + c] += wv * dz;"),
     "bwd_adjoint_after_output": ("Gs[(int64_t)p * N + n] += dyt[p] * (double)Ct[n];",
                                  "Gs[(int64_t)p * N + n] += 0.0 * dyt[p] * (double)Ct[n];"),
 }
