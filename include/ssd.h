@@ -197,6 +197,10 @@ typedef struct ssd_stream_args {
     const float *dt_bias;
     int dt_softplus;
     float dt_min, dt_max;
+    /* conv_ckpt [b][floor(L/s)][3][C_ch] (I/O dtype) or NULL: the conv buffer at every
+     * checkpoint, conv_ckpt[bi,k,r,:] = u[bi,(k+1)*s-3+r,:] -- with h_ckpt[k] it is
+     * what a cell's exact recompute needs (ssd_layer_backward). */
+    void *conv_ckpt;
 } ssd_stream_args;
 
 /*
@@ -206,8 +210,21 @@ typedef struct ssd_stream_args {
  * previous (h_final, tail_out), equals one call on the whole sequence
  * (sequence-axis checkpointing of pith_extraction.key_machinery, with the
  * conv buffer the skeptic_critique asks for).
+ * With v == NULL the conv output is not returned, and the call needs a
+ * workspace of ssd_stream_workspace_size() bytes instead of
+ * ssd_scan_workspace_size(): on the tensor-core scan's shapes (bf16, P = 64,
+ * N = 128, Q = 128, heads in pairs per group) the conv of x is then fused into
+ * the scan kernels, which read x's columns of u directly, and only the B and
+ * C channels' conv output passes through memory (in the workspace); on other
+ * shapes the whole conv output is kept in the workspace.
+ * tail_out is written last, so it may alias tail_in.
  */
 SSD_API int ssd_stream_forward(const ssd_stream_args *args, ssd_stream_t stream);
+
+/* Bytes of workspace ssd_stream_forward needs when v is NULL (the scan's
+ * workspace plus the conv output that still passes through memory), for
+ * dtype SSD_F32 or SSD_BF16 on the current device. */
+SSD_API size_t ssd_stream_workspace_size(int b, int64_t L, int H, int P, int N, int G, int Q, int dtype);
 
 /*
  * Arguments of one decode step: a single new token of b independent streams
@@ -325,6 +342,73 @@ SSD_API int ssd_scan_backward(const ssd_scan_bwd_args *args, ssd_stream_t stream
 /* Bytes of workspace ssd_scan_backward needs: per 64-token chunk and head two
  * P x N fp32 states, and per token and head two N-vectors of fp32. */
 SSD_API size_t ssd_scan_backward_workspace_size(int b, int64_t L, int H, int P, int N);
+
+/*
+ * Arguments of the backward pass of the whole layer (see ssd_layer_backward).
+ *   dtype, b, L, H, P, N, G, u (+ strides), conv_w, conv_bias, tail_in, dt, A,
+ *   D, h0: as given to the forward (ssd_stream_forward; dt is the step size the
+ *   scan used, see ssd_scan_bwd_args).
+ *   h_ckpt [b][floor(L/s)][H][P][N] float and conv_ckpt [b][floor(L/s)][3][C_ch]
+ *           (I/O dtype): the forward's state checkpoints and conv buffers, s a
+ *           multiple of 64.  Both or neither: without them the states and the
+ *           conv are rebuilt from h0 and tail_in over the whole sequence.
+ *   dy      dLoss/dy laid out as for ssd_scan_bwd_args; dh_final [b][H][P][N]
+ *           float or NULL; dtail_out [b][3][C_ch] float or NULL: dLoss/d(tail_out).
+ * Outputs, float, contiguous, every element written:
+ *   du [b][L][C_ch] (row-major, C_ch = H*P + 2*G*N); dtail_in [b][3][C_ch] or
+ *   NULL; dconv_w [C_ch][4]; dconv_bias [C_ch] or NULL; ddt [b][L][H]; dA [H];
+ *   dD [H] or NULL; dh0 [b][H][P][N] or NULL.  They must not overlap the inputs.
+ *   workspace: at least ssd_layer_backward_workspace_size() bytes, 256-byte
+ *   aligned; contents on entry are ignored.
+ */
+typedef struct ssd_layer_bwd_args {
+    int dtype;
+    int b;
+    int64_t L;
+    int H, P, N, G;
+    int64_t s;
+    const void *u;
+    int64_t u_batch_stride, u_row_stride;
+    const float *conv_w;
+    const float *conv_bias;
+    const void *tail_in;
+    const void *conv_ckpt;
+    const float *dt;
+    const float *A;
+    const float *D;
+    const float *h0;
+    const float *h_ckpt;
+    const void *dy;
+    int64_t dy_batch_stride, dy_row_stride;
+    const float *dh_final;
+    const float *dtail_out;
+    float *du, *dtail_in, *dconv_w, *dconv_bias, *ddt, *dA, *dD, *dh0;
+    void *workspace;
+    size_t workspace_bytes;
+} ssd_layer_bwd_args;
+
+/*
+ * ssd_layer_backward -- gradients of a scalar loss through the whole layer
+ * (conv1d + SiLU, then the scan), given dLoss/dy, dLoss/dh_final and
+ * dLoss/d(tail_out).  With checkpoints, each cell of s tokens is rebuilt on its
+ * own: its conv output from ITS OWN rows of u and the 3-row conv buffer stored
+ * with the checkpoint that starts it (tail_in for the first cell), its states
+ * from that checkpoint's state (h0 for the first cell) -- MA-GC's grid-cell
+ * recompute (pith_extraction.key_machinery, "Algorithm 1"), exact because the
+ * conv buffer is stored along with the SSD state (skeptic_critique.headline).
+ * Then the scan's reverse mode (as ssd_scan_backward) and the conv's:
+ *   dz = dv silu'(z), du[t'] = sum_j w[:,3-j] dz[t'+j], dw[:,k] = sum_t dz[t] u[t-3+k],
+ *   dbias = sum_t dz[t]; the gradient of a cell's conv buffer is that of the
+ *   rows of u it copies (of tail_in for the first cell).
+ * The rounding of the conv output to the I/O dtype is taken as the identity.
+ * All arithmetic is fp32 on CUDA cores.  Asynchronous on `stream`.
+ */
+SSD_API int ssd_layer_backward(const ssd_layer_bwd_args *args, ssd_stream_t stream);
+
+/* Bytes of workspace ssd_layer_backward needs: the rebuilt conv output, the
+ * conv output's gradients (fp32), per 64-token block partial sums of the conv
+ * weight gradients, and the scan backward's own workspace. */
+SSD_API size_t ssd_layer_backward_workspace_size(int b, int64_t L, int H, int P, int N, int G, int dtype);
 
 /*
  * ssd_gated_rmsnorm_forward -- the output norm of the Mamba-2 block on the

@@ -59,7 +59,8 @@ class StreamArgs(ctypes.Structure):
                 ("h_final", _vp), ("h_ckpt", _vp),
                 ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
                 ("dt_bias", _vp), ("dt_softplus", ctypes.c_int),
-                ("dt_min", ctypes.c_float), ("dt_max", ctypes.c_float)]
+                ("dt_min", ctypes.c_float), ("dt_max", ctypes.c_float),
+                ("conv_ckpt", _vp)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -85,6 +86,20 @@ class ScanBwdArgs(ctypes.Structure):
                 ("dh_final", _vp),
                 ("dx", _vp), ("dB", _vp), ("dC", _vp), ("ddt", _vp), ("dA", _vp), ("dD", _vp),
                 ("dh0", _vp),
+                ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
+
+
+class LayerBwdArgs(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int), ("b", ctypes.c_int), ("L", _i64),
+                ("H", ctypes.c_int), ("P", ctypes.c_int), ("N", ctypes.c_int),
+                ("G", ctypes.c_int), ("s", _i64),
+                ("u", _vp), ("u_batch_stride", _i64), ("u_row_stride", _i64),
+                ("conv_w", _vp), ("conv_bias", _vp), ("tail_in", _vp), ("conv_ckpt", _vp),
+                ("dt", _vp), ("A", _vp), ("D", _vp), ("h0", _vp), ("h_ckpt", _vp),
+                ("dy", _vp), ("dy_batch_stride", _i64), ("dy_row_stride", _i64),
+                ("dh_final", _vp), ("dtail_out", _vp),
+                ("du", _vp), ("dtail_in", _vp), ("dconv_w", _vp), ("dconv_bias", _vp),
+                ("ddt", _vp), ("dA", _vp), ("dD", _vp), ("dh0", _vp),
                 ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
 
 
@@ -116,6 +131,14 @@ def lib():
         L.ssd_scan_backward_workspace_size.argtypes = [ctypes.c_int, _i64, ctypes.c_int, ctypes.c_int,
                                                        ctypes.c_int]
         L.ssd_scan_backward_workspace_size.restype = ctypes.c_size_t
+        L.ssd_layer_backward.argtypes = [ctypes.POINTER(LayerBwdArgs), _vp]
+        L.ssd_layer_backward.restype = ctypes.c_int
+        L.ssd_layer_backward_workspace_size.argtypes = [ctypes.c_int, _i64, ctypes.c_int, ctypes.c_int,
+                                                        ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        L.ssd_layer_backward_workspace_size.restype = ctypes.c_size_t
+        L.ssd_stream_workspace_size.argtypes = [ctypes.c_int, _i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        L.ssd_stream_workspace_size.restype = ctypes.c_size_t
         L.ssd_scan_workspace_size.argtypes = [ctypes.c_int, _i64, ctypes.c_int, ctypes.c_int,
                                               ctypes.c_int, ctypes.c_int]
         L.ssd_scan_workspace_size.restype = ctypes.c_size_t
@@ -173,6 +196,11 @@ def _f32(t, name):
 
 def workspace_size(b, L, H, P, N, Q):
     return int(lib().ssd_scan_workspace_size(b, L, H, P, N, Q))
+
+
+def stream_workspace_size(b, L, H, P, N, G, Q, dtype):
+    """Workspace bytes of stream_forward without the conv output (keep_v=False)."""
+    return int(lib().ssd_stream_workspace_size(b, L, H, P, N, G, Q, dtype))
 
 
 def alloc_workspace(b, L, H, P, N, Q, device=None):
@@ -269,13 +297,18 @@ def scan_forward(x, B, C, dt, A, D=None, h0=None, *, H, G=1, Q=128, s=0, y=None,
 def stream_forward(u, conv_w, dt, A, D=None, *, H, P, N, G=1, Q=128, s=0, conv_bias=None,
                    tail_in=None, tail_out=None, h0=None, v=None, y=None, h_final=None,
                    h_ckpt=None, workspace=None, stream=None, dt_bias=None, dt_softplus=False,
-                   dt_limit=None):
-    """One streamed segment: conv (tail_in -> tail_out), then scan (h0 -> h_final)."""
+                   dt_limit=None, conv_ckpt=None, keep_v=True):
+    """One streamed segment: conv (tail_in -> tail_out), then scan (h0 -> h_final).
+
+    conv_ckpt: a [b, L//s, 3, C_ch] tensor (I/O dtype) to receive the conv buffer at
+    every checkpoint, True to allocate one, or None.  keep_v=False (and v None):
+    the conv output is not returned, and on the tensor-core shapes the conv of x is
+    fused into the scan kernels (the workspace is then ssd_stream_workspace_size)."""
     _cuda(u, conv_w, dt, A, D, conv_bias, tail_in, tail_out, h0, v, y, h_final, h_ckpt, workspace)
     b, L, cch = u.shape
     assert cch == H * P + 2 * G * N, "u must hold x|B|C channels"
     dev = u.device
-    if v is None:
+    if v is None and keep_v:
         v = torch.empty_like(u)
     if y is None:
         y = torch.empty(b, L, H, P, dtype=u.dtype, device=dev)
@@ -286,14 +319,21 @@ def stream_forward(u, conv_w, dt, A, D=None, *, H, P, N, G=1, Q=128, s=0, conv_b
     if h_ckpt is None and s > 0:
         h_ckpt = torch.empty(b, L // s, H, P, N, dtype=torch.float32, device=dev)
     if workspace is None:
-        workspace = alloc_workspace(b, L, H, P, N, Q, dev)
+        if v is None:
+            n = stream_workspace_size(b, L, H, P, N, G, Q, _dtype_code(u))
+            workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=dev)
+        else:
+            workspace = alloc_workspace(b, L, H, P, N, Q, dev)
+    if conv_ckpt is True:
+        conv_ckpt = torch.empty(b, L // s if s > 0 else 0, 3, cch, dtype=u.dtype, device=dev)
     a = StreamArgs()
     a.dtype = _dtype_code(u); a.b = b; a.L = L; a.H = H; a.P = P; a.N = N; a.G = G; a.Q = Q; a.s = s
     a.u = u.data_ptr(); a.u_batch_stride = u.stride(0); a.u_row_stride = u.stride(1)
     a.conv_w = conv_w.data_ptr(); a.conv_bias = conv_bias.data_ptr() if conv_bias is not None else None
     a.tail_in = tail_in.data_ptr() if tail_in is not None else None
     a.tail_out = tail_out.data_ptr()
-    a.v = v.data_ptr(); a.v_batch_stride = v.stride(0); a.v_row_stride = v.stride(1)
+    if v is not None:
+        a.v = v.data_ptr(); a.v_batch_stride = v.stride(0); a.v_row_stride = v.stride(1)
     a.dt = dt.data_ptr(); a.A = A.data_ptr(); a.D = D.data_ptr() if D is not None else None
     a.h0 = h0.data_ptr() if h0 is not None else None
     y2 = y.view(b, L, H * P)
@@ -302,8 +342,9 @@ def stream_forward(u, conv_w, dt, A, D=None, *, H, P, N, G=1, Q=128, s=0, conv_b
     a.h_ckpt = h_ckpt.data_ptr() if h_ckpt is not None else None
     a.workspace = workspace.data_ptr(); a.workspace_bytes = workspace.numel()
     _set_dt(a, dt_bias, dt_softplus, dt_limit)
+    a.conv_ckpt = conv_ckpt.data_ptr() if conv_ckpt is not None else None
     _check(lib().ssd_stream_forward(ctypes.byref(a), _stream(stream)))
-    return {"v": v, "y": y, "h_final": h_final, "h_ckpt": h_ckpt, "tail_out": tail_out}
+    return {"v": v, "y": y, "h_final": h_final, "h_ckpt": h_ckpt, "tail_out": tail_out, "conv_ckpt": conv_ckpt}
 
 
 def decode_step(u, conv_w, dt, A, D=None, *, H, P, N, G=1, conv_bias=None, tail_in=None,
@@ -386,6 +427,61 @@ def scan_backward(x, B, C, dt, A, D, dy, h0=None, h_ckpt=None, dh_final=None, *,
     a.workspace = workspace.data_ptr(); a.workspace_bytes = workspace.numel()
     _check(lib().ssd_scan_backward(ctypes.byref(a), _stream(stream)))
     return o
+
+
+def layer_backward_workspace_size(b, L, H, P, N, G=1, dtype=SSD_BF16):
+    return int(lib().ssd_layer_backward_workspace_size(b, L, H, P, N, G, dtype))
+
+
+def layer_backward(u, conv_w, dt, A, D, dy, *, H, P, N, G=1, s=0, conv_bias=None, tail_in=None, h0=None,
+                   h_ckpt=None, conv_ckpt=None, dh_final=None, dtail_out=None, workspace=None, out=None,
+                   stream=None):
+    """Gradients through the whole layer (conv1d + SiLU, then the scan): returns dict du,
+    dtail_in, dconv_w, dconv_bias, ddt, dA, dD, dh0 (float32).
+
+    u, conv_w, conv_bias, tail_in, dt, A, D, h0: the forward's inputs (as for
+    stream_forward); dy: [b, L, >=H*P] (I/O dtype); dh_final [b, H, P, N] and
+    dtail_out [b, 3, C_ch] float32 or None.  h_ckpt [b, L//s, H, P, N] and conv_ckpt
+    [b, L//s, 3, C_ch] (the forward's checkpoints, s a multiple of 64) rebuild each cell
+    of s tokens on its own; without them the whole sequence is rebuilt from h0, tail_in.
+    """
+    _cuda(u, conv_w, dt, A, D, dy, conv_bias, tail_in, h0, h_ckpt, conv_ckpt, dh_final, dtail_out, workspace)
+    b, L, cch = u.shape
+    assert cch == H * P + 2 * G * N, "u must hold x|B|C channels"
+    dev = u.device
+    o = dict(out or {})
+    shapes = {"du": (b, L, cch), "dtail_in": (b, 3, cch), "dconv_w": (cch, 4), "dconv_bias": (cch,),
+              "ddt": (b, L, H), "dA": (H,), "dD": (H,), "dh0": (b, H, P, N)}
+    for k, shp in shapes.items():
+        if k not in o:
+            o[k] = torch.empty(shp, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(layer_backward_workspace_size(b, L, H, P, N, G, _dtype_code(u)), 1),
+                                dtype=torch.uint8, device=dev)
+    for t, n in ((conv_w, "conv_w"), (conv_bias, "conv_bias"), (dt, "dt"), (A, "A"), (D, "D"), (h0, "h0"),
+                 (h_ckpt, "h_ckpt"), (dh_final, "dh_final"), (dtail_out, "dtail_out"),
+                 *((o[k], k) for k in shapes if o[k] is not None)):
+        _f32(t, n)
+    a = LayerBwdArgs()
+    a.dtype = _dtype_code(u); a.b = b; a.L = L; a.H = H; a.P = P; a.N = N; a.G = G
+    a.s = s if h_ckpt is not None else 0
+    a.u = u.data_ptr(); a.u_batch_stride = u.stride(0); a.u_row_stride = u.stride(1)
+    a.conv_w = conv_w.data_ptr(); a.conv_bias = _vp_of(conv_bias); a.tail_in = _vp_of(tail_in)
+    a.conv_ckpt = _vp_of(conv_ckpt)
+    a.dt = dt.data_ptr(); a.A = A.data_ptr(); a.D = _vp_of(D); a.h0 = _vp_of(h0); a.h_ckpt = _vp_of(h_ckpt)
+    dy3 = dy.reshape(b, L, -1) if dy.dim() == 4 else dy
+    a.dy = dy3.data_ptr(); a.dy_batch_stride = dy3.stride(0); a.dy_row_stride = dy3.stride(1)
+    a.dh_final = _vp_of(dh_final); a.dtail_out = _vp_of(dtail_out)
+    a.du = o["du"].data_ptr(); a.dtail_in = _vp_of(o["dtail_in"]); a.dconv_w = o["dconv_w"].data_ptr()
+    a.dconv_bias = _vp_of(o["dconv_bias"]); a.ddt = o["ddt"].data_ptr(); a.dA = o["dA"].data_ptr()
+    a.dD = _vp_of(o["dD"]); a.dh0 = _vp_of(o["dh0"])
+    a.workspace = workspace.data_ptr(); a.workspace_bytes = workspace.numel()
+    _check(lib().ssd_layer_backward(ctypes.byref(a), _stream(stream)))
+    return o
+
+
+def _vp_of(t):
+    return None if t is None else t.data_ptr()
 
 
 def gated_rmsnorm(y, z, weight, eps=1e-5, group_size=0, out=None, stream=None):

@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(kConvThreads, 2) conv1d_silu_kernel(ConvParams
     float w0[V], w1[V], w2[V], w3[V], bs[V];
     const T *u = reinterpret_cast<const T *>(p.u) + bi * p.ubs + c0;
     T *v = reinterpret_cast<T *>(p.v) + bi * p.vbs + c0;
-    const T *tin = p.tail_in ? reinterpret_cast<const T *>(p.tail_in) + bi * 3 * p.C_ch + c0 : nullptr;
+    const T *tin = p.tail_in ? reinterpret_cast<const T *>(p.tail_in) + bi * 3 * p.tail_rs + c0 : nullptr;
     const int64_t t0 = tb * kTokensPerThread;
     const int n = active ? (int)(min(p.L, t0 + kTokensPerThread) - t0) : 0;
     Vec16 *slot = &ring[0][threadIdx.x];
@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(kConvThreads, 2) conv1d_silu_kernel(ConvParams
             if (pos >= 0) {
                 IO::unpack(ld_stream(u + pos * p.urs), dst[k]);
             } else if (tin) {
-                IO::unpack(*reinterpret_cast<const Vec16 *>(tin + (3 + pos) * p.C_ch), dst[k]);
+                IO::unpack(*reinterpret_cast<const Vec16 *>(tin + (3 + pos) * p.tail_rs), dst[k]);
             } else {
 #pragma unroll
                 for (int i = 0; i < V; ++i) dst[k][i] = 0.0f;
@@ -188,17 +188,17 @@ __global__ void conv_tail_kernel(ConvParams p)
     const int64_t bi = gid / p.C_ch;
     const int c = (int)(gid % p.C_ch);
     const T *u = reinterpret_cast<const T *>(p.u) + bi * p.ubs + c;
-    const T *tin = p.tail_in ? reinterpret_cast<const T *>(p.tail_in) + bi * 3 * p.C_ch + c : nullptr;
+    const T *tin = p.tail_in ? reinterpret_cast<const T *>(p.tail_in) + bi * 3 * p.tail_rs + c : nullptr;
     T vals[3];
 #pragma unroll
     for (int r = 0; r < 3; ++r) {
         const int64_t pos = p.L - 3 + r;
         if (pos >= 0) vals[r] = u[pos * p.urs];
-        else vals[r] = tin ? tin[(3 + pos) * p.C_ch] : from_f32<T>(0.0f);
+        else vals[r] = tin ? tin[(3 + pos) * p.tail_rs] : from_f32<T>(0.0f);
     }
-    T *tout = reinterpret_cast<T *>(p.tail_out) + bi * 3 * p.C_ch + c;
+    T *tout = reinterpret_cast<T *>(p.tail_out) + bi * 3 * p.tail_rs + c;
 #pragma unroll
-    for (int r = 0; r < 3; ++r) tout[r * p.C_ch] = vals[r];
+    for (int r = 0; r < 3; ++r) tout[r * p.tail_rs] = vals[r];
 }
 
 template <typename T>
@@ -232,7 +232,87 @@ int launch_conv_t(const ConvParams &p, cudaStream_t st)
     return cudaGetLastError() == cudaSuccess ? 0 : 7;
 }
 
+// The conv output rebuilt cell by cell for the backward pass: v[bi, t, c] from
+// the cell's own rows of u and its conv buffer (cell_val), with the forward
+// kernel's arithmetic (same order of fused multiply-adds, same SiLU), so that a
+// cell rebuilt from exact buffers reproduces the forward's v bit for bit.
+template <typename T>
+__global__ void conv_cells_kernel(ConvBwdParams p)
+{
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= (int64_t)p.b * p.L * p.C_ch) return;
+    const int c = (int)(gid % p.C_ch);
+    const int64_t t = (gid / p.C_ch) % p.L;
+    const int64_t bi = gid / ((int64_t)p.C_ch * p.L);
+    const float4 wq = __ldg(reinterpret_cast<const float4 *>(p.w) + c);
+    float z = p.bias ? __ldg(p.bias + c) : 0.0f;
+    z = fmaf(wq.x, cell_val<T>(p, bi, t, t - 3, c), z);
+    z = fmaf(wq.y, cell_val<T>(p, bi, t, t - 2, c), z);
+    z = fmaf(wq.z, cell_val<T>(p, bi, t, t - 1, c), z);
+    z = fmaf(wq.w, cell_val<T>(p, bi, t, t, c), z);
+    reinterpret_cast<T *>(p.v)[(bi * p.L + t) * p.C_ch + c] = from_f32<T>(VecIO<T>::silu(z));
+}
+
+// conv_ckpt[bi, k, r, c] = u[bi, (k+1) s - 3 + r, c]: the conv buffer at every checkpoint
+template <typename T>
+__global__ void conv_ckpt_kernel(const T *u, int64_t ubs, int64_t urs, T *out, int b, int64_t n_ckpt, int C_ch,
+                                 int64_t s)
+{
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= (int64_t)b * n_ckpt * 3 * C_ch) return;
+    const int c = (int)(gid % C_ch);
+    const int64_t r = (gid / C_ch) % 3;
+    const int64_t k = (gid / ((int64_t)3 * C_ch)) % n_ckpt;
+    const int64_t bi = gid / ((int64_t)3 * C_ch * n_ckpt);
+    out[gid] = u[bi * ubs + ((k + 1) * s - 3 + r) * urs + c];
+}
+
 }  // namespace
+
+int launch_conv_cells(const ConvBwdParams &p, int dtype, cudaStream_t st)
+{
+    const int64_t n = (int64_t)p.b * p.L * p.C_ch;
+    if (n == 0) return 0;
+    const int64_t blocks = (n + 255) / 256;
+    if (blocks > 0x7fffffffLL) return 2;
+    prof_begin(st, kKConvCells);
+    if (dtype == 1) conv_cells_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(p);
+    else conv_cells_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(p);
+    prof_end(st, kKConvCells);
+    return cudaGetLastError() == cudaSuccess ? 0 : 7;
+}
+
+int launch_conv_ckpt(const void *u, int64_t ubs, int64_t urs, void *conv_ckpt, int b, int64_t L, int C_ch,
+                     int64_t s, int dtype, cudaStream_t st)
+{
+    const int64_t n_ckpt = s > 0 ? L / s : 0;
+    const int64_t n = (int64_t)b * n_ckpt * 3 * C_ch;
+    if (n == 0) return 0;
+    const int64_t blocks = (n + 255) / 256;
+    if (blocks > 0x7fffffffLL) return 2;
+    prof_begin(st, kKConvCkpt);
+    if (dtype == 1)
+        conv_ckpt_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
+            reinterpret_cast<const __nv_bfloat16 *>(u), ubs, urs, reinterpret_cast<__nv_bfloat16 *>(conv_ckpt), b,
+            n_ckpt, C_ch, s);
+    else
+        conv_ckpt_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<const float *>(u), ubs, urs,
+                                                                 reinterpret_cast<float *>(conv_ckpt), b, n_ckpt,
+                                                                 C_ch, s);
+    prof_end(st, kKConvCkpt);
+    return cudaGetLastError() == cudaSuccess ? 0 : 7;
+}
+
+int launch_conv_tail(const ConvParams &p, int dtype, cudaStream_t st)
+{
+    if (!p.tail_out || p.b <= 0) return 0;
+    const int64_t n = (int64_t)p.b * p.C_ch;
+    prof_begin(st, kKConvTail);
+    if (dtype == 1) conv_tail_kernel<__nv_bfloat16><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p);
+    else conv_tail_kernel<float><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p);
+    prof_end(st, kKConvTail);
+    return cudaGetLastError() == cudaSuccess ? 0 : 7;
+}
 
 int launch_conv(const ConvParams &p, int dtype, cudaStream_t st)
 {

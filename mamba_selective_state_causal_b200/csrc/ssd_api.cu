@@ -183,7 +183,17 @@ int check_rows(const char *name, const void *ptr, int64_t bs, int64_t rs, int64_
     return SSD_OK;
 }
 
-int scan_impl(const ssd_scan_args *a, cudaStream_t st)
+// The conv of x fused into the tensor-core scan (ssd_stream_forward without v): x is read
+// from u's x columns and turned into silu(conv(u)) inside the scan kernels.
+struct FusedConv {
+    const void *u;
+    int64_t ubs, urs;
+    const float *w, *bias;
+    const void *tail;
+    int C_ch;
+};
+
+int scan_impl(const ssd_scan_args *a, cudaStream_t st, const FusedConv *fc = nullptr)
 {
     if (!a) return fail(SSD_ERR_NULL, "args is NULL");
     int rc = check_scan_shape(a->dtype, a->b, a->L, a->H, a->P, a->N, a->G, a->Q, a->s);
@@ -241,6 +251,10 @@ int scan_impl(const ssd_scan_args *a, cudaStream_t st)
     }
     p.status = status_ptr();
     if (!p.status) return fail(SSD_ERR_LAUNCH, "no CUDA device available");
+    if (fc) {
+        p.conv_u = fc->u; p.conv_ubs = fc->ubs; p.conv_urs = fc->urs;
+        p.conv_w = fc->w; p.conv_bias = fc->bias; p.conv_tail = fc->tail; p.conv_cch = fc->C_ch;
+    }
     const EnvHooks &hooks = env_hooks();
     p.wait_limit_ns = hooks.wait_limit_ns;
     static std::atomic<bool> drop_used{false};
@@ -249,6 +263,7 @@ int scan_impl(const ssd_scan_args *a, cudaStream_t st)
     const bool force_generic = hooks.force_generic;
     rc = 6;
     if (!force_generic && ssd::tc_scan_supported(p, a->dtype)) rc = ssd::launch_scan_tc(p, st);
+    if (fc && rc == 6) return fail(SSD_ERR_UNSUPPORTED, "the fused conv needs the tensor-core scan (dt 8-byte aligned)");
     if (rc == 6) rc = ssd::launch_scan_generic(p, a->dtype, st);
     if (rc == 6) return fail(SSD_ERR_UNSUPPORTED, "no GPU kernel for this shape (P=%d N=%d Q=%d)", a->P, a->N, a->Q);
     if (rc) return fail(SSD_ERR_LAUNCH, "scan launch failed: %s", cudaGetErrorString(cudaGetLastError()));
@@ -351,6 +366,119 @@ int scan_bwd_impl(const ssd_scan_bwd_args *a, cudaStream_t st)
     return ok();
 }
 
+// Layer backward workspace: the rebuilt conv output v [b][L][C_ch] (I/O dtype); dx [b][L][H*P],
+// dB, dC [b][L][G*N] fp32; the conv weight partial sums [b*blocks][C_ch][4] and [b*blocks][C_ch]
+// fp32; then the scan backward's workspace.
+struct LayerBwdPlan {
+    size_t off_v = 0, off_dx = 0, off_dB = 0, off_dC = 0, off_pw = 0, off_pb = 0, off_scan = 0, bytes = 0;
+};
+
+LayerBwdPlan make_layer_bwd_plan(int b, int64_t L, int H, int P, int N, int G, int dtype)
+{
+    LayerBwdPlan pl;
+    if (b <= 0 || L <= 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0) return pl;
+    const size_t cch = (size_t)H * P + 2 * (size_t)G * N;
+    const size_t rows = (size_t)b * L;
+    const size_t parts = (size_t)b * ssd::conv_bwd_blocks(L);
+    pl.off_v = 0;
+    pl.off_dx = round256(rows * cch * elem_size(dtype));
+    pl.off_dB = pl.off_dx + round256(sizeof(float) * rows * H * P);
+    pl.off_dC = pl.off_dB + round256(sizeof(float) * rows * G * N);
+    pl.off_pw = pl.off_dC + round256(sizeof(float) * rows * G * N);
+    pl.off_pb = pl.off_pw + round256(sizeof(float) * parts * cch * 4);
+    pl.off_scan = pl.off_pb + round256(sizeof(float) * parts * cch);
+    pl.bytes = pl.off_scan + make_bwd_plan(b, L, H, P, N).bytes;
+    return pl;
+}
+
+int layer_bwd_impl(const ssd_layer_bwd_args *a, cudaStream_t st)
+{
+    if (!a) return fail(SSD_ERR_NULL, "args is NULL");
+    const bool ck = a->h_ckpt != nullptr || a->conv_ckpt != nullptr;
+    if ((a->h_ckpt == nullptr) != (a->conv_ckpt == nullptr))
+        return fail(SSD_ERR_NULL, "h_ckpt and conv_ckpt must be given together");
+    int rc = check_scan_shape(a->dtype, a->b, a->L, a->H, a->P, a->N, a->G, 64, ck ? a->s : 0);
+    if (rc) return rc;
+    if (ck && a->s <= 0) return fail(SSD_ERR_SHAPE, "checkpoints given with stride s=%lld", (long long)a->s);
+    if (a->b == 0) return ok();
+    const int HP = a->H * a->P, GN = a->G * a->N;
+    const int C_ch = HP + 2 * GN;
+    const size_t es = elem_size(a->dtype);
+    if (!a->dconv_w || !a->dA || !a->du || !a->ddt) return fail(SSD_ERR_NULL, "du, dconv_w, ddt and dA must not be NULL");
+    if (!a->conv_w || !aligned16(a->conv_w) || !aligned16(a->dconv_w))
+        return fail(SSD_ERR_ALIGN, "conv_w and dconv_w must be given, 16-byte aligned");
+    const void *vec[] = {a->tail_in, a->conv_ckpt, a->du, a->dtail_in, a->h0, a->h_ckpt, a->dh_final, a->dh0};
+    for (const void *v : vec)
+        if (v && !aligned16(v)) return fail(SSD_ERR_ALIGN, "buffers must be 16-byte aligned");
+    if (a->L == 0) {
+        // no token: tail_out is tail_in, every other gradient is zero or passes through
+        const size_t tail_bytes = sizeof(float) * (size_t)a->b * 3 * C_ch;
+        const size_t state_bytes = sizeof(float) * (size_t)a->b * a->H * a->P * a->N;
+        cudaError_t e = cudaMemsetAsync(a->dconv_w, 0, sizeof(float) * 4 * C_ch, st);
+        if (e == cudaSuccess && a->dconv_bias) e = cudaMemsetAsync(a->dconv_bias, 0, sizeof(float) * C_ch, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(a->dA, 0, sizeof(float) * a->H, st);
+        if (e == cudaSuccess && a->dD) e = cudaMemsetAsync(a->dD, 0, sizeof(float) * a->H, st);
+        if (e == cudaSuccess && a->dtail_in)
+            e = a->dtail_out ? cudaMemcpyAsync(a->dtail_in, a->dtail_out, tail_bytes, cudaMemcpyDeviceToDevice, st)
+                             : cudaMemsetAsync(a->dtail_in, 0, tail_bytes, st);
+        if (e == cudaSuccess && a->dh0)
+            e = a->dh_final ? cudaMemcpyAsync(a->dh0, a->dh_final, state_bytes, cudaMemcpyDeviceToDevice, st)
+                            : cudaMemsetAsync(a->dh0, 0, state_bytes, st);
+        if (e != cudaSuccess) return fail(SSD_ERR_LAUNCH, "%s", cudaGetErrorString(e));
+        return ok();
+    }
+    if ((rc = check_rows("u", a->u, a->u_batch_stride, a->u_row_stride, C_ch, a->b, a->L, a->dtype, true))) return rc;
+    (void)es;
+    const LayerBwdPlan pl = make_layer_bwd_plan(a->b, a->L, a->H, a->P, a->N, a->G, a->dtype);
+    if (!a->workspace || a->workspace_bytes < pl.bytes)
+        return fail(SSD_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", pl.bytes,
+                    a->workspace ? a->workspace_bytes : (size_t)0);
+    if ((reinterpret_cast<uintptr_t>(a->workspace) & 255u) != 0)
+        return fail(SSD_ERR_ALIGN, "workspace must be 256-byte aligned");
+    char *ws = static_cast<char *>(a->workspace);
+    ssd::ConvBwdParams cp{};
+    cp.b = a->b; cp.L = a->L; cp.C_ch = C_ch; cp.HP = HP; cp.GN = GN;
+    cp.u = a->u; cp.ubs = a->u_batch_stride; cp.urs = a->u_row_stride;
+    cp.w = a->conv_w; cp.bias = a->conv_bias; cp.tail_in = a->tail_in;
+    cp.conv_ckpt = ck ? a->conv_ckpt : nullptr;
+    cp.s = ck ? a->s : 0;
+    cp.n_ckpt = ck ? a->L / a->s : 0;
+    cp.v = ws + pl.off_v;
+    cp.dx = reinterpret_cast<float *>(ws + pl.off_dx);
+    cp.dB = reinterpret_cast<float *>(ws + pl.off_dB);
+    cp.dC = reinterpret_cast<float *>(ws + pl.off_dC);
+    cp.dtail_out = a->dtail_out;
+    cp.du = a->du; cp.dtail_in = a->dtail_in;
+    cp.ws_dw = reinterpret_cast<float *>(ws + pl.off_pw);
+    cp.ws_dbias = reinterpret_cast<float *>(ws + pl.off_pb);
+    cp.dw = a->dconv_w; cp.dbias = a->dconv_bias;
+    // 1. every cell's conv output from its own rows of u and its conv buffer
+    rc = ssd::launch_conv_cells(cp, a->dtype, st);
+    if (rc == 2) return fail(SSD_ERR_SHAPE, "layer backward grid too large");
+    if (rc) return fail(SSD_ERR_LAUNCH, "conv recompute launch failed: %s", cudaGetErrorString(cudaGetLastError()));
+    // 2. the scan's reverse mode on that output's x, B and C, each cell from its state checkpoint
+    ssd_scan_bwd_args sb{};
+    sb.dtype = a->dtype; sb.b = a->b; sb.L = a->L; sb.H = a->H; sb.P = a->P; sb.N = a->N; sb.G = a->G;
+    sb.s = ck ? a->s : 0;
+    const char *v = static_cast<const char *>(cp.v);
+    sb.x = v; sb.x_batch_stride = a->L * C_ch; sb.x_row_stride = C_ch;
+    sb.B = v + es * HP; sb.B_batch_stride = a->L * C_ch; sb.B_row_stride = C_ch;
+    sb.C = v + es * (HP + GN); sb.C_batch_stride = a->L * C_ch; sb.C_row_stride = C_ch;
+    sb.dt = a->dt; sb.A = a->A; sb.D = a->D; sb.h0 = a->h0; sb.h_ckpt = ck ? a->h_ckpt : nullptr;
+    sb.dy = a->dy; sb.dy_batch_stride = a->dy_batch_stride; sb.dy_row_stride = a->dy_row_stride;
+    sb.dh_final = a->dh_final;
+    sb.dx = const_cast<float *>(cp.dx); sb.dB = const_cast<float *>(cp.dB); sb.dC = const_cast<float *>(cp.dC);
+    sb.ddt = a->ddt; sb.dA = a->dA; sb.dD = a->dD; sb.dh0 = a->dh0;
+    sb.workspace = ws + pl.off_scan; sb.workspace_bytes = pl.bytes - pl.off_scan;
+    rc = scan_bwd_impl(&sb, st);
+    if (rc) return rc;
+    // 3. the conv's reverse mode
+    rc = ssd::launch_conv_backward(cp, a->dtype, st);
+    if (rc == 2) return fail(SSD_ERR_SHAPE, "layer backward grid too large");
+    if (rc) return fail(SSD_ERR_LAUNCH, "conv backward launch failed: %s", cudaGetErrorString(cudaGetLastError()));
+    return ok();
+}
+
 int conv_impl(const void *u, int64_t ubs, int64_t urs, const float *w, const float *bias,
               const void *tail_in, void *tail_out, void *v, int64_t vbs, int64_t vrs,
               int b, int64_t L, int C_ch, int dtype, cudaStream_t st)
@@ -374,6 +502,7 @@ int conv_impl(const void *u, int64_t ubs, int64_t urs, const float *w, const flo
     ssd::ConvParams p{};
     p.u = u; p.ubs = ubs; p.urs = urs; p.w = w; p.bias = bias; p.tail_in = tail_in;
     p.tail_out = tail_out; p.v = v; p.vbs = vbs; p.vrs = vrs; p.b = b; p.L = L; p.C_ch = C_ch;
+    p.tail_rs = C_ch;
     rc = ssd::launch_conv(p, dtype, st);
     if (rc == 2) return fail(SSD_ERR_SHAPE, "conv grid too large");
     if (rc) return fail(SSD_ERR_LAUNCH, "conv launch failed: %s", cudaGetErrorString(cudaGetLastError()));
@@ -384,7 +513,7 @@ int conv_impl(const void *u, int64_t ubs, int64_t urs, const float *w, const flo
 const char *const kKernelNames[ssd::kKCount] = {
     "conv1d_silu", "conv_tail", "stripe_state_tc", "stripe_chain", "chunk_output_tc",
     "stripe_state_generic", "chunk_output_generic", "decode_step", "bwd_chunk_summary", "bwd_chains",
-    "bwd_chunk_grad", "bwd_reduce", "gated_rmsnorm"};
+    "bwd_chunk_grad", "bwd_reduce", "gated_rmsnorm", "conv_cells", "conv_ckpt", "conv_bwd"};
 
 struct ProfRecord {
     int id;
@@ -431,6 +560,102 @@ void prof_end(cudaStream_t st, int id)
     g_prof.pending = nullptr;
 }
 }  // namespace ssd
+
+namespace {
+
+// Workspace of ssd_stream_forward without v: the scan's workspace, then the conv output
+// the scan still reads from memory -- B and C only ([b][L][2GN]) when the x conv is fused
+// into the tensor-core scan, all of v ([b][L][C_ch]) on the CUDA-core path.
+struct StreamPlan {
+    bool fused = false;
+    size_t off_v = 0, bytes = 0;
+};
+
+StreamPlan make_stream_plan(int b, int64_t L, int H, int P, int N, int G, int Q, int dtype)
+{
+    StreamPlan sp;
+    const Plan pl = make_plan(b, L, H, P, N, Q);
+    sp.fused = ssd::tc_scan_shape(dtype, H, P, N, G, Q);
+    const size_t cols = sp.fused ? 2 * (size_t)G * N : (size_t)H * P + 2 * (size_t)G * N;
+    sp.off_v = round256(pl.bytes_dt);
+    sp.bytes = sp.off_v + round256((size_t)b * L * cols * elem_size(dtype));
+    return sp;
+}
+
+int stream_fused_impl(const ssd_stream_args *a, cudaStream_t st)
+{
+    const int HP = a->H * a->P, GN = a->G * a->N;
+    const int C_ch = HP + 2 * GN;
+    const size_t es = elem_size(a->dtype);
+    const StreamPlan sp = make_stream_plan(a->b, a->L, a->H, a->P, a->N, a->G, a->Q, a->dtype);
+    if (!a->workspace || a->workspace_bytes < sp.bytes)
+        return fail(SSD_ERR_WORKSPACE, "workspace of %zu bytes needed (ssd_stream_workspace_size), %zu given",
+                    sp.bytes, a->workspace ? a->workspace_bytes : (size_t)0);
+    if ((reinterpret_cast<uintptr_t>(a->workspace) & 255u) != 0)
+        return fail(SSD_ERR_ALIGN, "workspace must be 256-byte aligned");
+    int rc = check_rows("u", a->u, a->u_batch_stride, a->u_row_stride, C_ch, a->b, a->L, a->dtype, true);
+    if (rc) return rc;
+    if (!a->conv_w || !aligned16(a->conv_w)) return fail(SSD_ERR_ALIGN, "conv_w must be given, 16-byte aligned");
+    if ((a->tail_in && !aligned16(a->tail_in)) || (a->tail_out && !aligned16(a->tail_out)) ||
+        (a->conv_ckpt && !aligned16(a->conv_ckpt)))
+        return fail(SSD_ERR_ALIGN, "conv tails must be 16-byte aligned");
+    char *vws = static_cast<char *>(a->workspace) + sp.off_v;
+    const char *u = static_cast<const char *>(a->u);
+    ssd_scan_args s{};
+    s.dtype = a->dtype; s.b = a->b; s.L = a->L; s.H = a->H; s.P = a->P; s.N = a->N; s.G = a->G;
+    s.Q = a->Q; s.s = a->s;
+    s.dt = a->dt; s.A = a->A; s.D = a->D; s.h0 = a->h0;
+    s.dt_bias = a->dt_bias; s.dt_softplus = a->dt_softplus; s.dt_min = a->dt_min; s.dt_max = a->dt_max;
+    s.y = a->y; s.y_batch_stride = a->y_batch_stride; s.y_row_stride = a->y_row_stride;
+    s.h_final = a->h_final; s.h_ckpt = a->h_ckpt;
+    s.workspace = a->workspace; s.workspace_bytes = sp.off_v;
+    if (sp.fused) {
+        // 1. the conv of the B and C channels only, into the workspace ([b][L][2GN]); their rows
+        //    before token 0 are tail_in's B/C columns
+        ssd::ConvParams cp{};
+        cp.u = u + es * HP; cp.ubs = a->u_batch_stride; cp.urs = a->u_row_stride;
+        cp.w = a->conv_w + 4 * HP; cp.bias = a->conv_bias ? a->conv_bias + HP : nullptr;
+        cp.tail_in = a->tail_in ? static_cast<const char *>(a->tail_in) + es * HP : nullptr;
+        cp.tail_rs = C_ch;
+        cp.v = vws; cp.vbs = a->L * 2 * GN; cp.vrs = 2 * GN; cp.b = a->b; cp.L = a->L; cp.C_ch = 2 * GN;
+        rc = ssd::launch_conv(cp, a->dtype, st);
+        if (rc == 2) return fail(SSD_ERR_SHAPE, "conv grid too large");
+        if (rc) return fail(SSD_ERR_LAUNCH, "conv launch failed: %s", cudaGetErrorString(cudaGetLastError()));
+        // 2. the scan, x read from u's x columns with its conv fused in
+        s.x = u; s.x_batch_stride = a->u_batch_stride; s.x_row_stride = a->u_row_stride;
+        s.B = vws; s.B_batch_stride = a->L * 2 * GN; s.B_row_stride = 2 * GN;
+        s.C = vws + es * GN; s.C_batch_stride = a->L * 2 * GN; s.C_row_stride = 2 * GN;
+        FusedConv fc{a->u, a->u_batch_stride, a->u_row_stride, a->conv_w, a->conv_bias, a->tail_in, C_ch};
+        rc = scan_impl(&s, st, &fc);
+        if (rc) return rc;
+    } else {
+        // CUDA-core path: the whole conv output in the workspace, then the scan
+        rc = conv_impl(a->u, a->u_batch_stride, a->u_row_stride, a->conv_w, a->conv_bias, a->tail_in, nullptr, vws,
+                       a->L * C_ch, C_ch, a->b, a->L, C_ch, a->dtype, st);
+        if (rc) return rc;
+        s.x = vws; s.x_batch_stride = a->L * C_ch; s.x_row_stride = C_ch;
+        s.B = vws + es * HP; s.B_batch_stride = a->L * C_ch; s.B_row_stride = C_ch;
+        s.C = vws + es * (HP + GN); s.C_batch_stride = a->L * C_ch; s.C_row_stride = C_ch;
+        rc = scan_impl(&s, st);
+        if (rc) return rc;
+    }
+    // 3. the conv buffers: at every checkpoint, and tail_out (last: it may alias tail_in)
+    if (a->conv_ckpt && a->s > 0 && a->L >= a->s) {
+        if (ssd::launch_conv_ckpt(a->u, a->u_batch_stride, a->u_row_stride, a->conv_ckpt, a->b, a->L, C_ch, a->s,
+                                  a->dtype, st))
+            return fail(SSD_ERR_LAUNCH, "conv checkpoint launch failed: %s", cudaGetErrorString(cudaGetLastError()));
+    }
+    if (a->tail_out) {
+        ssd::ConvParams tp{};
+        tp.u = a->u; tp.ubs = a->u_batch_stride; tp.urs = a->u_row_stride; tp.tail_in = a->tail_in;
+        tp.tail_out = a->tail_out; tp.b = a->b; tp.L = a->L; tp.C_ch = C_ch; tp.tail_rs = C_ch;
+        if (ssd::launch_conv_tail(tp, a->dtype, st))
+            return fail(SSD_ERR_LAUNCH, "conv tail launch failed: %s", cudaGetErrorString(cudaGetLastError()));
+    }
+    return ok();
+}
+
+}  // namespace
 
 extern "C" {
 
@@ -487,18 +712,35 @@ size_t ssd_scan_workspace_size(int b, int64_t L, int H, int P, int N, int Q)
     return make_plan(b, L, H, P, N, Q).bytes_dt;
 }
 
+size_t ssd_stream_workspace_size(int b, int64_t L, int H, int P, int N, int G, int Q, int dtype)
+{
+    if (b <= 0 || L <= 0 || H <= 0 || G <= 0) return 0;
+    return make_stream_plan(b, L, H, P, N, G, Q, dtype).bytes;
+}
+
 int ssd_stream_forward(const ssd_stream_args *a, ssd_stream_t stream)
 {
     if (!a) return fail(SSD_ERR_NULL, "args is NULL");
     int rc = check_scan_shape(a->dtype, a->b, a->L, a->H, a->P, a->N, a->G, a->Q, a->s);
     if (rc) return rc;
+    if (!a->v && a->L > 0 && a->b > 0) return stream_fused_impl(a, (cudaStream_t)stream);
     const int d_inner = a->H * a->P;
     const int C_ch = d_inner + 2 * a->G * a->N;
     if (a->L > 0 && !a->v) return fail(SSD_ERR_NULL, "v is NULL");
+    if (a->conv_ckpt && a->s > 0 && a->L >= a->s) {
+        if (!aligned16(a->conv_ckpt)) return fail(SSD_ERR_ALIGN, "conv_ckpt must be 16-byte aligned");
+        if (!a->u) return fail(SSD_ERR_NULL, "u is NULL");
+    }
     rc = conv_impl(a->u, a->u_batch_stride, a->u_row_stride, a->conv_w, a->conv_bias, a->tail_in,
                    a->tail_out, a->v, a->v_batch_stride, a->v_row_stride, a->b, a->L, C_ch,
                    a->dtype, (cudaStream_t)stream);
     if (rc) return rc;
+    if (a->conv_ckpt && a->s > 0 && a->L >= a->s && a->b > 0) {
+        // the conv buffer at every checkpoint: the 3 rows of u before it
+        if (ssd::launch_conv_ckpt(a->u, a->u_batch_stride, a->u_row_stride, a->conv_ckpt, a->b, a->L, C_ch, a->s,
+                                  a->dtype, (cudaStream_t)stream))
+            return fail(SSD_ERR_LAUNCH, "conv checkpoint launch failed: %s", cudaGetErrorString(cudaGetLastError()));
+    }
     const size_t es = elem_size(a->dtype);
     const char *v = static_cast<const char *>(a->v);
     ssd_scan_args s{};
@@ -520,6 +762,16 @@ int ssd_stream_forward(const ssd_stream_args *a, ssd_stream_t stream)
 int ssd_scan_backward(const ssd_scan_bwd_args *args, ssd_stream_t stream)
 {
     return scan_bwd_impl(args, (cudaStream_t)stream);
+}
+
+size_t ssd_layer_backward_workspace_size(int b, int64_t L, int H, int P, int N, int G, int dtype)
+{
+    return make_layer_bwd_plan(b, L, H, P, N, G, dtype).bytes;
+}
+
+int ssd_layer_backward(const ssd_layer_bwd_args *a, ssd_stream_t stream)
+{
+    return layer_bwd_impl(a, (cudaStream_t)stream);
 }
 
 size_t ssd_scan_backward_workspace_size(int b, int64_t L, int H, int P, int N)
@@ -605,6 +857,6 @@ int ssd_sync_status(ssd_stream_t stream)
 
 const char *ssd_last_error_string(void) { return g_last_error.c_str(); }
 
-int ssd_version(void) { return 200; }   // 0.2.0: backward, its workspace size, gated norm
+int ssd_version(void) { return 300; }   // 0.3.0: layer backward, conv buffers at the checkpoints
 
 }  // extern "C"

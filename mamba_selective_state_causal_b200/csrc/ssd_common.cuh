@@ -47,6 +47,15 @@ struct ScanParams {
     const float *dt_bias;
     int dt_softplus;
     float dt_min, dt_max;
+    // the conv of x fused into the tensor-core passes (ssd_stream_forward without v):
+    // x is then read from the conv input u (same columns) and turned into
+    // silu(conv(u)) in shared memory; NULL conv_w means x is given
+    const void *conv_u;
+    int64_t conv_ubs, conv_urs;
+    const float *conv_w;        // [C_ch][4]
+    const float *conv_bias;     // [C_ch] or NULL
+    const void *conv_tail;      // [b][3][C_ch] (the rows before token 0) or NULL (zeros)
+    int conv_cch;
 };
 
 struct ConvParams {
@@ -61,6 +70,7 @@ struct ConvParams {
     int b;
     int64_t L;
     int C_ch;
+    int64_t tail_rs;    // row stride of tail_in / tail_out (C_ch, or wider for a column slice)
 };
 
 // One decode step (decode.cu).
@@ -115,6 +125,28 @@ struct BwdParams {
     int stage_adjoint;      // set by the launcher: copy Gam and h_prev into shared memory
 };
 
+// The conv part of the layer's backward pass (conv1d_silu.cu, layer_bwd.cu): the
+// conv input u and its per-cell conv buffers, and the gradients of the conv output.
+struct ConvBwdParams {
+    int b;
+    int64_t L;
+    int C_ch, HP, GN;           // channels: x (HP), then B (GN), then C (GN)
+    const void *u;
+    int64_t ubs, urs;
+    const float *w;
+    const float *bias;
+    const void *tail_in;        // [b][3][C_ch] buffer of the first cell, or NULL (zeros)
+    const void *conv_ckpt;      // [b][n_ckpt][3][C_ch] buffer of cell k at k-1, or NULL (one cell)
+    int64_t s, n_ckpt;          // cell length and number of checkpoints (cells when conv_ckpt is set)
+    void *v;                    // recomputed conv output [b][L][C_ch] (I/O dtype, contiguous)
+    const float *dx, *dB, *dC;  // [b][L][HP], [b][L][GN], [b][L][GN] gradients of the conv output
+    const float *dtail_out;     // [b][3][C_ch] or NULL
+    float *du;                  // [b][L][C_ch]
+    float *dtail_in;            // [b][3][C_ch] or NULL
+    float *ws_dw, *ws_dbias;    // per (batch row, token block) partial sums [..][C_ch][4], [..][C_ch]
+    float *dw, *dbias;          // [C_ch][4], [C_ch] (dbias may be NULL)
+};
+
 // The gated RMS norm of the layer output (gated_norm.cu).
 struct NormParams {
     const void *y;
@@ -166,21 +198,44 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(v);
 }
 
+// Row tt of the conv input (channel c of batch row bi) as token t sees it when each cell
+// is rebuilt on its own: rows before t's cell come from that cell's 3-row conv buffer
+// (conv_ckpt[k-1] for cell k > 0, tail_in or zeros for the first cell), the others from u.
+template <typename T>
+__device__ __forceinline__ float cell_val(const ConvBwdParams &p, int64_t bi, int64_t t, int64_t tt, int c)
+{
+    const int64_t k = p.conv_ckpt ? t / p.s : 0;
+    const int64_t start = p.conv_ckpt ? k * p.s : 0;
+    if (tt >= start) return to_f32<T>(reinterpret_cast<const T *>(p.u)[bi * p.ubs + tt * p.urs + c]);
+    const int64_t r = tt - start + 3;
+    if (k == 0)
+        return p.tail_in ? to_f32<T>(reinterpret_cast<const T *>(p.tail_in)[(bi * 3 + r) * p.C_ch + c]) : 0.0f;
+    return to_f32<T>(reinterpret_cast<const T *>(p.conv_ckpt)[((bi * p.n_ckpt + (k - 1)) * 3 + r) * p.C_ch + c]);
+}
+
 // Kernel timing hooks (ssd_api.cu): no-ops unless ssd_profile_begin() is active
 // on the calling thread.
 enum KernelId : int {
     kKConv = 0, kKConvTail, kKStateTc, kKChain, kKOutputTc, kKStateGeneric, kKOutputGeneric, kKDecode,
-    kKBwdSummary, kKBwdChain, kKBwdGrad, kKBwdReduce, kKGatedNorm, kKCount
+    kKBwdSummary, kKBwdChain, kKBwdGrad, kKBwdReduce, kKGatedNorm, kKConvCells, kKConvCkpt, kKConvBwd,
+    kKCount
 };
 void prof_begin(cudaStream_t st, int id);
 void prof_end(cudaStream_t st, int id);
 
 // Launchers (defined in the .cu files).
 int launch_conv(const ConvParams &p, int dtype, cudaStream_t st);
+int launch_conv_cells(const ConvBwdParams &p, int dtype, cudaStream_t st);
+int launch_conv_ckpt(const void *u, int64_t ubs, int64_t urs, void *conv_ckpt, int b, int64_t L, int C_ch,
+                     int64_t s, int dtype, cudaStream_t st);
+int launch_conv_backward(const ConvBwdParams &p, int dtype, cudaStream_t st);
+int64_t conv_bwd_blocks(int64_t L);
 int launch_decode(const DecodeParams &p, int dtype, cudaStream_t st);
 int launch_scan_generic(const ScanParams &p, int dtype, cudaStream_t st);
 int launch_dt_prepare(const ScanParams &p, float *out, cudaStream_t st);
 bool tc_scan_supported(const ScanParams &p, int dtype);
+bool tc_scan_shape(int dtype, int H, int P, int N, int G, int Q);
+int launch_conv_tail(const ConvParams &p, int dtype, cudaStream_t st);
 int launch_scan_backward(const BwdParams &p, int dtype, cudaStream_t st);
 size_t bwd_grad_smem_bytes(int P, int N);
 int launch_gated_norm(const NormParams &p, int dtype, cudaStream_t st);

@@ -167,6 +167,16 @@ def make_grads(wl: Workload, L=None, b=None, device="cpu", seed=None):
     return dy, dhf
 
 
+def make_conv_grads(wl: Workload, b=None, device="cpu", seed=None):
+    """The upstream gradient of the conv buffer a segment hands on: dtail_out [b, 3, C_ch]
+    ~ N(0,1) fp32, and a conv bias ~ N(0, 0.3^2) [C_ch] fp32 for the gradient tests."""
+    b = wl.b if b is None else b
+    g = _gen((wl.seed if seed is None else seed) + 7000, device)
+    dto = torch.randn(b, 3, wl.cch, device=device, generator=g)
+    bias = torch.randn(wl.cch, device=device, generator=g) * 0.3
+    return dto, bias
+
+
 def scaled(wl: Workload, **changes) -> Workload:
     """A copy of a workload with some fields changed (e.g. a shorter L)."""
     d = dict(wl.__dict__)

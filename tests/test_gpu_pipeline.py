@@ -19,8 +19,9 @@ pytestmark = pytest.mark.gpu
 W = ssd_synth.WORKLOADS
 
 
-def gpu_layer(wl, u, prm, dt, segments=1, h0=None, tail=None, zero_tail_at=None):
-    """Run the layer on the GPU as `segments` consecutive resumed calls."""
+def gpu_layer(wl, u, prm, dt, segments=1, h0=None, tail=None, zero_tail_at=None, fused=False):
+    """Run the layer on the GPU as `segments` consecutive resumed calls; fused=True asks for
+    no conv output (the conv of x then runs inside the tensor-core scan kernels)."""
     d = "cuda"
     g = {k: v.to(d) for k, v in prm.items()}
     L = u.shape[1]
@@ -28,14 +29,19 @@ def gpu_layer(wl, u, prm, dt, segments=1, h0=None, tail=None, zero_tail_at=None)
     st = None if h0 is None else h0.to(d).clone()
     tl = None if tail is None else tail.to(d).clone()
     ys, cks = [], []
-    ws = ssd.alloc_workspace(wl.b, seg, wl.H, wl.P, wl.N, wl.Q, d)
+    if fused:
+        code = ssd.SSD_BF16 if wl.dtype == "bf16" else ssd.SSD_F32
+        ws = torch.empty(max(1, ssd.stream_workspace_size(wl.b, seg, wl.H, wl.P, wl.N, wl.G, wl.Q, code)),
+                         dtype=torch.uint8, device=d)
+    else:
+        ws = ssd.alloc_workspace(wl.b, seg, wl.H, wl.P, wl.N, wl.Q, d)
     for k in range(segments):
         sl = slice(k * seg, (k + 1) * seg if k < segments - 1 else L)
         if zero_tail_at is not None and k == zero_tail_at:
             tl = torch.zeros_like(tl)
         out = ssd.stream_forward(u[:, sl], g["w"], dt[:, sl], g["A"], g["D"], H=wl.H, P=wl.P,
                                  N=wl.N, G=wl.G, Q=wl.Q, s=wl.s, conv_bias=g["bias"], tail_in=tl,
-                                 h0=st, workspace=ws if sl.stop - sl.start == seg else None)
+                                 h0=st, workspace=ws if sl.stop - sl.start == seg else None, keep_v=not fused)
         st, tl = out["h_final"], out["tail_out"]
         ys.append(out["y"])
         if out["h_ckpt"] is not None:
@@ -66,30 +72,36 @@ def oracle_layer(wl, u, prm, dt, heads=None, h0=None, tail=None):
                         G=1, s=wl.s, io_round=io)
 
 
-def test_tiny_f32_workload():
+FUSED = pytest.mark.parametrize("fused", [False, True], ids=["two_call", "fused"])
+
+
+@FUSED
+def test_tiny_f32_workload(fused):
     wl = W[0]
     prm = ssd_synth.make_params(wl)
     u = ssd_synth.make_u(wl)
     dt = ssd_synth.make_dt(wl, prm["dt_bias"])
-    out = gpu_layer(wl, u.cuda(), prm, dt.cuda())
+    out = gpu_layer(wl, u.cuda(), prm, dt.cuda(), fused=fused)
     ref = oracle_layer(wl, u, prm, dt)
     check_outputs(out, ref, TOL["f32"])
     np.testing.assert_array_equal(host(out["tail_out"]), ref["tail_out"])
 
 
-def test_03b_L16k_workload_all_heads():
+@FUSED
+def test_03b_L16k_workload_all_heads(fused):
     wl = W[1]
     prm = ssd_synth.make_params(wl)
     u = ssd_synth.make_u(wl)
     dt = ssd_synth.make_dt(wl, prm["dt_bias"])
-    out = gpu_layer(wl, u.cuda(), prm, dt.cuda())
+    out = gpu_layer(wl, u.cuda(), prm, dt.cuda(), fused=fused)
     ref = oracle_layer(wl, u, prm, dt)
     errs = check_outputs(out, ref, TOL["bf16"])
     print("0.3B L16k relL2", errs)
 
 
+@FUSED
 @pytest.mark.parametrize("segments", [2, 8])
-def test_streamed_segments_equal_unsplit(segments):
+def test_streamed_segments_equal_unsplit(segments, fused):
     """Split/resume invariant: consecutive resumed calls reproduce the unsplit layer."""
     wl = ssd_synth.scaled(W[2], L=8 * 2048, H=4, s=1024)
     prm = ssd_synth.make_params(wl)
@@ -97,23 +109,25 @@ def test_streamed_segments_equal_unsplit(segments):
     dt = ssd_synth.make_dt(wl, prm["dt_bias"])
     h0 = ssd_synth.make_h0(wl, scale=0.5)
     tail = ssd_synth.make_tail(wl)
-    out = gpu_layer(wl, u.cuda(), prm, dt.cuda(), segments=segments, h0=h0, tail=tail)
+    out = gpu_layer(wl, u.cuda(), prm, dt.cuda(), segments=segments, h0=h0, tail=tail, fused=fused)
     ref = oracle_layer(wl, u, prm, dt, h0=h0, tail=tail)
     check_outputs(out, ref, TOL["bf16"])
     np.testing.assert_array_equal(host(out["tail_out"]), ref["tail_out"])
-    one = gpu_layer(wl, u.cuda(), prm, dt.cuda(), segments=1, h0=h0, tail=tail)
+    one = gpu_layer(wl, u.cuda(), prm, dt.cuda(), segments=1, h0=h0, tail=tail, fused=fused)
     assert rel_l2(host(out["y"]), host(one["y"])) < 1e-2
 
 
-def test_resume_without_conv_tail_differs():
+@FUSED
+def test_resume_without_conv_tail_differs(fused):
     """Negative control: resuming with a zero conv buffer changes the output."""
     wl = ssd_synth.scaled(W[2], L=4 * 512, H=2)
     prm = ssd_synth.make_params(wl)
     u = ssd_synth.make_u(wl)
     dt = ssd_synth.make_dt(wl, prm["dt_bias"])
-    good = gpu_layer(wl, u.cuda(), prm, dt.cuda(), segments=4, tail=torch.zeros(1, 3, wl.cch).to(torch.bfloat16))
+    good = gpu_layer(wl, u.cuda(), prm, dt.cuda(), segments=4, tail=torch.zeros(1, 3, wl.cch).to(torch.bfloat16),
+                     fused=fused)
     bad = gpu_layer(wl, u.cuda(), prm, dt.cuda(), segments=4, tail=torch.zeros(1, 3, wl.cch).to(torch.bfloat16),
-                    zero_tail_at=2)
+                    zero_tail_at=2, fused=fused)
     ref = oracle_layer(wl, u, prm, dt)
     check_outputs(good, ref, TOL["bf16"])
     yb = host(bad["y"])
@@ -121,12 +135,30 @@ def test_resume_without_conv_tail_differs():
     assert rel_l2(yb[:, 2 * seg:2 * seg + 3], ref["y"][:, 2 * seg:2 * seg + 3]) > 1e-2
 
 
-def _sampled_full_size(wl, heads):
+def test_fused_conv_equals_two_call_path_bitwise():
+    """The conv of x fused into the tensor-core scan computes x exactly as the conv kernel
+    does (same fused multiply-adds, same SiLU, same rounding), so the fused layer equals
+    the two-call layer bit for bit: several stripes, a ragged tail, a conv buffer and a
+    state handed in, two batch rows."""
+    wl = ssd_synth.scaled(W[1], L=3 * 2048 + 77, H=4, b=2, s=1024)
+    prm = ssd_synth.make_params(wl)
+    prm["bias"] = ssd_synth.make_conv_grads(wl)[1]
+    u = ssd_synth.make_u(wl).cuda()
+    dt = ssd_synth.make_dt(wl, prm["dt_bias"]).cuda()
+    h0 = ssd_synth.make_h0(wl, scale=0.5)
+    tail = ssd_synth.make_tail(wl)
+    a = gpu_layer(wl, u, prm, dt, h0=h0, tail=tail, fused=False)
+    b = gpu_layer(wl, u, prm, dt, h0=h0, tail=tail, fused=True)
+    for k in ("y", "h_final", "h_ckpt", "tail_out"):
+        assert torch.equal(a[k], b[k]), (k, rel_l2(host(a[k]), host(b[k])))
+
+
+def _sampled_full_size(wl, heads, fused=True):
     prm = ssd_synth.make_params(wl)
     d = "cuda"
     u = ssd_synth.make_u(wl, device=d)
     dt = ssd_synth.make_dt(wl, prm["dt_bias"].to(d), device=d)
-    out = gpu_layer(wl, u, prm, dt, segments=wl.segments)
+    out = gpu_layer(wl, u, prm, dt, segments=wl.segments, fused=fused)
     di = wl.H * wl.P
     cols = torch.cat([torch.arange(h * wl.P, (h + 1) * wl.P) for h in heads] +
                      [torch.arange(di, di + 2 * wl.N)]).to(d)
@@ -139,8 +171,9 @@ def _sampled_full_size(wl, heads):
 
 
 @pytest.mark.slow
-def test_03b_1M_stream_full_size_sampled_heads():
-    _sampled_full_size(W[2], heads=[0, 31])
+@FUSED
+def test_03b_1M_stream_full_size_sampled_heads(fused):
+    _sampled_full_size(W[2], heads=[0, 31], fused=fused)
 
 
 @pytest.mark.slow

@@ -115,13 +115,30 @@ def test_scan_linearity_in_h0():
     assert rel_l2(host(y2), 2 * host(ya)) < 1e-6
 
 
-def test_tensor_core_path_matches_cuda_core_path(monkeypatch):
+def _generic_path_child(out_path):
+    """Runs in a child process started with SSD_SCAN_PATH=generic (the library reads its
+    hooks once per process): the CUDA-core scan of the same case, saved for the parent."""
+    wl = ssd_synth.scaled(W[1], L=3000, H=4, b=2)
+    slow, _ = run_case(wl)
+    np.savez(out_path, **{k: host(v) for k, v in slow.items()})
+
+
+def test_tensor_core_path_matches_cuda_core_path(tmp_path):
     """The tcgen05 path (bf16, P=64, N=128, Q=128) and the CUDA-core path agree,
     and both stay within tolerance of the oracle."""
+    import os
+    import subprocess
+    import sys
     wl = ssd_synth.scaled(W[1], L=3000, H=4, b=2)
     fast, ref = run_case(wl)
-    monkeypatch.setenv("SSD_SCAN_PATH", "generic")
-    slow, _ = run_case(wl)
+    out = tmp_path / "generic.npz"
+    here = os.path.dirname(os.path.abspath(__file__))
+    code = (f"import sys; sys.path[:0] = [{here!r}, {os.path.dirname(here)!r}]; "
+            f"import test_gpu_scan as t; t._generic_path_child({str(out)!r})")
+    r = subprocess.run([sys.executable, "-c", code], env=dict(os.environ, SSD_SCAN_PATH="generic"),
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]
+    slow = dict(np.load(out))
     check_outputs(fast, ref, TOL["bf16"])
-    check_outputs(slow, ref, TOL["bf16"])
-    assert rel_l2(host(fast["y"]), host(slow["y"])) < 1e-2
+    check_outputs({k: torch.from_numpy(v) for k, v in slow.items()}, ref, TOL["bf16"])
+    assert rel_l2(host(fast["y"]), slow["y"]) < 1e-2
