@@ -57,6 +57,9 @@ def parse_args():
     ap.add_argument("--backward", action="store_true")
     # the gated RMS norm of the layer output on one 131072-token segment of the 0.3B shape
     ap.add_argument("--gated-norm", action="store_true")
+    # the layer as two library calls (conv over every channel, then the scan) instead of the
+    # default one call, whose first scan pass computes the conv of x itself
+    ap.add_argument("--two-call", action="store_true")
     return ap.parse_args()
 
 
@@ -70,6 +73,32 @@ def algorithmic_bytes_per_token(wl):
             + 4 * wl.H                                 # read dt
             + (4 * wl.H * wl.P * wl.N / wl.s if wl.s else 0))  # write checkpoints
     return conv, scan
+
+
+def layer_bytes_per_token(wl):
+    """Minimum HBM bytes per token of the layer itself: read u and dt, write y and the
+    checkpoints (the conv output need not leave the chip)."""
+    e = 2 if wl.dtype == "bf16" else 4
+    return (wl.cch * e + 4 * wl.H + wl.d_inner * e
+            + (4 * wl.H * wl.P * wl.N / wl.s if wl.s else 0))
+
+
+def issued_mma_flops_per_token(wl):
+    """Dense bf16 MMA flops the tensor-core output pass issues per token (per chunk of Q
+    tokens and head pair: G = C B^T, Ys = C hp^T, S = B^T (w o X), each Q x 128 x N (or
+    x Q), and Y = Pm X for both heads, Q x P x Q each)."""
+    per_pair_chunk = 2 * (wl.Q * 128 * wl.N * 2 + 128 * wl.N * wl.Q + 2 * wl.Q * wl.P * wl.Q)
+    return per_pair_chunk * (wl.H // 2) / wl.Q
+
+
+def bf16_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
 
 
 # ----------------------------------------------------------------- peaks
@@ -275,10 +304,12 @@ def job_throughput(wl, world, steps, ms_max):
 class Layer:
     """Device buffers and one step of the layer for a workload (one rank)."""
 
-    def __init__(self, wl, seed):
+    def __init__(self, wl, seed, fused=True):
         import mamba_selective_state_causal_b200 as ssd
         self.ssd = ssd
         self.wl = wl
+        self.fused = fused
+        self.two_call = not fused
         d = torch.device("cuda", torch.cuda.current_device())
         self.dev = d
         prm = ssd_synth.make_params(wl, device=d, seed=seed)
@@ -288,25 +319,41 @@ class Layer:
         seg = wl.seg_len
         self.seg = seg
         tdt = ssd_synth.torch_dtype(wl.dtype)
-        self.v = torch.empty(wl.b, seg, wl.cch, dtype=tdt, device=d)
+        self.v = None if fused else torch.empty(wl.b, seg, wl.cch, dtype=tdt, device=d)
         self.y = torch.empty(wl.b, wl.L, wl.H, wl.P, dtype=tdt, device=d)
         self.h = torch.empty(wl.b, wl.H, wl.P, wl.N, dtype=torch.float32, device=d)
         self.tail = torch.empty(wl.b, 3, wl.cch, dtype=tdt, device=d)
         n_ck = seg // wl.s if wl.s else 0
         self.ckpt = torch.empty(wl.b, wl.segments * n_ck, wl.H, wl.P, wl.N, dtype=torch.float32, device=d)
-        self.ws = ssd.alloc_workspace(wl.b, seg, wl.H, wl.P, wl.N, wl.Q, d)
+        if fused:
+            code = ssd.SSD_BF16 if wl.dtype == "bf16" else ssd.SSD_F32
+            self.ws = torch.empty(max(1, ssd.stream_workspace_size(wl.b, seg, wl.H, wl.P, wl.N, wl.G, wl.Q, code)),
+                                  dtype=torch.uint8, device=d)
+        else:
+            self.ws = ssd.alloc_workspace(wl.b, seg, wl.H, wl.P, wl.N, wl.Q, d)
         self.n_ck = n_ck
 
     def segment(self, k, stream=None):
         wl, ssd = self.wl, self.ssd
         t0, t1 = k * self.seg, (k + 1) * self.seg
+        if self.two_call:
+            # the conv over every channel, then the scan on its output: two library calls
+            di, gn = wl.H * wl.P, wl.G * wl.N
+            ssd.conv_forward(self.u[:, t0:t1], self.w, self.bias, tail_in=None if k == 0 else self.tail,
+                             tail_out=self.tail, v=self.v, stream=stream)
+            ssd.scan_forward(self.v[:, :, :di], self.v[:, :, di:di + gn], self.v[:, :, di + gn:],
+                             self.dt[:, t0:t1], self.A, self.D, None if k == 0 else self.h, H=wl.H, G=wl.G,
+                             Q=wl.Q, s=wl.s, y=self.y[:, t0:t1], h_final=self.h,
+                             h_ckpt=self.ckpt[:, k * self.n_ck:(k + 1) * self.n_ck] if self.n_ck else None,
+                             workspace=self.ws, stream=stream)
+            return
         ssd.stream_forward(
             self.u[:, t0:t1], self.w, self.dt[:, t0:t1], self.A, self.D, H=wl.H, P=wl.P, N=wl.N,
             G=wl.G, Q=wl.Q, s=wl.s, conv_bias=self.bias,
             tail_in=None if k == 0 else self.tail, tail_out=self.tail,
             h0=None if k == 0 else self.h, h_final=self.h, v=self.v, y=self.y[:, t0:t1],
             h_ckpt=self.ckpt[:, k * self.n_ck:(k + 1) * self.n_ck] if self.n_ck else None,
-            workspace=self.ws, stream=stream)
+            workspace=self.ws, stream=stream, keep_v=not self.fused)
 
     def step(self, stream=None):
         for k in range(self.wl.segments):
@@ -644,7 +691,7 @@ def main():
         return
     import __graft_entry__
     __graft_entry__.build()
-    layer = Layer(wl, seed=rank_seed(wl, rank))
+    layer = Layer(wl, seed=rank_seed(wl, rank), fused=not args.two_call)
 
     clocks = clock_sampler(local)
     clocks.start()
@@ -665,17 +712,25 @@ def main():
     launches_per_step = sum(v["launches"] for v in prof.values()) / prof_steps
 
     conv_b, scan_b = algorithmic_bytes_per_token(wl)
+    e = 2 if wl.dtype == "bf16" else 4
+    fused = layer.fused and "stripe_state_tc" in prof
     peak, peak_src = hbm_peak()
+    tpeak, tpeak_src = bf16_peak()
     per_launch = {k: v["total_ms"] / v["launches"] for k, v in prof.items()}
     dom = max(prof, key=lambda k: prof[k]["total_ms"])
     tokens_per_launch = {
         "conv1d_silu": wl.b * wl.seg_len, "chunk_output_tc": wl.b * wl.seg_len,
         "chunk_output_generic": wl.b * wl.seg_len, "stripe_state_tc": wl.b * wl.seg_len,
         "stripe_state_generic": wl.b * wl.seg_len}
-    alg_per_token = {"conv1d_silu": conv_b, "chunk_output_tc": scan_b, "chunk_output_generic": scan_b,
-                     # pass A's own necessary reads: x, B, dt
-                     "stripe_state_tc": 2 * wl.d_inner + 2 * wl.G * wl.N + 4 * wl.H,
-                     "stripe_state_generic": 2 * wl.d_inner + 2 * wl.G * wl.N + 4 * wl.H}
+    alg_per_token = {
+        # the conv kernel reads u and writes v: all channels, or only B/C's on the fused path
+        "conv1d_silu": 2 * 2 * wl.G * wl.N * e if fused else conv_b,
+        # the output pass reads x (or u's x columns), B, C, dt and writes y and the checkpoints
+        "chunk_output_tc": scan_b, "chunk_output_generic": scan_b,
+        # pass A's own necessary reads: x (u's x columns on the fused path, where it also
+        # writes the conv output of x), B, dt
+        "stripe_state_tc": (2 if fused else 1) * wl.d_inner * e + wl.G * wl.N * e + 4 * wl.H,
+        "stripe_state_generic": wl.d_inner * e + wl.G * wl.N * e + 4 * wl.H}
     dom_alg = alg_per_token.get(dom, 0) * tokens_per_launch.get(dom, 0)
     achieved = dom_alg / (per_launch[dom] / 1e3) / 1e9
     traffic_pt = recorded_traffic(dom)
@@ -683,8 +738,17 @@ def main():
                 "frac": achieved / peak, "peak_source": peak_src,
                 "traffic": None if traffic_pt is None else traffic_pt * tokens_per_launch.get(dom, 0),
                 "algorithmic_bytes_per_launch": dom_alg}
-    step_bytes = (conv_b + scan_b) * wl.tokens
+    if dom == "chunk_output_tc":
+        tflops = issued_mma_flops_per_token(wl) * tokens_per_launch[dom] / (per_launch[dom] / 1e3) / 1e12
+        roofline.update({"tensor_achieved_tflops": tflops, "tensor_peak_tflops": tpeak,
+                         "tensor_frac": tflops / tpeak, "tensor_peak_source": tpeak_src,
+                         "tensor_flops": "issued dense bf16 MMA flops of the kernel"})
+    # the whole step: the bytes the layer must move (read u and dt, write y and checkpoints)
+    # and, for the target as stated, the two-call path's bytes (conv output written and re-read)
+    layer_b = layer_bytes_per_token(wl)
+    step_bytes = layer_b * wl.tokens
     step_frac = step_bytes / (ms_step / 1e3) / 1e9 / peak
+    two_call_frac = (conv_b + scan_b) * wl.tokens / (ms_step / 1e3) / 1e9 / peak
     kernels = {k: {"launches_per_step": v["launches"] / prof_steps, "ms_per_launch": per_launch[k],
                    "share": v["total_ms"] / sum(x["total_ms"] for x in prof.values())}
                for k, v in prof.items()}
@@ -709,8 +773,10 @@ def main():
                    "ckpt_stride": wl.s, "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2 (u alone %.1f GB)" % (layer.u.numel() * 2 / 1e9)},
         "roofline": roofline,
-        "step_roofline": {"bound": "hbm", "algorithmic_bytes_per_token": conv_b + scan_b,
-                          "achieved": step_bytes / (ms_step / 1e3) / 1e9, "peak": peak, "frac": step_frac},
+        "step_roofline": {"bound": "hbm", "algorithmic_bytes_per_token": layer_b,
+                          "achieved": step_bytes / (ms_step / 1e3) / 1e9, "peak": peak, "frac": step_frac,
+                          "two_call_bytes_per_token": conv_b + scan_b, "two_call_frac": two_call_frac,
+                          "path": "fused conv" if fused else "two-call"},
         "kernels": kernels,
         "cpu_baseline": cpu,
         "e2e": e2e,

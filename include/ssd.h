@@ -210,20 +210,21 @@ typedef struct ssd_stream_args {
  * previous (h_final, tail_out), equals one call on the whole sequence
  * (sequence-axis checkpointing of pith_extraction.key_machinery, with the
  * conv buffer the skeptic_critique asks for).
- * With v == NULL the conv output is not returned, and the call needs a
- * workspace of ssd_stream_workspace_size() bytes instead of
- * ssd_scan_workspace_size(): on the tensor-core scan's shapes (bf16, P = 64,
- * N = 128, Q = 128, heads in pairs per group) the conv of x is then fused into
- * the scan kernels, which read x's columns of u directly, and only the B and
- * C channels' conv output passes through memory (in the workspace); on other
- * shapes the whole conv output is kept in the workspace.
+ * On the tensor-core scan's shapes (bf16, P = 64, N = 128, Q = 128, heads in
+ * pairs per group) with more than one stripe (ssd_scan_workspace_size > 0),
+ * the conv of x runs inside the scan's first pass, which reads x's columns of
+ * u and writes the conv output of x to v; a conv kernel covers only the B and
+ * C channels.  Elsewhere one conv kernel writes all of v.  Either way v ends
+ * up holding the whole conv output, bit for bit the same.
+ * v may be NULL: the conv output then lives in the workspace, which must hold
+ * ssd_stream_workspace_size() bytes instead of ssd_scan_workspace_size().
  * tail_out is written last, so it may alias tail_in.
  */
 SSD_API int ssd_stream_forward(const ssd_stream_args *args, ssd_stream_t stream);
 
 /* Bytes of workspace ssd_stream_forward needs when v is NULL (the scan's
- * workspace plus the conv output that still passes through memory), for
- * dtype SSD_F32 or SSD_BF16 on the current device. */
+ * workspace, then room for the conv output [b][L][C_ch]), for dtype SSD_F32
+ * or SSD_BF16 on the current device. */
 SSD_API size_t ssd_stream_workspace_size(int b, int64_t L, int H, int P, int N, int G, int Q, int dtype);
 
 /*

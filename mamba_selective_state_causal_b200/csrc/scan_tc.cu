@@ -139,10 +139,11 @@ __device__ __forceinline__ void raise_timeout(const ScanParams &p, volatile int 
 // MMAs; warp 17 runs the dt scan that yields w, up to three chunks ahead.
 // Fused conv (kFused): each X box holds the chunk's 128 rows of the conv
 // input u plus the 8 rows before it, and the scaling warps first turn u into
-// x = silu(conv(u)) (rounded to bf16, as the conv kernel stores it), then
-// scale: thread (head, 16-byte column, 4-row group) reads the 3 rows before
-// its group, waits until every thread has (a bounded barrier), then rewrites
-// its 4 rows in place.
+// x = silu(conv(u)) (rounded to bf16, as the conv kernel stores it), write
+// that x to global memory for the output pass (a warp writes 4 whole 128-byte
+// row segments per store), then scale: thread (head, 16-byte column, 4-row
+// group) reads the 3 rows before its group, waits until every thread has (a
+// bounded barrier), then rewrites its 4 rows in place.
 constexpr int kStagesA = 3;
 constexpr int kScaleWarpsA = 16;
 constexpr int kThreadsA = 32 * (kScaleWarpsA + 2);
@@ -251,6 +252,9 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
                     float cur[8];
                     unpack8(lds128(a), cur);
                     uint4 v = conv8(cw, cb, m3, m2, m1, cur);
+                    if (t0 + r < s1)
+                        *reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.conv_v) + (int64_t)bi * p.conv_vbs +
+                                                   (t0 + r) * p.conv_vrs + (ha + hd) * kP + 8 * ch) = v;
                     const float w = s.w[st][hd][r];
                     v.x = scale_bf16x2_int(v.x, w); v.y = scale_bf16x2_int(v.y, w);
                     v.z = scale_bf16x2_int(v.z, w); v.w = scale_bf16x2_int(v.w, w);
@@ -287,7 +291,7 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
                 for (int c32 = 0; c32 < 2; ++c32) {
                     uint32_t a[32];
                     tmem_ld32(tS + lane_base + 64 * hq + 32 * c32, a);
-                    tmem_wait_ld();
+                    tmem_wait_ld(a);
 #pragma unroll
                     for (int pp = 0; pp < 32; ++pp) dst[(int64_t)(32 * c32 + pp) * kN] = __uint_as_float(a[pp]);
                 }
@@ -437,60 +441,58 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
 }
 
 // =============================================================== pass C
-// One CTA per (stripe, head pair), one CTA per SM: 6 decay warps, 8 output
-// warps, a scan warp and an issuing warp (16 warps, four per SM sub-partition,
-// so that each thread may hold 128 registers).  The two heads share their B and C tiles and
-// G = C B^T; the chunks of the stripe are walked in order, two chunks in flight.
+// One CTA per (stripe, head pair), one CTA per SM: 16 compute warps and one
+// issuing warp.  The two heads share their B and C tiles and G = C B^T; the
+// chunks of the stripe are walked in order.
 //
-// Per chunk c (T = the output accumulator of chunk c, two of them alternate):
-//   G   = C B^T                     -> R (TMEM, fp32)
-//   Pm  = masked decay of G         -> R, in place (bf16, both heads)    decay warps
-//   Ys  = C [hp_a | hp_b]^T         -> T                                 (hp = bf16 h_prev)
-//   T  *= exp(cs_i) per row                                              output warps
-//   Y   = Pm X, accumulated into T  (both heads, A from TMEM)
-//   y   = T + D x  (fp32)  -> bf16 -> the X slot -> TMA store            output warps
-//   S   = B^T [Xw_a | Xw_b], accumulated into the fp32 state H (TMEM)
-//   H   = exp(cs_last) H + S, its bf16 copy hp feeding the next chunk's Ys  output warps
-// w o X (Xw) is written into the C half of the chunk's B/C slot once G and Ys
-// have read C.  The issuing warp issues each group of MMAs as soon as its
-// inputs are ready, so the Ys/S chain of chunk c runs while the decay warps
-// work on it, and G of chunk c+1 follows Y of chunk c.
-//
-// Decay warp (lane quarter q = warp & 3): a range of 32-token column blocks J
-// of its 32 rows, both heads -- warps 0 and 1 all four blocks of quarters 0
-// and 1, warps 2 and 3 blocks 0 and 1 of quarters 2 and 3, warps 14 and 15
-// blocks 2 and 3 of quarters 2 and 3 (the lower quarters carry less of the
-// triangle).  It reads G's block J (TMEM columns 32 J .. 32 J + 31) and writes
-// Pm of head a into columns 32 J .. 32 J + 15 and of head b into 32 J + 16 ..
-// 32 J + 31, i.e. only into columns it has read itself, so no other warp is
-// involved.
-//   Pm[i][j] = G[i][j] exp(cs_i - cs_j) dt_j  (j <= i), 0 above the diagonal.
-// Warp 13 publishes each chunk's cumsum of dt*A once every reader of the
-// previous chunk's values is done; warp 12 issues the TMA copies and MMAs.
-// Output warp (lane quarter q, head hd = (warp - 4) >> 2), per chunk c:
-//   state step c: H (h after chunk c-1; checkpointed when one ends there) ->
-//   hp, then H *= exp(cs_last(c)); the epilogue of chunk c-1; w o X of its 32
-//   token rows of head hd; T *= exp(cs_i) on its rows and head.
-// Every per-chunk barrier exists twice (chunk parity), so a barrier cannot
-// complete twice before its waiter looks.
-// TMEM (512 columns): R = 0..127, T0 = 128..255, T1 = 256..383, H = 384..511.
-constexpr int kDecayWarps = 6;
-constexpr int kOutWarps = 8;
-constexpr int kIssueWarp = 12, kScanWarp = 13;
-constexpr int kThreadsC = 32 * 16;
+// The output accumulator T of a chunk first receives Ys = C [hp_a | hp_b]^T
+// (the contribution of the state entering the chunk), which the compute warps
+// scale row by row by exp(cs_i); Y = Pm X then accumulates onto it, so the
+// epilogue only adds D x.  Ys of chunk c is computed while the warps work on
+// chunk c's masked decay, and G of chunk c+1 while they work on chunk c's
+// products and epilogue, so neither is on the chunk's critical path.
+// Issuing warp, per chunk c (the whole warp waits, one lane issues):
+//   Pm ready -> G of chunk c+1 into R0 (its B/C tile has landed; the decay has
+//   read G of chunk c); T scaled -> Y_a = Pm_a X_a, Y_b = Pm_b X_b accumulated
+//   into T; w o X ready -> S = B^T [Xw_a | Xw_b], accumulated straight into the
+//   fp32 state H in TMEM; products done -> the B/C slot is refilled and X of
+//   chunk c+1 is loaded into the X slot w o X came from; y staged (and hp of
+//   chunk c+1 written) -> TMA store of y, Ys of chunk c+1 into T, and, once the
+//   store has read its slot, chunk c+1 may write its w o X there.
+// The two X slots alternate: chunk c's X sits in slot c & 1, its w o X goes
+// to slot (c + 1) & 1 (so that scaling X never waits for Y = Pm X to read it)
+// and its y is staged back in slot c & 1.
+// Warp 4 (no masked-decay work of its own) also publishes the chunk cumsum of
+// dt*A of both heads for chunk c+1 once every warp has written chunk c's w o X.
+// Compute warp (TMEM lane quarter q = warp & 3, column slice cs = warp >> 2 of
+// the 128 (head, p) columns; head hd = cs >> 1), per chunk:
+//   mask: Pm columns 32 cs .. 32 cs + 31, i.e. head hd's 32-token column
+//         blocks 2 (cs & 1) and 2 (cs & 1) + 1 of its 32 rows:
+//         Pm[i][j] = G[i][j] exp(cs_i - cs_j) dt_j (j <= i), 0 above
+//   T *= exp(cs_i) on its rows and columns (T holds Ys)
+//   w o X of head hd into the other X slot (rows split over the head's 8 warps)
+//   y = T + D x in fp32 -> bf16 -> the X slot (same swizzle as the y map), and
+//   with it the state step of chunk c+1: H (h after chunk c) -> bf16 copy hp,
+//         checkpoint, then H = exp(cs_last(c+1)) H, to which S of chunk c+1 is added
+// A warp reads and writes only TMEM columns it owns (and G's, which nobody
+// writes while the decay runs), so no barrier among the compute warps is
+// needed; hand-offs go through mbarriers (one arrival per warp).
+// TMEM (512 columns): R0 = 0..127 G (fp32); R1 = 128..255 Pm_a | Pm_b (bf16);
+// T = 256..383 (a | b); H = 384..511 (a | b), the fp32 state, rows n.
+// Shared memory: B/C ring of 2, two X slots (a slot holds a chunk's X, then its
+// y, then the next chunk's w o X), hp, and the per-head scan values (about 227 KB).
+constexpr int kComputeWarps = 16;
+constexpr int kThreadsC = 32 * (kComputeWarps + 1);
 
 struct SmemC {
-    uint8_t bc[2][4 * kBox];   // C box 0, C box 1, B box 0, B box 1; the C half later holds w o X
-    uint8_t x[2][2 * kBox];    // X of head a, head b; then y
+    uint8_t bc[2][4 * kBox];   // ring slot: C box 0, C box 1, B box 0, B box 1
+    uint8_t x[2][2 * kBox];    // X slot: head a box, head b box (X, then y, then the next chunk's w o X)
     uint8_t hp[2 * kBox];      // bf16 h_prev of head a, head b (rows n, cols p), 128B-swizzled
     float cvs[2][kQ];          // chunk-inclusive cumsum of dt*A (log2 units), per head
     float dvs[2][kQ];          // dt, per head
     float fs[2][3 * 32];       // dt_j exp(cs_end(J) - cs_j) for the 32-token blocks J = 0..2
-    uint64_t full_bc[2], full_x[2];                       // TMA -> consumers (by slot)
-    uint64_t g_done[2], ys_done[2], s_done[2], y_done[2]; // MMA commits (by chunk parity)
-    uint64_t fin;
-    uint64_t pm_ready[2], st_ready[2], ts_ready[2], ep_done[2], xw_ready[2], scan_ready[2];
-    uint64_t conv_sync[2];     // fused conv: every output warp has read the rows before its group
+    uint64_t full_bc[2], full_x[2], g_done, ys_done, mma_done, fin, xslot_free; // TMA / MMA / issuer -> warps
+    uint64_t pm_ready, ts_ready, xw_ready, y_ready, st0_ready, scan_ready;     // warps -> issuing warp
     uint32_t tmem;
     int abort;
 };
@@ -507,7 +509,6 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b)
     return d;
 }
 
-template <bool kFused>
 __global__ void __launch_bounds__(kThreadsC, 1)
 chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
 {
@@ -532,22 +533,18 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
         return;
     }
     if (tid == 0) {
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&s.full_bc[i], 1);
-            mbar_init(&s.full_x[i], 1);
-            mbar_init(&s.g_done[i], 1);
-            mbar_init(&s.ys_done[i], 1);
-            mbar_init(&s.s_done[i], 1);
-            mbar_init(&s.y_done[i], 1);
-            mbar_init(&s.pm_ready[i], kDecayWarps);
-            mbar_init(&s.st_ready[i], kOutWarps);
-            mbar_init(&s.ts_ready[i], kOutWarps);
-            mbar_init(&s.ep_done[i], kOutWarps);
-            mbar_init(&s.xw_ready[i], kOutWarps);
-            mbar_init(&s.scan_ready[i], 1);
-            mbar_init(&s.conv_sync[i], kOutWarps);
-        }
+        for (int i = 0; i < 2; ++i) { mbar_init(&s.full_bc[i], 1); mbar_init(&s.full_x[i], 1); }
+        mbar_init(&s.g_done, 1);
+        mbar_init(&s.ys_done, 1);
+        mbar_init(&s.xslot_free, 1);
+        mbar_init(&s.mma_done, 1);
         mbar_init(&s.fin, 1);
+        mbar_init(&s.pm_ready, kComputeWarps);
+        mbar_init(&s.ts_ready, kComputeWarps);
+        mbar_init(&s.xw_ready, kComputeWarps);
+        mbar_init(&s.y_ready, kComputeWarps);
+        mbar_init(&s.st0_ready, kComputeWarps);
+        mbar_init(&s.scan_ready, 1);
         s.abort = 0;
         fence_mbar_init();
         prefetch_tmap(&maps.x);
@@ -559,26 +556,45 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = s.tmem;
-    const uint32_t tR = tm, tH = tm + 384;
+    const uint32_t tG = tm, tPm = tm + 128, tT = tm + 256, tH = tm + 384;
     volatile int *abort = &s.abort;
     const bool live = unit != p.test_drop_unit;
-    // wait for the completion that belongs to chunk c of a per-chunk-parity barrier pair
-    auto cwait = [&](uint64_t *bar2, int c) { return ewait(&bar2[c & 1], (uint32_t)(c >> 1) & 1, abort, lim); };
-    auto carrive = [&](uint64_t *bar2, int c) { if (lane == 0) mbar_arrive(&bar2[c & 1]); };
-    auto fail = [&]() { if (lane == 0) raise_timeout(p, abort); };
 
-    const bool decay_warp = warp < 4 || warp >= 14;
-    if (decay_warp || warp == kScanWarp) {
-        // ================================================= decay warps and the scan warp
-        const int q = warp & 3;
-        const int jlo = warp >= 14 ? 2 : 0;                 // column blocks of this decay warp
-        const int jhi = (warp >= 14 || q < 2) ? 3 : 1;
-        const int r = 32 * q + lane;                   // token row = TMEM lane
+    if (warp < kComputeWarps) {
+        // ================================================= compute warps
+        const int q = warp & 3, cs = warp >> 2, hd = cs >> 1, p0 = 32 * (cs & 1);
+        const int r = 32 * q + lane;             // token row / TMEM lane / state row n
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        const bool scan_warp = warp == kScanWarp;
-        // chunk cumsum of both heads (the scan warp): lane l holds tokens 4 l .. 4 l + 3; dt is
-        // prefetched a chunk ahead and the values are computed before the wait that lets
-        // them overwrite the previous chunk's
+        const int hh = ha + hd;
+        auto fail = [&]() { if (lane == 0) raise_timeout(p, abort); };
+
+        // state entering the stripe -> H: thread (n = r, cs) owns h[p0 .. p0 + 31][n] of head hh
+        {
+            const float *hin = (k == 0) ? (p.h0 ? p.h0 + ((int64_t)bi * p.H + hh) * PN : nullptr)
+                                        : p.ws_hin + (((int64_t)bi * p.ns + k) * p.H + hh) * PN;
+            uint32_t hv[32];
+#pragma unroll
+            for (int pp = 0; pp < 32; ++pp) hv[pp] = __float_as_uint(hin ? hin[(p0 + pp) * kN + r] : 0.0f);
+            tmem_st32(tH + lane_base + 32 * cs, hv);
+            tmem_wait_st();
+        }
+        // the checkpoint slot of the state after the chunk ending at t_end, or -1
+        const int64_t n_ckpt = p.s > 0 ? p.L / p.s : 0;
+        auto ckpt_slot = [&](int64_t t_end) -> int64_t {
+            if (!p.h_ckpt || p.s <= 0 || t_end > s1 || t_end % p.s != 0) return -1;
+            const int64_t kc = t_end / p.s - 1;
+            return kc < n_ckpt ? kc : -1;
+        };
+        auto store_state = [&](float *dst, const uint32_t (&hv)[32]) {
+#pragma unroll
+            for (int pp = 0; pp < 32; ++pp) dst[pp * kN] = __uint_as_float(hv[pp]);
+        };
+        auto ckpt_ptr = [&](int64_t kc) {
+            return p.h_ckpt + (((int64_t)bi * n_ckpt + kc) * p.H + hh) * PN + (int64_t)p0 * kN + r;
+        };
+
+        // chunk cumsum of both heads (warp 4, which has no masked-decay work): lane l holds
+        // tokens 4 l .. 4 l + 3; dt is prefetched a chunk ahead
         const float A2a = p.A[ha] * kLog2e, A2b = p.A[ha + 1] * kLog2e;
         float2 dtn[4];
         auto load_dt = [&](int c) {
@@ -590,8 +606,7 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
                                  : make_float2(0.0f, 0.0f);
             }
         };
-        // scan of chunk c (dt in dtn) -> registers, then -> the shared scan buffer
-        auto publish = [&](int c) -> bool {
+        auto scan = [&]() {
             float ca[4], cb[4];
             float sa = 0.0f, sb = 0.0f;
 #pragma unroll
@@ -613,49 +628,103 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
             // cumsum at the end of this lane's 32-token block (token 32 J + 31 = lane 8 J + 7)
             const float ea = __shfl_sync(0xffffffffu, ca[3], lane | 7);
             const float eb = __shfl_sync(0xffffffffu, cb[3], lane | 7);
-            const float4 fa = make_float4(dtn[0].x * ex2(ea - ca[0]), dtn[1].x * ex2(ea - ca[1]),
-                                          dtn[2].x * ex2(ea - ca[2]), dtn[3].x * ex2(ea - ca[3]));
-            const float4 fb = make_float4(dtn[0].y * ex2(eb - cb[0]), dtn[1].y * ex2(eb - cb[1]),
-                                          dtn[2].y * ex2(eb - cb[2]), dtn[3].y * ex2(eb - cb[3]));
-            // every reader of chunk c-1's values is done: its decay and the output warps' state step
-            if (c > 0 && !(cwait(s.pm_ready, c - 1) && cwait(s.st_ready, c - 1))) return false;
             reinterpret_cast<float4 *>(s.cvs[0])[lane] = make_float4(ca[0], ca[1], ca[2], ca[3]);
             reinterpret_cast<float4 *>(s.cvs[1])[lane] = make_float4(cb[0], cb[1], cb[2], cb[3]);
             reinterpret_cast<float4 *>(s.dvs[0])[lane] = make_float4(dtn[0].x, dtn[1].x, dtn[2].x, dtn[3].x);
             reinterpret_cast<float4 *>(s.dvs[1])[lane] = make_float4(dtn[0].y, dtn[1].y, dtn[2].y, dtn[3].y);
             if (lane < 24) {
-                reinterpret_cast<float4 *>(s.fs[0])[lane] = fa;
-                reinterpret_cast<float4 *>(s.fs[1])[lane] = fb;
+                reinterpret_cast<float4 *>(s.fs[0])[lane] =
+                    make_float4(dtn[0].x * ex2(ea - ca[0]), dtn[1].x * ex2(ea - ca[1]),
+                                dtn[2].x * ex2(ea - ca[2]), dtn[3].x * ex2(ea - ca[3]));
+                reinterpret_cast<float4 *>(s.fs[1])[lane] =
+                    make_float4(dtn[0].y * ex2(eb - cb[0]), dtn[1].y * ex2(eb - cb[1]),
+                                dtn[2].y * ex2(eb - cb[2]), dtn[3].y * ex2(eb - cb[3]));
             }
             __syncwarp();
-            carrive(s.scan_ready, c);
-            return true;
+            if (lane == 0) mbar_arrive(&s.scan_ready);
         };
-        if (scan_warp) load_dt(0);
 
-        bool ok = true;
-        for (int c = 0; c < nc; ++c) {
-            if (scan_warp) {
-                if (!publish(c)) { ok = false; break; }
-                if (c + 1 < nc) load_dt(c + 1);
-                continue;
-            }
-            if (!(cwait(s.scan_ready, c) && cwait(s.g_done, c))) { ok = false; break; }
-            tc_fence_after();
-            const float csa = s.cvs[0][r], csb = s.cvs[1][r];
-            for (int J = jlo; J <= jhi; ++J) {
-                const uint32_t tb = tR + lane_base + 32 * J;
-                if (J < q) {
-                    // whole block below the diagonal: exp(cs_r - cs_j) = exp(cs_r - m_J) exp(m_J - cs_j)
-                    uint32_t gv[32];
-                    tmem_ld32(tb, gv);
-                    tmem_wait_ld();
+        const bool scan_warp = warp == 4;
+        if (scan_warp && live) {
+            load_dt(0);
+            scan();
+            if (nc > 1) load_dt(1);
+        }
+        const float Dh = p.D ? p.D[hh] : 0.0f;
+
+        // H = h after chunk c-1: its bf16 copy feeds C hp^T of chunk c (checkpointed when a
+        // checkpoint ends there), then H *= exp(cs_last(c)), to which chunk c's S is added.
+        auto state_step = [&](int c, uint32_t (&hv)[32]) {
+            const int64_t kc = c > 0 ? ckpt_slot(s0 + (int64_t)c * kQ) : -1;
+            if (kc >= 0) store_state(ckpt_ptr(kc), hv);
+            uint8_t *dst = s.hp + hd * kBox;
 #pragma unroll
-                    for (int hd = 0; hd < 2; ++hd) {
-                        const float E = ex2((hd ? csb : csa) - s.cvs[hd][32 * J + 31]);
+            for (int c4 = 0; c4 < 4; ++c4) {
+                uint4 v;
+                v.x = pack_bf16x2_int(__uint_as_float(hv[8 * c4 + 0]), __uint_as_float(hv[8 * c4 + 1]));
+                v.y = pack_bf16x2_int(__uint_as_float(hv[8 * c4 + 2]), __uint_as_float(hv[8 * c4 + 3]));
+                v.z = pack_bf16x2_int(__uint_as_float(hv[8 * c4 + 4]), __uint_as_float(hv[8 * c4 + 5]));
+                v.w = pack_bf16x2_int(__uint_as_float(hv[8 * c4 + 6]), __uint_as_float(hv[8 * c4 + 7]));
+                sts128(dst + swz(r, (p0 >> 3) + c4), v);
+            }
+            const float dec = ex2(s.cvs[hd][kQ - 1]);
+#pragma unroll
+            for (int pp = 0; pp < 32; ++pp) hv[pp] = __float_as_uint(dec * __uint_as_float(hv[pp]));
+            tmem_st32(tH + lane_base + 32 * cs, hv);
+        };
+        // y = T + D x for 16 columns (fp32) -> bf16, in place over x in the X slot (same
+        // swizzle as the y map)
+        auto y_half = [&](uint8_t *xs, const uint32_t (&tv)[16], int hf) {
+            uint8_t *dst = xs + hd * kBox;
+#pragma unroll
+            for (int c2 = 0; c2 < 2; ++c2) {
+                uint8_t *a = dst + swz(r, (p0 >> 3) + 2 * hf + c2);
+                uint4 v = lds128(a);
+                uint32_t *vw = reinterpret_cast<uint32_t *>(&v);
+#pragma unroll
+                for (int e2 = 0; e2 < 4; ++e2) {
+                    const int i = 8 * c2 + 2 * e2;
+                    vw[e2] = pack_bf16x2(fmaf(Dh, bf16_lo(vw[e2]), __uint_as_float(tv[i])),
+                                         fmaf(Dh, bf16_hi(vw[e2]), __uint_as_float(tv[i + 1])));
+                }
+                sts128(a, v);
+            }
+        };
+
+        bool ok = ewait(&s.scan_ready, 0, abort, lim);
+        if (ok) {
+            uint32_t hv[32];
+            tmem_ld32(tH + lane_base + 32 * cs, hv);
+            tmem_wait_ld(hv);
+            state_step(0, hv);
+            tmem_wait_st();
+            fence_proxy_async_smem();   // hp, read by Ys of chunk 0
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.st0_ready);
+        } else {
+            fail();
+        }
+        for (int c = 0; ok && c < nc; ++c) {
+            uint8_t *xs = s.x[c & 1];
+
+            // ---- masked decay: column blocks J = 2 (cs & 1) + jb of head hd, rows of quarter q
+            if (!ewait(&s.g_done, c & 1, abort, lim)) { fail(); break; }
+            tc_fence_after();
+            {
+                const float csr = s.cvs[hd][r];
+#pragma unroll
+                for (int jb = 0; jb < 2; ++jb) {
+                    const int J = 2 * (cs & 1) + jb;
+                    uint32_t pk[16];
+                    if (J < q) {
+                        // whole block below the diagonal: exp(cs_r - cs_j) = exp(cs_r - m_J) exp(m_J - cs_j)
+                        const float E = ex2(csr - s.cvs[hd][32 * J + 31]);
                         const float2 E2 = make_float2(E, E);
+                        uint32_t gv[32];
+                        tmem_ld32(tG + lane_base + 32 * J, gv);
+                        tmem_wait_ld(gv);
                         const float4 *f4 = reinterpret_cast<const float4 *>(&s.fs[hd][32 * J]);
-                        uint32_t pk[16];
 #pragma unroll
                         for (int i4 = 0; i4 < 8; ++i4) {
                             const float4 f = f4[i4];
@@ -666,331 +735,153 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
                             pk[2 * i4] = pack_bf16x2(a.x, a.y);
                             pk[2 * i4 + 1] = pack_bf16x2(b.x, b.y);
                         }
-                        tmem_st16(tb + 16 * hd, pk);
-                    }
-                } else if (J == q) {
-                    // diagonal block as 16x16 quarters: the two on the diagonal exponentiate each
-                    // entry; the one below factors through m = cs at the block's column 15
-                    uint32_t gv[32];
-                    tmem_ld32(tb, gv);
-                    tmem_wait_ld();
-                    const bool lo = lane < 16;
-                    const int xo = lo ? 0 : 16;
-#pragma unroll
-                    for (int hd = 0; hd < 2; ++hd) {
-                        const float csr = hd ? csb : csa;
+                    } else if (J == q) {
+                        // diagonal block as 16x16 quarters: the two on the diagonal exponentiate each
+                        // entry; the one below factors through m = cs at the block's column 15
+                        uint32_t gv[32];
+                        tmem_ld32(tG + lane_base + 32 * J, gv);
+                        tmem_wait_ld(gv);
                         const float *cvb = &s.cvs[hd][32 * J], *dvb = &s.dvs[hd][32 * J];
                         const float m16 = cvb[15];
+                        const bool lo = lane < 16;
                         const float a_r = ex2(csr - m16);                                   // <= 1 for lane >= 16
                         const float b_own = dvb[lane & 15] * ex2(m16 - cvb[lane & 15]);     // <= dt for lane < 16
-                        uint32_t pk[16];
+                        const int xo = lo ? 0 : 16;
 #pragma unroll
                         for (int k2 = 0; k2 < 8; ++k2) {
                             float vl[2], vh[2];
 #pragma unroll
                             for (int e = 0; e < 2; ++e) {
-                                const int kk = 2 * k2 + e;
-                                const int x = xo + kk;
-                                const float g_x = __uint_as_float(lo ? gv[kk] : gv[16 + kk]);
+                                const int k = 2 * k2 + e;
+                                const int x = xo + k;
+                                const float g_x = __uint_as_float(lo ? gv[k] : gv[16 + k]);
                                 float t = g_x * ex2(csr - cvb[x]) * dvb[x];
                                 t = x > lane ? 0.0f : t;
-                                const float bk = __shfl_sync(0xffffffffu, b_own, kk);
-                                vl[e] = lo ? t : __uint_as_float(gv[kk]) * (a_r * bk);
+                                const float bk = __shfl_sync(0xffffffffu, b_own, k);
+                                vl[e] = lo ? t : __uint_as_float(gv[k]) * (a_r * bk);
                                 vh[e] = lo ? 0.0f : t;
                             }
                             pk[k2] = pack_bf16x2(vl[0], vl[1]);
                             pk[8 + k2] = pack_bf16x2(vh[0], vh[1]);
                         }
-                        tmem_st16(tb + 16 * hd, pk);
-                    }
-                } else {
-                    uint32_t pk[16];
+                    } else {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) pk[i] = 0u;
-                    tmem_st16(tb, pk);
-                    tmem_st16(tb + 16, pk);
+                        for (int i = 0; i < 16; ++i) pk[i] = 0u;
+                    }
+                    tmem_st16(tPm + lane_base + 16 * (2 * cs + jb), pk);
                 }
             }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            carrive(s.pm_ready, c);
-        }
-        if (!ok) fail();
-    } else if (warp < kIssueWarp) {
-        // ================================================= output warps
-        const int q = warp & 3, hd = (warp - 4) >> 2;
-        const int r = 32 * q + lane;             // token row of T / state row n of H
-        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        const int hh = ha + hd;
-        const uint32_t tHh = tH + lane_base + 64 * hd;
-        const float Dh = p.D ? p.D[hh] : 0.0f;
+            if (lane == 0) mbar_arrive(&s.pm_ready);
 
-        // the checkpoint slot of the state after the chunk ending at t_end, or -1
-        const int64_t n_ckpt = p.s > 0 ? p.L / p.s : 0;
-        auto ckpt_slot = [&](int64_t t_end) -> int64_t {
-            if (!p.h_ckpt || p.s <= 0 || t_end > s1 || t_end % p.s != 0) return -1;
-            const int64_t kc = t_end / p.s - 1;
-            return kc < n_ckpt ? kc : -1;
-        };
-        // thread (n = r) writes h[p][n] for p = 32 half .. 32 half + 31 of head hh
-        auto store_state = [&](float *base, int half, const uint32_t (&hv)[32]) {
-            float *dst = base + (int64_t)(32 * half) * kN + r;
-#pragma unroll
-            for (int pp = 0; pp < 32; ++pp) dst[pp * kN] = __uint_as_float(hv[pp]);
-        };
-        auto ckpt_base = [&](int64_t kc) { return p.h_ckpt + (((int64_t)bi * n_ckpt + kc) * p.H + hh) * PN; };
-
-        // state entering the stripe -> H
-        {
-            const float *hin = (k == 0) ? (p.h0 ? p.h0 + ((int64_t)bi * p.H + hh) * PN : nullptr)
-                                        : p.ws_hin + (((int64_t)bi * p.ns + k) * p.H + hh) * PN;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t hv[32];
-#pragma unroll
-                for (int pp = 0; pp < 32; ++pp)
-                    hv[pp] = __float_as_uint(hin ? hin[(32 * half + pp) * kN + r] : 0.0f);
-                tmem_st32(tHh + 32 * half, hv);
-            }
-            tmem_wait_st();
-        }
-
-        // y = T + D x of chunk c -> bf16, in place over x in the X slot
-        auto epilogue = [&](int c) -> bool {
-            if (!cwait(s.y_done, c)) return false;
+            // ---- T (= Ys of this chunk) *= exp(cs_r) on this warp's rows and columns
+            if (!ewait(&s.ys_done, c & 1, abort, lim)) { fail(); break; }
             tc_fence_after();
-            uint8_t *xs = s.x[c & 1] + hd * kBox;
-            const uint32_t tT = tm + 128 + 128 * (c & 1) + lane_base + 64 * hd;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
+            {
+                const float e_r = ex2(s.cvs[hd][r]);
                 uint32_t tv[32];
-                tmem_ld32(tT + 32 * half, tv);
-                tmem_wait_ld();
+                tmem_ld32(tT + lane_base + 32 * cs, tv);
+                tmem_wait_ld(tv);
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    uint8_t *a = xs + swz(r, 4 * half + cc);
-                    uint4 v = lds128(a);
-                    uint32_t *vw = reinterpret_cast<uint32_t *>(&v);
-#pragma unroll
-                    for (int e2 = 0; e2 < 4; ++e2) {
-                        const int i = 8 * cc + 2 * e2;
-                        vw[e2] = pack_bf16x2(fmaf(Dh, bf16_lo(vw[e2]), __uint_as_float(tv[i])),
-                                             fmaf(Dh, bf16_hi(vw[e2]), __uint_as_float(tv[i + 1])));
-                    }
-                    sts128(a, v);
-                }
-            }
-            tc_fence_before();
-            fence_proxy_async_smem();   // y, read by the TMA store
-            __syncwarp();
-            carrive(s.ep_done, c);
-            return true;
-        };
-
-        // fused conv of chunk c, in place over its X slot (u -> x = bf16(silu(conv(u)))): thread
-        // (head chd, 16-byte column cch, 8-row group rg) with rg = (cg + c) mod 16, so that the
-        // thread doing rows 120..127 of chunk c does rows 0..7 of chunk c+1 and carries the 3
-        // rows before them in registers; the other groups read those rows from the slot
-        const int ew = warp - 4, chd = ew >> 2, cch = lane & 7, cg = 4 * (ew & 3) + (lane >> 3);
-        const int cc0 = (ha + chd) * kP + 8 * cch;       // first of this thread's 8 channels
-        uint4 win3 = make_uint4(0u, 0u, 0u, 0u), win2 = win3, win1 = win3;
-        auto conv_chunk = [&](int c) -> bool {
-            uint8_t *xs = s.x[c & 1] + chd * kBox;
-            const int rg = (cg + c) & 15;
-            uint4 h3, h2, h1;
-            if (rg != 0) {
-                h3 = lds128(xs + swz(8 * rg - 3, cch));
-                h2 = lds128(xs + swz(8 * rg - 2, cch));
-                h1 = lds128(xs + swz(8 * rg - 1, cch));
-            } else if (c > 0) {
-                h3 = win3; h2 = win2; h1 = win1;
-            } else {
-                // the stripe's first chunk: the 3 rows before it, from u or the conv buffer handed in
-                uint4 hv[3];
-#pragma unroll
-                for (int rr = 0; rr < 3; ++rr) {
-                    const int64_t pos = s0 - 3 + rr;
-                    const __nv_bfloat16 *src = nullptr;
-                    if (pos >= 0)
-                        src = reinterpret_cast<const __nv_bfloat16 *>(p.conv_u) + (int64_t)bi * p.conv_ubs +
-                              pos * p.conv_urs + cc0;
-                    else if (p.conv_tail)
-                        src = reinterpret_cast<const __nv_bfloat16 *>(p.conv_tail) +
-                              ((int64_t)bi * 3 + 3 + pos) * p.conv_cch + cc0;
-                    hv[rr] = src ? *reinterpret_cast<const uint4 *>(src) : make_uint4(0u, 0u, 0u, 0u);
-                }
-                h3 = hv[0]; h2 = hv[1]; h1 = hv[2];
-            }
-            __syncwarp();
-            carrive(s.conv_sync, c);
-            if (!cwait(s.conv_sync, c)) return false;
-            float cw[8][4], cb[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float4 q4 = __ldg(reinterpret_cast<const float4 *>(p.conv_w) + cc0 + i);
-                cw[i][0] = q4.x; cw[i][1] = q4.y; cw[i][2] = q4.z; cw[i][3] = q4.w;
-                cb[i] = p.conv_bias ? __ldg(p.conv_bias + cc0 + i) : 0.0f;
-            }
-            float m3[8], m2[8], m1[8];
-            unpack8(h3, m3); unpack8(h2, m2); unpack8(h1, m1);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                uint8_t *a = xs + swz(8 * rg + i, cch);
-                const uint4 raw = lds128(a);
-                float cur[8];
-                unpack8(raw, cur);
-                sts128(a, conv8(cw, cb, m3, m2, m1, cur));
-#pragma unroll
-                for (int e = 0; e < 8; ++e) { m3[e] = m2[e]; m2[e] = m1[e]; m1[e] = cur[e]; }
-                if (i == 5) win3 = raw;
-                if (i == 6) win2 = raw;
-                if (i == 7) win1 = raw;
-            }
-            fence_proxy_async_smem();
-            return true;
-        };
-
-        bool ok = true;
-        float e_r = 0.0f, w_r = 0.0f;
-        for (int c = 0; c < nc; ++c) {
-            // ---- state step c: H = h after chunk c-1 -> checkpoint, hp; H *= exp(cs_last(c))
-            if (c > 0 && !cwait(s.s_done, c - 1)) { ok = false; break; }
-            if (!cwait(s.scan_ready, c)) { ok = false; break; }
-            tc_fence_after();
-            const float cl = s.cvs[hd][kQ - 1];
-            const float dec = ex2(cl);
-            e_r = ex2(s.cvs[hd][r]);
-            w_r = s.dvs[hd][r] * ex2(cl - s.cvs[hd][r]);
-            {
-                const int64_t kc = c > 0 ? ckpt_slot(s0 + (int64_t)c * kQ) : -1;
-                uint8_t *hdst = s.hp + hd * kBox;
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t hv[32];
-                    tmem_ld32(tHh + 32 * half, hv);
-                    tmem_wait_ld();
-                    if (kc >= 0) store_state(ckpt_base(kc), half, hv);
-#pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        uint4 v;
-                        v.x = pack_bf16x2_int(__uint_as_float(hv[8 * c4 + 0]), __uint_as_float(hv[8 * c4 + 1]));
-                        v.y = pack_bf16x2_int(__uint_as_float(hv[8 * c4 + 2]), __uint_as_float(hv[8 * c4 + 3]));
-                        v.z = pack_bf16x2_int(__uint_as_float(hv[8 * c4 + 4]), __uint_as_float(hv[8 * c4 + 5]));
-                        v.w = pack_bf16x2_int(__uint_as_float(hv[8 * c4 + 6]), __uint_as_float(hv[8 * c4 + 7]));
-                        sts128(hdst + swz(r, 4 * half + c4), v);
-                    }
-#pragma unroll
-                    for (int pp = 0; pp < 32; ++pp) hv[pp] = __float_as_uint(dec * __uint_as_float(hv[pp]));
-                    tmem_st32(tHh + 32 * half, hv);
-                }
-            }
-            tmem_wait_st();
-            fence_proxy_async_smem();   // hp, read by Ys
-            tc_fence_before();
-            __syncwarp();
-            carrive(s.st_ready, c);
-
-            // ---- the epilogue of chunk c-1
-            if (c > 0 && !epilogue(c - 1)) { ok = false; break; }
-
-            // ---- fused: the conv of chunk c once its rows of u have landed
-            if (kFused) {
-                if (!(ewait(&s.full_x[c & 1], (uint32_t)(c >> 1) & 1, abort, lim) && conv_chunk(c))) {
-                    ok = false;
-                    break;
-                }
-            }
-
-            // ---- w o X of chunk c (row r of head hd) into the C half of its B/C slot, once G and Ys
-            //      have read C; then T *= exp(cs_r)
-            if (!(cwait(s.ys_done, c) && ewait(&s.full_x[c & 1], (uint32_t)(c >> 1) & 1, abort, lim))) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            {
-                const uint8_t *src = s.x[c & 1] + hd * kBox;
-                uint8_t *dst = s.bc[c & 1] + hd * kBox;
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    uint4 v = lds128(src + swz(r, u));
-                    v.x = scale_bf16x2_int(v.x, w_r); v.y = scale_bf16x2_int(v.y, w_r);
-                    v.z = scale_bf16x2_int(v.z, w_r); v.w = scale_bf16x2_int(v.w, w_r);
-                    sts128(dst + swz(r, u), v);
-                }
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            carrive(s.xw_ready, c);
-            {
-                const uint32_t tT = tm + 128 + 128 * (c & 1) + lane_base + 64 * hd;
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t tv[32];
-                    tmem_ld32(tT + 32 * half, tv);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) tv[i] = __float_as_uint(e_r * __uint_as_float(tv[i]));
-                    tmem_st32(tT + 32 * half, tv);
-                }
+                for (int i = 0; i < 32; ++i) tv[i] = __float_as_uint(e_r * __uint_as_float(tv[i]));
+                tmem_st32(tT + lane_base + 32 * cs, tv);
             }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            carrive(s.ts_ready, c);
-        }
-        if (ok) {
-            // the state after the stripe's last chunk, then the last epilogue
-            if (cwait(s.s_done, nc - 1)) {
-                tc_fence_after();
-                const int64_t kc = ckpt_slot(s0 + (int64_t)nc * kQ);
-                const bool fin_state = p.h_final && s1 == p.L;
+            if (lane == 0) mbar_arrive(&s.ts_ready);
+
+            // ---- w o X of head hd into the other X slot (free once the previous y store has read it),
+            //      so that it need not wait for Y = Pm X: 4 chunks of 16 B per thread
+            if (!(ewait(&s.full_x[c & 1], (c >> 1) & 1, abort, lim) &&
+                  ewait(&s.xslot_free, c & 1, abort, lim))) { fail(); break; }
+            {
+                const int ti = 32 * (warp & 7) + lane;
+                const int j = ti >> 1, ch = 4 * (ti & 1);
+                const float w = s.dvs[hd][j] * ex2(s.cvs[hd][kQ - 1] - s.cvs[hd][j]);
+                const uint8_t *src = xs + hd * kBox;
+                uint8_t *dst = s.x[(c + 1) & 1] + hd * kBox;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t hv[32];
-                    tmem_ld32(tHh + 32 * half, hv);
-                    tmem_wait_ld();
-                    if (kc >= 0) store_state(ckpt_base(kc), half, hv);
-                    if (fin_state) store_state(p.h_final + ((int64_t)bi * p.H + hh) * PN, half, hv);
+                for (int u = 0; u < 4; ++u) {
+                    uint4 v = lds128(src + swz(j, ch + u));
+                    v.x = scale_bf16x2_int(v.x, w); v.y = scale_bf16x2_int(v.y, w);
+                    v.z = scale_bf16x2_int(v.z, w); v.w = scale_bf16x2_int(v.w, w);
+                    sts128(dst + swz(j, ch + u), v);
                 }
-                ok = epilogue(nc - 1);
-            } else {
-                ok = false;
             }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.xw_ready);
+            // every warp has read this chunk's scan values once all w o X are written: publish the next chunk's
+            if (scan_warp && c + 1 < nc) {
+                if (!ewait(&s.xw_ready, c & 1, abort, lim)) { fail(); break; }
+                scan();
+                if (c + 2 < nc) load_dt(c + 2);
+            }
+
+            // ---- once every product of the chunk is done: y of chunk c and the state step of chunk c+1
+            if (!ewait(&s.mma_done, c & 1, abort, lim)) { fail(); break; }
+            tc_fence_after();
+            if (c + 1 < nc) {
+                if (!ewait(&s.scan_ready, (c + 1) & 1, abort, lim)) { fail(); break; }
+                uint32_t hv[32], t0v[16], t1v[16];
+                tmem_ld32(tH + lane_base + 32 * cs, hv);
+                tmem_ld16(tT + lane_base + 32 * cs, t0v);
+                tmem_ld16(tT + lane_base + 32 * cs + 16, t1v);
+                tmem_wait_ld(t0v, t1v);
+                tmem_wait_ld(hv);
+                y_half(xs, t0v, 0);
+                y_half(xs, t1v, 1);
+                state_step(c + 1, hv);
+            } else {
+                uint32_t t0v[16], t1v[16];
+                tmem_ld16(tT + lane_base + 32 * cs, t0v);
+                tmem_ld16(tT + lane_base + 32 * cs + 16, t1v);
+                tmem_wait_ld(t0v, t1v);
+                y_half(xs, t0v, 0);
+                y_half(xs, t1v, 1);
+            }
+            tmem_wait_st();
+            fence_proxy_async_smem();   // y for the store, hp for the next C hp^T
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.y_ready);
         }
-        if (!ok) fail();
+        if (!__any_sync(0xffffffffu, *abort != 0)) {
+            // the state after the stripe's last chunk
+            uint32_t hv[32];
+            tmem_ld32(tH + lane_base + 32 * cs, hv);
+            tmem_wait_ld(hv);
+            const int64_t kc = ckpt_slot(s0 + (int64_t)nc * kQ);
+            if (kc >= 0) store_state(ckpt_ptr(kc), hv);
+            if (p.h_final && s1 == p.L) store_state(p.h_final + ((int64_t)bi * p.H + hh) * PN + (int64_t)p0 * kN + r, hv);
+        }
     } else {
         // ================================================= issuing warp
-        // The whole warp polls (lane 0's view decides, so every branch is warp-uniform); lane 0
-        // issues.  Counters: groups issued (i_*), completions observed (o_*), loads issued (n_*).
-        int i_g = 0, i_ys = 0, i_s = 0, i_y = 0, i_st = 0;
-        int o_bc = 0, o_x = 0, o_yd = 0, o_sd = 0, o_pm = 0, o_st = 0, o_ts = 0, o_ep = 0, o_xw = 0;
-        int n_bc = 0, n_x = 0;
+        int bc_issued = 0, bc_waited = 0, x_issued = 0, x_waited = 0;   // lane 0's bookkeeping
         auto issue_bc = [&](int c) {
-            if (lane == 0) {
-                const int t0 = (int)(s0 + (int64_t)c * kQ);
-                uint8_t *d = s.bc[c & 1];
-                uint64_t *bar = &s.full_bc[c & 1];
-                mbar_arrive_expect_tx(bar, 4 * kBox);
-                tma_load_3d(d, &maps.C, bar, g * kN, t0, bi);
-                tma_load_3d(d + kBox, &maps.C, bar, g * kN + 64, t0, bi);
-                tma_load_3d(d + 2 * kBox, &maps.B, bar, g * kN, t0, bi);
-                tma_load_3d(d + 3 * kBox, &maps.B, bar, g * kN + 64, t0, bi);
-            }
-            ++n_bc;
+            const int t0 = (int)(s0 + (int64_t)c * kQ);
+            uint8_t *d = s.bc[c & 1];
+            uint64_t *bar = &s.full_bc[c & 1];
+            mbar_arrive_expect_tx(bar, 4 * kBox);
+            tma_load_3d(d, &maps.C, bar, g * kN, t0, bi);
+            tma_load_3d(d + kBox, &maps.C, bar, g * kN + 64, t0, bi);
+            tma_load_3d(d + 2 * kBox, &maps.B, bar, g * kN, t0, bi);
+            tma_load_3d(d + 3 * kBox, &maps.B, bar, g * kN + 64, t0, bi);
+            ++bc_issued;
         };
         auto issue_x = [&](int c) {
-            if (lane == 0) {
-                const int t0 = (int)(s0 + (int64_t)c * kQ);
-                uint8_t *d = s.x[c & 1];
-                uint64_t *bar = &s.full_x[c & 1];
-                mbar_arrive_expect_tx(bar, 2 * kBox);
-                tma_load_3d(d, &maps.x, bar, ha * kP, t0, bi);
-                tma_load_3d(d + kBox, &maps.x, bar, (ha + 1) * kP, t0, bi);
-            }
-            ++n_x;
+            const int t0 = (int)(s0 + (int64_t)c * kQ);
+            uint8_t *d = s.x[c & 1];
+            uint64_t *bar = &s.full_x[c & 1];
+            mbar_arrive_expect_tx(bar, 2 * kBox);
+            tma_load_3d(d, &maps.x, bar, ha * kP, t0, bi);
+            tma_load_3d(d + kBox, &maps.x, bar, (ha + 1) * kP, t0, bi);
+            ++x_issued;
         };
+        // G = C B^T of chunk c into the TMEM columns at tG (its B/C slot has landed)
         // shared-memory descriptors of every operand tile, built once per slot: a K-step only adds
         // a constant to the start-address field (in 16-byte units; addresses stay below 256 KB)
         const uint32_t bc0 = smem_u32(s.bc[0]), bc1 = smem_u32(s.bc[1]);
@@ -998,137 +889,120 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
         const uint64_t dC0 = smem_desc(bc0, 16, 1024), dC1 = smem_desc(bc1, 16, 1024);   // C, K-major
         const uint64_t dBk0 = smem_desc(bc0 + 2 * kBox, 16, 1024), dBk1 = smem_desc(bc1 + 2 * kBox, 16, 1024);  // B, K-major
         const uint64_t dBt0 = smem_desc(bc0 + 2 * kBox, kBox, 1024), dBt1 = smem_desc(bc1 + 2 * kBox, kBox, 1024);  // B^T, MN-major
-        const uint64_t dXw0 = smem_desc(bc0, kBox, 1024), dXw1 = smem_desc(bc1, kBox, 1024);  // w o X (C half), N = 128
-        const uint64_t dX0 = smem_desc(x0, 0, 1024), dX1 = smem_desc(x1, 0, 1024);           // X of one head, N = 64
+        const uint64_t dX0 = smem_desc(x0, 0, 1024), dX1 = smem_desc(x1, 0, 1024);           // X of one head, MN-major, N = 64
+        const uint64_t dXw0 = smem_desc(x0, kBox, 1024), dXw1 = smem_desc(x1, kBox, 1024);    // w o X of both heads, N = 128
         const uint64_t dHp = smem_desc(smem_u32(s.hp), kBox, 1024);                          // hp of both heads, N = 128
         constexpr uint64_t kBoxD = kBox >> 4;
         auto koff = [](int kk) -> uint64_t { return (uint64_t)((kk >> 2) * kBoxD + (kk & 3) * 2); };  // K-major K-step
         auto moff = [](int kk) -> uint64_t { return (uint64_t)(kk * 128); };                          // MN-major K-step
-        const uint32_t id_g = idesc_bf16(128, 128, 0, 0);     // A = C (K-major), B = B (K-major)
-        const uint32_t id_pm = idesc_bf16(128, 64, 0, 1);     // A = Pm (TMEM), B = X (MN-major)
-        const uint32_t id_ys = idesc_bf16(128, 128, 0, 1);    // A = C (K-major), B = hp (MN-major)
-        const uint32_t id_s = idesc_bf16(128, 128, 1, 1);     // A = B^T (MN-major), B = w o X (MN-major)
-        auto poll = [&](uint64_t *bar2, int c) -> bool {
-            uint32_t v = 0;
-            if (lane == 0) v = mbar_try_wait(&bar2[c & 1], (uint32_t)(c >> 1) & 1) ? 1u : 0u;
-            return __shfl_sync(0xffffffffu, v, 0) != 0;
+        auto issue_g = [&](int c) {
+            const uint64_t dc = (c & 1) ? dC1 : dC0, db = (c & 1) ? dBk1 : dBk0;
+            const uint32_t id_g = idesc_bf16(128, 128, 0, 0);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) mma_ss(tG, dc + koff(kk), db + koff(kk), id_g, kk > 0);
+            mma_commit(&s.g_done);
         };
-
+        // Ys = C hp^T of chunk c into T (its B/C slot has landed, hp is written, T is free)
+        auto issue_ys = [&](int c) {
+            const uint64_t dc = (c & 1) ? dC1 : dC0;
+            const uint32_t id_ys = idesc_bf16(128, 128, 0, 1);    // A = C (K-major), B = hp (MN-major)
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) mma_ss(tT, dc + koff(kk), dHp + moff(kk), id_ys, kk > 0);
+            mma_commit(&s.ys_done);
+        };
+        const uint32_t id_pm = idesc_bf16(128, 64, 0, 1);     // A = Pm (TMEM), B = X (MN-major)
+        const uint32_t id_s = idesc_bf16(128, 128, 1, 1);     // A = B^T (MN-major), B = w o X (MN-major)
+        // The whole warp waits (warp-uniform outcome); lane 0 issues.
         bool ok = live;
         if (ok) {
-            issue_bc(0);
-            if (nc > 1) issue_bc(1);
-            issue_x(0);
-            if (nc > 1) issue_x(1);
-        }
-        uint64_t t_last = globaltimer_ns();
-        while (ok && (i_y < nc || i_s < nc || i_st < nc)) {
-            bool prog = false;
-            // observe completions, each barrier's next expected one
-            if (o_bc < n_bc && poll(s.full_bc, o_bc)) { ++o_bc; prog = true; }
-            if (o_x < n_x && poll(s.full_x, o_x)) { ++o_x; prog = true; }
-            if (o_yd < i_y && poll(s.y_done, o_yd)) { ++o_yd; prog = true; }
-            if (o_sd < i_s && poll(s.s_done, o_sd)) { ++o_sd; prog = true; }
-            if (o_pm < i_g && poll(s.pm_ready, o_pm)) { ++o_pm; prog = true; }
-            if (o_st < nc && poll(s.st_ready, o_st)) { ++o_st; prog = true; }
-            if (o_ts < i_ys && poll(s.ts_ready, o_ts)) { ++o_ts; prog = true; }
-            if (o_xw < i_ys && poll(s.xw_ready, o_xw)) { ++o_xw; prog = true; }
-            if (o_ep < i_y && poll(s.ep_done, o_ep)) { ++o_ep; prog = true; }
-            // G of chunk i_g into R: its B/C tile has landed and Y of the previous chunk has read R
-            if (i_g < nc && i_g <= i_y && o_bc > i_g && o_yd >= i_g) {
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint64_t dc = (i_g & 1) ? dC1 : dC0, db = (i_g & 1) ? dBk1 : dBk0;
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) mma_ss(tR, dc + koff(kk), db + koff(kk), id_g, kk > 0);
-                    mma_commit(&s.g_done[i_g & 1]);
-                }
-                ++i_g;
-                prog = true;
-            }
-            // Ys = C hp^T into T: hp of this chunk is ready and the epilogue two chunks back has read T
-            if (i_ys < i_g && o_st > i_ys && o_ep >= i_ys - 1) {
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint64_t dc = (i_ys & 1) ? dC1 : dC0;
-                    const uint32_t tT = tm + 128 + 128 * (i_ys & 1);
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) mma_ss(tT, dc + koff(kk), dHp + moff(kk), id_ys, kk > 0);
-                    mma_commit(&s.ys_done[i_ys & 1]);
-                }
-                ++i_ys;
-                prog = true;
-            }
-            // S = B^T (w o X) accumulated into H: w o X written (the state step decayed H before it)
-            if (i_s < i_ys && o_xw > i_s) {
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint64_t dbt = (i_s & 1) ? dBt1 : dBt0, dxw = (i_s & 1) ? dXw1 : dXw0;
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) mma_ss(tH, dbt + moff(kk), dxw + moff(kk), id_s, true);
-                    mma_commit(&s.s_done[i_s & 1]);
-                }
-                ++i_s;
-                prog = true;
-            }
-            // Y = Pm X accumulated into T: Pm written, T scaled, X landed
-            if (i_y < i_g && o_pm > i_y && o_ts > i_y && o_x > i_y) {
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint64_t dx = (i_y & 1) ? dX1 : dX0;
-                    const uint32_t tT = tm + 128 + 128 * (i_y & 1);
-#pragma unroll
-                    for (int hd = 0; hd < 2; ++hd)
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            mma_ts(tT + 64 * hd, tR + 32 * (kk >> 1) + 16 * hd + 8 * (kk & 1),
-                                   dx + hd * kBoxD + moff(kk), id_pm, true);
-                    mma_commit(&s.y_done[i_y & 1]);
-                }
-                ++i_y;
-                prog = true;
-            }
-            // refill a B/C slot once S (the last reader of the chunk two back) is complete
-            if (n_bc < nc && o_sd >= n_bc - 1) { issue_bc(n_bc); prog = true; }
-            // store y once staged
-            if (i_st < nc && o_ep > i_st) {
-                if (lane == 0) {
-                    const int t0 = (int)(s0 + (int64_t)i_st * kQ);
-                    uint8_t *xs = s.x[i_st & 1];
-                    tma_store_3d(&maps.y, xs, ha * kP, t0, bi);
-                    tma_store_3d(&maps.y, xs + kBox, (ha + 1) * kP, t0, bi);
-                    tma_store_commit();
-                }
-                ++i_st;
-                prog = true;
-            }
-            // refill an X slot once its y store has read it and its w o X is written
-            if (n_x < nc && i_st >= n_x - 1 && o_xw >= n_x - 1) {
-                if (lane == 0) tma_store_wait_read<0>();
-                __syncwarp();
-                issue_x(n_x);
-                prog = true;
-            }
-            // give up after lim without progress, or when another warp raised the abort flag
-            // (decided on lane 0's view, so that the loop stays warp-uniform)
-            uint32_t stop = 0;
             if (lane == 0) {
-                const uint64_t now = globaltimer_ns();
-                if (prog) t_last = now;
-                else if (now - t_last > lim || *abort) stop = 1;
+                issue_bc(0);
+                if (nc > 1) issue_bc(1);
+                issue_x(0);
+                mbar_arrive(&s.xslot_free);   // chunk 0's w o X goes into the untouched slot 1
             }
-            if (__shfl_sync(0xffffffffu, stop, 0)) ok = false;
+            ok = ewait(&s.full_bc[0], 0, abort, lim);
+            if (ok) {
+                tc_fence_after();
+                if (lane == 0) { ++bc_waited; issue_g(0); }
+                __syncwarp();
+                // Ys of chunk 0 once the warps have written hp of the state entering the stripe
+                ok = ewait(&s.st0_ready, 0, abort, lim);
+                if (ok) {
+                    tc_fence_after();
+                    if (lane == 0) issue_ys(0);
+                    __syncwarp();
+                }
+            }
+        }
+        for (int c = 0; ok && c < nc; ++c) {
+            const int64_t t0 = s0 + (int64_t)c * kQ;
+            uint8_t *xs = s.x[c & 1];
+            // the decay has read G: G of chunk c+1 into R0, under this chunk's products
+            ok = ewait(&s.pm_ready, c & 1, abort, lim);
+            if (!ok) break;
+            if (c + 1 < nc) {
+                ok = ewait(&s.full_bc[(c + 1) & 1], ((c + 1) >> 1) & 1, abort, lim);
+                if (!ok) break;
+                tc_fence_after();
+                if (lane == 0) { ++bc_waited; issue_g(c + 1); }
+                __syncwarp();
+            }
+            // Pm written, T (= Ys) scaled, X landed: Y_a, Y_b accumulate into T
+            ok = ewait(&s.ts_ready, c & 1, abort, lim) && ewait(&s.full_x[c & 1], (c >> 1) & 1, abort, lim);
+            if (!ok) break;
+            tc_fence_after();
+            if (lane == 0) {
+                ++x_waited;
+                const uint64_t dx = (c & 1) ? dX1 : dX0;
+#pragma unroll
+                for (int hd2 = 0; hd2 < 2; ++hd2)
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts(tT + 64 * hd2, tPm + 64 * hd2 + kk * 8, dx + hd2 * kBoxD + moff(kk), id_pm, true);
+            }
+            __syncwarp();
+            // w o X of both heads: S = B^T [Xw_a | Xw_b] accumulates into H
+            ok = ewait(&s.xw_ready, c & 1, abort, lim);
+            if (!ok) break;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint64_t dbt = (c & 1) ? dBt1 : dBt0, dxw = (c & 1) ? dXw0 : dXw1;   // w o X is in slot (c+1) & 1
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) mma_ss(tH, dbt + moff(kk), dxw + moff(kk), id_s, true);
+                mma_commit(&s.mma_done);
+            }
+            __syncwarp();
+            // products done: refill this B/C slot, and load chunk c+1's X into the slot S read w o X from
+            ok = ewait(&s.mma_done, c & 1, abort, lim);
+            if (!ok) break;
+            if (lane == 0 && c + 2 < nc) issue_bc(c + 2);
+            if (lane == 0 && c + 1 < nc) issue_x(c + 1);
+            __syncwarp();
+            // y staged and hp of chunk c+1 written: store y, start Ys of chunk c+1 (T has been read)
+            ok = ewait(&s.y_ready, c & 1, abort, lim);
+            if (!ok) break;
+            tc_fence_after();
+            if (lane == 0) {
+                tma_store_3d(&maps.y, xs, ha * kP, (int)t0, bi);
+                tma_store_3d(&maps.y, xs + kBox, (ha + 1) * kP, (int)t0, bi);
+                tma_store_commit();
+                if (c + 1 < nc) issue_ys(c + 1);
+                // once the store has read the slot, chunk c+1 may write its w o X there
+                tma_store_wait_read<0>();
+                mbar_arrive(&s.xslot_free);
+            }
+            __syncwarp();
         }
         if (lane == 0) {
             if (live && !ok) raise_timeout(p, abort);
-            // every MMA complete before TMEM is freed
+            // every MMA complete before TMEM is freed (after an abort: drain the loads too)
             mma_commit(&s.fin);
             mbar_wait(&s.fin, 0, nullptr, 100000000ull);
             if (*abort) {
-                // drain every load issued but not observed
-                for (int i = o_bc; i < n_bc; ++i)
+                for (int i = bc_waited; i < bc_issued; ++i)
                     mbar_wait(&s.full_bc[i & 1], (i >> 1) & 1, nullptr, 100000000ull);
-                for (int i = o_x; i < n_x; ++i)
+                for (int i = x_waited; i < x_issued; ++i)
                     mbar_wait(&s.full_x[i & 1], (i >> 1) & 1, nullptr, 100000000ull);
             }
             tma_store_wait<0>();
@@ -1139,6 +1013,8 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
     __syncthreads();
     if (warp == 0) tmem_dealloc(tm, 512);
 }
+
+// =============================================================== host side
 
 // =============================================================== host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -1202,11 +1078,10 @@ int launch_scan_tc(const ScanParams &p, cudaStream_t st)
     Maps maps;
     const int64_t gn = (int64_t)p.G * p.N;
     const bool fused = p.conv_w != nullptr;
-    if (fused && !encode_bf16(enc, &maps.ux, p.conv_u, (int64_t)p.H * p.P, p.L, p.b, p.conv_urs, p.conv_ubs,
-                              kQ + kHaloRows))
-        return 6;
-    if (!fused && !encode_bf16(enc, &maps.x, p.x, (int64_t)p.H * p.P, p.L, p.b, p.xrs, p.xbs)) return 6;
-    if ((fused && !encode_bf16(enc, &maps.x, p.conv_u, (int64_t)p.H * p.P, p.L, p.b, p.conv_urs, p.conv_ubs)) ||
+    if (fused && (p.ns <= 1 || !encode_bf16(enc, &maps.ux, p.conv_u, (int64_t)p.H * p.P, p.L, p.b, p.conv_urs,
+                                            p.conv_ubs, kQ + kHaloRows)))
+        return 6;   // the fused conv lives in pass A, which a single stripe does not run
+    if (!encode_bf16(enc, &maps.x, p.x, (int64_t)p.H * p.P, p.L, p.b, p.xrs, p.xbs) ||
         !encode_bf16(enc, &maps.B, p.B, gn, p.L, p.b, p.Brs, p.Bbs) ||
         !encode_bf16(enc, &maps.C, p.C, gn, p.L, p.b, p.Crs, p.Cbs) ||
         !encode_bf16(enc, &maps.y, p.y, (int64_t)p.H * p.P, p.L, p.b, p.yrs, p.ybs))
@@ -1217,8 +1092,7 @@ int launch_scan_tc(const ScanParams &p, cudaStream_t st)
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
         if (cudaFuncSetAttribute(stripe_state_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemA) != cudaSuccess ||
             cudaFuncSetAttribute(stripe_state_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemA) != cudaSuccess ||
-            cudaFuncSetAttribute(chunk_output_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemC) != cudaSuccess ||
-            cudaFuncSetAttribute(chunk_output_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemC) != cudaSuccess)
+            cudaFuncSetAttribute(chunk_output_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemC) != cudaSuccess)
             return 7;
         attr_set[dev] = true;
     }
@@ -1232,8 +1106,7 @@ int launch_scan_tc(const ScanParams &p, cudaStream_t st)
         if (rc) return rc;
     }
     prof_begin(st, kKOutputTc);
-    if (fused) chunk_output_tc_kernel<true><<<(unsigned)(units / 2), kThreadsC, kSmemC, st>>>(maps, p);
-    else chunk_output_tc_kernel<false><<<(unsigned)(units / 2), kThreadsC, kSmemC, st>>>(maps, p);
+    chunk_output_tc_kernel<<<(unsigned)(units / 2), kThreadsC, kSmemC, st>>>(maps, p);
     prof_end(st, kKOutputTc);
     return cudaGetLastError() == cudaSuccess ? 0 : 7;
 }

@@ -191,6 +191,8 @@ struct FusedConv {
     const float *w, *bias;
     const void *tail;
     int C_ch;
+    void *v;                 // where pass A writes the conv output of x
+    int64_t vbs, vrs;
 };
 
 int scan_impl(const ssd_scan_args *a, cudaStream_t st, const FusedConv *fc = nullptr)
@@ -254,6 +256,7 @@ int scan_impl(const ssd_scan_args *a, cudaStream_t st, const FusedConv *fc = nul
     if (fc) {
         p.conv_u = fc->u; p.conv_ubs = fc->ubs; p.conv_urs = fc->urs;
         p.conv_w = fc->w; p.conv_bias = fc->bias; p.conv_tail = fc->tail; p.conv_cch = fc->C_ch;
+        p.conv_v = fc->v; p.conv_vbs = fc->vbs; p.conv_vrs = fc->vrs;
     }
     const EnvHooks &hooks = env_hooks();
     p.wait_limit_ns = hooks.wait_limit_ns;
@@ -263,7 +266,7 @@ int scan_impl(const ssd_scan_args *a, cudaStream_t st, const FusedConv *fc = nul
     const bool force_generic = hooks.force_generic;
     rc = 6;
     if (!force_generic && ssd::tc_scan_supported(p, a->dtype)) rc = ssd::launch_scan_tc(p, st);
-    if (fc && rc == 6) return fail(SSD_ERR_UNSUPPORTED, "the fused conv needs the tensor-core scan (dt 8-byte aligned)");
+    if (fc && rc == 6) return fail(SSD_ERR_UNSUPPORTED, "the fused conv needs the tensor-core scan");
     if (rc == 6) rc = ssd::launch_scan_generic(p, a->dtype, st);
     if (rc == 6) return fail(SSD_ERR_UNSUPPORTED, "no GPU kernel for this shape (P=%d N=%d Q=%d)", a->P, a->N, a->Q);
     if (rc) return fail(SSD_ERR_LAUNCH, "scan launch failed: %s", cudaGetErrorString(cudaGetLastError()));
@@ -404,7 +407,8 @@ int layer_bwd_impl(const ssd_layer_bwd_args *a, cudaStream_t st)
     const int HP = a->H * a->P, GN = a->G * a->N;
     const int C_ch = HP + 2 * GN;
     const size_t es = elem_size(a->dtype);
-    if (!a->dconv_w || !a->dA || !a->du || !a->ddt) return fail(SSD_ERR_NULL, "du, dconv_w, ddt and dA must not be NULL");
+    if (!a->dconv_w || !a->dA || (a->L > 0 && (!a->du || !a->ddt)))
+        return fail(SSD_ERR_NULL, "du, dconv_w, ddt and dA must not be NULL");
     if (!a->conv_w || !aligned16(a->conv_w) || !aligned16(a->dconv_w))
         return fail(SSD_ERR_ALIGN, "conv_w and dconv_w must be given, 16-byte aligned");
     const void *vec[] = {a->tail_in, a->conv_ckpt, a->du, a->dtail_in, a->h0, a->h_ckpt, a->dh_final, a->dh0};
@@ -564,10 +568,8 @@ void prof_end(cudaStream_t st, int id)
 namespace {
 
 // Workspace of ssd_stream_forward without v: the scan's workspace, then the conv output
-// the scan still reads from memory -- B and C only ([b][L][2GN]) when the x conv is fused
-// into the tensor-core scan, all of v ([b][L][C_ch]) on the CUDA-core path.
+// v [b][L][C_ch] that the output pass reads.
 struct StreamPlan {
-    bool fused = false;
     size_t off_v = 0, bytes = 0;
 };
 
@@ -575,71 +577,78 @@ StreamPlan make_stream_plan(int b, int64_t L, int H, int P, int N, int G, int Q,
 {
     StreamPlan sp;
     const Plan pl = make_plan(b, L, H, P, N, Q);
-    sp.fused = ssd::tc_scan_shape(dtype, H, P, N, G, Q);
-    const size_t cols = sp.fused ? 2 * (size_t)G * N : (size_t)H * P + 2 * (size_t)G * N;
     sp.off_v = round256(pl.bytes_dt);
-    sp.bytes = sp.off_v + round256((size_t)b * L * cols * elem_size(dtype));
+    sp.bytes = sp.off_v + round256((size_t)b * L * ((size_t)H * P + 2 * (size_t)G * N) * elem_size(dtype));
     return sp;
 }
 
-int stream_fused_impl(const ssd_stream_args *a, cudaStream_t st)
+// One streamed segment, L > 0 and b > 0.  On the tensor-core shapes with more than one
+// stripe the conv of x runs inside pass A (which writes x = v[:, :H*P]) and a conv kernel
+// covers only the B and C channels; otherwise one conv kernel covers every channel.
+int stream_impl(const ssd_stream_args *a, cudaStream_t st)
 {
     const int HP = a->H * a->P, GN = a->G * a->N;
     const int C_ch = HP + 2 * GN;
     const size_t es = elem_size(a->dtype);
-    const StreamPlan sp = make_stream_plan(a->b, a->L, a->H, a->P, a->N, a->G, a->Q, a->dtype);
-    if (!a->workspace || a->workspace_bytes < sp.bytes)
-        return fail(SSD_ERR_WORKSPACE, "workspace of %zu bytes needed (ssd_stream_workspace_size), %zu given",
-                    sp.bytes, a->workspace ? a->workspace_bytes : (size_t)0);
-    if ((reinterpret_cast<uintptr_t>(a->workspace) & 255u) != 0)
-        return fail(SSD_ERR_ALIGN, "workspace must be 256-byte aligned");
     int rc = check_rows("u", a->u, a->u_batch_stride, a->u_row_stride, C_ch, a->b, a->L, a->dtype, true);
     if (rc) return rc;
-    if (!a->conv_w || !aligned16(a->conv_w)) return fail(SSD_ERR_ALIGN, "conv_w must be given, 16-byte aligned");
+    if (!a->conv_w) return fail(SSD_ERR_NULL, "conv weight w is NULL");
+    if (!aligned16(a->conv_w)) return fail(SSD_ERR_ALIGN, "conv weight w must be 16-byte aligned");
     if ((a->tail_in && !aligned16(a->tail_in)) || (a->tail_out && !aligned16(a->tail_out)) ||
         (a->conv_ckpt && !aligned16(a->conv_ckpt)))
-        return fail(SSD_ERR_ALIGN, "conv tails must be 16-byte aligned");
-    char *vws = static_cast<char *>(a->workspace) + sp.off_v;
-    const char *u = static_cast<const char *>(a->u);
+        return fail(SSD_ERR_ALIGN, "conv tails and conv_ckpt must be 16-byte aligned");
+    char *v;
+    int64_t vbs, vrs;
+    size_t scan_ws_bytes = a->workspace_bytes;
+    if (a->v) {
+        if ((rc = check_rows("v", a->v, a->v_batch_stride, a->v_row_stride, C_ch, a->b, a->L, a->dtype, true)))
+            return rc;
+        v = static_cast<char *>(a->v); vbs = a->v_batch_stride; vrs = a->v_row_stride;
+    } else {
+        const StreamPlan sp = make_stream_plan(a->b, a->L, a->H, a->P, a->N, a->G, a->Q, a->dtype);
+        if (!a->workspace || a->workspace_bytes < sp.bytes)
+            return fail(SSD_ERR_WORKSPACE, "workspace of %zu bytes needed (ssd_stream_workspace_size), %zu given",
+                        sp.bytes, a->workspace ? a->workspace_bytes : (size_t)0);
+        if ((reinterpret_cast<uintptr_t>(a->workspace) & 255u) != 0)
+            return fail(SSD_ERR_ALIGN, "workspace must be 256-byte aligned");
+        v = static_cast<char *>(a->workspace) + sp.off_v; vbs = a->L * C_ch; vrs = C_ch;
+        scan_ws_bytes = sp.off_v;
+    }
+    const Plan pl = make_plan(a->b, a->L, a->H, a->P, a->N, a->Q);
+    const bool fuse = ssd::tc_scan_shape(a->dtype, a->H, a->P, a->N, a->G, a->Q) && pl.ns > 1 &&
+                      !env_hooks().force_generic && (reinterpret_cast<uintptr_t>(a->dt) & 7u) == 0 &&
+                      a->L < (1LL << 31) && (int64_t)a->b * pl.ns * a->H < (1LL << 31);
+    ssd::ConvParams cp{};
+    cp.ubs = a->u_batch_stride; cp.urs = a->u_row_stride; cp.tail_rs = C_ch;
+    cp.vbs = vbs; cp.vrs = vrs; cp.b = a->b; cp.L = a->L;
+    if (fuse) {
+        // the B and C channels' conv into v[:, H*P:] (their rows before token 0 from tail_in's B/C columns)
+        cp.u = static_cast<const char *>(a->u) + es * HP;
+        cp.w = a->conv_w + 4 * HP; cp.bias = a->conv_bias ? a->conv_bias + HP : nullptr;
+        cp.tail_in = a->tail_in ? static_cast<const char *>(a->tail_in) + es * HP : nullptr;
+        cp.v = v + es * HP; cp.C_ch = 2 * GN;
+    } else {
+        cp.u = a->u; cp.w = a->conv_w; cp.bias = a->conv_bias; cp.tail_in = a->tail_in;
+        cp.v = v; cp.C_ch = C_ch;
+    }
+    rc = ssd::launch_conv(cp, a->dtype, st);
+    if (rc == 2) return fail(SSD_ERR_SHAPE, "conv grid too large");
+    if (rc) return fail(SSD_ERR_LAUNCH, "conv launch failed: %s", cudaGetErrorString(cudaGetLastError()));
     ssd_scan_args s{};
     s.dtype = a->dtype; s.b = a->b; s.L = a->L; s.H = a->H; s.P = a->P; s.N = a->N; s.G = a->G;
     s.Q = a->Q; s.s = a->s;
+    s.x = v; s.x_batch_stride = vbs; s.x_row_stride = vrs;
+    s.B = v + es * HP; s.B_batch_stride = vbs; s.B_row_stride = vrs;
+    s.C = v + es * (HP + GN); s.C_batch_stride = vbs; s.C_row_stride = vrs;
     s.dt = a->dt; s.A = a->A; s.D = a->D; s.h0 = a->h0;
     s.dt_bias = a->dt_bias; s.dt_softplus = a->dt_softplus; s.dt_min = a->dt_min; s.dt_max = a->dt_max;
     s.y = a->y; s.y_batch_stride = a->y_batch_stride; s.y_row_stride = a->y_row_stride;
     s.h_final = a->h_final; s.h_ckpt = a->h_ckpt;
-    s.workspace = a->workspace; s.workspace_bytes = sp.off_v;
-    if (sp.fused) {
-        // 1. the conv of the B and C channels only, into the workspace ([b][L][2GN]); their rows
-        //    before token 0 are tail_in's B/C columns
-        ssd::ConvParams cp{};
-        cp.u = u + es * HP; cp.ubs = a->u_batch_stride; cp.urs = a->u_row_stride;
-        cp.w = a->conv_w + 4 * HP; cp.bias = a->conv_bias ? a->conv_bias + HP : nullptr;
-        cp.tail_in = a->tail_in ? static_cast<const char *>(a->tail_in) + es * HP : nullptr;
-        cp.tail_rs = C_ch;
-        cp.v = vws; cp.vbs = a->L * 2 * GN; cp.vrs = 2 * GN; cp.b = a->b; cp.L = a->L; cp.C_ch = 2 * GN;
-        rc = ssd::launch_conv(cp, a->dtype, st);
-        if (rc == 2) return fail(SSD_ERR_SHAPE, "conv grid too large");
-        if (rc) return fail(SSD_ERR_LAUNCH, "conv launch failed: %s", cudaGetErrorString(cudaGetLastError()));
-        // 2. the scan, x read from u's x columns with its conv fused in
-        s.x = u; s.x_batch_stride = a->u_batch_stride; s.x_row_stride = a->u_row_stride;
-        s.B = vws; s.B_batch_stride = a->L * 2 * GN; s.B_row_stride = 2 * GN;
-        s.C = vws + es * GN; s.C_batch_stride = a->L * 2 * GN; s.C_row_stride = 2 * GN;
-        FusedConv fc{a->u, a->u_batch_stride, a->u_row_stride, a->conv_w, a->conv_bias, a->tail_in, C_ch};
-        rc = scan_impl(&s, st, &fc);
-        if (rc) return rc;
-    } else {
-        // CUDA-core path: the whole conv output in the workspace, then the scan
-        rc = conv_impl(a->u, a->u_batch_stride, a->u_row_stride, a->conv_w, a->conv_bias, a->tail_in, nullptr, vws,
-                       a->L * C_ch, C_ch, a->b, a->L, C_ch, a->dtype, st);
-        if (rc) return rc;
-        s.x = vws; s.x_batch_stride = a->L * C_ch; s.x_row_stride = C_ch;
-        s.B = vws + es * HP; s.B_batch_stride = a->L * C_ch; s.B_row_stride = C_ch;
-        s.C = vws + es * (HP + GN); s.C_batch_stride = a->L * C_ch; s.C_row_stride = C_ch;
-        rc = scan_impl(&s, st);
-        if (rc) return rc;
-    }
-    // 3. the conv buffers: at every checkpoint, and tail_out (last: it may alias tail_in)
+    s.workspace = a->workspace; s.workspace_bytes = scan_ws_bytes;
+    FusedConv fc{a->u, a->u_batch_stride, a->u_row_stride, a->conv_w, a->conv_bias, a->tail_in, C_ch, v, vbs, vrs};
+    rc = scan_impl(&s, st, fuse ? &fc : nullptr);
+    if (rc) return rc;
+    // the conv buffers: at every checkpoint, and tail_out (last: it may alias tail_in)
     if (a->conv_ckpt && a->s > 0 && a->L >= a->s) {
         if (ssd::launch_conv_ckpt(a->u, a->u_batch_stride, a->u_row_stride, a->conv_ckpt, a->b, a->L, C_ch, a->s,
                                   a->dtype, st))
@@ -723,10 +732,10 @@ int ssd_stream_forward(const ssd_stream_args *a, ssd_stream_t stream)
     if (!a) return fail(SSD_ERR_NULL, "args is NULL");
     int rc = check_scan_shape(a->dtype, a->b, a->L, a->H, a->P, a->N, a->G, a->Q, a->s);
     if (rc) return rc;
-    if (!a->v && a->L > 0 && a->b > 0) return stream_fused_impl(a, (cudaStream_t)stream);
+    if (a->L > 0 && a->b > 0) return stream_impl(a, (cudaStream_t)stream);
+    // no token (or no batch row): tail_out from tail_in, h_final from h0
     const int d_inner = a->H * a->P;
     const int C_ch = d_inner + 2 * a->G * a->N;
-    if (a->L > 0 && !a->v) return fail(SSD_ERR_NULL, "v is NULL");
     if (a->conv_ckpt && a->s > 0 && a->L >= a->s) {
         if (!aligned16(a->conv_ckpt)) return fail(SSD_ERR_ALIGN, "conv_ckpt must be 16-byte aligned");
         if (!a->u) return fail(SSD_ERR_NULL, "u is NULL");

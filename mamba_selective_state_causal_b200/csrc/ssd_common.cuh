@@ -47,11 +47,14 @@ struct ScanParams {
     const float *dt_bias;
     int dt_softplus;
     float dt_min, dt_max;
-    // the conv of x fused into the tensor-core passes (ssd_stream_forward without v):
-    // x is then read from the conv input u (same columns) and turned into
-    // silu(conv(u)) in shared memory; NULL conv_w means x is given
+    // the conv of x fused into pass A (ssd_stream_forward on the tensor-core shapes):
+    // pass A reads x's columns of the conv input u, turns them into
+    // silu(conv(u)) in shared memory and writes that x to conv_v (which the
+    // output pass then reads as x); NULL conv_w means x is given
     const void *conv_u;
     int64_t conv_ubs, conv_urs;
+    void *conv_v;
+    int64_t conv_vbs, conv_vrs;
     const float *conv_w;        // [C_ch][4]
     const float *conv_bias;     // [C_ch] or NULL
     const void *conv_tail;      // [b][3][C_ch] (the rows before token 0) or NULL (zeros)

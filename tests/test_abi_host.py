@@ -139,15 +139,16 @@ def test_conv_rejects_bad_arguments(ssd):
 
 
 def test_stream_without_v_needs_its_workspace(ssd):
-    """v = NULL asks for the fused path, whose workspace (ssd_stream_workspace_size) holds
-    only the B/C conv output on the tensor-core shapes and all of it elsewhere."""
+    """v = NULL keeps the conv output in the workspace (ssd_stream_workspace_size): the
+    scan's workspace, then [b][L][C_ch] of the I/O dtype."""
     a = ssd.StreamArgs()
     a.dtype = 1; a.b = 1; a.L = 64; a.H = 2; a.P = 64; a.N = 128; a.G = 1; a.Q = 128; a.s = 0
     a.u = 0x1000; a.u_row_stride = 384; a.u_batch_stride = 64 * 384
     a.conv_w = 0x2000; a.v = None
     assert ssd.lib().ssd_stream_forward(ctypes.byref(a), None) == 9
     scan = ssd.workspace_size(2, 131072, 32, 64, 128, 128)
-    tc = ssd.stream_workspace_size(2, 131072, 32, 64, 128, 1, 128, ssd.SSD_BF16)
-    assert tc >= scan + 2 * 131072 * 256 * 2 and tc < scan + 2 * 131072 * 256 * 2 + 1024
+    v = 2 * 131072 * (32 * 64 + 256)
+    bf = ssd.stream_workspace_size(2, 131072, 32, 64, 128, 1, 128, ssd.SSD_BF16)
+    assert scan + 2 * v <= bf < scan + 2 * v + 1024
     f32 = ssd.stream_workspace_size(2, 131072, 32, 64, 128, 1, 128, ssd.SSD_F32)
-    assert f32 >= 2 * 131072 * (32 * 64 + 256) * 4
+    assert scan + 4 * v <= f32 < scan + 4 * v + 1024

@@ -19,9 +19,11 @@ pytestmark = pytest.mark.gpu
 W = ssd_synth.WORKLOADS
 
 
-def gpu_layer(wl, u, prm, dt, segments=1, h0=None, tail=None, zero_tail_at=None, fused=False):
-    """Run the layer on the GPU as `segments` consecutive resumed calls; fused=True asks for
-    no conv output (the conv of x then runs inside the tensor-core scan kernels)."""
+def gpu_layer(wl, u, prm, dt, segments=1, h0=None, tail=None, zero_tail_at=None, fused=False, two_call=False):
+    """Run the layer on the GPU as `segments` consecutive resumed calls of ssd_stream_forward
+    (on the tensor-core shapes the conv of x runs inside the scan's first pass); fused=True
+    asks for no conv output (v in the workspace); two_call=True uses ssd_conv_forward then
+    ssd_scan_forward instead (one conv kernel over every channel)."""
     d = "cuda"
     g = {k: v.to(d) for k, v in prm.items()}
     L = u.shape[1]
@@ -39,9 +41,18 @@ def gpu_layer(wl, u, prm, dt, segments=1, h0=None, tail=None, zero_tail_at=None,
         sl = slice(k * seg, (k + 1) * seg if k < segments - 1 else L)
         if zero_tail_at is not None and k == zero_tail_at:
             tl = torch.zeros_like(tl)
-        out = ssd.stream_forward(u[:, sl], g["w"], dt[:, sl], g["A"], g["D"], H=wl.H, P=wl.P,
-                                 N=wl.N, G=wl.G, Q=wl.Q, s=wl.s, conv_bias=g["bias"], tail_in=tl,
-                                 h0=st, workspace=ws if sl.stop - sl.start == seg else None, keep_v=not fused)
+        if two_call:
+            to = torch.empty(wl.b, 3, wl.cch, dtype=u.dtype, device=d)
+            v, _ = ssd.conv_forward(u[:, sl], g["w"], g["bias"], tail_in=tl, tail_out=to)
+            di, gn = wl.H * wl.P, wl.G * wl.N
+            y, hf, hc = ssd.scan_forward(v[:, :, :di], v[:, :, di:di + gn], v[:, :, di + gn:], dt[:, sl], g["A"],
+                                         g["D"], st, H=wl.H, G=wl.G, Q=wl.Q, s=wl.s)
+            out = {"y": y, "h_final": hf, "h_ckpt": hc, "tail_out": to}
+        else:
+            out = ssd.stream_forward(u[:, sl], g["w"], dt[:, sl], g["A"], g["D"], H=wl.H, P=wl.P,
+                                     N=wl.N, G=wl.G, Q=wl.Q, s=wl.s, conv_bias=g["bias"], tail_in=tl,
+                                     h0=st, workspace=ws if sl.stop - sl.start == seg else None,
+                                     keep_v=not fused)
         st, tl = out["h_final"], out["tail_out"]
         ys.append(out["y"])
         if out["h_ckpt"] is not None:
@@ -72,7 +83,7 @@ def oracle_layer(wl, u, prm, dt, heads=None, h0=None, tail=None):
                         G=1, s=wl.s, io_round=io)
 
 
-FUSED = pytest.mark.parametrize("fused", [False, True], ids=["two_call", "fused"])
+FUSED = pytest.mark.parametrize("fused", [False, True], ids=["v_returned", "v_in_workspace"])
 
 
 @FUSED
@@ -136,10 +147,10 @@ def test_resume_without_conv_tail_differs(fused):
 
 
 def test_fused_conv_equals_two_call_path_bitwise():
-    """The conv of x fused into the tensor-core scan computes x exactly as the conv kernel
-    does (same fused multiply-adds, same SiLU, same rounding), so the fused layer equals
-    the two-call layer bit for bit: several stripes, a ragged tail, a conv buffer and a
-    state handed in, two batch rows."""
+    """The conv of x fused into the scan's first pass computes x exactly as the conv kernel
+    does (same fused multiply-adds, same SiLU, same rounding), so ssd_stream_forward equals
+    ssd_conv_forward followed by ssd_scan_forward bit for bit: several stripes, a ragged
+    tail, a conv buffer and a state handed in, two batch rows."""
     wl = ssd_synth.scaled(W[1], L=3 * 2048 + 77, H=4, b=2, s=1024)
     prm = ssd_synth.make_params(wl)
     prm["bias"] = ssd_synth.make_conv_grads(wl)[1]
@@ -147,10 +158,11 @@ def test_fused_conv_equals_two_call_path_bitwise():
     dt = ssd_synth.make_dt(wl, prm["dt_bias"]).cuda()
     h0 = ssd_synth.make_h0(wl, scale=0.5)
     tail = ssd_synth.make_tail(wl)
-    a = gpu_layer(wl, u, prm, dt, h0=h0, tail=tail, fused=False)
-    b = gpu_layer(wl, u, prm, dt, h0=h0, tail=tail, fused=True)
-    for k in ("y", "h_final", "h_ckpt", "tail_out"):
-        assert torch.equal(a[k], b[k]), (k, rel_l2(host(a[k]), host(b[k])))
+    a = gpu_layer(wl, u, prm, dt, h0=h0, tail=tail, two_call=True)
+    for fused in (False, True):
+        b = gpu_layer(wl, u, prm, dt, h0=h0, tail=tail, fused=fused)
+        for k in ("y", "h_final", "h_ckpt", "tail_out"):
+            assert torch.equal(a[k], b[k]), (fused, k, rel_l2(host(a[k]), host(b[k])))
 
 
 def _sampled_full_size(wl, heads, fused=True):
