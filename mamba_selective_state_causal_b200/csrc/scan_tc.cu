@@ -89,37 +89,65 @@ __device__ __forceinline__ uint32_t scale_bf16x2_int(uint32_t v, float w)
     return pack_bf16x2_int(bf16_lo(v) * w, bf16_hi(v) * w);
 }
 
-// SiLU(z) = z (1 + tanh(z / 2)) / 2 with the hardware tanh: the conv kernel's form, so that
-// a fused conv reproduces its bf16 output bit for bit
-__device__ __forceinline__ float silu_tanh(float z)
+// two fp32 products / fused multiply-adds in one instruction (sm_100 packed fp32); each lane
+// rounds exactly as the scalar instruction does
+__device__ __forceinline__ float2 mul2(float2 a, float2 b)
 {
-    float t;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
-    return z * fmaf(0.5f, t, 0.5f);
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
 }
 
-// Conv + SiLU of 8 channels of one token: window m3 = u[t-3], m2, m1, cur = u[t]
-__device__ __forceinline__ uint4 conv8(const float (&w)[8][4], const float (&bs)[8], const float (&m3)[8],
-                                       const float (&m2)[8], const float (&m1)[8], const float (&cur)[8])
+__device__ __forceinline__ float2 unpack2(uint32_t v) { return make_float2(bf16_lo(v), bf16_hi(v)); }
+
+// Conv + SiLU of 8 channels (4 pairs) of one token: window m3 = u[t-3], m2, m1, cur = u[t],
+// weights w[pair][tap] and bias as channel pairs.  The same operations, in the same order
+// and rounding, as the conv kernel's scalar code, two channels per instruction.
+__device__ __forceinline__ uint4 conv8(const float2 (&w)[4][4], const float2 (&bs)[4], const float2 (&m3)[4],
+                                       const float2 (&m2)[4], const float2 (&m1)[4], const float2 (&cur)[4])
 {
-    float o[8];
+    uint32_t o[4];
+    const float2 half = make_float2(0.5f, 0.5f);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        float z = bs[i];
-        z = fmaf(w[i][0], m3[i], z);
-        z = fmaf(w[i][1], m2[i], z);
-        z = fmaf(w[i][2], m1[i], z);
-        z = fmaf(w[i][3], cur[i], z);
-        o[i] = silu_tanh(z);
+    for (int i = 0; i < 4; ++i) {
+        float2 z = fma2(w[i][0], m3[i], bs[i]);
+        z = fma2(w[i][1], m2[i], z);
+        z = fma2(w[i][2], m1[i], z);
+        z = fma2(w[i][3], cur[i], z);
+        const float2 h = mul2(half, z);
+        float2 t;
+        asm("tanh.approx.f32 %0, %1;" : "=f"(t.x) : "f"(h.x));
+        asm("tanh.approx.f32 %0, %1;" : "=f"(t.y) : "f"(h.y));
+        const float2 sg = mul2(z, fma2(half, t, half));
+        o[i] = pack_bf16x2(sg.x, sg.y);
     }
-    return make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
-                      pack_bf16x2(o[6], o[7]));
+    return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-__device__ __forceinline__ void unpack8(uint4 v, float (&f)[8])
+__device__ __forceinline__ void unpack8(uint4 v, float2 (&f)[4])
 {
-    f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x); f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
-    f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z); f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+    f[0] = unpack2(v.x); f[1] = unpack2(v.y); f[2] = unpack2(v.z); f[3] = unpack2(v.w);
+}
+
+// bf16 pair times w, rounded to nearest even (cvt)
+__device__ __forceinline__ uint32_t scale_bf16x2_rn(uint32_t v, float2 w2)
+{
+    const float2 p = mul2(unpack2(v), w2);
+    return pack_bf16x2(p.x, p.y);
 }
 
 __device__ __forceinline__ void raise_timeout(const ScanParams &p, volatile int *abort)
@@ -204,14 +232,17 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
         const int hd = warp >> 3, j = 32 * (warp & 3) + lane, c0 = 4 * ((warp >> 2) & 1);
         // fused conv: 16-byte column ch (8 channels) of rows 4 rg .. 4 rg + 3 of head hd
         const int ch = lane & 7, rg = (lane >> 3) + 4 * (warp & 7);
-        float cw[8][4], cb[8];
+        float2 cw[4][4], cb[4];   // weights [channel pair][tap] and bias of this thread's 8 channels
         if (kFused) {
             const int c0ch = (ha + hd) * kP + 8 * ch;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float4 q4 = __ldg(reinterpret_cast<const float4 *>(p.conv_w) + c0ch + i);
-                cw[i][0] = q4.x; cw[i][1] = q4.y; cw[i][2] = q4.z; cw[i][3] = q4.w;
-                cb[i] = p.conv_bias ? __ldg(p.conv_bias + c0ch + i) : 0.0f;
+            for (int i = 0; i < 4; ++i) {
+                const float4 qa = __ldg(reinterpret_cast<const float4 *>(p.conv_w) + c0ch + 2 * i);
+                const float4 qb = __ldg(reinterpret_cast<const float4 *>(p.conv_w) + c0ch + 2 * i + 1);
+                cw[i][0] = make_float2(qa.x, qb.x); cw[i][1] = make_float2(qa.y, qb.y);
+                cw[i][2] = make_float2(qa.z, qb.z); cw[i][3] = make_float2(qa.w, qb.w);
+                cb[i] = p.conv_bias ? make_float2(__ldg(p.conv_bias + c0ch + 2 * i), __ldg(p.conv_bias + c0ch + 2 * i + 1))
+                                    : make_float2(0.0f, 0.0f);
             }
         }
         bool ok = true;
@@ -223,7 +254,7 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
             if (kFused) {
                 uint8_t *box = s.stage[st] + 2 * kBox + hd * kBoxX;   // row r of the chunk is box row r + 8
                 const int64_t t0 = s0 + (int64_t)(nc - 1 - it) * kQ;
-                float m3[8], m2[8], m1[8];
+                float2 m3[4], m2[4], m1[4];
                 if (t0 == 0 && rg == 0) {
                     // the rows before the sequence: the conv buffer handed in, or zeros
                     const __nv_bfloat16 *tin = p.conv_tail
@@ -249,28 +280,30 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
                 for (int i = 0; i < 4; ++i) {
                     const int r = 4 * rg + i;
                     uint8_t *a = box + swz(r + kHaloRows, ch);
-                    float cur[8];
+                    float2 cur[4];
                     unpack8(lds128(a), cur);
                     uint4 v = conv8(cw, cb, m3, m2, m1, cur);
                     if (t0 + r < s1)
                         *reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.conv_v) + (int64_t)bi * p.conv_vbs +
                                                    (t0 + r) * p.conv_vrs + (ha + hd) * kP + 8 * ch) = v;
                     const float w = s.w[st][hd][r];
-                    v.x = scale_bf16x2_int(v.x, w); v.y = scale_bf16x2_int(v.y, w);
-                    v.z = scale_bf16x2_int(v.z, w); v.w = scale_bf16x2_int(v.w, w);
+                    const float2 w2 = make_float2(w, w);
+                    v.x = scale_bf16x2_rn(v.x, w2); v.y = scale_bf16x2_rn(v.y, w2);
+                    v.z = scale_bf16x2_rn(v.z, w2); v.w = scale_bf16x2_rn(v.w, w2);
                     sts128(a, v);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) { m3[e] = m2[e]; m2[e] = m1[e]; m1[e] = cur[e]; }
+                    for (int e = 0; e < 4; ++e) { m3[e] = m2[e]; m2[e] = m1[e]; m1[e] = cur[e]; }
                 }
             } else {
                 const float w = s.w[st][hd][j];
+                const float2 w2 = make_float2(w, w);
                 uint8_t *xrow = s.stage[st] + 2 * kBox + hd * kBoxX + kHaloRows * 128;
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
                     const uint32_t o = swz(j, c0 + cc);
                     uint4 vv = lds128(xrow + o);
-                    vv.x = scale_bf16x2_int(vv.x, w); vv.y = scale_bf16x2_int(vv.y, w);
-                    vv.z = scale_bf16x2_int(vv.z, w); vv.w = scale_bf16x2_int(vv.w, w);
+                    vv.x = scale_bf16x2_rn(vv.x, w2); vv.y = scale_bf16x2_rn(vv.y, w2);
+                    vv.z = scale_bf16x2_rn(vv.z, w2); vv.w = scale_bf16x2_rn(vv.w, w2);
                     sts128(xrow + o, vv);
                 }
             }
@@ -448,66 +481,57 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
 // The output accumulator T of a chunk first receives Ys = C [hp_a | hp_b]^T
 // (the contribution of the state entering the chunk), which the compute warps
 // scale row by row by exp(cs_i); Y = Pm X then accumulates onto it, so the
-// epilogue only adds D x.  Ys of chunk c is computed while the warps work on
-// chunk c's masked decay, and G of chunk c+1 while they work on chunk c's
-// products and epilogue, so neither is on the chunk's critical path.
+// epilogue only adds D x.  w o X is formed first in each chunk, into the C
+// half of the chunk's B/C slot (spent once G and Ys have read C), so that S
+// runs under the masked decay; Ys of chunk c+1 runs while the warps form y of
+// chunk c, and G of chunk c+1 right behind chunk c's products, so only Y lies
+// between the decay and the epilogue on the chunk's critical path.  (Issuing
+// a group of MMAs holds the issuing lane for most of its run time, which is
+// what fixes this order.)
 // Issuing warp, per chunk c (the whole warp waits, one lane issues):
-//   Pm ready -> G of chunk c+1 into R0 (its B/C tile has landed; the decay has
-//   read G of chunk c); T scaled -> Y_a = Pm_a X_a, Y_b = Pm_b X_b accumulated
-//   into T; w o X ready -> S = B^T [Xw_a | Xw_b], accumulated straight into the
-//   fp32 state H in TMEM; products done -> the B/C slot is refilled and X of
-//   chunk c+1 is loaded into the X slot w o X came from; y staged (and hp of
-//   chunk c+1 written) -> TMA store of y, Ys of chunk c+1 into T, and, once the
-//   store has read its slot, chunk c+1 may write its w o X there.
-// The two X slots alternate: chunk c's X sits in slot c & 1, its w o X goes
-// to slot (c + 1) & 1 (so that scaling X never waits for Y = Pm X to read it)
-// and its y is staged back in slot c & 1.
+//   w o X ready -> S = B^T [Xw_a | Xw_b], accumulated straight into the fp32
+//   state H in TMEM; Pm written and T scaled -> Y_a = Pm_a X_a, Y_b = Pm_b X_b
+//   accumulated into T; G of chunk c+1 into R0 (the decay has read G of chunk
+//   c); products done -> the B/C slot is refilled with chunk c+2; T read and
+//   hp of chunk c+1 written -> Ys of chunk c+1 into T; y staged -> TMA store of
+//   y, and, once the store has read its slot, X of chunk c+2 is loaded there.
+// Chunk c's X sits in X slot c & 1 and its y is staged back in place.
 // Warp 4 (no masked-decay work of its own) also publishes the chunk cumsum of
-// dt*A of both heads for chunk c+1 once every warp has written chunk c's w o X.
+// dt*A of both heads for chunk c+1 once every warp has finished chunk c's mask.
 // Compute warp (TMEM lane quarter q = warp & 3, column slice cs = warp >> 2 of
 // the 128 (head, p) columns; head hd = cs >> 1), per chunk:
+//   w o X of head hd into the C half of the B/C slot (rows split over the
+//         head's 8 warps)
 //   mask: Pm columns 32 cs .. 32 cs + 31, i.e. head hd's 32-token column
 //         blocks 2 (cs & 1) and 2 (cs & 1) + 1 of its 32 rows:
 //         Pm[i][j] = G[i][j] exp(cs_i - cs_j) dt_j (j <= i), 0 above
 //   T *= exp(cs_i) on its rows and columns (T holds Ys)
-//   w o X of head hd into the other X slot (rows split over the head's 8 warps)
-//   y = T + D x in fp32 -> bf16 -> the X slot (same swizzle as the y map), and
-//   with it the state step of chunk c+1: H (h after chunk c) -> bf16 copy hp,
-//         checkpoint, then H = exp(cs_last(c+1)) H, to which S of chunk c+1 is added
+//   the state step of chunk c+1: H (h after chunk c) -> bf16 copy hp,
+//         checkpoint, then H = exp(cs_last(c+1)) H, to which S of chunk c+1 is added;
+//   then y = T + D x in fp32 -> bf16 -> the X slot (same swizzle as the y map)
 // A warp reads and writes only TMEM columns it owns (and G's, which nobody
 // writes while the decay runs), so no barrier among the compute warps is
 // needed; hand-offs go through mbarriers (one arrival per warp).
 // TMEM (512 columns): R0 = 0..127 G (fp32); R1 = 128..255 Pm_a | Pm_b (bf16);
 // T = 256..383 (a | b); H = 384..511 (a | b), the fp32 state, rows n.
-// Shared memory: B/C ring of 2, two X slots (a slot holds a chunk's X, then its
-// y, then the next chunk's w o X), hp, and the per-head scan values (about 227 KB).
+// Shared memory: B/C ring of 2 (a slot holds a chunk's C and B, then its w o X
+// in the C half), two X slots (a chunk's X, then its y), hp, and the per-head
+// scan values (about 227 KB).
 constexpr int kComputeWarps = 16;
 constexpr int kThreadsC = 32 * (kComputeWarps + 1);
 
 struct SmemC {
-    uint8_t bc[2][4 * kBox];   // ring slot: C box 0, C box 1, B box 0, B box 1
-    uint8_t x[2][2 * kBox];    // X slot: head a box, head b box (X, then y, then the next chunk's w o X)
+    uint8_t bc[2][4 * kBox];   // ring slot: C box 0, C box 1, B box 0, B box 1; later w o X in the C half
+    uint8_t x[2][2 * kBox];    // X slot: head a box, head b box (X, then y)
     uint8_t hp[2 * kBox];      // bf16 h_prev of head a, head b (rows n, cols p), 128B-swizzled
     float cvs[2][kQ];          // chunk-inclusive cumsum of dt*A (log2 units), per head
     float dvs[2][kQ];          // dt, per head
     float fs[2][3 * 32];       // dt_j exp(cs_end(J) - cs_j) for the 32-token blocks J = 0..2
-    uint64_t full_bc[2], full_x[2], g_done, ys_done, mma_done, fin, xslot_free; // TMA / MMA / issuer -> warps
-    uint64_t pm_ready, ts_ready, xw_ready, y_ready, st0_ready, scan_ready;     // warps -> issuing warp
+    uint64_t full_bc[2], full_x[2], g_done, ys_done, mma_done, fin;            // TMA / MMA / issuer -> warps
+    uint64_t pm_ready, xw_ready, ys_go, y_ready, st0_ready, scan_ready;        // warps -> issuing warp
     uint32_t tmem;
     int abort;
 };
-
-// two fp32 products in one instruction (sm_100 packed fp32)
-__device__ __forceinline__ float2 mul2(float2 a, float2 b)
-{
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
 
 __global__ void __launch_bounds__(kThreadsC, 1)
 chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
@@ -536,12 +560,11 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
         for (int i = 0; i < 2; ++i) { mbar_init(&s.full_bc[i], 1); mbar_init(&s.full_x[i], 1); }
         mbar_init(&s.g_done, 1);
         mbar_init(&s.ys_done, 1);
-        mbar_init(&s.xslot_free, 1);
         mbar_init(&s.mma_done, 1);
         mbar_init(&s.fin, 1);
         mbar_init(&s.pm_ready, kComputeWarps);
-        mbar_init(&s.ts_ready, kComputeWarps);
         mbar_init(&s.xw_ready, kComputeWarps);
+        mbar_init(&s.ys_go, kComputeWarps);
         mbar_init(&s.y_ready, kComputeWarps);
         mbar_init(&s.st0_ready, kComputeWarps);
         mbar_init(&s.scan_ready, 1);
@@ -708,8 +731,30 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
         for (int c = 0; ok && c < nc; ++c) {
             uint8_t *xs = s.x[c & 1];
 
-            // ---- masked decay: column blocks J = 2 (cs & 1) + jb of head hd, rows of quarter q
-            if (!ewait(&s.g_done, c & 1, abort, lim)) { fail(); break; }
+            // ---- w o X of head hd into the C half of this chunk's B/C slot (free once G and Ys have
+            //      read C), so that S = B^T (w o X) runs under the masked decay: 4 chunks of 16 B per thread
+            if (!(ewait(&s.g_done, c & 1, abort, lim) && ewait(&s.ys_done, c & 1, abort, lim) &&
+                  ewait(&s.full_x[c & 1], (c >> 1) & 1, abort, lim))) { fail(); break; }
+            {
+                const int ti = 32 * (warp & 7) + lane;
+                const int j = ti >> 1, ch = 4 * (ti & 1);
+                const float w = s.dvs[hd][j] * ex2(s.cvs[hd][kQ - 1] - s.cvs[hd][j]);
+                const uint8_t *src = xs + hd * kBox;
+                uint8_t *dst = s.bc[c & 1] + hd * kBox;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    uint4 v = lds128(src + swz(j, ch + u));
+                    v.x = scale_bf16x2_int(v.x, w); v.y = scale_bf16x2_int(v.y, w);
+                    v.z = scale_bf16x2_int(v.z, w); v.w = scale_bf16x2_int(v.w, w);
+                    sts128(dst + swz(j, ch + u), v);
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.xw_ready);
+
+            // ---- masked decay: column blocks J = 2 (cs & 1) + jb of head hd, rows of quarter q; then
+            //      T (= Ys of this chunk) *= exp(cs_r) on this warp's rows and columns
             tc_fence_after();
             {
                 const float csr = s.cvs[hd][r];
@@ -771,14 +816,6 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
                     tmem_st16(tPm + lane_base + 16 * (2 * cs + jb), pk);
                 }
             }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s.pm_ready);
-
-            // ---- T (= Ys of this chunk) *= exp(cs_r) on this warp's rows and columns
-            if (!ewait(&s.ys_done, c & 1, abort, lim)) { fail(); break; }
-            tc_fence_after();
             {
                 const float e_r = ex2(s.cvs[hd][r]);
                 uint32_t tv[32];
@@ -791,32 +828,12 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&s.ts_ready);
+            if (lane == 0) mbar_arrive(&s.pm_ready);   // Pm written and T scaled
 
-            // ---- w o X of head hd into the other X slot (free once the previous y store has read it),
-            //      so that it need not wait for Y = Pm X: 4 chunks of 16 B per thread
-            if (!(ewait(&s.full_x[c & 1], (c >> 1) & 1, abort, lim) &&
-                  ewait(&s.xslot_free, c & 1, abort, lim))) { fail(); break; }
-            {
-                const int ti = 32 * (warp & 7) + lane;
-                const int j = ti >> 1, ch = 4 * (ti & 1);
-                const float w = s.dvs[hd][j] * ex2(s.cvs[hd][kQ - 1] - s.cvs[hd][j]);
-                const uint8_t *src = xs + hd * kBox;
-                uint8_t *dst = s.x[(c + 1) & 1] + hd * kBox;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    uint4 v = lds128(src + swz(j, ch + u));
-                    v.x = scale_bf16x2_int(v.x, w); v.y = scale_bf16x2_int(v.y, w);
-                    v.z = scale_bf16x2_int(v.z, w); v.w = scale_bf16x2_int(v.w, w);
-                    sts128(dst + swz(j, ch + u), v);
-                }
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s.xw_ready);
-            // every warp has read this chunk's scan values once all w o X are written: publish the next chunk's
+            // every warp has read this chunk's scan values once all have written Pm and scaled T:
+            // publish the next chunk's
             if (scan_warp && c + 1 < nc) {
-                if (!ewait(&s.xw_ready, c & 1, abort, lim)) { fail(); break; }
+                if (!ewait(&s.pm_ready, c & 1, abort, lim)) { fail(); break; }
                 scan();
                 if (c + 2 < nc) load_dt(c + 2);
             }
@@ -832,9 +849,16 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
                 tmem_ld16(tT + lane_base + 32 * cs + 16, t1v);
                 tmem_wait_ld(t0v, t1v);
                 tmem_wait_ld(hv);
+                // the state step first: with T read and hp written, Ys of chunk c+1 may start
+                // while y is formed from the registers
+                state_step(c + 1, hv);
+                tmem_wait_st();
+                fence_proxy_async_smem();   // hp, read by Ys of chunk c+1
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s.ys_go);
                 y_half(xs, t0v, 0);
                 y_half(xs, t1v, 1);
-                state_step(c + 1, hv);
             } else {
                 uint32_t t0v[16], t1v[16];
                 tmem_ld16(tT + lane_base + 32 * cs, t0v);
@@ -844,7 +868,7 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
                 y_half(xs, t1v, 1);
             }
             tmem_wait_st();
-            fence_proxy_async_smem();   // y for the store, hp for the next C hp^T
+            fence_proxy_async_smem();   // y, read by the TMA store
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.y_ready);
@@ -890,7 +914,7 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
         const uint64_t dBk0 = smem_desc(bc0 + 2 * kBox, 16, 1024), dBk1 = smem_desc(bc1 + 2 * kBox, 16, 1024);  // B, K-major
         const uint64_t dBt0 = smem_desc(bc0 + 2 * kBox, kBox, 1024), dBt1 = smem_desc(bc1 + 2 * kBox, kBox, 1024);  // B^T, MN-major
         const uint64_t dX0 = smem_desc(x0, 0, 1024), dX1 = smem_desc(x1, 0, 1024);           // X of one head, MN-major, N = 64
-        const uint64_t dXw0 = smem_desc(x0, kBox, 1024), dXw1 = smem_desc(x1, kBox, 1024);    // w o X of both heads, N = 128
+        const uint64_t dXw0 = smem_desc(bc0, kBox, 1024), dXw1 = smem_desc(bc1, kBox, 1024);  // w o X (C half of the B/C slot), N = 128
         const uint64_t dHp = smem_desc(smem_u32(s.hp), kBox, 1024);                          // hp of both heads, N = 128
         constexpr uint64_t kBoxD = kBox >> 4;
         auto koff = [](int kk) -> uint64_t { return (uint64_t)((kk >> 2) * kBoxD + (kk & 3) * 2); };  // K-major K-step
@@ -919,7 +943,7 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
                 issue_bc(0);
                 if (nc > 1) issue_bc(1);
                 issue_x(0);
-                mbar_arrive(&s.xslot_free);   // chunk 0's w o X goes into the untouched slot 1
+                if (nc > 1) issue_x(1);
             }
             ok = ewait(&s.full_bc[0], 0, abort, lim);
             if (ok) {
@@ -938,18 +962,19 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
         for (int c = 0; ok && c < nc; ++c) {
             const int64_t t0 = s0 + (int64_t)c * kQ;
             uint8_t *xs = s.x[c & 1];
-            // the decay has read G: G of chunk c+1 into R0, under this chunk's products
-            ok = ewait(&s.pm_ready, c & 1, abort, lim);
+            // w o X of both heads written (into the C half of this chunk's B/C slot):
+            // S = B^T [Xw_a | Xw_b] accumulates into H while the warps compute the masked decay
+            ok = ewait(&s.xw_ready, c & 1, abort, lim);
             if (!ok) break;
-            if (c + 1 < nc) {
-                ok = ewait(&s.full_bc[(c + 1) & 1], ((c + 1) >> 1) & 1, abort, lim);
-                if (!ok) break;
-                tc_fence_after();
-                if (lane == 0) { ++bc_waited; issue_g(c + 1); }
-                __syncwarp();
+            tc_fence_after();
+            if (lane == 0) {
+                const uint64_t dbt = (c & 1) ? dBt1 : dBt0, dxw = (c & 1) ? dXw1 : dXw0;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) mma_ss(tH, dbt + moff(kk), dxw + moff(kk), id_s, true);
             }
-            // Pm written, T (= Ys) scaled, X landed: Y_a, Y_b accumulate into T
-            ok = ewait(&s.ts_ready, c & 1, abort, lim) && ewait(&s.full_x[c & 1], (c >> 1) & 1, abort, lim);
+            __syncwarp();
+            // Pm written and T (= Ys) scaled, X landed: Y_a, Y_b accumulate into T
+            ok = ewait(&s.pm_ready, c & 1, abort, lim) && ewait(&s.full_x[c & 1], (c >> 1) & 1, abort, lim);
             if (!ok) break;
             tc_fence_after();
             if (lane == 0) {
@@ -960,37 +985,41 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
                         mma_ts(tT + 64 * hd2, tPm + 64 * hd2 + kk * 8, dx + hd2 * kBoxD + moff(kk), id_pm, true);
-            }
-            __syncwarp();
-            // w o X of both heads: S = B^T [Xw_a | Xw_b] accumulates into H
-            ok = ewait(&s.xw_ready, c & 1, abort, lim);
-            if (!ok) break;
-            tc_fence_after();
-            if (lane == 0) {
-                const uint64_t dbt = (c & 1) ? dBt1 : dBt0, dxw = (c & 1) ? dXw0 : dXw1;   // w o X is in slot (c+1) & 1
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) mma_ss(tH, dbt + moff(kk), dxw + moff(kk), id_s, true);
                 mma_commit(&s.mma_done);
             }
             __syncwarp();
-            // products done: refill this B/C slot, and load chunk c+1's X into the slot S read w o X from
+            // G of chunk c+1 into R0 (the decay has read G of chunk c), behind this chunk's products
+            if (c + 1 < nc) {
+                ok = ewait(&s.full_bc[(c + 1) & 1], ((c + 1) >> 1) & 1, abort, lim);
+                if (!ok) break;
+                tc_fence_after();
+                if (lane == 0) { ++bc_waited; issue_g(c + 1); }
+                __syncwarp();
+            }
+            // products done: this B/C slot (C, B, w o X) is spent -- refill it with chunk c+2
             ok = ewait(&s.mma_done, c & 1, abort, lim);
             if (!ok) break;
             if (lane == 0 && c + 2 < nc) issue_bc(c + 2);
-            if (lane == 0 && c + 1 < nc) issue_x(c + 1);
             __syncwarp();
-            // y staged and hp of chunk c+1 written: store y, start Ys of chunk c+1 (T has been read)
+            // T read and hp of chunk c+1 written: Ys of chunk c+1 into T
+            if (c + 1 < nc) {
+                ok = ewait(&s.ys_go, c & 1, abort, lim);
+                if (!ok) break;
+                tc_fence_after();
+                if (lane == 0) issue_ys(c + 1);
+                __syncwarp();
+            }
+            // y staged: store it; once the store has read the slot, X of chunk c+2 is loaded there
             ok = ewait(&s.y_ready, c & 1, abort, lim);
             if (!ok) break;
-            tc_fence_after();
             if (lane == 0) {
                 tma_store_3d(&maps.y, xs, ha * kP, (int)t0, bi);
                 tma_store_3d(&maps.y, xs + kBox, (ha + 1) * kP, (int)t0, bi);
                 tma_store_commit();
-                if (c + 1 < nc) issue_ys(c + 1);
-                // once the store has read the slot, chunk c+1 may write its w o X there
-                tma_store_wait_read<0>();
-                mbar_arrive(&s.xslot_free);
+                if (c + 2 < nc) {
+                    tma_store_wait_read<0>();
+                    issue_x(c + 2);
+                }
             }
             __syncwarp();
         }
