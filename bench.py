@@ -45,7 +45,7 @@ def parse_args():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(ssd_synth.BY_NAME))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-sample-tokens", type=int, default=131072)
+    ap.add_argument("--cpu-sample-tokens", type=int, default=393216)
     # profiling aids: run a shorter stream of the same shape (not a bench line)
     ap.add_argument("--seq-len", type=int, default=None)
     ap.add_argument("--segments", type=int, default=None)

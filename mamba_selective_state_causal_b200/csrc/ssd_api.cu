@@ -406,7 +406,6 @@ int layer_bwd_impl(const ssd_layer_bwd_args *a, cudaStream_t st)
     if (a->b == 0) return ok();
     const int HP = a->H * a->P, GN = a->G * a->N;
     const int C_ch = HP + 2 * GN;
-    const size_t es = elem_size(a->dtype);
     if (!a->dconv_w || !a->dA || (a->L > 0 && (!a->du || !a->ddt)))
         return fail(SSD_ERR_NULL, "du, dconv_w, ddt and dA must not be NULL");
     if (!a->conv_w || !aligned16(a->conv_w) || !aligned16(a->dconv_w))
@@ -432,7 +431,6 @@ int layer_bwd_impl(const ssd_layer_bwd_args *a, cudaStream_t st)
         return ok();
     }
     if ((rc = check_rows("u", a->u, a->u_batch_stride, a->u_row_stride, C_ch, a->b, a->L, a->dtype, true))) return rc;
-    (void)es;
     const LayerBwdPlan pl = make_layer_bwd_plan(a->b, a->L, a->H, a->P, a->N, a->G, a->dtype);
     if (!a->workspace || a->workspace_bytes < pl.bytes)
         return fail(SSD_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", pl.bytes,
@@ -464,6 +462,7 @@ int layer_bwd_impl(const ssd_layer_bwd_args *a, cudaStream_t st)
     ssd_scan_bwd_args sb{};
     sb.dtype = a->dtype; sb.b = a->b; sb.L = a->L; sb.H = a->H; sb.P = a->P; sb.N = a->N; sb.G = a->G;
     sb.s = ck ? a->s : 0;
+    const size_t es = elem_size(a->dtype);
     const char *v = static_cast<const char *>(cp.v);
     sb.x = v; sb.x_batch_stride = a->L * C_ch; sb.x_row_stride = C_ch;
     sb.B = v + es * HP; sb.B_batch_stride = a->L * C_ch; sb.B_row_stride = C_ch;

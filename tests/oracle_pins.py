@@ -517,6 +517,38 @@ def pin_layer_backward_torch_autograd():
             assert _rel(got[k], ref[k]) < 1e-10, (k, (b, L, H, P, N, G), _rel(got[k], ref[k]))
 
 
+def pin_layer_backward_finite_differences():
+    """Every gradient of the layer's reverse mode against central differences of the forward
+    oracle (conv + SiLU, then the recurrence): Richardson-extrapolated for the inputs the loss
+    is nonlinear in (u, the conv buffer, w, bias, dt, A), fixed steps for D and h0."""
+    rng = RNG(43)
+    b, L, H, P, N, G = 1, 9, 2, 2, 2, 1
+    u, w, bias, tail, dt, A, D, h0, dy, dhf, dto = _layer_grad_inputs(rng, b, L, H, P, N, G)
+    args = dict(u=u, w=w, bias=bias, tail=tail, dt=dt, A=A, D=D, h0=h0)
+    got = oracle.layer_backward(u, w, dt, A, D, dy, bias=bias, tail_in=tail, h0=h0, dh_final=dhf,
+                                dtail_out=dto, H=H, P=P, N=N, G=G, io_round="none")
+
+    def loss_wrt(name):
+        def f(v):
+            kw = dict(args)
+            kw[name] = v
+            out = oracle.layer(kw["u"], kw["w"], kw["dt"], kw["A"], kw["D"], kw["bias"], kw["tail"], kw["h0"],
+                               H=H, P=P, N=N, G=G, s=0, io_round="none", want_ckpt=False)
+            return float(np.sum(out["y"] * dy) + np.sum(out["h_final"] * dhf) + np.sum(out["tail_out"] * dto))
+        return f
+
+    # the conv's inputs reach the loss through v, which the forward stores in float32: larger
+    # steps keep that rounding out of the differences
+    for name, key, step, tol in [("u", "du", 5e-2, 1e-4), ("tail", "dtail_in", 5e-2, 1e-4),
+                                 ("w", "dw", 5e-2, 1e-4), ("bias", "dbias", 5e-2, 1e-4),
+                                 ("dt", "ddt", 1e-2, 1e-6), ("A", "dA", 1e-2, 1e-6)]:
+        fd = _fd_grad(loss_wrt(name), args[name], rel_step=step)
+        assert _rel(got[key], fd) < tol, (name, _rel(got[key], fd))
+    for name, key in [("D", "dD"), ("h0", "dh0")]:
+        fd = _fd_grad(loss_wrt(name), args[name])
+        assert _rel(got[key], fd) < 1e-6, (name, _rel(got[key], fd))
+
+
 def _conv_ckpt_from_u(u, s):
     """The 3 rows of u before every checkpoint boundary: [b, L//s, 3, Cch]."""
     b, L, cch = u.shape
@@ -564,5 +596,6 @@ PINS = [pin_quadratic_form, pin_A_zero_prefix_sum, pin_constant_geometric, pin_s
         pin_bf16_rounding, pin_ckpt_indexing, pin_split_resume_bitwise,
         pin_resume_needs_conv_tail, pin_backward_finite_differences, pin_backward_cells_equal_full,
         pin_backward_without_input, pin_gated_norm_torch, pin_gated_norm_invariants,
-        pin_layer_backward_torch_autograd, pin_layer_backward_cells_equal_full,
+        pin_layer_backward_torch_autograd, pin_layer_backward_finite_differences,
+        pin_layer_backward_cells_equal_full,
         pin_layer_backward_needs_conv_buffer]
