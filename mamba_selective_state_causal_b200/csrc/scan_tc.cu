@@ -11,10 +11,10 @@
 // Per chunk of 128 tokens of one head (cs = chunk-local cumulative dt*A, kept
 // in log2 units so that exp(x) = ex2(x * log2 e)):
 //   G  = C B^T                                     tcgen05, 128x128x128, TMEM
-//   Pm = G o [exp(cs_i - cs_j) dt_j, j <= i] + D I CUDA cores, TMEM -> TMEM (bf16)
+//   Pm = G o [exp(cs_i - cs_j) dt_j, j <= i]       CUDA cores, TMEM -> TMEM (bf16)
 //   Yd = Pm X                                      tcgen05, A from TMEM, 128x64x128
 //   Yo = C h_prev^T                                tcgen05, 128x128x128 (both heads)
-//   y  = Yd + exp(cs_i) Yo                         CUDA cores -> smem -> TMA store
+//   y  = Yd + exp(cs_i) Yo + D x                   CUDA cores (fp32) -> smem -> TMA store
 //   S  = B^T (w o X),  w_j = dt_j exp(cs_last - cs_j)   tcgen05, 128x128x128 (both heads)
 //   h  = exp(cs_last) h + S                        fp32 state in TMEM, S accumulated into it
 // Only non-positive differences of cs are exponentiated.  The state is kept in
@@ -474,38 +474,41 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
 }
 
 // =============================================================== pass C
-// One CTA per (stripe, head pair), one CTA per SM: 16 compute warps and one
-// issuing warp.  The two heads share their B and C tiles and G = C B^T; the
+// One CTA per (stripe, head pair), one CTA per SM: 16 compute warps, one
+// issuing warp and one store warp.  The two heads share their B and C tiles and G = C B^T; the
 // chunks of the stripe are walked in order.
 //
 // The output accumulator T of a chunk first receives Ys = C [hp_a | hp_b]^T
 // (the contribution of the state entering the chunk), which the compute warps
 // scale row by row by exp(cs_i); Y = Pm X then accumulates onto it, so the
-// epilogue only adds D x.  w o X is formed first in each chunk, into the C
-// half of the chunk's B/C slot (spent once G and Ys have read C), so that S
-// runs under the masked decay; Ys of chunk c+1 runs while the warps form y of
-// chunk c, and G of chunk c+1 right behind chunk c's products, so only Y lies
-// between the decay and the epilogue on the chunk's critical path.  (Issuing
-// a group of MMAs holds the issuing lane for most of its run time, which is
-// what fixes this order.)
+// epilogue only adds D x.  Per chunk the warps first form the masked decay
+// (G was computed during the previous chunk, and it does not need Ys), then
+// scale T, so that Y = Pm X starts as early as possible; w o X follows, into
+// the C half of the chunk's B/C slot (spent once G and Ys have read C), while
+// Y runs, and S = B^T (w o X) right behind Y.  Ys of chunk c+1 runs while the
+// warps form y of chunk c and start the next decay.  (Issuing a group of MMAs
+// holds the issuing lane for most of its run time, which is what fixes this
+// order.)
 // Issuing warp, per chunk c (the whole warp waits, one lane issues):
-//   w o X ready -> S = B^T [Xw_a | Xw_b], accumulated straight into the fp32
-//   state H in TMEM; Pm written and T scaled -> Y_a = Pm_a X_a, Y_b = Pm_b X_b
-//   accumulated into T; G of chunk c+1 into R0 (the decay has read G of chunk
+//   Pm written and T scaled -> Y_a = Pm_a X_a, Y_b = Pm_b X_b accumulated into
+//   T; w o X ready -> S = B^T [Xw_a | Xw_b], accumulated straight into the fp32
+//   state H in TMEM; G of chunk c+1 into R0 (the decay has read G of chunk
 //   c); products done -> the B/C slot is refilled with chunk c+2; T read and
-//   hp of chunk c+1 written -> Ys of chunk c+1 into T; y staged -> TMA store of
-//   y, and, once the store has read its slot, X of chunk c+2 is loaded there.
-// Chunk c's X sits in X slot c & 1 and its y is staged back in place.
+//   hp of chunk c+1 written -> Ys of chunk c+1 into T.
+// Store warp, per chunk c: y staged -> TMA store of y, and, once the store has
+// read its slot, X of chunk c+2 is loaded there.  Chunk c's X sits in X slot
+// c & 1 and its y is staged back in place.
 // Warp 4 (no masked-decay work of its own) also publishes the chunk cumsum of
-// dt*A of both heads for chunk c+1 once every warp has finished chunk c's mask.
+// dt*A of both heads for chunk c+1 once every warp has written chunk c's w o X
+// (the last use of chunk c's values).
 // Compute warp (TMEM lane quarter q = warp & 3, column slice cs = warp >> 2 of
 // the 128 (head, p) columns; head hd = cs >> 1), per chunk:
-//   w o X of head hd into the C half of the B/C slot (rows split over the
-//         head's 8 warps)
 //   mask: Pm columns 32 cs .. 32 cs + 31, i.e. head hd's 32-token column
 //         blocks 2 (cs & 1) and 2 (cs & 1) + 1 of its 32 rows:
 //         Pm[i][j] = G[i][j] exp(cs_i - cs_j) dt_j (j <= i), 0 above
 //   T *= exp(cs_i) on its rows and columns (T holds Ys)
+//   w o X of head hd into the C half of the B/C slot (rows split over the
+//         head's 8 warps)
 //   the state step of chunk c+1: H (h after chunk c) -> bf16 copy hp,
 //         checkpoint, then H = exp(cs_last(c+1)) H, to which S of chunk c+1 is added;
 //   then y = T + D x in fp32 -> bf16 -> the X slot (same swizzle as the y map)
@@ -518,7 +521,7 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
 // in the C half), two X slots (a chunk's X, then its y), hp, and the per-head
 // scan values (about 227 KB).
 constexpr int kComputeWarps = 16;
-constexpr int kThreadsC = 32 * (kComputeWarps + 1);
+constexpr int kThreadsC = 32 * (kComputeWarps + 3);
 
 struct SmemC {
     uint8_t bc[2][4 * kBox];   // ring slot: C box 0, C box 1, B box 0, B box 1; later w o X in the C half
@@ -527,8 +530,11 @@ struct SmemC {
     float cvs[2][kQ];          // chunk-inclusive cumsum of dt*A (log2 units), per head
     float dvs[2][kQ];          // dt, per head
     float fs[2][3 * 32];       // dt_j exp(cs_end(J) - cs_j) for the 32-token blocks J = 0..2
-    uint64_t full_bc[2], full_x[2], g_done, ys_done, mma_done, fin;            // TMA / MMA / issuer -> warps
-    uint64_t pm_ready, xw_ready, ys_go, y_ready, st0_ready, scan_ready;        // warps -> issuing warp
+    uint64_t full_bc[2], full_x[2], g_done, ys_done, ymma_done, mma_done[2];   // TMA / MMA / issuer -> warps
+    uint64_t fin, fin2;                                                        // end of each issuing warp's MMAs
+    uint64_t pmw, pm_ready, xw_ready, ys_go, st0_ready, scan_ready;            // warps -> issuing warp
+    uint64_t y_ready[2];       // warps -> store warp, by X slot (the store warp may still be storing the
+                               // previous chunk's y when this one's is staged)
     uint32_t tmem;
     int abort;
 };
@@ -560,12 +566,17 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
         for (int i = 0; i < 2; ++i) { mbar_init(&s.full_bc[i], 1); mbar_init(&s.full_x[i], 1); }
         mbar_init(&s.g_done, 1);
         mbar_init(&s.ys_done, 1);
-        mbar_init(&s.mma_done, 1);
+        mbar_init(&s.ymma_done, 1);
+        mbar_init(&s.mma_done[0], 1);
+        mbar_init(&s.mma_done[1], 1);
         mbar_init(&s.fin, 1);
+        mbar_init(&s.fin2, 1);
+        mbar_init(&s.pmw, kComputeWarps);
         mbar_init(&s.pm_ready, kComputeWarps);
         mbar_init(&s.xw_ready, kComputeWarps);
         mbar_init(&s.ys_go, kComputeWarps);
-        mbar_init(&s.y_ready, kComputeWarps);
+        mbar_init(&s.y_ready[0], kComputeWarps);
+        mbar_init(&s.y_ready[1], kComputeWarps);
         mbar_init(&s.st0_ready, kComputeWarps);
         mbar_init(&s.scan_ready, 1);
         s.abort = 0;
@@ -714,6 +725,70 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
             }
         };
 
+        // masked decay of the chunk whose scan values are published: column blocks
+        // J = 2 (cs & 1) + jb of head hd, rows of quarter q (G of that chunk is in TMEM, and
+        // Y of the chunk before it has read Pm)
+        auto decay = [&]() {
+            const float csr = s.cvs[hd][r];
+#pragma unroll
+            for (int jb = 0; jb < 2; ++jb) {
+                const int J = 2 * (cs & 1) + jb;
+                uint32_t pk[16];
+                if (J < q) {
+                    // whole block below the diagonal: exp(cs_r - cs_j) = exp(cs_r - m_J) exp(m_J - cs_j)
+                    const float E = ex2(csr - s.cvs[hd][32 * J + 31]);
+                    const float2 E2 = make_float2(E, E);
+                    uint32_t gv[32];
+                    tmem_ld32(tG + lane_base + 32 * J, gv);
+                    tmem_wait_ld(gv);
+                    const float4 *f4 = reinterpret_cast<const float4 *>(&s.fs[hd][32 * J]);
+#pragma unroll
+                    for (int i4 = 0; i4 < 8; ++i4) {
+                        const float4 f = f4[i4];
+                        const float2 a = mul2(make_float2(__uint_as_float(gv[4 * i4]), __uint_as_float(gv[4 * i4 + 1])),
+                                              mul2(make_float2(f.x, f.y), E2));
+                        const float2 b = mul2(make_float2(__uint_as_float(gv[4 * i4 + 2]), __uint_as_float(gv[4 * i4 + 3])),
+                                              mul2(make_float2(f.z, f.w), E2));
+                        pk[2 * i4] = pack_bf16x2(a.x, a.y);
+                        pk[2 * i4 + 1] = pack_bf16x2(b.x, b.y);
+                    }
+                } else if (J == q) {
+                    // diagonal block as 16x16 quarters: the two on the diagonal exponentiate each
+                    // entry; the one below factors through m = cs at the block's column 15
+                    uint32_t gv[32];
+                    tmem_ld32(tG + lane_base + 32 * J, gv);
+                    tmem_wait_ld(gv);
+                    const float *cvb = &s.cvs[hd][32 * J], *dvb = &s.dvs[hd][32 * J];
+                    const float m16 = cvb[15];
+                    const bool lo = lane < 16;
+                    const float a_r = ex2(csr - m16);                                   // <= 1 for lane >= 16
+                    const float b_own = dvb[lane & 15] * ex2(m16 - cvb[lane & 15]);     // <= dt for lane < 16
+                    const int xo = lo ? 0 : 16;
+#pragma unroll
+                    for (int k2 = 0; k2 < 8; ++k2) {
+                        float vl[2], vh[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int k = 2 * k2 + e;
+                            const int x = xo + k;
+                            const float g_x = __uint_as_float(lo ? gv[k] : gv[16 + k]);
+                            float t = g_x * ex2(csr - cvb[x]) * dvb[x];
+                            t = x > lane ? 0.0f : t;
+                            const float bk = __shfl_sync(0xffffffffu, b_own, k);
+                            vl[e] = lo ? t : __uint_as_float(gv[k]) * (a_r * bk);
+                            vh[e] = lo ? 0.0f : t;
+                        }
+                        pk[k2] = pack_bf16x2(vl[0], vl[1]);
+                        pk[8 + k2] = pack_bf16x2(vh[0], vh[1]);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) pk[i] = 0u;
+                }
+                tmem_st16(tPm + lane_base + 16 * (2 * cs + jb), pk);
+            }
+        };
+
         bool ok = ewait(&s.scan_ready, 0, abort, lim);
         if (ok) {
             uint32_t hv[32];
@@ -725,16 +800,41 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.st0_ready);
-        } else {
-            fail();
+            // the masked decay of chunk 0
+            ok = ewait(&s.g_done, 0, abort, lim);
+            if (ok) {
+                tc_fence_after();
+                decay();
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s.pmw);
+            }
         }
+        if (!ok) fail();
         for (int c = 0; ok && c < nc; ++c) {
             uint8_t *xs = s.x[c & 1];
 
-            // ---- w o X of head hd into the C half of this chunk's B/C slot (free once G and Ys have
-            //      read C), so that S = B^T (w o X) runs under the masked decay: 4 chunks of 16 B per thread
-            if (!(ewait(&s.g_done, c & 1, abort, lim) && ewait(&s.ys_done, c & 1, abort, lim) &&
-                  ewait(&s.full_x[c & 1], (c >> 1) & 1, abort, lim))) { fail(); break; }
+            // ---- T (= Ys of this chunk) *= exp(cs_r) on this warp's rows and columns
+            if (!ewait(&s.ys_done, c & 1, abort, lim)) { fail(); break; }
+            tc_fence_after();
+            {
+                const float e_r = ex2(s.cvs[hd][r]);
+                uint32_t tv[32];
+                tmem_ld32(tT + lane_base + 32 * cs, tv);
+                tmem_wait_ld(tv);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) tv[i] = __float_as_uint(e_r * __uint_as_float(tv[i]));
+                tmem_st32(tT + lane_base + 32 * cs, tv);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.pm_ready);   // Pm written and T scaled
+
+            // ---- w o X of head hd into the C half of this chunk's B/C slot (free: G and Ys have read
+            //      C), for S = B^T (w o X), which runs after Y = Pm X: 4 chunks of 16 B per thread
+            if (!ewait(&s.full_x[c & 1], (c >> 1) & 1, abort, lim)) { fail(); break; }
             {
                 const int ti = 32 * (warp & 7) + lane;
                 const int j = ti >> 1, ch = 4 * (ti & 1);
@@ -753,96 +853,31 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.xw_ready);
 
-            // ---- masked decay: column blocks J = 2 (cs & 1) + jb of head hd, rows of quarter q; then
-            //      T (= Ys of this chunk) *= exp(cs_r) on this warp's rows and columns
-            tc_fence_after();
-            {
-                const float csr = s.cvs[hd][r];
-#pragma unroll
-                for (int jb = 0; jb < 2; ++jb) {
-                    const int J = 2 * (cs & 1) + jb;
-                    uint32_t pk[16];
-                    if (J < q) {
-                        // whole block below the diagonal: exp(cs_r - cs_j) = exp(cs_r - m_J) exp(m_J - cs_j)
-                        const float E = ex2(csr - s.cvs[hd][32 * J + 31]);
-                        const float2 E2 = make_float2(E, E);
-                        uint32_t gv[32];
-                        tmem_ld32(tG + lane_base + 32 * J, gv);
-                        tmem_wait_ld(gv);
-                        const float4 *f4 = reinterpret_cast<const float4 *>(&s.fs[hd][32 * J]);
-#pragma unroll
-                        for (int i4 = 0; i4 < 8; ++i4) {
-                            const float4 f = f4[i4];
-                            const float2 a = mul2(make_float2(__uint_as_float(gv[4 * i4]), __uint_as_float(gv[4 * i4 + 1])),
-                                                  mul2(make_float2(f.x, f.y), E2));
-                            const float2 b = mul2(make_float2(__uint_as_float(gv[4 * i4 + 2]), __uint_as_float(gv[4 * i4 + 3])),
-                                                  mul2(make_float2(f.z, f.w), E2));
-                            pk[2 * i4] = pack_bf16x2(a.x, a.y);
-                            pk[2 * i4 + 1] = pack_bf16x2(b.x, b.y);
-                        }
-                    } else if (J == q) {
-                        // diagonal block as 16x16 quarters: the two on the diagonal exponentiate each
-                        // entry; the one below factors through m = cs at the block's column 15
-                        uint32_t gv[32];
-                        tmem_ld32(tG + lane_base + 32 * J, gv);
-                        tmem_wait_ld(gv);
-                        const float *cvb = &s.cvs[hd][32 * J], *dvb = &s.dvs[hd][32 * J];
-                        const float m16 = cvb[15];
-                        const bool lo = lane < 16;
-                        const float a_r = ex2(csr - m16);                                   // <= 1 for lane >= 16
-                        const float b_own = dvb[lane & 15] * ex2(m16 - cvb[lane & 15]);     // <= dt for lane < 16
-                        const int xo = lo ? 0 : 16;
-#pragma unroll
-                        for (int k2 = 0; k2 < 8; ++k2) {
-                            float vl[2], vh[2];
-#pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                const int k = 2 * k2 + e;
-                                const int x = xo + k;
-                                const float g_x = __uint_as_float(lo ? gv[k] : gv[16 + k]);
-                                float t = g_x * ex2(csr - cvb[x]) * dvb[x];
-                                t = x > lane ? 0.0f : t;
-                                const float bk = __shfl_sync(0xffffffffu, b_own, k);
-                                vl[e] = lo ? t : __uint_as_float(gv[k]) * (a_r * bk);
-                                vh[e] = lo ? 0.0f : t;
-                            }
-                            pk[k2] = pack_bf16x2(vl[0], vl[1]);
-                            pk[8 + k2] = pack_bf16x2(vh[0], vh[1]);
-                        }
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) pk[i] = 0u;
-                    }
-                    tmem_st16(tPm + lane_base + 16 * (2 * cs + jb), pk);
-                }
-            }
-            {
-                const float e_r = ex2(s.cvs[hd][r]);
-                uint32_t tv[32];
-                tmem_ld32(tT + lane_base + 32 * cs, tv);
-                tmem_wait_ld(tv);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) tv[i] = __float_as_uint(e_r * __uint_as_float(tv[i]));
-                tmem_st32(tT + lane_base + 32 * cs, tv);
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s.pm_ready);   // Pm written and T scaled
-
-            // every warp has read this chunk's scan values once all have written Pm and scaled T:
+            // every warp has read this chunk's scan values once all have written w o X:
             // publish the next chunk's
             if (scan_warp && c + 1 < nc) {
-                if (!ewait(&s.pm_ready, c & 1, abort, lim)) { fail(); break; }
+                if (!ewait(&s.xw_ready, c & 1, abort, lim)) { fail(); break; }
                 scan();
                 if (c + 2 < nc) load_dt(c + 2);
             }
 
+            // ---- the masked decay of chunk c+1 while S of this chunk runs: Y has read Pm, G of
+            //      chunk c+1 is in TMEM, its scan values are published
+            if (c + 1 < nc) {
+                if (!(ewait(&s.ymma_done, c & 1, abort, lim) && ewait(&s.g_done, (c + 1) & 1, abort, lim) &&
+                      ewait(&s.scan_ready, (c + 1) & 1, abort, lim))) { fail(); break; }
+                tc_fence_after();
+                decay();
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s.pmw);
+            }
+
             // ---- once every product of the chunk is done: y of chunk c and the state step of chunk c+1
-            if (!ewait(&s.mma_done, c & 1, abort, lim)) { fail(); break; }
+            if (!ewait(&s.mma_done[c & 1], (c >> 1) & 1, abort, lim)) { fail(); break; }
             tc_fence_after();
             if (c + 1 < nc) {
-                if (!ewait(&s.scan_ready, (c + 1) & 1, abort, lim)) { fail(); break; }
                 uint32_t hv[32], t0v[16], t1v[16];
                 tmem_ld32(tH + lane_base + 32 * cs, hv);
                 tmem_ld16(tT + lane_base + 32 * cs, t0v);
@@ -871,7 +906,7 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
             fence_proxy_async_smem();   // y, read by the TMA store
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&s.y_ready);
+            if (lane == 0) mbar_arrive(&s.y_ready[c & 1]);
         }
         if (!__any_sync(0xffffffffu, *abort != 0)) {
             // the state after the stripe's last chunk
@@ -883,29 +918,6 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
             if (p.h_final && s1 == p.L) store_state(p.h_final + ((int64_t)bi * p.H + hh) * PN + (int64_t)p0 * kN + r, hv);
         }
     } else {
-        // ================================================= issuing warp
-        int bc_issued = 0, bc_waited = 0, x_issued = 0, x_waited = 0;   // lane 0's bookkeeping
-        auto issue_bc = [&](int c) {
-            const int t0 = (int)(s0 + (int64_t)c * kQ);
-            uint8_t *d = s.bc[c & 1];
-            uint64_t *bar = &s.full_bc[c & 1];
-            mbar_arrive_expect_tx(bar, 4 * kBox);
-            tma_load_3d(d, &maps.C, bar, g * kN, t0, bi);
-            tma_load_3d(d + kBox, &maps.C, bar, g * kN + 64, t0, bi);
-            tma_load_3d(d + 2 * kBox, &maps.B, bar, g * kN, t0, bi);
-            tma_load_3d(d + 3 * kBox, &maps.B, bar, g * kN + 64, t0, bi);
-            ++bc_issued;
-        };
-        auto issue_x = [&](int c) {
-            const int t0 = (int)(s0 + (int64_t)c * kQ);
-            uint8_t *d = s.x[c & 1];
-            uint64_t *bar = &s.full_x[c & 1];
-            mbar_arrive_expect_tx(bar, 2 * kBox);
-            tma_load_3d(d, &maps.x, bar, ha * kP, t0, bi);
-            tma_load_3d(d + kBox, &maps.x, bar, (ha + 1) * kP, t0, bi);
-            ++x_issued;
-        };
-        // G = C B^T of chunk c into the TMEM columns at tG (its B/C slot has landed)
         // shared-memory descriptors of every operand tile, built once per slot: a K-step only adds
         // a constant to the start-address field (in 16-byte units; addresses stay below 256 KB)
         const uint32_t bc0 = smem_u32(s.bc[0]), bc1 = smem_u32(s.bc[1]);
@@ -919,6 +931,7 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
         constexpr uint64_t kBoxD = kBox >> 4;
         auto koff = [](int kk) -> uint64_t { return (uint64_t)((kk >> 2) * kBoxD + (kk & 3) * 2); };  // K-major K-step
         auto moff = [](int kk) -> uint64_t { return (uint64_t)(kk * 128); };                          // MN-major K-step
+        // G = C B^T of chunk c into the TMEM columns at tG (its B/C slot has landed)
         auto issue_g = [&](int c) {
             const uint64_t dc = (c & 1) ? dC1 : dC0, db = (c & 1) ? dBk1 : dBk0;
             const uint32_t id_g = idesc_bf16(128, 128, 0, 0);
@@ -926,124 +939,191 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
             for (int kk = 0; kk < 8; ++kk) mma_ss(tG, dc + koff(kk), db + koff(kk), id_g, kk > 0);
             mma_commit(&s.g_done);
         };
-        // Ys = C hp^T of chunk c into T (its B/C slot has landed, hp is written, T is free)
-        auto issue_ys = [&](int c) {
-            const uint64_t dc = (c & 1) ? dC1 : dC0;
-            const uint32_t id_ys = idesc_bf16(128, 128, 0, 1);    // A = C (K-major), B = hp (MN-major)
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) mma_ss(tT, dc + koff(kk), dHp + moff(kk), id_ys, kk > 0);
-            mma_commit(&s.ys_done);
-        };
-        const uint32_t id_pm = idesc_bf16(128, 64, 0, 1);     // A = Pm (TMEM), B = X (MN-major)
-        const uint32_t id_s = idesc_bf16(128, 128, 1, 1);     // A = B^T (MN-major), B = w o X (MN-major)
         // The whole warp waits (warp-uniform outcome); lane 0 issues.
-        bool ok = live;
-        if (ok) {
-            if (lane == 0) {
-                issue_bc(0);
-                if (nc > 1) issue_bc(1);
-                issue_x(0);
-                if (nc > 1) issue_x(1);
-            }
-            ok = ewait(&s.full_bc[0], 0, abort, lim);
+        if (warp == kComputeWarps) {
+            // ============================================= issuing warp: Y, S, Ys (and G of chunk 0)
+            // Ys = C hp^T of chunk c into T (its B/C slot has landed, hp is written, T is free)
+            auto issue_ys = [&](int c) {
+                const uint64_t dc = (c & 1) ? dC1 : dC0;
+                const uint32_t id_ys = idesc_bf16(128, 128, 0, 1);    // A = C (K-major), B = hp (MN-major)
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) mma_ss(tT, dc + koff(kk), dHp + moff(kk), id_ys, kk > 0);
+                mma_commit(&s.ys_done);
+            };
+            const uint32_t id_pm = idesc_bf16(128, 64, 0, 1);     // A = Pm (TMEM), B = X (MN-major)
+            const uint32_t id_s = idesc_bf16(128, 128, 1, 1);     // A = B^T (MN-major), B = w o X (MN-major)
+            bool ok = live;
             if (ok) {
-                tc_fence_after();
-                if (lane == 0) { ++bc_waited; issue_g(0); }
-                __syncwarp();
-                // Ys of chunk 0 once the warps have written hp of the state entering the stripe
-                ok = ewait(&s.st0_ready, 0, abort, lim);
+                // G of chunk 0 once its B/C slot has landed, Ys of chunk 0 once the warps have
+                // written hp of the state entering the stripe
+                ok = ewait(&s.full_bc[0], 0, abort, lim);
                 if (ok) {
                     tc_fence_after();
-                    if (lane == 0) issue_ys(0);
+                    if (lane == 0) issue_g(0);
+                    __syncwarp();
+                    ok = ewait(&s.st0_ready, 0, abort, lim);
+                    if (ok) {
+                        tc_fence_after();
+                        if (lane == 0) issue_ys(0);
+                        __syncwarp();
+                    }
+                }
+            }
+            for (int c = 0; ok && c < nc; ++c) {
+                // Pm written and T (= Ys) scaled, X landed: Y_a, Y_b accumulate into T while the
+                // warps write w o X
+                ok = ewait(&s.pm_ready, c & 1, abort, lim) && ewait(&s.full_x[c & 1], (c >> 1) & 1, abort, lim);
+                if (!ok) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint64_t dx = (c & 1) ? dX1 : dX0;
+#pragma unroll
+                    for (int hd2 = 0; hd2 < 2; ++hd2)
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_ts(tT + 64 * hd2, tPm + 64 * hd2 + kk * 8, dx + hd2 * kBoxD + moff(kk), id_pm, true);
+                    mma_commit(&s.ymma_done);
+                }
+                __syncwarp();
+                // w o X of both heads written (into the C half of this chunk's B/C slot):
+                // S = B^T [Xw_a | Xw_b] accumulates into H
+                ok = ewait(&s.xw_ready, c & 1, abort, lim);
+                if (!ok) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint64_t dbt = (c & 1) ? dBt1 : dBt0, dxw = (c & 1) ? dXw1 : dXw0;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) mma_ss(tH, dbt + moff(kk), dxw + moff(kk), id_s, true);
+                    mma_commit(&s.mma_done[c & 1]);
+                }
+                __syncwarp();
+                // T read and hp of chunk c+1 written: Ys of chunk c+1 into T
+                if (c + 1 < nc) {
+                    ok = ewait(&s.ys_go, c & 1, abort, lim);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (lane == 0) issue_ys(c + 1);
                     __syncwarp();
                 }
             }
-        }
-        for (int c = 0; ok && c < nc; ++c) {
-            const int64_t t0 = s0 + (int64_t)c * kQ;
-            uint8_t *xs = s.x[c & 1];
-            // w o X of both heads written (into the C half of this chunk's B/C slot):
-            // S = B^T [Xw_a | Xw_b] accumulates into H while the warps compute the masked decay
-            ok = ewait(&s.xw_ready, c & 1, abort, lim);
-            if (!ok) break;
-            tc_fence_after();
             if (lane == 0) {
-                const uint64_t dbt = (c & 1) ? dBt1 : dBt0, dxw = (c & 1) ? dXw1 : dXw0;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) mma_ss(tH, dbt + moff(kk), dxw + moff(kk), id_s, true);
+                if (live && !ok) raise_timeout(p, abort);
+                // every MMA of this warp complete before TMEM is freed
+                mma_commit(&s.fin);
+                mbar_wait(&s.fin, 0, nullptr, 100000000ull);
             }
             __syncwarp();
-            // Pm written and T (= Ys) scaled, X landed: Y_a, Y_b accumulate into T
-            ok = ewait(&s.pm_ready, c & 1, abort, lim) && ewait(&s.full_x[c & 1], (c >> 1) & 1, abort, lim);
-            if (!ok) break;
-            tc_fence_after();
-            if (lane == 0) {
-                ++x_waited;
-                const uint64_t dx = (c & 1) ? dX1 : dX0;
-#pragma unroll
-                for (int hd2 = 0; hd2 < 2; ++hd2)
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ts(tT + 64 * hd2, tPm + 64 * hd2 + kk * 8, dx + hd2 * kBoxD + moff(kk), id_pm, true);
-                mma_commit(&s.mma_done);
+        } else if (warp == kComputeWarps + 1) {
+            // ============================================= store warp: y out, X in
+            // (kept off the issuing warp, whose lane would otherwise sit in the wait for the
+            // store to read its slot while the next products could be issued)
+            int x_issued = 0;   // lane 0's bookkeeping
+            auto issue_x = [&](int c) {
+                const int t0 = (int)(s0 + (int64_t)c * kQ);
+                uint8_t *d = s.x[c & 1];
+                uint64_t *bar = &s.full_x[c & 1];
+                mbar_arrive_expect_tx(bar, 2 * kBox);
+                tma_load_3d(d, &maps.x, bar, ha * kP, t0, bi);
+                tma_load_3d(d + kBox, &maps.x, bar, (ha + 1) * kP, t0, bi);
+                ++x_issued;
+            };
+            bool ok = live;
+            if (ok && lane == 0) {
+                issue_x(0);
+                if (nc > 1) issue_x(1);
             }
-            __syncwarp();
-            // G of chunk c+1 into R0 (the decay has read G of chunk c), behind this chunk's products
-            if (c + 1 < nc) {
-                ok = ewait(&s.full_bc[(c + 1) & 1], ((c + 1) >> 1) & 1, abort, lim);
+            for (int c = 0; ok && c < nc; ++c) {
+                const int64_t t0 = s0 + (int64_t)c * kQ;
+                uint8_t *xs = s.x[c & 1];
+                // y staged: store it; once the store has read the slot, X of chunk c+2 is loaded there
+                ok = ewait(&s.y_ready[c & 1], (c >> 1) & 1, abort, lim);
                 if (!ok) break;
-                tc_fence_after();
-                if (lane == 0) { ++bc_waited; issue_g(c + 1); }
+                if (lane == 0) {
+                    tma_store_3d(&maps.y, xs, ha * kP, (int)t0, bi);
+                    tma_store_3d(&maps.y, xs + kBox, (ha + 1) * kP, (int)t0, bi);
+                    tma_store_commit();
+                    if (c + 2 < nc) {
+                        tma_store_wait_read<0>();
+                        issue_x(c + 2);
+                    }
+                }
                 __syncwarp();
             }
-            // products done: this B/C slot (C, B, w o X) is spent -- refill it with chunk c+2
-            ok = ewait(&s.mma_done, c & 1, abort, lim);
-            if (!ok) break;
-            if (lane == 0 && c + 2 < nc) issue_bc(c + 2);
+            if (lane == 0) {
+                if (live && !ok) raise_timeout(p, abort);
+                if (*abort) {
+                    // the last load issued into each X slot lands before the CTA's shared memory is
+                    // released (an earlier load into the same slot has been waited on by the compute warps)
+                    for (int i = x_issued > 2 ? x_issued - 2 : 0; i < x_issued; ++i)
+                        mbar_wait(&s.full_x[i & 1], (i >> 1) & 1, nullptr, 100000000ull);
+                }
+                tma_store_wait<0>();
+            }
             __syncwarp();
-            // T read and hp of chunk c+1 written: Ys of chunk c+1 into T
-            if (c + 1 < nc) {
-                ok = ewait(&s.ys_go, c & 1, abort, lim);
+        } else {
+            // ============================================= B/C warp: B and C in, G of chunks 1..
+            // (G of chunk c+2 waits for its slot to land, which must not hold up Y and S)
+            int bc_issued = 0;   // lane 0's bookkeeping
+            auto issue_bc = [&](int c) {
+                const int t0 = (int)(s0 + (int64_t)c * kQ);
+                uint8_t *d = s.bc[c & 1];
+                uint64_t *bar = &s.full_bc[c & 1];
+                mbar_arrive_expect_tx(bar, 4 * kBox);
+                tma_load_3d(d, &maps.C, bar, g * kN, t0, bi);
+                tma_load_3d(d + kBox, &maps.C, bar, g * kN + 64, t0, bi);
+                tma_load_3d(d + 2 * kBox, &maps.B, bar, g * kN, t0, bi);
+                tma_load_3d(d + 3 * kBox, &maps.B, bar, g * kN + 64, t0, bi);
+                ++bc_issued;
+            };
+            bool ok = live;
+            if (ok) {
+                if (lane == 0) {
+                    issue_bc(0);
+                    if (nc > 1) issue_bc(1);
+                }
+                // G of chunk 1 once the warps have read G of chunk 0
+                if (nc > 1) {
+                    ok = ewait(&s.pmw, 0, abort, lim) && ewait(&s.full_bc[1], 0, abort, lim);
+                    if (ok) {
+                        tc_fence_after();
+                        if (lane == 0) issue_g(1);
+                        __syncwarp();
+                    }
+                }
+            }
+            for (int c = 0; ok && c + 2 < nc; ++c) {
+                // S of chunk c done: its B/C slot (C, B, w o X) is spent -- refill it with chunk c+2
+                ok = ewait(&s.mma_done[c & 1], (c >> 1) & 1, abort, lim);
+                if (!ok) break;
+                if (lane == 0) issue_bc(c + 2);
+                __syncwarp();
+                // G of chunk c+2 into R0 once the warps have read G of chunk c+1 and the slot has landed
+                ok = ewait(&s.pmw, (c + 1) & 1, abort, lim) &&
+                     ewait(&s.full_bc[c & 1], ((c + 2) >> 1) & 1, abort, lim);
                 if (!ok) break;
                 tc_fence_after();
-                if (lane == 0) issue_ys(c + 1);
+                if (lane == 0) issue_g(c + 2);
                 __syncwarp();
             }
-            // y staged: store it; once the store has read the slot, X of chunk c+2 is loaded there
-            ok = ewait(&s.y_ready, c & 1, abort, lim);
-            if (!ok) break;
             if (lane == 0) {
-                tma_store_3d(&maps.y, xs, ha * kP, (int)t0, bi);
-                tma_store_3d(&maps.y, xs + kBox, (ha + 1) * kP, (int)t0, bi);
-                tma_store_commit();
-                if (c + 2 < nc) {
-                    tma_store_wait_read<0>();
-                    issue_x(c + 2);
+                if (live && !ok) raise_timeout(p, abort);
+                // every MMA of this warp complete before TMEM is freed
+                mma_commit(&s.fin2);
+                mbar_wait(&s.fin2, 0, nullptr, 100000000ull);
+                if (*abort) {
+                    // the last load issued into each B/C slot lands before the CTA's shared memory
+                    // is released (an earlier load into the same slot has been waited on for its G)
+                    for (int i = bc_issued > 2 ? bc_issued - 2 : 0; i < bc_issued; ++i)
+                        mbar_wait(&s.full_bc[i & 1], (i >> 1) & 1, nullptr, 100000000ull);
                 }
             }
             __syncwarp();
         }
-        if (lane == 0) {
-            if (live && !ok) raise_timeout(p, abort);
-            // every MMA complete before TMEM is freed (after an abort: drain the loads too)
-            mma_commit(&s.fin);
-            mbar_wait(&s.fin, 0, nullptr, 100000000ull);
-            if (*abort) {
-                for (int i = bc_waited; i < bc_issued; ++i)
-                    mbar_wait(&s.full_bc[i & 1], (i >> 1) & 1, nullptr, 100000000ull);
-                for (int i = x_waited; i < x_issued; ++i)
-                    mbar_wait(&s.full_x[i & 1], (i >> 1) & 1, nullptr, 100000000ull);
-            }
-            tma_store_wait<0>();
-        }
-        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tm, 512);
 }
-
-// =============================================================== host side
 
 // =============================================================== host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
