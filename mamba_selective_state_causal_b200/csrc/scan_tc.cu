@@ -89,28 +89,11 @@ __device__ __forceinline__ uint32_t scale_bf16x2_int(uint32_t v, float w)
     return pack_bf16x2_int(bf16_lo(v) * w, bf16_hi(v) * w);
 }
 
-// two fp32 products / fused multiply-adds in one instruction (sm_100 packed fp32); each lane
-// rounds exactly as the scalar instruction does
-__device__ __forceinline__ float2 mul2(float2 a, float2 b)
-{
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c)
-{
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return d;
-}
+// two fp32 products / fused multiply-adds in one instruction (sm_100 packed fp32, through the
+// CUDA float2 intrinsics, which leave the register pairing to the compiler); each lane rounds
+// exactly as the scalar instruction does
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
 __device__ __forceinline__ float2 unpack2(uint32_t v) { return make_float2(bf16_lo(v), bf16_hi(v)); }
 
@@ -474,41 +457,44 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
 }
 
 // =============================================================== pass C
-// One CTA per (stripe, head pair), one CTA per SM: 16 compute warps, one
-// issuing warp and one store warp.  The two heads share their B and C tiles and G = C B^T; the
-// chunks of the stripe are walked in order.
+// One CTA per (stripe, head pair), one CTA per SM: 16 compute warps, an issuing
+// warp, a store warp and a B/C warp.  The two heads share their B and C tiles
+// and G = C B^T; the chunks of the stripe are walked in order.
 //
 // The output accumulator T of a chunk first receives Ys = C [hp_a | hp_b]^T
 // (the contribution of the state entering the chunk), which the compute warps
 // scale row by row by exp(cs_i); Y = Pm X then accumulates onto it, so the
-// epilogue only adds D x.  Per chunk the warps first form the masked decay
-// (G was computed during the previous chunk, and it does not need Ys), then
-// scale T, so that Y = Pm X starts as early as possible; w o X follows, into
-// the C half of the chunk's B/C slot (spent once G and Ys have read C), while
-// Y runs, and S = B^T (w o X) right behind Y.  Ys of chunk c+1 runs while the
-// warps form y of chunk c and start the next decay.  (Issuing a group of MMAs
-// holds the issuing lane for most of its run time, which is what fixes this
-// order.)
+// epilogue only adds D x.  The masked decay Pm of a chunk is formed during the
+// previous chunk, under its S, so per chunk the compute warps scale T (Y may
+// start at once), write w o X into the C half of the chunk's B/C slot (spent
+// once G and Ys have read C) while Y runs, form the next chunk's decay once Y
+// has read Pm while S = B^T (w o X) runs, and then take the state step and y.
+// Ys of chunk c+1 runs while the warps form y of chunk c.  (Issuing a group of
+// MMAs holds the issuing lane for most of its run time, and a load can take a
+// microsecond to land: loads, stores and G, whose operands arrive by TMA, are
+// kept off the warp that issues Y, S and Ys.)
 // Issuing warp, per chunk c (the whole warp waits, one lane issues):
 //   Pm written and T scaled -> Y_a = Pm_a X_a, Y_b = Pm_b X_b accumulated into
 //   T; w o X ready -> S = B^T [Xw_a | Xw_b], accumulated straight into the fp32
-//   state H in TMEM; G of chunk c+1 into R0 (the decay has read G of chunk
-//   c); products done -> the B/C slot is refilled with chunk c+2; T read and
-//   hp of chunk c+1 written -> Ys of chunk c+1 into T.
+//   state H in TMEM; T read and hp of chunk c+1 written -> Ys of chunk c+1
+//   into T.  (G and Ys of chunk 0 in the prologue.)
+// B/C warp, per chunk c: products done -> the B/C slot is refilled with chunk
+// c+2; the decay of chunk c+1 has read G, the slot has landed and Ys of chunk
+// c+1 is done -> G of chunk c+2 into R0.
 // Store warp, per chunk c: y staged -> TMA store of y, and, once the store has
 // read its slot, X of chunk c+2 is loaded there.  Chunk c's X sits in X slot
 // c & 1 and its y is staged back in place.
 // Warp 4 (no masked-decay work of its own) also publishes the chunk cumsum of
 // dt*A of both heads for chunk c+1 once every warp has written chunk c's w o X
-// (the last use of chunk c's values).
+// (the last use of chunk c's values before the next decay).
 // Compute warp (TMEM lane quarter q = warp & 3, column slice cs = warp >> 2 of
-// the 128 (head, p) columns; head hd = cs >> 1), per chunk:
-//   mask: Pm columns 32 cs .. 32 cs + 31, i.e. head hd's 32-token column
-//         blocks 2 (cs & 1) and 2 (cs & 1) + 1 of its 32 rows:
-//         Pm[i][j] = G[i][j] exp(cs_i - cs_j) dt_j (j <= i), 0 above
+// the 128 (head, p) columns; head hd = cs >> 1), per chunk c:
 //   T *= exp(cs_i) on its rows and columns (T holds Ys)
 //   w o X of head hd into the C half of the B/C slot (rows split over the
 //         head's 8 warps)
+//   mask of chunk c+1: Pm columns 32 cs .. 32 cs + 31, i.e. head hd's 32-token
+//         column blocks 2 (cs & 1) and 2 (cs & 1) + 1 of its 32 rows:
+//         Pm[i][j] = G[i][j] exp(cs_i - cs_j) dt_j (j <= i), 0 above
 //   the state step of chunk c+1: H (h after chunk c) -> bf16 copy hp,
 //         checkpoint, then H = exp(cs_last(c+1)) H, to which S of chunk c+1 is added;
 //   then y = T + D x in fp32 -> bf16 -> the X slot (same swizzle as the y map)
@@ -1097,9 +1083,12 @@ chunk_output_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
                 if (!ok) break;
                 if (lane == 0) issue_bc(c + 2);
                 __syncwarp();
-                // G of chunk c+2 into R0 once the warps have read G of chunk c+1 and the slot has landed
+                // G of chunk c+2 into R0 once the warps have read G of chunk c+1, the slot has landed
+                // and Ys of chunk c+1 is done (G must not sit in front of Ys in the tensor pipe: Ys
+                // is on the chunk's critical path, G of chunk c+2 is not needed for a while)
                 ok = ewait(&s.pmw, (c + 1) & 1, abort, lim) &&
-                     ewait(&s.full_bc[c & 1], ((c + 2) >> 1) & 1, abort, lim);
+                     ewait(&s.full_bc[c & 1], ((c + 2) >> 1) & 1, abort, lim) &&
+                     ewait(&s.ys_done, (c + 1) & 1, abort, lim);
                 if (!ok) break;
                 tc_fence_after();
                 if (lane == 0) issue_g(c + 2);
