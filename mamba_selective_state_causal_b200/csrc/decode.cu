@@ -11,8 +11,9 @@
 // The state is the traffic: 2 * P * N * 4 bytes per (stream, head), read and
 // written once.  One CTA per (stream, head): it recomputes the conv of the
 // channels it reads (its head's x, its group's B and C) from tail_in, then
-// streams its state with float4 loads (lane = 4 state columns, warp = P/8 rows)
-// and reduces y over n with shuffles.  The tail shift runs as a second kernel
+// streams its state with float4 loads (lane = 4 state columns, warp = P/8 rows;
+// streaming cache hints, since each state element is touched once per step) and
+// reduces y over n with shuffles.  The tail shift runs as a second kernel
 // after it, so that tail_out may alias tail_in.
 #include <algorithm>
 
@@ -85,7 +86,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(DecodeParams p
 #pragma unroll
         for (int k = 0; k < kBatch; ++k) {
             const int pr = pb + k * stride + sub;
-            hv[k] = (hin && pr < p.P) ? reinterpret_cast<const float4 *>(hin + (int64_t)pr * p.N)[col]
+            hv[k] = (hin && pr < p.P) ? __ldcs(reinterpret_cast<const float4 *>(hin + (int64_t)pr * p.N) + col)
                                       : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         }
 #pragma unroll
@@ -99,7 +100,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(DecodeParams p
                 o.y = fmaf(a, hv[k].y, dx * Bv.y);
                 o.z = fmaf(a, hv[k].z, dx * Bv.z);
                 o.w = fmaf(a, hv[k].w, dx * Bv.w);
-                reinterpret_cast<float4 *>(hout + (int64_t)pr * p.N)[col] = o;
+                __stcs(reinterpret_cast<float4 *>(hout + (int64_t)pr * p.N) + col, o);
                 part = fmaf(Cv.x, o.x, fmaf(Cv.y, o.y, fmaf(Cv.z, o.z, Cv.w * o.w)));
             }
             // sum over the nq lanes of this row

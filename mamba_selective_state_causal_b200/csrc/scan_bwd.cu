@@ -33,8 +33,10 @@
 // runs over the whole sequence, last chunk first, and ends in dh0.
 // Only non-positive differences of cs are exponentiated.
 #include <algorithm>
+#include <type_traits>
 
 #include "ssd_common.cuh"
+#include "tc_ptx.cuh"
 
 namespace ssd {
 namespace {
@@ -93,7 +95,148 @@ __device__ __forceinline__ void chunk_cumsum(const float *dts, float *cum, float
 }
 
 // ---------------------------------------------------------------- summaries
-// One CTA per (chunk, head, batch row): S_c, Gl_c and lam_c.
+// Tensor-core form for bf16 inputs with P = 64, N = 128: one CTA of 4 warps per
+// (chunk, head, batch row).  x, dy, B and C are bf16 values, exact as MMA operands;
+// the fp32 weights are applied to x and dy and each product is split into a bf16
+// high part and a bf16 remainder (hi + lo carries 16 significant bits), so that
+//   S^T  = B^T (w_x o x)_hi + B^T (w_x o x)_lo,   Gl^T = C^T (w_g o dy)_hi + C^T (w_g o dy)_lo
+// accumulate in fp32 in TMEM (M = n = 128 lanes, N = p = 64 columns each) with an
+// error of about 2^-17 of each term: far inside the backward's 1e-5.  Operand tiles
+// are written by the threads in the 128B-swizzled layout the MMA descriptors expect.
+using namespace tc;
+constexpr int kSumTcThreads = 128;
+constexpr uint32_t kSumBox = kQb * 128;              // 64 rows x 128 bytes: one 128B-swizzled box
+
+struct SmemSumTc {
+    uint8_t bt[2 * kSumBox];     // B rows of the chunk, n = 0..63 | 64..127 (A operand of S^T, MN-major)
+    uint8_t ct[2 * kSumBox];     // C rows, likewise (A operand of Gl^T)
+    uint8_t xh[kSumBox], xl[kSumBox];   // (w_x o x) high part and remainder (B operand, MN-major, N = 64)
+    uint8_t gh[kSumBox], gl[kSumBox];   // (w_g o dy) high part and remainder
+    float dts[kQb], cum[kQb];
+    uint64_t done;
+    uint32_t tmem;
+};
+
+__device__ __forceinline__ uint32_t sum_swz(int r, int c)
+{
+    return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
+}
+
+// 8 bf16 values scaled by w in fp32, split into the bf16 of the product and the bf16 of what it leaves
+__device__ __forceinline__ void split8(uint4 v, float w, uint4 &hi, uint4 &lo)
+{
+    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float a = bf16_lo(in[i]) * w, b = bf16_hi(in[i]) * w;
+        h[i] = pack_bf16x2(a, b);
+        l[i] = pack_bf16x2(a - bf16_lo(h[i]), b - bf16_hi(h[i]));
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+__global__ void __launch_bounds__(kSumTcThreads) bwd_chunk_summary_tc_kernel(BwdParams p)
+{
+    extern __shared__ __align__(1024) uint8_t sst_raw[];
+    SmemSumTc &s = *reinterpret_cast<SmemSumTc *>((reinterpret_cast<uintptr_t>(sst_raw) + 1023) & ~uintptr_t(1023));
+    const int c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    constexpr int P = 64, N = 128;
+    const int g = (int)((int64_t)h * p.G / p.H);
+    const int64_t t0 = (int64_t)c * kQb;
+    const int rows = (int)(p.L - t0 < kQb ? p.L - t0 : kQb);
+    if (tid == 0) {
+        mbar_init(&s.done, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) { tmem_alloc(&s.tmem, 128); tmem_relinquish(); }
+    for (int i = tid; i < kQb; i += kSumTcThreads)
+        s.dts[i] = i < rows ? p.dt[((int64_t)bi * p.L + t0 + i) * p.H + h] : 0.0f;
+    // B and C rows: 16 chunks of 16 bytes per row, chunk q of row j to box q >> 3
+    const __nv_bfloat16 *Bg = reinterpret_cast<const __nv_bfloat16 *>(p.B) + bi * p.Bbs + t0 * p.Brs + (int64_t)g * N;
+    const __nv_bfloat16 *Cg = reinterpret_cast<const __nv_bfloat16 *>(p.C) + bi * p.Cbs + t0 * p.Crs + (int64_t)g * N;
+    for (int i = tid; i < kQb * 16; i += kSumTcThreads) {
+        const int j = i >> 4, q = i & 15;
+        const uint32_t o = (uint32_t)(q >> 3) * kSumBox + sum_swz(j, q & 7);
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4 *>(s.bt + o) = j < rows ? *reinterpret_cast<const uint4 *>(Bg + j * p.Brs + 8 * q) : z;
+        *reinterpret_cast<uint4 *>(s.ct + o) = j < rows ? *reinterpret_cast<const uint4 *>(Cg + j * p.Crs + 8 * q) : z;
+    }
+    __syncthreads();
+    chunk_cumsum(s.dts, s.cum, p.A[h]);
+    __syncthreads();
+    const float lam = s.cum[kQb - 1];
+    // x and dy rows, weighted and split: 8 chunks of 16 bytes per row
+    const __nv_bfloat16 *xg = reinterpret_cast<const __nv_bfloat16 *>(p.x) + bi * p.xbs + t0 * p.xrs + (int64_t)h * P;
+    const __nv_bfloat16 *yg = reinterpret_cast<const __nv_bfloat16 *>(p.dy) + bi * p.dybs + t0 * p.dyrs + (int64_t)h * P;
+    for (int i = tid; i < kQb * 8; i += kSumTcThreads) {
+        const int j = i >> 3, q = i & 7;
+        const uint32_t o = sum_swz(j, q);
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        const uint4 xv = j < rows ? *reinterpret_cast<const uint4 *>(xg + j * p.xrs + 8 * q) : z;
+        const uint4 yv = j < rows ? *reinterpret_cast<const uint4 *>(yg + j * p.dyrs + 8 * q) : z;
+        uint4 hi, lo;
+        split8(xv, s.dts[j] * expf(lam - s.cum[j]), hi, lo);
+        *reinterpret_cast<uint4 *>(s.xh + o) = hi;
+        *reinterpret_cast<uint4 *>(s.xl + o) = lo;
+        split8(yv, expf(s.cum[j]), hi, lo);
+        *reinterpret_cast<uint4 *>(s.gh + o) = hi;
+        *reinterpret_cast<uint4 *>(s.gl + o) = lo;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = s.tmem;       // S^T at columns 0..63, Gl^T at 64..127
+    if (tid == 0) {
+        const uint32_t id = idesc_bf16(128, 64, 1, 1);
+        const uint64_t dB = smem_desc(smem_u32(s.bt), kSumBox, 1024), dC = smem_desc(smem_u32(s.ct), kSumBox, 1024);
+        const uint64_t dXh = smem_desc(smem_u32(s.xh), 0, 1024), dXl = smem_desc(smem_u32(s.xl), 0, 1024);
+        const uint64_t dGh = smem_desc(smem_u32(s.gh), 0, 1024), dGl = smem_desc(smem_u32(s.gl), 0, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) mma_ss(tm, dB + kk * 128, dXh + kk * 128, id, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) mma_ss(tm, dB + kk * 128, dXl + kk * 128, id, true);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) mma_ss(tm + 64, dC + kk * 128, dGh + kk * 128, id, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) mma_ss(tm + 64, dC + kk * 128, dGl + kk * 128, id, true);
+        mma_commit(&s.done);
+    }
+    __syncwarp();
+    const int64_t unit = ((int64_t)bi * p.H + h) * p.nch + c;
+    if (tid == 0) p.ws_lam[unit] = lam;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&s.done, 0, nullptr, p.wait_limit_ns));
+    if (ok) {
+        // lane quarter warp holds state rows n = 32 warp + lane: S[p][n] and Gl[p][n] for every p
+        tc_fence_after();
+        const int n = 32 * warp + lane;
+        const uint32_t lb = (uint32_t)(32 * warp) << 16;
+        float *S = p.ws_h + unit * (int64_t)P * N + n;
+        float *Gl = p.ws_g + unit * (int64_t)P * N + n;
+#pragma unroll
+        for (int half = 0; half < 4; ++half) {
+            uint32_t v[32];
+            tmem_ld32(tm + lb + 32 * half, v);
+            tmem_wait_ld(v);
+            float *dst = half < 2 ? S : Gl;
+            const int pb = 32 * (half & 1);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) dst[(int64_t)(pb + i) * N] = __uint_as_float(v[i]);
+        }
+    } else if (lane == 0) {
+        atomicOr(p.status, kDevTimeout);
+    }
+    // the products are complete before TMEM is freed (a longer bound after a timeout)
+    if (!ok && tid == 0) mbar_wait(&s.done, 0, nullptr, 100000000ull);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tm, 128);
+}
+
+// One CTA per (chunk, head, batch row): S_c, Gl_c and lam_c (CUDA cores, any shape).
 template <typename T>
 __global__ void __launch_bounds__(kBwdThreads) bwd_chunk_summary_kernel(BwdParams p)
 {
@@ -571,8 +714,15 @@ int launch_bwd_t(BwdParams p, cudaStream_t st)
             cudaSuccess)
         return 7;
     const dim3 grid((unsigned)p.nch, (unsigned)p.H, (unsigned)p.b);
+    // bf16 inputs at P = 64, N = 128: the summaries on the tensor cores
+    const bool tc_summary = std::is_same<T, __nv_bfloat16>::value && p.P == 64 && p.N == 128;
+    const size_t s_tc = sizeof(SmemSumTc) + 1024;
+    if (tc_summary && cudaFuncSetAttribute(bwd_chunk_summary_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)s_tc) != cudaSuccess)
+        return 7;
     prof_begin(st, kKBwdSummary);
-    bwd_chunk_summary_kernel<T><<<grid, kBwdThreads, s1, st>>>(p);
+    if (tc_summary) bwd_chunk_summary_tc_kernel<<<grid, kSumTcThreads, s_tc, st>>>(p);
+    else bwd_chunk_summary_kernel<T><<<grid, kBwdThreads, s1, st>>>(p);
     prof_end(st, kKBwdSummary);
     const int64_t PN = (int64_t)p.P * p.N;
     const unsigned slices = (unsigned)((PN + 4 * kBwdThreads - 1) / (4 * kBwdThreads));

@@ -361,6 +361,9 @@ int scan_bwd_impl(const ssd_scan_bwd_args *a, cudaStream_t st)
     p.ws_pD = reinterpret_cast<float *>(ws + pl.off_pD);
     p.ws_dBh = reinterpret_cast<float *>(ws + pl.off_dB);
     p.ws_dCh = reinterpret_cast<float *>(ws + pl.off_dC);
+    p.status = status_ptr();
+    if (!p.status) return fail(SSD_ERR_LAUNCH, "no CUDA device available");
+    p.wait_limit_ns = env_hooks().wait_limit_ns;
     if (p.nch > 2147483647LL || (int64_t)p.b * p.H > 65535LL * 65535LL)
         return fail(SSD_ERR_SHAPE, "sequence too long for the backward grid");
     if (a->H > 65535 || a->b > 65535) return fail(SSD_ERR_SHAPE, "H and b must be at most 65535");

@@ -126,6 +126,8 @@ struct BwdParams {
     float *ws_dBh, *ws_dCh; // [b][L][H][N] per-head dB and dC
     float *ws_pA, *ws_pD;   // [b][H][nch] per-chunk dA and dD
     int stage_adjoint;      // set by the launcher: copy Gam and h_prev into shared memory
+    unsigned int *status;   // device status word (a bounded wait that gave up)
+    uint64_t wait_limit_ns; // bound of every device-side wait
 };
 
 // The conv part of the layer's backward pass (conv1d_silu.cu, layer_bwd.cu): the
