@@ -55,6 +55,9 @@ def parse_args():
     # the backward pass of the scan instead of the headline step: gradients from the
     # forward's checkpoints, on the 0.3B 16384-token workload (its own JSON line)
     ap.add_argument("--backward", action="store_true")
+    # the backward pass of the whole layer (conv1d + SiLU, then the scan) from the forward's state
+    # checkpoints and conv buffers, on the same workload (its own JSON line)
+    ap.add_argument("--layer-backward", action="store_true")
     # the gated RMS norm of the layer output on one 131072-token segment of the 0.3B shape
     ap.add_argument("--gated-norm", action="store_true")
     # the layer as two library calls (conv over every channel, then the scan) instead of the
@@ -642,6 +645,74 @@ def run_backward(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_layer_backward(args, world, rank, local):
+    """Gradients through the whole layer (conv1d + SiLU, then the scan) from the forward's state
+    checkpoints and conv buffers (each cell of s tokens rebuilt on its own), timed with CUDA
+    events like the headline step; the forward runs once, before the timing."""
+    import __graft_entry__
+    __graft_entry__.build()
+    import mamba_selective_state_causal_b200 as ssd
+    wl = ssd_synth.BY_NAME["mamba2-0.3b-L16k"]
+    d = torch.device("cuda", torch.cuda.current_device())
+    seed = rank_seed(wl, rank)
+    prm = ssd_synth.make_params(wl, device=d, seed=seed)
+    u = ssd_synth.make_u(wl, device=d, seed=seed)
+    dt = ssd_synth.make_dt(wl, prm["dt_bias"], device=d, seed=seed)
+    dy, dhf = ssd_synth.make_grads(wl, device=d, seed=seed)
+    dto, _ = ssd_synth.make_conv_grads(wl, device=d, seed=seed)
+    cc = torch.empty(wl.b, wl.L // wl.s, 3, wl.cch, dtype=u.dtype, device=d)
+    fwd = ssd.stream_forward(u, prm["w"], dt, prm["A"], prm["D"], H=wl.H, P=wl.P, N=wl.N, G=wl.G, Q=wl.Q,
+                             s=wl.s, conv_bias=prm["bias"], conv_ckpt=cc, keep_v=False)
+    ws = torch.empty(ssd.layer_backward_workspace_size(wl.b, wl.L, wl.H, wl.P, wl.N, wl.G, ssd.SSD_BF16),
+                     dtype=torch.uint8, device=d)
+    kw = dict(H=wl.H, P=wl.P, N=wl.N, G=wl.G, s=wl.s, conv_bias=prm["bias"], h_ckpt=fwd["h_ckpt"],
+              conv_ckpt=cc, dh_final=dhf, dtail_out=dto, workspace=ws)
+    out = ssd.layer_backward(u, prm["w"], dt, prm["A"], prm["D"], dy, **kw)
+
+    def step():
+        ssd.layer_backward(u, prm["w"], dt, prm["A"], prm["D"], dy, out=out, **kw)
+
+    clocks = clock_sampler(local)
+    clocks.start()
+    ms = time_steps(step, args.steps, args.warmup, world, local)
+    clk = clocks.stop()
+    ssd.sync_status()
+    ms = max_over_ranks(world, ms)
+    ssd.profile_begin()
+    prof_steps = min(args.steps, 5)
+    for _ in range(prof_steps):
+        step()
+    torch.cuda.synchronize()
+    prof = ssd.profile_end()
+    per_launch = {k: v["total_ms"] / v["launches"] for k, v in prof.items()}
+    nch = -(-wl.L // 64)
+    _, f_grad = bwd_flops_per_chunk_head(wl.P, wl.N)
+    grad_flops = f_grad * nch * wl.H * wl.b
+    achieved = grad_flops / (per_launch["bwd_chunk_grad"] / 1e3) / 1e12
+    line = {
+        "metric": "SSD layer backward tokens/s (0.3B shape, L=16384, cells rebuilt from state checkpoints "
+                  "and conv buffers)",
+        "value": wl.tokens * world * args.steps / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": wl.name + "-layer-backward", "batch": wl.b, "seq_len": wl.L, "heads": wl.H,
+                   "headdim": wl.P, "d_state": wl.N, "ckpt_stride": wl.s, "io_dtype": wl.dtype,
+                   "l2": "workspace and outputs larger than L2 (%.1f GB)" % (ws.numel() / 1e9)},
+        "roofline": {"bound": "alu", "kernel": "bwd_chunk_grad", "achieved": achieved, "peak": FP32_ALU_TFLOPS,
+                     "unit": "TFLOP/s", "frac": achieved / FP32_ALU_TFLOPS,
+                     "peak_source": "derived: 148 SMs x 128 fp32 FMA lanes x 2 x 1.965 GHz", "traffic": None,
+                     "algorithmic_flops_per_launch": grad_flops},
+        "kernels": {k: {"launches_per_step": v["launches"] / prof_steps, "ms_per_launch": per_launch[k]}
+                    for k, v in prof.items()},
+        # per step: the cells' conv, the scan backward's six, the conv backward and its reduction
+        "gpu_launches": 9 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def run_gated_norm(args, world, rank, local):
     """out = rmsnorm(y * silu(z)) * w on 131072 rows of the 0.3B d_inner (2048), bf16, one group."""
     import __graft_entry__
@@ -700,6 +771,9 @@ def main():
         return
     if args.backward:
         run_backward(args, world, rank, local)
+        return
+    if args.layer_backward:
+        run_layer_backward(args, world, rank, local)
         return
     if args.gated_norm:
         run_gated_norm(args, world, rank, local)

@@ -84,6 +84,22 @@ def test_bf16_exact_checkpoints(L, s):
     _compare(got, ref, TOL["f32"], wl)
 
 
+@pytest.mark.parametrize("wl", [
+    ssd_synth.scaled(W[1], b=2, L=777, H=4, G=2, s=256),                 # tensor-core summaries, two groups
+    ssd_synth.scaled(W[1], b=1, L=600, H=2, P=32, N=64, Q=64, s=128),    # bf16 off the tensor-core shape
+], ids=["bf16-tc-summaries-two-groups", "bf16-cuda-core-summaries"])
+def test_bf16_summary_paths(wl):
+    """bf16 inputs through both forms of the chunk summaries (tensor cores at P = 64, N = 128 with
+    the group of every head; CUDA cores elsewhere), exact checkpoints, to 1e-5."""
+    prm, dt, x, Bm, Cm, h0, dy, dhf = _inputs(wl, seed=14)
+    ref = _oracle_bwd(wl, prm, dt, x, Bm, Cm, h0, dy, dhf)
+    fwd = oracle.scan(x.float().numpy(), Bm.float().numpy(), Cm.float().numpy(), dt.numpy(), prm["A"].numpy(),
+                      prm["D"].numpy(), h0.double().numpy(), s=wl.s, H=wl.H, P=wl.P, G=wl.G)
+    ck = torch.from_numpy(fwd["h_ckpt"]).float()
+    got = _gpu_bwd(wl, prm, dt, x, Bm, Cm, h0, dy, dhf, h_ckpt=ck, s=wl.s)
+    _compare(got, ref, TOL["f32"], wl)
+
+
 def test_bf16_with_gpu_forward_checkpoints():
     """The training pipeline: the tensor-core forward writes the checkpoints, the backward reads them."""
     wl = ssd_synth.scaled(W[1], b=2, L=2048, H=8, s=512)
