@@ -23,27 +23,48 @@ namespace {
 constexpr int kTB = 64;          // tokens per thread, walked from the last
 constexpr int kConvBwdThreads = 256;
 
+// dLoss/dv of channel c at row (bi, t)
+__device__ __forceinline__ float dv_at(const ConvBwdParams &p, int64_t bi, int64_t t, int c)
+{
+    const int64_t row = bi * p.L + t;
+    if (c < p.HP) return p.dx[row * p.HP + c];
+    if (c < p.HP + p.GN) return p.dB[row * p.GN + (c - p.HP)];
+    return p.dC[row * p.GN + (c - p.HP - p.GN)];
+}
+
+// dz = dv silu'(z) from the conv window u[t-3 .. t] (as token t's cell sees it)
+__device__ __forceinline__ float dz_of(float dv, const float4 &wq, float bs, const float (&uw)[4])
+{
+    float z = bs;
+    z = fmaf(wq.x, uw[0], z);
+    z = fmaf(wq.y, uw[1], z);
+    z = fmaf(wq.z, uw[2], z);
+    z = fmaf(wq.w, uw[3], z);
+    const float sg = 1.0f / (1.0f + expf(-z));
+    return dv * (sg * (1.0f + z * (1.0f - sg)));
+}
+
+template <typename T>
+__device__ __forceinline__ void load_window(const ConvBwdParams &p, int64_t bi, int64_t t, int c, float (&uw)[4])
+{
+#pragma unroll
+    for (int k = 0; k < 4; ++k) uw[k] = cell_val<T>(p, bi, t, t - 3 + k, c);
+}
+
 template <typename T>
 __device__ __forceinline__ float dz_at(const ConvBwdParams &p, int64_t bi, int64_t t, int c, const float4 &wq,
                                        float bs)
 {
     if (t >= p.L) return 0.0f;
-    float z = bs;
-    z = fmaf(wq.x, cell_val<T>(p, bi, t, t - 3, c), z);
-    z = fmaf(wq.y, cell_val<T>(p, bi, t, t - 2, c), z);
-    z = fmaf(wq.z, cell_val<T>(p, bi, t, t - 1, c), z);
-    z = fmaf(wq.w, cell_val<T>(p, bi, t, t, c), z);
-    const int64_t row = bi * p.L + t;
-    float dv;
-    if (c < p.HP) dv = p.dx[row * p.HP + c];
-    else if (c < p.HP + p.GN) dv = p.dB[row * p.GN + (c - p.HP)];
-    else dv = p.dC[row * p.GN + (c - p.HP - p.GN)];
-    const float sg = 1.0f / (1.0f + expf(-z));
-    return dv * (sg * (1.0f + z * (1.0f - sg)));
+    float uw[4];
+    load_window<T>(p, bi, t, c, uw);
+    return dz_of(dv_at(p, bi, t, c), wq, bs, uw);
 }
 
 // One thread per (batch row, block of kTB tokens, channel); consecutive threads
-// take consecutive channels, so every row access is coalesced.
+// take consecutive channels, so every row access is coalesced.  The thread walks
+// its block from the last token with the conv window of u in registers, one new
+// row per token (rows before a cell come from its conv buffer).
 template <typename T>
 __global__ void __launch_bounds__(kConvBwdThreads) conv_bwd_kernel(ConvBwdParams p, int64_t nblk)
 {
@@ -60,20 +81,37 @@ __global__ void __launch_bounds__(kConvBwdThreads) conv_bwd_kernel(ConvBwdParams
     float d1 = dz_at<T>(p, bi, t1, c, wq, bs), d2 = dz_at<T>(p, bi, t1 + 1, c, wq, bs),
           d3 = dz_at<T>(p, bi, t1 + 2, c, wq, bs);
     float gw0 = 0.0f, gw1 = 0.0f, gw2 = 0.0f, gw3 = 0.0f, gb = 0.0f;
-    for (int64_t t = t1 - 1; t >= t0; --t) {
-        const float d0 = dz_at<T>(p, bi, t, c, wq, bs);
-        float g = wq.w * d0;
-        g = fmaf(wq.z, d1, g);
-        g = fmaf(wq.y, d2, g);
-        g = fmaf(wq.x, d3, g);
-        if (p.dtail_out && t >= p.L - 3) g += p.dtail_out[(bi * 3 + (t - (p.L - 3))) * p.C_ch + c];
-        p.du[(bi * p.L + t) * p.C_ch + c] = g;
-        gb += d0;
-        gw0 = fmaf(d0, cell_val<T>(p, bi, t, t - 3, c), gw0);
-        gw1 = fmaf(d0, cell_val<T>(p, bi, t, t - 2, c), gw1);
-        gw2 = fmaf(d0, cell_val<T>(p, bi, t, t - 1, c), gw2);
-        gw3 = fmaf(d0, cell_val<T>(p, bi, t, t, c), gw3);
-        d3 = d2; d2 = d1; d1 = d0;
+    float uw[4];
+    load_window<T>(p, bi, t1 - 1, c, uw);
+    // a block never crosses a cell (blocks and cells are multiples of 64 tokens), so the window
+    // only slides; each group of four tokens issues its loads before it computes
+    for (int64_t tg = t1 - 1; tg >= t0; tg -= 4) {
+        float dvv[4], un[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int64_t t = tg - i;
+            dvv[i] = t >= t0 ? dv_at(p, bi, t, c) : 0.0f;
+            un[i] = t > t0 ? cell_val<T>(p, bi, t - 1, t - 4, c) : 0.0f;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int64_t t = tg - i;
+            if (t < t0) break;
+            const float d0 = dz_of(dvv[i], wq, bs, uw);
+            float g = wq.w * d0;
+            g = fmaf(wq.z, d1, g);
+            g = fmaf(wq.y, d2, g);
+            g = fmaf(wq.x, d3, g);
+            if (p.dtail_out && t >= p.L - 3) g += p.dtail_out[(bi * 3 + (t - (p.L - 3))) * p.C_ch + c];
+            p.du[(bi * p.L + t) * p.C_ch + c] = g;
+            gb += d0;
+            gw0 = fmaf(d0, uw[0], gw0);
+            gw1 = fmaf(d0, uw[1], gw1);
+            gw2 = fmaf(d0, uw[2], gw2);
+            gw3 = fmaf(d0, uw[3], gw3);
+            d3 = d2; d2 = d1; d1 = d0;
+            uw[3] = uw[2]; uw[2] = uw[1]; uw[1] = uw[0]; uw[0] = un[i];
+        }
     }
     const int64_t slot = (bi * nblk + blk) * p.C_ch + c;
     reinterpret_cast<float4 *>(p.ws_dw)[slot] = make_float4(gw0, gw1, gw2, gw3);

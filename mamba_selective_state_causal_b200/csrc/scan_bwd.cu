@@ -307,7 +307,7 @@ __device__ __forceinline__ float4 f4_fma(float a, float4 x, float4 y)
     return make_float4(fmaf(a, x.x, y.x), fmaf(a, x.y, y.y), fmaf(a, x.z, y.z), fmaf(a, x.w, y.w));
 }
 
-constexpr int kChainAhead = 8;    // chunk summaries loaded ahead of the chain
+constexpr int kChainAhead = 16;   // chunk summaries loaded ahead of the chain
 
 // State entering every chunk, per cell: h = start of the cell (h0 or the
 // checkpoint before it); for each chunk c of the cell: slot c := h, then
