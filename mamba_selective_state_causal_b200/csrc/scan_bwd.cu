@@ -455,23 +455,32 @@ __global__ void __launch_bounds__(kGradThreads) bwd_chunk_grad_kernel(BwdParams 
         ecs[i] = expf(cum[i]);
         eend[i] = expf(lam - cum[i]);
     }
-    // CB[t][j] = C_t . B_j and GX[t][j] = dy_t . x_j, all t, j (a tile's columns are c0 + 16q)
+    // CB[t][j] = C_t . B_j and GX[t][j] = dy_t . x_j, all t, j (a tile's columns are c0 + 16q);
+    // with 512 threads the first half forms CB's tiles and the second half GX's at the same time
     constexpr int kQt = kQb / 4;
-    for (int tile = tid; tile < kQt * kQt; tile += blockDim.x) {
+    const int half = blockDim.x >= 2 * kQt * kQt ? (int)(blockDim.x / 2) : 0;
+    for (int w = tid; w < (half ? (int)blockDim.x : kQt * kQt); w += blockDim.x) {
+        const bool do_cb = half ? w < half : true, do_gx = half ? w >= half : true;
+        const int tile = half ? w % half : w;
+        if (tile >= kQt * kQt) continue;
         const int r0 = (tile / kQt) * 4, c0 = tile % kQt;
         float acc[4][4];
-        zero4x4(acc);
-        mm4x4(acc, cs, N1, 1, bs, 1, N1, N, r0, 1, c0, kQt);
+        if (do_cb) {
+            zero4x4(acc);
+            mm4x4(acc, cs, N1, 1, bs, 1, N1, N, r0, 1, c0, kQt);
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+            for (int r = 0; r < 4; ++r)
 #pragma unroll
-            for (int q = 0; q < 4; ++q) CB[(r0 + r) * kQ1 + c0 + q * kQt] = acc[r][q];
-        zero4x4(acc);
-        mm4x4(acc, gs, P1, 1, xs, 1, P1, P, r0, 1, c0, kQt);
+                for (int q = 0; q < 4; ++q) CB[(r0 + r) * kQ1 + c0 + q * kQt] = acc[r][q];
+        }
+        if (do_gx) {
+            zero4x4(acc);
+            mm4x4(acc, gs, P1, 1, xs, 1, P1, P, r0, 1, c0, kQt);
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+            for (int r = 0; r < 4; ++r)
 #pragma unroll
-            for (int q = 0; q < 4; ++q) GX[(r0 + r) * kQ1 + c0 + q * kQt] = acc[r][q];
+                for (int q = 0; q < 4; ++q) GX[(r0 + r) * kQ1 + c0 + q * kQt] = acc[r][q];
+        }
     }
     __syncthreads();
     float gam_h = 0.0f;
