@@ -241,8 +241,9 @@ constexpr int kCellTB = 64;      // tokens per thread of the cell rebuild
 // One thread per (batch row, block of kCellTB tokens, channel), consecutive threads on consecutive
 // channels; the thread slides the conv window of u along its block in registers, one new row per
 // token (rows before a cell come from its conv buffer).
+// six CTAs per SM: more warps in flight beat the few registers spilled
 template <typename T>
-__global__ void conv_cells_kernel(ConvBwdParams p, int64_t nblk)
+__global__ void __launch_bounds__(256, 6) conv_cells_kernel(ConvBwdParams p, int64_t nblk)
 {
     const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (gid >= (int64_t)p.b * nblk * p.C_ch) return;

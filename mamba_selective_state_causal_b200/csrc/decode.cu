@@ -35,7 +35,8 @@ template <> __device__ __forceinline__ float dec_silu<__nv_bfloat16>(float z)
 template <> __device__ __forceinline__ float dec_silu<float>(float z) { return z / (1.0f + expf(-z)); }
 
 template <typename T>
-__global__ void __launch_bounds__(kDecThreads) decode_step_kernel(DecodeParams p)
+// six CTAs per SM (at most 40 registers): the state loads need the warps to cover their latency
+__global__ void __launch_bounds__(kDecThreads, 6) decode_step_kernel(DecodeParams p)
 {
     extern __shared__ float dsm[];          // x [P], B [N], C [N] of this (stream, head)
     float *xs = dsm, *Bs = dsm + p.P, *Cs = Bs + p.N;

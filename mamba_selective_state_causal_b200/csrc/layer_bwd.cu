@@ -65,8 +65,9 @@ __device__ __forceinline__ float dz_at(const ConvBwdParams &p, int64_t bi, int64
 // take consecutive channels, so every row access is coalesced.  The thread walks
 // its block from the last token with the conv window of u in registers, one new
 // row per token (rows before a cell come from its conv buffer).
+// four CTAs per SM (at most 64 registers): enough warps to cover the loads of the serial walk
 template <typename T>
-__global__ void __launch_bounds__(kConvBwdThreads) conv_bwd_kernel(ConvBwdParams p, int64_t nblk)
+__global__ void __launch_bounds__(kConvBwdThreads, 4) conv_bwd_kernel(ConvBwdParams p, int64_t nblk)
 {
     const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (gid >= (int64_t)p.b * nblk * p.C_ch) return;
