@@ -579,6 +579,50 @@ def bwd_flops_per_chunk_head(P, N, Q=64):
     return summary, grad
 
 
+def bwd_grad_bytes_per_chunk_head(wl, Q=64):
+    """Bytes one (64-token chunk, head) of the gradient kernel must move: read x and dy, the
+    chunk's Gam and h_prev (fp32, P x N each), dt and its share of the group's B and C rows;
+    write dx (fp32), the per-head dB and dC (fp32, Q x N each), ddt and the chunk's dA and dD
+    partials."""
+    e = 2 if wl.dtype == "bf16" else 4
+    reads = 2 * Q * wl.P * e + 2 * wl.P * wl.N * 4 + Q * 4 + 2 * Q * wl.N * e * wl.G / wl.H
+    writes = Q * wl.P * 4 + 2 * Q * wl.N * 4 + Q * 4 + 8
+    return reads + writes
+
+
+def bwd_grad_mma_flops_per_chunk_head(P, N, Q=64):
+    """Issued dense bf16 MMA flops of one (chunk, head) in the tensor-core gradient kernel:
+    C B^T and dy x^T; B Gam^T, C h_prev^T, Gam^T x^T and h_prev^T dy^T over the three bf16
+    pieces of Gam and h_prev; the three intra-chunk products over the two pieces of the
+    masked operand."""
+    return 2 * Q * Q * N + 2 * Q * Q * P + 3 * 4 * (2 * Q * P * N) + 2 * (2 * Q * Q * P + 2 * 2 * N * Q * Q)
+
+
+def bwd_grad_roofline(wl, ms_per_launch):
+    """Roofline of the gradient kernel: on the tensor-core form (bf16, P = 64, N = 128) the
+    bytes it must move against the HBM peak, with its issued MMA flops beside them; on the
+    CUDA-core form its fp32 multiply-add flops against the CUDA cores' FMA issue."""
+    units = -(-wl.L // 64) * wl.H * wl.b
+    if wl.dtype == "bf16" and wl.P == 64 and wl.N == 128:
+        peak, peak_src = hbm_peak()
+        tpeak, tpeak_src = bf16_peak()
+        alg = bwd_grad_bytes_per_chunk_head(wl) * units
+        achieved = alg / (ms_per_launch / 1e3) / 1e9
+        tflops = bwd_grad_mma_flops_per_chunk_head(wl.P, wl.N) * units / (ms_per_launch / 1e3) / 1e12
+        return {"bound": "hbm", "kernel": "bwd_chunk_grad_tc", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_source": peak_src, "traffic": None,
+                "algorithmic_bytes_per_launch": alg, "tensor_achieved_tflops": tflops,
+                "tensor_peak_tflops": tpeak, "tensor_frac": tflops / tpeak, "tensor_peak_source": tpeak_src,
+                "tensor_flops": "issued dense bf16 MMA flops of the kernel"}
+    _, f_grad = bwd_flops_per_chunk_head(wl.P, wl.N)
+    grad_flops = f_grad * units
+    achieved = grad_flops / (ms_per_launch / 1e3) / 1e12
+    return {"bound": "alu", "kernel": "bwd_chunk_grad", "achieved": achieved, "peak": FP32_ALU_TFLOPS,
+            "unit": "TFLOP/s", "frac": achieved / FP32_ALU_TFLOPS,
+            "peak_source": "derived: 148 SMs x 128 fp32 FMA lanes x 2 x 1.965 GHz", "traffic": None,
+            "algorithmic_flops_per_launch": grad_flops}
+
+
 def run_backward(args, world, rank, local):
     """Gradients through the scan from the forward's checkpoints (cell recompute), timed
     with CUDA events like the headline step; the forward runs once, before the timing."""
@@ -618,8 +662,6 @@ def run_backward(args, world, rank, local):
     per_launch = {k: v["total_ms"] / v["launches"] for k, v in prof.items()}
     nch = -(-wl.L // 64)
     f_sum, f_grad = bwd_flops_per_chunk_head(wl.P, wl.N)
-    grad_flops = f_grad * nch * wl.H * wl.b
-    achieved = grad_flops / (per_launch["bwd_chunk_grad"] / 1e3) / 1e12
     step_flops = (f_sum + f_grad) * nch * wl.H * wl.b
     line = {
         "metric": "SSD scan backward tokens/s (0.3B shape, L=16384, cells recomputed from checkpoints)",
@@ -630,10 +672,7 @@ def run_backward(args, world, rank, local):
         "config": {"workload": wl.name + "-backward", "batch": wl.b, "seq_len": wl.L, "heads": wl.H,
                    "headdim": wl.P, "d_state": wl.N, "ckpt_stride": wl.s, "io_dtype": wl.dtype,
                    "l2": "workspace and outputs larger than L2 (%.1f GB)" % (ws.numel() / 1e9)},
-        "roofline": {"bound": "alu", "kernel": "bwd_chunk_grad", "achieved": achieved, "peak": FP32_ALU_TFLOPS,
-                     "unit": "TFLOP/s", "frac": achieved / FP32_ALU_TFLOPS,
-                     "peak_source": "derived: 148 SMs x 128 fp32 FMA lanes x 2 x 1.965 GHz", "traffic": None,
-                     "algorithmic_flops_per_launch": grad_flops},
+        "roofline": bwd_grad_roofline(wl, per_launch["bwd_chunk_grad"]),
         "step_flops": step_flops,
         "kernels": {k: {"launches_per_step": v["launches"] / prof_steps, "ms_per_launch": per_launch[k]}
                     for k, v in prof.items()},
@@ -685,10 +724,6 @@ def run_layer_backward(args, world, rank, local):
     torch.cuda.synchronize()
     prof = ssd.profile_end()
     per_launch = {k: v["total_ms"] / v["launches"] for k, v in prof.items()}
-    nch = -(-wl.L // 64)
-    _, f_grad = bwd_flops_per_chunk_head(wl.P, wl.N)
-    grad_flops = f_grad * nch * wl.H * wl.b
-    achieved = grad_flops / (per_launch["bwd_chunk_grad"] / 1e3) / 1e12
     line = {
         "metric": "SSD layer backward tokens/s (0.3B shape, L=16384, cells rebuilt from state checkpoints "
                   "and conv buffers)",
@@ -699,10 +734,7 @@ def run_layer_backward(args, world, rank, local):
         "config": {"workload": wl.name + "-layer-backward", "batch": wl.b, "seq_len": wl.L, "heads": wl.H,
                    "headdim": wl.P, "d_state": wl.N, "ckpt_stride": wl.s, "io_dtype": wl.dtype,
                    "l2": "workspace and outputs larger than L2 (%.1f GB)" % (ws.numel() / 1e9)},
-        "roofline": {"bound": "alu", "kernel": "bwd_chunk_grad", "achieved": achieved, "peak": FP32_ALU_TFLOPS,
-                     "unit": "TFLOP/s", "frac": achieved / FP32_ALU_TFLOPS,
-                     "peak_source": "derived: 148 SMs x 128 fp32 FMA lanes x 2 x 1.965 GHz", "traffic": None,
-                     "algorithmic_flops_per_launch": grad_flops},
+        "roofline": bwd_grad_roofline(wl, per_launch["bwd_chunk_grad"]),
         "kernels": {k: {"launches_per_step": v["launches"] / prof_steps, "ms_per_launch": per_launch[k]}
                     for k, v in prof.items()},
         # per step: the cells' conv, the scan backward's six, the conv backward and its reduction

@@ -1,5 +1,6 @@
 // scan_bwd.cu -- gradients of the selective scan, recomputing each cell of s
-// tokens from its checkpoint (CUDA cores, fp32 math).
+// tokens from its checkpoint (fp32 math; for bf16 inputs at P = 64, N = 128 the
+// chunk summaries and the gradient contractions run on tcgen05).
 //
 // The layer is the recurrence h_t = a_t h_{t-1} + dt_t x_t B_t^T,
 // y_t = C_t^T h_t + D x_t with a_t = exp(dt_t A) (pith.science verdict for
@@ -643,6 +644,491 @@ __global__ void __launch_bounds__(kGradThreads) bwd_chunk_grad_kernel(BwdParams 
     }
 }
 
+// ---------------------------------------------------------------- gradients on tcgen05
+// Tensor-core form of the gradient kernel for bf16 inputs with P = 64, N = 128: one CTA of
+// 8 warps per (chunk, head, batch row).  Every contraction of the chunk runs as tcgen05
+// products with fp32 accumulators in TMEM; x, dy, B, C are exact bf16 operands.  Gam and
+// h_prev enter as three bf16 pieces (high, middle, low: 24 significant bits, as fp32 has),
+// because dA sums dt_t dl_t over the whole sequence with cancellation and its terms al_t and
+// be_j come from them; the masked decayed CB and GX enter as a bf16 high part plus a bf16
+// remainder (about 2^-17 of each term), as in the summaries above.
+//   phase 1 (inputs only):         CB = C B^T, GX = dy x^T            (M = 64: t x j)
+//                                  dxI = B Gam^T, Yo = C h_prev^T     (M = 64: j x p, t x p)
+//                                  dBr^T = Gam^T x^T, dC^T = h_prev^T dy^T   (M = 128: n x j, n x t)
+//   CUDA cores:                    mask and decay CB, GX (and GX dt_j) into operand tiles,
+//                                  K and its prefix sums, al_t from Yo, be_j from dxI, and
+//                                  the inter-chunk accumulators rescaled in TMEM
+//                                  (dxI and dBr^T by e^{lam - cs_j}, dC^T by e^{cs_t})
+//   phase 2 (accumulate on top):   dx += CBm^T dy, dBr^T += C^T GXm, dC^T += B^T (GXm dt)^T
+// An M = 64 accumulator keeps row m in TMEM lane (m mod 16) + 32 (m / 16): lanes 0..15 of
+// each warp's lane quarter.
+constexpr int kGradTcThreads = 256;
+constexpr uint32_t kColCB = 0, kColGX = 64, kColDX = 128, kColYO = 192, kColBR = 256, kColDC = 320;
+
+struct SmemGradTc {
+    uint8_t x[kSumBox];                    // x rows [t][p]
+    uint8_t dy[kSumBox];                   // dy rows [t][p]
+    uint8_t b[2 * kSumBox];                // B rows [j][n], n = 0..63 | 64..127
+    uint8_t c[2 * kSumBox];                // C rows [t][n]
+    union {
+        struct {                           // phase 1
+            uint8_t g[3][2 * kSumBox];     // Gam [p][n]: high, middle and low pieces
+            uint8_t hs[3][2 * kSumBox];    // h_prev [p][n]
+        } in;
+        struct {                           // phase 2, once phase 1 has read the above
+            uint8_t cb[2][kSumBox];        // CBm [t][j] = e^{cs_t - cs_j} C_t.B_j (j <= t): high, remainder
+            uint8_t gx[2][kSumBox];        // GXm [t][j] = e^{cs_t - cs_j} dy_t.x_j (j <= t)
+            uint8_t gd[2][kSumBox];        // GXm [t][j] dt_j
+            float kp[kQb * kQb];           // row-exclusive prefix sums of K, row t rotated by t
+        } mid;
+    } u;
+    float dts[kQb], cum[kQb], ecs[kQb], eend[kQb];
+    float al[kQb], be[kQb], dl0[kQb], din[kQb];
+    float red[4][kQb];                     // din partials, one row per lane quarter
+    float part[kGradTcThreads / 32];       // <Gam, h_prev> partials
+    float pdd[4], pa[2];
+    uint64_t done1, done2;
+    uint32_t tmem;
+    int ok;
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// bf16 element (r, col) of a 64-row tile of 128-byte rows in the 128B-swizzled layout;
+// columns 64..127 live in a second tile kSumBox further on
+__device__ __forceinline__ float tile_at(const uint8_t *tile, int r, int col)
+{
+    const uint32_t off = (uint32_t)(col >> 6) * kSumBox + sum_swz(r, (col & 63) >> 3) + (uint32_t)(col & 7) * 2u;
+    const uint16_t v = *reinterpret_cast<const uint16_t *>(tile + off);
+    return __uint_as_float((uint32_t)v << 16);
+}
+
+// fp32 pair -> bf16 high parts and bf16 remainders (each difference is exact in fp32)
+__device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t &lo)
+{
+    hi = pack_bf16x2(a, b);
+    lo = pack_bf16x2(a - bf16_lo(hi), b - bf16_hi(hi));
+}
+
+// fp32 pair -> three bf16 pieces whose sum is the pair to about 2^-27
+__device__ __forceinline__ void split3(float a, float b, uint32_t &hi, uint32_t &md, uint32_t &lo)
+{
+    hi = pack_bf16x2(a, b);
+    const float ra = a - bf16_lo(hi), rb = b - bf16_hi(hi);
+    md = pack_bf16x2(ra, rb);
+    lo = pack_bf16x2(ra - bf16_lo(md), rb - bf16_hi(md));
+}
+
+__global__ void __launch_bounds__(kGradTcThreads, 1) bwd_chunk_grad_tc_kernel(BwdParams p)
+{
+    extern __shared__ __align__(1024) uint8_t sgt_raw[];
+    SmemGradTc &s = *reinterpret_cast<SmemGradTc *>((reinterpret_cast<uintptr_t>(sgt_raw) + 1023) & ~uintptr_t(1023));
+    const int c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    constexpr int P = 64, N = 128;
+    const int g = (int)((int64_t)h * p.G / p.H);
+    const int64_t t0 = (int64_t)c * kQb;
+    const int rows = (int)(p.L - t0 < kQb ? p.L - t0 : kQb);
+    const int64_t unit = ((int64_t)bi * p.H + h) * p.nch + c;
+    const float Ah = p.A[h];
+    const float Dh = p.D ? p.D[h] : 0.0f;
+    if (tid == 0) {
+        mbar_init(&s.done1, 1);
+        mbar_init(&s.done2, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) { tmem_alloc(&s.tmem, 512); tmem_relinquish(); }
+
+    // x, dy, B, C rows: 16-byte asynchronous copies into the swizzled tiles, rows past L zero
+    {
+        const __nv_bfloat16 *xg = reinterpret_cast<const __nv_bfloat16 *>(p.x) + bi * p.xbs + t0 * p.xrs + (int64_t)h * P;
+        const __nv_bfloat16 *yg = reinterpret_cast<const __nv_bfloat16 *>(p.dy) + bi * p.dybs + t0 * p.dyrs + (int64_t)h * P;
+        const __nv_bfloat16 *Bg = reinterpret_cast<const __nv_bfloat16 *>(p.B) + bi * p.Bbs + t0 * p.Brs + (int64_t)g * N;
+        const __nv_bfloat16 *Cg = reinterpret_cast<const __nv_bfloat16 *>(p.C) + bi * p.Cbs + t0 * p.Crs + (int64_t)g * N;
+        for (int i = tid; i < kQb * 8; i += kGradTcThreads) {
+            const int r = i >> 3, q = i & 7;
+            const bool v = r < rows;
+            const int64_t rs = v ? r : 0;
+            const uint32_t o = sum_swz(r, q);
+            cp_async16(smem_u32(s.x) + o, xg + rs * p.xrs + 8 * q, v);
+            cp_async16(smem_u32(s.dy) + o, yg + rs * p.dyrs + 8 * q, v);
+        }
+        for (int i = tid; i < kQb * 16; i += kGradTcThreads) {
+            const int r = i >> 4, q = i & 15;
+            const bool v = r < rows;
+            const int64_t rs = v ? r : 0;
+            const uint32_t o = (uint32_t)(q >> 3) * kSumBox + sum_swz(r, q & 7);
+            cp_async16(smem_u32(s.b) + o, Bg + rs * p.Brs + 8 * q, v);
+            cp_async16(smem_u32(s.c) + o, Cg + rs * p.Crs + 8 * q, v);
+        }
+    }
+    for (int i = tid; i < kQb; i += kGradTcThreads) s.dts[i] = i < rows ? p.dt[((int64_t)bi * p.L + t0 + i) * p.H + h] : 0.0f;
+    // Gam and h_prev of the chunk: fp32 in, three bf16 pieces out; <Gam, h_prev> on the way
+    {
+        constexpr int kPer = P * N / 4 / kGradTcThreads;
+        const float4 *Gg = reinterpret_cast<const float4 *>(p.ws_g + unit * (int64_t)P * N);
+        const float4 *Hg = reinterpret_cast<const float4 *>(p.ws_h + unit * (int64_t)P * N);
+        float4 gv[kPer], hv[kPer];
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            gv[k] = Gg[tid + k * kGradTcThreads];
+            hv[k] = Hg[tid + k * kGradTcThreads];
+        }
+        float part = 0.0f;
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            const int i = tid + k * kGradTcThreads;
+            const int pr = i >> 5, n = (i & 31) * 4;
+            part = fmaf(gv[k].x, hv[k].x, part);
+            part = fmaf(gv[k].y, hv[k].y, part);
+            part = fmaf(gv[k].z, hv[k].z, part);
+            part = fmaf(gv[k].w, hv[k].w, part);
+            const uint32_t o = (uint32_t)(n >> 6) * kSumBox + sum_swz(pr, (n & 63) >> 3) + (uint32_t)(n & 7) * 2u;
+            uint32_t a0[3], a1[3];
+            split3(gv[k].x, gv[k].y, a0[0], a0[1], a0[2]);
+            split3(gv[k].z, gv[k].w, a1[0], a1[1], a1[2]);
+#pragma unroll
+            for (int pc = 0; pc < 3; ++pc) *reinterpret_cast<uint2 *>(s.u.in.g[pc] + o) = make_uint2(a0[pc], a1[pc]);
+            split3(hv[k].x, hv[k].y, a0[0], a0[1], a0[2]);
+            split3(hv[k].z, hv[k].w, a1[0], a1[1], a1[2]);
+#pragma unroll
+            for (int pc = 0; pc < 3; ++pc) *reinterpret_cast<uint2 *>(s.u.in.hs[pc] + o) = make_uint2(a0[pc], a1[pc]);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if (lane == 0) s.part[warp] = part;
+    }
+    cp_async_wait_all();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = s.tmem;
+    constexpr uint64_t kBoxD = kSumBox >> 4;
+    auto koff = [](int kk) -> uint64_t { return (uint64_t)((kk >> 2) * kBoxD + (kk & 3) * 2); };   // K-major K-step
+    if (tid == 0) {
+        // phase 1: every product of the inputs alone
+        const uint32_t id64 = idesc_bf16(64, 64, 0, 0), id128 = idesc_bf16(128, 64, 1, 0);
+        const uint64_t kC = smem_desc(smem_u32(s.c), 16, 1024), kB = smem_desc(smem_u32(s.b), 16, 1024);
+        const uint64_t kY = smem_desc(smem_u32(s.dy), 16, 1024), kX = smem_desc(smem_u32(s.x), 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) mma_ss(tm + kColCB, kC + koff(kk), kB + koff(kk), id64, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColGX, kY + koff(kk), kX + koff(kk), id64, kk > 0);
+#pragma unroll
+        for (int pc = 0; pc < 3; ++pc) {
+            const uint64_t kG = smem_desc(smem_u32(s.u.in.g[pc]), 16, 1024);
+            const uint64_t kH = smem_desc(smem_u32(s.u.in.hs[pc]), 16, 1024);
+            const uint64_t mG = smem_desc(smem_u32(s.u.in.g[pc]), kSumBox, 1024);
+            const uint64_t mH = smem_desc(smem_u32(s.u.in.hs[pc]), kSumBox, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) mma_ss(tm + kColDX, kB + koff(kk), kG + koff(kk), id64, pc > 0 || kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) mma_ss(tm + kColYO, kC + koff(kk), kH + koff(kk), id64, pc > 0 || kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColBR, mG + kk * 128, kX + koff(kk), id128, pc > 0 || kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColDC, mH + kk * 128, kY + koff(kk), id128, pc > 0 || kk > 0);
+        }
+        mma_commit(&s.done1);
+    }
+    if (tid == 32) {
+        float acc = 0.0f;
+        for (int i = 0; i < kQb; ++i) { acc = fmaf(s.dts[i], Ah, acc); s.cum[i] = acc; }
+    }
+    __syncthreads();
+    const float lam = s.cum[kQb - 1];
+    if (tid < kQb) {
+        s.ecs[tid] = expf(s.cum[tid]);
+        s.eend[tid] = expf(lam - s.cum[tid]);
+    }
+    float gam_h = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kGradTcThreads / 32; ++w) gam_h += s.part[w];
+    const float term3 = expf(lam) * gam_h;
+    if (tid == 0) s.ok = mbar_wait(&s.done1, 0, nullptr, p.wait_limit_ns) ? 1 : 0;
+    __syncthreads();
+    const bool ok1 = s.ok != 0;
+    if (ok1) {
+        tc_fence_after();
+        if (warp < 4) {
+            // rows t of CB and GX: mask and decay into the phase-2 operand tiles; K's prefix sums
+            const int q = warp, t = 16 * q + (lane & 15);
+            const bool act = lane < 16;
+            const uint32_t lb = (uint32_t)(32 * q) << 16;
+            const float cum_t = s.cum[t];
+            float *kprow = s.u.mid.kp + t * kQb;
+            float run = 0.0f, dd = 0.0f;
+#pragma unroll 1
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t cbv[32], gxv[32];
+                tmem_ld32(tm + kColCB + lb + 32 * hf, cbv);
+                tmem_ld32(tm + kColGX + lb + 32 * hf, gxv);
+                tmem_wait_ld(cbv);
+                tmem_wait_ld(gxv);
+#pragma unroll
+                for (int k8 = 0; k8 < 4; ++k8) {
+                    uint32_t ch[4], cl[4], xh[4], xl[4], dh[4], dl[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float cm[2], xm[2], dm[2];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int k = 8 * k8 + 2 * e + u, j = 32 * hf + k;
+                            const float cb = __uint_as_float(cbv[k]), gx = __uint_as_float(gxv[k]);
+                            const float seg = j <= t ? expf(cum_t - s.cum[j]) : 0.0f;
+                            const float gxm = seg * gx, gd = gxm * s.dts[j];
+                            cm[u] = seg * cb;
+                            xm[u] = gxm;
+                            dm[u] = gd;
+                            if (act) kprow[(j + t) & (kQb - 1)] = run;
+                            run += j < t ? gd * cb : 0.0f;
+                            if (j == t) dd = gx;
+                        }
+                        split2(cm[0], cm[1], ch[e], cl[e]);
+                        split2(xm[0], xm[1], xh[e], xl[e]);
+                        split2(dm[0], dm[1], dh[e], dl[e]);
+                    }
+                    if (act) {
+                        const uint32_t o = sum_swz(t, 4 * hf + k8);
+                        *reinterpret_cast<uint4 *>(s.u.mid.cb[0] + o) = make_uint4(ch[0], ch[1], ch[2], ch[3]);
+                        *reinterpret_cast<uint4 *>(s.u.mid.cb[1] + o) = make_uint4(cl[0], cl[1], cl[2], cl[3]);
+                        *reinterpret_cast<uint4 *>(s.u.mid.gx[0] + o) = make_uint4(xh[0], xh[1], xh[2], xh[3]);
+                        *reinterpret_cast<uint4 *>(s.u.mid.gx[1] + o) = make_uint4(xl[0], xl[1], xl[2], xl[3]);
+                        *reinterpret_cast<uint4 *>(s.u.mid.gd[0] + o) = make_uint4(dh[0], dh[1], dh[2], dh[3]);
+                        *reinterpret_cast<uint4 *>(s.u.mid.gd[1] + o) = make_uint4(dl[0], dl[1], dl[2], dl[3]);
+                    }
+                }
+            }
+            // dD of the chunk: the diagonal of GX (decay 1 there)
+            dd = act ? dd : 0.0f;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) dd += __shfl_xor_sync(0xffffffffu, dd, o);
+            if (lane == 0) s.pdd[q] = dd;
+        } else {
+            // the inter-chunk accumulators: be_j, al_t, then rescaled in place
+            const int q = warp - 4;
+            const bool act = lane < 16;
+            const int r16 = 16 * q + (lane & 15);
+            const uint32_t lb = (uint32_t)(32 * q) << 16;
+            {
+                // dxI[j][p] = B_j . Gam[p]: be_j = e^{lam - cs_j} dt_j x_j . dxI[j]; dxI *= e^{lam - cs_j}
+                const int j = r16;
+                const float ej = s.eend[j];
+                float sbe = 0.0f;
+#pragma unroll 1
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t v[32];
+                    tmem_ld32(tm + kColDX + lb + 32 * hf, v);
+                    tmem_wait_ld(v);
+#pragma unroll
+                    for (int k8 = 0; k8 < 4; ++k8) {
+                        const uint4 xv = *reinterpret_cast<const uint4 *>(s.x + sum_swz(j, 4 * hf + k8));
+                        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            sbe = fmaf(bf16_lo(xw[e]), __uint_as_float(v[8 * k8 + 2 * e]), sbe);
+                            sbe = fmaf(bf16_hi(xw[e]), __uint_as_float(v[8 * k8 + 2 * e + 1]), sbe);
+                        }
+                    }
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * ej);
+                    tmem_st32(tm + kColDX + lb + 32 * hf, v);
+                }
+                if (act) s.be[j] = ej * s.dts[j] * sbe;
+            }
+            {
+                // Yo[t][p] = C_t . h_prev[p]: al_t = e^{cs_t} dy_t . Yo[t]
+                const int t = r16;
+                float sal = 0.0f;
+#pragma unroll 1
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t v[32];
+                    tmem_ld32(tm + kColYO + lb + 32 * hf, v);
+                    tmem_wait_ld(v);
+#pragma unroll
+                    for (int k8 = 0; k8 < 4; ++k8) {
+                        const uint4 yv = *reinterpret_cast<const uint4 *>(s.dy + sum_swz(t, 4 * hf + k8));
+                        const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            sal = fmaf(bf16_lo(yw[e]), __uint_as_float(v[8 * k8 + 2 * e]), sal);
+                            sal = fmaf(bf16_hi(yw[e]), __uint_as_float(v[8 * k8 + 2 * e + 1]), sal);
+                        }
+                    }
+                }
+                if (act) s.al[t] = s.ecs[t] * sal;
+            }
+            // dBr^T[n][j] *= e^{lam - cs_j}, dC^T[n][t] *= e^{cs_t}
+#pragma unroll 1
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t v[32];
+                tmem_ld32(tm + kColBR + lb + 32 * hf, v);
+                tmem_wait_ld(v);
+#pragma unroll
+                for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * s.eend[32 * hf + k]);
+                tmem_st32(tm + kColBR + lb + 32 * hf, v);
+                tmem_ld32(tm + kColDC + lb + 32 * hf, v);
+                tmem_wait_ld(v);
+#pragma unroll
+                for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * s.ecs[32 * hf + k]);
+                tmem_st32(tm + kColDC + lb + 32 * hf, v);
+            }
+            tmem_wait_st();
+        }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (ok1 && tid == 0) {
+        // phase 2: the intra-chunk products, accumulated onto the rescaled inter-chunk terms
+        const uint32_t idx = idesc_bf16(64, 64, 1, 1), idbr = idesc_bf16(128, 64, 1, 1), iddc = idesc_bf16(128, 64, 1, 0);
+        const uint64_t mCBh = smem_desc(smem_u32(s.u.mid.cb[0]), kSumBox, 1024), mCBl = smem_desc(smem_u32(s.u.mid.cb[1]), kSumBox, 1024);
+        const uint64_t mY = smem_desc(smem_u32(s.dy), kSumBox, 1024);
+        const uint64_t mC = smem_desc(smem_u32(s.c), kSumBox, 1024), mB = smem_desc(smem_u32(s.b), kSumBox, 1024);
+        const uint64_t mGXh = smem_desc(smem_u32(s.u.mid.gx[0]), kSumBox, 1024), mGXl = smem_desc(smem_u32(s.u.mid.gx[1]), kSumBox, 1024);
+        const uint64_t kGDh = smem_desc(smem_u32(s.u.mid.gd[0]), 16, 1024), kGDl = smem_desc(smem_u32(s.u.mid.gd[1]), 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColDX, mCBh + kk * 128, mY + kk * 128, idx, true);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColDX, mCBl + kk * 128, mY + kk * 128, idx, true);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColBR, mC + kk * 128, mGXh + kk * 128, idbr, true);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColBR, mC + kk * 128, mGXl + kk * 128, idbr, true);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColDC, mB + kk * 128, kGDh + koff(kk), iddc, true);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColDC, mB + kk * 128, kGDl + koff(kk), iddc, true);
+        mma_commit(&s.done2);
+    }
+    if (ok1 && tid < kQb) {
+        // dl_t without the B_t . dBr_t term: sum_{u>=t} al_u + sum_{t'>=t} sum_{j<t} K[t'][j]
+        //   + e^{lam} <Gam, h_prev> + sum_{j<t} be_j
+        const int t = tid;
+        float rr = 0.0f, suf = 0.0f, pre = 0.0f;
+        for (int u = t; u < kQb; ++u) {
+            rr += s.u.mid.kp[u * kQb + ((t + u) & (kQb - 1))];
+            suf += s.al[u];
+        }
+        for (int j = 0; j < t; ++j) pre += s.be[j];
+        s.dl0[t] = suf + rr + term3 + pre;
+    }
+    if (ok1 && tid == kQb) p.ws_pD[unit] = s.pdd[0] + s.pdd[1] + s.pdd[2] + s.pdd[3];
+    if (tid == 0) s.ok = ok1 && mbar_wait(&s.done2, 0, nullptr, p.wait_limit_ns) ? 1 : 0;
+    __syncthreads();
+    const bool ok2 = s.ok != 0;
+    if (ok2) {
+        tc_fence_after();
+        const int64_t rstride = (int64_t)p.H * N;    // floats between tokens of dBh and dCh
+        if (warp < 4) {
+            // dBr^T[n][j]: dB_j = dt_j dBr_j (per head), and B_j . dBr_j summed over n
+            const int q = warp, n = 32 * q + lane;
+            const uint32_t lb = (uint32_t)(32 * q) << 16;
+            float *dBh = p.ws_dBh + (((int64_t)bi * p.L + t0) * p.H + h) * N + n;
+            float pr[kQb];
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t v[32];
+                tmem_ld32(tm + kColBR + lb + 32 * hf, v);
+                tmem_wait_ld(v);
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    const int j = 32 * hf + k;
+                    const float br = __uint_as_float(v[k]);
+                    if (j < rows) dBh[j * rstride] = s.dts[j] * br;
+                    pr[j] = tile_at(s.b, j, n) * br;
+                }
+            }
+            // sums over the warp's 32 values of n for all 64 j: each halving step keeps one half
+            // of the remaining j and adds the partner lane's copy of it; lane l ends with j = 2l, 2l+1
+#pragma unroll
+            for (int w = 32; w >= 2; w >>= 1) {
+                const bool up = (lane & (w >> 1)) != 0;
+#pragma unroll
+                for (int k = 0; k < w; ++k) {
+                    const float send = up ? pr[k] : pr[k + w];
+                    const float keep = up ? pr[k + w] : pr[k];
+                    pr[k] = keep + __shfl_xor_sync(0xffffffffu, send, w >> 1);
+                }
+            }
+            s.red[q][2 * lane] = pr[0];
+            s.red[q][2 * lane + 1] = pr[1];
+        } else {
+            const int q = warp - 4, n = 32 * q + lane;
+            const uint32_t lb = (uint32_t)(32 * q) << 16;
+            // dC^T[n][t] is dC_t (per head)
+            float *dCh = p.ws_dCh + (((int64_t)bi * p.L + t0) * p.H + h) * N + n;
+#pragma unroll 1
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t v[32];
+                tmem_ld32(tm + kColDC + lb + 32 * hf, v);
+                tmem_wait_ld(v);
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    const int t = 32 * hf + k;
+                    if (t < rows) dCh[t * rstride] = __uint_as_float(v[k]);
+                }
+            }
+            // dx_j = D dy_j + dt_j (dx accumulator row j)
+            const int j = 16 * q + (lane & 15);
+            const bool act = lane < 16 && j < rows;
+            float *dxr = p.dx + ((int64_t)bi * p.L + t0 + j) * p.H * P + (int64_t)h * P;
+            const float dtj = s.dts[j];
+#pragma unroll 1
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t v[32];
+                tmem_ld32(tm + kColDX + lb + 32 * hf, v);
+                tmem_wait_ld(v);
+#pragma unroll
+                for (int k8 = 0; k8 < 4; ++k8) {
+                    const uint4 yv = *reinterpret_cast<const uint4 *>(s.dy + sum_swz(j, 4 * hf + k8));
+                    const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
+                    float o[8];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        o[2 * e] = fmaf(Dh, bf16_lo(yw[e]), dtj * __uint_as_float(v[8 * k8 + 2 * e]));
+                        o[2 * e + 1] = fmaf(Dh, bf16_hi(yw[e]), dtj * __uint_as_float(v[8 * k8 + 2 * e + 1]));
+                    }
+                    if (act) {
+                        float4 *d4 = reinterpret_cast<float4 *>(dxr + 32 * hf + 8 * k8);
+                        d4[0] = make_float4(o[0], o[1], o[2], o[3]);
+                        d4[1] = make_float4(o[4], o[5], o[6], o[7]);
+                    }
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (ok2 && tid < kQb) {
+        // dl_t, ddt_t = A dl_t + B_t . dBr_t, and this chunk's share of dA
+        const int t = tid;
+        const float din = s.red[0][t] + s.red[1][t] + s.red[2][t] + s.red[3][t];
+        const float dl = s.dl0[t];
+        if (t < rows) p.ddt[((int64_t)bi * p.L + t0 + t) * p.H + h] = fmaf(Ah, dl, din);
+        float a = s.dts[t] * dl;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        if (lane == 0) s.pa[warp] = a;
+    }
+    __syncthreads();
+    if (ok2 && tid == 0) p.ws_pA[unit] = s.pa[0] + s.pa[1];
+    if (tid == 0 && !ok2) {
+        // a bounded wait gave up: report it, and let the products in flight finish before TMEM is freed
+        atomicOr(p.status, kDevTimeout);
+        mbar_wait(ok1 ? &s.done2 : &s.done1, 0, nullptr, 100000000ull);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tm, 512);
+}
+
 // dB, dC: sum of the per-head partials over the heads of each group;
 // one thread per (batch row, token, group, n).
 __global__ void bwd_group_sum_kernel(BwdParams p)
@@ -723,11 +1209,13 @@ int launch_bwd_t(BwdParams p, cudaStream_t st)
             cudaSuccess)
         return 7;
     const dim3 grid((unsigned)p.nch, (unsigned)p.H, (unsigned)p.b);
-    // bf16 inputs at P = 64, N = 128: the summaries on the tensor cores
+    // bf16 inputs at P = 64, N = 128: the summaries and the gradients on the tensor cores
     const bool tc_summary = std::is_same<T, __nv_bfloat16>::value && p.P == 64 && p.N == 128;
-    const size_t s_tc = sizeof(SmemSumTc) + 1024;
-    if (tc_summary && cudaFuncSetAttribute(bwd_chunk_summary_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)s_tc) != cudaSuccess)
+    const size_t s_tc = sizeof(SmemSumTc) + 1024, s_gt = sizeof(SmemGradTc) + 1024;
+    if (tc_summary && (cudaFuncSetAttribute(bwd_chunk_summary_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            (int)s_tc) != cudaSuccess ||
+                       cudaFuncSetAttribute(bwd_chunk_grad_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            (int)s_gt) != cudaSuccess))
         return 7;
     prof_begin(st, kKBwdSummary);
     if (tc_summary) bwd_chunk_summary_tc_kernel<<<grid, kSumTcThreads, s_tc, st>>>(p);
@@ -741,7 +1229,8 @@ int launch_bwd_t(BwdParams p, cudaStream_t st)
     bwd_adjoint_chain_kernel<<<dim3(slices, (unsigned)p.H, (unsigned)p.b), kBwdThreads, 0, st>>>(p);
     prof_end(st, kKBwdChain);
     prof_begin(st, kKBwdGrad);
-    bwd_chunk_grad_kernel<T><<<grid, kGradThreads, s2, st>>>(p);
+    if (tc_summary) bwd_chunk_grad_tc_kernel<<<grid, kGradTcThreads, s_gt, st>>>(p);
+    else bwd_chunk_grad_kernel<T><<<grid, kGradThreads, s2, st>>>(p);
     prof_end(st, kKBwdGrad);
     prof_begin(st, kKBwdReduce);
     const int64_t total = (int64_t)p.b * p.L * p.G * p.N;
