@@ -646,48 +646,48 @@ __global__ void __launch_bounds__(kGradThreads) bwd_chunk_grad_kernel(BwdParams 
 
 // ---------------------------------------------------------------- gradients on tcgen05
 // Tensor-core form of the gradient kernel for bf16 inputs with P = 64, N = 128: one CTA of
-// 8 warps per (chunk, head, batch row).  Every contraction of the chunk runs as tcgen05
-// products with fp32 accumulators in TMEM; x, dy, B, C are exact bf16 operands.  Gam and
-// h_prev enter as three bf16 pieces (high, middle, low: 24 significant bits, as fp32 has),
-// because dA sums dt_t dl_t over the whole sequence with cancellation and its terms al_t and
-// be_j come from them; the masked decayed CB and GX enter as a bf16 high part plus a bf16
-// remainder (about 2^-17 of each term), as in the summaries above.
-//   phase 1 (inputs only):         CB = C B^T, GX = dy x^T            (M = 64: t x j)
-//                                  dxI = B Gam^T, Yo = C h_prev^T     (M = 64: j x p, t x p)
-//                                  dBr^T = Gam^T x^T, dC^T = h_prev^T dy^T   (M = 128: n x j, n x t)
-//   CUDA cores:                    mask and decay CB, GX (and GX dt_j) into operand tiles,
-//                                  K and its prefix sums, al_t from Yo, be_j from dxI, and
-//                                  the inter-chunk accumulators rescaled in TMEM
-//                                  (dxI and dBr^T by e^{lam - cs_j}, dC^T by e^{cs_t})
-//   phase 2 (accumulate on top):   dx += CBm^T dy, dBr^T += C^T GXm, dC^T += B^T (GXm dt)^T
-// An M = 64 accumulator keeps row m in TMEM lane (m mod 16) + 32 (m / 16): lanes 0..15 of
-// each warp's lane quarter.
+// 8 warps per (chunk, head, batch row), two CTAs per SM.  Every contraction of the chunk
+// runs as tcgen05 products with fp32 accumulators in TMEM; x, dy, B, C are exact bf16
+// operands.  Gam and h_prev enter as three bf16 pieces (high, middle, low: 24 significant
+// bits, as fp32 has), because dA sums dt_t dl_t over the whole sequence with cancellation
+// and its terms al_t and be_j come from them; the masked decayed CB and GX enter as a bf16
+// high part plus a bf16 remainder (about 2^-17 of each term), as in the summaries above.
+//   phase 1a:  CB = C B^T, GX = dy x^T (M = 64: t x j), dxI = B Gam^T (M = 64: j x p),
+//              dBr^T = Gam^T x^T (M = 128: n x j)
+//   phase 1b:  dC^T = h_prev^T dy^T (M = 128: n x t), h_prev in Gam's shared memory
+//   CUDA cores: mask and decay CB, GX (and GX dt_j) into the operand tiles of phase 2; K and
+//              its prefix sums; be_j = e^{lam-cs_j} dt_j x_j . dxI_j; al_t = e^{cs_t} C_t . dC^T_t;
+//              the inter-chunk accumulators rescaled in TMEM (dxI and dBr^T by e^{lam - cs_j},
+//              dC^T by e^{cs_t})
+//   phase 2:   dx += CBm^T dy, dBr^T += C^T GXm, dC^T += B^T (GXm dt)^T
+// An M = 64 accumulator keeps row m in TMEM lane (m mod 16) + 32 (m / 16), or 16 lanes
+// higher when its address says so: CB and GX share their 64 columns that way.
 constexpr int kGradTcThreads = 256;
-constexpr uint32_t kColCB = 0, kColGX = 64, kColDX = 128, kColYO = 192, kColBR = 256, kColDC = 320;
+constexpr uint32_t kColCG = 0, kColDX = 64, kColBR = 128, kColDC = 192, kGradTcCols = 256;
+constexpr uint32_t kLane16 = 16u << 16;   // TMEM address offset of lane 16
 
 struct SmemGradTc {
-    uint8_t x[kSumBox];                    // x rows [t][p]
     uint8_t dy[kSumBox];                   // dy rows [t][p]
     uint8_t b[2 * kSumBox];                // B rows [j][n], n = 0..63 | 64..127
     uint8_t c[2 * kSumBox];                // C rows [t][n]
     union {
         struct {                           // phase 1
-            uint8_t g[3][2 * kSumBox];     // Gam [p][n]: high, middle and low pieces
-            uint8_t hs[3][2 * kSumBox];    // h_prev [p][n]
+            uint8_t gh[3][2 * kSumBox];    // Gam [p][n] (1a), then h_prev [p][n] (1b): three pieces
+            uint8_t x[kSumBox];            // x rows [j][p] (1a)
         } in;
-        struct {                           // phase 2, once phase 1 has read the above
+        struct {                           // phase 2
             uint8_t cb[2][kSumBox];        // CBm [t][j] = e^{cs_t - cs_j} C_t.B_j (j <= t): high, remainder
             uint8_t gx[2][kSumBox];        // GXm [t][j] = e^{cs_t - cs_j} dy_t.x_j (j <= t)
             uint8_t gd[2][kSumBox];        // GXm [t][j] dt_j
-            float kp[kQb * kQb];           // row-exclusive prefix sums of K, row t rotated by t
+            float kp[kQb * kQb];           // prefix sums of K along each row half, row t rotated by t
         } mid;
     } u;
     float dts[kQb], cum[kQb], ecs[kQb], eend[kQb];
-    float al[kQb], be[kQb], dl0[kQb], din[kQb];
-    float red[4][kQb];                     // din partials, one row per lane quarter
+    float be[kQb], dl0[kQb], rowoff[kQb];  // rowoff[t] = sum_{j<32} K[t][j]
+    float red[4][kQb];                     // per lane quarter: C_t . dC^T_t (E1), B_j . dBr_j (E2)
     float part[kGradTcThreads / 32];       // <Gam, h_prev> partials
     float pdd[4], pa[2];
-    uint64_t done1, done2;
+    uint64_t done1, done3, done2;
     uint32_t tmem;
     int ok;
 };
@@ -724,7 +724,40 @@ __device__ __forceinline__ void split3(float a, float b, uint32_t &hi, uint32_t 
     lo = pack_bf16x2(ra - bf16_lo(md), rb - bf16_hi(md));
 }
 
-__global__ void __launch_bounds__(kGradTcThreads, 1) bwd_chunk_grad_tc_kernel(BwdParams p)
+// 64 values per lane -> their sums over the warp's 32 lanes: each halving step keeps one half
+// of the remaining values and adds the partner lane's copy of it; lane l ends with the sums of
+// values 2l and 2l+1 in v[0], v[1]
+__device__ __forceinline__ void warp_sum64(float (&v)[kQb], int lane)
+{
+#pragma unroll
+    for (int w = 32; w >= 2; w >>= 1) {
+        const bool up = (lane & (w >> 1)) != 0;
+#pragma unroll
+        for (int k = 0; k < w; ++k) {
+            const float send = up ? v[k] : v[k + w];
+            const float keep = up ? v[k + w] : v[k];
+            v[k] = keep + __shfl_xor_sync(0xffffffffu, send, w >> 1);
+        }
+    }
+}
+
+// Gam or h_prev (fp32 pieces of 4 in registers) -> the three bf16 pieces in the swizzled tiles
+__device__ __forceinline__ void store_pieces3(uint8_t (&dst)[3][2 * kSumBox], const float4 (&v)[8], int tid)
+{
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int i = tid + k * kGradTcThreads;
+        const int pr = i >> 5, n = (i & 31) * 4;
+        const uint32_t o = (uint32_t)(n >> 6) * kSumBox + sum_swz(pr, (n & 63) >> 3) + (uint32_t)(n & 7) * 2u;
+        uint32_t a0[3], a1[3];
+        split3(v[k].x, v[k].y, a0[0], a0[1], a0[2]);
+        split3(v[k].z, v[k].w, a1[0], a1[1], a1[2]);
+#pragma unroll
+        for (int pc = 0; pc < 3; ++pc) *reinterpret_cast<uint2 *>(dst[pc] + o) = make_uint2(a0[pc], a1[pc]);
+    }
+}
+
+__global__ void __launch_bounds__(kGradTcThreads, 2) bwd_chunk_grad_tc_kernel(BwdParams p)
 {
     extern __shared__ __align__(1024) uint8_t sgt_raw[];
     SmemGradTc &s = *reinterpret_cast<SmemGradTc *>((reinterpret_cast<uintptr_t>(sgt_raw) + 1023) & ~uintptr_t(1023));
@@ -737,16 +770,17 @@ __global__ void __launch_bounds__(kGradTcThreads, 1) bwd_chunk_grad_tc_kernel(Bw
     const int64_t unit = ((int64_t)bi * p.H + h) * p.nch + c;
     const float Ah = p.A[h];
     const float Dh = p.D ? p.D[h] : 0.0f;
+    const __nv_bfloat16 *xg = reinterpret_cast<const __nv_bfloat16 *>(p.x) + bi * p.xbs + t0 * p.xrs + (int64_t)h * P;
     if (tid == 0) {
         mbar_init(&s.done1, 1);
+        mbar_init(&s.done3, 1);
         mbar_init(&s.done2, 1);
         fence_mbar_init();
     }
-    if (warp == 0) { tmem_alloc(&s.tmem, 512); tmem_relinquish(); }
+    if (warp == 0) { tmem_alloc(&s.tmem, kGradTcCols); tmem_relinquish(); }
 
     // x, dy, B, C rows: 16-byte asynchronous copies into the swizzled tiles, rows past L zero
     {
-        const __nv_bfloat16 *xg = reinterpret_cast<const __nv_bfloat16 *>(p.x) + bi * p.xbs + t0 * p.xrs + (int64_t)h * P;
         const __nv_bfloat16 *yg = reinterpret_cast<const __nv_bfloat16 *>(p.dy) + bi * p.dybs + t0 * p.dyrs + (int64_t)h * P;
         const __nv_bfloat16 *Bg = reinterpret_cast<const __nv_bfloat16 *>(p.B) + bi * p.Bbs + t0 * p.Brs + (int64_t)g * N;
         const __nv_bfloat16 *Cg = reinterpret_cast<const __nv_bfloat16 *>(p.C) + bi * p.Cbs + t0 * p.Crs + (int64_t)g * N;
@@ -755,7 +789,7 @@ __global__ void __launch_bounds__(kGradTcThreads, 1) bwd_chunk_grad_tc_kernel(Bw
             const bool v = r < rows;
             const int64_t rs = v ? r : 0;
             const uint32_t o = sum_swz(r, q);
-            cp_async16(smem_u32(s.x) + o, xg + rs * p.xrs + 8 * q, v);
+            cp_async16(smem_u32(s.u.in.x) + o, xg + rs * p.xrs + 8 * q, v);
             cp_async16(smem_u32(s.dy) + o, yg + rs * p.dyrs + 8 * q, v);
         }
         for (int i = tid; i < kQb * 16; i += kGradTcThreads) {
@@ -768,40 +802,30 @@ __global__ void __launch_bounds__(kGradTcThreads, 1) bwd_chunk_grad_tc_kernel(Bw
         }
     }
     for (int i = tid; i < kQb; i += kGradTcThreads) s.dts[i] = i < rows ? p.dt[((int64_t)bi * p.L + t0 + i) * p.H + h] : 0.0f;
-    // Gam and h_prev of the chunk: fp32 in, three bf16 pieces out; <Gam, h_prev> on the way
+    // Gam and h_prev of the chunk (fp32); <Gam, h_prev> on the way; Gam's pieces to shared memory,
+    // h_prev's kept in registers until phase 1a has read Gam's
+    float4 hv[8];
     {
-        constexpr int kPer = P * N / 4 / kGradTcThreads;
         const float4 *Gg = reinterpret_cast<const float4 *>(p.ws_g + unit * (int64_t)P * N);
         const float4 *Hg = reinterpret_cast<const float4 *>(p.ws_h + unit * (int64_t)P * N);
-        float4 gv[kPer], hv[kPer];
+        float4 gv[8];
 #pragma unroll
-        for (int k = 0; k < kPer; ++k) {
+        for (int k = 0; k < 8; ++k) {
             gv[k] = Gg[tid + k * kGradTcThreads];
             hv[k] = Hg[tid + k * kGradTcThreads];
         }
         float part = 0.0f;
 #pragma unroll
-        for (int k = 0; k < kPer; ++k) {
-            const int i = tid + k * kGradTcThreads;
-            const int pr = i >> 5, n = (i & 31) * 4;
+        for (int k = 0; k < 8; ++k) {
             part = fmaf(gv[k].x, hv[k].x, part);
             part = fmaf(gv[k].y, hv[k].y, part);
             part = fmaf(gv[k].z, hv[k].z, part);
             part = fmaf(gv[k].w, hv[k].w, part);
-            const uint32_t o = (uint32_t)(n >> 6) * kSumBox + sum_swz(pr, (n & 63) >> 3) + (uint32_t)(n & 7) * 2u;
-            uint32_t a0[3], a1[3];
-            split3(gv[k].x, gv[k].y, a0[0], a0[1], a0[2]);
-            split3(gv[k].z, gv[k].w, a1[0], a1[1], a1[2]);
-#pragma unroll
-            for (int pc = 0; pc < 3; ++pc) *reinterpret_cast<uint2 *>(s.u.in.g[pc] + o) = make_uint2(a0[pc], a1[pc]);
-            split3(hv[k].x, hv[k].y, a0[0], a0[1], a0[2]);
-            split3(hv[k].z, hv[k].w, a1[0], a1[1], a1[2]);
-#pragma unroll
-            for (int pc = 0; pc < 3; ++pc) *reinterpret_cast<uint2 *>(s.u.in.hs[pc] + o) = make_uint2(a0[pc], a1[pc]);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
         if (lane == 0) s.part[warp] = part;
+        store_pieces3(s.u.in.gh, gv, tid);
     }
     cp_async_wait_all();
     fence_proxy_async_smem();
@@ -811,31 +835,27 @@ __global__ void __launch_bounds__(kGradTcThreads, 1) bwd_chunk_grad_tc_kernel(Bw
     const uint32_t tm = s.tmem;
     constexpr uint64_t kBoxD = kSumBox >> 4;
     auto koff = [](int kk) -> uint64_t { return (uint64_t)((kk >> 2) * kBoxD + (kk & 3) * 2); };   // K-major K-step
+    const uint32_t id64 = idesc_bf16(64, 64, 0, 0), id128 = idesc_bf16(128, 64, 1, 0);
+    uint64_t *last = nullptr;      // the barrier of the last commit (issuing thread)
     if (tid == 0) {
-        // phase 1: every product of the inputs alone
-        const uint32_t id64 = idesc_bf16(64, 64, 0, 0), id128 = idesc_bf16(128, 64, 1, 0);
+        // phase 1a
         const uint64_t kC = smem_desc(smem_u32(s.c), 16, 1024), kB = smem_desc(smem_u32(s.b), 16, 1024);
-        const uint64_t kY = smem_desc(smem_u32(s.dy), 16, 1024), kX = smem_desc(smem_u32(s.x), 16, 1024);
+        const uint64_t kY = smem_desc(smem_u32(s.dy), 16, 1024), kX = smem_desc(smem_u32(s.u.in.x), 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_ss(tm + kColCB, kC + koff(kk), kB + koff(kk), id64, kk > 0);
+        for (int kk = 0; kk < 8; ++kk) mma_ss(tm + kColCG, kC + koff(kk), kB + koff(kk), id64, kk > 0);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColGX, kY + koff(kk), kX + koff(kk), id64, kk > 0);
+        for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColCG + kLane16, kY + koff(kk), kX + koff(kk), id64, kk > 0);
 #pragma unroll
         for (int pc = 0; pc < 3; ++pc) {
-            const uint64_t kG = smem_desc(smem_u32(s.u.in.g[pc]), 16, 1024);
-            const uint64_t kH = smem_desc(smem_u32(s.u.in.hs[pc]), 16, 1024);
-            const uint64_t mG = smem_desc(smem_u32(s.u.in.g[pc]), kSumBox, 1024);
-            const uint64_t mH = smem_desc(smem_u32(s.u.in.hs[pc]), kSumBox, 1024);
+            const uint64_t kG = smem_desc(smem_u32(s.u.in.gh[pc]), 16, 1024);
+            const uint64_t mG = smem_desc(smem_u32(s.u.in.gh[pc]), kSumBox, 1024);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) mma_ss(tm + kColDX, kB + koff(kk), kG + koff(kk), id64, pc > 0 || kk > 0);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) mma_ss(tm + kColYO, kC + koff(kk), kH + koff(kk), id64, pc > 0 || kk > 0);
-#pragma unroll
             for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColBR, mG + kk * 128, kX + koff(kk), id128, pc > 0 || kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColDC, mH + kk * 128, kY + koff(kk), id128, pc > 0 || kk > 0);
         }
         mma_commit(&s.done1);
+        last = &s.done1;
     }
     if (tid == 32) {
         float acc = 0.0f;
@@ -853,83 +873,109 @@ __global__ void __launch_bounds__(kGradTcThreads, 1) bwd_chunk_grad_tc_kernel(Bw
     const float term3 = expf(lam) * gam_h;
     if (tid == 0) s.ok = mbar_wait(&s.done1, 0, nullptr, p.wait_limit_ns) ? 1 : 0;
     __syncthreads();
+    // phase 1b: h_prev's pieces over Gam's (phase 1a has read them)
+    if (s.ok) store_pieces3(s.u.in.gh, hv, tid);
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0 && s.ok) {
+        tc_fence_after();
+        const uint64_t kY = smem_desc(smem_u32(s.dy), 16, 1024);
+#pragma unroll
+        for (int pc = 0; pc < 3; ++pc) {
+            const uint64_t mH = smem_desc(smem_u32(s.u.in.gh[pc]), kSumBox, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColDC, mH + kk * 128, kY + koff(kk), id128, pc > 0 || kk > 0);
+        }
+        mma_commit(&s.done3);
+        last = &s.done3;
+        s.ok = mbar_wait(&s.done3, 0, nullptr, p.wait_limit_ns) ? 1 : 0;
+    }
+    __syncthreads();
     const bool ok1 = s.ok != 0;
     if (ok1) {
         tc_fence_after();
         if (warp < 4) {
-            // rows t of CB and GX: mask and decay into the phase-2 operand tiles; K's prefix sums
-            const int q = warp, t = 16 * q + (lane & 15);
-            const bool act = lane < 16;
+            // row t of CB (lanes 0..15) and of GX (lanes 16..31); after one exchange lanes 0..15
+            // hold columns j = 0..31 of both and lanes 16..31 columns 32..63
+            const int q = warp, hi = lane >> 4, t = 16 * q + (lane & 15);
             const uint32_t lb = (uint32_t)(32 * q) << 16;
+            float cbk[32], gxk[32];
+            {
+                uint32_t v0[32], v1[32];
+                tmem_ld32(tm + kColCG + lb, v0);
+                tmem_ld32(tm + kColCG + lb + 32, v1);
+                tmem_wait_ld(v0);
+                tmem_wait_ld(v1);
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    const uint32_t send = hi ? v0[k] : v1[k];
+                    const float keep = __uint_as_float(hi ? v1[k] : v0[k]);
+                    const float recv = __uint_as_float(__shfl_xor_sync(0xffffffffu, send, 16));
+                    cbk[k] = hi ? recv : keep;
+                    gxk[k] = hi ? keep : recv;
+                }
+            }
             const float cum_t = s.cum[t];
             float *kprow = s.u.mid.kp + t * kQb;
             float run = 0.0f, dd = 0.0f;
-#pragma unroll 1
-            for (int hf = 0; hf < 2; ++hf) {
-                uint32_t cbv[32], gxv[32];
-                tmem_ld32(tm + kColCB + lb + 32 * hf, cbv);
-                tmem_ld32(tm + kColGX + lb + 32 * hf, gxv);
-                tmem_wait_ld(cbv);
-                tmem_wait_ld(gxv);
 #pragma unroll
-                for (int k8 = 0; k8 < 4; ++k8) {
-                    uint32_t ch[4], cl[4], xh[4], xl[4], dh[4], dl[4];
+            for (int k8 = 0; k8 < 4; ++k8) {
+                uint32_t ch[4], cl[4], xh[4], xl[4], dh[4], dl[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        float cm[2], xm[2], dm[2];
+                for (int e = 0; e < 4; ++e) {
+                    float cm[2], xm[2], dm[2];
 #pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const int k = 8 * k8 + 2 * e + u, j = 32 * hf + k;
-                            const float cb = __uint_as_float(cbv[k]), gx = __uint_as_float(gxv[k]);
-                            const float seg = j <= t ? expf(cum_t - s.cum[j]) : 0.0f;
-                            const float gxm = seg * gx, gd = gxm * s.dts[j];
-                            cm[u] = seg * cb;
-                            xm[u] = gxm;
-                            dm[u] = gd;
-                            if (act) kprow[(j + t) & (kQb - 1)] = run;
-                            run += j < t ? gd * cb : 0.0f;
-                            if (j == t) dd = gx;
-                        }
-                        split2(cm[0], cm[1], ch[e], cl[e]);
-                        split2(xm[0], xm[1], xh[e], xl[e]);
-                        split2(dm[0], dm[1], dh[e], dl[e]);
+                    for (int u = 0; u < 2; ++u) {
+                        const int k = 8 * k8 + 2 * e + u, j = 32 * hi + k;
+                        const float seg = j <= t ? expf(cum_t - s.cum[j]) : 0.0f;
+                        const float gxm = seg * gxk[k], gd = gxm * s.dts[j];
+                        cm[u] = seg * cbk[k];
+                        xm[u] = gxm;
+                        dm[u] = gd;
+                        kprow[(j + t) & (kQb - 1)] = run;
+                        run += j < t ? gd * cbk[k] : 0.0f;
+                        if (j == t) dd = gxk[k];
                     }
-                    if (act) {
-                        const uint32_t o = sum_swz(t, 4 * hf + k8);
-                        *reinterpret_cast<uint4 *>(s.u.mid.cb[0] + o) = make_uint4(ch[0], ch[1], ch[2], ch[3]);
-                        *reinterpret_cast<uint4 *>(s.u.mid.cb[1] + o) = make_uint4(cl[0], cl[1], cl[2], cl[3]);
-                        *reinterpret_cast<uint4 *>(s.u.mid.gx[0] + o) = make_uint4(xh[0], xh[1], xh[2], xh[3]);
-                        *reinterpret_cast<uint4 *>(s.u.mid.gx[1] + o) = make_uint4(xl[0], xl[1], xl[2], xl[3]);
-                        *reinterpret_cast<uint4 *>(s.u.mid.gd[0] + o) = make_uint4(dh[0], dh[1], dh[2], dh[3]);
-                        *reinterpret_cast<uint4 *>(s.u.mid.gd[1] + o) = make_uint4(dl[0], dl[1], dl[2], dl[3]);
-                    }
+                    split2(cm[0], cm[1], ch[e], cl[e]);
+                    split2(xm[0], xm[1], xh[e], xl[e]);
+                    split2(dm[0], dm[1], dh[e], dl[e]);
                 }
+                const uint32_t o = sum_swz(t, 4 * hi + k8);
+                *reinterpret_cast<uint4 *>(s.u.mid.cb[0] + o) = make_uint4(ch[0], ch[1], ch[2], ch[3]);
+                *reinterpret_cast<uint4 *>(s.u.mid.cb[1] + o) = make_uint4(cl[0], cl[1], cl[2], cl[3]);
+                *reinterpret_cast<uint4 *>(s.u.mid.gx[0] + o) = make_uint4(xh[0], xh[1], xh[2], xh[3]);
+                *reinterpret_cast<uint4 *>(s.u.mid.gx[1] + o) = make_uint4(xl[0], xl[1], xl[2], xl[3]);
+                *reinterpret_cast<uint4 *>(s.u.mid.gd[0] + o) = make_uint4(dh[0], dh[1], dh[2], dh[3]);
+                *reinterpret_cast<uint4 *>(s.u.mid.gd[1] + o) = make_uint4(dl[0], dl[1], dl[2], dl[3]);
             }
+            if (!hi) s.rowoff[t] = run;
             // dD of the chunk: the diagonal of GX (decay 1 there)
-            dd = act ? dd : 0.0f;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) dd += __shfl_xor_sync(0xffffffffu, dd, o);
             if (lane == 0) s.pdd[q] = dd;
         } else {
-            // the inter-chunk accumulators: be_j, al_t, then rescaled in place
             const int q = warp - 4;
-            const bool act = lane < 16;
-            const int r16 = 16 * q + (lane & 15);
             const uint32_t lb = (uint32_t)(32 * q) << 16;
             {
-                // dxI[j][p] = B_j . Gam[p]: be_j = e^{lam - cs_j} dt_j x_j . dxI[j]; dxI *= e^{lam - cs_j}
-                const int j = r16;
+                // dx accumulator, row j in lanes 0..15: be_j = e^{lam - cs_j} dt_j x_j . dxI_j (x from
+                // global memory: its tile is gone), then dxI *= e^{lam - cs_j}
+                const int j = 16 * q + (lane & 15);
                 const float ej = s.eend[j];
+                uint4 xv[8];
+#pragma unroll
+                for (int c8 = 0; c8 < 8; ++c8)
+                    xv[c8] = j < rows ? *reinterpret_cast<const uint4 *>(xg + (int64_t)j * p.xrs + 8 * c8)
+                                      : make_uint4(0u, 0u, 0u, 0u);
                 float sbe = 0.0f;
-#pragma unroll 1
+#pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     uint32_t v[32];
                     tmem_ld32(tm + kColDX + lb + 32 * hf, v);
                     tmem_wait_ld(v);
 #pragma unroll
                     for (int k8 = 0; k8 < 4; ++k8) {
-                        const uint4 xv = *reinterpret_cast<const uint4 *>(s.x + sum_swz(j, 4 * hf + k8));
-                        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                        const uint32_t xw[4] = {xv[4 * hf + k8].x, xv[4 * hf + k8].y, xv[4 * hf + k8].z,
+                                                xv[4 * hf + k8].w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             sbe = fmaf(bf16_lo(xw[e]), __uint_as_float(v[8 * k8 + 2 * e]), sbe);
@@ -940,32 +986,33 @@ __global__ void __launch_bounds__(kGradTcThreads, 1) bwd_chunk_grad_tc_kernel(Bw
                     for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * ej);
                     tmem_st32(tm + kColDX + lb + 32 * hf, v);
                 }
-                if (act) s.be[j] = ej * s.dts[j] * sbe;
+                if (lane < 16) s.be[j] = ej * s.dts[j] * sbe;
             }
             {
-                // Yo[t][p] = C_t . h_prev[p]: al_t = e^{cs_t} dy_t . Yo[t]
-                const int t = r16;
-                float sal = 0.0f;
-#pragma unroll 1
+                // dC^T[n][t] = h_prev[.][n] . dy_t: C_t[n] dC^T[n][t] summed over n gives al_t / e^{cs_t};
+                // then dC^T *= e^{cs_t}
+                const int n = 32 * q + lane;
+                float pr[kQb];
+#pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     uint32_t v[32];
-                    tmem_ld32(tm + kColYO + lb + 32 * hf, v);
+                    tmem_ld32(tm + kColDC + lb + 32 * hf, v);
                     tmem_wait_ld(v);
 #pragma unroll
-                    for (int k8 = 0; k8 < 4; ++k8) {
-                        const uint4 yv = *reinterpret_cast<const uint4 *>(s.dy + sum_swz(t, 4 * hf + k8));
-                        const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            sal = fmaf(bf16_lo(yw[e]), __uint_as_float(v[8 * k8 + 2 * e]), sal);
-                            sal = fmaf(bf16_hi(yw[e]), __uint_as_float(v[8 * k8 + 2 * e + 1]), sal);
-                        }
+                    for (int k = 0; k < 32; ++k) {
+                        const int t = 32 * hf + k;
+                        const float a = __uint_as_float(v[k]);
+                        pr[t] = tile_at(s.c, t, n) * a;
+                        v[k] = __float_as_uint(a * s.ecs[t]);
                     }
+                    tmem_st32(tm + kColDC + lb + 32 * hf, v);
                 }
-                if (act) s.al[t] = s.ecs[t] * sal;
+                warp_sum64(pr, lane);
+                s.red[q][2 * lane] = pr[0];
+                s.red[q][2 * lane + 1] = pr[1];
             }
-            // dBr^T[n][j] *= e^{lam - cs_j}, dC^T[n][t] *= e^{cs_t}
-#pragma unroll 1
+            // dBr^T[n][j] *= e^{lam - cs_j}
+#pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 uint32_t v[32];
                 tmem_ld32(tm + kColBR + lb + 32 * hf, v);
@@ -973,11 +1020,6 @@ __global__ void __launch_bounds__(kGradTcThreads, 1) bwd_chunk_grad_tc_kernel(Bw
 #pragma unroll
                 for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * s.eend[32 * hf + k]);
                 tmem_st32(tm + kColBR + lb + 32 * hf, v);
-                tmem_ld32(tm + kColDC + lb + 32 * hf, v);
-                tmem_wait_ld(v);
-#pragma unroll
-                for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * s.ecs[32 * hf + k]);
-                tmem_st32(tm + kColDC + lb + 32 * hf, v);
             }
             tmem_wait_st();
         }
@@ -988,39 +1030,39 @@ __global__ void __launch_bounds__(kGradTcThreads, 1) bwd_chunk_grad_tc_kernel(Bw
     tc_fence_after();
     if (ok1 && tid == 0) {
         // phase 2: the intra-chunk products, accumulated onto the rescaled inter-chunk terms
-        const uint32_t idx = idesc_bf16(64, 64, 1, 1), idbr = idesc_bf16(128, 64, 1, 1), iddc = idesc_bf16(128, 64, 1, 0);
-        const uint64_t mCBh = smem_desc(smem_u32(s.u.mid.cb[0]), kSumBox, 1024), mCBl = smem_desc(smem_u32(s.u.mid.cb[1]), kSumBox, 1024);
+        const uint32_t idx = idesc_bf16(64, 64, 1, 1), idbr = idesc_bf16(128, 64, 1, 1);
         const uint64_t mY = smem_desc(smem_u32(s.dy), kSumBox, 1024);
         const uint64_t mC = smem_desc(smem_u32(s.c), kSumBox, 1024), mB = smem_desc(smem_u32(s.b), kSumBox, 1024);
-        const uint64_t mGXh = smem_desc(smem_u32(s.u.mid.gx[0]), kSumBox, 1024), mGXl = smem_desc(smem_u32(s.u.mid.gx[1]), kSumBox, 1024);
-        const uint64_t kGDh = smem_desc(smem_u32(s.u.mid.gd[0]), 16, 1024), kGDl = smem_desc(smem_u32(s.u.mid.gd[1]), 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColDX, mCBh + kk * 128, mY + kk * 128, idx, true);
+        for (int pc = 0; pc < 2; ++pc) {
+            const uint64_t mCB = smem_desc(smem_u32(s.u.mid.cb[pc]), kSumBox, 1024);
+            const uint64_t mGX = smem_desc(smem_u32(s.u.mid.gx[pc]), kSumBox, 1024);
+            const uint64_t kGD = smem_desc(smem_u32(s.u.mid.gd[pc]), 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColDX, mCBl + kk * 128, mY + kk * 128, idx, true);
+            for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColDX, mCB + kk * 128, mY + kk * 128, idx, true);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColBR, mC + kk * 128, mGXh + kk * 128, idbr, true);
+            for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColBR, mC + kk * 128, mGX + kk * 128, idbr, true);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColBR, mC + kk * 128, mGXl + kk * 128, idbr, true);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColDC, mB + kk * 128, kGDh + koff(kk), iddc, true);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColDC, mB + kk * 128, kGDl + koff(kk), iddc, true);
+            for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColDC, mB + kk * 128, kGD + koff(kk), id128, true);
+        }
         mma_commit(&s.done2);
+        last = &s.done2;
     }
     if (ok1 && tid < kQb) {
         // dl_t without the B_t . dBr_t term: sum_{u>=t} al_u + sum_{t'>=t} sum_{j<t} K[t'][j]
         //   + e^{lam} <Gam, h_prev> + sum_{j<t} be_j
         const int t = tid;
+        const bool upper = t >= 32;
         float rr = 0.0f, suf = 0.0f, pre = 0.0f;
         for (int u = t; u < kQb; ++u) {
-            rr += s.u.mid.kp[u * kQb + ((t + u) & (kQb - 1))];
-            suf += s.al[u];
+            rr += s.u.mid.kp[u * kQb + ((t + u) & (kQb - 1))] + (upper ? s.rowoff[u] : 0.0f);
+            suf += s.ecs[u] * (s.red[0][u] + s.red[1][u] + s.red[2][u] + s.red[3][u]);
         }
         for (int j = 0; j < t; ++j) pre += s.be[j];
         s.dl0[t] = suf + rr + term3 + pre;
     }
     if (ok1 && tid == kQb) p.ws_pD[unit] = s.pdd[0] + s.pdd[1] + s.pdd[2] + s.pdd[3];
+    __syncthreads();   // red is read before E2 writes it again
     if (tid == 0) s.ok = ok1 && mbar_wait(&s.done2, 0, nullptr, p.wait_limit_ns) ? 1 : 0;
     __syncthreads();
     const bool ok2 = s.ok != 0;
@@ -1046,18 +1088,7 @@ __global__ void __launch_bounds__(kGradTcThreads, 1) bwd_chunk_grad_tc_kernel(Bw
                     pr[j] = tile_at(s.b, j, n) * br;
                 }
             }
-            // sums over the warp's 32 values of n for all 64 j: each halving step keeps one half
-            // of the remaining j and adds the partner lane's copy of it; lane l ends with j = 2l, 2l+1
-#pragma unroll
-            for (int w = 32; w >= 2; w >>= 1) {
-                const bool up = (lane & (w >> 1)) != 0;
-#pragma unroll
-                for (int k = 0; k < w; ++k) {
-                    const float send = up ? pr[k] : pr[k + w];
-                    const float keep = up ? pr[k + w] : pr[k];
-                    pr[k] = keep + __shfl_xor_sync(0xffffffffu, send, w >> 1);
-                }
-            }
+            warp_sum64(pr, lane);
             s.red[q][2 * lane] = pr[0];
             s.red[q][2 * lane + 1] = pr[1];
         } else {
@@ -1065,7 +1096,7 @@ __global__ void __launch_bounds__(kGradTcThreads, 1) bwd_chunk_grad_tc_kernel(Bw
             const uint32_t lb = (uint32_t)(32 * q) << 16;
             // dC^T[n][t] is dC_t (per head)
             float *dCh = p.ws_dCh + (((int64_t)bi * p.L + t0) * p.H + h) * N + n;
-#pragma unroll 1
+#pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 uint32_t v[32];
                 tmem_ld32(tm + kColDC + lb + 32 * hf, v);
@@ -1076,12 +1107,12 @@ __global__ void __launch_bounds__(kGradTcThreads, 1) bwd_chunk_grad_tc_kernel(Bw
                     if (t < rows) dCh[t * rstride] = __uint_as_float(v[k]);
                 }
             }
-            // dx_j = D dy_j + dt_j (dx accumulator row j)
+            // dx_j = D dy_j + dt_j (dx accumulator row j, lanes 0..15)
             const int j = 16 * q + (lane & 15);
             const bool act = lane < 16 && j < rows;
             float *dxr = p.dx + ((int64_t)bi * p.L + t0 + j) * p.H * P + (int64_t)h * P;
             const float dtj = s.dts[j];
-#pragma unroll 1
+#pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 uint32_t v[32];
                 tmem_ld32(tm + kColDX + lb + 32 * hf, v);
@@ -1122,11 +1153,11 @@ __global__ void __launch_bounds__(kGradTcThreads, 1) bwd_chunk_grad_tc_kernel(Bw
     if (tid == 0 && !ok2) {
         // a bounded wait gave up: report it, and let the products in flight finish before TMEM is freed
         atomicOr(p.status, kDevTimeout);
-        mbar_wait(ok1 ? &s.done2 : &s.done1, 0, nullptr, 100000000ull);
+        if (last) mbar_wait(last, 0, nullptr, 100000000ull);
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tm, 512);
+    if (warp == 0) tmem_dealloc(tm, kGradTcCols);
 }
 
 // dB, dC: sum of the per-head partials over the heads of each group;
@@ -1215,7 +1246,9 @@ int launch_bwd_t(BwdParams p, cudaStream_t st)
     if (tc_summary && (cudaFuncSetAttribute(bwd_chunk_summary_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             (int)s_tc) != cudaSuccess ||
                        cudaFuncSetAttribute(bwd_chunk_grad_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            (int)s_gt) != cudaSuccess))
+                                            (int)s_gt) != cudaSuccess ||
+                       cudaFuncSetAttribute(bwd_chunk_grad_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                            (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess))
         return 7;
     prof_begin(st, kKBwdSummary);
     if (tc_summary) bwd_chunk_summary_tc_kernel<<<grid, kSumTcThreads, s_tc, st>>>(p);
