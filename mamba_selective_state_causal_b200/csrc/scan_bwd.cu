@@ -655,8 +655,9 @@ __global__ void __launch_bounds__(kGradThreads) bwd_chunk_grad_kernel(BwdParams 
 //   phase 1a:  CB = C B^T, GX = dy x^T (M = 64: t x j), dxI = B Gam^T (M = 64: j x p),
 //              dBr^T = Gam^T x^T (M = 128: n x j)
 //   phase 1b:  dC^T = h_prev^T dy^T (M = 128: n x t), h_prev in Gam's shared memory
-//   CUDA cores: mask and decay CB, GX (and GX dt_j) into the operand tiles of phase 2; K and
-//              its prefix sums; be_j = e^{lam-cs_j} dt_j x_j . dxI_j; al_t = e^{cs_t} C_t . dC^T_t;
+//   CUDA cores: mask and decay CB, GX (and GX dt_j) into the operand tiles of phase 2; K, its
+//              prefix sums and their column sums; be_j = e^{lam-cs_j} dt_j x_j . dxI_j;
+//              al_t = e^{cs_t} C_t . dC^T_t;
 //              the inter-chunk accumulators rescaled in TMEM (dxI and dBr^T by e^{lam - cs_j},
 //              dC^T by e^{cs_t})
 //   phase 2:   dx += CBm^T dy, dBr^T += C^T GXm, dC^T += B^T (GXm dt)^T
@@ -668,25 +669,25 @@ constexpr uint32_t kLane16 = 16u << 16;   // TMEM address offset of lane 16
 
 struct SmemGradTc {
     uint8_t dy[kSumBox];                   // dy rows [t][p]
+    uint8_t x[kSumBox];                    // x rows [j][p]
     uint8_t b[2 * kSumBox];                // B rows [j][n], n = 0..63 | 64..127
     uint8_t c[2 * kSumBox];                // C rows [t][n]
     union {
-        struct {                           // phase 1
-            uint8_t gh[3][2 * kSumBox];    // Gam [p][n] (1a), then h_prev [p][n] (1b): three pieces
-            uint8_t x[kSumBox];            // x rows [j][p] (1a)
-        } in;
+        uint8_t gh[3][2 * kSumBox];        // phase 1: Gam [p][n] (1a), then h_prev [p][n] (1b), three pieces
         struct {                           // phase 2
             uint8_t cb[2][kSumBox];        // CBm [t][j] = e^{cs_t - cs_j} C_t.B_j (j <= t): high, remainder
             uint8_t gx[2][kSumBox];        // GXm [t][j] = e^{cs_t - cs_j} dy_t.x_j (j <= t)
             uint8_t gd[2][kSumBox];        // GXm [t][j] dt_j
-            float kp[kQb * kQb];           // prefix sums of K along each row half, row t rotated by t
         } mid;
     } u;
-    float dts[kQb], cum[kQb], ecs[kQb], eend[kQb];
-    float be[kQb], dl0[kQb], rowoff[kQb];  // rowoff[t] = sum_{j<32} K[t][j]
-    float red[4][kQb];                     // per lane quarter: C_t . dC^T_t (E1), B_j . dBr_j (E2)
+    float dts[kQb], cum[kQb], ecs[kQb], eend[kQb], be[kQb], sbe[kQb];
+    float rrp[4][kQb];                     // sum_{t' >= t} of each row half's part of sum_{j < t} K[t'][j],
+                                           // over each quarter of rows t'
+    float rowoff[kQb];                     // sum_{j < 32} K[t][j]
+    float ral[4][kQb];                     // C_t . dC^T_t over each quarter of n (before the rescale)
+    float rdin[4][kQb];                    // sum_t GXm[t][j] CB[t][j] over each quarter of rows t
     float part[kGradTcThreads / 32];       // <Gam, h_prev> partials
-    float pdd[4], pa[2];
+    float pdd[4];
     uint64_t done1, done3, done2;
     uint32_t tmem;
     int ok;
@@ -706,6 +707,17 @@ __device__ __forceinline__ float tile_at(const uint8_t *tile, int r, int col)
     const uint32_t off = (uint32_t)(col >> 6) * kSumBox + sum_swz(r, (col & 63) >> 3) + (uint32_t)(col & 7) * 2u;
     const uint16_t v = *reinterpret_cast<const uint16_t *>(tile + off);
     return __uint_as_float((uint32_t)v << 16);
+}
+
+// e^d for d <= 0 as 2^(d log2 e) on the hardware's base-2 exponential (relative error about
+// 2^-22, and |d| 2^-24 from the rounding of d log2 e): the decay e^{cs_t - cs_j} of a
+// chunk-local cumsum difference
+constexpr float kLog2e = 1.44269504088896341f;
+__device__ __forceinline__ float exp2_approx(float a)
+{
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(a));
+    return r;
 }
 
 // fp32 pair -> bf16 high parts and bf16 remainders (each difference is exact in fp32)
@@ -741,19 +753,45 @@ __device__ __forceinline__ void warp_sum64(float (&v)[kQb], int lane)
     }
 }
 
-// Gam or h_prev (fp32 pieces of 4 in registers) -> the three bf16 pieces in the swizzled tiles
-__device__ __forceinline__ void store_pieces3(uint8_t (&dst)[3][2 * kSumBox], const float4 (&v)[8], int tid)
+// 16 values per lane -> their sums over each half warp (lanes 0..15, 16..31); lane l of a half
+// ends with the sum of value l in v[0]
+__device__ __forceinline__ void half_warp_sum16(float (&v)[16], int lane)
+{
+#pragma unroll
+    for (int w = 8; w >= 1; w >>= 1) {
+        const bool up = (lane & w) != 0;
+#pragma unroll
+        for (int k = 0; k < w; ++k) {
+            const float send = up ? v[k] : v[k + w];
+            const float keep = up ? v[k + w] : v[k];
+            v[k] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+        }
+    }
+}
+
+// Gam or h_prev (fp32, four consecutive n per piece of the thread's share) -> three bf16 pieces
+__device__ __forceinline__ void split_pieces3(const float4 (&v)[8], uint2 (&pc3)[8][3])
+{
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        uint32_t a0[3], a1[3];
+        split3(v[k].x, v[k].y, a0[0], a0[1], a0[2]);
+        split3(v[k].z, v[k].w, a1[0], a1[1], a1[2]);
+#pragma unroll
+        for (int pc = 0; pc < 3; ++pc) pc3[k][pc] = make_uint2(a0[pc], a1[pc]);
+    }
+}
+
+// the thread's share of the three pieces -> the swizzled [p][n] tiles
+__device__ __forceinline__ void store_pieces3(uint8_t (&dst)[3][2 * kSumBox], const uint2 (&pc3)[8][3], int tid)
 {
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
         const int i = tid + k * kGradTcThreads;
         const int pr = i >> 5, n = (i & 31) * 4;
         const uint32_t o = (uint32_t)(n >> 6) * kSumBox + sum_swz(pr, (n & 63) >> 3) + (uint32_t)(n & 7) * 2u;
-        uint32_t a0[3], a1[3];
-        split3(v[k].x, v[k].y, a0[0], a0[1], a0[2]);
-        split3(v[k].z, v[k].w, a1[0], a1[1], a1[2]);
 #pragma unroll
-        for (int pc = 0; pc < 3; ++pc) *reinterpret_cast<uint2 *>(dst[pc] + o) = make_uint2(a0[pc], a1[pc]);
+        for (int pc = 0; pc < 3; ++pc) *reinterpret_cast<uint2 *>(dst[pc] + o) = pc3[k][pc];
     }
 }
 
@@ -789,7 +827,7 @@ __global__ void __launch_bounds__(kGradTcThreads, 2) bwd_chunk_grad_tc_kernel(Bw
             const bool v = r < rows;
             const int64_t rs = v ? r : 0;
             const uint32_t o = sum_swz(r, q);
-            cp_async16(smem_u32(s.u.in.x) + o, xg + rs * p.xrs + 8 * q, v);
+            cp_async16(smem_u32(s.x) + o, xg + rs * p.xrs + 8 * q, v);
             cp_async16(smem_u32(s.dy) + o, yg + rs * p.dyrs + 8 * q, v);
         }
         for (int i = tid; i < kQb * 16; i += kGradTcThreads) {
@@ -802,8 +840,7 @@ __global__ void __launch_bounds__(kGradTcThreads, 2) bwd_chunk_grad_tc_kernel(Bw
         }
     }
     for (int i = tid; i < kQb; i += kGradTcThreads) s.dts[i] = i < rows ? p.dt[((int64_t)bi * p.L + t0 + i) * p.H + h] : 0.0f;
-    // Gam and h_prev of the chunk (fp32); <Gam, h_prev> on the way; Gam's pieces to shared memory,
-    // h_prev's kept in registers until phase 1a has read Gam's
+    // Gam and h_prev of the chunk (fp32); <Gam, h_prev> on the way; Gam's pieces to shared memory
     float4 hv[8];
     {
         const float4 *Gg = reinterpret_cast<const float4 *>(p.ws_g + unit * (int64_t)P * N);
@@ -825,7 +862,9 @@ __global__ void __launch_bounds__(kGradTcThreads, 2) bwd_chunk_grad_tc_kernel(Bw
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
         if (lane == 0) s.part[warp] = part;
-        store_pieces3(s.u.in.gh, gv, tid);
+        uint2 gp[8][3];
+        split_pieces3(gv, gp);
+        store_pieces3(s.u.gh, gp, tid);
     }
     cp_async_wait_all();
     fence_proxy_async_smem();
@@ -840,15 +879,15 @@ __global__ void __launch_bounds__(kGradTcThreads, 2) bwd_chunk_grad_tc_kernel(Bw
     if (tid == 0) {
         // phase 1a
         const uint64_t kC = smem_desc(smem_u32(s.c), 16, 1024), kB = smem_desc(smem_u32(s.b), 16, 1024);
-        const uint64_t kY = smem_desc(smem_u32(s.dy), 16, 1024), kX = smem_desc(smem_u32(s.u.in.x), 16, 1024);
+        const uint64_t kY = smem_desc(smem_u32(s.dy), 16, 1024), kX = smem_desc(smem_u32(s.x), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) mma_ss(tm + kColCG, kC + koff(kk), kB + koff(kk), id64, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColCG + kLane16, kY + koff(kk), kX + koff(kk), id64, kk > 0);
 #pragma unroll
         for (int pc = 0; pc < 3; ++pc) {
-            const uint64_t kG = smem_desc(smem_u32(s.u.in.gh[pc]), 16, 1024);
-            const uint64_t mG = smem_desc(smem_u32(s.u.in.gh[pc]), kSumBox, 1024);
+            const uint64_t kG = smem_desc(smem_u32(s.u.gh[pc]), 16, 1024);
+            const uint64_t mG = smem_desc(smem_u32(s.u.gh[pc]), kSumBox, 1024);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) mma_ss(tm + kColDX, kB + koff(kk), kG + koff(kk), id64, pc > 0 || kk > 0);
 #pragma unroll
@@ -857,24 +896,38 @@ __global__ void __launch_bounds__(kGradTcThreads, 2) bwd_chunk_grad_tc_kernel(Bw
         mma_commit(&s.done1);
         last = &s.done1;
     }
-    if (tid == 32) {
-        float acc = 0.0f;
-        for (int i = 0; i < kQb; ++i) { acc = fmaf(s.dts[i], Ah, acc); s.cum[i] = acc; }
+    // h_prev's pieces, made while phase 1a runs and stored once it has read Gam's
+    uint2 hp[8][3];
+    split_pieces3(hv, hp);
+    if (warp == 1) {
+        // chunk-local inclusive cumsum of dt A: two tokens per lane, then a scan over the lanes
+        const float a0 = s.dts[2 * lane] * Ah, a1 = s.dts[2 * lane + 1] * Ah;
+        float v = a0 + a1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float n = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += n;
+        }
+        float ex = __shfl_up_sync(0xffffffffu, v, 1);
+        ex = lane == 0 ? 0.0f : ex;
+        const float c0 = ex + a0;
+        const float lamw = __shfl_sync(0xffffffffu, v, 31);
+        s.cum[2 * lane] = c0;
+        s.cum[2 * lane + 1] = v;
+        s.ecs[2 * lane] = expf(c0);
+        s.ecs[2 * lane + 1] = expf(v);
+        s.eend[2 * lane] = expf(lamw - c0);
+        s.eend[2 * lane + 1] = expf(lamw - v);
     }
+    if (tid == 0) s.ok = mbar_wait(&s.done1, 0, nullptr, p.wait_limit_ns) ? 1 : 0;
     __syncthreads();
     const float lam = s.cum[kQb - 1];
-    if (tid < kQb) {
-        s.ecs[tid] = expf(s.cum[tid]);
-        s.eend[tid] = expf(lam - s.cum[tid]);
-    }
     float gam_h = 0.0f;
 #pragma unroll
     for (int w = 0; w < kGradTcThreads / 32; ++w) gam_h += s.part[w];
     const float term3 = expf(lam) * gam_h;
-    if (tid == 0) s.ok = mbar_wait(&s.done1, 0, nullptr, p.wait_limit_ns) ? 1 : 0;
-    __syncthreads();
     // phase 1b: h_prev's pieces over Gam's (phase 1a has read them)
-    if (s.ok) store_pieces3(s.u.in.gh, hv, tid);
+    if (s.ok) store_pieces3(s.u.gh, hp, tid);
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0 && s.ok) {
@@ -882,7 +935,7 @@ __global__ void __launch_bounds__(kGradTcThreads, 2) bwd_chunk_grad_tc_kernel(Bw
         const uint64_t kY = smem_desc(smem_u32(s.dy), 16, 1024);
 #pragma unroll
         for (int pc = 0; pc < 3; ++pc) {
-            const uint64_t mH = smem_desc(smem_u32(s.u.in.gh[pc]), kSumBox, 1024);
+            const uint64_t mH = smem_desc(smem_u32(s.u.gh[pc]), kSumBox, 1024);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) mma_ss(tm + kColDC, mH + kk * 128, kY + koff(kk), id128, pc > 0 || kk > 0);
         }
@@ -895,60 +948,77 @@ __global__ void __launch_bounds__(kGradTcThreads, 2) bwd_chunk_grad_tc_kernel(Bw
     if (ok1) {
         tc_fence_after();
         if (warp < 4) {
-            // row t of CB (lanes 0..15) and of GX (lanes 16..31); after one exchange lanes 0..15
-            // hold columns j = 0..31 of both and lanes 16..31 columns 32..63
+            // row t of CB (lanes 0..15) and of GX (lanes 16..31), 16 columns at a time: after one
+            // exchange lanes 0..15 hold columns j = 16 g .. 16 g + 15 of both, lanes 16..31 the
+            // same columns of the upper half (32 + 16 g ..)
             const int q = warp, hi = lane >> 4, t = 16 * q + (lane & 15);
             const uint32_t lb = (uint32_t)(32 * q) << 16;
-            float cbk[32], gxk[32];
-            {
-                uint32_t v0[32], v1[32];
-                tmem_ld32(tm + kColCG + lb, v0);
-                tmem_ld32(tm + kColCG + lb + 32, v1);
-                tmem_wait_ld(v0);
-                tmem_wait_ld(v1);
-#pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    const uint32_t send = hi ? v0[k] : v1[k];
-                    const float keep = __uint_as_float(hi ? v1[k] : v0[k]);
-                    const float recv = __uint_as_float(__shfl_xor_sync(0xffffffffu, send, 16));
-                    cbk[k] = hi ? recv : keep;
-                    gxk[k] = hi ? keep : recv;
-                }
-            }
             const float cum_t = s.cum[t];
-            float *kprow = s.u.mid.kp + t * kQb;
-            float run = 0.0f, dd = 0.0f;
+            float run = 0.0f, dd = 0.0f;     // run: sum of K[t][j'] over this half's columns so far
+#pragma unroll 1
+            for (int g = 0; g < 2; ++g) {
+                float cbv[16], gxv[16];
+                {
+                    uint32_t a[16], b[16];
+                    tmem_ld16(tm + kColCG + lb + 16 * g, a);
+                    tmem_ld16(tm + kColCG + lb + 32 + 16 * g, b);
+                    tmem_wait_ld(a, b);
 #pragma unroll
-            for (int k8 = 0; k8 < 4; ++k8) {
-                uint32_t ch[4], cl[4], xh[4], xl[4], dh[4], dl[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float cm[2], xm[2], dm[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int k = 8 * k8 + 2 * e + u, j = 32 * hi + k;
-                        const float seg = j <= t ? expf(cum_t - s.cum[j]) : 0.0f;
-                        const float gxm = seg * gxk[k], gd = gxm * s.dts[j];
-                        cm[u] = seg * cbk[k];
-                        xm[u] = gxm;
-                        dm[u] = gd;
-                        kprow[(j + t) & (kQb - 1)] = run;
-                        run += j < t ? gd * cbk[k] : 0.0f;
-                        if (j == t) dd = gxk[k];
+                    for (int k = 0; k < 16; ++k) {
+                        const uint32_t send = hi ? a[k] : b[k];
+                        const float keep = __uint_as_float(hi ? b[k] : a[k]);
+                        const float recv = __uint_as_float(__shfl_xor_sync(0xffffffffu, send, 16));
+                        cbv[k] = hi ? recv : keep;
+                        gxv[k] = hi ? keep : recv;
                     }
-                    split2(cm[0], cm[1], ch[e], cl[e]);
-                    split2(xm[0], xm[1], xh[e], xl[e]);
-                    split2(dm[0], dm[1], dh[e], dl[e]);
                 }
-                const uint32_t o = sum_swz(t, 4 * hi + k8);
-                *reinterpret_cast<uint4 *>(s.u.mid.cb[0] + o) = make_uint4(ch[0], ch[1], ch[2], ch[3]);
-                *reinterpret_cast<uint4 *>(s.u.mid.cb[1] + o) = make_uint4(cl[0], cl[1], cl[2], cl[3]);
-                *reinterpret_cast<uint4 *>(s.u.mid.gx[0] + o) = make_uint4(xh[0], xh[1], xh[2], xh[3]);
-                *reinterpret_cast<uint4 *>(s.u.mid.gx[1] + o) = make_uint4(xl[0], xl[1], xl[2], xl[3]);
-                *reinterpret_cast<uint4 *>(s.u.mid.gd[0] + o) = make_uint4(dh[0], dh[1], dh[2], dh[3]);
-                *reinterpret_cast<uint4 *>(s.u.mid.gd[1] + o) = make_uint4(dl[0], dl[1], dl[2], dl[3]);
+                const int jb = 32 * hi + 16 * g;
+#pragma unroll
+                for (int k8 = 0; k8 < 2; ++k8) {
+                    const float4 c4a = *reinterpret_cast<const float4 *>(s.cum + jb + 8 * k8);
+                    const float4 c4b = *reinterpret_cast<const float4 *>(s.cum + jb + 8 * k8 + 4);
+                    const float4 d4a = *reinterpret_cast<const float4 *>(s.dts + jb + 8 * k8);
+                    const float4 d4b = *reinterpret_cast<const float4 *>(s.dts + jb + 8 * k8 + 4);
+                    const float cj[8] = {c4a.x, c4a.y, c4a.z, c4a.w, c4b.x, c4b.y, c4b.z, c4b.w};
+                    const float dj[8] = {d4a.x, d4a.y, d4a.z, d4a.w, d4b.x, d4b.y, d4b.z, d4b.w};
+                    uint32_t ch[4], cl[4], xh[4], xl[4], dh[4], dl[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float cm[2], xm[2], dm[2];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int k = 8 * k8 + 2 * e + u, j = jb + k;
+                            const float ex = exp2_approx(fminf(cum_t - cj[2 * e + u], 0.0f) * kLog2e);
+                            const float seg = j <= t ? ex : 0.0f;
+                            const float cb = cbv[k], gx = gxv[k];
+                            const float gxm = seg * gx, gd = gxm * dj[2 * e + u];
+                            cm[u] = seg * cb;
+                            xm[u] = gxm;
+                            dm[u] = gd;
+                            cbv[k] = t >= j ? run : 0.0f;    // this half's part of sum_{j' < j} K[t][j'], rows t >= j
+                            gxv[k] = gxm * cb;               // GXm[t][j] CB[t][j], for B_j . dBr_j
+                            run += j < t ? gd * cb : 0.0f;
+                            dd = j == t ? gx : dd;
+                        }
+                        split2(cm[0], cm[1], ch[e], cl[e]);
+                        split2(xm[0], xm[1], xh[e], xl[e]);
+                        split2(dm[0], dm[1], dh[e], dl[e]);
+                    }
+                    const uint32_t o = sum_swz(t, (jb >> 3) + k8);
+                    *reinterpret_cast<uint4 *>(s.u.mid.cb[0] + o) = make_uint4(ch[0], ch[1], ch[2], ch[3]);
+                    *reinterpret_cast<uint4 *>(s.u.mid.cb[1] + o) = make_uint4(cl[0], cl[1], cl[2], cl[3]);
+                    *reinterpret_cast<uint4 *>(s.u.mid.gx[0] + o) = make_uint4(xh[0], xh[1], xh[2], xh[3]);
+                    *reinterpret_cast<uint4 *>(s.u.mid.gx[1] + o) = make_uint4(xl[0], xl[1], xl[2], xl[3]);
+                    *reinterpret_cast<uint4 *>(s.u.mid.gd[0] + o) = make_uint4(dh[0], dh[1], dh[2], dh[3]);
+                    *reinterpret_cast<uint4 *>(s.u.mid.gd[1] + o) = make_uint4(dl[0], dl[1], dl[2], dl[3]);
+                }
+                // column sums over this warp's 16 rows: lane l of each half gets column jb + l
+                half_warp_sum16(cbv, lane);
+                half_warp_sum16(gxv, lane);
+                s.rrp[q][jb + (lane & 15)] = cbv[0];
+                s.rdin[q][jb + (lane & 15)] = gxv[0];
             }
-            if (!hi) s.rowoff[t] = run;
+            if (!hi) s.rowoff[t] = run;      // sum_{j < 32} K[t][j], added to the upper half's columns below
             // dD of the chunk: the diagonal of GX (decay 1 there)
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) dd += __shfl_xor_sync(0xffffffffu, dd, o);
@@ -957,15 +1027,10 @@ __global__ void __launch_bounds__(kGradTcThreads, 2) bwd_chunk_grad_tc_kernel(Bw
             const int q = warp - 4;
             const uint32_t lb = (uint32_t)(32 * q) << 16;
             {
-                // dx accumulator, row j in lanes 0..15: be_j = e^{lam - cs_j} dt_j x_j . dxI_j (x from
-                // global memory: its tile is gone), then dxI *= e^{lam - cs_j}
+                // dx accumulator, row j in lanes 0..15: be_j = e^{lam - cs_j} dt_j x_j . dxI_j,
+                // then dxI *= e^{lam - cs_j}
                 const int j = 16 * q + (lane & 15);
                 const float ej = s.eend[j];
-                uint4 xv[8];
-#pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8)
-                    xv[c8] = j < rows ? *reinterpret_cast<const uint4 *>(xg + (int64_t)j * p.xrs + 8 * c8)
-                                      : make_uint4(0u, 0u, 0u, 0u);
                 float sbe = 0.0f;
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
@@ -974,8 +1039,8 @@ __global__ void __launch_bounds__(kGradTcThreads, 2) bwd_chunk_grad_tc_kernel(Bw
                     tmem_wait_ld(v);
 #pragma unroll
                     for (int k8 = 0; k8 < 4; ++k8) {
-                        const uint32_t xw[4] = {xv[4 * hf + k8].x, xv[4 * hf + k8].y, xv[4 * hf + k8].z,
-                                                xv[4 * hf + k8].w};
+                        const uint4 xv = *reinterpret_cast<const uint4 *>(s.x + sum_swz(j, 4 * hf + k8));
+                        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             sbe = fmaf(bf16_lo(xw[e]), __uint_as_float(v[8 * k8 + 2 * e]), sbe);
@@ -986,7 +1051,10 @@ __global__ void __launch_bounds__(kGradTcThreads, 2) bwd_chunk_grad_tc_kernel(Bw
                     for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * ej);
                     tmem_st32(tm + kColDX + lb + 32 * hf, v);
                 }
-                if (lane < 16) s.be[j] = ej * s.dts[j] * sbe;
+                if (lane < 16) {
+                    s.sbe[j] = ej * sbe;       // e^{lam - cs_j} x_j^T Gam B_j
+                    s.be[j] = ej * s.dts[j] * sbe;
+                }
             }
             {
                 // dC^T[n][t] = h_prev[.][n] . dy_t: C_t[n] dC^T[n][t] summed over n gives al_t / e^{cs_t};
@@ -1008,8 +1076,8 @@ __global__ void __launch_bounds__(kGradTcThreads, 2) bwd_chunk_grad_tc_kernel(Bw
                     tmem_st32(tm + kColDC + lb + 32 * hf, v);
                 }
                 warp_sum64(pr, lane);
-                s.red[q][2 * lane] = pr[0];
-                s.red[q][2 * lane + 1] = pr[1];
+                s.ral[q][2 * lane] = pr[0];
+                s.ral[q][2 * lane + 1] = pr[1];
             }
             // dBr^T[n][j] *= e^{lam - cs_j}
 #pragma unroll
@@ -1048,21 +1116,47 @@ __global__ void __launch_bounds__(kGradTcThreads, 2) bwd_chunk_grad_tc_kernel(Bw
         mma_commit(&s.done2);
         last = &s.done2;
     }
-    if (ok1 && tid < kQb) {
-        // dl_t without the B_t . dBr_t term: sum_{u>=t} al_u + sum_{t'>=t} sum_{j<t} K[t'][j]
-        //   + e^{lam} <Gam, h_prev> + sum_{j<t} be_j
-        const int t = tid;
-        const bool upper = t >= 32;
-        float rr = 0.0f, suf = 0.0f, pre = 0.0f;
-        for (int u = t; u < kQb; ++u) {
-            rr += s.u.mid.kp[u * kQb + ((t + u) & (kQb - 1))] + (upper ? s.rowoff[u] : 0.0f);
-            suf += s.ecs[u] * (s.red[0][u] + s.red[1][u] + s.red[2][u] + s.red[3][u]);
+    if (ok1 && warp == 1) {
+        // while phase 2 runs, tokens t = 2 lane, 2 lane + 1:
+        //   dl_t = sum_{u>=t} al_u + sum_{t'>=t} sum_{j<t} K[t'][j] + e^{lam} <Gam, h_prev> + sum_{j<t} be_j
+        //   ddt_t = A dl_t + B_t . dBr_t, and this chunk's share of dA = sum_t dt_t dl_t, with
+        //   B_j . dBr_j = sum_t GXm[t][j] CB[t][j] + e^{lam - cs_j} x_j^T Gam B_j
+        const int ta = 2 * lane, tb = ta + 1;
+        auto qsum = [](const float (&r)[4][kQb], int t) { return r[0][t] + r[1][t] + r[2][t] + r[3][t]; };
+        const float ala = s.ecs[ta] * qsum(s.ral, ta), alb = s.ecs[tb] * qsum(s.ral, tb);
+        float suf = ala + alb, pre = s.be[ta] + s.be[tb];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float sn = __shfl_down_sync(0xffffffffu, suf, o), pn = __shfl_up_sync(0xffffffffu, pre, o);
+            if (lane + o < 32) suf += sn;
+            if (lane >= o) pre += pn;
         }
-        for (int j = 0; j < t; ++j) pre += s.be[j];
-        s.dl0[t] = suf + rr + term3 + pre;
+        float sufn = __shfl_down_sync(0xffffffffu, suf, 1), pren = __shfl_up_sync(0xffffffffu, pre, 1);
+        sufn = lane == 31 ? 0.0f : sufn;           // sum of al over the later lanes
+        pren = lane == 0 ? 0.0f : pren;            // sum of be over the earlier lanes
+        // columns t >= 32 add sum_{t' >= t} sum_{j < 32} K[t'][j]
+        const float roa = s.rowoff[ta], rob = s.rowoff[tb];
+        float ros = roa + rob;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float n = __shfl_down_sync(0xffffffffu, ros, o);
+            if (lane + o < 32) ros += n;
+        }
+        float rosn = __shfl_down_sync(0xffffffffu, ros, 1);
+        rosn = lane == 31 ? 0.0f : rosn;
+        const float rra = qsum(s.rrp, ta) + (ta >= 32 ? roa + rob + rosn : 0.0f);
+        const float rrb = qsum(s.rrp, tb) + (tb >= 32 ? rob + rosn : 0.0f);
+        const float dlb = (alb + sufn) + rrb + term3 + (pren + s.be[ta]);
+        const float dla = (ala + alb + sufn) + rra + term3 + pren;
+        const float dina = qsum(s.rdin, ta) + s.sbe[ta], dinb = qsum(s.rdin, tb) + s.sbe[tb];
+        if (ta < rows) p.ddt[((int64_t)bi * p.L + t0 + ta) * p.H + h] = fmaf(Ah, dla, dina);
+        if (tb < rows) p.ddt[((int64_t)bi * p.L + t0 + tb) * p.H + h] = fmaf(Ah, dlb, dinb);
+        float a = fmaf(s.dts[ta], dla, s.dts[tb] * dlb);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        if (lane == 0) p.ws_pA[unit] = a;
     }
     if (ok1 && tid == kQb) p.ws_pD[unit] = s.pdd[0] + s.pdd[1] + s.pdd[2] + s.pdd[3];
-    __syncthreads();   // red is read before E2 writes it again
     if (tid == 0) s.ok = ok1 && mbar_wait(&s.done2, 0, nullptr, p.wait_limit_ns) ? 1 : 0;
     __syncthreads();
     const bool ok2 = s.ok != 0;
@@ -1070,11 +1164,10 @@ __global__ void __launch_bounds__(kGradTcThreads, 2) bwd_chunk_grad_tc_kernel(Bw
         tc_fence_after();
         const int64_t rstride = (int64_t)p.H * N;    // floats between tokens of dBh and dCh
         if (warp < 4) {
-            // dBr^T[n][j]: dB_j = dt_j dBr_j (per head), and B_j . dBr_j summed over n
+            // dBr^T[n][j]: dB_j = dt_j dBr_j (per head)
             const int q = warp, n = 32 * q + lane;
             const uint32_t lb = (uint32_t)(32 * q) << 16;
             float *dBh = p.ws_dBh + (((int64_t)bi * p.L + t0) * p.H + h) * N + n;
-            float pr[kQb];
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 uint32_t v[32];
@@ -1083,14 +1176,9 @@ __global__ void __launch_bounds__(kGradTcThreads, 2) bwd_chunk_grad_tc_kernel(Bw
 #pragma unroll
                 for (int k = 0; k < 32; ++k) {
                     const int j = 32 * hf + k;
-                    const float br = __uint_as_float(v[k]);
-                    if (j < rows) dBh[j * rstride] = s.dts[j] * br;
-                    pr[j] = tile_at(s.b, j, n) * br;
+                    if (j < rows) dBh[j * rstride] = s.dts[j] * __uint_as_float(v[k]);
                 }
             }
-            warp_sum64(pr, lane);
-            s.red[q][2 * lane] = pr[0];
-            s.red[q][2 * lane + 1] = pr[1];
         } else {
             const int q = warp - 4, n = 32 * q + lane;
             const uint32_t lb = (uint32_t)(32 * q) << 16;
@@ -1136,20 +1224,6 @@ __global__ void __launch_bounds__(kGradTcThreads, 2) bwd_chunk_grad_tc_kernel(Bw
             }
         }
     }
-    __syncthreads();
-    if (ok2 && tid < kQb) {
-        // dl_t, ddt_t = A dl_t + B_t . dBr_t, and this chunk's share of dA
-        const int t = tid;
-        const float din = s.red[0][t] + s.red[1][t] + s.red[2][t] + s.red[3][t];
-        const float dl = s.dl0[t];
-        if (t < rows) p.ddt[((int64_t)bi * p.L + t0 + t) * p.H + h] = fmaf(Ah, dl, din);
-        float a = s.dts[t] * dl;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-        if (lane == 0) s.pa[warp] = a;
-    }
-    __syncthreads();
-    if (ok2 && tid == 0) p.ws_pA[unit] = s.pa[0] + s.pa[1];
     if (tid == 0 && !ok2) {
         // a bounded wait gave up: report it, and let the products in flight finish before TMEM is freed
         atomicOr(p.status, kDevTimeout);
