@@ -1124,26 +1124,21 @@ __global__ void __launch_bounds__(kGradTcThreads, 2) bwd_chunk_grad_tc_kernel(Bw
         const int ta = 2 * lane, tb = ta + 1;
         auto qsum = [](const float (&r)[4][kQb], int t) { return r[0][t] + r[1][t] + r[2][t] + r[3][t]; };
         const float ala = s.ecs[ta] * qsum(s.ral, ta), alb = s.ecs[tb] * qsum(s.ral, tb);
-        float suf = ala + alb, pre = s.be[ta] + s.be[tb];
+        // columns t >= 32 also add sum_{t' >= t} sum_{j < 32} K[t'][j]
+        const float roa = s.rowoff[ta], rob = s.rowoff[tb];
+        float suf = ala + alb, pre = s.be[ta] + s.be[tb], ros = roa + rob;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const float sn = __shfl_down_sync(0xffffffffu, suf, o), pn = __shfl_up_sync(0xffffffffu, pre, o);
-            if (lane + o < 32) suf += sn;
+            const float rn = __shfl_down_sync(0xffffffffu, ros, o);
+            if (lane + o < 32) { suf += sn; ros += rn; }
             if (lane >= o) pre += pn;
         }
         float sufn = __shfl_down_sync(0xffffffffu, suf, 1), pren = __shfl_up_sync(0xffffffffu, pre, 1);
-        sufn = lane == 31 ? 0.0f : sufn;           // sum of al over the later lanes
-        pren = lane == 0 ? 0.0f : pren;            // sum of be over the earlier lanes
-        // columns t >= 32 add sum_{t' >= t} sum_{j < 32} K[t'][j]
-        const float roa = s.rowoff[ta], rob = s.rowoff[tb];
-        float ros = roa + rob;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float n = __shfl_down_sync(0xffffffffu, ros, o);
-            if (lane + o < 32) ros += n;
-        }
         float rosn = __shfl_down_sync(0xffffffffu, ros, 1);
+        sufn = lane == 31 ? 0.0f : sufn;           // sum of al over the later lanes
         rosn = lane == 31 ? 0.0f : rosn;
+        pren = lane == 0 ? 0.0f : pren;            // sum of be over the earlier lanes
         const float rra = qsum(s.rrp, ta) + (ta >= 32 ? roa + rob + rosn : 0.0f);
         const float rrb = qsum(s.rrp, tb) + (tb >= 32 ? rob + rosn : 0.0f);
         const float dlb = (alb + sufn) + rrb + term3 + (pren + s.be[ta]);
@@ -1195,31 +1190,32 @@ __global__ void __launch_bounds__(kGradTcThreads, 2) bwd_chunk_grad_tc_kernel(Bw
                     if (t < rows) dCh[t * rstride] = __uint_as_float(v[k]);
                 }
             }
-            // dx_j = D dy_j + dt_j (dx accumulator row j, lanes 0..15)
+        }
+        {
+            // dx_j = D dy_j + dt_j (dx accumulator row j, lanes 0..15); each team takes 32 of the p columns
+            const int q = warp & 3, hf = warp >> 2;
+            const uint32_t lb = (uint32_t)(32 * q) << 16;
             const int j = 16 * q + (lane & 15);
             const bool act = lane < 16 && j < rows;
             float *dxr = p.dx + ((int64_t)bi * p.L + t0 + j) * p.H * P + (int64_t)h * P;
             const float dtj = s.dts[j];
+            uint32_t v[32];
+            tmem_ld32(tm + kColDX + lb + 32 * hf, v);
+            tmem_wait_ld(v);
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                uint32_t v[32];
-                tmem_ld32(tm + kColDX + lb + 32 * hf, v);
-                tmem_wait_ld(v);
+            for (int k8 = 0; k8 < 4; ++k8) {
+                const uint4 yv = *reinterpret_cast<const uint4 *>(s.dy + sum_swz(j, 4 * hf + k8));
+                const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
+                float o[8];
 #pragma unroll
-                for (int k8 = 0; k8 < 4; ++k8) {
-                    const uint4 yv = *reinterpret_cast<const uint4 *>(s.dy + sum_swz(j, 4 * hf + k8));
-                    const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
-                    float o[8];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        o[2 * e] = fmaf(Dh, bf16_lo(yw[e]), dtj * __uint_as_float(v[8 * k8 + 2 * e]));
-                        o[2 * e + 1] = fmaf(Dh, bf16_hi(yw[e]), dtj * __uint_as_float(v[8 * k8 + 2 * e + 1]));
-                    }
-                    if (act) {
-                        float4 *d4 = reinterpret_cast<float4 *>(dxr + 32 * hf + 8 * k8);
-                        d4[0] = make_float4(o[0], o[1], o[2], o[3]);
-                        d4[1] = make_float4(o[4], o[5], o[6], o[7]);
-                    }
+                for (int e = 0; e < 4; ++e) {
+                    o[2 * e] = fmaf(Dh, bf16_lo(yw[e]), dtj * __uint_as_float(v[8 * k8 + 2 * e]));
+                    o[2 * e + 1] = fmaf(Dh, bf16_hi(yw[e]), dtj * __uint_as_float(v[8 * k8 + 2 * e + 1]));
+                }
+                if (act) {
+                    float4 *d4 = reinterpret_cast<float4 *>(dxr + 32 * hf + 8 * k8);
+                    d4[0] = make_float4(o[0], o[1], o[2], o[3]);
+                    d4[1] = make_float4(o[4], o[5], o[6], o[7]);
                 }
             }
         }
