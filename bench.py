@@ -609,8 +609,10 @@ def bwd_grad_roofline(wl, ms_per_launch):
         alg = bwd_grad_bytes_per_chunk_head(wl) * units
         achieved = alg / (ms_per_launch / 1e3) / 1e9
         tflops = bwd_grad_mma_flops_per_chunk_head(wl.P, wl.N) * units / (ms_per_launch / 1e3) / 1e12
+        traffic_pt = recorded_traffic("bwd_chunk_grad_tc")
         return {"bound": "hbm", "kernel": "bwd_chunk_grad_tc", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "peak_source": peak_src, "traffic": None,
+                "frac": achieved / peak, "peak_source": peak_src,
+                "traffic": None if traffic_pt is None else traffic_pt * wl.L * wl.b,
                 "algorithmic_bytes_per_launch": alg, "tensor_achieved_tflops": tflops,
                 "tensor_peak_tflops": tpeak, "tensor_frac": tflops / tpeak, "tensor_peak_source": tpeak_src,
                 "tensor_flops": "issued dense bf16 MMA flops of the kernel"}
