@@ -31,7 +31,9 @@ def _check(got, ref, dtype):
 
 
 @pytest.mark.parametrize("dtype,d,group,rows", [
-    (torch.bfloat16, 2048, 0, 2000),      # the 0.3B d_inner, one group
+    (torch.bfloat16, 2048, 0, 2000),      # the 0.3B d_inner, one group (a warp per row)
+    (torch.bfloat16, 2048, 512, 999),     # four groups of 512, a warp per row
+    (torch.bfloat16, 768, 256, 333),      # three chunks of 256, a warp per row
     (torch.bfloat16, 5120, 640, 300),     # the 2.7B d_inner, eight groups
     (torch.float32, 256, 64, 777),
     (torch.float32, 8, 8, 5),
