@@ -368,22 +368,34 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_adjoint_chain_kernel(BwdParam
                            : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     float *base = p.ws_g + hu * p.nch * PN + e;
     const float *lam = p.ws_lam + hu * p.nch;
-    for (int64_t cb = p.nch - 1; cb >= 0; cb -= kChainAhead) {
-        float4 sv[kChainAhead];
-        float lv[kChainAhead];
+    // two halves of kChainAhead chunks in turn: the loads of one half are in flight while the
+    // other half's steps run
+    constexpr int kHalf = kChainAhead / 2;
+    float4 sa[kHalf], sb[kHalf];
+    float la[kHalf], lb[kHalf];
+    auto load = [&](int64_t c, float4 (&sv)[kHalf], float (&lv)[kHalf]) {
 #pragma unroll
-        for (int i = 0; i < kChainAhead; ++i) {
-            const bool in = cb - i >= 0;
-            sv[i] = in ? *reinterpret_cast<const float4 *>(base + (cb - i) * PN) : make_float4(0.f, 0.f, 0.f, 0.f);
-            lv[i] = in ? lam[cb - i] : 0.0f;
+        for (int i = 0; i < kHalf; ++i) {
+            const bool in = c - i >= 0;
+            sv[i] = in ? *reinterpret_cast<const float4 *>(base + (c - i) * PN) : make_float4(0.f, 0.f, 0.f, 0.f);
+            lv[i] = in ? lam[c - i] : 0.0f;
         }
+    };
+    auto steps = [&](int64_t c, const float4 (&sv)[kHalf], const float (&lv)[kHalf]) {
 #pragma unroll
-        for (int i = 0; i < kChainAhead; ++i) {
-            if (cb - i >= 0) {
-                *reinterpret_cast<float4 *>(base + (cb - i) * PN) = gv;
+        for (int i = 0; i < kHalf; ++i) {
+            if (c - i >= 0) {
+                *reinterpret_cast<float4 *>(base + (c - i) * PN) = gv;
                 gv = f4_fma(expf(lv[i]), gv, sv[i]);
             }
         }
+    };
+    load(p.nch - 1, sa, la);
+    for (int64_t cb = p.nch - 1; cb >= 0; cb -= 2 * kHalf) {
+        load(cb - kHalf, sb, lb);
+        steps(cb, sa, la);
+        load(cb - 2 * kHalf, sa, la);
+        steps(cb - kHalf, sb, lb);
     }
     if (p.dh0) *reinterpret_cast<float4 *>(p.dh0 + hu * PN + e) = gv;
 }
@@ -1329,8 +1341,10 @@ int launch_bwd_t(BwdParams p, cudaStream_t st)
     const int64_t cells = (p.nch + p.cell_chunks - 1) / p.cell_chunks;
     prof_begin(st, kKBwdChain);
     bwd_state_chain_kernel<<<dim3(slices * (unsigned)cells, (unsigned)p.H, (unsigned)p.b), kBwdThreads, 0, st>>>(p);
-    bwd_adjoint_chain_kernel<<<dim3(slices, (unsigned)p.H, (unsigned)p.b), kBwdThreads, 0, st>>>(p);
     prof_end(st, kKBwdChain);
+    prof_begin(st, kKBwdAdjoint);
+    bwd_adjoint_chain_kernel<<<dim3(slices, (unsigned)p.H, (unsigned)p.b), kBwdThreads, 0, st>>>(p);
+    prof_end(st, kKBwdAdjoint);
     prof_begin(st, kKBwdGrad);
     if (tc_summary) bwd_chunk_grad_tc_kernel<<<grid, kGradTcThreads, s_gt, st>>>(p);
     else bwd_chunk_grad_kernel<T><<<grid, kGradThreads, s2, st>>>(p);

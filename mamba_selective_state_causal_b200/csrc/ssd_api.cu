@@ -518,8 +518,8 @@ int conv_impl(const void *u, int64_t ubs, int64_t urs, const float *w, const flo
 // ---------------------------------------------------------------- kernel timing
 const char *const kKernelNames[ssd::kKCount] = {
     "conv1d_silu", "conv_tail", "stripe_state_tc", "stripe_chain", "chunk_output_tc",
-    "stripe_state_generic", "chunk_output_generic", "decode_step", "bwd_chunk_summary", "bwd_chains",
-    "bwd_chunk_grad", "bwd_reduce", "gated_rmsnorm", "conv_cells", "conv_ckpt", "conv_bwd"};
+    "stripe_state_generic", "chunk_output_generic", "decode_step", "bwd_chunk_summary", "bwd_state_chain",
+    "bwd_chunk_grad", "bwd_reduce", "gated_rmsnorm", "conv_cells", "conv_ckpt", "conv_bwd", "bwd_adjoint_chain"};
 
 struct ProfRecord {
     int id;

@@ -223,7 +223,7 @@ __device__ __forceinline__ float cell_val(const ConvBwdParams &p, int64_t bi, in
 enum KernelId : int {
     kKConv = 0, kKConvTail, kKStateTc, kKChain, kKOutputTc, kKStateGeneric, kKOutputGeneric, kKDecode,
     kKBwdSummary, kKBwdChain, kKBwdGrad, kKBwdReduce, kKGatedNorm, kKConvCells, kKConvCkpt, kKConvBwd,
-    kKCount
+    kKBwdAdjoint, kKCount
 };
 void prof_begin(cudaStream_t st, int id);
 void prof_end(cudaStream_t st, int id);
