@@ -314,7 +314,8 @@ constexpr int kChainAhead = 16;   // chunk summaries loaded ahead of the chain
 // checkpoint before it); for each chunk c of the cell: slot c := h, then
 // h = e^{lam_c} h + S_c (the slot held S_c).  Grid: (slices * cells, H, b);
 // a thread carries 4 consecutive state elements.
-__global__ void __launch_bounds__(kBwdThreads) bwd_state_chain_kernel(BwdParams p)
+// (three CTAs per SM: at one, set by its registers, too few loads were in flight)
+__global__ void __launch_bounds__(kBwdThreads, 3) bwd_state_chain_kernel(BwdParams p)
 {
     const int64_t PN = (int64_t)p.P * p.N;
     const int slices = (int)((PN + 4 * kBwdThreads - 1) / (4 * kBwdThreads));
