@@ -140,20 +140,192 @@ __global__ void __launch_bounds__(kConvBwdThreads, 4) conv_bwd_kernel(ConvBwdPar
     }
 }
 
-// dw and dbias: the partial sums of every (batch row, token block), added in a fixed order
-__global__ void conv_bwd_reduce_kernel(ConvBwdParams p, int64_t nparts)
+// ---- two consecutive channels per thread (8-byte loads of dv and stores of du, 4 bytes of bf16 u)
+__device__ __forceinline__ float2 ld2(const float *q) { return *reinterpret_cast<const float2 *>(q); }
+__device__ __forceinline__ float2 ld2(const __nv_bfloat16 *q)
 {
-    const int c = blockIdx.x * blockDim.x + threadIdx.x;
-    if (c >= p.C_ch) return;
+    const uint32_t v = *reinterpret_cast<const uint32_t *>(q);
+    return make_float2(bf16_lo(v), bf16_hi(v));
+}
+
+// dLoss/dv of channels c, c+1 (both in one of x, B, C) at row (bi, t)
+__device__ __forceinline__ float2 dv2_at(const ConvBwdParams &p, int64_t bi, int64_t t, int c)
+{
+    const int64_t row = bi * p.L + t;
+    if (c < p.HP) return ld2(p.dx + row * p.HP + c);
+    if (c < p.HP + p.GN) return ld2(p.dB + row * p.GN + (c - p.HP));
+    return ld2(p.dC + row * p.GN + (c - p.HP - p.GN));
+}
+
+// cell_val of channels c, c+1 at position tt, for a token of cell k (which starts at `start`)
+template <typename T>
+__device__ __forceinline__ float2 cell2k(const ConvBwdParams &p, int64_t bi, int64_t k, int64_t start, int64_t tt, int c)
+{
+    if (tt >= start) return ld2(reinterpret_cast<const T *>(p.u) + bi * p.ubs + tt * p.urs + c);
+    const int64_t r = tt - start + 3;
+    if (k == 0)
+        return p.tail_in ? ld2(reinterpret_cast<const T *>(p.tail_in) + (bi * 3 + r) * p.C_ch + c)
+                         : make_float2(0.0f, 0.0f);
+    return ld2(reinterpret_cast<const T *>(p.conv_ckpt) + ((bi * p.n_ckpt + (k - 1)) * 3 + r) * p.C_ch + c);
+}
+
+// cell_val of channels c, c+1 for token t
+template <typename T>
+__device__ __forceinline__ float2 cell2(const ConvBwdParams &p, int64_t bi, int64_t t, int64_t tt, int c)
+{
+    const int64_t k = p.conv_ckpt ? t / p.s : 0;
+    return cell2k<T>(p, bi, k, p.conv_ckpt ? k * p.s : 0, tt, c);
+}
+
+template <typename T>
+__device__ __forceinline__ float2 dz2_at(const ConvBwdParams &p, int64_t bi, int64_t t, int c, const float4 (&wq)[2],
+                                         const float2 &bs)
+{
+    if (t >= p.L) return make_float2(0.0f, 0.0f);
+    float2 uw[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) uw[k] = cell2<T>(p, bi, t, t - 3 + k, c);
+    const float2 dv = dv2_at(p, bi, t, c);
+    const float wa[4] = {uw[0].x, uw[1].x, uw[2].x, uw[3].x}, wb[4] = {uw[0].y, uw[1].y, uw[2].y, uw[3].y};
+    return make_float2(dz_of(dv.x, wq[0], bs.x, wa), dz_of(dv.y, wq[1], bs.y, wb));
+}
+
+// The same walk as conv_bwd_kernel with two consecutive channels per thread (one thread per
+// (batch row, block of kTB tokens, channel pair), consecutive threads on consecutive pairs) and
+// eight tokens' loads issued before their arithmetic.  two CTAs per SM (at most 128 registers)
+constexpr int kAhead2 = 8;
+template <typename T>
+__global__ void __launch_bounds__(kConvBwdThreads, 2) conv_bwd2_kernel(ConvBwdParams p, int64_t nblk)
+{
+    const int np = p.C_ch >> 1;
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= (int64_t)p.b * nblk * np) return;
+    const int c = 2 * (int)(gid % np);
+    const int64_t blk = (gid / np) % nblk;
+    const int64_t bi = gid / ((int64_t)np * nblk);
+    const int64_t t0 = blk * kTB;
+    const int64_t t1 = min(p.L, t0 + kTB);
+    float4 wq[2];
+    wq[0] = __ldg(reinterpret_cast<const float4 *>(p.w) + c);
+    wq[1] = __ldg(reinterpret_cast<const float4 *>(p.w) + c + 1);
+    const float2 bs = p.bias ? make_float2(__ldg(p.bias + c), __ldg(p.bias + c + 1)) : make_float2(0.0f, 0.0f);
+    // window of dz at t'+0 .. t'+3, walked from t' = t1-1 down to t0
+    float2 d1 = dz2_at<T>(p, bi, t1, c, wq, bs), d2 = dz2_at<T>(p, bi, t1 + 1, c, wq, bs),
+           d3 = dz2_at<T>(p, bi, t1 + 2, c, wq, bs);
+    float2 gw[4] = {}, gb = make_float2(0.0f, 0.0f);
+    // the block's tokens are all in one cell (blocks and cells are multiples of 64 tokens)
+    const int64_t kc = p.conv_ckpt ? t0 / p.s : 0;
+    const int64_t cstart = p.conv_ckpt ? kc * p.s : 0;
+    float2 uw[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) uw[k] = cell2k<T>(p, bi, kc, cstart, t1 - 4 + k, c);
+    for (int64_t tg = t1 - 1; tg >= t0; tg -= kAhead2) {
+        float2 dvv[kAhead2], un[kAhead2];
+#pragma unroll
+        for (int i = 0; i < kAhead2; ++i) {
+            const int64_t t = tg - i;
+            dvv[i] = t >= t0 ? dv2_at(p, bi, t, c) : make_float2(0.0f, 0.0f);
+            un[i] = t > t0 ? cell2k<T>(p, bi, kc, cstart, t - 4, c) : make_float2(0.0f, 0.0f);
+        }
+#pragma unroll
+        for (int i = 0; i < kAhead2; ++i) {
+            const int64_t t = tg - i;
+            if (t < t0) break;
+            const float wa[4] = {uw[0].x, uw[1].x, uw[2].x, uw[3].x}, wb[4] = {uw[0].y, uw[1].y, uw[2].y, uw[3].y};
+            const float2 d0 = make_float2(dz_of(dvv[i].x, wq[0], bs.x, wa), dz_of(dvv[i].y, wq[1], bs.y, wb));
+            float2 g;
+            g.x = fmaf(wq[0].x, d3.x, fmaf(wq[0].y, d2.x, fmaf(wq[0].z, d1.x, wq[0].w * d0.x)));
+            g.y = fmaf(wq[1].x, d3.y, fmaf(wq[1].y, d2.y, fmaf(wq[1].z, d1.y, wq[1].w * d0.y)));
+            if (p.dtail_out && t >= p.L - 3) {
+                const float2 dto = ld2(p.dtail_out + (bi * 3 + (t - (p.L - 3))) * p.C_ch + c);
+                g.x += dto.x;
+                g.y += dto.y;
+            }
+            *reinterpret_cast<float2 *>(p.du + (bi * p.L + t) * p.C_ch + c) = g;
+            gb.x += d0.x;
+            gb.y += d0.y;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                gw[k].x = fmaf(d0.x, wa[k], gw[k].x);
+                gw[k].y = fmaf(d0.y, wb[k], gw[k].y);
+            }
+            d3 = d2; d2 = d1; d1 = d0;
+            uw[3] = uw[2]; uw[2] = uw[1]; uw[1] = uw[0]; uw[0] = un[i];
+        }
+    }
+    const int64_t slot = (bi * nblk + blk) * p.C_ch + c;
+    reinterpret_cast<float4 *>(p.ws_dw)[slot] = make_float4(gw[0].x, gw[1].x, gw[2].x, gw[3].x);
+    reinterpret_cast<float4 *>(p.ws_dw)[slot + 1] = make_float4(gw[0].y, gw[1].y, gw[2].y, gw[3].y);
+    p.ws_dbias[slot] = gb.x;
+    p.ws_dbias[slot + 1] = gb.y;
+    if (blk == 0 && p.dtail_in) {
+        // the rows before the sequence (positions -3, -2, -1): d1, d2, d3 now hold dz at 0, 1, 2
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+            float *dt = p.dtail_in + bi * 3 * p.C_ch + c + ch;
+            const float e1 = ch ? d1.y : d1.x, e2 = ch ? d2.y : d2.x, e3 = ch ? d3.y : d3.x;
+            float g2 = fmaf(wq[ch].z, e1, fmaf(wq[ch].y, e2, wq[ch].x * e3));   // position -1
+            float g1 = fmaf(wq[ch].y, e1, wq[ch].x * e2);                        // position -2
+            float g0 = wq[ch].x * e1;                                            // position -3
+            if (p.dtail_out) {
+                for (int r = 0; r < 3; ++r) {
+                    const int64_t pos = p.L - 3 + r;
+                    if (pos >= 0) continue;
+                    const float gt = p.dtail_out[(bi * 3 + r) * p.C_ch + c + ch];
+                    if (pos == -3) g0 += gt;
+                    else if (pos == -2) g1 += gt;
+                    else g2 += gt;
+                }
+            }
+            dt[0] = g0;
+            dt[p.C_ch] = g1;
+            dt[2 * p.C_ch] = g2;
+        }
+    }
+}
+
+// dw and dbias: the partial sums of every (batch row, token block), added in a fixed order.  A CTA
+// takes 32 channels; its 8 warps each add every 8th partial of them (8 loads in flight per
+// thread), then warp 0 adds the 8 warp sums in order.
+constexpr int kRedSlices = 8;
+__global__ void __launch_bounds__(32 * kRedSlices) conv_bwd_reduce_kernel(ConvBwdParams p, int64_t nparts)
+{
+    __shared__ float4 sw[kRedSlices][32];
+    __shared__ float sb[kRedSlices][32];
+    const int cl = threadIdx.x & 31, sl = threadIdx.x >> 5;
+    const int c = blockIdx.x * 32 + cl;
     float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     float ab = 0.0f;
-    for (int64_t i = 0; i < nparts; ++i) {
-        const float4 v = reinterpret_cast<const float4 *>(p.ws_dw)[i * p.C_ch + c];
-        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-        ab += p.ws_dbias[i * p.C_ch + c];
+    if (c < p.C_ch) {
+        for (int64_t i0 = sl; i0 < nparts; i0 += 8 * kRedSlices) {
+            float4 v[8];
+            float b[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int64_t i = i0 + (int64_t)u * kRedSlices;
+                v[u] = i < nparts ? reinterpret_cast<const float4 *>(p.ws_dw)[i * p.C_ch + c]
+                                  : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                b[u] = i < nparts ? p.ws_dbias[i * p.C_ch + c] : 0.0f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                acc.x += v[u].x; acc.y += v[u].y; acc.z += v[u].z; acc.w += v[u].w;
+                ab += b[u];
+            }
+        }
     }
-    reinterpret_cast<float4 *>(p.dw)[c] = acc;
-    if (p.dbias) p.dbias[c] = ab;
+    sw[sl][cl] = acc;
+    sb[sl][cl] = ab;
+    __syncthreads();
+    if (sl == 0 && c < p.C_ch) {
+        for (int k = 1; k < kRedSlices; ++k) {
+            const float4 v = sw[k][cl];
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+            ab += sb[k][cl];
+        }
+        reinterpret_cast<float4 *>(p.dw)[c] = acc;
+        if (p.dbias) p.dbias[c] = ab;
+    }
 }
 
 }  // namespace
@@ -163,15 +335,22 @@ int64_t conv_bwd_blocks(int64_t L) { return (L + kTB - 1) / kTB; }
 int launch_conv_backward(const ConvBwdParams &p, int dtype, cudaStream_t st)
 {
     const int64_t nblk = conv_bwd_blocks(p.L);
-    const int64_t n = (int64_t)p.b * nblk * p.C_ch;
+    // two channels per thread when every channel pair lies in one of x, B, C
+    const bool pairs = p.C_ch % 2 == 0 && p.HP % 2 == 0 && p.GN % 2 == 0;
+    const int64_t n = (int64_t)p.b * nblk * (pairs ? p.C_ch / 2 : p.C_ch);
     const int64_t blocks = (n + kConvBwdThreads - 1) / kConvBwdThreads;
     if (blocks > 0x7fffffffLL) return 2;
     prof_begin(st, kKConvBwd);
     if (n > 0) {
-        if (dtype == 1) conv_bwd_kernel<__nv_bfloat16><<<(unsigned)blocks, kConvBwdThreads, 0, st>>>(p, nblk);
-        else conv_bwd_kernel<float><<<(unsigned)blocks, kConvBwdThreads, 0, st>>>(p, nblk);
+        if (pairs) {
+            if (dtype == 1) conv_bwd2_kernel<__nv_bfloat16><<<(unsigned)blocks, kConvBwdThreads, 0, st>>>(p, nblk);
+            else conv_bwd2_kernel<float><<<(unsigned)blocks, kConvBwdThreads, 0, st>>>(p, nblk);
+        } else {
+            if (dtype == 1) conv_bwd_kernel<__nv_bfloat16><<<(unsigned)blocks, kConvBwdThreads, 0, st>>>(p, nblk);
+            else conv_bwd_kernel<float><<<(unsigned)blocks, kConvBwdThreads, 0, st>>>(p, nblk);
+        }
     }
-    conv_bwd_reduce_kernel<<<(unsigned)((p.C_ch + 127) / 128), 128, 0, st>>>(p, (int64_t)p.b * nblk);
+    conv_bwd_reduce_kernel<<<(unsigned)((p.C_ch + 31) / 32), 32 * kRedSlices, 0, st>>>(p, (int64_t)p.b * nblk);
     prof_end(st, kKConvBwd);
     return cudaGetLastError() == cudaSuccess ? 0 : 7;
 }
