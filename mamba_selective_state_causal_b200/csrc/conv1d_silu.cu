@@ -273,6 +273,76 @@ __global__ void __launch_bounds__(256, 6) conv_cells_kernel(ConvBwdParams p, int
     }
 }
 
+// The same rebuild with two consecutive channels per thread (4-byte bf16 pairs in and out), the
+// block's cell found once (a block never crosses a cell), and the next eight rows of u loaded
+// before their arithmetic.  The arithmetic of each channel is the scalar kernel's, in its order.
+__device__ __forceinline__ float2 cells_ld2(const float *q) { return *reinterpret_cast<const float2 *>(q); }
+__device__ __forceinline__ float2 cells_ld2(const __nv_bfloat16 *q)
+{
+    const uint32_t v = *reinterpret_cast<const uint32_t *>(q);
+    return make_float2(bf16_lo(v), bf16_hi(v));
+}
+__device__ __forceinline__ void cells_st2(float *q, float a, float b) { *reinterpret_cast<float2 *>(q) = make_float2(a, b); }
+__device__ __forceinline__ void cells_st2(__nv_bfloat16 *q, float a, float b)
+{
+    const __nv_bfloat16 ha = __float2bfloat16_rn(a), hb = __float2bfloat16_rn(b);
+    *reinterpret_cast<uint32_t *>(q) = (uint32_t)__bfloat16_as_ushort(ha) | ((uint32_t)__bfloat16_as_ushort(hb) << 16);
+}
+
+constexpr int kCellAhead = 8;
+template <typename T>
+__global__ void __launch_bounds__(256, 3) conv_cells2_kernel(ConvBwdParams p, int64_t nblk)
+{
+    const int np = p.C_ch >> 1;
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= (int64_t)p.b * nblk * np) return;
+    const int c = 2 * (int)(gid % np);
+    const int64_t blk = (gid / np) % nblk;
+    const int64_t bi = gid / ((int64_t)np * nblk);
+    const int64_t t0 = blk * kCellTB;
+    const int64_t t1 = min(p.L, t0 + kCellTB);
+    const float4 wa = __ldg(reinterpret_cast<const float4 *>(p.w) + c);
+    const float4 wb = __ldg(reinterpret_cast<const float4 *>(p.w) + c + 1);
+    const float ba = p.bias ? __ldg(p.bias + c) : 0.0f, bb = p.bias ? __ldg(p.bias + c + 1) : 0.0f;
+    const T *u = reinterpret_cast<const T *>(p.u) + bi * p.ubs + c;
+    // the window u[t0-3 .. t0-1]: rows before the cell come from its conv buffer
+    const int64_t kc = p.conv_ckpt ? t0 / p.s : 0;
+    const int64_t cstart = p.conv_ckpt ? kc * p.s : 0;
+    float2 uw[3];
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+        const int64_t tt = t0 - 3 + k;
+        if (tt >= cstart) {
+            uw[k] = cells_ld2(u + tt * p.urs);
+        } else {
+            const int64_t r = tt - cstart + 3;
+            if (kc == 0)
+                uw[k] = p.tail_in ? cells_ld2(reinterpret_cast<const T *>(p.tail_in) + (bi * 3 + r) * p.C_ch + c)
+                                  : make_float2(0.0f, 0.0f);
+            else
+                uw[k] = cells_ld2(reinterpret_cast<const T *>(p.conv_ckpt) + ((bi * p.n_ckpt + (kc - 1)) * 3 + r) * p.C_ch + c);
+        }
+    }
+    T *v = reinterpret_cast<T *>(p.v) + (bi * p.L) * p.C_ch + c;
+    for (int64_t tg = t0; tg < t1; tg += kCellAhead) {
+        float2 un[kCellAhead];
+#pragma unroll
+        for (int i = 0; i < kCellAhead; ++i) un[i] = tg + i < t1 ? cells_ld2(u + (tg + i) * p.urs) : make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int i = 0; i < kCellAhead; ++i) {
+            const int64_t t = tg + i;
+            if (t >= t1) break;
+            float za = ba, zb = bb;
+            za = fmaf(wa.x, uw[0].x, za); zb = fmaf(wb.x, uw[0].y, zb);
+            za = fmaf(wa.y, uw[1].x, za); zb = fmaf(wb.y, uw[1].y, zb);
+            za = fmaf(wa.z, uw[2].x, za); zb = fmaf(wb.z, uw[2].y, zb);
+            za = fmaf(wa.w, un[i].x, za); zb = fmaf(wb.w, un[i].y, zb);
+            cells_st2(v + t * p.C_ch, VecIO<T>::silu(za), VecIO<T>::silu(zb));
+            uw[0] = uw[1]; uw[1] = uw[2]; uw[2] = un[i];
+        }
+    }
+}
+
 // conv_ckpt[bi, k, r, c] = u[bi, (k+1) s - 3 + r, c]: the conv buffer at every checkpoint
 template <typename T>
 __global__ void conv_ckpt_kernel(const T *u, int64_t ubs, int64_t urs, T *out, int b, int64_t n_ckpt, int C_ch,
@@ -292,13 +362,20 @@ __global__ void conv_ckpt_kernel(const T *u, int64_t ubs, int64_t urs, T *out, i
 int launch_conv_cells(const ConvBwdParams &p, int dtype, cudaStream_t st)
 {
     const int64_t nblk = (p.L + kCellTB - 1) / kCellTB;
-    const int64_t n = (int64_t)p.b * nblk * p.C_ch;
+    const bool pairs = p.C_ch % 2 == 0;
+    const int64_t n = (int64_t)p.b * nblk * (pairs ? p.C_ch / 2 : p.C_ch);
     if (n == 0) return 0;
     const int64_t blocks = (n + 255) / 256;
     if (blocks > 0x7fffffffLL) return 2;
     prof_begin(st, kKConvCells);
-    if (dtype == 1) conv_cells_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(p, nblk);
-    else conv_cells_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(p, nblk);
+    if (pairs) {
+        if (dtype == 1) conv_cells2_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(p, nblk);
+        else conv_cells2_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(p, nblk);
+    } else if (dtype == 1) {
+        conv_cells_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(p, nblk);
+    } else {
+        conv_cells_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(p, nblk);
+    }
     prof_end(st, kKConvCells);
     return cudaGetLastError() == cudaSuccess ? 0 : 7;
 }
