@@ -190,21 +190,71 @@ __device__ __forceinline__ float2 dz2_at(const ConvBwdParams &p, int64_t bi, int
     return make_float2(dz_of(dv.x, wq[0], bs.x, wa), dz_of(dv.y, wq[1], bs.y, wb));
 }
 
+// asynchronous copies of 4 or 8 bytes into shared memory (the stream of one thread)
+template <int kBytes>
+__device__ __forceinline__ void cp_async_small(void *dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src),
+                 "n"(kBytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_b() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_b() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 // The same walk as conv_bwd_kernel with two consecutive channels per thread (one thread per
-// (batch row, block of kTB tokens, channel pair), consecutive threads on consecutive pairs) and
-// eight tokens' loads issued before their arithmetic.  two CTAs per SM (at most 128 registers)
-constexpr int kAhead2 = 8;
+// (batch row, block of kTB tokens, channel pair), consecutive threads on consecutive pairs).  Each
+// thread streams its tokens' dv and the u rows its window needs through its own slots of a ring
+// in shared memory (kRingB tokens in flight, 4- and 8-byte asynchronous copies), so the loads in
+// flight cost no registers; the block's cell (where its conv buffer starts) is found once.
+constexpr int kRingB = 16;
 template <typename T>
 __global__ void __launch_bounds__(kConvBwdThreads, 2) conv_bwd2_kernel(ConvBwdParams p, int64_t nblk)
 {
+    extern __shared__ __align__(16) uint8_t cbw_raw[];
+    float2 *rdv = reinterpret_cast<float2 *>(cbw_raw);                                   // [kRingB][threads]
+    T *ru = reinterpret_cast<T *>(cbw_raw + sizeof(float2) * kRingB * kConvBwdThreads);   // [kRingB][threads][2]
+    const int tid = threadIdx.x;
     const int np = p.C_ch >> 1;
-    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + tid;
     if (gid >= (int64_t)p.b * nblk * np) return;
     const int c = 2 * (int)(gid % np);
     const int64_t blk = (gid / np) % nblk;
     const int64_t bi = gid / ((int64_t)np * nblk);
     const int64_t t0 = blk * kTB;
     const int64_t t1 = min(p.L, t0 + kTB);
+    const int n = (int)(t1 - t0);
+    // the block's tokens are all in one cell (blocks and cells are multiples of 64 tokens)
+    const int64_t kc = p.conv_ckpt ? t0 / p.s : 0;
+    const int64_t cstart = p.conv_ckpt ? kc * p.s : 0;
+    auto dv_ptr = [&](int64_t t) -> const float * {
+        const int64_t row = bi * p.L + t;
+        if (c < p.HP) return p.dx + row * p.HP + c;
+        if (c < p.HP + p.GN) return p.dB + row * p.GN + (c - p.HP);
+        return p.dC + row * p.GN + (c - p.HP - p.GN);
+    };
+    auto u_ptr = [&](int64_t tt) -> const T * {
+        if (tt >= cstart) return reinterpret_cast<const T *>(p.u) + bi * p.ubs + tt * p.urs + c;
+        const int64_t r = tt - cstart + 3;
+        if (kc == 0) return p.tail_in ? reinterpret_cast<const T *>(p.tail_in) + (bi * 3 + r) * p.C_ch + c : nullptr;
+        return reinterpret_cast<const T *>(p.conv_ckpt) + ((bi * p.n_ckpt + (kc - 1)) * 3 + r) * p.C_ch + c;
+    };
+    // token j of the walk is t = t1 - 1 - j: its dv, and u[t - 4], the row its window takes next
+    auto issue = [&](int j) {
+        if (j < n) {
+            const int64_t t = t1 - 1 - j;
+            const int sl = (j % kRingB) * kConvBwdThreads + tid;
+            cp_async_small<8>(&rdv[sl], dv_ptr(t));
+            if (t > t0) {
+                const T *q = u_ptr(t - 4);
+                if (q) cp_async_small<2 * sizeof(T)>(&ru[2 * sl], q);
+            }
+        }
+        cp_async_commit_b();
+    };
+#pragma unroll 1
+    for (int j = 0; j < kRingB; ++j) issue(j);
+
     float4 wq[2];
     wq[0] = __ldg(reinterpret_cast<const float4 *>(p.w) + c);
     wq[1] = __ldg(reinterpret_cast<const float4 *>(p.w) + c + 1);
@@ -213,46 +263,47 @@ __global__ void __launch_bounds__(kConvBwdThreads, 2) conv_bwd2_kernel(ConvBwdPa
     float2 d1 = dz2_at<T>(p, bi, t1, c, wq, bs), d2 = dz2_at<T>(p, bi, t1 + 1, c, wq, bs),
            d3 = dz2_at<T>(p, bi, t1 + 2, c, wq, bs);
     float2 gw[4] = {}, gb = make_float2(0.0f, 0.0f);
-    // the block's tokens are all in one cell (blocks and cells are multiples of 64 tokens)
-    const int64_t kc = p.conv_ckpt ? t0 / p.s : 0;
-    const int64_t cstart = p.conv_ckpt ? kc * p.s : 0;
     float2 uw[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) uw[k] = cell2k<T>(p, bi, kc, cstart, t1 - 4 + k, c);
-    for (int64_t tg = t1 - 1; tg >= t0; tg -= kAhead2) {
-        float2 dvv[kAhead2], un[kAhead2];
-#pragma unroll
-        for (int i = 0; i < kAhead2; ++i) {
-            const int64_t t = tg - i;
-            dvv[i] = t >= t0 ? dv2_at(p, bi, t, c) : make_float2(0.0f, 0.0f);
-            un[i] = t > t0 ? cell2k<T>(p, bi, kc, cstart, t - 4, c) : make_float2(0.0f, 0.0f);
-        }
-#pragma unroll
-        for (int i = 0; i < kAhead2; ++i) {
-            const int64_t t = tg - i;
-            if (t < t0) break;
-            const float wa[4] = {uw[0].x, uw[1].x, uw[2].x, uw[3].x}, wb[4] = {uw[0].y, uw[1].y, uw[2].y, uw[3].y};
-            const float2 d0 = make_float2(dz_of(dvv[i].x, wq[0], bs.x, wa), dz_of(dvv[i].y, wq[1], bs.y, wb));
-            float2 g;
-            g.x = fmaf(wq[0].x, d3.x, fmaf(wq[0].y, d2.x, fmaf(wq[0].z, d1.x, wq[0].w * d0.x)));
-            g.y = fmaf(wq[1].x, d3.y, fmaf(wq[1].y, d2.y, fmaf(wq[1].z, d1.y, wq[1].w * d0.y)));
-            if (p.dtail_out && t >= p.L - 3) {
-                const float2 dto = ld2(p.dtail_out + (bi * 3 + (t - (p.L - 3))) * p.C_ch + c);
-                g.x += dto.x;
-                g.y += dto.y;
+#pragma unroll 1
+    for (int j = 0; j < n; ++j) {
+        const int64_t t = t1 - 1 - j;
+        cp_async_wait_b<kRingB - 1>();          // token j's group is the oldest
+        const int sl = (j % kRingB) * kConvBwdThreads + tid;
+        const float2 dvv = rdv[sl];
+        float2 un = make_float2(0.0f, 0.0f);
+        if (t > t0 && u_ptr(t - 4)) {
+            if (sizeof(T) == 2) {
+                const uint32_t v = *reinterpret_cast<const uint32_t *>(&ru[2 * sl]);
+                un = make_float2(bf16_lo(v), bf16_hi(v));
+            } else {
+                un = *reinterpret_cast<const float2 *>(&ru[2 * sl]);
             }
-            *reinterpret_cast<float2 *>(p.du + (bi * p.L + t) * p.C_ch + c) = g;
-            gb.x += d0.x;
-            gb.y += d0.y;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                gw[k].x = fmaf(d0.x, wa[k], gw[k].x);
-                gw[k].y = fmaf(d0.y, wb[k], gw[k].y);
-            }
-            d3 = d2; d2 = d1; d1 = d0;
-            uw[3] = uw[2]; uw[2] = uw[1]; uw[1] = uw[0]; uw[0] = un[i];
         }
+        issue(j + kRingB);                       // refill the slot just read
+        const float wa[4] = {uw[0].x, uw[1].x, uw[2].x, uw[3].x}, wb[4] = {uw[0].y, uw[1].y, uw[2].y, uw[3].y};
+        const float2 d0 = make_float2(dz_of(dvv.x, wq[0], bs.x, wa), dz_of(dvv.y, wq[1], bs.y, wb));
+        float2 g;
+        g.x = fmaf(wq[0].x, d3.x, fmaf(wq[0].y, d2.x, fmaf(wq[0].z, d1.x, wq[0].w * d0.x)));
+        g.y = fmaf(wq[1].x, d3.y, fmaf(wq[1].y, d2.y, fmaf(wq[1].z, d1.y, wq[1].w * d0.y)));
+        if (p.dtail_out && t >= p.L - 3) {
+            const float2 dto = ld2(p.dtail_out + (bi * 3 + (t - (p.L - 3))) * p.C_ch + c);
+            g.x += dto.x;
+            g.y += dto.y;
+        }
+        *reinterpret_cast<float2 *>(p.du + (bi * p.L + t) * p.C_ch + c) = g;
+        gb.x += d0.x;
+        gb.y += d0.y;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            gw[k].x = fmaf(d0.x, wa[k], gw[k].x);
+            gw[k].y = fmaf(d0.y, wb[k], gw[k].y);
+        }
+        d3 = d2; d2 = d1; d1 = d0;
+        uw[3] = uw[2]; uw[2] = uw[1]; uw[1] = uw[0]; uw[0] = un;
     }
+    cp_async_wait_b<0>();
     const int64_t slot = (bi * nblk + blk) * p.C_ch + c;
     reinterpret_cast<float4 *>(p.ws_dw)[slot] = make_float4(gw[0].x, gw[1].x, gw[2].x, gw[3].x);
     reinterpret_cast<float4 *>(p.ws_dw)[slot + 1] = make_float4(gw[0].y, gw[1].y, gw[2].y, gw[3].y);
@@ -343,8 +394,18 @@ int launch_conv_backward(const ConvBwdParams &p, int dtype, cudaStream_t st)
     prof_begin(st, kKConvBwd);
     if (n > 0) {
         if (pairs) {
-            if (dtype == 1) conv_bwd2_kernel<__nv_bfloat16><<<(unsigned)blocks, kConvBwdThreads, 0, st>>>(p, nblk);
-            else conv_bwd2_kernel<float><<<(unsigned)blocks, kConvBwdThreads, 0, st>>>(p, nblk);
+            const int smem = (int)((sizeof(float2) + 2 * (dtype == 1 ? 2 : 4)) * kRingB * kConvBwdThreads);
+            if (dtype == 1) {
+                if (cudaFuncSetAttribute(conv_bwd2_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem) != cudaSuccess)
+                    return 7;
+                conv_bwd2_kernel<__nv_bfloat16><<<(unsigned)blocks, kConvBwdThreads, smem, st>>>(p, nblk);
+            } else {
+                if (cudaFuncSetAttribute(conv_bwd2_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+                    cudaSuccess)
+                    return 7;
+                conv_bwd2_kernel<float><<<(unsigned)blocks, kConvBwdThreads, smem, st>>>(p, nblk);
+            }
         } else {
             if (dtype == 1) conv_bwd_kernel<__nv_bfloat16><<<(unsigned)blocks, kConvBwdThreads, 0, st>>>(p, nblk);
             else conv_bwd_kernel<float><<<(unsigned)blocks, kConvBwdThreads, 0, st>>>(p, nblk);
