@@ -118,6 +118,14 @@ struct SmemSumTc {
     uint32_t tmem;
 };
 
+// 16-byte asynchronous copy into shared memory; a row past the sequence reads zeros
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t sum_swz(int r, int c)
 {
     return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
@@ -153,39 +161,51 @@ __global__ void __launch_bounds__(kSumTcThreads) bwd_chunk_summary_tc_kernel(Bwd
         fence_mbar_init();
     }
     if (warp == 0) { tmem_alloc(&s.tmem, 128); tmem_relinquish(); }
-    for (int i = tid; i < kQb; i += kSumTcThreads)
-        s.dts[i] = i < rows ? p.dt[((int64_t)bi * p.L + t0 + i) * p.H + h] : 0.0f;
-    // B and C rows: 16 chunks of 16 bytes per row, chunk q of row j to box q >> 3
+    // B and C rows, 16 chunks of 16 bytes per row (chunk q of row j to box q >> 3), as asynchronous
+    // copies; x and dy rows (8 chunks per row) into registers, all before the chunk's cumsum
     const __nv_bfloat16 *Bg = reinterpret_cast<const __nv_bfloat16 *>(p.B) + bi * p.Bbs + t0 * p.Brs + (int64_t)g * N;
     const __nv_bfloat16 *Cg = reinterpret_cast<const __nv_bfloat16 *>(p.C) + bi * p.Cbs + t0 * p.Crs + (int64_t)g * N;
     for (int i = tid; i < kQb * 16; i += kSumTcThreads) {
         const int j = i >> 4, q = i & 15;
+        const bool v = j < rows;
+        const int64_t js = v ? j : 0;
         const uint32_t o = (uint32_t)(q >> 3) * kSumBox + sum_swz(j, q & 7);
-        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4 *>(s.bt + o) = j < rows ? *reinterpret_cast<const uint4 *>(Bg + j * p.Brs + 8 * q) : z;
-        *reinterpret_cast<uint4 *>(s.ct + o) = j < rows ? *reinterpret_cast<const uint4 *>(Cg + j * p.Crs + 8 * q) : z;
+        cp_async16(smem_u32(s.bt) + o, Bg + js * p.Brs + 8 * q, v);
+        cp_async16(smem_u32(s.ct) + o, Cg + js * p.Crs + 8 * q, v);
     }
+    const __nv_bfloat16 *xg = reinterpret_cast<const __nv_bfloat16 *>(p.x) + bi * p.xbs + t0 * p.xrs + (int64_t)h * P;
+    const __nv_bfloat16 *yg = reinterpret_cast<const __nv_bfloat16 *>(p.dy) + bi * p.dybs + t0 * p.dyrs + (int64_t)h * P;
+    constexpr int kXPer = kQb * 8 / kSumTcThreads;
+    uint4 xr[kXPer], yr[kXPer];
+#pragma unroll
+    for (int k = 0; k < kXPer; ++k) {
+        const int i = tid + k * kSumTcThreads;
+        const int j = i >> 3, q = i & 7;
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        xr[k] = j < rows ? *reinterpret_cast<const uint4 *>(xg + j * p.xrs + 8 * q) : z;
+        yr[k] = j < rows ? *reinterpret_cast<const uint4 *>(yg + j * p.dyrs + 8 * q) : z;
+    }
+    for (int i = tid; i < kQb; i += kSumTcThreads)
+        s.dts[i] = i < rows ? p.dt[((int64_t)bi * p.L + t0 + i) * p.H + h] : 0.0f;
     __syncthreads();
     chunk_cumsum(s.dts, s.cum, p.A[h]);
     __syncthreads();
     const float lam = s.cum[kQb - 1];
-    // x and dy rows, weighted and split: 8 chunks of 16 bytes per row
-    const __nv_bfloat16 *xg = reinterpret_cast<const __nv_bfloat16 *>(p.x) + bi * p.xbs + t0 * p.xrs + (int64_t)h * P;
-    const __nv_bfloat16 *yg = reinterpret_cast<const __nv_bfloat16 *>(p.dy) + bi * p.dybs + t0 * p.dyrs + (int64_t)h * P;
-    for (int i = tid; i < kQb * 8; i += kSumTcThreads) {
+    // x and dy rows, weighted and split
+#pragma unroll
+    for (int k = 0; k < kXPer; ++k) {
+        const int i = tid + k * kSumTcThreads;
         const int j = i >> 3, q = i & 7;
         const uint32_t o = sum_swz(j, q);
-        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-        const uint4 xv = j < rows ? *reinterpret_cast<const uint4 *>(xg + j * p.xrs + 8 * q) : z;
-        const uint4 yv = j < rows ? *reinterpret_cast<const uint4 *>(yg + j * p.dyrs + 8 * q) : z;
         uint4 hi, lo;
-        split8(xv, s.dts[j] * expf(lam - s.cum[j]), hi, lo);
+        split8(xr[k], s.dts[j] * expf(lam - s.cum[j]), hi, lo);
         *reinterpret_cast<uint4 *>(s.xh + o) = hi;
         *reinterpret_cast<uint4 *>(s.xl + o) = lo;
-        split8(yv, expf(s.cum[j]), hi, lo);
+        split8(yr[k], expf(s.cum[j]), hi, lo);
         *reinterpret_cast<uint4 *>(s.gh + o) = hi;
         *reinterpret_cast<uint4 *>(s.gl + o) = lo;
     }
+    cp_async_wait_all();
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -706,12 +726,6 @@ struct SmemGradTc {
     int ok;
 };
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // bf16 element (r, col) of a 64-row tile of 128-byte rows in the 128B-swizzled layout;
 // columns 64..127 live in a second tile kSumBox further on
