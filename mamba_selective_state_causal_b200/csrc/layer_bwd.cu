@@ -14,7 +14,7 @@
 // pith_extraction.key_machinery): z of a token reads the rows before its cell
 // from that cell's stored 3-row conv buffer, which is what makes the
 // recompute exact (skeptic_critique.headline).  The rounding of v to the I/O
-// dtype is taken as the identity, and dz is fp32 with an accurate exponential.
+// dtype is taken as the identity, and dz is fp32 (sigma through the hardware exponential).
 #include "ssd_common.cuh"
 
 namespace ssd {
@@ -40,7 +40,9 @@ __device__ __forceinline__ float dz_of(float dv, const float4 &wq, float bs, con
     z = fmaf(wq.y, uw[1], z);
     z = fmaf(wq.z, uw[2], z);
     z = fmaf(wq.w, uw[3], z);
-    const float sg = 1.0f / (1.0f + expf(-z));
+    // sigma(z) with the hardware exponential and a fast division; -z is clamped at 80 inside the
+    // exponential so the divisor stays below 2^126 (sigma(z) is below 2e-35 there either way)
+    const float sg = __fdividef(1.0f, 1.0f + __expf(fminf(-z, 80.0f)));
     return dv * (sg * (1.0f + z * (1.0f - sg)));
 }
 
