@@ -233,49 +233,16 @@ int launch_conv_t(const ConvParams &p, cudaStream_t st)
 }
 
 // The conv output rebuilt cell by cell for the backward pass: v[bi, t, c] from
-// the cell's own rows of u and its conv buffer (cell_val), with the forward
+// the cell's own rows of u and its 3-row conv buffer, with the forward
 // kernel's arithmetic (same order of fused multiply-adds, same SiLU), so that a
 // cell rebuilt from exact buffers reproduces the forward's v bit for bit.
 constexpr int kCellTB = 64;      // tokens per thread of the cell rebuild
 
-// One thread per (batch row, block of kCellTB tokens, channel), consecutive threads on consecutive
-// channels; the thread slides the conv window of u along its block in registers, one new row per
-// token (rows before a cell come from its conv buffer).
-// six CTAs per SM: more warps in flight beat the few registers spilled
-template <typename T>
-__global__ void __launch_bounds__(256, 6) conv_cells_kernel(ConvBwdParams p, int64_t nblk)
-{
-    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (gid >= (int64_t)p.b * nblk * p.C_ch) return;
-    const int c = (int)(gid % p.C_ch);
-    const int64_t blk = (gid / p.C_ch) % nblk;
-    const int64_t bi = gid / ((int64_t)p.C_ch * nblk);
-    const int64_t t0 = blk * kCellTB;
-    const int64_t t1 = min(p.L, t0 + kCellTB);
-    const float4 wq = __ldg(reinterpret_cast<const float4 *>(p.w) + c);
-    const float bs = p.bias ? __ldg(p.bias + c) : 0.0f;
-    float uw[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) uw[k] = cell_val<T>(p, bi, t0, t0 - 3 + k, c);
-    // a block never crosses a cell (blocks and cells are multiples of 64 tokens), so the window
-    // only slides
-    for (int64_t t = t0; t < t1; ++t) {
-        float z = bs;
-        z = fmaf(wq.x, uw[0], z);
-        z = fmaf(wq.y, uw[1], z);
-        z = fmaf(wq.z, uw[2], z);
-        z = fmaf(wq.w, uw[3], z);
-        reinterpret_cast<T *>(p.v)[(bi * p.L + t) * p.C_ch + c] = from_f32<T>(VecIO<T>::silu(z));
-        if (t + 1 < t1) {
-            uw[0] = uw[1]; uw[1] = uw[2]; uw[2] = uw[3];
-            uw[3] = cell_val<T>(p, bi, t + 1, t + 1, c);
-        }
-    }
-}
-
-// The same rebuild with two consecutive channels per thread (4-byte bf16 pairs in and out), the
-// block's cell found once (a block never crosses a cell), and the next eight rows of u loaded
-// before their arithmetic.  The arithmetic of each channel is the scalar kernel's, in its order.
+// One thread per (batch row, block of kCellTB tokens, channel pair), consecutive threads on
+// consecutive pairs (4-byte bf16 pairs in and out); the block's cell is found once (a block never
+// crosses a cell: blocks and cells are multiples of 64 tokens), the thread slides the conv window
+// of u along its block in registers, and the next eight rows of u are loaded before their
+// arithmetic.  The arithmetic of each channel is the forward conv's, in its order.
 __device__ __forceinline__ float2 cells_ld2(const float *q) { return *reinterpret_cast<const float2 *>(q); }
 __device__ __forceinline__ float2 cells_ld2(const __nv_bfloat16 *q)
 {
@@ -362,20 +329,14 @@ __global__ void conv_ckpt_kernel(const T *u, int64_t ubs, int64_t urs, T *out, i
 int launch_conv_cells(const ConvBwdParams &p, int dtype, cudaStream_t st)
 {
     const int64_t nblk = (p.L + kCellTB - 1) / kCellTB;
-    const bool pairs = p.C_ch % 2 == 0;
-    const int64_t n = (int64_t)p.b * nblk * (pairs ? p.C_ch / 2 : p.C_ch);
+    // two channels per thread: P and N are multiples of 16, so C_ch is even
+    const int64_t n = (int64_t)p.b * nblk * (p.C_ch / 2);
     if (n == 0) return 0;
     const int64_t blocks = (n + 255) / 256;
     if (blocks > 0x7fffffffLL) return 2;
     prof_begin(st, kKConvCells);
-    if (pairs) {
-        if (dtype == 1) conv_cells2_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(p, nblk);
-        else conv_cells2_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(p, nblk);
-    } else if (dtype == 1) {
-        conv_cells_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(p, nblk);
-    } else {
-        conv_cells_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(p, nblk);
-    }
+    if (dtype == 1) conv_cells2_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(p, nblk);
+    else conv_cells2_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(p, nblk);
     prof_end(st, kKConvCells);
     return cudaGetLastError() == cudaSuccess ? 0 : 7;
 }

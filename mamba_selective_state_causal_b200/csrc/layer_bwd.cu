@@ -23,15 +23,6 @@ namespace {
 constexpr int kTB = 64;          // tokens per thread, walked from the last
 constexpr int kConvBwdThreads = 256;
 
-// dLoss/dv of channel c at row (bi, t)
-__device__ __forceinline__ float dv_at(const ConvBwdParams &p, int64_t bi, int64_t t, int c)
-{
-    const int64_t row = bi * p.L + t;
-    if (c < p.HP) return p.dx[row * p.HP + c];
-    if (c < p.HP + p.GN) return p.dB[row * p.GN + (c - p.HP)];
-    return p.dC[row * p.GN + (c - p.HP - p.GN)];
-}
-
 // dz = dv silu'(z) from the conv window u[t-3 .. t] (as token t's cell sees it)
 __device__ __forceinline__ float dz_of(float dv, const float4 &wq, float bs, const float (&uw)[4])
 {
@@ -44,102 +35,6 @@ __device__ __forceinline__ float dz_of(float dv, const float4 &wq, float bs, con
     // exponential so the divisor stays below 2^126 (sigma(z) is below 2e-35 there either way)
     const float sg = __fdividef(1.0f, 1.0f + __expf(fminf(-z, 80.0f)));
     return dv * (sg * (1.0f + z * (1.0f - sg)));
-}
-
-template <typename T>
-__device__ __forceinline__ void load_window(const ConvBwdParams &p, int64_t bi, int64_t t, int c, float (&uw)[4])
-{
-#pragma unroll
-    for (int k = 0; k < 4; ++k) uw[k] = cell_val<T>(p, bi, t, t - 3 + k, c);
-}
-
-template <typename T>
-__device__ __forceinline__ float dz_at(const ConvBwdParams &p, int64_t bi, int64_t t, int c, const float4 &wq,
-                                       float bs)
-{
-    if (t >= p.L) return 0.0f;
-    float uw[4];
-    load_window<T>(p, bi, t, c, uw);
-    return dz_of(dv_at(p, bi, t, c), wq, bs, uw);
-}
-
-// One thread per (batch row, block of kTB tokens, channel); consecutive threads
-// take consecutive channels, so every row access is coalesced.  The thread walks
-// its block from the last token with the conv window of u in registers, one new
-// row per token (rows before a cell come from its conv buffer).
-// four CTAs per SM (at most 64 registers): enough warps to cover the loads of the serial walk
-template <typename T>
-__global__ void __launch_bounds__(kConvBwdThreads, 4) conv_bwd_kernel(ConvBwdParams p, int64_t nblk)
-{
-    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (gid >= (int64_t)p.b * nblk * p.C_ch) return;
-    const int c = (int)(gid % p.C_ch);
-    const int64_t blk = (gid / p.C_ch) % nblk;
-    const int64_t bi = gid / ((int64_t)p.C_ch * nblk);
-    const int64_t t0 = blk * kTB;
-    const int64_t t1 = min(p.L, t0 + kTB);
-    const float4 wq = __ldg(reinterpret_cast<const float4 *>(p.w) + c);
-    const float bs = p.bias ? __ldg(p.bias + c) : 0.0f;
-    // window of dz at t'+0 .. t'+3, walked from t' = t1-1 down to t0
-    float d1 = dz_at<T>(p, bi, t1, c, wq, bs), d2 = dz_at<T>(p, bi, t1 + 1, c, wq, bs),
-          d3 = dz_at<T>(p, bi, t1 + 2, c, wq, bs);
-    float gw0 = 0.0f, gw1 = 0.0f, gw2 = 0.0f, gw3 = 0.0f, gb = 0.0f;
-    float uw[4];
-    load_window<T>(p, bi, t1 - 1, c, uw);
-    // a block never crosses a cell (blocks and cells are multiples of 64 tokens), so the window
-    // only slides; each group of four tokens issues its loads before it computes
-    for (int64_t tg = t1 - 1; tg >= t0; tg -= 4) {
-        float dvv[4], un[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int64_t t = tg - i;
-            dvv[i] = t >= t0 ? dv_at(p, bi, t, c) : 0.0f;
-            un[i] = t > t0 ? cell_val<T>(p, bi, t - 1, t - 4, c) : 0.0f;
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int64_t t = tg - i;
-            if (t < t0) break;
-            const float d0 = dz_of(dvv[i], wq, bs, uw);
-            float g = wq.w * d0;
-            g = fmaf(wq.z, d1, g);
-            g = fmaf(wq.y, d2, g);
-            g = fmaf(wq.x, d3, g);
-            if (p.dtail_out && t >= p.L - 3) g += p.dtail_out[(bi * 3 + (t - (p.L - 3))) * p.C_ch + c];
-            p.du[(bi * p.L + t) * p.C_ch + c] = g;
-            gb += d0;
-            gw0 = fmaf(d0, uw[0], gw0);
-            gw1 = fmaf(d0, uw[1], gw1);
-            gw2 = fmaf(d0, uw[2], gw2);
-            gw3 = fmaf(d0, uw[3], gw3);
-            d3 = d2; d2 = d1; d1 = d0;
-            uw[3] = uw[2]; uw[2] = uw[1]; uw[1] = uw[0]; uw[0] = un[i];
-        }
-    }
-    const int64_t slot = (bi * nblk + blk) * p.C_ch + c;
-    reinterpret_cast<float4 *>(p.ws_dw)[slot] = make_float4(gw0, gw1, gw2, gw3);
-    p.ws_dbias[slot] = gb;
-    if (blk == 0 && p.dtail_in) {
-        // the rows before the sequence (positions -3, -2, -1): d1, d2, d3 now hold dz at 0, 1, 2
-        float *dt = p.dtail_in + bi * 3 * p.C_ch + c;
-        float g2 = fmaf(wq.z, d1, fmaf(wq.y, d2, wq.x * d3));   // position -1
-        float g1 = fmaf(wq.y, d1, wq.x * d2);                   // position -2
-        float g0 = wq.x * d1;                                   // position -3
-        if (p.dtail_out) {
-            // tail_out rows that are rows of tail_in when L < 3
-            for (int r = 0; r < 3; ++r) {
-                const int64_t pos = p.L - 3 + r;
-                if (pos >= 0) continue;
-                const float gt = p.dtail_out[(bi * 3 + r) * p.C_ch + c];
-                if (pos == -3) g0 += gt;
-                else if (pos == -2) g1 += gt;
-                else g2 += gt;
-            }
-        }
-        dt[0] = g0;
-        dt[p.C_ch] = g1;
-        dt[2 * p.C_ch] = g2;
-    }
 }
 
 // ---- two consecutive channels per thread (8-byte loads of dv and stores of du, 4 bytes of bf16 u)
@@ -159,7 +54,9 @@ __device__ __forceinline__ float2 dv2_at(const ConvBwdParams &p, int64_t bi, int
     return ld2(p.dC + row * p.GN + (c - p.HP - p.GN));
 }
 
-// cell_val of channels c, c+1 at position tt, for a token of cell k (which starts at `start`)
+// Row tt of the conv input, channels c and c+1, as a token of cell k (which starts at `start`)
+// sees it when each cell is rebuilt on its own: rows before the cell come from its 3-row conv
+// buffer (conv_ckpt[k-1] for cell k > 0, tail_in or zeros for the first cell), the others from u
 template <typename T>
 __device__ __forceinline__ float2 cell2k(const ConvBwdParams &p, int64_t bi, int64_t k, int64_t start, int64_t tt, int c)
 {
@@ -171,7 +68,7 @@ __device__ __forceinline__ float2 cell2k(const ConvBwdParams &p, int64_t bi, int
     return ld2(reinterpret_cast<const T *>(p.conv_ckpt) + ((bi * p.n_ckpt + (k - 1)) * 3 + r) * p.C_ch + c);
 }
 
-// cell_val of channels c, c+1 for token t
+// the same for token t (its cell found from t)
 template <typename T>
 __device__ __forceinline__ float2 cell2(const ConvBwdParams &p, int64_t bi, int64_t t, int64_t tt, int c)
 {
@@ -204,8 +101,10 @@ __device__ __forceinline__ void cp_async_commit_b() { asm volatile("cp.async.com
 template <int N>
 __device__ __forceinline__ void cp_async_wait_b() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// The same walk as conv_bwd_kernel with two consecutive channels per thread (one thread per
-// (batch row, block of kTB tokens, channel pair), consecutive threads on consecutive pairs).  Each
+// One thread per (batch row, block of kTB tokens, channel pair), consecutive threads on
+// consecutive pairs; the thread walks its block from the last token with the conv window of u
+// and a 4-deep window of dz in registers (a block never crosses a cell: blocks and cells are
+// multiples of 64 tokens).  Each
 // thread streams its tokens' dv and the u rows its window needs through its own slots of a ring
 // in shared memory (kRingB tokens in flight, 4- and 8-byte asynchronous copies), so the loads in
 // flight cost no registers; the block's cell (where its conv buffer starts) is found once.
@@ -388,29 +287,23 @@ int64_t conv_bwd_blocks(int64_t L) { return (L + kTB - 1) / kTB; }
 int launch_conv_backward(const ConvBwdParams &p, int dtype, cudaStream_t st)
 {
     const int64_t nblk = conv_bwd_blocks(p.L);
-    // two channels per thread when every channel pair lies in one of x, B, C
-    const bool pairs = p.C_ch % 2 == 0 && p.HP % 2 == 0 && p.GN % 2 == 0;
-    const int64_t n = (int64_t)p.b * nblk * (pairs ? p.C_ch / 2 : p.C_ch);
+    // two channels per thread: P and N are multiples of 16, so a channel pair never straddles x, B, C
+    const int64_t n = (int64_t)p.b * nblk * (p.C_ch / 2);
     const int64_t blocks = (n + kConvBwdThreads - 1) / kConvBwdThreads;
     if (blocks > 0x7fffffffLL) return 2;
     prof_begin(st, kKConvBwd);
     if (n > 0) {
-        if (pairs) {
-            const int smem = (int)((sizeof(float2) + 2 * (dtype == 1 ? 2 : 4)) * kRingB * kConvBwdThreads);
-            if (dtype == 1) {
-                if (cudaFuncSetAttribute(conv_bwd2_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         smem) != cudaSuccess)
-                    return 7;
-                conv_bwd2_kernel<__nv_bfloat16><<<(unsigned)blocks, kConvBwdThreads, smem, st>>>(p, nblk);
-            } else {
-                if (cudaFuncSetAttribute(conv_bwd2_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-                    cudaSuccess)
-                    return 7;
-                conv_bwd2_kernel<float><<<(unsigned)blocks, kConvBwdThreads, smem, st>>>(p, nblk);
-            }
+        const int smem = (int)((sizeof(float2) + 2 * (dtype == 1 ? 2 : 4)) * kRingB * kConvBwdThreads);
+        if (dtype == 1) {
+            if (cudaFuncSetAttribute(conv_bwd2_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     smem) != cudaSuccess)
+                return 7;
+            conv_bwd2_kernel<__nv_bfloat16><<<(unsigned)blocks, kConvBwdThreads, smem, st>>>(p, nblk);
         } else {
-            if (dtype == 1) conv_bwd_kernel<__nv_bfloat16><<<(unsigned)blocks, kConvBwdThreads, 0, st>>>(p, nblk);
-            else conv_bwd_kernel<float><<<(unsigned)blocks, kConvBwdThreads, 0, st>>>(p, nblk);
+            if (cudaFuncSetAttribute(conv_bwd2_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+                cudaSuccess)
+                return 7;
+            conv_bwd2_kernel<float><<<(unsigned)blocks, kConvBwdThreads, smem, st>>>(p, nblk);
         }
     }
     conv_bwd_reduce_kernel<<<(unsigned)((p.C_ch + 31) / 32), 32 * kRedSlices, 0, st>>>(p, (int64_t)p.b * nblk);

@@ -203,21 +203,6 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(v);
 }
 
-// Row tt of the conv input (channel c of batch row bi) as token t sees it when each cell
-// is rebuilt on its own: rows before t's cell come from that cell's 3-row conv buffer
-// (conv_ckpt[k-1] for cell k > 0, tail_in or zeros for the first cell), the others from u.
-template <typename T>
-__device__ __forceinline__ float cell_val(const ConvBwdParams &p, int64_t bi, int64_t t, int64_t tt, int c)
-{
-    const int64_t k = p.conv_ckpt ? t / p.s : 0;
-    const int64_t start = p.conv_ckpt ? k * p.s : 0;
-    if (tt >= start) return to_f32<T>(reinterpret_cast<const T *>(p.u)[bi * p.ubs + tt * p.urs + c]);
-    const int64_t r = tt - start + 3;
-    if (k == 0)
-        return p.tail_in ? to_f32<T>(reinterpret_cast<const T *>(p.tail_in)[(bi * 3 + r) * p.C_ch + c]) : 0.0f;
-    return to_f32<T>(reinterpret_cast<const T *>(p.conv_ckpt)[((bi * p.n_ckpt + (k - 1)) * 3 + r) * p.C_ch + c]);
-}
-
 // Kernel timing hooks (ssd_api.cu): no-ops unless ssd_profile_begin() is active
 // on the calling thread.
 enum KernelId : int {
