@@ -450,9 +450,14 @@ def run_reference(args, wl, world, rank):
 
 def run_e2e(layer, steps=3):
     """Same metric through the library with host buffers: every step copies the
-    inputs in from pinned host memory and the outputs back.  Segment k's input
-    copy, segment k-1's compute and segment k-2's output copy overlap on three
-    streams, as a caller streaming a long input would run them."""
+    inputs in from pinned host memory and the outputs back (y, the checkpoints and
+    h_final).  Copies in, compute and copies out run on three streams, as a caller
+    streaming a long input would run them, with dependencies per segment: a
+    segment's input copy waits only for the previous step's compute of that
+    segment (its slice of the device input), and a segment's compute for the
+    previous step's output copy of that segment (its slices of y and of the
+    checkpoints; the last segment's copy also holds h_final, which segment 0
+    rewrites)."""
     wl = layer.wl
     comp = torch.cuda.current_stream()
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
@@ -463,42 +468,54 @@ def run_e2e(layer, steps=3):
     o_y = torch.empty(layer.y.shape, dtype=layer.y.dtype, pin_memory=True)
     o_h = torch.empty(layer.h.shape, dtype=layer.h.dtype, pin_memory=True)
     o_ck = torch.empty(layer.ckpt.shape, dtype=layer.ckpt.dtype, pin_memory=True)
-    seg = layer.seg
+    seg, nseg, nck = layer.seg, wl.segments, layer.n_ck
 
     layer.cur = 0                     # the host copies land in the first input set
+    prev_comp = [None] * nseg         # the previous step's compute of each segment
+    prev_out = [None] * nseg          # the previous step's output copy of each segment
 
     def step():
-        s_in.wait_stream(comp)        # the previous step is done with the device buffers
-        s_out.wait_stream(comp)
         landed = []
-        for k in range(wl.segments):
+        for k in range(nseg):
             t0, t1 = k * seg, (k + 1) * seg
+            if prev_comp[k] is not None:
+                s_in.wait_event(prev_comp[k])
             with torch.cuda.stream(s_in):
                 layer.u[:, t0:t1].copy_(h_u[:, t0:t1], non_blocking=True)
                 layer.dt[:, t0:t1].copy_(h_dt[:, t0:t1], non_blocking=True)
                 ev = torch.cuda.Event()
                 ev.record(s_in)
                 landed.append(ev)
-        for k in range(wl.segments):
+        for k in range(nseg):
             t0, t1 = k * seg, (k + 1) * seg
             comp.wait_event(landed[k])
+            if prev_out[k] is not None:
+                comp.wait_event(prev_out[k])
+            if k == 0 and prev_out[nseg - 1] is not None:
+                comp.wait_event(prev_out[nseg - 1])   # h_final of the previous step is out
             layer.segment(k, comp)
             done = torch.cuda.Event()
             done.record(comp)
+            prev_comp[k] = done
             s_out.wait_event(done)
             with torch.cuda.stream(s_out):
                 o_y[:, t0:t1].copy_(layer.y[:, t0:t1], non_blocking=True)
-        with torch.cuda.stream(s_out):
-            o_h.copy_(layer.h, non_blocking=True)
-            o_ck.copy_(layer.ckpt, non_blocking=True)
-        comp.wait_stream(s_out)
+                if nck:
+                    o_ck[:, k * nck:(k + 1) * nck].copy_(layer.ckpt[:, k * nck:(k + 1) * nck], non_blocking=True)
+                if k == nseg - 1:
+                    o_h.copy_(layer.h, non_blocking=True)
+                out = torch.cuda.Event()
+                out.record(s_out)
+                prev_out[k] = out
     step()
+    comp.wait_stream(s_out)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(comp)
     for _ in range(steps):
         step()
+    comp.wait_stream(s_out)           # every step's results are on the host
     e1.record(comp)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
@@ -506,7 +523,7 @@ def run_e2e(layer, steps=3):
     d2h = sum(t.numel() * t.element_size() for t in (o_y, o_h, o_ck))
     return {"value": wl.tokens / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps,
-            "overlap": "input copy of segment k, compute of k-1 and output copy of k-2 on three streams"}
+            "overlap": "copies in, compute and copies out on three streams, ordered per segment"}
 
 
 def run_decode(args, world, rank, local):
