@@ -94,6 +94,24 @@ def test_without_conv_buffers_the_recompute_is_wrong():
     assert e["dconv_w"] > 1e-3 and e["du"] > 1e-4, e
 
 
+def test_saturated_conv_activations():
+    """u and the conv buffer scaled so that the conv's pre-activations reach past the clamp of the
+    sigmoid in the conv's reverse mode (|z| beyond 80 on both sides): both tails of silu' in every
+    gradient, to 1e-5."""
+    wl = ssd_synth.scaled(PAGE_TEST, L=512)
+    prm, u, dt, h0, tail, dy, dhf, dto = _case(wl, seed=9)
+    u, tail = u * 60.0, tail * 60.0
+    # the pre-activations the layer sees: bias + sum_k w[c, k] u[t - 3 + k, c]
+    un, tn, w, b = u[0].double().numpy(), tail[0].double().numpy(), prm["w"].double().numpy(), prm["bias"].double().numpy()
+    ext = np.concatenate([tn, un], axis=0)
+    z = b + sum(w[:, k] * ext[k:k + wl.L] for k in range(4))
+    assert (z > 80).any() and (z < -80).any(), (z.min(), z.max())
+    case = (prm, u, dt, h0, tail, dy, dhf, dto)
+    got, _ = _gpu(wl, *case)
+    errs = _errs(got, _oracle(wl, *case))
+    assert all(e <= 1e-5 for e in errs.values()), errs
+
+
 def test_full_recompute_without_checkpoints():
     wl = ssd_synth.scaled(PAGE_TEST, L=1000)
     case = _case(wl, seed=3)
