@@ -164,3 +164,28 @@ def test_empty_sequence():
     ssd.sync_status()
     assert torch.equal(out["dh0"], dhf)
     assert torch.all(out["dA"] == 0) and torch.all(out["dD"] == 0)
+
+
+def test_full_size_bench_configuration():
+    """The configuration the backward bench times: b = 1, L = 16384, 32 heads of P = 64, N = 128,
+    s = 1024, no h0, dh_final given, the caller's workspace and output buffers (the no-allocation
+    form).  Checkpoints come from the oracle's exact forward, so every gradient, dB and dC summed
+    over the 32 heads included, is held to 1e-5 against the oracle's reverse mode per cell."""
+    wl = ssd_synth.BY_NAME["mamba2-0.3b-L16k"]
+    prm, dt, x, Bm, Cm, _, dy, dhf = _inputs(wl, seed=17, h0=False)
+    args = (x.float().numpy(), Bm.float().numpy(), Cm.float().numpy(), dt.numpy(), prm["A"].numpy(),
+            prm["D"].numpy())
+    fwd = oracle.scan(*args, None, s=wl.s, H=wl.H, P=wl.P)
+    ref = oracle.scan_backward(*args, dy.float().numpy().reshape(wl.b, wl.L, wl.H, wl.P), h0=None,
+                               h_ckpt=fwd["h_ckpt"], dh_final=dhf.double().numpy(), s=wl.s, H=wl.H, P=wl.P)
+    d = "cuda"
+    ws = torch.empty(ssd.backward_workspace_size(wl.b, wl.L, wl.H, wl.P, wl.N), dtype=torch.uint8, device=d)
+    out = {"dx": torch.empty(wl.b, wl.L, wl.H, wl.P, device=d), "dB": torch.empty(wl.b, wl.L, wl.G, wl.N, device=d),
+           "dC": torch.empty(wl.b, wl.L, wl.G, wl.N, device=d), "ddt": torch.empty(wl.b, wl.L, wl.H, device=d),
+           "dA": torch.empty(wl.H, device=d), "dD": torch.empty(wl.H, device=d),
+           "dh0": torch.empty(wl.b, wl.H, wl.P, wl.N, device=d)}
+    ck = torch.from_numpy(fwd["h_ckpt"]).float().to(d)
+    ssd.scan_backward(x.to(d), Bm.to(d), Cm.to(d), dt.to(d), prm["A"].to(d), prm["D"].to(d), dy.to(d), h_ckpt=ck,
+                      dh_final=dhf.to(d), H=wl.H, G=wl.G, s=wl.s, workspace=ws, out=out)
+    ssd.sync_status()
+    _compare({k: host(v) for k, v in out.items()}, ref, TOL["f32"], wl)

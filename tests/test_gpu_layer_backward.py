@@ -159,3 +159,86 @@ def test_empty_sequence():
     assert torch.equal(got["dtail_in"].cpu(), dto)
     assert torch.equal(got["dh0"].cpu(), dhf)
     assert float(got["dconv_w"].abs().max()) == 0.0 and float(got["dA"].abs().max()) == 0.0
+
+
+
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+def test_full_size_bench_configuration(io):
+    """The configuration the layer-backward bench times: b = 1, L = 16384, the 0.3B mixer (32 heads
+    of P = 64, N = 128, 2304 conv channels), s = 1024, no h0 or tail_in, the caller's workspace,
+    then its output buffers (the no-allocation form); bf16 I/O as the bench runs it, and fp32.
+    The state checkpoints come from the oracle's exact forward and the conv buffers are the 3 rows
+    of u before each cell.  A second call, into the first call's outputs, must reproduce it bit
+    for bit (every reduction runs in a fixed order).
+
+    fp32 I/O: every gradient to 1e-5.  bf16 I/O rounds the conv output v to bf16, a decision
+    that the GPU takes on an fp32 value and the oracle on an fp64 one, so a few elements of v
+    round to the other neighbour (the two are then one bf16 spacing apart, 2^-7 relative at
+    most).  The test checks that every element of the GPU's v is a valid rounding (within one
+    spacing of the exact SiLU, plus the fp32 rounding of the four-tap sum, plus the hardware
+    tanh's approximation of sigma, 2^-12 absolute), that at most 1e-3 of them round the other
+    way, and hence that v's relL2 against the oracle's rounding is at most
+    sqrt(1e-3) * 2^-7 = 2.5e-4; the gradients, which carry that difference of v with a gain
+    of about 2, are held to 5e-4."""
+    wl = ssd_synth.scaled(ssd_synth.BY_NAME["mamba2-0.3b-L16k"], dtype=io)
+    seed = 18
+    prm = ssd_synth.make_params(wl, seed=seed)
+    dto, _ = ssd_synth.make_conv_grads(wl, seed=seed)
+    u = ssd_synth.make_u(wl, seed=seed)
+    dt = ssd_synth.make_dt(wl, prm["dt_bias"], seed=seed)
+    dy, dhf = ssd_synth.make_grads(wl, seed=seed)
+    un = host(u)
+    fwd = oracle.layer(un, prm["w"].numpy(), dt.numpy(), prm["A"].numpy(), prm["D"].numpy(), bias=prm["bias"].numpy(),
+                       H=wl.H, P=wl.P, N=wl.N, G=wl.G, s=wl.s, io_round=io)
+    cc = torch.stack([u[:, (j + 1) * wl.s - 3:(j + 1) * wl.s] for j in range(wl.L // wl.s)], dim=1)
+    ref = oracle.layer_backward(un, prm["w"].numpy(), dt.numpy(), prm["A"].numpy(), prm["D"].numpy(),
+                                host(dy).reshape(wl.b, wl.L, wl.H, wl.P), bias=prm["bias"].numpy(),
+                                h_ckpt=fwd["h_ckpt"], conv_ckpt=host(cc), dh_final=dhf.double().numpy(),
+                                dtail_out=dto.double().numpy(), H=wl.H, P=wl.P, N=wl.N, G=wl.G, s=wl.s,
+                                io_round=io)
+    d = "cuda"
+    g = {k: v.to(d) for k, v in prm.items()}
+    gf = ssd.stream_forward(u.to(d), g["w"], dt.to(d), g["A"], g["D"], H=wl.H, P=wl.P, N=wl.N, G=wl.G, Q=wl.Q,
+                            s=wl.s, conv_bias=g["bias"])
+    ssd.sync_status()
+    vg = host(gf["v"]).astype(np.float64)
+    vo = np.asarray(fwd["v"], dtype=np.float64)
+    if io == "bf16":
+        ve = oracle.conv(un, prm["w"].numpy(), prm["bias"].numpy())[0].astype(np.float64)
+        # size of the conv's pre-activation terms, for the fp32 rounding of their sum
+        w, b = prm["w"].double().numpy(), prm["bias"].double().numpy()
+        ext = np.concatenate([np.zeros((wl.b, 3, wl.cch)), un.astype(np.float64)], axis=1)
+        zabs = np.abs(b) + sum(np.abs(w[:, k] * ext[:, k:k + wl.L]) for k in range(4))
+        z = b + sum(w[:, k] * ext[:, k:k + wl.L] for k in range(4))
+        mant, ex = np.frexp(np.abs(ve))
+        spacing = np.where(ve == 0.0, 0.0, np.ldexp(1.0, ex - 8))
+        bound = spacing + 1.1 * 5 * 2.0 ** -24 * zabs + np.abs(z) * 2.0 ** -12
+        over = np.abs(vg - ve) > bound
+        assert not over.any(), (int(over.sum()), float(np.abs(vg - ve)[over].max()))
+        flips = float(np.mean(vg != vo))
+        assert flips <= 1e-3, flips
+        ev = rel_l2(vg, vo)
+        assert ev <= 2.5e-4, ev
+        tol = 5e-4
+    else:
+        assert rel_l2(vg, vo) <= 1e-6
+        tol = 1e-5
+    ws = torch.empty(ssd.layer_backward_workspace_size(wl.b, wl.L, wl.H, wl.P, wl.N, wl.G,
+                                                      ssd.SSD_BF16 if io == "bf16" else ssd.SSD_F32),
+                     dtype=torch.uint8, device=d)
+    kw = dict(H=wl.H, P=wl.P, N=wl.N, G=wl.G, s=wl.s, conv_bias=g["bias"],
+              h_ckpt=torch.from_numpy(fwd["h_ckpt"]).float().to(d), conv_ckpt=cc.to(d), dh_final=dhf.to(d),
+              dtail_out=dto.to(d), workspace=ws)
+    args = (u.to(d), g["w"], dt.to(d), g["A"], g["D"], dy.to(d))
+    first = ssd.layer_backward(*args, **kw)
+    ssd.sync_status()
+    snap = {k: host(first[k]).copy() for k in KEYS}
+    for v in first.values():
+        if torch.is_tensor(v):
+            v.fill_(float("nan"))
+    again = ssd.layer_backward(*args, out=first, **kw)
+    ssd.sync_status()
+    errs = _errs(again, ref)
+    assert all(e <= tol for e in errs.values()), errs
+    for k in KEYS:
+        assert np.array_equal(host(again[k]), snap[k]), k
