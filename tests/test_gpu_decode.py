@@ -118,3 +118,33 @@ def test_decode_continues_a_streamed_prefix():
     assert rel_l2(got_y, ref["y"].reshape(1, 528, -1)) <= TOL["bf16"]
     assert rel_l2(host(h), ref["h_final"]) <= TOL["bf16"]
     np.testing.assert_array_equal(host(tl), ref["tail_out"])
+
+
+def test_bench_configuration_256_streams():
+    """The configuration the decode bench times: 256 independent streams of the 0.3B shape (32 heads
+    of P = 64, N = 128, 2304 conv channels, bf16), each from an empty state and conv tail, eight
+    steps with the state and tail updated in place and y written into the caller's buffer; every
+    step's y and the final state against the oracle's layer over the eight tokens of each stream,
+    the conv tail bitwise."""
+    wl = ssd_synth.scaled(W[1], b=256, L=8, segments=1)
+    prm, u, dt = _inputs(wl, seed=21)
+    d = "cuda"
+    g = {k: v.to(d) for k, v in prm.items()}
+    u_steps = u.to(d).transpose(0, 1).contiguous()
+    dt_steps = dt.to(d).transpose(0, 1).contiguous()
+    h = torch.zeros(wl.b, wl.H, wl.P, wl.N, device=d)
+    tl = torch.zeros(wl.b, 3, wl.cch, dtype=u.dtype, device=d)
+    y = torch.empty(wl.b, wl.H, wl.P, dtype=u.dtype, device=d)
+    ys = []
+    for t in range(wl.L):
+        ssd.decode_step(u_steps[t], g["w"], dt_steps[t], g["A"], g["D"], H=wl.H, P=wl.P, N=wl.N, G=wl.G,
+                        conv_bias=g["bias"], tail_in=tl, tail_out=tl, h_in=h, h_out=h, y=y)
+        ys.append(y.clone())
+    ssd.sync_status()
+    ref = _oracle(wl, u, prm, dt)
+    got = host(torch.stack(ys, 1)).reshape(wl.b, wl.L, -1)
+    want = ref["y"].reshape(wl.b, wl.L, -1)
+    for t in range(wl.L):
+        assert rel_l2(got[:, t], want[:, t]) <= TOL["bf16"], t
+    assert rel_l2(host(h), ref["h_final"]) <= TOL["bf16"]
+    np.testing.assert_array_equal(host(tl), ref["tail_out"])

@@ -81,3 +81,20 @@ def test_norm_after_the_scan():
                      prm["D"].numpy(), s=0, H=wl.H, P=wl.P, want_ckpt=False)["y"]
     ref = oracle.gated_rmsnorm(ys.reshape(wl.b, wl.L, -1), z.float().numpy(), w.numpy(), io_round="bf16")
     assert rel_l2(host(out).astype(np.float32), ref) <= TOL["bf16"]
+
+
+def test_norm_bench_configuration_sampled_rows():
+    """The configuration the norm bench times: 131072 rows of 2048 (the 0.3B d_inner), bf16, one
+    group, so that each warp of the 296-CTA grid walks about 55 rows; the first and last 64 rows
+    and every 61st row between them against the oracle, row by row."""
+    rows, d = 131072, 2048
+    y = _gen((rows, d), torch.bfloat16, 7)
+    z = _gen((rows, d), torch.bfloat16, 8, scale=3.0)
+    w = _gen((d,), torch.float32, 9)
+    out = torch.empty(rows, d, dtype=torch.bfloat16, device="cuda")
+    ssd.gated_rmsnorm(y.cuda(), z.cuda(), w.cuda(), eps=1e-5, out=out)
+    ssd.sync_status()
+    idx = np.unique(np.r_[0:64, 64:rows - 64:61, rows - 64:rows])
+    ref = oracle.gated_rmsnorm(y[idx].float().numpy(), z[idx].float().numpy(), w.numpy(), eps=1e-5,
+                               io_round="bf16")
+    _check(out[torch.from_numpy(idx).cuda()], ref, torch.bfloat16)
