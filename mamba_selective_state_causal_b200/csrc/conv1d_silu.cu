@@ -46,14 +46,16 @@ template <> struct VecIO<__nv_bfloat16> {
         for (int i = 0; i < 4; ++i) v.w[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
         return v;
     }
-    // SiLU(z) = z sigmoid(z) = z (1 + tanh(z / 2)) / 2 with one hardware tanh
-    // (relative error about 2^-11) instead of an exponential and a reciprocal;
-    // the result is rounded to bf16 right after
-    __device__ __forceinline__ static float silu(float z)
+    // The conv sums with halved weights and bias (kPre; a power-of-two scale, exact), so
+    // that silu() receives h = z / 2, and SiLU(z) = z sigmoid(z) = h + h tanh(h): one
+    // hardware tanh (relative error about 2^-11) and one fma instead of an exponential and
+    // a reciprocal; the result is rounded to bf16 right after
+    static constexpr float kPre = 0.5f;
+    __device__ __forceinline__ static float silu(float h)
     {
         float t;
-        asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
-        return z * fmaf(0.5f, t, 0.5f);
+        asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+        return fmaf(h, t, h);
     }
 };
 template <> struct VecIO<float> {
@@ -70,7 +72,8 @@ template <> struct VecIO<float> {
         for (int i = 0; i < 4; ++i) v.w[i] = __float_as_uint(f[i]);
         return v;
     }
-    // accurate SiLU for the fp32 I/O path
+    // accurate SiLU for the fp32 I/O path, on the unscaled sum
+    static constexpr float kPre = 1.0f;
     __device__ __forceinline__ static float silu(float z) { return z / (1.0f + expf(-z)); }
 };
 
@@ -125,8 +128,8 @@ __global__ void __launch_bounds__(kConvThreads, 2) conv1d_silu_kernel(ConvParams
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             float4 q = __ldg(wp + i);
-            w0[i] = q.x; w1[i] = q.y; w2[i] = q.z; w3[i] = q.w;
-            bs[i] = p.bias ? __ldg(p.bias + c0 + i) : 0.0f;
+            w0[i] = IO::kPre * q.x; w1[i] = IO::kPre * q.y; w2[i] = IO::kPre * q.z; w3[i] = IO::kPre * q.w;
+            bs[i] = p.bias ? IO::kPre * __ldg(p.bias + c0 + i) : 0.0f;
         }
     }
     // halo: m3 = u[t-3], m2 = u[t-2], m1 = u[t-1]
@@ -268,9 +271,13 @@ __global__ void __launch_bounds__(256, 3) conv_cells2_kernel(ConvBwdParams p, in
     const int64_t bi = gid / ((int64_t)np * nblk);
     const int64_t t0 = blk * kCellTB;
     const int64_t t1 = min(p.L, t0 + kCellTB);
-    const float4 wa = __ldg(reinterpret_cast<const float4 *>(p.w) + c);
-    const float4 wb = __ldg(reinterpret_cast<const float4 *>(p.w) + c + 1);
-    const float ba = p.bias ? __ldg(p.bias + c) : 0.0f, bb = p.bias ? __ldg(p.bias + c + 1) : 0.0f;
+    // weights and bias scaled as the forward conv scales them (VecIO::kPre)
+    constexpr float pre = VecIO<T>::kPre;
+    const float4 qa = __ldg(reinterpret_cast<const float4 *>(p.w) + c);
+    const float4 qb = __ldg(reinterpret_cast<const float4 *>(p.w) + c + 1);
+    const float4 wa = make_float4(pre * qa.x, pre * qa.y, pre * qa.z, pre * qa.w);
+    const float4 wb = make_float4(pre * qb.x, pre * qb.y, pre * qb.z, pre * qb.w);
+    const float ba = p.bias ? pre * __ldg(p.bias + c) : 0.0f, bb = p.bias ? pre * __ldg(p.bias + c + 1) : 0.0f;
     const T *u = reinterpret_cast<const T *>(p.u) + bi * p.ubs + c;
     // the window u[t0-3 .. t0-1]: rows before the cell come from its conv buffer
     const int64_t kc = p.conv_ckpt ? t0 / p.s : 0;

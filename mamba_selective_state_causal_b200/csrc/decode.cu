@@ -24,13 +24,17 @@ namespace {
 
 constexpr int kDecThreads = 256;
 
+// SiLU of the conv sum, as the layer's conv computes it: for bf16 the weights and bias are
+// halved (kDecPre, exact), the sum is h = z / 2 and SiLU(z) = h + h tanh(h) with one hardware
+// tanh, the result rounded to bf16 right after; for fp32 the accurate form on z itself
+template <typename T> constexpr float kDecPre = 1.0f;
+template <> constexpr float kDecPre<__nv_bfloat16> = 0.5f;
 template <typename T> __device__ __forceinline__ float dec_silu(float z);
-// one hardware tanh, the result is rounded to bf16 right after
-template <> __device__ __forceinline__ float dec_silu<__nv_bfloat16>(float z)
+template <> __device__ __forceinline__ float dec_silu<__nv_bfloat16>(float h)
 {
     float t;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
-    return z * fmaf(0.5f, t, 0.5f);
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+    return fmaf(h, t, h);
 }
 template <> __device__ __forceinline__ float dec_silu<float>(float z) { return z / (1.0f + expf(-z)); }
 
@@ -51,8 +55,10 @@ __global__ void __launch_bounds__(kDecThreads, 6) decode_step_kernel(DecodeParam
     for (int i = threadIdx.x; i < p.P + 2 * p.N; i += blockDim.x) {
         const int c = i < p.P ? h * p.P + i : (i < p.P + p.N ? din + g * p.N + (i - p.P)
                                                              : din + p.G * p.N + g * p.N + (i - p.P - p.N));
-        const float4 w = reinterpret_cast<const float4 *>(p.w)[c];
-        float z = p.bias ? p.bias[c] : 0.0f;
+        constexpr float pre = kDecPre<T>;
+        const float4 wq = reinterpret_cast<const float4 *>(p.w)[c];
+        const float4 w = make_float4(pre * wq.x, pre * wq.y, pre * wq.z, pre * wq.w);
+        float z = p.bias ? pre * p.bias[c] : 0.0f;
         if (tin) {
             z = fmaf(w.x, to_f32(tin[c]), z);
             z = fmaf(w.y, to_f32(tin[C_ch + c]), z);

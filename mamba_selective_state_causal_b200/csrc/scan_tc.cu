@@ -98,24 +98,24 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __
 __device__ __forceinline__ float2 unpack2(uint32_t v) { return make_float2(bf16_lo(v), bf16_hi(v)); }
 
 // Conv + SiLU of 8 channels (4 pairs) of one token: window m3 = u[t-3], m2, m1, cur = u[t],
-// weights w[pair][tap] and bias as channel pairs.  The same operations, in the same order
-// and rounding, as the conv kernel's scalar code, two channels per instruction.
+// weights w[pair][tap] and bias as channel pairs, both already halved, so that the sum is
+// h = z / 2 and SiLU(z) = z sigmoid(z) = h + h tanh(h) takes one hardware tanh and one fma.
+// The same operations, in the same order and rounding, as the conv kernel's scalar code,
+// two channels per instruction.
 __device__ __forceinline__ uint4 conv8(const float2 (&w)[4][4], const float2 (&bs)[4], const float2 (&m3)[4],
                                        const float2 (&m2)[4], const float2 (&m1)[4], const float2 (&cur)[4])
 {
     uint32_t o[4];
-    const float2 half = make_float2(0.5f, 0.5f);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        float2 z = fma2(w[i][0], m3[i], bs[i]);
-        z = fma2(w[i][1], m2[i], z);
-        z = fma2(w[i][2], m1[i], z);
-        z = fma2(w[i][3], cur[i], z);
-        const float2 h = mul2(half, z);
+        float2 h = fma2(w[i][0], m3[i], bs[i]);
+        h = fma2(w[i][1], m2[i], h);
+        h = fma2(w[i][2], m1[i], h);
+        h = fma2(w[i][3], cur[i], h);
         float2 t;
         asm("tanh.approx.f32 %0, %1;" : "=f"(t.x) : "f"(h.x));
         asm("tanh.approx.f32 %0, %1;" : "=f"(t.y) : "f"(h.y));
-        const float2 sg = mul2(z, fma2(half, t, half));
+        const float2 sg = fma2(h, t, h);
         o[i] = pack_bf16x2(sg.x, sg.y);
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
@@ -222,9 +222,10 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
             for (int i = 0; i < 4; ++i) {
                 const float4 qa = __ldg(reinterpret_cast<const float4 *>(p.conv_w) + c0ch + 2 * i);
                 const float4 qb = __ldg(reinterpret_cast<const float4 *>(p.conv_w) + c0ch + 2 * i + 1);
-                cw[i][0] = make_float2(qa.x, qb.x); cw[i][1] = make_float2(qa.y, qb.y);
-                cw[i][2] = make_float2(qa.z, qb.z); cw[i][3] = make_float2(qa.w, qb.w);
-                cb[i] = p.conv_bias ? make_float2(__ldg(p.conv_bias + c0ch + 2 * i), __ldg(p.conv_bias + c0ch + 2 * i + 1))
+                // halved (exact) for conv8's h = z / 2
+                cw[i][0] = make_float2(0.5f * qa.x, 0.5f * qb.x); cw[i][1] = make_float2(0.5f * qa.y, 0.5f * qb.y);
+                cw[i][2] = make_float2(0.5f * qa.z, 0.5f * qb.z); cw[i][3] = make_float2(0.5f * qa.w, 0.5f * qb.w);
+                cb[i] = p.conv_bias ? make_float2(0.5f * __ldg(p.conv_bias + c0ch + 2 * i), 0.5f * __ldg(p.conv_bias + c0ch + 2 * i + 1))
                                     : make_float2(0.0f, 0.0f);
             }
         }
@@ -259,6 +260,10 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
                 if (lane == 0) mbar_arrive(&s.halo_read[st]);
                 ok = ewait(&s.halo_read[st], ph, abort, lim);
                 if (!ok) break;
+                // x rows 4 rg .. 4 rg + 3 of the chunk in global memory (rows past the sequence end skipped)
+                __nv_bfloat16 *xo = reinterpret_cast<__nv_bfloat16 *>(p.conv_v) + (int64_t)bi * p.conv_vbs +
+                                    (t0 + 4 * rg) * p.conv_vrs + (ha + hd) * kP + 8 * ch;
+                const int64_t nrows = s1 - t0 - 4 * rg;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int r = 4 * rg + i;
@@ -266,9 +271,8 @@ stripe_state_tc_kernel(const __grid_constant__ Maps maps, const ScanParams p)
                     float2 cur[4];
                     unpack8(lds128(a), cur);
                     uint4 v = conv8(cw, cb, m3, m2, m1, cur);
-                    if (t0 + r < s1)
-                        *reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.conv_v) + (int64_t)bi * p.conv_vbs +
-                                                   (t0 + r) * p.conv_vrs + (ha + hd) * kP + 8 * ch) = v;
+                    if (i < nrows) *reinterpret_cast<uint4 *>(xo) = v;
+                    xo += p.conv_vrs;
                     const float w = s.w[st][hd][r];
                     const float2 w2 = make_float2(w, w);
                     v.x = scale_bf16x2_rn(v.x, w2); v.y = scale_bf16x2_rn(v.y, w2);
