@@ -50,6 +50,14 @@ __global__ void __launch_bounds__(kDecThreads, 6) decode_step_kernel(DecodeParam
     const int C_ch = din + 2 * p.G * p.N;
     const T *u = reinterpret_cast<const T *>(p.u) + (int64_t)bi * p.ubs;
     const T *tin = p.tail_in ? reinterpret_cast<const T *>(p.tail_in) + (int64_t)bi * 3 * C_ch : nullptr;
+    // start this (stream, head)'s state on its way into L2 while the conv below runs: one bulk
+    // prefetch of its P x N floats (a hint, no registers or shared memory held).  The host
+    // checks h_in for 16-byte alignment and P, N are powers of two from 16 to 128, so every
+    // state starts on a 16-byte boundary and P N 4 bytes is a multiple of 16
+    if (threadIdx.x == 0 && p.h_in) {
+        const float *hpf = p.h_in + ((int64_t)bi * p.H + h) * (int64_t)p.P * p.N;
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(hpf), "r"((uint32_t)(p.P * p.N * 4)) : "memory");
+    }
 
     // conv + SiLU of the P + 2N channels this head reads
     for (int i = threadIdx.x; i < p.P + 2 * p.N; i += blockDim.x) {
