@@ -822,6 +822,10 @@ __device__ __forceinline__ void store_pieces3(uint8_t (&dst)[3][2 * kSumBox], co
     }
 }
 
+// how far ahead (in CTAs) the gradient kernel prefetches Gam and h_prev: measured 0.504 ms per
+// launch at 32 and 48, 0.509 at 74, 0.512 at 110, no gain at a whole wave (296), 0.535 without
+constexpr int kGradAhead = 32;
+
 __global__ void __launch_bounds__(kGradTcThreads, 2) bwd_chunk_grad_tc_kernel(BwdParams p)
 {
     extern __shared__ __align__(1024) uint8_t sgt_raw[];
@@ -843,6 +847,16 @@ __global__ void __launch_bounds__(kGradTcThreads, 2) bwd_chunk_grad_tc_kernel(Bw
         fence_mbar_init();
     }
     if (warp == 0) { tmem_alloc(&s.tmem, kGradTcCols); tmem_relinquish(); }
+    // Gam and h_prev of the unit kGradAhead CTAs further on (which starts a few microseconds
+    // later, CTAs being scheduled in order) started into L2 with one bulk prefetch each: its
+    // loads below then find them there (a hint; the blocks are 32 KB each, 256-byte aligned)
+    if (tid == 32 || tid == 33) {
+        const int64_t ahead = unit + kGradAhead;
+        if (ahead < (int64_t)p.b * p.H * p.nch) {
+            const float *src = (tid == 32 ? p.ws_g : p.ws_h) + ahead * (int64_t)P * N;
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"((uint32_t)(P * N * 4)) : "memory");
+        }
+    }
 
     // x, dy, B, C rows: 16-byte asynchronous copies into the swizzled tiles, rows past L zero
     {
