@@ -329,6 +329,7 @@ __device__ __forceinline__ float4 f4_fma(float a, float4 x, float4 y)
 }
 
 constexpr int kChainAhead = 16;   // chunk summaries loaded ahead of the chain
+constexpr int kChainPrefetch = 32; // CTAs ahead whose summaries the state chain starts into L2
 
 // State entering every chunk, per cell: h = start of the cell (h0 or the
 // checkpoint before it); for each chunk c of the cell: slot c := h, then
@@ -342,6 +343,23 @@ __global__ void __launch_bounds__(kBwdThreads, 3) bwd_state_chain_kernel(BwdPara
     const int sl = blockIdx.x % slices;
     const int64_t k = blockIdx.x / slices;
     const int h = blockIdx.y, bi = blockIdx.z;
+    if (threadIdx.x < kChainAhead) {
+        // the chunk summaries of the CTA kChainPrefetch further on (one contiguous slice of up to
+        // 4 KB per chunk), started into L2 with one bulk prefetch per chunk: CTAs run in order, so
+        // that CTA's loads below find them there (0.115 -> 0.093 ms per launch at the 0.3B shape)
+        const int64_t ahead = ((int64_t)bi * p.H + h) * gridDim.x + blockIdx.x + kChainPrefetch;
+        if (ahead < (int64_t)gridDim.x * p.H * p.b) {
+            const int64_t xa = ahead % gridDim.x, hua = ahead / gridDim.x;
+            const int64_t e0 = (xa % slices) * 4 * kBwdThreads, ka = xa / slices;
+            const int64_t ca = ka * p.cell_chunks + threadIdx.x;
+            const int64_t ce = p.nch < (ka + 1) * p.cell_chunks ? p.nch : (ka + 1) * p.cell_chunks;
+            if (ca < ce) {
+                const int64_t n = PN - e0 < 4 * kBwdThreads ? PN - e0 : 4 * kBwdThreads;
+                const float *src = p.ws_h + (hua * p.nch + ca) * PN + e0;
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"((uint32_t)(n * 4)) : "memory");
+            }
+        }
+    }
     const int64_t e = (int64_t)sl * 4 * kBwdThreads + 4 * threadIdx.x;
     if (e >= PN) return;
     const int64_t hu = (int64_t)bi * p.H + h;
